@@ -1,0 +1,528 @@
+/*
+ * moe_oracle.c -- plain single-threaded CPU oracle of the Sparsely-Gated MoE
+ * layer forward pass.  TEST INFRASTRUCTURE ONLY (see moe_oracle.h): it is
+ * loaded by tests, the smoke check and the bench's CPU-baseline leg, never by
+ * the product path.  Loops are written in the order of the formulas they
+ * follow; no blocking, fusion or reordering beyond that.
+ */
+#include "moe_oracle.h"
+
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+/* ======================================================================= */
+/* Noise: StandardNormal() of the noisy gate.                               */
+/* [SGMoE-xyz] "Noisy Top-K 門控" writes H(x)_i = (x W_g)_i +                */
+/* StandardNormal() * Softplus((x W_noise)_i) without saying how the normal */
+/* deviate is drawn.  Our reading: a counter-based stream, so that every    */
+/* (seed, token, expert, gate) has one fixed deviate on any machine:        */
+/*   key = (seed low 32 bits, seed high 32 bits)                            */
+/*   ctr = (token, expert / 2, gate_id, 0)                                  */
+/*   words (w0,w1) feed the even expert of the pair, (w2,w3) the odd one,   */
+/*   each through one Box-Muller cosine branch.                             */
+/* ======================================================================= */
+
+/* Philox4x32-10 [Philox]: ten rounds of the 4x32 S-box.  Each round
+ * multiplies words 0 and 2 by the two round multipliers, swaps the halves and
+ * folds in the key; the key is bumped by the two Weyl constants between
+ * rounds. */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4])
+{
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;  /* round multipliers */
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;  /* key bumps (Weyl)  */
+  uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    uint64_t p0 = (uint64_t)M0 * (uint64_t)x0;
+    uint64_t p1 = (uint64_t)M1 * (uint64_t)x2;
+    uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    uint32_t y0 = hi1 ^ x1 ^ k0;
+    uint32_t y1 = lo1;
+    uint32_t y2 = hi0 ^ x3 ^ k1;
+    uint32_t y3 = lo0;
+    x0 = y0; x1 = y1; x2 = y2; x3 = y3;
+  }
+  out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
+}
+
+/* Box-Muller [Box-Muller], cosine branch.  u1 = (top 24 bits of w0 + 1)/2^24
+ * lies in (0,1] so the logarithm is finite; u2 = (top 24 bits of w1)/2^24
+ * lies in [0,1). */
+double orc_box_muller(uint32_t w0, uint32_t w1)
+{
+  double u1 = ((double)(w0 >> 8) + 1.0) / 16777216.0;
+  double u2 = (double)(w1 >> 8) / 16777216.0;
+  const double two_pi = 6.283185307179586476925286766559;
+  return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+}
+
+double orc_noise(uint64_t seed, uint32_t token, uint32_t expert, uint32_t gate_id)
+{
+  uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
+  uint32_t ctr[4] = {token, expert >> 1, gate_id, 0u};
+  uint32_t w[4];
+  orc_philox4x32_10(ctr, key, w);
+  if ((expert & 1u) == 0u) return orc_box_muller(w[0], w[1]);
+  return orc_box_muller(w[2], w[3]);
+}
+
+/* ======================================================================= */
+/* Closed-form helpers                                                     */
+/* ======================================================================= */
+
+/* Softplus(z) = log(1 + e^z), written in the overflow-free form. */
+double orc_softplus(double z)
+{
+  double a = fabs(z);
+  return (z > 0.0 ? z : 0.0) + log1p(exp(-a));
+}
+
+/* Phi: the standard Normal CDF used by the smoothed load estimator
+ * ([SGMoE-xyz] "負載平衡損失"). */
+double orc_phi(double z)
+{
+  return 0.5 * erfc(-z / sqrt(2.0));
+}
+
+/* Squared coefficient of variation: population variance over squared mean.
+ * [SGMoE-xyz] "負載平衡損失" defines L = w * CV(.)^2 without fixing the
+ * variance convention; our reading is the population variance.  A zero mean
+ * gives 0. */
+double orc_cv2(const double *v, int n)
+{
+  if (n <= 0) return 0.0;
+  double sum = 0.0;
+  for (int i = 0; i < n; ++i) sum += v[i];
+  double mean = sum / (double)n;
+  if (mean == 0.0) return 0.0;
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += (v[i] - mean) * (v[i] - mean);
+  double var = ss / (double)n;
+  return var / (mean * mean);
+}
+
+/* Round an fp32 value to the nearest bf16 (ties to even), returned as fp32. */
+float orc_bf16_round(float v)
+{
+  uint32_t u;
+  memcpy(&u, &v, 4);
+  if ((u & 0x7f800000u) == 0x7f800000u && (u & 0x007fffffu) != 0u) {
+    u = (u | 0x00400000u) & 0xffff0000u; /* keep NaN a (quiet) NaN */
+  } else {
+    uint32_t lsb = (u >> 16) & 1u;
+    u += 0x7fffu + lsb;
+    u &= 0xffff0000u;
+  }
+  float r;
+  memcpy(&r, &u, 4);
+  return r;
+}
+
+static double bf16_bits_to_double(uint16_t b)
+{
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* Expert capacity, [MoE-deep] §3.2: C = tokens per batch / E * capacity
+ * factor.  With k slots per token our reading counts T*k routed slots, and
+ * rounds up.  No limit when the factor is not positive. */
+int64_t orc_capacity(int T, int k, int n, double capacity_factor)
+{
+  if (capacity_factor <= 0.0) return INT64_MAX;
+  return (int64_t)ceil((double)T * (double)k * capacity_factor / (double)n);
+}
+
+/* ======================================================================= */
+/* Gate                                                                     */
+/* ======================================================================= */
+
+typedef struct { float h; int i; } keyed;
+
+/* Order: larger H first; equal H -> lower index first (the pages do not say
+ * how ties are broken; our reading is lower index). */
+static int keyed_cmp(const void *pa, const void *pb)
+{
+  const keyed *a = (const keyed *)pa, *b = (const keyed *)pb;
+  if (a->h > b->h) return -1;
+  if (a->h < b->h) return 1;
+  return (a->i < b->i) ? -1 : (a->i > b->i);
+}
+
+/* Noisy top-k gating, [SGMoE-xyz] "Noisy Top-K 門控" and [SGMoE-note] "Noisy
+ * Top-K Gating":
+ *   H(x)_i = (x W_g)_i + StandardNormal() * Softplus((x W_noise)_i)
+ *   KeepTopK(v,k)_i = v_i if v_i is among the top k of v, else -inf
+ *   G(x) = Softmax(KeepTopK(H(x), k))
+ * The optional per-expert bias b_g is part of the clean logit (x W_g)_i.
+ * Router 1 is the Switch router of [MoE-deep] §3.1: p = softmax(x W_r) over
+ * all experts, the token goes to argmax p and is weighted by p_argmax (no
+ * renormalisation over the kept expert). */
+void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
+                  uint32_t token, uint32_t gate_id, const float *x,
+                  const float *Wg, const float *bg, const float *Wn,
+                  double *c, double *s, float *H, int *order, double *gates,
+                  double *p)
+{
+  for (int i = 0; i < n; ++i) { c[i] = 0.0; s[i] = 0.0; }
+  for (int j = 0; j < d; ++j) {
+    double xj = (double)x[j];
+    for (int i = 0; i < n; ++i) c[i] += xj * (double)Wg[(size_t)j * n + i];
+    if (noise)
+      for (int i = 0; i < n; ++i) s[i] += xj * (double)Wn[(size_t)j * n + i];
+  }
+  for (int i = 0; i < n; ++i) {
+    if (bg) c[i] += (double)bg[i];
+    if (noise) {
+      s[i] = orc_softplus(s[i]);
+      double eps = orc_noise(seed, token, (uint32_t)i, gate_id);
+      H[i] = (float)(c[i] + eps * s[i]);
+    } else {
+      s[i] = 0.0;
+      H[i] = (float)c[i];
+    }
+  }
+
+  keyed *kv = (keyed *)malloc(sizeof(keyed) * (size_t)n);
+  for (int i = 0; i < n; ++i) { kv[i].h = H[i]; kv[i].i = i; }
+  qsort(kv, (size_t)n, sizeof(keyed), keyed_cmp);
+  for (int i = 0; i < n; ++i) order[i] = kv[i].i;
+  free(kv);
+
+  if (router == 1) {
+    double m = c[0];
+    for (int i = 1; i < n; ++i) if (c[i] > m) m = c[i];
+    double den = 0.0;
+    for (int i = 0; i < n; ++i) den += exp(c[i] - m);
+    for (int i = 0; i < n; ++i) {
+      double pi = exp(c[i] - m) / den;
+      if (p) p[i] = pi;
+      if (i == order[0]) gates[0] = pi;
+    }
+    return;
+  }
+
+  /* softmax over the kept k; every other entry is -inf and gets 0. */
+  double hmax = (double)H[order[0]];
+  double den = 0.0;
+  for (int j = 0; j < k; ++j) den += exp((double)H[order[j]] - hmax);
+  for (int j = 0; j < k; ++j) gates[j] = exp((double)H[order[j]] - hmax) / den;
+}
+
+/* Smoothed load, [SGMoE-xyz] "負載平衡損失":
+ *   P(x,i) = Phi( ((x W_g)_i - kth_excluding(H(x), k, i)) / Softplus((x W_noise)_i) )
+ * kth_excluding(H,k,i) is the k-th largest entry of H once entry i is left
+ * out.  With H sorted, that is the (k+1)-th largest when i itself is among the
+ * first k, and the k-th largest otherwise; -inf (P = 1) when fewer than k
+ * other entries exist.  Without noise the estimator has no spread; we use
+ * its zero-noise limit, the indicator of i being kept. */
+void orc_load_row(int n, int k, int noise, const double *c, const double *s,
+                  const float *H, double *P)
+{
+  int *rank = (int *)malloc(sizeof(int) * (size_t)n);
+  keyed *kv = (keyed *)malloc(sizeof(keyed) * (size_t)n);
+  for (int i = 0; i < n; ++i) { kv[i].h = H[i]; kv[i].i = i; }
+  qsort(kv, (size_t)n, sizeof(keyed), keyed_cmp);
+  for (int r = 0; r < n; ++r) rank[kv[r].i] = r;
+  double v_k = (double)kv[k - 1].h;
+  double v_k1 = (k < n) ? (double)kv[k].h : -INFINITY;
+  for (int i = 0; i < n; ++i) {
+    int kept = rank[i] < k;
+    if (!noise) { P[i] = kept ? 1.0 : 0.0; continue; }
+    double thr = kept ? v_k1 : v_k;
+    if (thr == -INFINITY) { P[i] = 1.0; continue; }
+    double num = c[i] - thr;
+    if (s[i] == 0.0) { P[i] = num > 0.0 ? 1.0 : (num < 0.0 ? 0.0 : 0.5); continue; }
+    P[i] = orc_phi(num / s[i]);
+  }
+  free(kv);
+  free(rank);
+}
+
+/* ======================================================================= */
+/* Dispatch                                                                 */
+/* ======================================================================= */
+
+/* [SGMoE-note] "Sparsely-Gated MoE 层架构": E_i(x) need not be computed when
+ * G(x)_i = 0, so each token is sent only to its kept experts.  Slots are
+ * visited token by token, slot by slot; a slot's rank is the number of
+ * earlier slots sent to the same expert.  [MoE-deep] §3.2: an expert takes
+ * at most C tokens, the rest overflow (our reading: the later tokens, in
+ * this visiting order, are the ones that overflow). */
+void orc_dispatch(int T, int k, int n, int64_t C, const int32_t *idx,
+                  int32_t *counts, int32_t *offsets, int32_t *perm_token,
+                  int32_t *perm_slot, int32_t *row_of, int64_t *n_invalid)
+{
+  int64_t invalid = 0;
+  for (int e = 0; e < n; ++e) counts[e] = 0;
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      int32_t e = idx[(size_t)t * k + j];
+      if (e < 0 || e >= n) invalid++;
+      else counts[e]++;
+    }
+  offsets[0] = 0;
+  for (int e = 0; e < n; ++e) {
+    int64_t kept = counts[e] < C ? counts[e] : C;
+    offsets[e + 1] = offsets[e] + (int32_t)kept;
+  }
+  int32_t *seen = (int32_t *)calloc((size_t)(n > 0 ? n : 1), sizeof(int32_t));
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j) {
+      size_t p = (size_t)t * k + j;
+      int32_t e = idx[p];
+      if (e < 0 || e >= n) { row_of[p] = -1; continue; }
+      int32_t r = seen[e]++;
+      if ((int64_t)r < C) {
+        int32_t row = offsets[e] + r;
+        row_of[p] = row;
+        perm_token[row] = t;
+        perm_slot[row] = j;
+      } else {
+        row_of[p] = -1;
+      }
+    }
+  free(seen);
+  if (n_invalid) *n_invalid = invalid;
+}
+
+/* ======================================================================= */
+/* Expert                                                                   */
+/* ======================================================================= */
+
+/* [SGMoE-note] "Sparsely-Gated MoE 层架构": every expert is a feed-forward
+ * network with one ReLU hidden layer, same shape, own parameters:
+ *   E(x) = ReLU(x W1^T + b1) W2^T + b2      (W1: [f][d], W2: [d][f])
+ * bf16 experts take bf16 activations: x and the hidden layer are rounded to
+ * bf16, all sums are fp64. */
+void orc_expert_row(int d, int f, int bf16, const float *x, const void *W1,
+                    const float *b1, const void *W2, const float *b2, double *y)
+{
+  double *h = (double *)malloc(sizeof(double) * (size_t)(f > 0 ? f : 1));
+  for (int j = 0; j < f; ++j) {
+    double acc = 0.0;
+    for (int q = 0; q < d; ++q) {
+      double xv, wv;
+      if (bf16) {
+        xv = (double)orc_bf16_round(x[q]);
+        wv = bf16_bits_to_double(((const uint16_t *)W1)[(size_t)j * d + q]);
+      } else {
+        xv = (double)x[q];
+        wv = (double)((const float *)W1)[(size_t)j * d + q];
+      }
+      acc += xv * wv;
+    }
+    if (b1) acc += (double)b1[j];
+    double r = acc > 0.0 ? acc : 0.0;
+    h[j] = bf16 ? (double)orc_bf16_round((float)r) : r;
+  }
+  for (int q = 0; q < d; ++q) {
+    double acc = 0.0;
+    for (int j = 0; j < f; ++j) {
+      double wv = bf16 ? bf16_bits_to_double(((const uint16_t *)W2)[(size_t)q * f + j])
+                       : (double)((const float *)W2)[(size_t)q * f + j];
+      acc += h[j] * wv;
+    }
+    if (b2) acc += (double)b2[q];
+    y[q] = acc;
+  }
+  free(h);
+}
+
+/* ======================================================================= */
+/* Whole layer                                                              */
+/* ======================================================================= */
+
+static float min_gap(const float *H, const int *order, int n, int k)
+{
+  float g = INFINITY;
+  int last = k < n - 1 ? k : n - 1;
+  for (int j = 1; j <= last; ++j) {
+    float d = H[order[j - 1]] - H[order[j]];
+    if (d < g) g = d;
+  }
+  return g;
+}
+
+static int valid_cfg(const orc_cfg *c)
+{
+  if (c->T < 0 || c->d < 1 || c->f < 1 || c->n < 1 || c->k < 1 || c->k > c->n) return 0;
+  if (c->router != 0 && c->router != 1) return 0;
+  if (c->router == 1 && (c->k != 1 || c->noise || c->hier_a)) return 0;
+  if (c->hier_a) {
+    if (c->hier_b < 1 || c->hier_a * c->hier_b != c->n) return 0;
+    if (c->hier_k1 < 1 || c->hier_k1 > c->hier_a) return 0;
+    if (c->hier_k2 < 1 || c->hier_k2 > c->hier_b) return 0;
+    if (c->hier_k1 * c->hier_k2 != c->k) return 0;
+  }
+  return 1;
+}
+
+/* y = sum_i G(x)_i E_i(x)  ([SGMoE-note] "Sparsely-Gated MoE 层架构"),
+ * over the kept experts only.  A dropped slot adds nothing and the other
+ * gates are not renormalised (the pages are silent; plainest reading).  A
+ * token whose every slot overflowed passes through the residual
+ * ([MoE-deep] §3.2): our reading is that the layer's output for it is x.
+ *
+ * losses[0] L_importance = w_importance * CV(Importance)^2
+ * losses[1] L_load       = w_load * CV(Load)^2
+ * losses[2] N * sum_i f_i P_i  (Switch; f_i = routed fraction before the
+ *           capacity cut, P_i = mean router probability), 0 for router 0
+ * losses[3] alpha * losses[2]  ([MoE-deep] §3.2)
+ * losses[4] dropped slots / (T k)
+ * losses[5] CV(Importance)^2, losses[6] CV(Load)^2, losses[7] dropped slots
+ *
+ * Hierarchical layer ([SGMoE-note] "分层 MoE"): the primary gate picks k1
+ * groups, group i's own gate picks k2 of its b experts for the tokens sent
+ * to it; expert (i,j) has flat id i*b+j and gate G_p(x)_i * G_i(x)_j; slot
+ * order is primary slot major.  Losses (our reading, parity unpinned beyond
+ * the zero-noise limit): Importance over the a*b experts is the sum of the
+ * combined gates; Load(i*b+j) = Load_p(X)_i * Load_i(X_i)_j / |X_i|. */
+int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
+{
+  if (!valid_cfg(cfg)) return -1;
+  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f;
+  const int hier = cfg->hier_a > 0;
+  const int ng = hier ? (cfg->hier_a > cfg->hier_b ? cfg->hier_a : cfg->hier_b) : n;
+
+  double *c = (double *)malloc(sizeof(double) * (size_t)ng);
+  double *s = (double *)malloc(sizeof(double) * (size_t)ng);
+  double *P = (double *)malloc(sizeof(double) * (size_t)ng);
+  double *pr = (double *)malloc(sizeof(double) * (size_t)ng);
+  float *H = (float *)malloc(sizeof(float) * (size_t)ng);
+  int *order = (int *)malloc(sizeof(int) * (size_t)ng);
+  double *g1 = (double *)malloc(sizeof(double) * (size_t)(k + 1));
+  double *g2 = (double *)malloc(sizeof(double) * (size_t)(k + 1));
+  int *pidx = (int *)malloc(sizeof(int) * (size_t)(k + 1));
+
+  for (int e = 0; e < n; ++e) {
+    out->importance[e] = 0.0;
+    out->load[e] = 0.0;
+    if (out->prob_sum) out->prob_sum[e] = 0.0;
+  }
+
+  if (!hier) {
+    for (int t = 0; t < T; ++t) {
+      const float *xt = in->x + (size_t)t * d;
+      orc_gate_row(d, n, k, cfg->router, cfg->noise, cfg->seed, (uint32_t)t, 0u,
+                   xt, in->Wg, in->bg, in->Wn, c, s, H, order, g1, pr);
+      for (int j = 0; j < k; ++j) {
+        out->topk_idx[(size_t)t * k + j] = order[j];
+        out->topk_gate[(size_t)t * k + j] = g1[j];
+      }
+      orc_load_row(n, k, cfg->noise, c, s, H, P);
+      for (int i = 0; i < n; ++i) out->load[i] += P[i];
+      if (cfg->router == 1 && out->prob_sum)
+        for (int i = 0; i < n; ++i) out->prob_sum[i] += pr[i];
+      if (out->near_tie) out->near_tie[t] = min_gap(H, order, n, k);
+    }
+  } else {
+    const int a = cfg->hier_a, b = cfg->hier_b, k1 = cfg->hier_k1, k2 = cfg->hier_k2;
+    double *load_p = (double *)calloc((size_t)a, sizeof(double));
+    double *load_s = (double *)calloc((size_t)a * b, sizeof(double));
+    int64_t *cnt = (int64_t *)calloc((size_t)a, sizeof(int64_t));
+    for (int t = 0; t < T; ++t) {
+      const float *xt = in->x + (size_t)t * d;
+      orc_gate_row(d, a, k1, 0, cfg->noise, cfg->seed, (uint32_t)t, 0u, xt,
+                   in->Wg, in->bg, in->Wn, c, s, H, order, g1, NULL);
+      float gap = min_gap(H, order, a, k1);
+      orc_load_row(a, k1, cfg->noise, c, s, H, P);
+      for (int i = 0; i < a; ++i) load_p[i] += P[i];
+      for (int ps = 0; ps < k1; ++ps) pidx[ps] = order[ps];
+      for (int ps = 0; ps < k1; ++ps) {
+        int gi = pidx[ps];
+        cnt[gi]++;
+        const float *Wg2 = in->Wg2 + (size_t)gi * d * b;
+        const float *Wn2 = in->Wn2 ? in->Wn2 + (size_t)gi * d * b : NULL;
+        const float *bg2 = in->bg2 ? in->bg2 + (size_t)gi * b : NULL;
+        orc_gate_row(d, b, k2, 0, cfg->noise, cfg->seed, (uint32_t)t, (uint32_t)(1 + gi),
+                     xt, Wg2, bg2, Wn2, c, s, H, order, g2, NULL);
+        float gap2 = min_gap(H, order, b, k2);
+        if (gap2 < gap) gap = gap2;
+        orc_load_row(b, k2, cfg->noise, c, s, H, P);
+        for (int j = 0; j < b; ++j) load_s[(size_t)gi * b + j] += P[j];
+        for (int ss = 0; ss < k2; ++ss) {
+          size_t slot = (size_t)t * k + (size_t)ps * k2 + ss;
+          out->topk_idx[slot] = gi * b + order[ss];
+          out->topk_gate[slot] = g1[ps] * g2[ss];
+        }
+      }
+      if (out->near_tie) out->near_tie[t] = gap;
+    }
+    for (int i = 0; i < a; ++i)
+      for (int j = 0; j < b; ++j)
+        out->load[(size_t)i * b + j] =
+            cnt[i] > 0 ? load_p[i] * load_s[(size_t)i * b + j] / (double)cnt[i] : 0.0;
+    free(load_p); free(load_s); free(cnt);
+  }
+
+  /* Importance(X) = sum over the batch of G(x) ([SGMoE-xyz] "負載平衡損失"). */
+  for (int t = 0; t < T; ++t)
+    for (int j = 0; j < k; ++j)
+      out->importance[out->topk_idx[(size_t)t * k + j]] += out->topk_gate[(size_t)t * k + j];
+
+  /* dispatch with capacity */
+  int64_t C = orc_capacity(T, k, n, cfg->capacity_factor);
+  int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
+  size_t S = (size_t)T * k;
+  int32_t *perm_token = (int32_t *)malloc(sizeof(int32_t) * (S > 0 ? S : 1));
+  int32_t *perm_slot = (int32_t *)malloc(sizeof(int32_t) * (S > 0 ? S : 1));
+  orc_dispatch(T, k, n, C, out->topk_idx, out->counts, offsets, perm_token, perm_slot,
+               out->row_of, NULL);
+
+  /* experts and the gate-weighted sum */
+  double *ye = (double *)malloc(sizeof(double) * (size_t)d);
+  const size_t w1_stride = (size_t)f * d, w2_stride = (size_t)d * f;
+  const size_t esz = cfg->expert_bf16 ? 2 : 4;
+  int64_t dropped = 0;
+  for (int t = 0; t < T; ++t) {
+    double *yt = out->y + (size_t)t * d;
+    for (int q = 0; q < d; ++q) yt[q] = 0.0;
+    int kept_slots = 0;
+    for (int j = 0; j < k; ++j) {
+      size_t pj = (size_t)t * k + j;
+      if (out->row_of[pj] < 0) { dropped++; continue; }
+      kept_slots++;
+      int e = out->topk_idx[pj];
+      const char *W1e = (const char *)in->W1 + (size_t)e * w1_stride * esz;
+      const char *W2e = (const char *)in->W2 + (size_t)e * w2_stride * esz;
+      const float *b1e = in->b1 ? in->b1 + (size_t)e * f : NULL;
+      const float *b2e = in->b2 ? in->b2 + (size_t)e * d : NULL;
+      orc_expert_row(d, f, cfg->expert_bf16, in->x + (size_t)t * d, W1e, b1e, W2e, b2e, ye);
+      double g = out->topk_gate[pj];
+      for (int q = 0; q < d; ++q) yt[q] += g * ye[q];
+    }
+    if (kept_slots == 0 && k > 0 && cfg->passthrough)
+      for (int q = 0; q < d; ++q) yt[q] = (double)in->x[(size_t)t * d + q];
+  }
+
+  double cv2_imp = orc_cv2(out->importance, n);
+  double cv2_load = orc_cv2(out->load, n);
+  double aux = 0.0;
+  if (cfg->router == 1 && T > 0 && out->prob_sum) {
+    for (int i = 0; i < n; ++i)
+      aux += ((double)out->counts[i] / (double)T) * (out->prob_sum[i] / (double)T);
+    aux *= (double)n;
+  }
+  out->losses[0] = cfg->w_importance * cv2_imp;
+  out->losses[1] = cfg->w_load * cv2_load;
+  out->losses[2] = aux;
+  out->losses[3] = cfg->alpha * aux;
+  out->losses[4] = S > 0 ? (double)dropped / (double)S : 0.0;
+  out->losses[5] = cv2_imp;
+  out->losses[6] = cv2_load;
+  out->losses[7] = (double)dropped;
+
+  free(ye); free(offsets); free(perm_token); free(perm_slot);
+  free(c); free(s); free(P); free(pr); free(H); free(order); free(g1); free(g2); free(pidx);
+  return 0;
+}

@@ -1,0 +1,132 @@
+/*
+ * moe_oracle.h -- plain single-threaded CPU oracle for the forward pass of the
+ * Sparsely-Gated Mixture-of-Experts layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  This code exists to check the CUDA path; it is
+ * never part of the product path.  Only tests/, the smoke check and the
+ * bench's CPU-baseline leg may load it.  It shares no source, header, table or
+ * helper with the CUDA library: every formula below is written out again from
+ * the pages it cites.
+ *
+ * Arithmetic: fp64 accumulation everywhere.  Two results are deliberately
+ * taken in fp32 because an integer decision hangs on them and the kernel takes
+ * that decision in fp32: the gate logits H used for KeepTopK / argmax.
+ *
+ * Sources (page title, section):
+ *  [SGMoE-note]  "Outrageously Large Neural Networks: The Sparsely-Gated
+ *                Mixture-of-Experts Layer" reading note (chenshi221.pages.dev),
+ *                sections "Sparsely-Gated MoE 层架构", "Noisy Top-K Gating",
+ *                "负载均衡", "分层 MoE", "缺点与局限性".
+ *  [SGMoE-xyz]   "極大規模神經網路：稀疏門控專家混合層" (xyznot.com, arXiv
+ *                1701.06538), section "方法（與關鍵公式）": "Noisy Top-K 門控" and
+ *                "負載平衡損失".
+ *  [MoE-intro]   "MoE (Mixture-of-Experts) 算法介绍" (wkbse.com), "工作流程".
+ *  [MoE-deep]    "MoE 稀疏架构深度解析" (tufusi.com), §3.1 核心架构 and
+ *                §3.2 负载均衡问题.
+ *  [Philox]      Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
+ *                as 1, 2, 3", SC'11 (Philox4x32-10).
+ *  [Box-Muller]  Box & Muller, "A note on the generation of random normal
+ *                deviates", Ann. Math. Stat. 1958.
+ *
+ * Parity pins for every function are in tests/test_oracle_*.py.  Parity
+ * unpinned: the exact form of the hierarchical Load (the pages give the
+ * structure of the two-level gate but no formula for its balancing losses);
+ * it is pinned only through its zero-noise limit.
+ */
+#ifndef MOE_ORACLE_H
+#define MOE_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Layer description.  Flat layer: hier_a == 0.  Hierarchical layer: the
+ * primary gate picks hier_k1 of hier_a groups, each group's secondary gate
+ * picks hier_k2 of hier_b experts; then n must be hier_a*hier_b and
+ * k == hier_k1*hier_k2. */
+typedef struct {
+  int T, d, n, k, f;
+  int hier_a, hier_b, hier_k1, hier_k2;
+  int router;               /* 0: noisy top-k softmax gate; 1: Switch top-1 router */
+  int noise;                /* 1: add StandardNormal * Softplus(x W_noise)        */
+  uint64_t seed;
+  double capacity_factor;   /* <= 0: no capacity limit                           */
+  int passthrough;          /* 1: a token whose every slot overflowed gets y = x  */
+  int expert_bf16;          /* 1: expert weights and activations are bf16         */
+  double w_importance, w_load, alpha;
+} orc_cfg;
+
+/* ---- noise ------------------------------------------------------------ */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
+double orc_box_muller(uint32_t w0, uint32_t w1);
+double orc_noise(uint64_t seed, uint32_t token, uint32_t expert, uint32_t gate_id);
+
+/* ---- small helpers with a closed form ---------------------------------- */
+double orc_softplus(double z);
+double orc_phi(double z);
+double orc_cv2(const double *v, int n);
+float  orc_bf16_round(float v);
+int64_t orc_capacity(int T, int k, int n, double capacity_factor);
+
+/* ---- gate, one token (one row of the batch) ---------------------------- */
+/* x[d]; Wg, Wn: [d][n] row-major; bg: [n] or NULL; Wn may be NULL when noise
+ * is off.  Writes c[n] = (x Wg)+bg, s[n] = Softplus(x Wn) (0 if noise off),
+ * H[n] (fp32), order[n] = indices sorted by (H desc, index asc), gates[k]
+ * (softmax over the kept k for router 0; the full-softmax probability of the
+ * argmax for router 1, k must be 1) and, for router 1, p[n] (may be NULL). */
+void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
+                  uint32_t token, uint32_t gate_id, const float *x,
+                  const float *Wg, const float *bg, const float *Wn,
+                  double *c, double *s, float *H, int *order, double *gates,
+                  double *p);
+
+/* P(x,i) of the smoothed load estimator for every i, from one token's c, s
+ * and H (as written by orc_gate_row). */
+void orc_load_row(int n, int k, int noise, const double *c, const double *s,
+                  const float *H, double *P);
+
+/* ---- dispatch: stable expert-major permutation with capacity ------------ */
+/* idx[T][k] (any value outside [0,n) is ignored and counted in *n_invalid).
+ * counts[n] (before capacity), offsets[n+1] (exclusive scan of min(count,C)),
+ * perm_token/perm_slot[offsets[n]], row_of[T][k] (-1: dropped or invalid). */
+void orc_dispatch(int T, int k, int n, int64_t C, const int32_t *idx,
+                  int32_t *counts, int32_t *offsets, int32_t *perm_token,
+                  int32_t *perm_slot, int32_t *row_of, int64_t *n_invalid);
+
+/* ---- one expert applied to one token ----------------------------------- */
+/* W1: [f][d], b1: [f], W2: [d][f], b2: [d].  bf16 == 1: W1/W2 hold bf16 bit
+ * patterns (uint16), x and the hidden layer are rounded to bf16. */
+void orc_expert_row(int d, int f, int bf16, const float *x, const void *W1,
+                    const float *b1, const void *W2, const float *b2, double *y);
+
+/* ---- whole forward pass ------------------------------------------------- */
+typedef struct {
+  const float *x;                /* [T][d]                                    */
+  const float *Wg, *bg, *Wn;     /* flat/primary gate: [d][n'] , [n'], [d][n'] */
+  const float *Wg2, *bg2, *Wn2;  /* hierarchical secondary gates: [a][d][b], [a][b], [a][d][b] */
+  const void *W1; const float *b1;   /* [n][f][d], [n][f] */
+  const void *W2; const float *b2;   /* [n][d][f], [n][d] */
+} orc_inputs;
+
+typedef struct {
+  double *y;            /* [T][d]                                   */
+  int32_t *topk_idx;    /* [T][k]                                   */
+  double *topk_gate;    /* [T][k]                                   */
+  double *importance;   /* [n]                                      */
+  double *load;         /* [n]                                      */
+  double *prob_sum;     /* [n]   sum over tokens of the router softmax (router 1) */
+  int32_t *counts;      /* [n]                                      */
+  int32_t *row_of;      /* [T][k]                                   */
+  double *losses;       /* [8]   see orc_forward                    */
+  float *near_tie;      /* [T]   H_(k) - H_(k+1) of the deciding gate, or NULL */
+} orc_outputs;
+
+/* Returns 0 on success, -1 on an invalid configuration. */
+int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
