@@ -1,0 +1,256 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) forward pass of the Sparsely-Gated
+ * Mixture-of-Experts layer,  y = sum_i G(x)_i * E_i(x).
+ *
+ * Library: libmoe_b200.so.  Every entry point is `extern "C"`, takes plain
+ * pointers and sizes, returns an int status (MOE_OK = 0, negative = error)
+ * and is asynchronous on the given CUDA stream.
+ *
+ * Sources (page title, section), cited per entry point below:
+ *  [SGMoE-note] "Outrageously Large Neural Networks: The Sparsely-Gated
+ *               Mixture-of-Experts Layer" reading note (chenshi221.pages.dev),
+ *               "Sparsely-Gated MoE 层架构", "Noisy Top-K Gating", "负载均衡",
+ *               "分层 MoE".
+ *  [SGMoE-xyz]  "極大規模神經網路：稀疏門控專家混合層" (xyznot.com, arXiv
+ *               1701.06538), "方法（與關鍵公式）": "Noisy Top-K 門控",
+ *               "負載平衡損失".
+ *  [MoE-deep]   "MoE 稀疏架构深度解析" (tufusi.com), §3.1 核心架构,
+ *               §3.2 负载均衡问题.
+ *
+ * Conventions shared by every call
+ *  - Memory ownership: every pointer argument is caller-owned DEVICE memory
+ *    (the moe_config / parameter structs themselves are host memory and are
+ *    read during the call only).  The library allocates nothing; scratch
+ *    space is the caller's workspace `ws` of at least
+ *    moe_workspace_size() bytes, 256-byte aligned.
+ *  - Layouts are row-major.  x is [T][d] fp32.  Gate weights are stored as in
+ *    the pages' x*W products: W_g, W_noise are [d][n] fp32.  Expert weights
+ *    are stored K-major, as each linear map's [out][in]: W1 is [n][f][d],
+ *    W2 is [n][d][f], bf16 (MOE_BF16) or fp32 (MOE_F32); biases b1 [n][f],
+ *    b2 [n][d] are fp32 and may be NULL (zero).
+ *  - Alignment: every array pointer must be 16-byte aligned; d and f must be
+ *    multiples of 8.
+ *  - Routing slots: topk_idx / topk_gate are [T][k]; slot j of a token holds
+ *    its j-th largest noisy logit (ties: lower expert index first).
+ *  - Errors: argument problems are found on the host before any launch and
+ *    returned as MOE_EINVAL / MOE_EWORKSPACE; a failed launch returns
+ *    MOE_ECUDA.  Problems that only the device can see (a NaN logit, an
+ *    expert id out of range, a bounded wait that ran out) are OR-ed into the
+ *    caller's device word `*status` as MOE_STATUS_* bits; no kernel ever
+ *    traps.  The library never clears *status: the caller zeroes it and reads
+ *    it after synchronising.
+ *  - Determinism: for fixed inputs every output is bitwise reproducible
+ *    (fixed-order reductions, stable permutation).
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Every entry point is exported from the shared library. */
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+/* cudaStream_t without pulling in the CUDA headers. */
+typedef struct CUstream_st *moe_stream_t;
+
+enum {
+  MOE_OK = 0,
+  MOE_EINVAL = -1,      /* invalid configuration or NULL required pointer */
+  MOE_EWORKSPACE = -2,  /* workspace smaller than moe_workspace_size()    */
+  MOE_ECUDA = -3,       /* a CUDA call or kernel launch failed            */
+  MOE_EDEVICE = -4      /* no usable sm_100 device                        */
+};
+
+enum { MOE_ROUTER_NOISY_TOPK = 0, MOE_ROUTER_SWITCH = 1 };
+enum { MOE_F32 = 0, MOE_BF16 = 1 };
+
+/* bits OR-ed into *status by the kernels */
+enum {
+  MOE_STATUS_NONFINITE = 1,  /* a gate logit (or its noise scale) was NaN/Inf */
+  MOE_STATUS_BAD_INDEX = 2,  /* an expert id outside [0,n) was ignored        */
+  MOE_STATUS_TIMEOUT = 4,    /* a bounded on-chip wait gave up; outputs void  */
+  MOE_STATUS_OVERFLOW = 8    /* a size exceeded a kernel limit                */
+};
+
+/* Layer description.
+ *   T tokens, d model width, n experts, k experts per token, f hidden width.
+ *   Hierarchical layer ([SGMoE-note] "分层 MoE"): hier_a > 0 groups of hier_b
+ *   experts each; the primary gate keeps hier_k1 groups, each group's gate
+ *   keeps hier_k2 of its experts; then n = hier_a*hier_b, k = hier_k1*hier_k2.
+ *   router: MOE_ROUTER_NOISY_TOPK ([SGMoE-xyz] "Noisy Top-K 門控") or
+ *   MOE_ROUTER_SWITCH ([MoE-deep] §3.1: softmax over all experts, top-1, gate
+ *   = the winner's probability, no noise).
+ *   noise: 1 adds StandardNormal() * Softplus(x W_noise); the deviate for
+ *   (seed, token t, expert i, gate g) is the cosine branch of Box-Muller on
+ *   Philox4x32-10 words with key (seed lo, seed hi) and counter
+ *   (t, i/2, g, 0) -- words 0,1 for even i, words 2,3 for odd i; g = 0 for
+ *   the flat/primary gate and 1+group for a secondary gate.
+ *   capacity_factor > 0 limits every expert to C = ceil(T*k*cf/n) slots
+ *   ([MoE-deep] §3.2); slots beyond C (in token order) are dropped.
+ *   overflow_passthrough: 1 gives a token whose every slot was dropped the
+ *   output y = x (it "goes through the residual", [MoE-deep] §3.2).
+ *   w_importance, w_load: weights of the two CV^2 losses ([SGMoE-xyz]
+ *   "負載平衡損失"; 0.1 each in [SGMoE-note] "缺点与局限性"); alpha_aux: the
+ *   Switch loss coefficient ([MoE-deep] §3.2). */
+typedef struct moe_config {
+  int32_t T, d, n, k, f;
+  int32_t hier_a, hier_b, hier_k1, hier_k2;
+  int32_t router;
+  int32_t noise;
+  int32_t expert_dtype;       /* MOE_F32 or MOE_BF16 */
+  uint64_t seed;
+  double capacity_factor;
+  int32_t overflow_passthrough;
+  float w_importance, w_load, alpha_aux;
+  int32_t reserved;           /* must be 0 */
+} moe_config;
+
+/* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
+ * clean-logit bias, may be NULL).  Hierarchical layer: the same three for the
+ * primary gate over hier_a groups, plus the secondary gates W_g2, W_noise2
+ * [hier_a][d][hier_b] and b_g2 [hier_a][hier_b] (may be NULL).  W_noise /
+ * W_noise2 may be NULL when noise == 0. */
+typedef struct moe_gate_params {
+  const float *W_g, *b_g, *W_noise;
+  const float *W_g2, *b_g2, *W_noise2;
+} moe_gate_params;
+
+/* Expert parameters: W1 [n][f][d], W2 [n][d][f] of expert_dtype; b1 [n][f],
+ * b2 [n][d] fp32 or NULL. */
+typedef struct moe_expert_params {
+  const void *W1;
+  const float *b1;
+  const void *W2;
+  const float *b2;
+} moe_expert_params;
+
+/* Text for a return code. */
+MOE_API const char *moe_strerror(int code);
+
+/* Validates cfg.  MOE_OK or MOE_EINVAL.  Limits: T >= 0, 1 <= k <= min(n,8),
+ * 1 <= n <= 8192, d, f multiples of 8, d <= 16384, f <= 65536; Switch router:
+ * k = 1, no noise, n <= 4096, flat only. */
+MOE_API int moe_validate(const moe_config *cfg);
+
+/* Expert capacity C = ceil(T*k*capacity_factor/n), or INT64_MAX when
+ * capacity_factor <= 0 ([MoE-deep] §3.2: C = tokens per batch / E * factor;
+ * with k slots per token the routed slots are T*k). */
+MOE_API int moe_capacity(const moe_config *cfg, int64_t *C);
+
+/* Bytes of workspace that every call below accepts for this cfg (the same
+ * number for every entry point; moe_forward needs all of it). */
+MOE_API int moe_workspace_size(const moe_config *cfg, size_t *bytes);
+
+/* ---------------------------------------------------------------- steps */
+
+/* Gate: H(x)_i = (x W_g)_i + b_g,i + StandardNormal()*Softplus((x W_noise)_i),
+ * KeepTopK(H, k), G(x) = Softmax(KeepTopK(H, k))  ([SGMoE-xyz] "Noisy Top-K
+ * 門控"; [SGMoE-note] "Noisy Top-K Gating"); Switch router per [MoE-deep]
+ * §3.1; hierarchical gate per [SGMoE-note] "分层 MoE" (slot ps*k2+ss holds
+ * expert g*b+j with gate G_p(x)_g * G_g(x)_j, g the ps-th kept group).
+ * Outputs: topk_idx [T][k] int32, topk_gate [T][k] fp32,
+ *   load [n]: the smoothed load Load(X)_i = sum_x P(x,i),
+ *     P(x,i) = Phi(((x W_g)_i - kth_excluding(H(x),k,i)) / Softplus((x W_noise)_i))
+ *     ([SGMoE-xyz] "負載平衡損失"); without noise its zero-noise limit, the
+ *     number of tokens that keep expert i.  Hierarchical: Load_p(X)_g *
+ *     Load_g(X_g)_j / |X_g| for expert g*b+j, 0 for an empty group.
+ *   prob_sum [n] (may be NULL): sum over tokens of the Switch router's
+ *     softmax (zeros for the noisy gate).
+ * Errors: MOE_EINVAL for a NULL x / W_g / outputs (or W_noise with noise on,
+ * W_g2 for a hierarchical cfg). */
+MOE_API int moe_gate(const moe_config *cfg, const float *x, const moe_gate_params *gp,
+             int32_t *topk_idx, float *topk_gate, float *load, float *prob_sum,
+             void *ws, size_t ws_bytes, int32_t *status, moe_stream_t stream);
+
+/* Dispatch: E_i(x) is only evaluated where G(x)_i != 0 ([SGMoE-note]
+ * "Sparsely-Gated MoE 层架构"), so every (token, slot) pair goes to its
+ * expert.  Pairs are taken in (token, slot) order; the r-th pair of expert e
+ * is kept iff r < C ([MoE-deep] §3.2) and lands in row offsets[e] + r.
+ * Outputs: counts [n] (pairs per expert before the capacity cut), offsets
+ * [n+1] (exclusive scan of min(count, C)), perm_token [T*k] (token of every
+ * kept row; rows >= offsets[n] untouched), row_of [T][k] (row of a kept
+ * pair, -1 if dropped or its id was out of range -- the latter also sets
+ * MOE_STATUS_BAD_INDEX), x_perm [T*k][d] (x rows gathered into the kept rows,
+ * cast to expert_dtype; may be NULL together with x to skip the gather). */
+MOE_API int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *topk_idx,
+                 int32_t *counts, int32_t *offsets, int32_t *perm_token,
+                 int32_t *row_of, void *x_perm, void *ws, size_t ws_bytes,
+                 int32_t *status, moe_stream_t stream);
+
+/* Expert FFN on the expert-contiguous rows: rows offsets[e] .. offsets[e+1]-1
+ * of x_perm go through expert e ([SGMoE-note] "Sparsely-Gated MoE 层架构":
+ * one hidden ReLU layer):  y_perm = ReLU(x_perm W1_e^T + b1_e) W2_e^T + b2_e.
+ * bf16 experts: bf16 operands, fp32 accumulation (tcgen05 tensor cores), the
+ * hidden layer rounded to bf16, y_perm written as bf16.  fp32 experts: fp32
+ * throughout.  x_perm, y_perm: [T*k][d] of expert_dtype. */
+MOE_API int moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                   const moe_expert_params *ep, void *y_perm, void *ws,
+                   size_t ws_bytes, int32_t *status, moe_stream_t stream);
+
+/* Combine: y_t = sum_j topk_gate[t][j] * y_perm[row_of[t][j]] over the kept
+ * slots j (in slot order) ([SGMoE-note] "Sparsely-Gated MoE 层架构": y = sum_i
+ * G(x)_i E_i(x)).  A dropped slot adds nothing (gates are not renormalised);
+ * with overflow_passthrough a token with no kept slot gets y_t = x_t
+ * ([MoE-deep] §3.2), otherwise 0.  y: [T][d] fp32; x may be NULL without
+ * pass-through. */
+MOE_API int moe_combine(const moe_config *cfg, const void *y_perm, const float *topk_gate,
+                const int32_t *row_of, const float *x, float *y, int32_t *status,
+                moe_stream_t stream);
+
+/* Balancing statistics ([SGMoE-xyz] "負載平衡損失"; [MoE-deep] §3.2).
+ * importance [n]: Importance(X)_i = sum_x G(x)_i.
+ * losses [8]:
+ *   [0] L_importance = w_importance * CV(Importance)^2
+ *   [1] L_load       = w_load * CV(load)^2
+ *   [2] N * sum_i f_i P_i  (Switch: f_i = counts_i / T before the capacity
+ *       cut, P_i = prob_sum_i / T); 0 for the noisy gate
+ *   [3] alpha_aux * [2]
+ *   [4] dropped slots / (T*k),   [5] CV(Importance)^2,   [6] CV(load)^2,
+ *   [7] dropped slots
+ * CV^2 is the population variance over the squared mean (0 for a zero
+ * mean), evaluated in fp64.  counts and load come from moe_dispatch /
+ * moe_gate; prob_sum may be NULL for the noisy gate. */
+MOE_API int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx,
+                       const float *topk_gate, const int32_t *counts,
+                       const float *load, const float *prob_sum, float *importance,
+                       float *losses, void *ws, size_t ws_bytes, int32_t *status,
+                       moe_stream_t stream);
+
+/* ---------------------------------------------------------------- fused */
+
+/* The whole layer on one stream: gate, dispatch, experts, combine and the
+ * balancing statistics, every intermediate in ws.  Outputs as the step calls
+ * above: y [T][d], topk_idx, topk_gate [T][k], importance, load [n],
+ * counts [n], losses [8]. */
+MOE_API int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
+                const moe_expert_params *ep, float *y, int32_t *topk_idx,
+                float *topk_gate, float *importance, float *load, int32_t *counts,
+                float *losses, void *ws, size_t ws_bytes, int32_t *status,
+                moe_stream_t stream);
+
+/* ---------------------------------------------------------------- tracing */
+
+/* Per-kernel timing with CUDA events recorded around every launch on its own
+ * stream.  Off by default.  moe_trace_count/get synchronise on the recorded
+ * events and report, per kernel name, the launches and total milliseconds
+ * since the last reset.  moe_launch_count counts every kernel the library
+ * launched since load (tracing on or off).  Not thread-safe. */
+MOE_API int moe_trace_enable(int on);
+MOE_API int moe_trace_reset(void);
+MOE_API int moe_trace_count(void);
+MOE_API int moe_trace_get(int i, const char **name, int *launches, double *total_ms);
+MOE_API long long moe_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MOE_B200_H */

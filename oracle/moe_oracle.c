@@ -367,30 +367,22 @@ static int valid_cfg(const orc_cfg *c)
   return 1;
 }
 
-/* y = sum_i G(x)_i E_i(x)  ([SGMoE-note] "Sparsely-Gated MoE 层架构"),
- * over the kept experts only.  A dropped slot adds nothing and the other
- * gates are not renormalised (the pages are silent; plainest reading).  A
- * token whose every slot overflowed passes through the residual
- * ([MoE-deep] §3.2): our reading is that the layer's output for it is x.
- *
- * losses[0] L_importance = w_importance * CV(Importance)^2
- * losses[1] L_load       = w_load * CV(Load)^2
- * losses[2] N * sum_i f_i P_i  (Switch; f_i = routed fraction before the
- *           capacity cut, P_i = mean router probability), 0 for router 0
- * losses[3] alpha * losses[2]  ([MoE-deep] §3.2)
- * losses[4] dropped slots / (T k)
- * losses[5] CV(Importance)^2, losses[6] CV(Load)^2, losses[7] dropped slots
+/* Gate over a whole batch (flat, Switch or hierarchical): topk_idx /
+ * topk_gate [T][k], load [n] (smoothed load, or its zero-noise limit),
+ * prob_sum [n] (Switch: sum of router probabilities; else 0), near_tie [T]
+ * (smallest gap between neighbouring sorted logits among the first k+1 of any
+ * gate that decided the token; may be NULL).
  *
  * Hierarchical layer ([SGMoE-note] "分层 MoE"): the primary gate picks k1
  * groups, group i's own gate picks k2 of its b experts for the tokens sent
  * to it; expert (i,j) has flat id i*b+j and gate G_p(x)_i * G_i(x)_j; slot
- * order is primary slot major.  Losses (our reading, parity unpinned beyond
- * the zero-noise limit): Importance over the a*b experts is the sum of the
- * combined gates; Load(i*b+j) = Load_p(X)_i * Load_i(X_i)_j / |X_i|. */
-int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
+ * order is primary slot major.  Load (our reading, parity unpinned beyond
+ * the zero-noise limit): Load(i*b+j) = Load_p(X)_i * Load_i(X_i)_j / |X_i|. */
+int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
+                   double *topk_gate, double *load, double *prob_sum, float *near_tie)
 {
   if (!valid_cfg(cfg)) return -1;
-  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f;
+  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k;
   const int hier = cfg->hier_a > 0;
   const int ng = hier ? (cfg->hier_a > cfg->hier_b ? cfg->hier_a : cfg->hier_b) : n;
 
@@ -405,9 +397,8 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
   int *pidx = (int *)malloc(sizeof(int) * (size_t)(k + 1));
 
   for (int e = 0; e < n; ++e) {
-    out->importance[e] = 0.0;
-    out->load[e] = 0.0;
-    if (out->prob_sum) out->prob_sum[e] = 0.0;
+    load[e] = 0.0;
+    if (prob_sum) prob_sum[e] = 0.0;
   }
 
   if (!hier) {
@@ -416,14 +407,14 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
       orc_gate_row(d, n, k, cfg->router, cfg->noise, cfg->seed, (uint32_t)t, 0u,
                    xt, in->Wg, in->bg, in->Wn, c, s, H, order, g1, pr);
       for (int j = 0; j < k; ++j) {
-        out->topk_idx[(size_t)t * k + j] = order[j];
-        out->topk_gate[(size_t)t * k + j] = g1[j];
+        topk_idx[(size_t)t * k + j] = order[j];
+        topk_gate[(size_t)t * k + j] = g1[j];
       }
       orc_load_row(n, k, cfg->noise, c, s, H, P);
-      for (int i = 0; i < n; ++i) out->load[i] += P[i];
-      if (cfg->router == 1 && out->prob_sum)
-        for (int i = 0; i < n; ++i) out->prob_sum[i] += pr[i];
-      if (out->near_tie) out->near_tie[t] = min_gap(H, order, n, k);
+      for (int i = 0; i < n; ++i) load[i] += P[i];
+      if (cfg->router == 1 && prob_sum)
+        for (int i = 0; i < n; ++i) prob_sum[i] += pr[i];
+      if (near_tie) near_tie[t] = min_gap(H, order, n, k);
     }
   } else {
     const int a = cfg->hier_a, b = cfg->hier_b, k1 = cfg->hier_k1, k2 = cfg->hier_k2;
@@ -452,25 +443,100 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
         for (int j = 0; j < b; ++j) load_s[(size_t)gi * b + j] += P[j];
         for (int ss = 0; ss < k2; ++ss) {
           size_t slot = (size_t)t * k + (size_t)ps * k2 + ss;
-          out->topk_idx[slot] = gi * b + order[ss];
-          out->topk_gate[slot] = g1[ps] * g2[ss];
+          topk_idx[slot] = gi * b + order[ss];
+          topk_gate[slot] = g1[ps] * g2[ss];
         }
       }
-      if (out->near_tie) out->near_tie[t] = gap;
+      if (near_tie) near_tie[t] = gap;
     }
     for (int i = 0; i < a; ++i)
       for (int j = 0; j < b; ++j)
-        out->load[(size_t)i * b + j] =
+        load[(size_t)i * b + j] =
             cnt[i] > 0 ? load_p[i] * load_s[(size_t)i * b + j] / (double)cnt[i] : 0.0;
     free(load_p); free(load_s); free(cnt);
   }
+  free(c); free(s); free(P); free(pr); free(H); free(order); free(g1); free(g2); free(pidx);
+  return 0;
+}
 
-  /* Importance(X) = sum over the batch of G(x) ([SGMoE-xyz] "負載平衡損失"). */
+/* Gate-weighted sum of expert rows, y = sum_i G(x)_i E_i(x) ([SGMoE-note]
+ * "Sparsely-Gated MoE 层架构"), with E_i(x) already computed as row
+ * row_of[t][j] of Y.  A dropped slot (row -1) adds nothing and the other
+ * gates are not renormalised (the pages are silent; plainest reading).  A
+ * token whose every slot was dropped passes through the residual ([MoE-deep]
+ * §3.2): with passthrough its output is x, else 0. */
+void orc_combine(int T, int k, int d, const double *Y, const double *gate,
+                 const int32_t *row_of, const float *x, int passthrough, double *y)
+{
+  for (int t = 0; t < T; ++t) {
+    double *yt = y + (size_t)t * d;
+    for (int q = 0; q < d; ++q) yt[q] = 0.0;
+    int kept = 0;
+    for (int j = 0; j < k; ++j) {
+      int32_t r = row_of[(size_t)t * k + j];
+      if (r < 0) continue;
+      kept++;
+      double g = gate[(size_t)t * k + j];
+      for (int q = 0; q < d; ++q) yt[q] += g * Y[(size_t)r * d + q];
+    }
+    if (kept == 0 && passthrough)
+      for (int q = 0; q < d; ++q) yt[q] = (double)x[(size_t)t * d + q];
+  }
+}
+
+/* Balancing statistics ([SGMoE-xyz] "負載平衡損失"; [MoE-deep] §3.2):
+ * importance[i] = sum over tokens of G(x)_i (from the kept-expert lists);
+ * losses[0] L_importance = w_importance * CV(Importance)^2
+ * losses[1] L_load       = w_load * CV(Load)^2
+ * losses[2] N * sum_i f_i P_i  (Switch; f_i = counts_i / T, before the
+ *           capacity cut, P_i = prob_sum_i / T), 0 for router 0
+ * losses[3] alpha * losses[2]
+ * losses[4] dropped slots / (T k)  (dropped = sum_i max(counts_i - C, 0))
+ * losses[5] CV(Importance)^2, losses[6] CV(Load)^2, losses[7] dropped slots */
+void orc_balance(int n, int T, int k, const int32_t *topk_idx, const double *topk_gate,
+                 const int32_t *counts, const double *load, const double *prob_sum,
+                 int64_t C, int router, double w_importance, double w_load, double alpha,
+                 double *importance, double *losses)
+{
+  for (int e = 0; e < n; ++e) importance[e] = 0.0;
   for (int t = 0; t < T; ++t)
-    for (int j = 0; j < k; ++j)
-      out->importance[out->topk_idx[(size_t)t * k + j]] += out->topk_gate[(size_t)t * k + j];
+    for (int j = 0; j < k; ++j) {
+      int32_t e = topk_idx[(size_t)t * k + j];
+      if (e >= 0 && e < n) importance[e] += topk_gate[(size_t)t * k + j];
+    }
+  double dropped = 0.0;
+  for (int e = 0; e < n; ++e)
+    if ((int64_t)counts[e] > C) dropped += (double)((int64_t)counts[e] - C);
+  double aux = 0.0;
+  if (router == 1 && T > 0 && prob_sum) {
+    for (int i = 0; i < n; ++i)
+      aux += ((double)counts[i] / (double)T) * (prob_sum[i] / (double)T);
+    aux *= (double)n;
+  }
+  double cv2_imp = orc_cv2(importance, n);
+  double cv2_load = orc_cv2(load, n);
+  double S = (double)T * (double)k;
+  losses[0] = w_importance * cv2_imp;
+  losses[1] = w_load * cv2_load;
+  losses[2] = aux;
+  losses[3] = alpha * aux;
+  losses[4] = S > 0 ? dropped / S : 0.0;
+  losses[5] = cv2_imp;
+  losses[6] = cv2_load;
+  losses[7] = dropped;
+}
 
-  /* dispatch with capacity */
+/* The whole layer, y = sum_i G(x)_i E_i(x) over the kept experts
+ * ([SGMoE-note] "Sparsely-Gated MoE 层架构"): gate, capacity-limited
+ * dispatch, each kept expert applied to the token directly, gate-weighted
+ * sum, pass-through of fully dropped tokens, balancing statistics.  Losses
+ * as in orc_balance. */
+int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
+{
+  if (orc_gate_batch(cfg, in, out->topk_idx, out->topk_gate, out->load, out->prob_sum,
+                     out->near_tie) != 0)
+    return -1;
+  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f;
   int64_t C = orc_capacity(T, k, n, cfg->capacity_factor);
   int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
   size_t S = (size_t)T * k;
@@ -479,18 +545,16 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
   orc_dispatch(T, k, n, C, out->topk_idx, out->counts, offsets, perm_token, perm_slot,
                out->row_of, NULL);
 
-  /* experts and the gate-weighted sum */
   double *ye = (double *)malloc(sizeof(double) * (size_t)d);
   const size_t w1_stride = (size_t)f * d, w2_stride = (size_t)d * f;
   const size_t esz = cfg->expert_bf16 ? 2 : 4;
-  int64_t dropped = 0;
   for (int t = 0; t < T; ++t) {
     double *yt = out->y + (size_t)t * d;
     for (int q = 0; q < d; ++q) yt[q] = 0.0;
     int kept_slots = 0;
     for (int j = 0; j < k; ++j) {
       size_t pj = (size_t)t * k + j;
-      if (out->row_of[pj] < 0) { dropped++; continue; }
+      if (out->row_of[pj] < 0) continue;
       kept_slots++;
       int e = out->topk_idx[pj];
       const char *W1e = (const char *)in->W1 + (size_t)e * w1_stride * esz;
@@ -505,24 +569,9 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
       for (int q = 0; q < d; ++q) yt[q] = (double)in->x[(size_t)t * d + q];
   }
 
-  double cv2_imp = orc_cv2(out->importance, n);
-  double cv2_load = orc_cv2(out->load, n);
-  double aux = 0.0;
-  if (cfg->router == 1 && T > 0 && out->prob_sum) {
-    for (int i = 0; i < n; ++i)
-      aux += ((double)out->counts[i] / (double)T) * (out->prob_sum[i] / (double)T);
-    aux *= (double)n;
-  }
-  out->losses[0] = cfg->w_importance * cv2_imp;
-  out->losses[1] = cfg->w_load * cv2_load;
-  out->losses[2] = aux;
-  out->losses[3] = cfg->alpha * aux;
-  out->losses[4] = S > 0 ? (double)dropped / (double)S : 0.0;
-  out->losses[5] = cv2_imp;
-  out->losses[6] = cv2_load;
-  out->losses[7] = (double)dropped;
-
+  orc_balance(n, T, k, out->topk_idx, out->topk_gate, out->counts, out->load, out->prob_sum, C,
+              cfg->router, cfg->w_importance, cfg->w_load, cfg->alpha, out->importance,
+              out->losses);
   free(ye); free(offsets); free(perm_token); free(perm_slot);
-  free(c); free(s); free(P); free(pr); free(H); free(order); free(g1); free(g2); free(pidx);
   return 0;
 }

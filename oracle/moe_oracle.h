@@ -123,6 +123,21 @@ typedef struct {
   float *near_tie;      /* [T]   H_(k) - H_(k+1) of the deciding gate, or NULL */
 } orc_outputs;
 
+/* Gate over a whole batch: topk_idx / topk_gate [T][k], load [n],
+ * prob_sum [n] (may be NULL), near_tie [T] (may be NULL).  0 or -1. */
+int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
+                   double *topk_gate, double *load, double *prob_sum, float *near_tie);
+
+/* y[T][d] from expert rows Y[*][d] (row_of[T][k], -1 = dropped). */
+void orc_combine(int T, int k, int d, const double *Y, const double *gate,
+                 const int32_t *row_of, const float *x, int passthrough, double *y);
+
+/* importance [n] and losses [8] from routing, counts, load, prob_sum. */
+void orc_balance(int n, int T, int k, const int32_t *topk_idx, const double *topk_gate,
+                 const int32_t *counts, const double *load, const double *prob_sum,
+                 int64_t C, int router, double w_importance, double w_load, double alpha,
+                 double *importance, double *losses);
+
 /* Returns 0 on success, -1 on an invalid configuration. */
 int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
 

@@ -83,6 +83,11 @@ def lib():
         L.orc_load_row.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.orc_dispatch.argtypes = [i32, i32, i32, C.c_int64, vp, vp, vp, vp, vp, vp, vp]
         L.orc_expert_row.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
+        L.orc_gate_batch.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, vp, vp, vp, vp]
+        L.orc_gate_batch.restype = i32
+        L.orc_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp]
+        L.orc_balance.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, C.c_int64, i32, f64, f64, f64,
+                                  vp, vp]
         L.orc_forward.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), C.POINTER(OrcOutputs)]
         L.orc_forward.restype = i32
         _lib = L
@@ -198,19 +203,59 @@ def make_cfg(**kw) -> OrcCfg:
     return OrcCfg(**{k: base[k] for k in _CFG_KEYS})
 
 
-def forward(cfg: dict, inp: dict) -> dict:
-    """Run the whole layer.  ``cfg`` holds the fields of ``OrcCfg``; ``inp``
-    holds numpy arrays x, Wg, bg, Wn, Wg2, bg2, Wn2, W1, b1, W2, b2 (bf16
-    expert weights as uint16 bit patterns)."""
-    oc = make_cfg(**cfg)
-    T, d, n, k = oc.T, oc.d, oc.n, oc.k
+def _inputs(oc, inp):
     wdt = np.uint16 if oc.expert_bf16 else np.float32
     keep = {}
     for name, dt in (("x", np.float32), ("Wg", np.float32), ("bg", np.float32), ("Wn", np.float32),
                      ("Wg2", np.float32), ("bg2", np.float32), ("Wn2", np.float32),
                      ("W1", wdt), ("b1", np.float32), ("W2", wdt), ("b2", np.float32)):
         keep[name] = _c(inp.get(name), dt)
-    ins = OrcInputs(**{name: _p(a) for name, a in keep.items()})
+    return keep, OrcInputs(**{name: _p(a) for name, a in keep.items()})
+
+
+def gate_batch(cfg: dict, inp: dict) -> dict:
+    """Gate of the whole batch (flat, Switch or hierarchical); expert weights
+    are not needed."""
+    oc = make_cfg(**cfg)
+    keep, ins = _inputs(oc, inp)
+    T, n, k = oc.T, oc.n, oc.k
+    out = dict(topk_idx=np.zeros((T, k), np.int32), topk_gate=np.zeros((T, k)), load=np.zeros(n),
+               prob_sum=np.zeros(n), near_tie=np.zeros(T, np.float32))
+    rc = lib().orc_gate_batch(C.byref(oc), C.byref(ins), _p(out["topk_idx"]), _p(out["topk_gate"]),
+                              _p(out["load"]), _p(out["prob_sum"]), _p(out["near_tie"]))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the configuration {cfg}")
+    return out
+
+
+def combine(Y, gate, row_of, x=None, passthrough=False) -> np.ndarray:
+    Y = _c(Y, np.float64); gate = _c(gate, np.float64); row_of = _c(row_of, np.int32)
+    T, k = row_of.shape
+    d = Y.shape[1]
+    x = _c(x, np.float32)
+    y = np.zeros((T, d))
+    lib().orc_combine(T, k, d, _p(Y), _p(gate), _p(row_of), _p(x), int(bool(passthrough)), _p(y))
+    return y
+
+
+def balance(n, topk_idx, topk_gate, counts, load, prob_sum=None, C=2**63 - 1, router=0,
+            w_importance=0.1, w_load=0.1, alpha=0.01):
+    idx = _c(topk_idx, np.int32); g = _c(topk_gate, np.float64)
+    T, k = idx.shape
+    counts = _c(counts, np.int32); load = _c(load, np.float64); ps = _c(prob_sum, np.float64)
+    imp = np.zeros(n); losses = np.zeros(8)
+    lib().orc_balance(n, T, k, _p(idx), _p(g), _p(counts), _p(load), _p(ps), C, router,
+                      w_importance, w_load, alpha, _p(imp), _p(losses))
+    return imp, losses
+
+
+def forward(cfg: dict, inp: dict) -> dict:
+    """Run the whole layer.  ``cfg`` holds the fields of ``OrcCfg``; ``inp``
+    holds numpy arrays x, Wg, bg, Wn, Wg2, bg2, Wn2, W1, b1, W2, b2 (bf16
+    expert weights as uint16 bit patterns)."""
+    oc = make_cfg(**cfg)
+    T, d, n, k = oc.T, oc.d, oc.n, oc.k
+    keep, ins = _inputs(oc, inp)
     out = dict(y=np.zeros((T, d)), topk_idx=np.zeros((T, k), np.int32), topk_gate=np.zeros((T, k)),
                importance=np.zeros(n), load=np.zeros(n), prob_sum=np.zeros(n),
                counts=np.zeros(n, np.int32), row_of=np.zeros((T, k), np.int32),

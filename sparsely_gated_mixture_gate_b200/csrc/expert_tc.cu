@@ -1,0 +1,433 @@
+// expert_tc.cu -- the experts' two dense contractions on the 5th-generation
+// tensor cores (tcgen05, accumulators in tensor memory, operands by TMA).
+//
+// [SGMoE-note] "Sparsely-Gated MoE 层架构": every expert is a feed-forward
+// network with one ReLU hidden layer.  With the kept rows of expert e stored
+// contiguously (rows offsets[e] .. offsets[e+1]-1 of x_perm):
+//   GEMM1: hid    = ReLU(x_perm_e W1_e^T + b1_e)   (bf16 out)
+//   GEMM2: y_perm = hid_e W2_e^T + b2_e            (bf16 out)
+// Both are "grouped" GEMMs with a ragged M per expert and K-major operands.
+//
+// One persistent kernel, one CTA per SM, 192 threads:
+//   warp 0  TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte
+//           swizzle), 4 stages, mbarrier transaction counts
+//   warp 1  MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128,
+//           N=256, K=16, four per stage; tcgen05.commit frees the stage
+//   warps 2-5  epilogue: tcgen05.ld of the 128x256 fp32 accumulator, bias,
+//           ReLU, bf16, masked stores of the expert's valid rows
+// Two accumulators of 256 columns (all 512 TMEM columns) let the epilogue of
+// one tile overlap the main loop of the next.  Tiles are ordered expert by
+// expert, N-block by N-block, M-block fastest, so the M-blocks that share a
+// weight tile run at the same time and the weights stream from HBM once.
+// No cluster multicast anywhere.
+//
+// Every mbarrier wait is bounded (about two seconds of %globaltimer); a wait
+// that runs out sets MOE_STATUS_TIMEOUT, raises an abort flag seen by the
+// other roles, drains the copies and MMAs this CTA issued (again bounded),
+// frees its tensor memory and returns.
+#include <cuda.h>
+
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kExpertBM, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;
+constexpr int B_BYTES = BN * BK * 2;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int NUM_THREADS = 192;
+constexpr uint32_t TMEM_COLS = 2 * BN;
+constexpr int BAR_BYTES = 256;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+constexpr unsigned long long kWaitNs = 2000000000ull;
+
+// instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
+// = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N>>3 at bits
+// 17-22, M>>4 at bits 24-28.
+constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
+                           ((uint32_t)(BM >> 4) << 24);
+
+struct TcArgs {
+  const int *offsets;
+  const int *mprefix;
+  int n, N, K, nblk;
+  const float *bias;     // [n][N] or nullptr
+  __nv_bfloat16 *D;      // [S][N]
+  int relu;
+  int *status;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return (uint32_t)__cvta_generic_to_shared(p);
+}
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+__device__ __forceinline__ unsigned long long globaltimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+// Bounded wait for the phase with the given parity.  false: gave up (time
+// limit, or another role raised the abort flag).
+__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
+                                       unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0u) {
+      if (abort_flag && *abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                       uint32_t accum) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   bar)
+               : "memory");
+}
+
+// Shared-memory matrix descriptor of a K-major tile in the 128-byte swizzle
+// layout that TMA writes: rows of 128 bytes, atoms of 8 rows (1024 bytes)
+// stacked at a stride of 1024 bytes.  Fields: start address >> 4 (bits
+// 0-13), leading byte offset >> 4 (bits 16-29; not used by swizzled K-major
+// layouts, set to 1), stride byte offset >> 4 (bits 32-45), version 1 (bits
+// 46-47), swizzle mode 2 = 128-byte (bits 61-63).
+__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
+  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
+         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// tile -> (expert, M-block, N-block); tiles of expert e are
+// [mprefix[e]*nblk, mprefix[e+1]*nblk), N-block major, M-block minor.
+__device__ __forceinline__ void decode_tile(const TcArgs &a, int tile, int &e, int &mb, int &nbk) {
+  const int v = tile / a.nblk;
+  int lo = 0, hi = a.n - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (__ldg(a.mprefix + mid) <= v) lo = mid; else hi = mid - 1;
+  }
+  e = lo;
+  const int base = __ldg(a.mprefix + e);
+  const int mbe = __ldg(a.mprefix + e + 1) - base;
+  const int local = tile - base * a.nblk;
+  nbk = local / mbe;
+  mb = local - nbk * mbe;
+}
+
+__global__ void __launch_bounds__(NUM_THREADS, 1)
+    expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + STAGES * STAGE_BYTES);
+  // bars: full[STAGES] empty[STAGES] tfull[2] tempty[2] drain[1]
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 5);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  const uint32_t bar0 = smem_u32(bars);
+  auto full = [&](int s) { return bar0 + 8u * s; };
+  auto empty = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull = [&](int c) { return bar0 + 8u * (2 * STAGES + c); };
+  auto tempty = [&](int c) { return bar0 + 8u * (2 * STAGES + 2 + c); };
+  const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
+  const uint32_t sbase = smem_u32(smem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full(s), 1);
+      mbar_init(empty(s), 1);
+    }
+    for (int c = 0; c < 2; ++c) {
+      mbar_init(tfull(c), 1);
+      mbar_init(tempty(c), 128);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_slot)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int total = __ldg(a.mprefix + a.n) * a.nblk;
+  const int nkb = (a.K + BK - 1) / BK;
+  bool failed = false;
+
+  if (warp == 0 && lane == 0) {
+    // ------------------------------------------------ TMA producer
+    int stage = 0;
+    uint32_t phase = 0;
+    int issued[STAGES];
+    for (int s = 0; s < STAGES; ++s) issued[s] = -1;
+    for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      int e, mb, nbk;
+      decode_tile(a, tile, e, mb, nbk);
+      const int row0 = __ldg(a.offsets + e) + mb * BM;
+      const int brow = e * a.N + nbk * BN;
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
+        const uint32_t sa = sbase + stage * STAGE_BYTES;
+        mbar_expect_tx(full(stage), STAGE_BYTES);
+        tma_load_2d(sa, &tmA, full(stage), kb * BK, row0);
+        tma_load_2d(sa + A_BYTES, &tmB, full(stage), kb * BK, brow);
+        issued[stage] = (int)phase;
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+    }
+    if (failed || *abort_flag) {
+      *abort_flag = 1;
+      // let the copies this thread started land before the CTA exits
+      for (int s = 0; s < STAGES; ++s)
+        if (issued[s] >= 0) mbar_wait(full(s), (uint32_t)issued[s], nullptr, 100000000ull);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ------------------------------------------------ MMA issuer
+    int stage = 0, acc = 0;
+    uint32_t phase = 0, acc_phase = 0;
+    bool issued_any = false;
+    for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      if (!mbar_wait(tempty(acc), acc_phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
+      for (int kb = 0; kb < nkb; ++kb) {
+        if (!mbar_wait(full(stage), phase, abort_flag, kWaitNs)) { failed = true; break; }
+        tc_fence_after();
+        const uint32_t sa = sbase + stage * STAGE_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / 16; ++kk)
+          tc_mma(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sa + A_BYTES + kk * 32),
+                 (kb | kk) != 0);
+        issued_any = true;
+        tc_commit(empty(stage));
+        if (++stage == STAGES) { stage = 0; phase ^= 1u; }
+      }
+      if (failed) break;
+      tc_commit(tfull(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (failed || *abort_flag) {
+      *abort_flag = 1;
+      if (issued_any) {  // wait until every MMA issued so far has finished
+        tc_commit(drain);
+        mbar_wait(drain, 0u, nullptr, 100000000ull);
+      }
+    }
+  } else if (warp >= 2) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
+    int acc = 0;
+    uint32_t acc_phase = 0;
+    for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      int e, mb, nbk;
+      decode_tile(a, tile, e, mb, nbk);
+      const int off = __ldg(a.offsets + e);
+      const int Me = __ldg(a.offsets + e + 1) - off;
+      const int r_in = mb * BM + q * 32 + lane;
+      const bool row_ok = r_in < Me;
+      __nv_bfloat16 *drow = a.D + (size_t)(off + r_in) * a.N;
+      const float *brow = a.bias ? a.bias + (size_t)e * a.N : nullptr;
+      // every lane waits; the outcome is made warp-uniform so that the
+      // .sync.aligned tensor-memory loads below always see the full warp
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
+      if (!ok) { failed = true; break; }
+      tc_fence_after();
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
+        const int col0 = nbk * BN + c * 32;
+        if (row_ok && col0 < a.N) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            float x0 = __uint_as_float(v[2 * j]), x1 = __uint_as_float(v[2 * j + 1]);
+            const int cc = col0 + 2 * j;
+            if (brow) {
+              x0 += cc < a.N ? __ldg(brow + cc) : 0.f;
+              x1 += cc + 1 < a.N ? __ldg(brow + cc + 1) : 0.f;
+            }
+            if (a.relu) {
+              x0 = fmaxf(x0, 0.f);
+              x1 = fmaxf(x1, 0.f);
+            }
+            __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+            pk[j] = *reinterpret_cast<uint32_t *>(&h);
+          }
+          if (col0 + 32 <= a.N) {
+            uint4 *dst = reinterpret_cast<uint4 *>(drow + col0);
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          } else {
+            for (int j = 0; j < 32 && col0 + j < a.N; ++j)
+              reinterpret_cast<uint16_t *>(drow)[col0 + j] =
+                  (uint16_t)((pk[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty(acc));
+      if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+    }
+    if (failed) *abort_flag = 1;
+  }
+
+  if (failed && a.status) atomicOr(a.status, MOE_STATUS_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor [rows][inner] (inner contiguous), box [box_rows][64],
+// 128-byte swizzle, out-of-range elements read as zero.
+int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return MOE_ECUDA;
+  cuuint64_t dims[2] = {inner, rows};
+  cuuint64_t strides[1] = {inner * 2};
+  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? MOE_OK : MOE_ECUDA;
+}
+
+int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const float *bias, void *D,
+             int relu, const int *offsets, const int *mprefix, int *status, cudaStream_t st,
+             const char *name) {
+  CUtensorMap ta, tb;
+  MOE_TRY(make_map(&ta, A, (uint64_t)K, (uint64_t)S, BM));
+  MOE_TRY(make_map(&tb, B, (uint64_t)K, (uint64_t)n * N, BN));
+  TcArgs a;
+  a.offsets = offsets;
+  a.mprefix = mprefix;
+  a.n = n;
+  a.N = N;
+  a.K = K;
+  a.nblk = (N + BN - 1) / BN;
+  a.bias = bias;
+  a.D = static_cast<__nv_bfloat16 *>(D);
+  a.relu = relu;
+  a.status = status;
+  const int64_t upper = (ceil_div(S, BM) + n) * (int64_t)a.nblk;
+  const int grid = (int)(upper < num_sms() ? upper : num_sms());
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    if (cudaFuncSetAttribute(expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return MOE_ECUDA;
+    attr_dev = dev;
+  }
+  return launch(name, expert_gemm_kernel, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, ta, tb, a);
+}
+
+}  // namespace
+
+int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
+  if (a.S == 0) return MOE_OK;
+  int *mprefix = const_cast<int *>(a.mprefix);
+  MOE_TRY(launch_block_prefix(a.offsets, a.n, BM, mprefix, st));
+  MOE_TRY(run_gemm(a.x_perm, a.S, a.d, a.W1, a.n, a.f, a.b1, a.hid, 1, a.offsets, a.mprefix,
+                   a.status, st, "expert_gemm1_tcgen05"));
+  MOE_TRY(run_gemm(a.hid, a.S, a.f, a.W2, a.n, a.d, a.b2, a.y_perm, 0, a.offsets, a.mprefix,
+                   a.status, st, "expert_gemm2_tcgen05"));
+  return MOE_OK;
+}
+
+}  // namespace moe

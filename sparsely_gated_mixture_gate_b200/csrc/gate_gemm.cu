@@ -1,0 +1,177 @@
+// gate_gemm.cu -- the gate's two projections in fp32:
+//   c = x W_g (+ b_g)          (clean logits)
+//   s = Softplus(x W_noise)    (noise scale)
+// [SGMoE-xyz] "Noisy Top-K 門控": H(x)_i = (x W_g)_i + StandardNormal() *
+// Softplus((x W_noise)_i); [SGMoE-note] "缺点与局限性": the gate needs fp32
+// (bf16 made training diverge), so this contraction stays on the FP32 pipes.
+//
+// One kernel serves the flat gate, the primary gate and the grouped
+// secondary gates of the hierarchical layer: rows can be gathered from x
+// through row_token, and rows are split into groups (ragged M) that each use
+// their own weights.  The output columns [0,nb) of W_g and of W_noise are
+// separate N-tiles (blockIdx.y), so one launch computes both c and s.
+//
+// Tile: 128 x 128 x 8, 256 threads, 8x8 outputs per thread held as two 4x4
+// quadrants (rows ty*4, 64+ty*4; cols tx*4, 64+tx*4) so the shared-memory
+// reads of a warp are broadcast / conflict free.  Double-buffered shared
+// memory, global loads of the next K-slice overlap the FMAs of the current.
+#include "internal.h"
+
+namespace moe {
+namespace {
+
+constexpr int BM = kGateBM, BN = kGateBN, BK = 8, NT = 256;
+constexpr int APAD = 4;  // As row padding (keeps 16-byte alignment)
+
+__device__ __forceinline__ float softplus_f(float z) {
+  return fmaxf(z, 0.0f) + log1pf(expf(-fabsf(z)));
+}
+
+__global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
+  __shared__ __align__(16) float As[2][BK][BM + APAD];
+  __shared__ __align__(16) float Bs[2][BK][BN];
+
+  // ---- which group, which rows
+  const int mblk = blockIdx.x;
+  int g = 0, row0, row_end;
+  if (a.seg_mblk) {
+    const int total = a.seg_mblk[a.G];
+    if (mblk >= total) return;
+    int lo = 0, hi = a.G - 1;  // largest g with seg_mblk[g] <= mblk
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.seg_mblk[mid] <= mblk) lo = mid; else hi = mid - 1;
+    }
+    g = lo;
+    row0 = a.seg_off[g] + (mblk - a.seg_mblk[g]) * BM;
+    row_end = a.seg_off[g + 1];
+  } else {
+    row0 = mblk * BM;
+    row_end = a.R;
+    if (row0 >= row_end) return;
+  }
+  const int ntn = (a.nb + BN - 1) / BN;
+  const int which = blockIdx.y / ntn;          // 0: W_g -> c, 1: W_noise -> s
+  const int col0 = (blockIdx.y % ntn) * BN;
+  const float *B = (which ? a.Wn : a.Wg) + (size_t)g * a.d * a.nb;
+  const int nb = a.nb;
+  const bool vecB = (nb & 3) == 0;
+
+  const int tid = threadIdx.x;
+  // A loader: row ar = tid/2, k quad aq = (tid&1)*4
+  const int ar = tid >> 1, aq = (tid & 1) * 4;
+  const int arow = row0 + ar;
+  const bool a_ok = arow < row_end;
+  const float *Arow = nullptr;
+  if (a_ok) {
+    const int tok = a.row_token ? a.row_token[arow] : arow;
+    Arow = a.x + (size_t)tok * a.d;
+  }
+  // B loader: k row bk = tid/32, col quad bc = (tid&31)*4
+  const int bk = tid >> 5, bc = (tid & 31) * 4;
+  const int bcol = col0 + bc;
+
+  auto load_a = [&](int k0) -> float4 {
+    if (!a_ok) return make_float4(0.f, 0.f, 0.f, 0.f);
+    return __ldg(reinterpret_cast<const float4 *>(Arow + k0 + aq));
+  };
+  auto load_b = [&](int k0) -> float4 {
+    const float *p = B + (size_t)(k0 + bk) * nb + bcol;
+    if (vecB && bcol + 3 < nb) return __ldg(reinterpret_cast<const float4 *>(p));
+    float4 v;
+    v.x = bcol + 0 < nb ? __ldg(p + 0) : 0.f;
+    v.y = bcol + 1 < nb ? __ldg(p + 1) : 0.f;
+    v.z = bcol + 2 < nb ? __ldg(p + 2) : 0.f;
+    v.w = bcol + 3 < nb ? __ldg(p + 3) : 0.f;
+    return v;
+  };
+  auto store_tiles = [&](int buf, float4 av, float4 bv) {
+    As[buf][aq + 0][ar] = av.x;
+    As[buf][aq + 1][ar] = av.y;
+    As[buf][aq + 2][ar] = av.z;
+    As[buf][aq + 3][ar] = av.w;
+    *reinterpret_cast<float4 *>(&Bs[buf][bk][bc]) = bv;
+  };
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+
+  const int tx = tid & 15, ty = tid >> 4;
+  const int nk = a.d / BK;  // d is a multiple of 8
+  float4 av = load_a(0), bv = load_b(0);
+  store_tiles(0, av, bv);
+  __syncthreads();
+
+  for (int kt = 0; kt < nk; ++kt) {
+    const int buf = kt & 1;
+    if (kt + 1 < nk) {
+      av = load_a((kt + 1) * BK);
+      bv = load_b((kt + 1) * BK);
+    }
+#pragma unroll
+    for (int kk = 0; kk < BK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+      const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
+      const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+      const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
+      const float ar_[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float br_[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(ar_[i], br_[j], acc[i][j]);
+    }
+    if (kt + 1 < nk) {
+      store_tiles(buf ^ 1, av, bv);
+    }
+    __syncthreads();
+  }
+
+  // ---- epilogue
+  float *out = which ? a.s : a.c;
+  const float *bias = (which == 0 && a.bias) ? a.bias + (size_t)g * nb : nullptr;
+  bool bad = false;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = row0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
+    if (row >= row_end) continue;
+    float *orow = out + (size_t)row * nb;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int col = col0 + h * 64 + tx * 4;
+      float v[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float z = acc[i][h * 4 + j];
+        const int cc = col + j;
+        if (cc < nb) {
+          if (which) z = softplus_f(z);
+          else if (bias) z += bias[cc];
+        }
+        bad |= !isfinite(z);
+        v[j] = z;
+      }
+      if (vecB && col + 3 < nb) {
+        *reinterpret_cast<float4 *>(orow + col) = make_float4(v[0], v[1], v[2], v[3]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (col + j < nb) orow[col + j] = v[j];
+      }
+    }
+  }
+  if (bad && a.status) atomicOr(a.status, MOE_STATUS_NONFINITE);
+}
+
+}  // namespace
+
+int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st) {
+  const int ntn = (a.nb + BN - 1) / BN;
+  dim3 grid(mblk_upper, ntn * (a.noise ? 2 : 1));
+  return launch("gate_gemm_fp32", gate_gemm_kernel, grid, dim3(NT), 0, st, a);
+}
+
+}  // namespace moe

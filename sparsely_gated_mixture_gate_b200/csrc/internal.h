@@ -1,0 +1,147 @@
+// internal.h -- declarations shared by the library's translation units.
+// Not part of the ABI (that is include/moe.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/moe.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- launches
+// Every kernel goes through launch(): it counts the launch, records CUDA
+// events around it when tracing is on, and turns a launch error into
+// MOE_ECUDA.
+void trace_begin(const char *name, cudaStream_t st, int *slot);
+void trace_end(int slot, cudaStream_t st);
+void count_launch();
+
+template <class Kernel, class... Args>
+int launch(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+           Args... args) {
+  if (grid.x == 0 || grid.y == 0 || grid.z == 0) return MOE_OK;
+  int slot = -1;
+  trace_begin(name, st, &slot);
+  kernel<<<grid, block, smem, st>>>(args...);
+  cudaError_t e = cudaGetLastError();
+  trace_end(slot, st);
+  count_launch();
+  return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+#define MOE_TRY(expr)            \
+  do {                           \
+    int _rc = (expr);            \
+    if (_rc != MOE_OK) return _rc; \
+  } while (0)
+
+int num_sms();
+
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- tiling constants
+constexpr int kGateBM = 128, kGateBN = 128;   // SIMT gate GEMM tile
+constexpr int kExpertBM = 128;                // tcgen05 grouped GEMM rows per tile
+constexpr int kMaxK = 8;                      // largest supported top-k
+
+// tokens per dispatch block, rows per routing tile: functions of the sizes
+// only, so results never depend on the device.
+int dispatch_tokens_per_block(int T);
+int route_rows_per_tile(int R);
+
+// ---------------------------------------------------------------- kernels (host launchers)
+struct GateGemmArgs {
+  const float *x;          // [T][d]
+  int d;
+  const int *row_token;    // [R] token of every GEMM row, or nullptr (row r = token r)
+  const int *seg_off;      // [G+1] first row of every group, or nullptr (one group of R rows)
+  const int *seg_mblk;     // [G+1] exclusive scan of ceil(rows_g / kGateBM), or nullptr
+  int R, G;
+  const float *Wg, *Wn, *bias;  // group g: Wg + g*d*nb, Wn + g*d*nb, bias + g*nb
+  int nb, noise;
+  float *c, *s;            // [R][nb]
+  int *status;
+};
+int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st);
+
+struct RouteArgs {
+  const float *c, *s;      // [R][nb]
+  int R, nb, k, router, noise;
+  uint64_t seed;
+  const int *row_token;    // [R] or nullptr
+  const int *row_slot;     // [R] primary slot of the row (secondary gate), or nullptr
+  const int *seg_off;      // [G+1] or nullptr
+  const int *seg_tiles;    // [G+1] exclusive scan of ceil(rows_g / RT), or nullptr
+  int G, RT;
+  int secondary;           // 0: gate id 0; 1: gate id 1 + group
+  int *out_idx;            // [T][K]
+  float *out_gate;         // [T][K]
+  int K;                   // slots per token in out_idx/out_gate
+  int expert_stride;       // secondary: expert id = g * expert_stride + j
+  const float *gate_mult;  // secondary: primary gates [T][k1]
+  int k1;
+  float *load_part;        // [tiles][nb]
+  float *psum_part;        // [tiles][nb] or nullptr
+  int *status;
+};
+int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st);
+// out[g][j] = sum over the tiles of group g (in order) of part[tile][j]
+int launch_route_reduce(const float *part, const int *seg_tiles, int G, int ntiles_flat, int nb,
+                        float *out, cudaStream_t st);
+// Hierarchical load: load[g*b+j] = cnt_g ? load_p[g] * load2[g*b+j] / cnt_g : 0
+int launch_hier_load(const float *load_p, const float *load2, const int *cnt, int a, int b,
+                     float *load, cudaStream_t st);
+
+struct DispatchArgs {
+  const int *idx;          // [T][k]
+  int T, k, n;
+  int64_t C;               // capacity (INT64_MAX: none)
+  const float *gate;       // [T][k] or nullptr; with it gate_sorted is written
+  int *hist, *base;        // [B][n] scratch
+  int *counts;             // [n]
+  int *offsets;            // [n+1]
+  int *ucoff;              // [n+1] scratch (uncapped offsets)
+  int *perm_token;         // [T*k]
+  int *perm_slot;          // [T*k] or nullptr
+  int *row_of;             // [T][k]
+  float *gate_sorted;      // [T*k] or nullptr
+  int *seg_mblk;           // [n+1] or nullptr: exclusive scan of ceil(kept_e / mblk_rows)
+  int mblk_rows;
+  int *seg_tiles;          // [n+1] or nullptr: exclusive scan of ceil(kept_e / tile_rows)
+  int tile_rows;
+  int *status;
+};
+int launch_dispatch(const DispatchArgs &a, cudaStream_t st);
+int launch_gather(const float *x, const int *row_of, int T, int k, int d, int bf16, void *x_perm,
+                  cudaStream_t st);
+// exclusive scan of ceil((offsets[e+1]-offsets[e]) / rows) into out[n+1]
+int launch_block_prefix(const int *offsets, int n, int rows, int *out, cudaStream_t st);
+
+struct ExpertArgs {
+  const void *x_perm;      // [S][d]
+  const int *offsets;      // [n+1]
+  const int *mprefix;      // [n+1] exclusive scan of ceil(M_e / kExpertBM)
+  int n, d, f, S;
+  const void *W1, *W2;
+  const float *b1, *b2;
+  void *hid;               // [S][f]
+  void *y_perm;            // [S][d]
+  int *status;
+};
+int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st);
+int launch_expert_f32(const ExpertArgs &a, cudaStream_t st);
+
+int launch_combine(const void *y_perm, int bf16, const float *gate, const int *row_of,
+                   const float *x, int passthrough, int T, int k, int d, float *y,
+                   cudaStream_t st);
+
+int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
+                      cudaStream_t st);
+int launch_losses(const float *importance, const float *load, const int *counts,
+                  const float *prob_sum, int n, int T, int k, int64_t C, int router,
+                  float w_imp, float w_load, float alpha, float *losses, cudaStream_t st);
+
+}  // namespace moe

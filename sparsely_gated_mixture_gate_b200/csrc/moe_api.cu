@@ -1,0 +1,615 @@
+// moe_api.cu -- the C ABI declared in include/moe.h: argument validation,
+// workspace layout, the launch sequence of every entry point, and tracing.
+// Host code only; the arithmetic is in the kernels of the other files.
+#include <limits.h>
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "internal.h"
+
+namespace moe {
+
+// ---------------------------------------------------------------- tracing
+namespace {
+struct TraceRec {
+  const char *name;
+  cudaEvent_t a, b;
+};
+struct TraceAgg {
+  std::string name;
+  int launches;
+  double ms;
+};
+bool g_trace = false;
+std::vector<TraceRec> g_pending;
+std::vector<cudaEvent_t> g_pool;
+std::vector<TraceAgg> g_agg;
+long long g_launches = 0;
+
+cudaEvent_t pooled_event() {
+  if (!g_pool.empty()) {
+    cudaEvent_t e = g_pool.back();
+    g_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+void trace_collect() {
+  for (auto &r : g_pending) {
+    float ms = 0.f;
+    cudaEventSynchronize(r.b);
+    cudaEventElapsedTime(&ms, r.a, r.b);
+    bool found = false;
+    for (auto &g : g_agg)
+      if (g.name == r.name) {
+        g.launches += 1;
+        g.ms += ms;
+        found = true;
+        break;
+      }
+    if (!found) g_agg.push_back({r.name, 1, (double)ms});
+    g_pool.push_back(r.a);
+    g_pool.push_back(r.b);
+  }
+  g_pending.clear();
+}
+}  // namespace
+
+void trace_begin(const char *name, cudaStream_t st, int *slot) {
+  if (!g_trace) return;
+  TraceRec r{name, pooled_event(), pooled_event()};
+  cudaEventRecord(r.a, st);
+  g_pending.push_back(r);
+  *slot = (int)g_pending.size() - 1;
+}
+void trace_end(int slot, cudaStream_t st) {
+  if (slot >= 0) cudaEventRecord(g_pending[slot].b, st);
+}
+void count_launch() { ++g_launches; }
+
+int num_sms() {
+  static int cached_dev = -1, cached = 148;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev != cached_dev) {
+    int v = 0;
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+      cached = v;
+    cached_dev = dev;
+  }
+  return cached;
+}
+
+int route_rows_per_tile(int R) {
+  // about four routing tiles per SM of a 148-SM part, 16..256 rows each
+  int64_t rt = ceil_div(R, 592);
+  rt = ceil_div(rt, 4) * 4;
+  if (rt < 16) rt = 16;
+  if (rt > 256) rt = 256;
+  return (int)rt;
+}
+
+// ---------------------------------------------------------------- workspace layout
+namespace {
+
+struct Layout {
+  size_t c, s, load_part, psum_part, prob_sum;
+  size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
+      g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
+  size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch;
+  size_t mprefix, x_perm, hid, y_perm;
+  size_t total;
+  int RT1, tiles1, RT2, tiles2_upper, B;
+};
+
+struct Bump {
+  size_t off = 0;
+  size_t take(size_t bytes) {
+    const size_t at = off;
+    off += (bytes + 255) & ~(size_t)255;
+    return at;
+  }
+};
+
+Layout make_layout(const moe_config &c) {
+  Layout L;
+  Bump bp;
+  const size_t T = (size_t)c.T, n = (size_t)c.n, k = (size_t)c.k;
+  const bool hier = c.hier_a > 0;
+  const size_t ng = hier ? (size_t)c.hier_a : n;
+  const size_t S = T * k;
+  const size_t esz = c.expert_dtype == MOE_BF16 ? 2 : 4;
+  L.RT1 = route_rows_per_tile(c.T);
+  L.tiles1 = (int)ceil_div(c.T, L.RT1);
+  size_t R2 = 0;
+  if (hier) {
+    R2 = T * (size_t)c.hier_k1;
+    L.RT2 = route_rows_per_tile((int)R2);
+    L.tiles2_upper = (int)ceil_div((int64_t)R2, L.RT2) + c.hier_a;
+  } else {
+    L.RT2 = 0;
+    L.tiles2_upper = 0;
+  }
+  const size_t cs = T * ng > R2 * (size_t)c.hier_b ? T * ng : R2 * (size_t)c.hier_b;
+  L.c = bp.take(4 * cs);
+  L.s = bp.take(4 * cs);
+  const size_t lp1 = (size_t)L.tiles1 * ng, lp2 = (size_t)L.tiles2_upper * (size_t)c.hier_b;
+  L.load_part = bp.take(4 * (lp1 > lp2 ? lp1 : lp2));
+  L.psum_part = bp.take(c.router == MOE_ROUTER_SWITCH ? 4 * (size_t)L.tiles1 * n : 0);
+  L.prob_sum = bp.take(4 * n);
+  L.B = (int)ceil_div(c.T, dispatch_tokens_per_block(c.T));
+  if (hier) {
+    const size_t a = (size_t)c.hier_a, k1 = (size_t)c.hier_k1;
+    L.pidx = bp.take(4 * T * k1);
+    L.pgate = bp.take(4 * T * k1);
+    L.load_p = bp.take(4 * a);
+    L.g_hist = bp.take(4 * (size_t)L.B * a);
+    L.g_base = bp.take(4 * (size_t)L.B * a);
+    L.g_counts = bp.take(4 * a);
+    L.g_offsets = bp.take(4 * (a + 1));
+    L.g_ucoff = bp.take(4 * (a + 1));
+    L.g_perm_token = bp.take(4 * T * k1);
+    L.g_perm_slot = bp.take(4 * T * k1);
+    L.g_row_of = bp.take(4 * T * k1);
+    L.g_mblk = bp.take(4 * (a + 1));
+    L.g_tiles = bp.take(4 * (a + 1));
+    L.load2_part = L.load_part;  // the primary partial sums are reduced first
+    L.load2 = bp.take(4 * n);
+  } else {
+    L.pidx = L.pgate = L.load_p = L.g_hist = L.g_base = L.g_counts = L.g_offsets = L.g_ucoff =
+        L.g_perm_token = L.g_perm_slot = L.g_row_of = L.g_mblk = L.g_tiles = L.load2_part =
+            L.load2 = 0;
+  }
+  L.hist = bp.take(4 * (size_t)L.B * n);
+  L.base = bp.take(4 * (size_t)L.B * n);
+  L.ucoff = bp.take(4 * (n + 1));
+  L.offsets = bp.take(4 * (n + 1));
+  L.perm_token = bp.take(4 * S);
+  L.row_of = bp.take(4 * S);
+  L.gate_sorted = bp.take(4 * S);
+  L.counts_scratch = bp.take(4 * n);
+  L.mprefix = bp.take(4 * (n + 1));
+  L.x_perm = bp.take(esz * S * (size_t)c.d);
+  L.hid = bp.take(esz * S * (size_t)c.f);
+  L.y_perm = bp.take(esz * S * (size_t)c.d);
+  L.total = bp.off;
+  return L;
+}
+
+template <class P>
+P *at(void *ws, size_t off) {
+  return reinterpret_cast<P *>(static_cast<char *>(ws) + off);
+}
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int64_t capacity_of(const moe_config &c) {
+  if (!(c.capacity_factor > 0.0)) return INT64_MAX;
+  return (int64_t)ceil((double)c.T * (double)c.k * c.capacity_factor / (double)c.n);
+}
+
+int check_device() {
+  static int checked_dev = -1;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_EDEVICE;
+  if (dev == checked_dev) return MOE_OK;
+  int major = 0, minor = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+    return MOE_EDEVICE;
+  if (major != 10 || minor != 0) return MOE_EDEVICE;  // built for sm_100a only
+  checked_dev = dev;
+  return MOE_OK;
+}
+
+int common_checks(const moe_config *cfg, void *ws, size_t ws_bytes, int32_t *status,
+                  Layout *L) {
+  const int v = moe_validate(cfg);
+  if (v != MOE_OK) return v;
+  if (!status) return MOE_EINVAL;
+  *L = make_layout(*cfg);
+  if (ws_bytes < L->total) return MOE_EWORKSPACE;
+  if (L->total > 0 && (!ws || !aligned(ws, 256))) return MOE_EWORKSPACE;
+  return check_device();
+}
+
+// ---------------------------------------------------------------- stage drivers
+int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gate_params &gp,
+             int *idx, float *gate, float *load, float *prob_sum, void *ws, int *status,
+             cudaStream_t st) {
+  if (c.T == 0) {
+    if (cudaMemsetAsync(load, 0, 4 * (size_t)c.n, st) != cudaSuccess) return MOE_ECUDA;
+    if (prob_sum && cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess)
+      return MOE_ECUDA;
+    return MOE_OK;
+  }
+  float *cbuf = at<float>(ws, L.c), *sbuf = at<float>(ws, L.s);
+  const bool hier = c.hier_a > 0;
+  const int ng = hier ? c.hier_a : c.n;
+
+  GateGemmArgs g{};
+  g.x = x;
+  g.d = c.d;
+  g.R = c.T;
+  g.G = 1;
+  g.Wg = gp.W_g;
+  g.Wn = gp.W_noise;
+  g.bias = gp.b_g;
+  g.nb = ng;
+  g.noise = c.noise;
+  g.c = cbuf;
+  g.s = sbuf;
+  g.status = status;
+  MOE_TRY(launch_gate_gemm(g, (int)ceil_div(c.T, kGateBM), st));
+
+  RouteArgs r{};
+  r.c = cbuf;
+  r.s = sbuf;
+  r.R = c.T;
+  r.nb = ng;
+  r.router = c.router;
+  r.noise = c.noise;
+  r.seed = c.seed;
+  r.G = 1;
+  r.RT = L.RT1;
+  r.load_part = at<float>(ws, L.load_part);
+  r.status = status;
+  if (!hier) {
+    r.k = c.k;
+    r.out_idx = idx;
+    r.out_gate = gate;
+    r.K = c.k;
+    const bool sw = c.router == MOE_ROUTER_SWITCH;
+    r.psum_part = sw ? at<float>(ws, L.psum_part) : nullptr;
+    MOE_TRY(launch_route(r, L.tiles1, st));
+    MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, c.n, load, st));
+    if (sw) {
+      float *ps = prob_sum ? prob_sum : at<float>(ws, L.prob_sum);
+      MOE_TRY(launch_route_reduce(r.psum_part, nullptr, 1, L.tiles1, c.n, ps, st));
+    } else if (prob_sum) {
+      if (cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess) return MOE_ECUDA;
+    }
+    return MOE_OK;
+  }
+
+  // ---- hierarchical: primary gate over groups
+  const int a = c.hier_a, b = c.hier_b, k1 = c.hier_k1, k2 = c.hier_k2;
+  int *pidx = at<int>(ws, L.pidx);
+  float *pgate = at<float>(ws, L.pgate);
+  r.k = k1;
+  r.out_idx = pidx;
+  r.out_gate = pgate;
+  r.K = k1;
+  MOE_TRY(launch_route(r, L.tiles1, st));
+  MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, a, at<float>(ws, L.load_p), st));
+
+  // ---- tokens grouped by their kept groups (stable), tile prefixes per group
+  DispatchArgs da{};
+  da.idx = pidx;
+  da.T = c.T;
+  da.k = k1;
+  da.n = a;
+  da.C = INT64_MAX;
+  da.hist = at<int>(ws, L.g_hist);
+  da.base = at<int>(ws, L.g_base);
+  da.counts = at<int>(ws, L.g_counts);
+  da.offsets = at<int>(ws, L.g_offsets);
+  da.ucoff = at<int>(ws, L.g_ucoff);
+  da.perm_token = at<int>(ws, L.g_perm_token);
+  da.perm_slot = at<int>(ws, L.g_perm_slot);
+  da.row_of = at<int>(ws, L.g_row_of);
+  da.seg_mblk = at<int>(ws, L.g_mblk);
+  da.mblk_rows = kGateBM;
+  da.seg_tiles = at<int>(ws, L.g_tiles);
+  da.tile_rows = L.RT2;
+  da.status = status;
+  MOE_TRY(launch_dispatch(da, st));
+
+  // ---- secondary gates: grouped fp32 GEMM over each group's tokens
+  const int R2 = c.T * k1;
+  GateGemmArgs g2 = g;
+  g2.row_token = da.perm_token;
+  g2.seg_off = da.offsets;
+  g2.seg_mblk = da.seg_mblk;
+  g2.R = R2;
+  g2.G = a;
+  g2.Wg = gp.W_g2;
+  g2.Wn = gp.W_noise2;
+  g2.bias = gp.b_g2;
+  g2.nb = b;
+  MOE_TRY(launch_gate_gemm(g2, (int)ceil_div(R2, kGateBM) + a, st));
+
+  RouteArgs r2 = r;
+  r2.R = R2;
+  r2.nb = b;
+  r2.k = k2;
+  r2.router = MOE_ROUTER_NOISY_TOPK;
+  r2.row_token = da.perm_token;
+  r2.row_slot = da.perm_slot;
+  r2.seg_off = da.offsets;
+  r2.seg_tiles = da.seg_tiles;
+  r2.G = a;
+  r2.RT = L.RT2;
+  r2.secondary = 1;
+  r2.out_idx = idx;
+  r2.out_gate = gate;
+  r2.K = c.k;
+  r2.expert_stride = b;
+  r2.gate_mult = pgate;
+  r2.k1 = k1;
+  r2.load_part = at<float>(ws, L.load2_part);
+  r2.psum_part = nullptr;
+  MOE_TRY(launch_route(r2, L.tiles2_upper, st));
+  MOE_TRY(launch_route_reduce(r2.load_part, da.seg_tiles, a, 0, b, at<float>(ws, L.load2), st));
+  MOE_TRY(launch_hier_load(at<float>(ws, L.load_p), at<float>(ws, L.load2), da.counts, a, b, load,
+                           st));
+  if (prob_sum && cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess)
+    return MOE_ECUDA;
+  return MOE_OK;
+}
+
+int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const float *gate,
+                 int64_t C, int *counts, int *offsets, int *perm_token, int *row_of, void *ws,
+                 int *status, cudaStream_t st) {
+  DispatchArgs da{};
+  da.idx = idx;
+  da.T = c.T;
+  da.k = c.k;
+  da.n = c.n;
+  da.C = C;
+  da.gate = gate;
+  da.hist = at<int>(ws, L.hist);
+  da.base = at<int>(ws, L.base);
+  da.counts = counts;
+  da.offsets = offsets;
+  da.ucoff = at<int>(ws, L.ucoff);
+  da.perm_token = perm_token;
+  da.perm_slot = nullptr;
+  da.row_of = row_of;
+  da.gate_sorted = gate ? at<float>(ws, L.gate_sorted) : nullptr;
+  da.status = status;
+  return launch_dispatch(da, st);
+}
+
+int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const int *offsets,
+                const moe_expert_params &ep, void *y_perm, void *ws, int *status,
+                cudaStream_t st) {
+  ExpertArgs e{};
+  e.x_perm = x_perm;
+  e.offsets = offsets;
+  e.mprefix = at<int>(ws, L.mprefix);
+  e.n = c.n;
+  e.d = c.d;
+  e.f = c.f;
+  e.S = c.T * c.k;
+  e.W1 = ep.W1;
+  e.W2 = ep.W2;
+  e.b1 = ep.b1;
+  e.b2 = ep.b2;
+  e.hid = at<void>(ws, L.hid);
+  e.y_perm = y_perm;
+  e.status = status;
+  return c.expert_dtype == MOE_BF16 ? launch_expert_bf16(e, st) : launch_expert_f32(e, st);
+}
+
+bool gate_params_ok(const moe_config &c, const moe_gate_params *gp) {
+  if (!gp || !gp->W_g || !aligned(gp->W_g, 16)) return false;
+  if (c.noise && !gp->W_noise) return false;
+  if (c.hier_a > 0 && (!gp->W_g2 || (c.noise && !gp->W_noise2))) return false;
+  return true;
+}
+
+bool expert_params_ok(const moe_expert_params *ep) {
+  return ep && ep->W1 && ep->W2 && aligned(ep->W1, 16) && aligned(ep->W2, 16);
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char *moe_strerror(int code) {
+  switch (code) {
+    case MOE_OK: return "ok";
+    case MOE_EINVAL: return "invalid argument or configuration";
+    case MOE_EWORKSPACE: return "workspace too small or misaligned";
+    case MOE_ECUDA: return "CUDA call or kernel launch failed";
+    case MOE_EDEVICE: return "no usable sm_100 (B200) device";
+    default: return "unknown error";
+  }
+}
+
+int moe_validate(const moe_config *c) {
+  if (!c) return MOE_EINVAL;
+  if (c->reserved != 0) return MOE_EINVAL;
+  if (c->T < 0 || c->n < 1 || c->n > 8192 || c->k < 1 || c->k > kMaxK || c->k > c->n)
+    return MOE_EINVAL;
+  if (c->d < 8 || c->d % 8 || c->d > 16384 || c->f < 8 || c->f % 8 || c->f > 65536)
+    return MOE_EINVAL;
+  if (c->router != MOE_ROUTER_NOISY_TOPK && c->router != MOE_ROUTER_SWITCH) return MOE_EINVAL;
+  if (c->noise != 0 && c->noise != 1) return MOE_EINVAL;
+  if (c->expert_dtype != MOE_F32 && c->expert_dtype != MOE_BF16) return MOE_EINVAL;
+  if (c->overflow_passthrough != 0 && c->overflow_passthrough != 1) return MOE_EINVAL;
+  if (!(c->capacity_factor == c->capacity_factor)) return MOE_EINVAL;  // NaN
+  if (c->router == MOE_ROUTER_SWITCH && (c->k != 1 || c->noise || c->hier_a || c->n > 4096))
+    return MOE_EINVAL;
+  if (c->hier_a < 0) return MOE_EINVAL;
+  if (c->hier_a > 0) {
+    if (c->hier_b < 1 || (int64_t)c->hier_a * c->hier_b != c->n) return MOE_EINVAL;
+    if (c->hier_k1 < 1 || c->hier_k1 > c->hier_a || c->hier_k1 > kMaxK) return MOE_EINVAL;
+    if (c->hier_k2 < 1 || c->hier_k2 > c->hier_b || c->hier_k2 > kMaxK) return MOE_EINVAL;
+    if (c->hier_k1 * c->hier_k2 != c->k) return MOE_EINVAL;
+  }
+  if ((int64_t)c->T * c->k > INT_MAX / 2) return MOE_EINVAL;
+  return MOE_OK;
+}
+
+int moe_capacity(const moe_config *cfg, int64_t *C) {
+  const int v = moe_validate(cfg);
+  if (v != MOE_OK) return v;
+  if (!C) return MOE_EINVAL;
+  *C = capacity_of(*cfg);
+  return MOE_OK;
+}
+
+int moe_workspace_size(const moe_config *cfg, size_t *bytes) {
+  const int v = moe_validate(cfg);
+  if (v != MOE_OK) return v;
+  if (!bytes) return MOE_EINVAL;
+  *bytes = make_layout(*cfg).total;
+  return MOE_OK;
+}
+
+int moe_gate(const moe_config *cfg, const float *x, const moe_gate_params *gp, int32_t *topk_idx,
+             float *topk_gate, float *load, float *prob_sum, void *ws, size_t ws_bytes,
+             int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if ((c.T > 0 && (!x || !aligned(x, 16))) || !topk_idx || !topk_gate || !load ||
+      !gate_params_ok(c, gp))
+    return MOE_EINVAL;
+  return run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status,
+                  reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *topk_idx, int32_t *counts,
+                 int32_t *offsets, int32_t *perm_token, int32_t *row_of, void *x_perm, void *ws,
+                 size_t ws_bytes, int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if (!counts || !offsets || !perm_token || !row_of || (c.T > 0 && !topk_idx)) return MOE_EINVAL;
+  if ((x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
+  if (x && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  MOE_TRY(run_dispatch(c, L, topk_idx, nullptr, capacity_of(c), counts, offsets, perm_token, row_of,
+                       ws, status, st));
+  if (x && c.T > 0)
+    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, c.expert_dtype == MOE_BF16, x_perm, st));
+  return MOE_OK;
+}
+
+int moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
+                   const moe_expert_params *ep, void *y_perm, void *ws, size_t ws_bytes,
+                   int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if (!offsets || !expert_params_ok(ep)) return MOE_EINVAL;
+  if (c.T > 0 && (!x_perm || !y_perm || !aligned(x_perm, 16) || !aligned(y_perm, 16)))
+    return MOE_EINVAL;
+  return run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status,
+                     reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_combine(const moe_config *cfg, const void *y_perm, const float *topk_gate,
+                const int32_t *row_of, const float *x, float *y, int32_t *status,
+                moe_stream_t stream) {
+  const int v = moe_validate(cfg);
+  if (v != MOE_OK) return v;
+  const moe_config &c = *cfg;
+  if (!status) return MOE_EINVAL;
+  if (c.T > 0 && (!y_perm || !topk_gate || !row_of || !y || !aligned(y, 16) ||
+                  !aligned(y_perm, 16)))
+    return MOE_EINVAL;
+  if (c.T > 0 && c.overflow_passthrough && (!x || !aligned(x, 16))) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
+                        c.overflow_passthrough, c.T, c.k, c.d, y,
+                        reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx, const float *topk_gate,
+                       const int32_t *counts, const float *load, const float *prob_sum,
+                       float *importance, float *losses, void *ws, size_t ws_bytes,
+                       int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if (!counts || !load || !importance || !losses) return MOE_EINVAL;
+  if (c.T > 0 && (!topk_idx || !topk_gate)) return MOE_EINVAL;
+  if (c.router == MOE_ROUTER_SWITCH && !prob_sum) return MOE_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  // gates sorted by expert (stable), from a capacity-free dispatch into scratch
+  MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, INT64_MAX, at<int>(ws, L.counts_scratch),
+                       at<int>(ws, L.offsets), at<int>(ws, L.perm_token), at<int>(ws, L.row_of), ws,
+                       status, st));
+  MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
+                            st));
+  return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, capacity_of(c), c.router,
+                       c.w_importance, c.w_load, c.alpha_aux, losses, st);
+}
+
+int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
+                const moe_expert_params *ep, float *y, int32_t *topk_idx, float *topk_gate,
+                float *importance, float *load, int32_t *counts, float *losses, void *ws,
+                size_t ws_bytes, int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if (!topk_idx || !topk_gate || !importance || !load || !counts || !losses) return MOE_EINVAL;
+  if (c.T > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_EINVAL;
+  if (!gate_params_ok(c, gp) || !expert_params_ok(ep)) return MOE_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool sw = c.router == MOE_ROUTER_SWITCH;
+  float *prob_sum = sw ? at<float>(ws, L.prob_sum) : nullptr;
+  const int64_t C = capacity_of(c);
+  int *offsets = at<int>(ws, L.offsets);
+  int *row_of = at<int>(ws, L.row_of);
+  void *x_perm = at<void>(ws, L.x_perm);
+  void *y_perm = at<void>(ws, L.y_perm);
+
+  MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st));
+  MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, C, counts, offsets, at<int>(ws, L.perm_token),
+                       row_of, ws, status, st));
+  if (c.T > 0) {
+    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, c.expert_dtype == MOE_BF16, x_perm, st));
+    MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st));
+    MOE_TRY(launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
+                           c.overflow_passthrough, c.T, c.k, c.d, y, st));
+  }
+  MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
+                            st));
+  return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, C, c.router,
+                       c.w_importance, c.w_load, c.alpha_aux, losses, st);
+}
+
+int moe_trace_enable(int on) {
+  g_trace = on != 0;
+  return MOE_OK;
+}
+
+int moe_trace_reset(void) {
+  trace_collect();
+  g_agg.clear();
+  return MOE_OK;
+}
+
+int moe_trace_count(void) {
+  trace_collect();
+  return (int)g_agg.size();
+}
+
+int moe_trace_get(int i, const char **name, int *launches, double *total_ms) {
+  trace_collect();
+  if (i < 0 || i >= (int)g_agg.size()) return MOE_EINVAL;
+  if (name) *name = g_agg[i].name.c_str();
+  if (launches) *launches = g_agg[i].launches;
+  if (total_ms) *total_ms = g_agg[i].ms;
+  return MOE_OK;
+}
+
+long long moe_launch_count(void) { return g_launches; }
+
+}  // extern "C"

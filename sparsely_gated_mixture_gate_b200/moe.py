@@ -1,0 +1,325 @@
+"""Thin Python binding of the C ABI: argument marshalling over torch device
+memory and the current CUDA stream.  Every step of the layer runs in the CUDA
+library; this module only allocates outputs / workspace with torch and passes
+pointers.  There is no CPU path: calls fail loudly when the library or a CUDA
+device is missing.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import dataclasses
+from typing import Optional
+
+import torch
+
+from . import _lib
+from ._lib import moe_config, moe_expert_params, moe_gate_params
+
+
+class MoEError(RuntimeError):
+    pass
+
+
+def _check(rc: int, what: str):
+    if rc != _lib.MOE_OK:
+        msg = _lib.load().moe_strerror(rc).decode()
+        raise MoEError(f"{what}: {msg} ({rc})")
+
+
+@dataclasses.dataclass
+class Config:
+    """Mirror of ``moe_config`` (include/moe.h)."""
+    T: int
+    d: int
+    n: int
+    k: int
+    f: int
+    hier_a: int = 0
+    hier_b: int = 0
+    hier_k1: int = 0
+    hier_k2: int = 0
+    router: int = 0
+    noise: int = 1
+    expert_bf16: int = 1
+    seed: int = 0
+    capacity_factor: float = 0.0
+    passthrough: int = 0
+    w_importance: float = 0.1
+    w_load: float = 0.1
+    alpha: float = 0.01
+
+    @classmethod
+    def from_workload(cls, w, T: Optional[int] = None) -> "Config":
+        kw = {f.name: getattr(w, f.name) for f in dataclasses.fields(cls) if hasattr(w, f.name)}
+        if T is not None:
+            kw["T"] = T
+        return cls(**kw)
+
+    def c(self) -> moe_config:
+        return moe_config(T=self.T, d=self.d, n=self.n, k=self.k, f=self.f, hier_a=self.hier_a,
+                          hier_b=self.hier_b, hier_k1=self.hier_k1, hier_k2=self.hier_k2,
+                          router=self.router, noise=self.noise,
+                          expert_dtype=_lib.BF16 if self.expert_bf16 else _lib.F32,
+                          seed=self.seed, capacity_factor=float(self.capacity_factor),
+                          overflow_passthrough=self.passthrough, w_importance=self.w_importance,
+                          w_load=self.w_load, alpha_aux=self.alpha, reserved=0)
+
+    @property
+    def expert_dtype(self):
+        return torch.bfloat16 if self.expert_bf16 else torch.float32
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else C.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _need(t: Optional[torch.Tensor], name: str, dtype, shape=None, device=None, optional=False):
+    if t is None:
+        if optional:
+            return
+        raise MoEError(f"{name} is required")
+    if not t.is_cuda:
+        raise MoEError(f"{name} must be a CUDA tensor (the layer has no CPU path)")
+    if t.dtype != dtype:
+        raise MoEError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise MoEError(f"{name} must be contiguous")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise MoEError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if device is not None and t.device != device:
+        raise MoEError(f"{name} is on {t.device}, expected {device}")
+
+
+def validate(cfg: Config) -> bool:
+    c = cfg.c()
+    return _lib.load().moe_validate(C.byref(c)) == _lib.MOE_OK
+
+
+def workspace_size(cfg: Config) -> int:
+    c = cfg.c()
+    out = C.c_size_t(0)
+    _check(_lib.load().moe_workspace_size(C.byref(c), C.byref(out)), "moe_workspace_size")
+    return int(out.value)
+
+
+def capacity(cfg: Config) -> int:
+    c = cfg.c()
+    out = C.c_int64(0)
+    _check(_lib.load().moe_capacity(C.byref(c), C.byref(out)), "moe_capacity")
+    return int(out.value)
+
+
+def workspace(cfg: Config, device) -> torch.Tensor:
+    # torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(workspace_size(cfg), 256), dtype=torch.uint8, device=device)
+
+
+def gate_params(params: dict) -> moe_gate_params:
+    return moe_gate_params(W_g=_ptr(params.get("Wg")), b_g=_ptr(params.get("bg")),
+                           W_noise=_ptr(params.get("Wn")), W_g2=_ptr(params.get("Wg2")),
+                           b_g2=_ptr(params.get("bg2")), W_noise2=_ptr(params.get("Wn2")))
+
+
+def expert_params(params: dict) -> moe_expert_params:
+    return moe_expert_params(W1=_ptr(params.get("W1")), b1=_ptr(params.get("b1")),
+                             W2=_ptr(params.get("W2")), b2=_ptr(params.get("b2")))
+
+
+def _check_params(cfg: Config, p: dict, dev, gate=True, experts=True):
+    gn = cfg.hier_a if cfg.hier_a else cfg.n
+    if gate:
+        _need(p.get("Wg"), "Wg", torch.float32, (cfg.d, gn), dev)
+        _need(p.get("Wn"), "Wn", torch.float32, (cfg.d, gn), dev, optional=not cfg.noise)
+        _need(p.get("bg"), "bg", torch.float32, (gn,), dev, optional=True)
+        if cfg.hier_a:
+            sh = (cfg.hier_a, cfg.d, cfg.hier_b)
+            _need(p.get("Wg2"), "Wg2", torch.float32, sh, dev)
+            _need(p.get("Wn2"), "Wn2", torch.float32, sh, dev, optional=not cfg.noise)
+            _need(p.get("bg2"), "bg2", torch.float32, (cfg.hier_a, cfg.hier_b), dev, optional=True)
+    if experts:
+        _need(p.get("W1"), "W1", cfg.expert_dtype, (cfg.n, cfg.f, cfg.d), dev)
+        _need(p.get("W2"), "W2", cfg.expert_dtype, (cfg.n, cfg.d, cfg.f), dev)
+        _need(p.get("b1"), "b1", torch.float32, (cfg.n, cfg.f), dev, optional=True)
+        _need(p.get("b2"), "b2", torch.float32, (cfg.n, cfg.d), dev, optional=True)
+
+
+def new_status(device) -> torch.Tensor:
+    return torch.zeros(1, dtype=torch.int32, device=device)
+
+
+def status_bits(status: torch.Tensor) -> int:
+    return int(status.item())
+
+
+# ---------------------------------------------------------------- step calls
+def gate(cfg: Config, x: torch.Tensor, params: dict, ws=None, status=None):
+    dev = x.device
+    _need(x, "x", torch.float32, (cfg.T, cfg.d))
+    _check_params(cfg, params, dev, experts=False)
+    idx = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    g = torch.empty(cfg.T, cfg.k, dtype=torch.float32, device=dev)
+    load = torch.empty(cfg.n, dtype=torch.float32, device=dev)
+    psum = torch.empty(cfg.n, dtype=torch.float32, device=dev)
+    ws = workspace(cfg, dev) if ws is None else ws
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    gp = gate_params(params)
+    _check(_lib.load().moe_gate(C.byref(c), _ptr(x), C.byref(gp), _ptr(idx), _ptr(g), _ptr(load),
+                                _ptr(psum), _ptr(ws), ws.numel(), _ptr(status), _stream()), "moe_gate")
+    return dict(topk_idx=idx, topk_gate=g, load=load, prob_sum=psum, status=status)
+
+
+def dispatch(cfg: Config, x: Optional[torch.Tensor], topk_idx: torch.Tensor, ws=None, status=None):
+    dev = topk_idx.device
+    _need(topk_idx, "topk_idx", torch.int32, (cfg.T, cfg.k))
+    if x is not None:
+        _need(x, "x", torch.float32, (cfg.T, cfg.d), dev)
+    S = cfg.T * cfg.k
+    counts = torch.empty(cfg.n, dtype=torch.int32, device=dev)
+    offsets = torch.empty(cfg.n + 1, dtype=torch.int32, device=dev)
+    perm_token = torch.full((max(S, 1),), -1, dtype=torch.int32, device=dev)
+    row_of = torch.empty(cfg.T, cfg.k, dtype=torch.int32, device=dev)
+    x_perm = torch.empty(max(S, 1), cfg.d, dtype=cfg.expert_dtype, device=dev) if x is not None else None
+    ws = workspace(cfg, dev) if ws is None else ws
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    _check(_lib.load().moe_dispatch(C.byref(c), _ptr(x), _ptr(topk_idx), _ptr(counts), _ptr(offsets),
+                                    _ptr(perm_token), _ptr(row_of), _ptr(x_perm), _ptr(ws), ws.numel(),
+                                    _ptr(status), _stream()), "moe_dispatch")
+    return dict(counts=counts, offsets=offsets, perm_token=perm_token, row_of=row_of, x_perm=x_perm,
+                status=status)
+
+
+def expert_ffn(cfg: Config, x_perm: torch.Tensor, offsets: torch.Tensor, params: dict, ws=None,
+               status=None):
+    dev = x_perm.device
+    S = cfg.T * cfg.k
+    _need(x_perm, "x_perm", cfg.expert_dtype, (max(S, 1), cfg.d))
+    _need(offsets, "offsets", torch.int32, (cfg.n + 1,), dev)
+    _check_params(cfg, params, dev, gate=False)
+    y_perm = torch.empty(max(S, 1), cfg.d, dtype=cfg.expert_dtype, device=dev)
+    ws = workspace(cfg, dev) if ws is None else ws
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    ep = expert_params(params)
+    _check(_lib.load().moe_expert_ffn(C.byref(c), _ptr(x_perm), _ptr(offsets), C.byref(ep), _ptr(y_perm),
+                                      _ptr(ws), ws.numel(), _ptr(status), _stream()), "moe_expert_ffn")
+    return dict(y_perm=y_perm, status=status)
+
+
+def combine(cfg: Config, y_perm: torch.Tensor, topk_gate: torch.Tensor, row_of: torch.Tensor,
+            x: Optional[torch.Tensor] = None, status=None):
+    dev = y_perm.device
+    _need(y_perm, "y_perm", cfg.expert_dtype, None)
+    _need(topk_gate, "topk_gate", torch.float32, (cfg.T, cfg.k), dev)
+    _need(row_of, "row_of", torch.int32, (cfg.T, cfg.k), dev)
+    if x is not None:
+        _need(x, "x", torch.float32, (cfg.T, cfg.d), dev)
+    y = torch.empty(cfg.T, cfg.d, dtype=torch.float32, device=dev)
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    _check(_lib.load().moe_combine(C.byref(c), _ptr(y_perm), _ptr(topk_gate), _ptr(row_of), _ptr(x),
+                                   _ptr(y), _ptr(status), _stream()), "moe_combine")
+    return dict(y=y, status=status)
+
+
+def balance_losses(cfg: Config, topk_idx, topk_gate, counts, load, prob_sum=None, ws=None, status=None):
+    dev = topk_idx.device
+    importance = torch.empty(cfg.n, dtype=torch.float32, device=dev)
+    losses = torch.empty(8, dtype=torch.float32, device=dev)
+    ws = workspace(cfg, dev) if ws is None else ws
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    _check(_lib.load().moe_balance_losses(C.byref(c), _ptr(topk_idx), _ptr(topk_gate), _ptr(counts),
+                                          _ptr(load), _ptr(prob_sum), _ptr(importance), _ptr(losses),
+                                          _ptr(ws), ws.numel(), _ptr(status), _stream()),
+           "moe_balance_losses")
+    return dict(importance=importance, losses=losses, status=status)
+
+
+# ---------------------------------------------------------------- fused layer
+class MoELayer:
+    """Parameters plus pre-allocated workspace and outputs for repeated calls
+    of the fused ``moe_forward`` on one device."""
+
+    def __init__(self, cfg: Config, params: dict, device=None):
+        self.cfg = cfg
+        self.params = params
+        dev = torch.device(device) if device is not None else params["Wg"].device
+        self.device = dev
+        _check_params(cfg, params, dev)
+        _lib.load()
+        self._c = cfg.c()
+        self._gp = gate_params(params)
+        self._ep = expert_params(params)
+        self.ws = workspace(cfg, dev)
+        self.status = new_status(dev)
+        T, k, n, d = cfg.T, cfg.k, cfg.n, cfg.d
+        self.y = torch.empty(T, d, dtype=torch.float32, device=dev)
+        self.topk_idx = torch.empty(T, k, dtype=torch.int32, device=dev)
+        self.topk_gate = torch.empty(T, k, dtype=torch.float32, device=dev)
+        self.importance = torch.empty(n, dtype=torch.float32, device=dev)
+        self.load = torch.empty(n, dtype=torch.float32, device=dev)
+        self.counts = torch.empty(n, dtype=torch.int32, device=dev)
+        self.losses = torch.empty(8, dtype=torch.float32, device=dev)
+
+    def forward_(self, x: torch.Tensor, stream=None):
+        """Run the layer on device-resident x; outputs land in this object's
+        buffers (asynchronous on the current stream)."""
+        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        st = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+        _check(_lib.load().moe_forward(C.byref(self._c), _ptr(x), C.byref(self._gp), C.byref(self._ep),
+                                       _ptr(self.y), _ptr(self.topk_idx), _ptr(self.topk_gate),
+                                       _ptr(self.importance), _ptr(self.load), _ptr(self.counts),
+                                       _ptr(self.losses), _ptr(self.ws), self.ws.numel(),
+                                       _ptr(self.status), st), "moe_forward")
+        return self.y
+
+    def outputs(self) -> dict:
+        return dict(y=self.y, topk_idx=self.topk_idx, topk_gate=self.topk_gate,
+                    importance=self.importance, load=self.load, counts=self.counts,
+                    losses=self.losses, status=self.status)
+
+    def forward_host(self, x_host: torch.Tensor, y_host: torch.Tensor, losses_host: torch.Tensor,
+                     x_dev: torch.Tensor):
+        """End-to-end call from host memory: copy x in (pinned host -> device),
+        run the layer, copy y and the losses back, all on the current stream."""
+        x_dev.copy_(x_host, non_blocking=True)
+        self.forward_(x_dev)
+        y_host.copy_(self.y, non_blocking=True)
+        losses_host.copy_(self.losses, non_blocking=True)
+
+
+def forward(cfg: Config, x: torch.Tensor, params: dict) -> dict:
+    layer = MoELayer(cfg, params, x.device)
+    layer.forward_(x)
+    return layer.outputs()
+
+
+# ---------------------------------------------------------------- tracing
+def trace_enable(on: bool = True):
+    _lib.load().moe_trace_enable(int(bool(on)))
+
+
+def trace_reset():
+    _lib.load().moe_trace_reset()
+
+
+def trace_read() -> dict:
+    L = _lib.load()
+    out = {}
+    for i in range(L.moe_trace_count()):
+        name = C.c_char_p()
+        nl = C.c_int()
+        ms = C.c_double()
+        _check(L.moe_trace_get(i, C.byref(name), C.byref(nl), C.byref(ms)), "moe_trace_get")
+        out[name.value.decode()] = dict(launches=nl.value, ms=ms.value)
+    return out
+
+
+def launch_count() -> int:
+    return int(_lib.load().moe_launch_count())

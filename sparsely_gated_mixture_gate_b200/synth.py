@@ -156,6 +156,8 @@ def random_routing(T: int, k: int, n: int, device="cpu", seed: int = 0, skew: fl
     """Synthetic expert choices [T][k] for stand-alone dispatch tests: k
     distinct experts per token, drawn with optional Zipf-like skew; a fraction
     of entries can be replaced by out-of-range ids."""
+    if T == 0:
+        return torch.zeros(0, k, dtype=torch.int32, device=device)
     g = _gen(device, seed, 11)
     if skew > 0:
         w = torch.arange(1, n + 1, device=device, dtype=torch.float64).pow(-skew)

@@ -255,3 +255,42 @@ def test_hierarchical_structure_and_zero_noise(orc):
     inp["Wn2"] = torch.full_like(inp["Wn2"], -40.0)
     o = _fwd(orc, w, inp)
     np.testing.assert_allclose(o["load"], o["counts"].astype(np.float64), rtol=1e-12)
+
+
+def test_combine_hand(orc):
+    """y_0 = 1/4 (1,2) + 3/4 (5,6) = (4,5); token 1 has no kept slot and
+    passes through (9,8), or gets 0 without pass-through."""
+    Y = np.array([[1.0, 2.0], [3.0, 4.0], [5.0, 6.0]])
+    gate = np.array([[0.25, 0.75], [1.0, 0.0]])
+    row_of = np.array([[0, 2], [-1, -1]], np.int32)
+    x = np.array([[0.0, 0.0], [9.0, 8.0]], np.float32)
+    y = orc.combine(Y, gate, row_of, x, passthrough=True)
+    assert y.tolist() == [[4.0, 5.0], [9.0, 8.0]]
+    y = orc.combine(Y, gate, row_of, x, passthrough=False)
+    assert y.tolist() == [[4.0, 5.0], [0.0, 0.0]]
+
+
+def test_balance_hand(orc):
+    """idx (0,0,1), gates (1/2,1/2,1): Importance = (1,1) -> CV^2 = 0;
+    Load = (2,0) -> mean 1, population variance 1 -> CV^2 = 1, L_load = 0.1;
+    counts (2,1) with C = 1: one slot dropped of 3."""
+    imp, losses = orc.balance(2, [[0], [0], [1]], [[0.5], [0.5], [1.0]], [2, 1], [2.0, 0.0], C=1)
+    assert imp.tolist() == [1.0, 1.0]
+    assert losses[0] == 0.0 and losses[5] == 0.0
+    assert losses[1] == pytest.approx(0.1) and losses[6] == pytest.approx(1.0)
+    assert losses[4] == pytest.approx(1 / 3) and losses[7] == 1.0
+    assert losses[2] == 0.0  # noisy-gate router: no Switch loss
+    # Switch: f = (2/3, 1/3), P = (0.6, 0.4) -> 2 * (0.4 + 0.4/3)
+    imp, losses = orc.balance(2, [[0], [0], [1]], [[0.5], [0.5], [1.0]], [2, 1], [2.0, 1.0],
+                              prob_sum=[1.8, 1.2], router=1, alpha=0.01)
+    assert losses[2] == pytest.approx(2 * (2 / 3 * 0.6 + 1 / 3 * 0.4))
+    assert losses[3] == pytest.approx(0.01 * losses[2])
+
+
+def test_gate_batch_matches_forward(orc, tiny):
+    w, inp = tiny
+    o = _fwd(orc, w, inp)
+    g = orc.gate_batch(w.cfg(), _np_inputs(inp))
+    assert np.array_equal(g["topk_idx"], o["topk_idx"])
+    assert np.array_equal(g["topk_gate"], o["topk_gate"])
+    assert np.array_equal(g["load"], o["load"])
