@@ -1,0 +1,430 @@
+"""Benchmark of the Sparsely-Gated MoE layer forward pass on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload lm-flat] [--impl ours|reference]
+
+One step = one full forward pass (gate, dispatch, experts, combine, balancing
+statistics) of one batch of the workload through the fused C-ABI call
+``moe_forward``.  Inputs are resident in HBM; L2 is flushed (256 MiB write)
+before every timed step, and every step is timed on the device with CUDA
+events on the launching stream; the total is the max over ranks.  With N > 1
+(launched by torchrun) every rank runs its own independent batch on its own
+GPU (replicas, weak scaling; the layer has no cross-batch exchange).
+
+The JSON line also carries: e2e (same metric through the Python/C-ABI call
+with pinned host buffers, copies inside the timed region), the roofline of the
+dominant kernel (per-kernel CUDA-event times recorded by the library around
+its own launches), the expert-FFN TFLOP/s and routing GB/s of the metric,
+clocks sampled during the timed region, the count of library kernel launches,
+and the oracle's CPU baseline on a bounded sample.  ``--impl reference`` times
+the oracle itself (the reference arm of this comparison).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "MoE-layer fwd tokens/s; expert-FFN TFLOP/s vs bf16 peak; routing HBM GB/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                  "sm_max_mhz": 1965.0}
+SMS, FP32_LANES = 148, 128  # B200: 148 SMs x 128 FP32 lanes
+
+
+# ------------------------------------------------------------------ helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    d = dict(FALLBACK_PEAKS)
+    d["source"] = "fallback"
+    return d
+
+
+def dist_info():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def aggregate(total_ms: float, tokens_per_rank: int, steps: int, world: int, group=None):
+    """Max of the device time over ranks; value = tokens of all ranks / that
+    time.  Works for any torch.distributed backend (the test uses gloo)."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([total_ms], dtype=torch.float64)
+    if world > 1:
+        if dist.get_backend(group) == "nccl":
+            t = t.cuda()
+        dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    ms = float(t.item())
+    value = world * tokens_per_rank * steps / (ms / 1e3) if ms > 0 else 0.0
+    return ms, value
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons during a region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.path = tempfile.mktemp(prefix="clocks_", suffix=".csv")
+        self.proc = None
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={gpu_index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    rows.append(dict(sm=float(parts[1]), max=float(parts[2]), power=float(parts[3]),
+                                     hw=parts[5], hwt=parts[6], swt=parts[7], pcap=parts[8]))
+                except ValueError:
+                    continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200.0] or rows
+        reasons = set()
+        for r in load:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                              ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[key].lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["max"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(load)}
+
+
+def src_sha(name: str) -> str:
+    with open(os.path.join(ROOT, "sparsely_gated_mixture_gate_b200", "csrc", name), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+KERNEL_SRC = {"expert_gemm1_tcgen05": "expert_tc.cu", "expert_gemm2_tcgen05": "expert_tc.cu",
+              "gate_gemm_fp32": "gate_gemm.cu", "route_topk": "route.cu", "combine": "combine.cu",
+              "dispatch_gather": "dispatch.cu", "dispatch_rank": "dispatch.cu"}
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel's source changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    if not os.path.exists(p) or kernel not in KERNEL_SRC:
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(workload, {}).get(kernel)
+    if not rec or rec.get("csrc_sha") != src_sha(KERNEL_SRC[kernel]):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+def kernel_work(w, name: str, S_kept: int):
+    """Algorithmic work of one launch: (bound, flops, bytes)."""
+    T, d, n, k, f = w.T, w.d, w.n, w.k, w.f
+    S = T * k
+    ng = w.hier_a if w.hier_a else n
+    esz = 2 if w.expert_bf16 else 4
+    if name == "expert_gemm1_tcgen05":
+        return "tensor", 2.0 * S_kept * d * f, n * f * d * esz + S_kept * d * esz + S_kept * f * esz
+    if name == "expert_gemm2_tcgen05":
+        return "tensor", 2.0 * S_kept * d * f, n * d * f * esz + S_kept * f * esz + S_kept * d * esz
+    if name == "gate_gemm_fp32":
+        return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
+    if name == "route_topk":
+        return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
+    if name == "combine":
+        return "hbm", 0.0, S_kept * d * esz + T * d * 4 + 8 * T * k
+    if name == "dispatch_gather":
+        return "hbm", 0.0, T * d * 4 + S_kept * d * esz + 4 * S
+    return None, 0.0, 0.0
+
+
+# ------------------------------------------------------------------ arms
+def run_ours(args, w, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    from sparsely_gated_mixture_gate_b200 import moe as M
+    from sparsely_gated_mixture_gate_b200 import synth
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    pk = peaks()
+    # every rank: its own batch (x seeded by rank), the same weights
+    inp = synth.make_inputs(w, device=dev)
+    if rank:
+        inp["x"] = synth.make_inputs(w.with_(seed=rank), device=dev, experts=False)["x"]
+    cfg = M.Config.from_workload(w)
+    layer = M.MoELayer(cfg, inp, dev)
+    x = inp["x"]
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.fill_(1.0)
+        layer.forward_(x)
+    torch.cuda.synchronize()
+    st = M.status_bits(layer.status)
+    if st:
+        raise SystemExit(f"device status {st} after warm-up")
+    S_kept = int(layer.counts.clamp(max=M.capacity(cfg) if w.capacity_factor > 0 else 2**31 - 1).sum())
+
+    # ---- timed region: K device-timed steps
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    M.trace_reset()
+    M.trace_enable(True)
+    launches0 = M.launch_count()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(args.steps):
+        flush.fill_(float(i))
+        starts[i].record(stream)
+        layer.forward_(x)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    wall = time.perf_counter() - wall0
+    launches = M.launch_count() - launches0
+    M.trace_enable(False)
+    per_kernel = M.trace_read()
+    clk = clocks.stop()
+    total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
+    ms, value = aggregate(total_ms, w.T, args.steps, world)
+
+    # ---- e2e: host buffers, copies inside the timed region
+    xh = x.cpu().pin_memory()
+    yh = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+    lh = torch.empty(8, dtype=torch.float32).pin_memory()
+    xd = torch.empty_like(x)
+    e_steps = max(3, min(args.steps, 200))
+    for _ in range(3):
+        layer.forward_host(xh, yh, lh, xd)
+    torch.cuda.synchronize()
+    es = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    for i in range(e_steps):
+        flush.fill_(float(i))
+        es[i].record(stream)
+        layer.forward_host(xh, yh, lh, xd)
+        ee[i].record(stream)
+    torch.cuda.synchronize()
+    e_ms, e_value = aggregate(sum(a.elapsed_time(b) for a, b in zip(es, ee)), w.T, e_steps, world)
+    st = M.status_bits(layer.status)
+
+    if rank != 0:
+        return None
+
+    # ---- roofline of the dominant kernel and the metric's two side figures
+    kstats = {}
+    for name, rec in per_kernel.items():
+        per_launch_ms = rec["ms"] / max(rec["launches"], 1)
+        bound, flops, nbytes = kernel_work(w, name, S_kept)
+        e = {"launches": rec["launches"], "ms_per_launch": round(per_launch_ms, 5),
+             "share": round(rec["ms"] / max(sum(r["ms"] for r in per_kernel.values()), 1e-9), 4)}
+        if bound:
+            e["gbs"] = round(nbytes / (per_launch_ms / 1e3) / 1e9, 1)
+            if flops:
+                e["tflops"] = round(flops / (per_launch_ms / 1e3) / 1e12, 2)
+        kstats[name] = e
+    dom = max(per_kernel, key=lambda k: per_kernel[k]["ms"])
+    bound, flops, nbytes = kernel_work(w, dom, S_kept)
+    dom_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
+    sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
+    if bound == "tensor":
+        ai = flops / nbytes
+        ridge = sustained * 1e12 / (pk["hbm_gbs"] * 1e9)
+        if ai < ridge:  # the weights stream from HBM: bandwidth bound
+            roof = {"bound": "hbm", "achieved": nbytes / (dom_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                    "unit": "GB/s"}
+        else:
+            roof = {"bound": "tensor", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": sustained,
+                    "unit": "TFLOP/s"}
+    elif bound == "alu":
+        fp32_peak = SMS * FP32_LANES * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+        roof = {"bound": "alu", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": round(fp32_peak, 1),
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": nbytes / (dom_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["achieved"] = round(roof["achieved"], 2)
+    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof["kernel"] = dom
+    roof["peak_source"] = pk["source"]
+    roof["traffic"] = ncu_traffic(dom, w.name)
+
+    ffn_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in per_kernel
+                 if k.startswith("expert_gemm"))
+    ffn_flops = 4.0 * S_kept * w.d * w.f
+    route_names = [k for k in per_kernel if k.startswith(("route", "dispatch", "combine"))]
+    route_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in route_names)
+    route_bytes = sum(kernel_work(w, k, S_kept)[2] for k in route_names)
+
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32",
+        "data": "synthetic (seeded; random-init weights of the workload's shapes)",
+        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k,
+                   "d_ff": w.f, "hier": [w.hier_a, w.hier_b] if w.hier_a else None,
+                   "router": "switch-top1" if w.router else "noisy-top-k",
+                   "capacity_factor": w.capacity_factor or None,
+                   "l2": "flushed before every timed step (256 MiB write)",
+                   "parallelism": f"replicas x{world}"},
+        "expert_ffn_tflops": round(ffn_flops / (ffn_ms / 1e3) / 1e12, 2) if ffn_ms else None,
+        "expert_ffn_frac_bf16_peak": round(ffn_flops / (ffn_ms / 1e3) / 1e12 / sustained, 4) if ffn_ms else None,
+        "routing_hbm_gbs": round(route_bytes / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
+        "roofline": roof,
+        "kernels": kstats,
+        "gpu_launches": int(launches),
+        "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * 4,
+                "d2h_bytes_per_step": w.T * w.d * 4 + 32, "steps": e_steps},
+        "clocks": clk,
+        "wall_s": round(wall, 3),
+        "device_status": st,
+    }
+    return line
+
+
+def oracle_sample_inputs(w, T_s):
+    import torch
+
+    from sparsely_gated_mixture_gate_b200 import synth
+    inp = synth.make_inputs(w, T=T_s)
+    return {k: (None if v is None else (synth.bf16_bits(v) if v.dtype == torch.bfloat16 else v.numpy()))
+            for k, v in inp.items()}
+
+
+def time_oracle(w, T_s, reps=1):
+    from oracle import oracle as orc
+    orc.build()
+    npin = oracle_sample_inputs(w, T_s)
+    cfg = dict(w.cfg(), T=T_s)
+    t0 = time.perf_counter()
+    for _ in range(reps):
+        orc.forward(cfg, npin)
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w, budget_s=12.0):
+    """The oracle (single-threaded C, as it stands) on the first tokens of the
+    workload: calibrate on 8 tokens, then run a sample of about budget_s."""
+    t8 = time_oracle(w, 8)
+    T_s = int(max(8, min(w.T, budget_s / max(t8 / 8, 1e-6))))
+    t = time_oracle(w, T_s)
+    return {"value": round(T_s / t, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+            "sample": f"first {T_s} tokens of {w.name} as one batch (same weights), {t:.1f} s"}
+
+
+def run_reference(args, w):
+    """The reference arm: the oracle itself, each step a bounded sample of the
+    workload sized so the whole run stays within about two minutes."""
+    t8 = time_oracle(w, 8)
+    per_tok = max(t8 / 8, 1e-6)
+    budget = 90.0 / max(args.steps + args.warmup, 1)
+    T_s = int(max(1, min(w.T, budget / per_tok)))
+    from oracle import oracle as orc
+    npin = oracle_sample_inputs(w, T_s)
+    cfg = dict(w.cfg(), T=T_s)
+    for _ in range(args.warmup):
+        orc.forward(cfg, npin)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        orc.forward(cfg, npin)
+    t = time.perf_counter() - t0
+    value = T_s * args.steps / t
+    sample = f"first {T_s} tokens of {w.name} per step (same weights)"
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k, "d_ff": w.f,
+                       "sample_tokens_per_step": T_s},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--workload", default="lm-flat")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be at least 3")
+
+    from sparsely_gated_mixture_gate_b200 import synth
+    w = synth.WORKLOADS[args.workload]
+    world, rank, local = dist_info()
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args, w)), flush=True)
+        return
+
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, w, world, rank, local)
+        if rank == 0 and line is not None:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(w)
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -476,9 +476,8 @@ int moe_gate(const moe_config *cfg, const float *x, const moe_gate_params *gp, i
   Layout L;
   MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
   const moe_config &c = *cfg;
-  if ((c.T > 0 && (!x || !aligned(x, 16))) || !topk_idx || !topk_gate || !load ||
-      !gate_params_ok(c, gp))
-    return MOE_EINVAL;
+  if (!load || !gate_params_ok(c, gp)) return MOE_EINVAL;
+  if (c.T > 0 && (!x || !aligned(x, 16) || !topk_idx || !topk_gate)) return MOE_EINVAL;
   return run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status,
                   reinterpret_cast<cudaStream_t>(stream));
 }
@@ -489,9 +488,10 @@ int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *topk_idx,
   Layout L;
   MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
   const moe_config &c = *cfg;
-  if (!counts || !offsets || !perm_token || !row_of || (c.T > 0 && !topk_idx)) return MOE_EINVAL;
-  if ((x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
-  if (x && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_EINVAL;
+  if (!counts || !offsets) return MOE_EINVAL;
+  if (c.T > 0 && (!topk_idx || !perm_token || !row_of)) return MOE_EINVAL;
+  if (c.T > 0 && (x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
+  if (c.T > 0 && x && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   MOE_TRY(run_dispatch(c, L, topk_idx, nullptr, capacity_of(c), counts, offsets, perm_token, row_of,
                        ws, status, st));
@@ -558,8 +558,9 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   Layout L;
   MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
   const moe_config &c = *cfg;
-  if (!topk_idx || !topk_gate || !importance || !load || !counts || !losses) return MOE_EINVAL;
-  if (c.T > 0 && (!x || !y || !aligned(x, 16) || !aligned(y, 16))) return MOE_EINVAL;
+  if (!importance || !load || !counts || !losses) return MOE_EINVAL;
+  if (c.T > 0 && (!x || !y || !topk_idx || !topk_gate || !aligned(x, 16) || !aligned(y, 16)))
+    return MOE_EINVAL;
   if (!gate_params_ok(c, gp) || !expert_params_ok(ep)) return MOE_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool sw = c.router == MOE_ROUTER_SWITCH;
