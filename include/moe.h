@@ -186,6 +186,32 @@ MOE_API int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *t
                  int32_t *row_of, void *x_perm, void *ws, size_t ws_bytes,
                  int32_t *status, moe_stream_t stream);
 
+/* Allocation-free variant of moe_dispatch.  The pages have no counterpart:
+ * this entry point exists for callers that are given only their input and
+ * output buffers and cannot obtain scratch device memory -- e.g. a plugin of
+ * a host inference engine that plans all memory up front and passes no
+ * allocator, or a serving loop that must not call cudaMalloc after start-up
+ * (it synchronises the device and can fail under memory pressure).
+ * Same arguments, outputs and status bits as moe_dispatch, without ws.  Its
+ * scratch (per-block histograms and their scanned bases, uncapped offsets)
+ * takes 2*B*n + n + 1 int32, B = ceil(T / t) dispatch blocks of t tokens,
+ * t = T/296 rounded up to a multiple of 32 and clamped to [32, 256].  It
+ * lives in one fixed device array of MOE_DISPATCH_NOALLOC_SCRATCH_INTS int32
+ * (4 MiB) that every GPU loading the library keeps until the process exits.
+ * A call needing more returns MOE_EWORKSPACE before any device work (n = 256
+ * experts fit up to T = 524032 tokens, n = 4096 up to T = 4064).  The first
+ * call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current), so make that first call before any stream
+ * capture.  All calls share the array: every element a call reads is written
+ * earlier in the same call, so results never depend on earlier calls, but
+ * calls that overlap on the GPU (other streams, unordered host threads) race
+ * on it.  It calls no allocator. */
+#define MOE_DISPATCH_NOALLOC_SCRATCH_INTS (1 << 20)
+MOE_API int moe_dispatch_noalloc(const moe_config *cfg, const float *x,
+                                 const int32_t *topk_idx, int32_t *counts,
+                                 int32_t *offsets, int32_t *perm_token, int32_t *row_of,
+                                 void *x_perm, int32_t *status, moe_stream_t stream);
+
 /* Expert FFN on the expert-contiguous rows: rows offsets[e] .. offsets[e+1]-1
  * of x_perm go through expert e ([SGMoE-note] "Sparsely-Gated MoE 层架构":
  * one hidden ReLU layer):  y_perm = ReLU(x_perm W1_e^T + b1_e) W2_e^T + b2_e.

@@ -16,7 +16,7 @@ STATUS_NONFINITE, STATUS_BAD_INDEX, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 EXPORTS = ("moe_strerror", "moe_validate", "moe_capacity", "moe_workspace_size", "moe_gate",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_balance_losses", "moe_forward",
            "moe_trace_enable", "moe_trace_reset", "moe_trace_count", "moe_trace_get",
-           "moe_launch_count")
+           "moe_launch_count", "moe_dispatch_noalloc")
 
 
 class moe_config(C.Structure):
@@ -60,6 +60,7 @@ def load():
     L.moe_workspace_size.argtypes = [cfgp, C.POINTER(C.c_size_t)]
     L.moe_gate.argtypes = [cfgp, vp, C.POINTER(moe_gate_params), vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_dispatch.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.moe_dispatch_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_expert_ffn.argtypes = [cfgp, vp, vp, C.POINTER(moe_expert_params), vp, vp, sz, vp, vp]
     L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_balance_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
