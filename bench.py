@@ -164,6 +164,10 @@ def kernel_work(w, name: str, S_kept: int):
         return "tensor", 2.0 * S_kept * d * f, n * d * f * esz + S_kept * f * esz + S_kept * d * esz
     if name == "gate_gemm_fp32":
         return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
+    if name == "gate_gemm_tf32x3":
+        # the fp32-equivalent contraction; three tf32 MMAs carry it
+        return "tensor_tf32x3", 2.0 * T * d * ng * (2 if w.noise else 1), \
+            4 * (2 * T * d + 2 * d * ng * 2 + 2 * T * ng)
     if name == "route_topk":
         return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
     if name == "combine":
@@ -282,6 +286,11 @@ def run_ours(args, w, world, rank, local):
         else:
             roof = {"bound": "tensor", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": sustained,
                     "unit": "TFLOP/s"}
+    elif bound == "tensor_tf32x3":
+        # tf32 dense peak = bf16 peak / 2 (nominal ratio); three MMAs per product
+        tf32_peak = sustained / 2.0
+        roof = {"bound": "tensor", "achieved": 3 * flops / (dom_ms / 1e3) / 1e12, "peak": tf32_peak,
+                "unit": "TFLOP/s (tf32, 3 MMAs per fp32 product)"}
     elif bound == "alu":
         fp32_peak = SMS * FP32_LANES * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
         roof = {"bound": "alu", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": round(fp32_peak, 1),
@@ -310,6 +319,8 @@ def run_ours(args, w, world, rank, local):
         "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k,
                    "d_ff": w.f, "hier": [w.hier_a, w.hier_b] if w.hier_a else None,
                    "router": "switch-top1" if w.router else "noisy-top-k",
+                   "gate": "3-pass TF32 on tensor cores (fp32-level)" if w.gate_precision
+                   else "fp32 multiply-adds",
                    "capacity_factor": w.capacity_factor or None,
                    "l2": "flushed before every timed step (256 MiB write)",
                    "parallelism": f"replicas x{world}"},
@@ -395,13 +406,15 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--workload", default="lm-flat")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
+                    help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
 
     from sparsely_gated_mixture_gate_b200 import synth
-    w = synth.WORKLOADS[args.workload]
+    w = synth.WORKLOADS[args.workload].with_(gate_precision=1 if args.gate == "tf32x3" else 0)
     world, rank, local = dist_info()
 
     if args.impl == "reference":

@@ -72,6 +72,12 @@ enum {
 
 enum { MOE_ROUTER_NOISY_TOPK = 0, MOE_ROUTER_SWITCH = 1 };
 enum { MOE_F32 = 0, MOE_BF16 = 1 };
+/* How the gate's fp32 projections x W_g, x W_noise are computed:
+ * MOE_GATE_FP32   fp32 fused multiply-adds on the CUDA cores;
+ * MOE_GATE_TF32X3 tensor cores with a three-pass TF32 split (hi*hi + hi*lo +
+ *                 lo*hi, hi = nearest tf32, lo = remainder), fp32 accumulation:
+ *                 about the accuracy of fp32 multiply-adds, several times faster. */
+enum { MOE_GATE_FP32 = 0, MOE_GATE_TF32X3 = 1 };
 
 /* bits OR-ed into *status by the kernels */
 enum {
@@ -90,17 +96,19 @@ enum {
  *   MOE_ROUTER_SWITCH ([MoE-deep] §3.1: softmax over all experts, top-1, gate
  *   = the winner's probability, no noise).
  *   noise: 1 adds StandardNormal() * Softplus(x W_noise); the deviate for
- *   (seed, token t, expert i, gate g) is the cosine branch of Box-Muller on
- *   Philox4x32-10 words with key (seed lo, seed hi) and counter
- *   (t, i/2, g, 0) -- words 0,1 for even i, words 2,3 for odd i; g = 0 for
- *   the flat/primary gate and 1+group for a secondary gate.
+ *   (seed, token t, expert i, gate g) comes from Philox4x32-10 with key
+ *   (seed lo, seed hi) and counter (t, i/4, g, 0): words 0,1 give the cosine
+ *   and sine branches of one Box-Muller transform for experts 4m, 4m+1,
+ *   words 2,3 those of a second one for 4m+2, 4m+3; g = 0 for the
+ *   flat/primary gate and 1+group for a secondary gate.
  *   capacity_factor > 0 limits every expert to C = ceil(T*k*cf/n) slots
  *   ([MoE-deep] §3.2); slots beyond C (in token order) are dropped.
  *   overflow_passthrough: 1 gives a token whose every slot was dropped the
  *   output y = x (it "goes through the residual", [MoE-deep] §3.2).
  *   w_importance, w_load: weights of the two CV^2 losses ([SGMoE-xyz]
  *   "負載平衡損失"; 0.1 each in [SGMoE-note] "缺点与局限性"); alpha_aux: the
- *   Switch loss coefficient ([MoE-deep] §3.2). */
+ *   Switch loss coefficient ([MoE-deep] §3.2).  gate_precision: see
+ *   MOE_GATE_* ([SGMoE-note] "缺点与局限性": the gate needs fp32). */
 typedef struct moe_config {
   int32_t T, d, n, k, f;
   int32_t hier_a, hier_b, hier_k1, hier_k2;
@@ -111,7 +119,7 @@ typedef struct moe_config {
   double capacity_factor;
   int32_t overflow_passthrough;
   float w_importance, w_load, alpha_aux;
-  int32_t reserved;           /* must be 0 */
+  int32_t gate_precision;     /* MOE_GATE_FP32 or MOE_GATE_TF32X3 */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert

@@ -19,9 +19,10 @@
 /* deviate is drawn.  Our reading: a counter-based stream, so that every    */
 /* (seed, token, expert, gate) has one fixed deviate on any machine:        */
 /*   key = (seed low 32 bits, seed high 32 bits)                            */
-/*   ctr = (token, expert / 2, gate_id, 0)                                  */
-/*   words (w0,w1) feed the even expert of the pair, (w2,w3) the odd one,   */
-/*   each through one Box-Muller cosine branch.                             */
+/*   ctr = (token, expert / 4, gate_id, 0)                                  */
+/*   the four words feed four consecutive experts 4m .. 4m+3: words (0,1)   */
+/*   give the cosine and sine branches of one Box-Muller transform for      */
+/*   experts 4m and 4m+1, words (2,3) those of a second one for 4m+2, 4m+3. */
 /* ======================================================================= */
 
 /* Philox4x32-10 [Philox]: ten rounds of the 4x32 S-box.  Each round
@@ -52,25 +53,27 @@ void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
   out[0] = x0; out[1] = x1; out[2] = x2; out[3] = x3;
 }
 
-/* Box-Muller [Box-Muller], cosine branch.  u1 = (top 24 bits of w0 + 1)/2^24
- * lies in (0,1] so the logarithm is finite; u2 = (top 24 bits of w1)/2^24
- * lies in [0,1). */
-double orc_box_muller(uint32_t w0, uint32_t w1)
+/* Box-Muller [Box-Muller]: from two uniforms, r = sqrt(-2 ln u1) and angle
+ * 2 pi u2 give two independent standard normals r cos(2 pi u2) (branch 0) and
+ * r sin(2 pi u2) (branch 1).  u1 = (top 24 bits of w0 + 1)/2^24 lies in (0,1]
+ * so the logarithm is finite; u2 = (top 24 bits of w1)/2^24 lies in [0,1). */
+double orc_box_muller(uint32_t w0, uint32_t w1, int branch)
 {
   double u1 = ((double)(w0 >> 8) + 1.0) / 16777216.0;
   double u2 = (double)(w1 >> 8) / 16777216.0;
   const double two_pi = 6.283185307179586476925286766559;
-  return sqrt(-2.0 * log(u1)) * cos(two_pi * u2);
+  double r = sqrt(-2.0 * log(u1));
+  return branch ? r * sin(two_pi * u2) : r * cos(two_pi * u2);
 }
 
 double orc_noise(uint64_t seed, uint32_t token, uint32_t expert, uint32_t gate_id)
 {
   uint32_t key[2] = {(uint32_t)(seed & 0xffffffffu), (uint32_t)(seed >> 32)};
-  uint32_t ctr[4] = {token, expert >> 1, gate_id, 0u};
+  uint32_t ctr[4] = {token, expert >> 2, gate_id, 0u};
   uint32_t w[4];
   orc_philox4x32_10(ctr, key, w);
-  if ((expert & 1u) == 0u) return orc_box_muller(w[0], w[1]);
-  return orc_box_muller(w[2], w[3]);
+  uint32_t q = expert & 3u;
+  return orc_box_muller(w[2 * (q >> 1)], w[2 * (q >> 1) + 1], (int)(q & 1u));
 }
 
 /* ======================================================================= */
@@ -367,6 +370,10 @@ static int valid_cfg(const orc_cfg *c)
   return 1;
 }
 
+int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tokens, int ntok,
+                    int32_t *topk_idx, double *topk_gate, double *load, double *prob_sum,
+                    float *near_tie);
+
 /* Gate over a whole batch (flat, Switch or hierarchical): topk_idx /
  * topk_gate [T][k], load [n] (smoothed load, or its zero-noise limit),
  * prob_sum [n] (Switch: sum of router probabilities; else 0), near_tie [T]
@@ -381,8 +388,20 @@ static int valid_cfg(const orc_cfg *c)
 int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
                    double *topk_gate, double *load, double *prob_sum, float *near_tie)
 {
+  return orc_gate_tokens(cfg, in, NULL, cfg->T, topk_idx, topk_gate, load, prob_sum, near_tie);
+}
+
+/* The gate for a list of tokens (row r of the outputs is token tokens[r]:
+ * its x row and its noise counter); tokens == NULL means 0 .. ntok-1.  load
+ * and prob_sum are summed over the listed tokens only (for the hierarchical
+ * layer Load is a whole-batch quantity and is only meaningful for the whole
+ * batch). */
+int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tokens, int ntok,
+                    int32_t *topk_idx, double *topk_gate, double *load, double *prob_sum,
+                    float *near_tie)
+{
   if (!valid_cfg(cfg)) return -1;
-  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k;
+  const int T = ntok, d = cfg->d, n = cfg->n, k = cfg->k;
   const int hier = cfg->hier_a > 0;
   const int ng = hier ? (cfg->hier_a > cfg->hier_b ? cfg->hier_a : cfg->hier_b) : n;
 
@@ -403,8 +422,9 @@ int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
 
   if (!hier) {
     for (int t = 0; t < T; ++t) {
-      const float *xt = in->x + (size_t)t * d;
-      orc_gate_row(d, n, k, cfg->router, cfg->noise, cfg->seed, (uint32_t)t, 0u,
+      const int tok = tokens ? tokens[t] : t;
+      const float *xt = in->x + (size_t)tok * d;
+      orc_gate_row(d, n, k, cfg->router, cfg->noise, cfg->seed, (uint32_t)tok, 0u,
                    xt, in->Wg, in->bg, in->Wn, c, s, H, order, g1, pr);
       for (int j = 0; j < k; ++j) {
         topk_idx[(size_t)t * k + j] = order[j];
@@ -422,8 +442,9 @@ int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
     double *load_s = (double *)calloc((size_t)a * b, sizeof(double));
     int64_t *cnt = (int64_t *)calloc((size_t)a, sizeof(int64_t));
     for (int t = 0; t < T; ++t) {
-      const float *xt = in->x + (size_t)t * d;
-      orc_gate_row(d, a, k1, 0, cfg->noise, cfg->seed, (uint32_t)t, 0u, xt,
+      const int tok = tokens ? tokens[t] : t;
+      const float *xt = in->x + (size_t)tok * d;
+      orc_gate_row(d, a, k1, 0, cfg->noise, cfg->seed, (uint32_t)tok, 0u, xt,
                    in->Wg, in->bg, in->Wn, c, s, H, order, g1, NULL);
       float gap = min_gap(H, order, a, k1);
       orc_load_row(a, k1, cfg->noise, c, s, H, P);
@@ -435,7 +456,7 @@ int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
         const float *Wg2 = in->Wg2 + (size_t)gi * d * b;
         const float *Wn2 = in->Wn2 ? in->Wn2 + (size_t)gi * d * b : NULL;
         const float *bg2 = in->bg2 ? in->bg2 + (size_t)gi * b : NULL;
-        orc_gate_row(d, b, k2, 0, cfg->noise, cfg->seed, (uint32_t)t, (uint32_t)(1 + gi),
+        orc_gate_row(d, b, k2, 0, cfg->noise, cfg->seed, (uint32_t)tok, (uint32_t)(1 + gi),
                      xt, Wg2, bg2, Wn2, c, s, H, order, g2, NULL);
         float gap2 = min_gap(H, order, b, k2);
         if (gap2 < gap) gap = gap2;

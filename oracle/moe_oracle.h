@@ -60,7 +60,7 @@ typedef struct {
 
 /* ---- noise ------------------------------------------------------------ */
 void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]);
-double orc_box_muller(uint32_t w0, uint32_t w1);
+double orc_box_muller(uint32_t w0, uint32_t w1, int branch);
 double orc_noise(uint64_t seed, uint32_t token, uint32_t expert, uint32_t gate_id);
 
 /* ---- small helpers with a closed form ---------------------------------- */
@@ -127,6 +127,12 @@ typedef struct {
  * prob_sum [n] (may be NULL), near_tie [T] (may be NULL).  0 or -1. */
 int orc_gate_batch(const orc_cfg *cfg, const orc_inputs *in, int32_t *topk_idx,
                    double *topk_gate, double *load, double *prob_sum, float *near_tie);
+
+/* The gate for the tokens listed in tokens[0..ntok-1] (NULL: 0..ntok-1):
+ * output row r belongs to token tokens[r] (x row and noise counter). */
+int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tokens, int ntok,
+                    int32_t *topk_idx, double *topk_gate, double *load, double *prob_sum,
+                    float *near_tie);
 
 /* y[T][d] from expert rows Y[*][d] (row_of[T][k], -1 = dropped). */
 void orc_combine(int T, int k, int d, const double *Y, const double *gate,

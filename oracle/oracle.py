@@ -64,7 +64,7 @@ def lib():
         L = C.CDLL(_SO)
         vp, u32, i32, f64 = C.c_void_p, C.c_uint32, C.c_int, C.c_double
         L.orc_philox4x32_10.argtypes = [vp, vp, vp]
-        L.orc_box_muller.argtypes = [u32, u32]
+        L.orc_box_muller.argtypes = [u32, u32, i32]
         L.orc_box_muller.restype = f64
         L.orc_noise.argtypes = [C.c_uint64, u32, u32, u32]
         L.orc_noise.restype = f64
@@ -85,6 +85,9 @@ def lib():
         L.orc_expert_row.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
         L.orc_gate_batch.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, vp, vp, vp, vp]
         L.orc_gate_batch.restype = i32
+        L.orc_gate_tokens.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, i32, vp, vp, vp, vp,
+                                      vp]
+        L.orc_gate_tokens.restype = i32
         L.orc_combine.argtypes = [i32, i32, i32, vp, vp, vp, vp, i32, vp]
         L.orc_balance.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, C.c_int64, i32, f64, f64, f64,
                                   vp, vp]
@@ -111,8 +114,9 @@ def philox4x32_10(ctr, key) -> np.ndarray:
     return out
 
 
-def box_muller(w0: int, w1: int) -> float:
-    return lib().orc_box_muller(w0, w1)
+def box_muller(w0: int, w1: int, branch: int = 0) -> float:
+    """branch 0: r cos(2 pi u2); branch 1: r sin(2 pi u2)."""
+    return lib().orc_box_muller(w0, w1, branch)
 
 
 def noise(seed: int, token: int, expert: int, gate_id: int = 0) -> float:
@@ -223,6 +227,23 @@ def gate_batch(cfg: dict, inp: dict) -> dict:
                prob_sum=np.zeros(n), near_tie=np.zeros(T, np.float32))
     rc = lib().orc_gate_batch(C.byref(oc), C.byref(ins), _p(out["topk_idx"]), _p(out["topk_gate"]),
                               _p(out["load"]), _p(out["prob_sum"]), _p(out["near_tie"]))
+    if rc != 0:
+        raise ValueError(f"oracle rejected the configuration {cfg}")
+    return out
+
+
+def gate_tokens(cfg: dict, inp: dict, tokens) -> dict:
+    """The gate for the listed tokens only (x rows and noise counters of those
+    tokens); load / prob_sum are sums over the listed tokens."""
+    oc = make_cfg(**cfg)
+    keep, ins = _inputs(oc, inp)
+    toks = _c(tokens, np.int32)
+    m, n, k = toks.size, oc.n, oc.k
+    out = dict(topk_idx=np.zeros((m, k), np.int32), topk_gate=np.zeros((m, k)), load=np.zeros(n),
+               prob_sum=np.zeros(n), near_tie=np.zeros(m, np.float32))
+    rc = lib().orc_gate_tokens(C.byref(oc), C.byref(ins), _p(toks), m, _p(out["topk_idx"]),
+                               _p(out["topk_gate"]), _p(out["load"]), _p(out["prob_sum"]),
+                               _p(out["near_tie"]))
     if rc != 0:
         raise ValueError(f"oracle rejected the configuration {cfg}")
     return out

@@ -10,6 +10,7 @@ LIB_PATH = os.path.join(_HERE, "libmoe_b200.so")
 MOE_OK, MOE_EINVAL, MOE_EWORKSPACE, MOE_ECUDA, MOE_EDEVICE = 0, -1, -2, -3, -4
 ROUTER_NOISY_TOPK, ROUTER_SWITCH = 0, 1
 F32, BF16 = 0, 1
+GATE_FP32, GATE_TF32X3 = 0, 1
 STATUS_NONFINITE, STATUS_BAD_INDEX, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 
 # every symbol include/moe.h declares
@@ -26,7 +27,7 @@ class moe_config(C.Structure):
         ("router", C.c_int32), ("noise", C.c_int32), ("expert_dtype", C.c_int32),
         ("seed", C.c_uint64), ("capacity_factor", C.c_double), ("overflow_passthrough", C.c_int32),
         ("w_importance", C.c_float), ("w_load", C.c_float), ("alpha_aux", C.c_float),
-        ("reserved", C.c_int32),
+        ("gate_precision", C.c_int32),
     ]
 
 

@@ -47,25 +47,32 @@ __global__ void dispatch_hist_kernel(const int *idx, int T, int k, int n, int tp
   for (int e = threadIdx.x; e < n; e += NT) out[e] = sh[e];
 }
 
-__global__ void dispatch_scan_cols_kernel(const int *hist, int B, int n, int *base, int *counts) {
-  const int e = blockIdx.x * NT + threadIdx.x;
-  if (e >= n) return;
+// base[b][e] = sum of hist[b'][e] over b' < b.  A block takes 32 experts
+// (coalesced columns) and splits the B blocks into SC contiguous ranges:
+// range sums, their prefix in shared memory, then a second pass writes the
+// bases.  counts[e] = the total.
+constexpr int SC = 8;
+__global__ void __launch_bounds__(32 * SC) dispatch_scan_cols_kernel(const int *hist, int B, int n,
+                                                                     int *base, int *counts) {
+  __shared__ int tot[SC][33];
+  const int e = blockIdx.x * 32 + threadIdx.x;
+  const int r = threadIdx.y;
+  const int chunk = (B + SC - 1) / SC;
+  const int b0 = min(B, r * chunk), b1 = min(B, b0 + chunk);
+  int s = 0;
+  if (e < n)
+    for (int b = b0; b < b1; ++b) s += hist[(size_t)b * n + e];
+  tot[r][threadIdx.x] = s;
+  __syncthreads();
   int run = 0;
-  int b = 0;
-  for (; b + 4 <= B; b += 4) {
-    const int h0 = hist[(size_t)(b + 0) * n + e], h1 = hist[(size_t)(b + 1) * n + e];
-    const int h2 = hist[(size_t)(b + 2) * n + e], h3 = hist[(size_t)(b + 3) * n + e];
-    base[(size_t)(b + 0) * n + e] = run; run += h0;
-    base[(size_t)(b + 1) * n + e] = run; run += h1;
-    base[(size_t)(b + 2) * n + e] = run; run += h2;
-    base[(size_t)(b + 3) * n + e] = run; run += h3;
-  }
-  for (; b < B; ++b) {
+  for (int q = 0; q < r; ++q) run += tot[q][threadIdx.x];
+  if (e >= n) return;
+  for (int b = b0; b < b1; ++b) {
     const int h = hist[(size_t)b * n + e];
     base[(size_t)b * n + e] = run;
     run += h;
   }
-  counts[e] = run;
+  if (r == SC - 1) counts[e] = run;
 }
 
 // Block-wide exclusive scan: returns the sum of `v` over all threads with a
@@ -268,8 +275,8 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
     MOE_TRY(launch("dispatch_hist", dispatch_hist_kernel, dim3(B), dim3(NT), sh, st, a.idx, a.T,
                    a.k, a.n, tpb, a.hist, a.status));
     MOE_TRY(launch("dispatch_scan_cols", dispatch_scan_cols_kernel,
-                   dim3((unsigned)ceil_div(a.n, NT)), dim3(NT), 0, st, (const int *)a.hist, B, a.n,
-                   a.base, a.counts));
+                   dim3((unsigned)ceil_div(a.n, 32)), dim3(32, SC), 0, st, (const int *)a.hist, B,
+                   a.n, a.base, a.counts));
   } else {
     cudaMemsetAsync(a.counts, 0, sizeof(int) * a.n, st);
   }

@@ -8,13 +8,16 @@
 //   GEMM2: y_perm = hid_e W2_e^T + b2_e            (bf16 out)
 // Both are "grouped" GEMMs with a ragged M per expert and K-major operands.
 //
-// One persistent kernel, one CTA per SM, 192 threads:
+// One persistent kernel, one CTA per SM, 320 threads:
 //   warp 0  TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte
 //           swizzle), 4 stages, mbarrier transaction counts
 //   warp 1  MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128,
 //           N=256, K=16, four per stage; tcgen05.commit frees the stage
-//   warps 2-5  epilogue: tcgen05.ld of the 128x256 fp32 accumulator, bias,
-//           ReLU, bf16, masked stores of the expert's valid rows
+//   warps 2-9  epilogue: two warps per 32-lane quarter of tensor memory, one
+//           per 128-column half; tcgen05.ld of the fp32 accumulator 64
+//           columns at a time, bias (prefetched into registers before the
+//           wait, broadcast by shuffles), ReLU, bf16, masked stores of the
+//           expert's valid rows
 // Two accumulators of 256 columns (all 512 TMEM columns) let the epilogue of
 // one tile overlap the main loop of the next.  Tiles are ordered expert by
 // expert, N-block by N-block, M-block fastest, so the M-blocks that share a
@@ -25,18 +28,18 @@
 // that runs out sets MOE_STATUS_TIMEOUT, raises an abort flag seen by the
 // other roles, drains the copies and MMAs this CTA issued (again bounded),
 // frees its tensor memory and returns.
-#include <cuda.h>
-
-#include "internal.h"
+#include "tc_common.cuh"
 
 namespace moe {
 namespace {
+using namespace tc;
 
 constexpr int BM = kExpertBM, BN = 256, BK = 64, STAGES = 4;
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
-constexpr int NUM_THREADS = 192;
+constexpr int NUM_EPI = 256;                 // epilogue threads (warps 2-9)
+constexpr int NUM_THREADS = 64 + NUM_EPI;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int BAR_BYTES = 256;
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
@@ -57,105 +60,6 @@ struct TcArgs {
   int relu;
   int *status;
 };
-
-__device__ __forceinline__ uint32_t smem_u32(const void *p) {
-  return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
-               : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-__device__ __forceinline__ unsigned long long globaltimer() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-// Bounded wait for the phase with the given parity.  false: gave up (time
-// limit, or another role raised the abort flag).
-__device__ __noinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag,
-                                       unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = globaltimer();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0u) {
-      if (abort_flag && *abort_flag) return false;
-      if (globaltimer() - t0 > limit_ns) return false;
-    }
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *map, uint32_t bar,
-                                            int x, int y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
-                                       uint32_t accum) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(adesc), "l"(bdesc), "r"(IDESC), "r"(accum)
-      : "memory");
-}
-__device__ __forceinline__ void tc_commit(uint32_t bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   bar)
-               : "memory");
-}
-
-// Shared-memory matrix descriptor of a K-major tile in the 128-byte swizzle
-// layout that TMA writes: rows of 128 bytes, atoms of 8 rows (1024 bytes)
-// stacked at a stride of 1024 bytes.  Fields: start address >> 4 (bits
-// 0-13), leading byte offset >> 4 (bits 16-29; not used by swizzled K-major
-// layouts, set to 1), stride byte offset >> 4 (bits 32-45), version 1 (bits
-// 46-47), swizzle mode 2 = 128-byte (bits 61-63).
-__device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr) {
-  return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)1 << 16) | ((uint64_t)(1024 >> 4) << 32) |
-         ((uint64_t)1 << 46) | ((uint64_t)2 << 61);
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
-      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
-        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
-        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-      : "r"(taddr));
-  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
 
 // tile -> (expert, M-block, N-block); tiles of expert e are
 // [mprefix[e]*nblk, mprefix[e+1]*nblk), N-block major, M-block minor.
@@ -200,19 +104,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
     for (int c = 0; c < 2; ++c) {
       mbar_init(tfull(c), 1);
-      mbar_init(tempty(c), 128);
+      mbar_init(tempty(c), NUM_EPI);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
-  if (warp == 1) {
-    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                     smem_u32(tmem_slot)),
-                 "r"(TMEM_COLS)
-                 : "memory");
-    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
-  }
+  if (warp == 1) tmem_alloc(smem_u32(tmem_slot), TMEM_COLS);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -264,8 +162,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint32_t sa = sbase + stage * STAGE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < BK / 16; ++kk)
-          tc_mma(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sa + A_BYTES + kk * 32),
-                 (kb | kk) != 0);
+          tc_mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sa + A_BYTES + kk * 32), IDESC,
+                     (kb | kk) != 0);
         issued_any = true;
         tc_commit(empty(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -283,7 +181,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= 2) {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lanes 32q .. 32q+31 belong to this warp
+    const int q = warp & 3;                 // TMEM lanes 32q .. 32q+31 belong to this warp
+    const int half = (warp - 2) >> 2;       // columns [128*half, 128*half + 128) of the tile
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
@@ -291,44 +190,52 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       decode_tile(a, tile, e, mb, nbk);
       const int off = __ldg(a.offsets + e);
       const int Me = __ldg(a.offsets + e + 1) - off;
+      // bias of this warp's 128 columns, lane l holding columns l, l+32, ...;
+      // loaded before the wait so the latency hides behind the main loop
+      float breg[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int col = nbk * BN + half * 128 + u * 32 + lane;
+        breg[u] = (a.bias && col < a.N) ? __ldg(a.bias + (size_t)e * a.N + col) : 0.f;
+      }
       const int r_in = mb * BM + q * 32 + lane;
       const bool row_ok = r_in < Me;
       __nv_bfloat16 *drow = a.D + (size_t)(off + r_in) * a.N;
-      const float *brow = a.bias ? a.bias + (size_t)e * a.N : nullptr;
       // every lane waits; the outcome is made warp-uniform so that the
       // .sync.aligned tensor-memory loads below always see the full warp
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
       if (!ok) { failed = true; break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + c * 32), v);
-        const int col0 = nbk * BN + c * 32;
-        if (row_ok && col0 < a.N) {
-          uint32_t pk[16];
+      for (int c = 0; c < 2; ++c) {
+        const int cl = half * 128 + c * 64;  // column inside the tile
+        uint32_t v[64];
+        tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cl), v);
+        const int col0 = nbk * BN + cl;
+        // conversion by the whole warp (the shuffles need every lane), stores
+        // only for valid rows and columns
+        uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            float x0 = __uint_as_float(v[2 * j]), x1 = __uint_as_float(v[2 * j + 1]);
-            const int cc = col0 + 2 * j;
-            if (brow) {
-              x0 += cc < a.N ? __ldg(brow + cc) : 0.f;
-              x1 += cc + 1 < a.N ? __ldg(brow + cc + 1) : 0.f;
-            }
-            if (a.relu) {
-              x0 = fmaxf(x0, 0.f);
-              x1 = fmaxf(x1, 0.f);
-            }
-            __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-            pk[j] = *reinterpret_cast<uint32_t *>(&h);
+        for (int j = 0; j < 32; ++j) {
+          const float b0 = __shfl_sync(0xffffffffu, breg[2 * c + (j >> 4)], (2 * j) & 31);
+          const float b1 = __shfl_sync(0xffffffffu, breg[2 * c + (j >> 4)], (2 * j + 1) & 31);
+          float x0 = __uint_as_float(v[2 * j]) + b0;
+          float x1 = __uint_as_float(v[2 * j + 1]) + b1;
+          if (a.relu) {
+            x0 = fmaxf(x0, 0.f);
+            x1 = fmaxf(x1, 0.f);
           }
-          if (col0 + 32 <= a.N) {
+          __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+          pk[j] = *reinterpret_cast<uint32_t *>(&h);
+        }
+        if (row_ok && col0 < a.N) {
+          if (col0 + 64 <= a.N) {
             uint4 *dst = reinterpret_cast<uint4 *>(drow + col0);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
+            for (int u = 0; u < 8; ++u)
               dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
           } else {
-            for (int j = 0; j < 32 && col0 + j < a.N; ++j)
+            for (int j = 0; j < 64 && col0 + j < a.N; ++j)
               reinterpret_cast<uint16_t *>(drow)[col0 + j] =
                   (uint16_t)((pk[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
           }
@@ -346,52 +253,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
-                 "r"(TMEM_COLS)
-                 : "memory");
+    tmem_dealloc(tmem_base, TMEM_COLS);
   }
 }
 
 // ---------------------------------------------------------------- host side
-typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  if (!fn) {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  }
-  return fn;
-}
-
-// 2-D bf16 tensor [rows][inner] (inner contiguous), box [box_rows][64],
-// 128-byte swizzle, out-of-range elements read as zero.
-int make_map(CUtensorMap *m, const void *base, uint64_t inner, uint64_t rows, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return MOE_ECUDA;
-  cuuint64_t dims[2] = {inner, rows};
-  cuuint64_t strides[1] = {inner * 2};
-  cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
-  cuuint32_t estr[2] = {1, 1};
-  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides,
-                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  return r == CUDA_SUCCESS ? MOE_OK : MOE_ECUDA;
-}
-
 int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const float *bias, void *D,
              int relu, const int *offsets, const int *mprefix, int *status, cudaStream_t st,
              const char *name) {
   CUtensorMap ta, tb;
-  MOE_TRY(make_map(&ta, A, (uint64_t)K, (uint64_t)S, BM));
-  MOE_TRY(make_map(&tb, B, (uint64_t)K, (uint64_t)n * N, BN));
+  MOE_TRY(tc::make_map_2d(&ta, A, 2, (uint64_t)K, (uint64_t)S, BM));
+  MOE_TRY(tc::make_map_2d(&tb, B, 2, (uint64_t)K, (uint64_t)n * N, BN));
   TcArgs a;
   a.offsets = offsets;
   a.mprefix = mprefix;
@@ -421,8 +293,8 @@ int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const flo
 
 int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   if (a.S == 0) return MOE_OK;
-  int *mprefix = const_cast<int *>(a.mprefix);
-  MOE_TRY(launch_block_prefix(a.offsets, a.n, BM, mprefix, st));
+  if (!a.mprefix_ready)
+    MOE_TRY(launch_block_prefix(a.offsets, a.n, BM, const_cast<int *>(a.mprefix), st));
   MOE_TRY(run_gemm(a.x_perm, a.S, a.d, a.W1, a.n, a.f, a.b1, a.hid, 1, a.offsets, a.mprefix,
                    a.status, st, "expert_gemm1_tcgen05"));
   MOE_TRY(run_gemm(a.hid, a.S, a.f, a.W2, a.n, a.d, a.b2, a.y_perm, 0, a.offsets, a.mprefix,

@@ -66,6 +66,10 @@ struct GateGemmArgs {
   int *status;
 };
 int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st);
+// the same on the tensor cores (three-pass TF32 split); xhi/xlo: [R][d],
+// whi/wlo: [G][nb*(noise?2:1)][d] scratch
+int launch_gate_tf32x3(const GateGemmArgs &a, int mblk_upper, float *xhi, float *xlo, float *whi,
+                       float *wlo, cudaStream_t st);
 
 struct RouteArgs {
   const float *c, *s;      // [R][nb]
@@ -124,6 +128,7 @@ struct ExpertArgs {
   const void *x_perm;      // [S][d]
   const int *offsets;      // [n+1]
   const int *mprefix;      // [n+1] exclusive scan of ceil(M_e / kExpertBM)
+  int mprefix_ready;       // 1: mprefix already holds it (written by the dispatch)
   int n, d, f, S;
   const void *W1, *W2;
   const float *b1, *b2;

@@ -89,10 +89,10 @@ int num_sms() {
 }
 
 int route_rows_per_tile(int R) {
-  // about four routing tiles per SM of a 148-SM part, 16..256 rows each
-  int64_t rt = ceil_div(R, 592);
+  // about eight routing tiles per SM of a 148-SM part, 4..256 rows each
+  int64_t rt = ceil_div(R, 1184);
   rt = ceil_div(rt, 4) * 4;
-  if (rt < 16) rt = 16;
+  if (rt < 4) rt = 4;
   if (rt > 256) rt = 256;
   return (int)rt;
 }
@@ -106,6 +106,7 @@ struct Layout {
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch;
   size_t mprefix, x_perm, hid, y_perm;
+  size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
 };
@@ -180,6 +181,18 @@ Layout make_layout(const moe_config &c) {
   L.x_perm = bp.take(esz * S * (size_t)c.d);
   L.hid = bp.take(esz * S * (size_t)c.f);
   L.y_perm = bp.take(esz * S * (size_t)c.d);
+  if (c.gate_precision == MOE_GATE_TF32X3) {
+    const size_t rows = hier ? (T > R2 ? T : R2) : T;
+    const size_t nw = (size_t)(c.noise ? 2 : 1);
+    const size_t wr1 = nw * ng, wr2 = hier ? nw * (size_t)c.hier_a * c.hier_b : 0;
+    const size_t wrows = wr1 > wr2 ? wr1 : wr2;
+    L.xhi = bp.take(4 * rows * (size_t)c.d);
+    L.xlo = bp.take(4 * rows * (size_t)c.d);
+    L.whi = bp.take(4 * wrows * (size_t)c.d);
+    L.wlo = bp.take(4 * wrows * (size_t)c.d);
+  } else {
+    L.xhi = L.xlo = L.whi = L.wlo = 0;
+  }
   L.total = bp.off;
   return L;
 }
@@ -248,7 +261,13 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   g.c = cbuf;
   g.s = sbuf;
   g.status = status;
-  MOE_TRY(launch_gate_gemm(g, (int)ceil_div(c.T, kGateBM), st));
+  auto gate_gemm = [&](const GateGemmArgs &ga, int mblk_upper) -> int {
+    if (c.gate_precision == MOE_GATE_TF32X3)
+      return launch_gate_tf32x3(ga, mblk_upper, at<float>(ws, L.xhi), at<float>(ws, L.xlo),
+                                at<float>(ws, L.whi), at<float>(ws, L.wlo), st);
+    return launch_gate_gemm(ga, mblk_upper, st);
+  };
+  MOE_TRY(gate_gemm(g, (int)ceil_div(c.T, kGateBM)));
 
   RouteArgs r{};
   r.c = cbuf;
@@ -325,7 +344,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   g2.Wn = gp.W_noise2;
   g2.bias = gp.b_g2;
   g2.nb = b;
-  MOE_TRY(launch_gate_gemm(g2, (int)ceil_div(R2, kGateBM) + a, st));
+  MOE_TRY(gate_gemm(g2, (int)ceil_div(R2, kGateBM) + a));
 
   RouteArgs r2 = r;
   r2.R = R2;
@@ -358,7 +377,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
 
 int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const float *gate,
                  int64_t C, int *counts, int *offsets, int *perm_token, int *row_of, void *ws,
-                 int *status, cudaStream_t st) {
+                 int *status, cudaStream_t st, int *mprefix = nullptr) {
   DispatchArgs da{};
   da.idx = idx;
   da.T = c.T;
@@ -375,17 +394,20 @@ int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const flo
   da.perm_slot = nullptr;
   da.row_of = row_of;
   da.gate_sorted = gate ? at<float>(ws, L.gate_sorted) : nullptr;
+  da.seg_mblk = mprefix;  // expert GEMM tile prefix, when the experts follow
+  da.mblk_rows = kExpertBM;
   da.status = status;
   return launch_dispatch(da, st);
 }
 
 int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const int *offsets,
                 const moe_expert_params &ep, void *y_perm, void *ws, int *status,
-                cudaStream_t st) {
+                cudaStream_t st, int mprefix_ready = 0) {
   ExpertArgs e{};
   e.x_perm = x_perm;
   e.offsets = offsets;
   e.mprefix = at<int>(ws, L.mprefix);
+  e.mprefix_ready = mprefix_ready;
   e.n = c.n;
   e.d = c.d;
   e.f = c.f;
@@ -431,7 +453,7 @@ const char *moe_strerror(int code) {
 
 int moe_validate(const moe_config *c) {
   if (!c) return MOE_EINVAL;
-  if (c->reserved != 0) return MOE_EINVAL;
+  if (c->gate_precision != MOE_GATE_FP32 && c->gate_precision != MOE_GATE_TF32X3) return MOE_EINVAL;
   if (c->T < 0 || c->n < 1 || c->n > 8192 || c->k < 1 || c->k > kMaxK || c->k > c->n)
     return MOE_EINVAL;
   if (c->d < 8 || c->d % 8 || c->d > 16384 || c->f < 8 || c->f % 8 || c->f > 65536)
@@ -572,11 +594,12 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   void *y_perm = at<void>(ws, L.y_perm);
 
   MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st));
+  const bool tc = c.expert_dtype == MOE_BF16;
   MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, C, counts, offsets, at<int>(ws, L.perm_token),
-                       row_of, ws, status, st));
+                       row_of, ws, status, st, tc ? at<int>(ws, L.mprefix) : nullptr));
   if (c.T > 0) {
-    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, c.expert_dtype == MOE_BF16, x_perm, st));
-    MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st));
+    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, tc, x_perm, st));
+    MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));
     MOE_TRY(launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
                            c.overflow_passthrough, c.T, c.k, c.d, y, st));
   }

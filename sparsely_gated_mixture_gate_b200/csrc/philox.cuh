@@ -4,12 +4,14 @@
 // numbers: as easy as 1, 2, 3" (SC'11): ten rounds, each multiplying words 0
 // and 2 by the two round multipliers, exchanging the product halves across the
 // words and folding in the key, which is bumped by the two Weyl constants
-// between rounds.  Box-Muller (Box & Muller 1958), cosine branch, turns two
-// words into one standard normal deviate.
+// between rounds.  Box-Muller (Box & Muller 1958) turns two words into two
+// independent standard normal deviates (its cosine and sine branches).
 //
 // Stream convention (the pages only say "StandardNormal()", [SGMoE-xyz]
-// "Noisy Top-K 門控"): key (seed lo, seed hi), counter (token, expert/2,
-// gate id, 0); words (0,1) feed the even expert of the pair, (2,3) the odd one.
+// "Noisy Top-K 門控"): key (seed lo, seed hi), counter (token, expert/4,
+// gate id, 0); words (0,1) give the cosine and sine branches of one
+// Box-Muller transform for experts 4m and 4m+1, words (2,3) those of a second
+// transform for experts 4m+2 and 4m+3.
 #pragma once
 #include <stdint.h>
 
@@ -28,11 +30,16 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 ctr, uint32_t k0, uint32_t 
 }
 
 // u1 = (top 24 bits of w0 + 1) / 2^24 in (0,1], u2 = (top 24 bits of w1) / 2^24
-// in [0,1); both exact in fp32.  eps = sqrt(-2 ln u1) cos(2 pi u2).
-__device__ __forceinline__ float box_muller(uint32_t w0, uint32_t w1) {
+// in [0,1); both exact in fp32.  r = sqrt(-2 ln u1); z0 = r cos(2 pi u2),
+// z1 = r sin(2 pi u2).
+__device__ __forceinline__ void box_muller2(uint32_t w0, uint32_t w1, float &z0, float &z1) {
   const float u1 = (float)((w0 >> 8) + 1u) * 5.9604644775390625e-8f;  // 2^-24
   const float u2 = (float)(w1 >> 8) * 5.9604644775390625e-8f;
-  return sqrtf(-2.0f * logf(u1)) * cospif(2.0f * u2);
+  const float r = sqrtf(-2.0f * logf(u1));
+  float sn, cs;
+  sincospif(2.0f * u2, &sn, &cs);
+  z0 = r * cs;
+  z1 = r * sn;
 }
 
 }  // namespace moe

@@ -8,12 +8,14 @@
 //     kth_excluding is the (k+1)-th largest H when i is kept, the k-th otherwise
 //   Switch router ([MoE-deep] §3.1): p = softmax(c) over all experts, the row
 //   goes to argmax p with gate p_argmax; sum_t p_i is accumulated too.
-// One warp per row; each lane scans column pairs (2m, 2m+1), which share one
-// Philox call.  Each lane keeps a sorted top-(k+1) list in registers and the
-// warp merges the 32 lists with shuffles.  Column sums of P (and of p) are
-// accumulated per warp in shared memory, summed over the 4 warps in fixed
-// order, and written per tile; route_reduce sums the tiles in fixed order,
-// so the load is bitwise reproducible.
+// Pass 1, one warp per row: each lane scans column quads 4m .. 4m+3 (16-byte
+// loads, one Philox call per quad), keeps a sorted top-(k+1) list in
+// registers, and the warp merges the 32 lists with shuffles; the row's kept
+// ids and its two thresholds go to shared memory.  Pass 2, one thread per
+// column quad: the thread walks the tile's rows in order and sums P (and the
+// Switch probabilities) in registers, then writes the tile's column sums;
+// route_reduce adds the tiles in a fixed order, so the load is bitwise
+// reproducible.
 #include <float.h>
 #include <limits.h>
 
@@ -23,7 +25,7 @@
 namespace moe {
 namespace {
 
-constexpr int NW = 4;  // warps per routing block
+constexpr int NW = 8;  // warps per routing block
 
 struct Cand {
   float v;
@@ -50,12 +52,18 @@ __device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
   }
 }
 
-template <int K1>
+// K1 = k + 1; MAXQ = column quads per thread (nb <= MAXQ * 4 * 256); SW =
+// Switch router (probability sums kept).
+template <int K1, int MAXQ, bool SW>
 __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
-  extern __shared__ float smem[];
+  constexpr int KM = K1 - 1;  // k
+  constexpr int PQ = SW ? MAXQ : 1;
+  __shared__ int sel_s[NW][KM];
+  __shared__ float thr_s[NW][2];   // (k+1)-th largest, k-th largest
+  __shared__ float sm_s[NW][2];    // Switch: max and sum of exp of the clean logits
+  __shared__ float4 red_s[NW * 32];
+  __shared__ float4 redp_s[NW * 32];
   const int nb = a.nb;
-  float *part = smem;                                   // [NW][nb]
-  float *psum = a.psum_part ? smem + NW * nb : nullptr; // [NW][nb]
 
   // ---- which group, which rows
   const int tile = blockIdx.x;
@@ -75,167 +83,275 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
     row_end = min(row0 + a.RT, a.R);
   }
 
-  for (int i = threadIdx.x; i < NW * nb * (psum ? 2 : 1); i += NW * 32) smem[i] = 0.f;
-  __syncthreads();
-
   const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int k = a.k;
+  const bool vec4 = (nb & 3) == 0;  // rows start 16-byte aligned
+  constexpr bool sw = SW;
   const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
   const uint32_t gate_id = a.secondary ? (uint32_t)(1 + g) : 0u;
-  float *mypart = part + w * nb;
-  float *mypsum = psum ? psum + w * nb : nullptr;
   bool bad = false;
 
-  for (int row = row0 + w; row < row_end; row += NW) {
-    const int t = a.row_token ? a.row_token[row] : row;
-    const float *crow = a.c + (size_t)row * nb;
-    const float *srow = a.s + (size_t)row * nb;
+  // pass-2 thread layout: thread per column quad; with fewer quads than
+  // threads, RG groups of threads split the rows of each block
+  const int nq = (nb + 3) >> 2;
+  const int RG = nq >= NW * 32 ? 1 : min((NW * 32) / nq, NW);
+  const int rg = nq >= NW * 32 ? 0 : (int)threadIdx.x / nq;
+  const int nqpass = (nq + NW * 32 - 1) / (NW * 32);  // quads per thread when RG == 1
+  float acc[MAXQ][4], pacc[PQ][4];
+#pragma unroll
+  for (int u = 0; u < MAXQ; ++u)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[u][j] = 0.f;
+#pragma unroll
+  for (int u = 0; u < PQ; ++u)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) pacc[u][j] = 0.f;
 
-    Cand L[K1];
-#pragma unroll
-    for (int j = 0; j < K1; ++j) { L[j].v = -INFINITY; L[j].i = INT_MAX; }
-    float mx = -INFINITY, se = 0.f;  // online softmax of c (Switch)
+  for (int rb = row0; rb < row_end; rb += NW) {
+    // ================= pass 1: routing of row rb + w (warp per row)
+    const int row = rb + w;
+    if (row < row_end) {
+      const int t = a.row_token ? a.row_token[row] : row;
+      const float *crow = a.c + (size_t)row * nb;
+      const float *srow = a.s + (size_t)row * nb;
 
-    // ---- pass 1: noisy logits, per-lane top-(k+1)
-    for (int m = lane; 2 * m < nb; m += 32) {
-      const int i0 = 2 * m, i1 = 2 * m + 1;
-      const bool has1 = i1 < nb;
-      const float c0 = crow[i0], c1 = has1 ? crow[i1] : 0.f;
-      float h0 = c0, h1 = c1;
-      if (a.noise) {
-        const uint4 wd = philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, gate_id, 0u), key0, key1);
-        const float s0 = srow[i0], s1 = has1 ? srow[i1] : 0.f;
-        h0 = fmaf(box_muller(wd.x, wd.y), s0, c0);
-        h1 = fmaf(box_muller(wd.z, wd.w), s1, c1);
-      }
-      bad |= !isfinite(h0) || (has1 && !isfinite(h1));
-      insert<K1>(L, h0, i0);
-      if (has1) insert<K1>(L, h1, i1);
-      if (a.router == MOE_ROUTER_SWITCH) {
-        const float m2 = fmaxf(mx, has1 ? fmaxf(c0, c1) : c0);
-        se = se * expf(mx - m2) + expf(c0 - m2) + (has1 ? expf(c1 - m2) : 0.f);
-        mx = m2;
-      }
-    }
+      Cand L[K1];
+#pragma unroll
+      for (int j = 0; j < K1; ++j) { L[j].v = -INFINITY; L[j].i = INT_MAX; }
+      float mx = -INFINITY, se = 0.f;  // online softmax of c (Switch)
 
-    // ---- warp merge: K1 rounds of a warp-wide arg-max with the same order
-    Cand S[K1];
+      for (int m = lane; 4 * m < nb; m += 32) {
+        const int i0 = 4 * m;
+        float cv[4], sv[4] = {0.f, 0.f, 0.f, 0.f};
+        if (vec4) {
+          const float4 c4 = *reinterpret_cast<const float4 *>(crow + i0);
+          cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+          if (a.noise) {
+            const float4 s4 = *reinterpret_cast<const float4 *>(srow + i0);
+            sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+          }
+        } else {
 #pragma unroll
-    for (int r = 0; r < K1; ++r) {
-      float bv = L[0].v;
-      int bi = L[0].i;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-        if (before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
-      }
-      S[r].v = bv;
-      S[r].i = bi;
-      if (L[0].i == bi && bi != INT_MAX) {  // the owner pops its head
-#pragma unroll
-        for (int j = 0; j < K1 - 1; ++j) L[j] = L[j + 1];
-        L[K1 - 1].v = -INFINITY;
-        L[K1 - 1].i = INT_MAX;
-      }
-    }
-
-    // ---- gates
-    float M = 0.f, SE = 1.f;
-    if (a.router == MOE_ROUTER_SWITCH) {
-      M = mx; SE = se;
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) {
-        const float om = __shfl_xor_sync(0xffffffffu, M, off);
-        const float os = __shfl_xor_sync(0xffffffffu, SE, off);
-        const float m2 = fmaxf(M, om);
-        const float a1 = (M == -INFINITY) ? 0.f : SE * expf(M - m2);
-        const float a2 = (om == -INFINITY) ? 0.f : os * expf(om - m2);
-        M = m2;
-        SE = a1 + a2;
-      }
-    }
-    float gate_j = 0.f;
-    int idx_j = 0;
-    {
-      float den = 0.f;
-#pragma unroll
-      for (int j = 0; j < K1 - 1; ++j)
-        if (j < k) den += expf(S[j].v - S[0].v);
-#pragma unroll
-      for (int j = 0; j < K1 - 1; ++j)
-        if (j == lane) {
-          idx_j = S[j].i;
-          gate_j = (a.router == MOE_ROUTER_SWITCH) ? expf(crow[S[0].i] - M) / SE
-                                                   : expf(S[j].v - S[0].v) / den;
+          for (int j = 0; j < 4; ++j) {
+            cv[j] = i0 + j < nb ? crow[i0 + j] : -INFINITY;
+            if (a.noise) sv[j] = i0 + j < nb ? srow[i0 + j] : 0.f;
+          }
         }
-    }
-    if (lane < k) {
-      int slot = lane, outrow = t;
-      float gmul = 1.f;
-      int ebase = 0;
-      if (a.secondary) {
-        const int ps = a.row_slot[row];
-        slot = ps * k + lane;
-        gmul = a.gate_mult[(size_t)t * a.k1 + ps];
-        ebase = g * a.expert_stride;
-      }
-      a.out_idx[(size_t)outrow * a.K + slot] = ebase + idx_j;
-      a.out_gate[(size_t)outrow * a.K + slot] = gmul * gate_j;
-    }
-
-    // ---- pass 2: smoothed load (and Switch probabilities)
-    const float thr_kept = S[K1 - 1].v;  // (k+1)-th largest, -inf if it does not exist
-    const float thr_out = S[K1 - 2].v;   // k-th largest
-    for (int i = lane; i < nb; i += 32) {
-      bool kept = false;
+        float h[4] = {cv[0], cv[1], cv[2], cv[3]};
+        if (a.noise) {
+          const uint4 wd =
+              philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, gate_id, 0u), key0, key1);
+          float z[4];
+          box_muller2(wd.x, wd.y, z[0], z[1]);
+          box_muller2(wd.z, wd.w, z[2], z[3]);
 #pragma unroll
-      for (int j = 0; j < K1 - 1; ++j) kept |= (S[j].i == i) && (j < k);
-      float P;
-      if (!a.noise) {
-        P = kept ? 1.f : 0.f;
-      } else {
-        const float thr = kept ? thr_kept : thr_out;
-        const float ci = crow[i], si = srow[i];
-        if (thr == -INFINITY) P = 1.f;
-        else if (si == 0.f) P = ci > thr ? 1.f : (ci < thr ? 0.f : 0.5f);
-        else P = normcdff((ci - thr) / si);
+          for (int j = 0; j < 4; ++j) h[j] = fmaf(z[j], sv[j], cv[j]);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          if (i0 + j >= nb) break;
+          bad |= !isfinite(h[j]);
+          insert<K1>(L, h[j], i0 + j);
+          if (sw) {
+            const float m2 = fmaxf(mx, cv[j]);
+            se = se * expf(mx - m2) + expf(cv[j] - m2);
+            mx = m2;
+          }
+        }
       }
-      mypart[i] += P;
-      if (mypsum) mypsum[i] += expf(crow[i] - M) / SE;
+
+      // warp merge: K1 rounds of a warp-wide arg-max with the same order
+      Cand S[K1];
+#pragma unroll
+      for (int r = 0; r < K1; ++r) {
+        float bv = L[0].v;
+        int bi = L[0].i;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+          if (before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+        }
+        S[r].v = bv;
+        S[r].i = bi;
+        if (L[0].i == bi && bi != INT_MAX) {  // the owner pops its head
+#pragma unroll
+          for (int j = 0; j < K1 - 1; ++j) L[j] = L[j + 1];
+          L[K1 - 1].v = -INFINITY;
+          L[K1 - 1].i = INT_MAX;
+        }
+      }
+
+      float M = 0.f, SE = 1.f;
+      if (sw) {
+        M = mx; SE = se;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          const float om = __shfl_xor_sync(0xffffffffu, M, off);
+          const float os = __shfl_xor_sync(0xffffffffu, SE, off);
+          const float m2 = fmaxf(M, om);
+          const float a1 = (M == -INFINITY) ? 0.f : SE * expf(M - m2);
+          const float a2 = (om == -INFINITY) ? 0.f : os * expf(om - m2);
+          M = m2;
+          SE = a1 + a2;
+        }
+      }
+
+      // gates: softmax over the kept k (Switch: the winner's full-softmax p)
+      float gate_j = 0.f;
+      int idx_j = 0;
+      {
+        float den = 0.f;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) den += expf(S[j].v - S[0].v);
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+          if (j == lane) {
+            idx_j = S[j].i;
+            gate_j = sw ? expf(crow[S[0].i] - M) / SE : expf(S[j].v - S[0].v) / den;
+          }
+      }
+      if (lane < k) {
+        int slot = lane;
+        float gmul = 1.f;
+        int ebase = 0;
+        if (a.secondary) {
+          const int ps = a.row_slot[row];
+          slot = ps * k + lane;
+          gmul = a.gate_mult[(size_t)t * a.k1 + ps];
+          ebase = g * a.expert_stride;
+        }
+        a.out_idx[(size_t)t * a.K + slot] = ebase + idx_j;
+        a.out_gate[(size_t)t * a.K + slot] = gmul * gate_j;
+      }
+      if (lane == 0) {
+#pragma unroll
+        for (int j = 0; j < KM; ++j) sel_s[w][j] = S[j].i;
+        thr_s[w][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
+        thr_s[w][1] = S[K1 - 2].v;
+        sm_s[w][0] = M;
+        sm_s[w][1] = SE;
+      }
     }
+    __syncthreads();
+
+    // ================= pass 2: this block's rows into the column sums
+    const int nrow_blk = min(NW, row_end - rb);
+    if (rg < RG) {
+#pragma unroll
+      for (int u = 0; u < MAXQ; ++u) {
+        if (u >= nqpass) break;
+        const int m = (RG == 1) ? u * NW * 32 + (int)threadIdx.x : (int)threadIdx.x % nq;
+        if (m >= nq) break;
+        const int i0 = 4 * m;
+        for (int r = rg; r < nrow_blk; r += RG) {
+          const float *crow = a.c + (size_t)(rb + r) * nb;
+          const float *srow = a.s + (size_t)(rb + r) * nb;
+          float cv[4], sv[4] = {1.f, 1.f, 1.f, 1.f};
+          if (vec4) {
+            const float4 c4 = *reinterpret_cast<const float4 *>(crow + i0);
+            cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+            if (a.noise) {
+              const float4 s4 = *reinterpret_cast<const float4 *>(srow + i0);
+              sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              cv[j] = i0 + j < nb ? crow[i0 + j] : 0.f;
+              if (a.noise) sv[j] = i0 + j < nb ? srow[i0 + j] : 1.f;
+            }
+          }
+          const float thr_kept = thr_s[r][0], thr_out = thr_s[r][1];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const int i = i0 + j;
+            bool kept = false;
+#pragma unroll
+            for (int q = 0; q < KM; ++q) kept |= (sel_s[r][q] == i);
+            float P;
+            if (!a.noise) {
+              P = kept ? 1.f : 0.f;
+            } else {
+              const float thr = kept ? thr_kept : thr_out;
+              if (thr == -INFINITY) P = 1.f;
+              else if (sv[j] == 0.f) P = cv[j] > thr ? 1.f : (cv[j] < thr ? 0.f : 0.5f);
+              else P = normcdff((cv[j] - thr) / sv[j]);
+            }
+            acc[u][j] += P;
+            if (SW) pacc[u < PQ ? u : 0][j] += expf(cv[j] - sm_s[r][0]) / sm_s[r][1];
+          }
+        }
+      }
+    }
+    __syncthreads();  // the next block of rows reuses sel_s / thr_s / sm_s
   }
   if (bad && a.status) atomicOr(a.status, MOE_STATUS_NONFINITE);
 
-  __syncthreads();
+  // ---- the tile's column sums: row groups added in group order
   float *outp = a.load_part + (size_t)tile * nb;
-  for (int i = threadIdx.x; i < nb; i += NW * 32) {
-    float sum = 0.f;
+  float *outq = sw && a.psum_part ? a.psum_part + (size_t)tile * nb : nullptr;
+  auto store4 = [&](int i0, const float *v, float *dst) {
+    if (vec4) {
+      *reinterpret_cast<float4 *>(dst + i0) = make_float4(v[0], v[1], v[2], v[3]);
+    } else {
 #pragma unroll
-    for (int q = 0; q < NW; ++q) sum += part[q * nb + i];
-    outp[i] = sum;
-  }
-  if (psum) {
-    float *outq = a.psum_part + (size_t)tile * nb;
-    for (int i = threadIdx.x; i < nb; i += NW * 32) {
-      float sum = 0.f;
+      for (int j = 0; j < 4; ++j)
+        if (i0 + j < nb) dst[i0 + j] = v[j];
+    }
+  };
+  if (RG == 1) {
 #pragma unroll
-      for (int q = 0; q < NW; ++q) sum += psum[q * nb + i];
-      outq[i] = sum;
+    for (int u = 0; u < MAXQ; ++u) {
+      if (u >= nqpass) break;
+      const int m = u * NW * 32 + (int)threadIdx.x;
+      if (m >= nq) break;
+      store4(4 * m, acc[u], outp);
+      if (SW && outq) store4(4 * m, pacc[u < PQ ? u : 0], outq);
+    }
+  } else {
+    red_s[threadIdx.x] = make_float4(acc[0][0], acc[0][1], acc[0][2], acc[0][3]);
+    redp_s[threadIdx.x] = make_float4(pacc[0][0], pacc[0][1], pacc[0][2], pacc[0][3]);
+    __syncthreads();
+    if ((int)threadIdx.x < nq) {
+      float t4[4] = {0.f, 0.f, 0.f, 0.f}, p4[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < RG; ++q) {
+        const float4 u = red_s[q * nq + threadIdx.x], v = redp_s[q * nq + threadIdx.x];
+        t4[0] += u.x; t4[1] += u.y; t4[2] += u.z; t4[3] += u.w;
+        p4[0] += v.x; p4[1] += v.y; p4[2] += v.z; p4[3] += v.w;
+      }
+      store4(4 * threadIdx.x, t4, outp);
+      if (outq) store4(4 * threadIdx.x, p4, outq);
     }
   }
 }
 
-__global__ void route_reduce_kernel(const float *part, const int *seg_tiles, int ntiles_flat,
-                                    int nb, float *out) {
+// out[g][j] = sum over the tiles of group g, in tile order within each of
+// RR interleaved lanes of tiles, then the RR partial sums in fixed order:
+// the same summation order on every run.
+constexpr int RC = 32, RR = 32;  // columns x tile-lanes per block
+__global__ void __launch_bounds__(RC * RR) route_reduce_kernel(const float *part,
+                                                               const int *seg_tiles,
+                                                               int ntiles_flat, int nb,
+                                                               float *out) {
+  __shared__ float acc[RR][RC + 1];
   const int g = blockIdx.y;
-  const int j = blockIdx.x * blockDim.x + threadIdx.x;
-  if (j >= nb) return;
+  const int j = blockIdx.x * RC + threadIdx.x;
   const int t0 = seg_tiles ? seg_tiles[g] : 0;
   const int t1 = seg_tiles ? seg_tiles[g + 1] : ntiles_flat;
   float sum = 0.f;
-  for (int t = t0; t < t1; ++t) sum += part[(size_t)t * nb + j];
-  out[(size_t)g * nb + j] = sum;
+  if (j < nb) {
+#pragma unroll 8
+    for (int t = t0 + (int)threadIdx.y; t < t1; t += RR) sum += part[(size_t)t * nb + j];
+  }
+  acc[threadIdx.y][threadIdx.x] = sum;
+  __syncthreads();
+  if (threadIdx.y == 0 && j < nb) {
+    float s = 0.f;
+#pragma unroll
+    for (int r = 0; r < RR; ++r) s += acc[r][threadIdx.x];
+    out[(size_t)g * nb + j] = s;
+  }
 }
 
 __global__ void hier_load_kernel(const float *load_p, const float *load2, const int *cnt, int a,
@@ -250,32 +366,35 @@ __global__ void hier_load_kernel(const float *load_p, const float *load2, const 
 }  // namespace
 
 int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st) {
-  const size_t smem = sizeof(float) * NW * a.nb * (a.psum_part ? 2 : 1);
-  static bool attr_done[kMaxK + 2] = {};
-  auto go = [&](auto kern, int K1) -> int {
-    if (!attr_done[K1]) {
-      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-      attr_done[K1] = true;
-    }
-    return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), smem, st, a);
+  auto go = [&](auto kern) -> int {
+    return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), 0, st, a);
   };
+  const bool wide = a.nb > 4 * 4 * NW * 32;  // more than 4096 columns
+  if (a.router == MOE_ROUTER_SWITCH) {
+    if (a.k != 1 || wide) return MOE_EINVAL;
+    return go(route_kernel<2, 4, true>);
+  }
+#define MOE_ROUTE_CASE(K1)                                                      \
+  case K1:                                                                      \
+    return wide ? go(route_kernel<K1, 8, false>) : go(route_kernel<K1, 4, false>);
   switch (a.k + 1) {
-    case 2: return go(route_kernel<2>, 2);
-    case 3: return go(route_kernel<3>, 3);
-    case 4: return go(route_kernel<4>, 4);
-    case 5: return go(route_kernel<5>, 5);
-    case 6: return go(route_kernel<6>, 6);
-    case 7: return go(route_kernel<7>, 7);
-    case 8: return go(route_kernel<8>, 8);
-    case 9: return go(route_kernel<9>, 9);
+    MOE_ROUTE_CASE(2)
+    MOE_ROUTE_CASE(3)
+    MOE_ROUTE_CASE(4)
+    MOE_ROUTE_CASE(5)
+    MOE_ROUTE_CASE(6)
+    MOE_ROUTE_CASE(7)
+    MOE_ROUTE_CASE(8)
+    MOE_ROUTE_CASE(9)
     default: return MOE_EINVAL;
   }
+#undef MOE_ROUTE_CASE
 }
 
 int launch_route_reduce(const float *part, const int *seg_tiles, int G, int ntiles_flat, int nb,
                         float *out, cudaStream_t st) {
-  dim3 grid((unsigned)ceil_div(nb, 256), G);
-  return launch("route_reduce", route_reduce_kernel, grid, dim3(256), 0, st, part, seg_tiles,
+  dim3 grid((unsigned)ceil_div(nb, RC), G);
+  return launch("route_reduce", route_reduce_kernel, grid, dim3(RC, RR), 0, st, part, seg_tiles,
                 ntiles_flat, nb, out);
 }
 

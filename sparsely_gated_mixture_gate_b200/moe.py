@@ -47,6 +47,7 @@ class Config:
     w_importance: float = 0.1
     w_load: float = 0.1
     alpha: float = 0.01
+    gate_precision: int = 0   # 0: fp32 multiply-adds, 1: tensor cores, 3-pass TF32 split
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -62,7 +63,8 @@ class Config:
                           expert_dtype=_lib.BF16 if self.expert_bf16 else _lib.F32,
                           seed=self.seed, capacity_factor=float(self.capacity_factor),
                           overflow_passthrough=self.passthrough, w_importance=self.w_importance,
-                          w_load=self.w_load, alpha_aux=self.alpha, reserved=0)
+                          w_load=self.w_load, alpha_aux=self.alpha,
+                          gate_precision=self.gate_precision)
 
     @property
     def expert_dtype(self):
@@ -75,6 +77,13 @@ def _ptr(t: Optional[torch.Tensor]):
 
 def _stream():
     return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dev(device) -> torch.device:
+    d = torch.device(device)
+    if d.type == "cuda" and d.index is None:
+        d = torch.device("cuda", torch.cuda.current_device())
+    return d
 
 
 def _need(t: Optional[torch.Tensor], name: str, dtype, shape=None, device=None, optional=False):
@@ -90,7 +99,7 @@ def _need(t: Optional[torch.Tensor], name: str, dtype, shape=None, device=None, 
         raise MoEError(f"{name} must be contiguous")
     if shape is not None and tuple(t.shape) != tuple(shape):
         raise MoEError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
-    if device is not None and t.device != device:
+    if device is not None and t.device != _dev(device):
         raise MoEError(f"{name} is on {t.device}, expected {device}")
 
 
@@ -249,7 +258,7 @@ class MoELayer:
     def __init__(self, cfg: Config, params: dict, device=None):
         self.cfg = cfg
         self.params = params
-        dev = torch.device(device) if device is not None else params["Wg"].device
+        dev = _dev(device) if device is not None else params["Wg"].device
         self.device = dev
         _check_params(cfg, params, dev)
         _lib.load()

@@ -50,6 +50,7 @@ class Workload:
     w_importance: float = 0.1
     w_load: float = 0.1
     alpha: float = 0.01
+    gate_precision: int = 0     # library option; the oracle is always fp64
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)

@@ -46,7 +46,7 @@ def test_struct_layout_matches_c(tmp_path):
 #include "{HEADER}"
 int main(void) {{
   printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config), offsetof(moe_config, seed),
-         offsetof(moe_config, capacity_factor), offsetof(moe_config, reserved),
+         offsetof(moe_config, capacity_factor), offsetof(moe_config, gate_precision),
          sizeof(moe_gate_params), sizeof(moe_expert_params),
          offsetof(moe_config, alpha_aux));
   return 0;
@@ -56,7 +56,7 @@ int main(void) {{
     subprocess.check_call(["gcc", "-std=c11", "-o", str(exe), str(src)])
     vals = [int(v) for v in subprocess.check_output([str(exe)]).split()]
     want = [C.sizeof(_lib.moe_config), _lib.moe_config.seed.offset,
-            _lib.moe_config.capacity_factor.offset, _lib.moe_config.reserved.offset,
+            _lib.moe_config.capacity_factor.offset, _lib.moe_config.gate_precision.offset,
             C.sizeof(_lib.moe_gate_params), C.sizeof(_lib.moe_expert_params),
             _lib.moe_config.alpha_aux.offset]
     assert vals == want
@@ -82,7 +82,7 @@ BAD = [
     dict(hier_a=4, hier_b=2, hier_k1=2, hier_k2=2, n=8, k=2),
     dict(hier_a=4, hier_b=2, hier_k1=5, hier_k2=1, n=8, k=5),
     dict(passthrough=2), dict(capacity_factor=float("nan")),
-    dict(raw_expert_dtype=3), dict(raw_reserved=1),
+    dict(raw_expert_dtype=3), dict(raw_gate_precision=2),
 ]
 
 

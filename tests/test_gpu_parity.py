@@ -81,9 +81,13 @@ def check_routing(out_idx, out_gate, ref, what):
     return int(tie.sum())
 
 
+GP = [pytest.param(0, id="fp32fma"), pytest.param(1, id="tf32x3")]
+
+
+@pytest.mark.parametrize("gp", GP)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_gate_matches_oracle(orc, name):
-    w = SMALL[name]
+def test_gate_matches_oracle(orc, name, gp):
+    w = SMALL[name].with_(gate_precision=gp)
     inp = synth.make_inputs(w, experts=False)
     cfg = M.Config.from_workload(w)
     out = M.gate(cfg, inp["x"].to(DEV), to_dev(inp))
@@ -249,9 +253,10 @@ def run_layer(w, inp):
     return {k: v.cpu() for k, v in out.items()}
 
 
+@pytest.mark.parametrize("gp", GP)
 @pytest.mark.parametrize("name", list(SMALL))
-def test_forward_matches_oracle(orc, name):
-    w = SMALL[name]
+def test_forward_matches_oracle(orc, name, gp):
+    w = SMALL[name].with_(gate_precision=gp)
     inp = synth.make_inputs(w)
     out = run_layer(w, inp)
     assert M.status_bits(out["status"]) == 0
@@ -302,3 +307,26 @@ def test_bad_expert_id_sets_status_and_is_ignored(orc):
     assert M.status_bits(out["status"]) == M._lib.STATUS_BAD_INDEX
     ref = orc.dispatch(idx.numpy(), 3, 2**62)
     assert np.array_equal(out["row_of"].cpu().numpy(), ref["row_of"])
+
+
+# ------------------------------------------------------------------ balance losses (stage-wise)
+@pytest.mark.parametrize("router,T,n,k,cf", [(0, 3000, 64, 4, 0.0), (0, 5000, 1000, 2, 1.0),
+                                             (1, 4096, 128, 1, 1.25), (0, 0, 16, 2, 0.0)])
+def test_balance_losses_matches_oracle(orc, router, T, n, k, cf):
+    idx = synth.random_routing(T, k, n, skew=0.9, seed=n)
+    g = torch.Generator().manual_seed(4)
+    gate = torch.rand(T, k, generator=g)
+    gate = gate / gate.sum(1, keepdim=True) if T else gate
+    C = orc.capacity(T, k, n, cf)
+    counts = orc.dispatch(idx.numpy(), n, C)["counts"]
+    load = (torch.rand(n, generator=g) * T / n * 2).numpy().astype(np.float32)
+    psum = (torch.rand(n, generator=g) * T / n).numpy().astype(np.float32) if router else None
+    cfg = M.Config(T=T, d=8, n=n, k=k, f=8, router=router, noise=0 if router else 1, capacity_factor=cf)
+    out = M.balance_losses(cfg, idx.to(DEV), gate.to(DEV), torch.from_numpy(counts).to(DEV),
+                           torch.from_numpy(load).to(DEV),
+                           torch.from_numpy(psum).to(DEV) if psum is not None else None)
+    torch.cuda.synchronize()
+    imp_ref, losses_ref = orc.balance(n, idx.numpy(), gate.double().numpy(), counts, load.astype(np.float64),
+                                      None if psum is None else psum.astype(np.float64), C, router)
+    assert_rel(out["importance"].cpu().numpy(), imp_ref, 1e-5, 1e-6, "importance")
+    assert_rel(out["losses"].cpu().numpy(), losses_ref, 1e-5, 1e-7, "losses")

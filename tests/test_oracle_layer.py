@@ -294,3 +294,21 @@ def test_gate_batch_matches_forward(orc, tiny):
     assert np.array_equal(g["topk_idx"], o["topk_idx"])
     assert np.array_equal(g["topk_gate"], o["topk_gate"])
     assert np.array_equal(g["load"], o["load"])
+
+
+def test_gate_tokens_is_gate_batch_restricted(orc, tiny):
+    """The gate of a token does not depend on the other tokens of the batch:
+    a token list gives the same rows as the whole batch."""
+    w, inp = tiny
+    npin = _np_inputs(inp)
+    full = orc.gate_batch(w.cfg(), npin)
+    toks = np.array([5, 0, 63, 17], np.int32)
+    part = orc.gate_tokens(w.cfg(), npin, toks)
+    assert np.array_equal(part["topk_idx"], full["topk_idx"][toks])
+    assert np.array_equal(part["topk_gate"], full["topk_gate"][toks])
+    hw = synth.Workload("h", T=30, d=16, n=4 * 6, k=4, f=8, hier_a=4, hier_b=6, hier_k1=2, hier_k2=2,
+                        expert_bf16=0)
+    hin = _np_inputs(synth.make_inputs(hw))
+    hf = orc.gate_batch(hw.cfg(), hin)
+    hp = orc.gate_tokens(hw.cfg(), hin, [29, 3])
+    assert np.array_equal(hp["topk_idx"], hf["topk_idx"][[29, 3]])

@@ -38,25 +38,39 @@ def test_philox_matches_triton_library(orc):
 
 
 def test_box_muller_closed_forms(orc):
-    # u1 = 1 (top 24 bits of w0 all ones) -> sqrt(-2 ln 1) = 0
-    assert orc.box_muller(0xFFFFFFFF, 0x12345678) == 0.0
-    # u2 = 0 -> cos 0 = 1: eps = sqrt(-2 ln u1); w0 = 0 -> u1 = 2^-24
-    assert orc.box_muller(0, 0) == pytest.approx(math.sqrt(48 * math.log(2)), rel=1e-15)
-    # u2 = 1/2 -> cos(pi) = -1
-    assert orc.box_muller(0, 0x80000000) == pytest.approx(-math.sqrt(48 * math.log(2)), rel=1e-15)
-    # u2 = 1/4 -> cos(pi/2) = 0
-    assert abs(orc.box_muller(0, 0x40000000)) < 1e-15
+    r24 = math.sqrt(48 * math.log(2))  # w0 = 0 -> u1 = 2^-24 -> r = sqrt(-2 ln 2^-24)
+    # u1 = 1 (top 24 bits of w0 all ones) -> r = 0 on both branches
+    assert orc.box_muller(0xFFFFFFFF, 0x12345678, 0) == 0.0
+    assert orc.box_muller(0xFFFFFFFF, 0x12345678, 1) == 0.0
+    # u2 = 0: cos = 1, sin = 0
+    assert orc.box_muller(0, 0, 0) == pytest.approx(r24, rel=1e-15)
+    assert orc.box_muller(0, 0, 1) == 0.0
+    # u2 = 1/2: cos = -1, sin = 0
+    assert orc.box_muller(0, 0x80000000, 0) == pytest.approx(-r24, rel=1e-15)
+    assert abs(orc.box_muller(0, 0x80000000, 1)) < 1e-14
+    # u2 = 1/4: cos = 0, sin = 1
+    assert abs(orc.box_muller(0, 0x40000000, 0)) < 1e-15
+    assert orc.box_muller(0, 0x40000000, 1) == pytest.approx(r24, rel=1e-15)
+    # u2 = 3/4: sin = -1
+    assert orc.box_muller(0, 0xC0000000, 1) == pytest.approx(-r24, rel=1e-15)
     # u1 = 1/2 exactly: w0 >> 8 = 2^23 - 1
-    assert orc.box_muller((2**23 - 1) << 8, 0) == pytest.approx(math.sqrt(2 * math.log(2)), rel=1e-15)
+    assert orc.box_muller((2**23 - 1) << 8, 0, 0) == pytest.approx(math.sqrt(2 * math.log(2)), rel=1e-15)
+    # the two branches lie on one circle of radius r
+    for w0, w1 in [(123456789, 987654321), (2**31, 2**30 + 12345), (77, 2**32 - 1)]:
+        c, s_ = orc.box_muller(w0, w1, 0), orc.box_muller(w0, w1, 1)
+        r = math.sqrt(-2 * math.log(((w0 >> 8) + 1) / 2**24))
+        assert c * c + s_ * s_ == pytest.approx(r * r, rel=1e-13)
 
 
 def test_noise_stream_convention(orc):
-    """The even expert of a pair takes Philox words (0,1), the odd one (2,3),
-    with counter (token, expert/2, gate, 0) and key (seed lo, seed hi)."""
+    """Experts 4m..4m+3 share counter (token, m, gate, 0) under key (seed lo,
+    seed hi): words (0,1) give the cosine / sine branches for 4m, 4m+1,
+    words (2,3) those for 4m+2, 4m+3."""
     seed = 0x0123456789ABCDEF
-    for t, e, g in [(0, 0, 0), (5, 7, 0), (123, 4094, 3), (65535, 4095, 64)]:
-        w = orc.philox4x32_10([t, e >> 1, g, 0], [seed & 0xFFFFFFFF, seed >> 32])
-        want = orc.box_muller(int(w[0]), int(w[1])) if e % 2 == 0 else orc.box_muller(int(w[2]), int(w[3]))
+    for t, e, g in [(0, 0, 0), (5, 7, 0), (123, 4094, 3), (65535, 4095, 64), (9, 1, 2), (9, 2, 2)]:
+        w = orc.philox4x32_10([t, e >> 2, g, 0], [seed & 0xFFFFFFFF, seed >> 32])
+        q = e % 4
+        want = orc.box_muller(int(w[2 * (q // 2)]), int(w[2 * (q // 2) + 1]), q % 2)
         assert orc.noise(seed, t, e, g) == want
 
 
@@ -66,10 +80,15 @@ def test_noise_is_standard_normal(orc):
     assert abs(vals.mean()) < 5 / math.sqrt(N)
     assert abs(vals.var() - 1.0) < 5 * math.sqrt(2.0 / N)
     assert scipy.stats.kstest(vals, "norm").pvalue > 1e-4
-    # even/odd partners come from disjoint words: no correlation
-    ev = vals.reshape(500, 100, 2)
-    r = np.corrcoef(ev[..., 0].ravel(), ev[..., 1].ravel())[0, 1]
-    assert abs(r) < 5 / math.sqrt(ev[..., 0].size)
+    # the cosine / sine partners and the two word pairs of one counter are
+    # uncorrelated
+    q = vals.reshape(500, 50, 4)
+    for a, b in [(0, 1), (2, 3), (0, 2), (1, 3)]:
+        r = np.corrcoef(q[..., a].ravel(), q[..., b].ravel())[0, 1]
+        assert abs(r) < 5 / math.sqrt(q[..., 0].size)
+    # cos^2 + sin^2 of one pair is a chi-square with 2 degrees of freedom
+    r2 = (q[..., 0] ** 2 + q[..., 1] ** 2).ravel()
+    assert scipy.stats.kstest(r2, "chi2", args=(2,)).pvalue > 1e-4
     # different gates / seeds give different deviates
     assert orc.noise(0, 3, 4, 0) != orc.noise(0, 3, 4, 1)
     assert orc.noise(0, 3, 4, 0) != orc.noise(1, 3, 4, 0)
