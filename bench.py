@@ -207,13 +207,11 @@ def run_ours(args, w, world, rank, local):
         raise SystemExit(f"device status {st} after warm-up")
     S_kept = int(layer.counts.clamp(max=M.capacity(cfg) if w.capacity_factor > 0 else 2**31 - 1).sum())
 
-    # ---- timed region: K device-timed steps
+    # ---- timed region: K device-timed steps (no per-kernel events inside)
     clocks = ClockSampler(local)
     time.sleep(0.3)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    M.trace_reset()
-    M.trace_enable(True)
     launches0 = M.launch_count()
     if world > 1:
         dist.barrier()
@@ -229,34 +227,69 @@ def run_ours(args, w, world, rank, local):
         dist.barrier()
     wall = time.perf_counter() - wall0
     launches = M.launch_count() - launches0
-    M.trace_enable(False)
-    per_kernel = M.trace_read()
     clk = clocks.stop()
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms, value = aggregate(total_ms, w.T, args.steps, world)
 
-    # ---- e2e: host buffers, copies inside the timed region
-    xh = x.cpu().pin_memory()
-    yh = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
-    lh = torch.empty(8, dtype=torch.float32).pin_memory()
-    xd = torch.empty_like(x)
-    e_steps = max(3, min(args.steps, 200))
-    for _ in range(3):
-        layer.forward_host(xh, yh, lh, xd)
+    # ---- second timed pass for the roofline: CUDA events recorded by the
+    # library around each of its launches, on the launching stream (the
+    # events add a little time per launch, so this pass is not the value)
+    t_steps = max(3, min(args.steps, 300))
+    M.trace_reset()
+    M.trace_enable(True)
     torch.cuda.synchronize()
-    es = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
-    ee = [torch.cuda.Event(enable_timing=True) for _ in range(e_steps)]
+    for i in range(t_steps):
+        flush.fill_(float(i))
+        layer.forward_(x)
+    torch.cuda.synchronize()
+    M.trace_enable(False)
+    per_kernel = M.trace_read()
+
+    # ---- e2e: host buffers, copies inside the timed region.  Every step
+    # copies its batch from pinned host memory and its y and losses back;
+    # consecutive steps overlap copies with compute on separate streams.
+    e_steps = max(3, min(args.steps, 200))
+    xh = x.cpu().pin_memory()
+    yh = [torch.empty(w.T, w.d, dtype=torch.float32).pin_memory() for _ in range(2)]
+    lh = [torch.empty(8, dtype=torch.float32).pin_memory() for _ in range(2)]
+    layer.forward_host_batches([xh] * 3, [yh[i & 1] for i in range(3)], [lh[i & 1] for i in range(3)])
+    torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    for i in range(e_steps):
-        flush.fill_(float(i))
-        es[i].record(stream)
-        layer.forward_host(xh, yh, lh, xd)
-        ee[i].record(stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    d2h = layer.forward_host_batches([xh] * e_steps, [yh[i & 1] for i in range(e_steps)],
+                                     [lh[i & 1] for i in range(e_steps)])
+    stream.wait_stream(d2h)
+    e1.record(stream)
     torch.cuda.synchronize()
-    e_ms, e_value = aggregate(sum(a.elapsed_time(b) for a, b in zip(es, ee)), w.T, e_steps, world)
+    e_ms, e_value = aggregate(e0.elapsed_time(e1), w.T, e_steps, world)
     st = M.status_bits(layer.status)
+
+    # ---- the other gate mode on the same weights (short run, reported apart)
+    alt = None
+    if args.alt_gate and world == 1:
+        other = 0 if w.gate_precision else 1
+        alt_layer = M.MoELayer(M.Config.from_workload(w.with_(gate_precision=other)), inp, dev)
+        for _ in range(3):
+            flush.fill_(1.0)
+            alt_layer.forward_(x)
+        torch.cuda.synchronize()
+        a_steps = max(3, min(args.steps, 300))
+        as_ = [torch.cuda.Event(enable_timing=True) for _ in range(a_steps)]
+        ae_ = [torch.cuda.Event(enable_timing=True) for _ in range(a_steps)]
+        for i in range(a_steps):
+            flush.fill_(float(i))
+            as_[i].record(stream)
+            alt_layer.forward_(x)
+            ae_[i].record(stream)
+        torch.cuda.synchronize()
+        a_ms = sum(p.elapsed_time(q) for p, q in zip(as_, ae_))
+        alt = {"gate": "tf32x3" if other else "fp32", "value": round(w.T * a_steps / (a_ms / 1e3), 1),
+               "ms_per_step": round(a_ms / a_steps, 5), "steps": a_steps,
+               "device_status": M.status_bits(alt_layer.status)}
+        del alt_layer
 
     if rank != 0:
         return None
@@ -329,10 +362,14 @@ def run_ours(args, w, world, rank, local):
         "routing_hbm_gbs": round(route_bytes / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
         "roofline": roof,
         "kernels": kstats,
+        "kernel_timing": f"second pass of {t_steps} steps, CUDA events around every library launch",
         "gpu_launches": int(launches),
         "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * 4,
-                "d2h_bytes_per_step": w.T * w.d * 4 + 32, "steps": e_steps},
+                "d2h_bytes_per_step": w.T * w.d * 4 + 32, "steps": e_steps,
+                "how": "pinned host x in, y and losses out every step; copies of neighbouring "
+                       "steps overlap compute on two copy streams"},
         "clocks": clk,
+        "alt_gate_mode": alt,
         "wall_s": round(wall, 3),
         "device_status": st,
     }
@@ -409,6 +446,8 @@ def main():
     ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
                     help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-alt-gate", dest="alt_gate", action="store_false",
+                    help="skip the short run of the other gate mode")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")

@@ -109,9 +109,18 @@ constexpr int SCAN_NT = 1024, SCAN_PER = 8;  // n <= 8192
 
 // offsets[e] = sum_{e'<e} min(count, C); ucoff: the same without the cap;
 // seg_mblk / seg_tiles: exclusive scans of ceil(kept/rows).
+// One expert's tiles of a grouped GEMM: N-block major, M-block minor.
+__device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_base, int mbe,
+                                            int row_base, int rows) {
+  for (int nbk = 0; nbk < nblk; ++nbk)
+    for (int mb = 0; mb < mbe; ++mb)
+      tab[(size_t)(mb_base * nblk + nbk * mbe + mb)] =
+          make_int4(e, row_base + mb * kExpertBM, min(kExpertBM, rows - mb * kExpertBM), nbk);
+}
+
 __global__ void __launch_bounds__(SCAN_NT) dispatch_offsets_kernel(
     const int *counts, int n, long long C, int *offsets, int *ucoff, int *seg_mblk, int mblk_rows,
-    int *seg_tiles, int tile_rows) {
+    int *seg_tiles, int tile_rows, int4 *tab1, int nblk1, int4 *tab2, int nblk2) {
   const int e0 = threadIdx.x * SCAN_PER;
   long long kept[SCAN_PER], raw[SCAN_PER], mb[SCAN_PER], tl[SCAN_PER];
 #pragma unroll
@@ -148,6 +157,19 @@ __global__ void __launch_bounds__(SCAN_NT) dispatch_offsets_kernel(
       ucoff[n] = (int)q;
       if (seg_mblk) seg_mblk[n] = (int)pm;
       if (seg_tiles) seg_tiles[n] = (int)pt;
+    }
+  }
+  if (tab1) {  // expert GEMM tile tables (seg_mblk holds the M-block prefix)
+    long long p2 = block_exclusive_scan(sk), pm2 = block_exclusive_scan(sm);
+#pragma unroll 1
+    for (int j = 0; j < SCAN_PER; ++j) {
+      const int e = e0 + j;
+      if (e < n) {
+        write_tiles(tab1, nblk1, e, (int)pm2, (int)mb[j], (int)p2, (int)kept[j]);
+        write_tiles(tab2, nblk2, e, (int)pm2, (int)mb[j], (int)p2, (int)kept[j]);
+      }
+      p2 += kept[j];
+      pm2 += mb[j];
     }
   }
 }
@@ -233,26 +255,31 @@ __global__ void dispatch_gather_kernel(const float *x, const int *row_of, int T,
   }
 }
 
-__global__ void __launch_bounds__(SCAN_NT) block_prefix_kernel(const int *offsets, int n, int rows,
-                                                               int *out) {
+__global__ void __launch_bounds__(SCAN_NT) expert_plan_kernel(const int *offsets, int n,
+                                                              int *mprefix, int4 *tab1, int nblk1,
+                                                              int4 *tab2, int nblk2) {
   const int e0 = threadIdx.x * SCAN_PER;
-  long long v[SCAN_PER];
+  long long m[SCAN_PER], mb[SCAN_PER];
 #pragma unroll
   for (int j = 0; j < SCAN_PER; ++j) {
     const int e = e0 + j;
-    const long long m = e < n ? (long long)(offsets[e + 1] - offsets[e]) : 0;
-    v[j] = (m + rows - 1) / rows;
+    m[j] = e < n ? (long long)(offsets[e + 1] - offsets[e]) : 0;
+    mb[j] = (m[j] + kExpertBM - 1) / kExpertBM;
   }
-  long long sv = 0;
+  long long sm = 0;
 #pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) sv += v[j];
-  long long p = block_exclusive_scan(sv);
-#pragma unroll
+  for (int j = 0; j < SCAN_PER; ++j) sm += mb[j];
+  long long p = block_exclusive_scan(sm);
+#pragma unroll 1
   for (int j = 0; j < SCAN_PER; ++j) {
     const int e = e0 + j;
-    if (e < n) out[e] = (int)p;
-    p += v[j];
-    if (e == n - 1) out[n] = (int)p;
+    if (e < n) {
+      mprefix[e] = (int)p;
+      write_tiles(tab1, nblk1, e, (int)p, (int)mb[j], offsets[e], (int)m[j]);
+      write_tiles(tab2, nblk2, e, (int)p, (int)mb[j], offsets[e], (int)m[j]);
+    }
+    p += mb[j];
+    if (e == n - 1) mprefix[n] = (int)p;
   }
 }
 
@@ -283,7 +310,7 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
   const long long C = a.C;
   MOE_TRY(launch("dispatch_offsets", dispatch_offsets_kernel, dim3(1), dim3(SCAN_NT), 0, st,
                  (const int *)a.counts, a.n, C, a.offsets, a.ucoff, a.seg_mblk, a.mblk_rows,
-                 a.seg_tiles, a.tile_rows));
+                 a.seg_tiles, a.tile_rows, a.tab1, a.nblk1, a.tab2, a.nblk2));
   if (B > 0)
     MOE_TRY(launch("dispatch_rank", dispatch_rank_kernel, dim3(B), dim3(128), sh, st, a.idx,
                    a.gate, a.T, a.k, a.n, tpb, C, (const int *)a.base, (const int *)a.offsets,
@@ -301,10 +328,11 @@ int launch_gather(const float *x, const int *row_of, int T, int k, int d, int bf
                 T, k, d, x_perm);
 }
 
-int launch_block_prefix(const int *offsets, int n, int rows, int *out, cudaStream_t st) {
+int launch_expert_plan(const int *offsets, int n, int *mprefix, int4 *tab1, int nblk1, int4 *tab2,
+                       int nblk2, cudaStream_t st) {
   if (n > SCAN_NT * SCAN_PER) return MOE_EINVAL;
-  return launch("expert_tile_prefix", block_prefix_kernel, dim3(1), dim3(SCAN_NT), 0, st, offsets,
-                n, rows, out);
+  return launch("expert_plan", expert_plan_kernel, dim3(1), dim3(SCAN_NT), 0, st, offsets, n,
+                mprefix, tab1, nblk1, tab2, nblk2);
 }
 
 }  // namespace moe

@@ -52,31 +52,14 @@ constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >
                            ((uint32_t)(BM >> 4) << 24);
 
 struct TcArgs {
-  const int *offsets;
-  const int *mprefix;
+  const int4 *tiles;     // per tile: {expert, first row, valid rows, N-block}
+  const int *mprefix;    // [n+1]; mprefix[n] * nblk tiles in total
   int n, N, K, nblk;
   const float *bias;     // [n][N] or nullptr
   __nv_bfloat16 *D;      // [S][N]
   int relu;
   int *status;
 };
-
-// tile -> (expert, M-block, N-block); tiles of expert e are
-// [mprefix[e]*nblk, mprefix[e+1]*nblk), N-block major, M-block minor.
-__device__ __forceinline__ void decode_tile(const TcArgs &a, int tile, int &e, int &mb, int &nbk) {
-  const int v = tile / a.nblk;
-  int lo = 0, hi = a.n - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (__ldg(a.mprefix + mid) <= v) lo = mid; else hi = mid - 1;
-  }
-  e = lo;
-  const int base = __ldg(a.mprefix + e);
-  const int mbe = __ldg(a.mprefix + e + 1) - base;
-  const int local = tile - base * a.nblk;
-  nbk = local / mbe;
-  mb = local - nbk * mbe;
-}
 
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -126,11 +109,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     int issued[STAGES];
     for (int s = 0; s < STAGES; ++s) issued[s] = -1;
+    int4 cur = blockIdx.x < total ? __ldg(a.tiles + blockIdx.x) : make_int4(0, 0, 0, 0);
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      int e, mb, nbk;
-      decode_tile(a, tile, e, mb, nbk);
-      const int row0 = __ldg(a.offsets + e) + mb * BM;
-      const int brow = e * a.N + nbk * BN;
+      // the next tile's entry is fetched while this tile's loads go out
+      const int nxt = tile + gridDim.x;
+      const int4 next = nxt < total ? __ldg(a.tiles + nxt) : cur;
+      const int row0 = cur.y;
+      const int brow = cur.x * a.N + cur.w * BN;
+      cur = next;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
         const uint32_t sa = sbase + stage * STAGE_BYTES;
@@ -186,10 +172,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      int e, mb, nbk;
-      decode_tile(a, tile, e, mb, nbk);
-      const int off = __ldg(a.offsets + e);
-      const int Me = __ldg(a.offsets + e + 1) - off;
+      const int4 ti = __ldg(a.tiles + tile);
+      const int e = ti.x, nbk = ti.w;
       // bias of this warp's 128 columns, lane l holding columns l, l+32, ...;
       // loaded before the wait so the latency hides behind the main loop
       float breg[4];
@@ -198,9 +182,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int col = nbk * BN + half * 128 + u * 32 + lane;
         breg[u] = (a.bias && col < a.N) ? __ldg(a.bias + (size_t)e * a.N + col) : 0.f;
       }
-      const int r_in = mb * BM + q * 32 + lane;
-      const bool row_ok = r_in < Me;
-      __nv_bfloat16 *drow = a.D + (size_t)(off + r_in) * a.N;
+      const int r_in = q * 32 + lane;
+      const bool row_ok = r_in < ti.z;
+      __nv_bfloat16 *drow = a.D + (size_t)(ti.y + r_in) * a.N;
       // every lane waits; the outcome is made warp-uniform so that the
       // .sync.aligned tensor-memory loads below always see the full warp
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
@@ -259,13 +243,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 // ---------------------------------------------------------------- host side
 int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const float *bias, void *D,
-             int relu, const int *offsets, const int *mprefix, int *status, cudaStream_t st,
+             int relu, const int4 *tiles, const int *mprefix, int *status, cudaStream_t st,
              const char *name) {
   CUtensorMap ta, tb;
   MOE_TRY(tc::make_map_2d(&ta, A, 2, (uint64_t)K, (uint64_t)S, BM));
   MOE_TRY(tc::make_map_2d(&tb, B, 2, (uint64_t)K, (uint64_t)n * N, BN));
   TcArgs a;
-  a.offsets = offsets;
+  a.tiles = tiles;
   a.mprefix = mprefix;
   a.n = n;
   a.N = N;
@@ -293,12 +277,15 @@ int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const flo
 
 int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   if (a.S == 0) return MOE_OK;
-  if (!a.mprefix_ready)
-    MOE_TRY(launch_block_prefix(a.offsets, a.n, BM, const_cast<int *>(a.mprefix), st));
-  MOE_TRY(run_gemm(a.x_perm, a.S, a.d, a.W1, a.n, a.f, a.b1, a.hid, 1, a.offsets, a.mprefix,
-                   a.status, st, "expert_gemm1_tcgen05"));
-  MOE_TRY(run_gemm(a.hid, a.S, a.f, a.W2, a.n, a.d, a.b2, a.y_perm, 0, a.offsets, a.mprefix,
-                   a.status, st, "expert_gemm2_tcgen05"));
+  static_assert(BN == kExpertBN, "tile tables assume the GEMM's N-block width");
+  const int nblk1 = (a.f + BN - 1) / BN, nblk2 = (a.d + BN - 1) / BN;
+  if (!a.plan_ready)
+    MOE_TRY(launch_expert_plan(a.offsets, a.n, const_cast<int *>(a.mprefix), a.tab1, nblk1, a.tab2,
+                               nblk2, st));
+  MOE_TRY(run_gemm(a.x_perm, a.S, a.d, a.W1, a.n, a.f, a.b1, a.hid, 1, a.tab1, a.mprefix, a.status,
+                   st, "expert_gemm1_tcgen05"));
+  MOE_TRY(run_gemm(a.hid, a.S, a.f, a.W2, a.n, a.d, a.b2, a.y_perm, 0, a.tab2, a.mprefix, a.status,
+                   st, "expert_gemm2_tcgen05"));
   return MOE_OK;
 }
 

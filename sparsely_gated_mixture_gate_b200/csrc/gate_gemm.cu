@@ -11,7 +11,7 @@
 // their own weights.  The output columns [0,nb) of W_g and of W_noise are
 // separate N-tiles (blockIdx.y), so one launch computes both c and s.
 //
-// Tile: 128 x 128 x 8, 256 threads, 8x8 outputs per thread held as two 4x4
+// Tile: 128 x 128 x 16, 256 threads, 8x8 outputs per thread held as two 4x4
 // quadrants (rows ty*4, 64+ty*4; cols tx*4, 64+tx*4) so the shared-memory
 // reads of a warp are broadcast / conflict free.  Double-buffered shared
 // memory, global loads of the next K-slice overlap the FMAs of the current.
@@ -20,7 +20,7 @@
 namespace moe {
 namespace {
 
-constexpr int BM = kGateBM, BN = kGateBN, BK = 8, NT = 256;
+constexpr int BM = kGateBM, BN = kGateBN, BK = 16, NT = 256;
 constexpr int APAD = 4;  // As row padding (keeps 16-byte alignment)
 
 __device__ __forceinline__ float softplus_f(float z) {
@@ -58,25 +58,31 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
   const bool vecB = (nb & 3) == 0;
 
   const int tid = threadIdx.x;
-  // A loader: row ar = tid/2, k quad aq = (tid&1)*4
-  const int ar = tid >> 1, aq = (tid & 1) * 4;
-  const int arow = row0 + ar;
-  const bool a_ok = arow < row_end;
-  const float *Arow = nullptr;
-  if (a_ok) {
-    const int tok = a.row_token ? a.row_token[arow] : arow;
-    Arow = a.x + (size_t)tok * a.d;
+  // A loader: rows ar and ar + 64 (ar = tid/4), k quad aq = (tid&3)*4
+  const int ar = tid >> 2, aq = (tid & 3) * 4;
+  const float *Arow[2] = {nullptr, nullptr};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const int arow = row0 + ar + 64 * h;
+    if (arow < row_end) {
+      const int tok = a.row_token ? a.row_token[arow] : arow;
+      Arow[h] = a.x + (size_t)tok * a.d;
+    }
   }
-  // B loader: k row bk = tid/32, col quad bc = (tid&31)*4
+  // B loader: k rows bk and bk + 8 (bk = tid/32), col quad bc = (tid&31)*4
   const int bk = tid >> 5, bc = (tid & 31) * 4;
   const int bcol = col0 + bc;
 
-  auto load_a = [&](int k0) -> float4 {
-    if (!a_ok) return make_float4(0.f, 0.f, 0.f, 0.f);
-    return __ldg(reinterpret_cast<const float4 *>(Arow + k0 + aq));
+  auto load_a = [&](int k0, int h) -> float4 {
+    if (!Arow[h]) return make_float4(0.f, 0.f, 0.f, 0.f);
+    // d is a multiple of 8: a K tail inside a 16-wide slice reads zeros
+    if (k0 + aq >= a.d) return make_float4(0.f, 0.f, 0.f, 0.f);
+    return __ldg(reinterpret_cast<const float4 *>(Arow[h] + k0 + aq));
   };
-  auto load_b = [&](int k0) -> float4 {
-    const float *p = B + (size_t)(k0 + bk) * nb + bcol;
+  auto load_b = [&](int k0, int h) -> float4 {
+    const int kr = k0 + bk + 8 * h;
+    if (kr >= a.d) return make_float4(0.f, 0.f, 0.f, 0.f);
+    const float *p = B + (size_t)kr * nb + bcol;
     if (vecB && bcol + 3 < nb) return __ldg(reinterpret_cast<const float4 *>(p));
     float4 v;
     v.x = bcol + 0 < nb ? __ldg(p + 0) : 0.f;
@@ -85,12 +91,15 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     v.w = bcol + 3 < nb ? __ldg(p + 3) : 0.f;
     return v;
   };
-  auto store_tiles = [&](int buf, float4 av, float4 bv) {
-    As[buf][aq + 0][ar] = av.x;
-    As[buf][aq + 1][ar] = av.y;
-    As[buf][aq + 2][ar] = av.z;
-    As[buf][aq + 3][ar] = av.w;
-    *reinterpret_cast<float4 *>(&Bs[buf][bk][bc]) = bv;
+  auto store_tiles = [&](int buf, const float4 (&av)[2], const float4 (&bv)[2]) {
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      As[buf][aq + 0][ar + 64 * h] = av[h].x;
+      As[buf][aq + 1][ar + 64 * h] = av[h].y;
+      As[buf][aq + 2][ar + 64 * h] = av[h].z;
+      As[buf][aq + 3][ar + 64 * h] = av[h].w;
+      *reinterpret_cast<float4 *>(&Bs[buf][bk + 8 * h][bc]) = bv[h];
+    }
   };
 
   float acc[8][8];
@@ -100,16 +109,19 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
   const int tx = tid & 15, ty = tid >> 4;
-  const int nk = a.d / BK;  // d is a multiple of 8
-  float4 av = load_a(0), bv = load_b(0);
+  const int nk = (a.d + BK - 1) / BK;
+  float4 av[2] = {load_a(0, 0), load_a(0, 1)}, bv[2] = {load_b(0, 0), load_b(0, 1)};
   store_tiles(0, av, bv);
   __syncthreads();
 
   for (int kt = 0; kt < nk; ++kt) {
     const int buf = kt & 1;
     if (kt + 1 < nk) {
-      av = load_a((kt + 1) * BK);
-      bv = load_b((kt + 1) * BK);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        av[h] = load_a((kt + 1) * BK, h);
+        bv[h] = load_b((kt + 1) * BK, h);
+      }
     }
 #pragma unroll
     for (int kk = 0; kk < BK; ++kk) {

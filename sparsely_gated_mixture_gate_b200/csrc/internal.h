@@ -116,19 +116,27 @@ struct DispatchArgs {
   int mblk_rows;
   int *seg_tiles;          // [n+1] or nullptr: exclusive scan of ceil(kept_e / tile_rows)
   int tile_rows;
+  int4 *tab1, *tab2;       // expert GEMM tile tables (see ExpertArgs), or nullptr
+  int nblk1, nblk2;
   int *status;
 };
 int launch_dispatch(const DispatchArgs &a, cudaStream_t st);
 int launch_gather(const float *x, const int *row_of, int T, int k, int d, int bf16, void *x_perm,
                   cudaStream_t st);
-// exclusive scan of ceil((offsets[e+1]-offsets[e]) / rows) into out[n+1]
-int launch_block_prefix(const int *offsets, int n, int rows, int *out, cudaStream_t st);
+// Expert GEMM plan from offsets: mprefix[n+1] = exclusive scan of
+// ceil(M_e / kExpertBM); tab1 / tab2: one int4 per tile of the two GEMMs
+// (nblk1 / nblk2 N-blocks): {expert, first row, valid rows, N-block}, tiles
+// of an expert N-block major, M-block minor.
+int launch_expert_plan(const int *offsets, int n, int *mprefix, int4 *tab1, int nblk1, int4 *tab2,
+                       int nblk2, cudaStream_t st);
+constexpr int kExpertBN = 256;
 
 struct ExpertArgs {
   const void *x_perm;      // [S][d]
   const int *offsets;      // [n+1]
   const int *mprefix;      // [n+1] exclusive scan of ceil(M_e / kExpertBM)
-  int mprefix_ready;       // 1: mprefix already holds it (written by the dispatch)
+  int4 *tab1, *tab2;       // tile tables of GEMM1 / GEMM2
+  int plan_ready;          // 1: mprefix and the tables were written by the dispatch
   int n, d, f, S;
   const void *W1, *W2;
   const float *b1, *b2;

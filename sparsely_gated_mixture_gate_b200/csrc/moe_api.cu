@@ -105,7 +105,7 @@ struct Layout {
   size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch;
-  size_t mprefix, x_perm, hid, y_perm;
+  size_t mprefix, tab1, tab2, x_perm, hid, y_perm;
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
@@ -178,6 +178,11 @@ Layout make_layout(const moe_config &c) {
   L.gate_sorted = bp.take(4 * S);
   L.counts_scratch = bp.take(4 * n);
   L.mprefix = bp.take(4 * (n + 1));
+  {
+    const size_t mb_upper = (size_t)ceil_div((int64_t)S, kExpertBM) + n;
+    L.tab1 = bp.take(16 * mb_upper * (size_t)ceil_div(c.f, kExpertBN));
+    L.tab2 = bp.take(16 * mb_upper * (size_t)ceil_div(c.d, kExpertBN));
+  }
   L.x_perm = bp.take(esz * S * (size_t)c.d);
   L.hid = bp.take(esz * S * (size_t)c.f);
   L.y_perm = bp.take(esz * S * (size_t)c.d);
@@ -377,7 +382,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
 
 int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const float *gate,
                  int64_t C, int *counts, int *offsets, int *perm_token, int *row_of, void *ws,
-                 int *status, cudaStream_t st, int *mprefix = nullptr) {
+                 int *status, cudaStream_t st, bool plan_experts = false) {
   DispatchArgs da{};
   da.idx = idx;
   da.T = c.T;
@@ -394,20 +399,28 @@ int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const flo
   da.perm_slot = nullptr;
   da.row_of = row_of;
   da.gate_sorted = gate ? at<float>(ws, L.gate_sorted) : nullptr;
-  da.seg_mblk = mprefix;  // expert GEMM tile prefix, when the experts follow
-  da.mblk_rows = kExpertBM;
+  if (plan_experts) {  // expert GEMM tile prefix and tile tables, when the experts follow
+    da.seg_mblk = at<int>(ws, L.mprefix);
+    da.mblk_rows = kExpertBM;
+    da.tab1 = at<int4>(ws, L.tab1);
+    da.tab2 = at<int4>(ws, L.tab2);
+    da.nblk1 = (int)ceil_div(c.f, kExpertBN);
+    da.nblk2 = (int)ceil_div(c.d, kExpertBN);
+  }
   da.status = status;
   return launch_dispatch(da, st);
 }
 
 int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const int *offsets,
                 const moe_expert_params &ep, void *y_perm, void *ws, int *status,
-                cudaStream_t st, int mprefix_ready = 0) {
+                cudaStream_t st, int plan_ready = 0) {
   ExpertArgs e{};
   e.x_perm = x_perm;
   e.offsets = offsets;
   e.mprefix = at<int>(ws, L.mprefix);
-  e.mprefix_ready = mprefix_ready;
+  e.tab1 = at<int4>(ws, L.tab1);
+  e.tab2 = at<int4>(ws, L.tab2);
+  e.plan_ready = plan_ready;
   e.n = c.n;
   e.d = c.d;
   e.f = c.f;
@@ -596,7 +609,7 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st));
   const bool tc = c.expert_dtype == MOE_BF16;
   MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, C, counts, offsets, at<int>(ws, L.perm_token),
-                       row_of, ws, status, st, tc ? at<int>(ws, L.mprefix) : nullptr));
+                       row_of, ws, status, st, tc));
   if (c.T > 0) {
     MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, tc, x_perm, st));
     MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));

@@ -276,17 +276,20 @@ class MoELayer:
         self.counts = torch.empty(n, dtype=torch.int32, device=dev)
         self.losses = torch.empty(8, dtype=torch.float32, device=dev)
 
-    def forward_(self, x: torch.Tensor, stream=None):
+    def forward_(self, x: torch.Tensor, stream=None, y: Optional[torch.Tensor] = None,
+                 losses: Optional[torch.Tensor] = None):
         """Run the layer on device-resident x; outputs land in this object's
-        buffers (asynchronous on the current stream)."""
+        buffers, or in y / losses when given (asynchronous on the stream)."""
         _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        y = self.y if y is None else y
+        losses = self.losses if losses is None else losses
         st = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
         _check(_lib.load().moe_forward(C.byref(self._c), _ptr(x), C.byref(self._gp), C.byref(self._ep),
-                                       _ptr(self.y), _ptr(self.topk_idx), _ptr(self.topk_gate),
+                                       _ptr(y), _ptr(self.topk_idx), _ptr(self.topk_gate),
                                        _ptr(self.importance), _ptr(self.load), _ptr(self.counts),
-                                       _ptr(self.losses), _ptr(self.ws), self.ws.numel(),
+                                       _ptr(losses), _ptr(self.ws), self.ws.numel(),
                                        _ptr(self.status), st), "moe_forward")
-        return self.y
+        return y
 
     def outputs(self) -> dict:
         return dict(y=self.y, topk_idx=self.topk_idx, topk_gate=self.topk_gate,
@@ -301,6 +304,46 @@ class MoELayer:
         self.forward_(x_dev)
         y_host.copy_(self.y, non_blocking=True)
         losses_host.copy_(self.losses, non_blocking=True)
+
+    def forward_host_batches(self, x_hosts, y_hosts, losses_hosts):
+        """End-to-end calls over a sequence of batches in pinned host memory,
+        pipelined: the copy of batch i+1 to the device and the copy of batch
+        i-1's y and losses to the host run on their own streams while batch i
+        runs on the current stream (double-buffered device copies).  Returns
+        after queuing; the caller synchronises."""
+        if not hasattr(self, "_pipe"):
+            dev = self.device
+            self._pipe = dict(
+                h2d=torch.cuda.Stream(device=dev), d2h=torch.cuda.Stream(device=dev),
+                x=[torch.empty_like(self.y) for _ in range(2)],
+                y=[torch.empty_like(self.y) for _ in range(2)],
+                losses=[torch.empty_like(self.losses) for _ in range(2)])
+        P = self._pipe
+        comp = torch.cuda.current_stream(self.device)
+        x_free = [None, None]   # event: device x buffer b may be overwritten
+        y_free = [None, None]   # event: device y buffer b has been copied out
+        for i, (xh, yh, lh) in enumerate(zip(x_hosts, y_hosts, losses_hosts)):
+            b = i & 1
+            with torch.cuda.stream(P["h2d"]):
+                if x_free[b] is not None:
+                    P["h2d"].wait_event(x_free[b])
+                P["x"][b].copy_(xh, non_blocking=True)
+                x_ready = torch.cuda.Event()
+                x_ready.record(P["h2d"])
+            comp.wait_event(x_ready)
+            if y_free[b] is not None:
+                comp.wait_event(y_free[b])
+            self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
+            done = torch.cuda.Event()
+            done.record(comp)
+            x_free[b] = done
+            with torch.cuda.stream(P["d2h"]):
+                P["d2h"].wait_event(done)
+                yh.copy_(P["y"][b], non_blocking=True)
+                lh.copy_(P["losses"][b], non_blocking=True)
+                y_free[b] = torch.cuda.Event()
+                y_free[b].record(P["d2h"])
+        return P["d2h"]
 
 
 def forward(cfg: Config, x: torch.Tensor, params: dict) -> dict:

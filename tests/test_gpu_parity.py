@@ -330,3 +330,23 @@ def test_balance_losses_matches_oracle(orc, router, T, n, k, cf):
                                       None if psum is None else psum.astype(np.float64), C, router)
     assert_rel(out["importance"].cpu().numpy(), imp_ref, 1e-5, 1e-6, "importance")
     assert_rel(out["losses"].cpu().numpy(), losses_ref, 1e-5, 1e-7, "losses")
+
+
+def test_pipelined_host_batches_match_device_calls():
+    """The overlapped host-memory path returns, batch by batch, exactly what
+    the device-resident call computes (double buffers never mix batches)."""
+    w = SMALL["lm-flat-512"]
+    inp = synth.make_inputs(w)
+    cfg = M.Config.from_workload(w)
+    layer = M.MoELayer(cfg, to_dev(inp), torch.device(DEV))
+    g = torch.Generator().manual_seed(21)
+    xs = [torch.randn(w.T, w.d, generator=g).pin_memory() for _ in range(5)]
+    ys = [torch.empty(w.T, w.d).pin_memory() for _ in range(5)]
+    ls = [torch.empty(8).pin_memory() for _ in range(5)]
+    layer.forward_host_batches(xs, ys, ls)
+    torch.cuda.synchronize()
+    for i in range(5):
+        layer.forward_(xs[i].to(DEV))
+        torch.cuda.synchronize()
+        assert torch.equal(ys[i], layer.y.cpu()), i
+        assert torch.equal(ls[i], layer.losses.cpu()), i
