@@ -58,7 +58,7 @@ template <int K1, int MAXQ, bool SW>
 __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
   constexpr int KM = K1 - 1;  // k
   constexpr int PQ = SW ? MAXQ : 1;
-  __shared__ int sel_s[NW][KM];
+  __shared__ uint32_t kept_s[NW][MAXQ * NW * 32 * 4 / 32];  // kept columns of each row, one bit each
   __shared__ float thr_s[NW][2];   // (k+1)-th largest, k-th largest
   __shared__ float sm_s[NW][2];    // Switch: max and sum of exp of the clean logits
   __shared__ float4 red_s[NW * 32];
@@ -107,9 +107,12 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) pacc[u][j] = 0.f;
 
+  const int nwords = (nb + 31) >> 5;
   for (int rb = row0; rb < row_end; rb += NW) {
     // ================= pass 1: routing of row rb + w (warp per row)
     const int row = rb + w;
+    for (int q = lane; q < nwords; q += 32) kept_s[w][q] = 0u;  // read by the last pass 2
+    __syncwarp();
     if (row < row_end) {
       const int t = a.row_token ? a.row_token[row] : row;
       const float *crow = a.c + (size_t)row * nb;
@@ -226,7 +229,8 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
       }
       if (lane == 0) {
 #pragma unroll
-        for (int j = 0; j < KM; ++j) sel_s[w][j] = S[j].i;
+        for (int j = 0; j < KM; ++j)
+          if (S[j].i >= 0 && S[j].i < nb) kept_s[w][S[j].i >> 5] |= 1u << (S[j].i & 31);
         thr_s[w][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
         thr_s[w][1] = S[K1 - 2].v;
         sm_s[w][0] = M;
@@ -263,12 +267,10 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
             }
           }
           const float thr_kept = thr_s[r][0], thr_out = thr_s[r][1];
+          const uint32_t kbits = kept_s[r][i0 >> 5] >> (i0 & 31);  // the quad's 4 bits
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            const int i = i0 + j;
-            bool kept = false;
-#pragma unroll
-            for (int q = 0; q < KM; ++q) kept |= (sel_s[r][q] == i);
+            const bool kept = (kbits >> j) & 1u;
             float P;
             if (!a.noise) {
               P = kept ? 1.f : 0.f;
@@ -276,7 +278,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
               const float thr = kept ? thr_kept : thr_out;
               if (thr == -INFINITY) P = 1.f;
               else if (sv[j] == 0.f) P = cv[j] > thr ? 1.f : (cv[j] < thr ? 0.f : 0.5f);
-              else P = normcdff((cv[j] - thr) / sv[j]);
+              else P = normcdff(__fdividef(cv[j] - thr, sv[j]));
             }
             acc[u][j] += P;
             if (SW) pacc[u < PQ ? u : 0][j] += expf(cv[j] - sm_s[r][0]) / sm_s[r][1];
@@ -284,7 +286,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
         }
       }
     }
-    __syncthreads();  // the next block of rows reuses sel_s / thr_s / sm_s
+    __syncthreads();  // the next block of rows reuses kept_s / thr_s / sm_s
   }
   if (bad && a.status) atomicOr(a.status, MOE_STATUS_NONFINITE);
 

@@ -68,6 +68,11 @@ SMALL = {
     "switch-skew-small": V["switch-skew"].with_(T=2048, d=256, n=64, f=512),
     "hier-small": W["hierarchical"].with_(T=256, d=64, n=8 * 16, hier_a=8, hier_b=16, f=128),
     "kn-equal": W["tiny-flat"].with_(T=33, n=3, k=3, d=16, f=24),
+    "k8-n64": W["lm-flat"].with_(T=200, n=64, k=8, d=64, f=64),
+    "flat-n8192": W["many-expert"].with_(T=96, n=8192, d=64, f=16),
+    "one-token": W["lm-flat"].with_(T=1, n=16, k=2, d=64, f=64),
+    "bf16-narrow": W["lm-flat"].with_(T=100, n=5, k=2, d=40, f=24),
+    "hier-nonoise": W["hierarchical"].with_(T=256, d=64, n=8 * 16, hier_a=8, hier_b=16, f=128, noise=0),
 }
 
 
