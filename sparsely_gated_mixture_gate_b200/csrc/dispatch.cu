@@ -51,7 +51,7 @@ __global__ void dispatch_hist_kernel(const int *idx, int T, int k, int n, int tp
 // (coalesced columns) and splits the B blocks into SC contiguous ranges:
 // range sums, their prefix in shared memory, then a second pass writes the
 // bases.  counts[e] = the total.
-constexpr int SC = 8;
+constexpr int SC = 32;
 __global__ void __launch_bounds__(32 * SC) dispatch_scan_cols_kernel(const int *hist, int B, int n,
                                                                      int *base, int *counts) {
   __shared__ int tot[SC][33];
@@ -121,55 +121,49 @@ __device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_b
 __global__ void __launch_bounds__(SCAN_NT) dispatch_offsets_kernel(
     const int *counts, int n, long long C, int *offsets, int *ucoff, int *seg_mblk, int mblk_rows,
     int *seg_tiles, int tile_rows, int4 *tab1, int nblk1, int4 *tab2, int nblk2) {
-  const int e0 = threadIdx.x * SCAN_PER;
-  long long kept[SCAN_PER], raw[SCAN_PER], mb[SCAN_PER], tl[SCAN_PER];
-#pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) {
-    const int e = e0 + j;
-    const long long c = e < n ? counts[e] : 0;
-    raw[j] = c;
-    kept[j] = c < C ? c : C;
-    mb[j] = mblk_rows > 0 ? (kept[j] + mblk_rows - 1) / mblk_rows : 0;
-    tl[j] = tile_rows > 0 ? (kept[j] + tile_rows - 1) / tile_rows : 0;
-  }
+  // each thread takes a contiguous run of per <= SCAN_PER experts, so that
+  // small n still spreads over the whole block
+  const int per = (n + SCAN_NT - 1) / SCAN_NT;
+  const int e0 = threadIdx.x * per;
+  auto values = [&](int e, long long &raw, long long &kept, long long &mb, long long &tl) {
+    raw = e < n ? counts[e] : 0;
+    kept = raw < C ? raw : C;
+    mb = mblk_rows > 0 ? (kept + mblk_rows - 1) / mblk_rows : 0;
+    tl = tile_rows > 0 ? (kept + tile_rows - 1) / tile_rows : 0;
+  };
   long long sk = 0, sr = 0, sm = 0, st = 0;
-#pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) { sk += kept[j]; sr += raw[j]; sm += mb[j]; st += tl[j]; }
+  for (int j = 0; j < per; ++j) {
+    long long raw, kept, mb, tl;
+    values(e0 + j, raw, kept, mb, tl);
+    sk += kept; sr += raw; sm += mb; st += tl;
+  }
   long long p = block_exclusive_scan(sk);
   long long q = block_exclusive_scan(sr);
   long long pm = block_exclusive_scan(sm);
   long long pt = block_exclusive_scan(st);
-#pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) {
+  for (int j = 0; j < per; ++j) {
     const int e = e0 + j;
+    long long raw, kept, mb, tl;
+    values(e, raw, kept, mb, tl);
     if (e < n) {
       offsets[e] = (int)p;
       ucoff[e] = (int)q;
       if (seg_mblk) seg_mblk[e] = (int)pm;
       if (seg_tiles) seg_tiles[e] = (int)pt;
+      if (tab1) {  // expert GEMM tile tables
+        write_tiles(tab1, nblk1, e, (int)pm, (int)mb, (int)p, (int)kept);
+        write_tiles(tab2, nblk2, e, (int)pm, (int)mb, (int)p, (int)kept);
+      }
     }
-    p += kept[j];
-    q += raw[j];
-    pm += mb[j];
-    pt += tl[j];
+    p += kept;
+    q += raw;
+    pm += mb;
+    pt += tl;
     if (e == n - 1) {
       offsets[n] = (int)p;
       ucoff[n] = (int)q;
       if (seg_mblk) seg_mblk[n] = (int)pm;
       if (seg_tiles) seg_tiles[n] = (int)pt;
-    }
-  }
-  if (tab1) {  // expert GEMM tile tables (seg_mblk holds the M-block prefix)
-    long long p2 = block_exclusive_scan(sk), pm2 = block_exclusive_scan(sm);
-#pragma unroll 1
-    for (int j = 0; j < SCAN_PER; ++j) {
-      const int e = e0 + j;
-      if (e < n) {
-        write_tiles(tab1, nblk1, e, (int)pm2, (int)mb[j], (int)p2, (int)kept[j]);
-        write_tiles(tab2, nblk2, e, (int)pm2, (int)mb[j], (int)p2, (int)kept[j]);
-      }
-      p2 += kept[j];
-      pm2 += mb[j];
     }
   }
 }
@@ -258,27 +252,21 @@ __global__ void dispatch_gather_kernel(const float *x, const int *row_of, int T,
 __global__ void __launch_bounds__(SCAN_NT) expert_plan_kernel(const int *offsets, int n,
                                                               int *mprefix, int4 *tab1, int nblk1,
                                                               int4 *tab2, int nblk2) {
-  const int e0 = threadIdx.x * SCAN_PER;
-  long long m[SCAN_PER], mb[SCAN_PER];
-#pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) {
-    const int e = e0 + j;
-    m[j] = e < n ? (long long)(offsets[e + 1] - offsets[e]) : 0;
-    mb[j] = (m[j] + kExpertBM - 1) / kExpertBM;
-  }
+  const int per = (n + SCAN_NT - 1) / SCAN_NT;
+  const int e0 = threadIdx.x * per;
+  auto rows = [&](int e) -> long long { return e < n ? (long long)(offsets[e + 1] - offsets[e]) : 0; };
   long long sm = 0;
-#pragma unroll
-  for (int j = 0; j < SCAN_PER; ++j) sm += mb[j];
+  for (int j = 0; j < per; ++j) sm += (rows(e0 + j) + kExpertBM - 1) / kExpertBM;
   long long p = block_exclusive_scan(sm);
-#pragma unroll 1
-  for (int j = 0; j < SCAN_PER; ++j) {
+  for (int j = 0; j < per; ++j) {
     const int e = e0 + j;
+    const long long m = rows(e), mb = (m + kExpertBM - 1) / kExpertBM;
     if (e < n) {
       mprefix[e] = (int)p;
-      write_tiles(tab1, nblk1, e, (int)p, (int)mb[j], offsets[e], (int)m[j]);
-      write_tiles(tab2, nblk2, e, (int)p, (int)mb[j], offsets[e], (int)m[j]);
+      write_tiles(tab1, nblk1, e, (int)p, (int)mb, offsets[e], (int)m);
+      write_tiles(tab2, nblk2, e, (int)p, (int)mb, offsets[e], (int)m);
     }
-    p += mb[j];
+    p += mb;
     if (e == n - 1) mprefix[n] = (int)p;
   }
 }
