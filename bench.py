@@ -168,6 +168,9 @@ def kernel_work(w, name: str, S_kept: int):
         # the fp32-equivalent contraction; three tf32 MMAs carry it
         return "tensor_tf32x3", 2.0 * T * d * ng * (2 if w.noise else 1), \
             4 * (2 * T * d + 2 * d * ng * 2 + 2 * T * ng)
+    if name == "expert_ffn_fp32":
+        # both layers of every expert on its rows, fp32 weights streamed once
+        return "hbm", 4.0 * S_kept * d * f, n * 2 * d * f * 4 + S_kept * d * 4 * 2
     if name == "route_topk":
         return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
     if name == "combine":
