@@ -201,8 +201,8 @@ MOE_API int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *t
  * allocator, or a serving loop that must not call cudaMalloc after start-up
  * (it synchronises the device and can fail under memory pressure).
  * Same arguments, outputs and status bits as moe_dispatch, without ws.  Its
- * scratch (per-block histograms and their scanned bases, uncapped offsets)
- * takes 2*B*n + n + 1 int32, B = ceil(T / t) dispatch blocks of t tokens,
+ * scratch (per-block histograms and their scanned bases, uncapped offsets,
+ * one counter) takes 2*B*n + n + 2 int32, B = ceil(T / t) dispatch blocks of t tokens,
  * t = T/296 rounded up to a multiple of 32 and clamped to [32, 256].  It
  * lives in one fixed device array of MOE_DISPATCH_NOALLOC_SCRATCH_INTS int32
  * (4 MiB) that every GPU loading the library keeps until the process exits.

@@ -6,17 +6,21 @@
 //
 // Pairs are visited in (token, slot) order.  The r-th pair of expert e goes to
 // row offsets[e] + r when r < C, offsets being the exclusive scan of
-// min(count, C): a stable counting sort, built from
-//   1. dispatch_hist      per-block histograms hist[b][e] (shared-memory atomics;
-//                         counts are order-free)
-//   2. dispatch_scan_cols base[b][e] = sum of hist[b'][e] over b' < b (one thread
-//                         per expert, blocks in order), counts[e]
-//   3. dispatch_offsets   one block: offsets / uncapped offsets / tile prefixes
-//   4. dispatch_rank      per block, one warp walks the block's pairs in order
-//                         (32 at a time, __match_any_sync groups equal experts)
-//                         and assigns ranks -> row_of, perm_token, sorted gates
-//   5. dispatch_gather    x rows copied (and cast) into their rows, one warp
-//                         per token, 16-byte stores
+// min(count, C): a stable counting sort over blocks of tpb tokens, in three
+// launches:
+//   1. dispatch_hist   per block: the block's expert ids staged in shared
+//                      memory, one warp walks its pairs in order (32 at a time,
+//                      __match_any_sync groups equal experts) and hands out
+//                      the rank of every pair among the block's pairs of the
+//                      same expert (kept in row_of until step 3) -> hist[b][e]
+//   2. dispatch_scan   base[b][e] = sum of hist[b'][e] over b' < b, counts[e];
+//                      the last block to finish (atomic ticket, no waiting)
+//                      then writes offsets / uncapped offsets / tile prefixes
+//                      and the expert GEMM tile tables
+//   3. dispatch_place  one warp per token: rank = base[b][e] + block rank ->
+//                      row_of, perm_token, sorted gates; optionally the token's
+//                      x row copied (and cast) into its expert rows, 16-byte
+//                      stores
 // No step depends on scheduling order, so the permutation is deterministic.
 #include <limits.h>
 
@@ -27,52 +31,42 @@ namespace {
 
 constexpr int NT = 256;
 
-__global__ void dispatch_hist_kernel(const int *idx, int T, int k, int n, int tpb, int *hist,
-                                     int *status) {
+// smem: cnt[n] then the block's ids [tpb * k]
+__global__ void __launch_bounds__(NT) dispatch_hist_kernel(const int *idx, int T, int k, int n,
+                                                           int tpb, int *hist, int *brank,
+                                                           int *ticket, int *status) {
   extern __shared__ int sh[];
+  int *cnt = sh, *ids = sh + n;
   const int b = blockIdx.x;
-  for (int e = threadIdx.x; e < n; e += NT) sh[e] = 0;
-  __syncthreads();
+  if (b == 0 && threadIdx.x == 0) *ticket = 0;  // the scan kernel's last-block election
   const int64_t p0 = (int64_t)b * tpb * k;
-  const int64_t p1 = min((int64_t)(b + 1) * tpb, (int64_t)T) * k;
-  bool bad = false;
-  for (int64_t p = p0 + threadIdx.x; p < p1; p += NT) {
-    const int e = idx[p];
-    if (e >= 0 && e < n) atomicAdd(&sh[e], 1);
-    else bad = true;
+  const int np = (int)(min((int64_t)(b + 1) * tpb, (int64_t)T) * k - p0);
+  for (int e = threadIdx.x; e < n; e += NT) cnt[e] = 0;
+  for (int i = threadIdx.x; i < np; i += NT) ids[i] = idx[p0 + i];
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    bool bad = false;
+    for (int q = 0; q < np; q += 32) {
+      const int i = q + lane;
+      const bool valid = i < np;
+      const int e = valid ? ids[i] : -1;
+      const bool ok = valid && e >= 0 && e < n;
+      const unsigned grp = __match_any_sync(0xffffffffu, ok ? e : n + lane);
+      const int before_me = __popc(grp & lt_mask);
+      const int r_local = ok ? cnt[e] + before_me : -1;  // -1: an id outside [0, n)
+      __syncwarp();
+      if (ok && before_me == 0) cnt[e] += __popc(grp);
+      __syncwarp();
+      if (valid) brank[p0 + i] = r_local;
+      bad |= valid && !ok;
+    }
+    if (__any_sync(0xffffffffu, bad) && lane == 0 && status) atomicOr(status, MOE_STATUS_BAD_INDEX);
   }
-  if (bad && status) atomicOr(status, MOE_STATUS_BAD_INDEX);
   __syncthreads();
   int *out = hist + (size_t)b * n;
-  for (int e = threadIdx.x; e < n; e += NT) out[e] = sh[e];
-}
-
-// base[b][e] = sum of hist[b'][e] over b' < b.  A block takes 32 experts
-// (coalesced columns) and splits the B blocks into SC contiguous ranges:
-// range sums, their prefix in shared memory, then a second pass writes the
-// bases.  counts[e] = the total.
-constexpr int SC = 32;
-__global__ void __launch_bounds__(32 * SC) dispatch_scan_cols_kernel(const int *hist, int B, int n,
-                                                                     int *base, int *counts) {
-  __shared__ int tot[SC][33];
-  const int e = blockIdx.x * 32 + threadIdx.x;
-  const int r = threadIdx.y;
-  const int chunk = (B + SC - 1) / SC;
-  const int b0 = min(B, r * chunk), b1 = min(B, b0 + chunk);
-  int s = 0;
-  if (e < n)
-    for (int b = b0; b < b1; ++b) s += hist[(size_t)b * n + e];
-  tot[r][threadIdx.x] = s;
-  __syncthreads();
-  int run = 0;
-  for (int q = 0; q < r; ++q) run += tot[q][threadIdx.x];
-  if (e >= n) return;
-  for (int b = b0; b < b1; ++b) {
-    const int h = hist[(size_t)b * n + e];
-    base[(size_t)b * n + e] = run;
-    run += h;
-  }
-  if (r == SC - 1) counts[e] = run;
+  for (int e = threadIdx.x; e < n; e += NT) out[e] = cnt[e];
 }
 
 // Block-wide exclusive scan: returns the sum of `v` over all threads with a
@@ -107,8 +101,6 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v) {
 
 constexpr int SCAN_NT = 1024, SCAN_PER = 8;  // n <= 8192
 
-// offsets[e] = sum_{e'<e} min(count, C); ucoff: the same without the cap;
-// seg_mblk / seg_tiles: exclusive scans of ceil(kept/rows).
 // One expert's tiles of a grouped GEMM: N-block major, M-block minor.
 __device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_base, int mbe,
                                             int row_base, int rows) {
@@ -118,15 +110,29 @@ __device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_b
           make_int4(e, row_base + mb * kExpertBM, min(kExpertBM, rows - mb * kExpertBM), nbk);
 }
 
-__global__ void __launch_bounds__(SCAN_NT) dispatch_offsets_kernel(
-    const int *counts, int n, long long C, int *offsets, int *ucoff, int *seg_mblk, int mblk_rows,
-    int *seg_tiles, int tile_rows, int4 *tab1, int nblk1, int4 *tab2, int nblk2) {
+struct PlanOut {
+  long long C;
+  int *offsets, *ucoff, *seg_mblk, *seg_tiles;
+  int mblk_rows, tile_rows;
+  int4 *tab1, *tab2;
+  int nblk1, nblk2;
+};
+
+// offsets[e] = sum_{e'<e} min(count, C); ucoff: the same without the cap;
+// seg_mblk / seg_tiles: exclusive scans of ceil(kept/rows); the expert GEMM
+// tile tables.  Run by one whole block of SCAN_NT threads.
+__device__ void write_plan(const int *counts, int n, const PlanOut &o) {
+  const long long C = o.C;
+  int *offsets = o.offsets, *ucoff = o.ucoff, *seg_mblk = o.seg_mblk, *seg_tiles = o.seg_tiles;
+  const int mblk_rows = o.mblk_rows, tile_rows = o.tile_rows;
+  int4 *tab1 = o.tab1, *tab2 = o.tab2;
+  const int nblk1 = o.nblk1, nblk2 = o.nblk2;
   // each thread takes a contiguous run of per <= SCAN_PER experts, so that
   // small n still spreads over the whole block
   const int per = (n + SCAN_NT - 1) / SCAN_NT;
   const int e0 = threadIdx.x * per;
   auto values = [&](int e, long long &raw, long long &kept, long long &mb, long long &tl) {
-    raw = e < n ? counts[e] : 0;
+    raw = e < n ? __ldcg(counts + e) : 0;
     kept = raw < C ? raw : C;
     mb = mblk_rows > 0 ? (kept + mblk_rows - 1) / mblk_rows : 0;
     tl = tile_rows > 0 ? (kept + tile_rows - 1) / tile_rows : 0;
@@ -168,83 +174,105 @@ __global__ void __launch_bounds__(SCAN_NT) dispatch_offsets_kernel(
   }
 }
 
-__global__ void dispatch_rank_kernel(const int *idx, const float *gate, int T, int k, int n,
-                                     int tpb, long long C, const int *base, const int *offsets,
-                                     const int *ucoff, int *row_of, int *perm_token,
-                                     int *perm_slot, float *gate_sorted) {
-  extern __shared__ int cnt[];  // [n] ranks handed out so far in this block
-  const int b = blockIdx.x;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) cnt[e] = 0;
+// base[b][e] = sum of hist[b'][e] over b' < b.  A block takes 32 experts
+// (coalesced columns) and splits the B blocks into SC contiguous ranges:
+// range sums, their prefix in shared memory, then a second pass writes the
+// bases.  counts[e] = the total.  The last block to finish writes the plan.
+constexpr int SC = SCAN_NT / 32;
+__global__ void __launch_bounds__(SCAN_NT) dispatch_scan_kernel(const int *hist, int B, int n,
+                                                                int *base, int *counts,
+                                                                int *ticket, PlanOut o) {
+  __shared__ int tot[SC][33];
+  __shared__ int last;
+  const int tx = threadIdx.x & 31, r = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + tx;
+  const int chunk = (B + SC - 1) / SC;
+  const int b0 = min(B, r * chunk), b1 = min(B, b0 + chunk);
+  int s = 0;
+  if (e < n)
+    for (int b = b0; b < b1; ++b) s += hist[(size_t)b * n + e];
+  tot[r][tx] = s;
   __syncthreads();
-  if (threadIdx.x >= 32) return;
-  const int lane = threadIdx.x;
-  const unsigned lt_mask = (1u << lane) - 1u;
-  const int64_t p0 = (int64_t)b * tpb * k;
-  const int64_t p1 = min((int64_t)(b + 1) * tpb, (int64_t)T) * k;
-  const int *bbase = base + (size_t)b * n;
-  for (int64_t q = p0; q < p1; q += 32) {
-    const int64_t p = q + lane;
-    const bool valid = p < p1;
-    const int e = valid ? idx[p] : -1;
-    const bool ok = valid && e >= 0 && e < n;
-    const unsigned grp = __match_any_sync(0xffffffffu, ok ? e : n + lane);
-    const int before_me = __popc(grp & lt_mask);
-    const int r_local = ok ? cnt[e] + before_me : 0;
-    __syncwarp();
-    if (ok && before_me == 0) cnt[e] += __popc(grp);
-    __syncwarp();
-    if (!valid) continue;
-    if (!ok) {
-      row_of[p] = -1;
-      continue;
+  int run = 0;
+  for (int q = 0; q < r; ++q) run += tot[q][tx];
+  if (e < n) {
+    for (int b = b0; b < b1; ++b) {
+      const int h = hist[(size_t)b * n + e];
+      base[(size_t)b * n + e] = run;
+      run += h;
     }
-    const int rank = bbase[e] + r_local;
-    if (gate_sorted) gate_sorted[ucoff[e] + rank] = gate[p];
-    if ((long long)rank < C) {
-      const int row = offsets[e] + rank;
-      row_of[p] = row;
-      perm_token[row] = (int)(p / k);
-      if (perm_slot) perm_slot[row] = (int)(p % k);
-    } else {
-      row_of[p] = -1;
-    }
+    if (r == SC - 1) counts[e] = run;
   }
+  // counts visible device-wide before the ticket is taken
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(ticket, 1) == (int)gridDim.x - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  write_plan(counts, n, o);
 }
 
-// x rows into their expert rows, cast to the expert dtype; warp per token.
-template <bool BF16>
-__global__ void dispatch_gather_kernel(const float *x, const int *row_of, int T, int k, int d,
-                                       void *x_perm) {
+// One warp per token.  Lanes j < k finish the pairs of the token (row_of
+// holds each pair's rank inside its block on entry, its row on exit); with
+// COPY the whole warp then writes the token's x row into its expert rows,
+// cast to bf16 for the tensor-core experts.
+template <bool COPY, bool BF16>
+__global__ void __launch_bounds__(NT) dispatch_place_kernel(
+    const int *idx, const float *gate, int T, int k, int n, int tpb, long long C,
+    const int *base, const int *offsets, const int *ucoff, int *row_of, int *perm_token,
+    int *perm_slot, float *gate_sorted, const float *x, int d, void *x_perm) {
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
-  int rows[kMaxK];
+  int myrow = -1;
+  if (lane < k) {
+    const int64_t p = (int64_t)t * k + lane;
+    const int r_local = row_of[p];
+    if (r_local >= 0) {
+      const int e = idx[p];
+      const int rank = base[(size_t)(t / tpb) * n + e] + r_local;
+      if (gate_sorted) gate_sorted[ucoff[e] + rank] = gate[p];
+      if ((long long)rank < C) {
+        myrow = offsets[e] + rank;
+        perm_token[myrow] = t;
+        if (perm_slot) perm_slot[myrow] = lane;
+      }
+    }
+    row_of[p] = myrow;
+  }
+  if constexpr (COPY) {
+    int rows[kMaxK];
 #pragma unroll
-  for (int j = 0; j < kMaxK; ++j) rows[j] = j < k ? row_of[(size_t)t * k + j] : -1;
-  const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)t * d);
-  const int nchunk = d >> 3;  // 8 elements per chunk
-  for (int c = lane; c < nchunk; c += 32) {
-    const float4 u = __ldg(xr + 2 * c), v = __ldg(xr + 2 * c + 1);
-    if (BF16) {
-      __nv_bfloat162 p0 = __floats2bfloat162_rn(u.x, u.y), p1 = __floats2bfloat162_rn(u.z, u.w);
-      __nv_bfloat162 p2 = __floats2bfloat162_rn(v.x, v.y), p3 = __floats2bfloat162_rn(v.z, v.w);
-      uint4 pk;
-      pk.x = *reinterpret_cast<uint32_t *>(&p0);
-      pk.y = *reinterpret_cast<uint32_t *>(&p1);
-      pk.z = *reinterpret_cast<uint32_t *>(&p2);
-      pk.w = *reinterpret_cast<uint32_t *>(&p3);
+    for (int j = 0; j < kMaxK; ++j) {
+      const int v = __shfl_sync(0xffffffffu, myrow, j);
+      rows[j] = j < k ? v : -1;
+    }
+    const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)t * d);
+    const int nchunk = d >> 3;  // 8 elements per chunk
+    for (int c = lane; c < nchunk; c += 32) {
+      const float4 u = __ldg(xr + 2 * c), v = __ldg(xr + 2 * c + 1);
+      if (BF16) {
+        __nv_bfloat162 p0 = __floats2bfloat162_rn(u.x, u.y), p1 = __floats2bfloat162_rn(u.z, u.w);
+        __nv_bfloat162 p2 = __floats2bfloat162_rn(v.x, v.y), p3 = __floats2bfloat162_rn(v.z, v.w);
+        uint4 pk;
+        pk.x = *reinterpret_cast<uint32_t *>(&p0);
+        pk.y = *reinterpret_cast<uint32_t *>(&p1);
+        pk.z = *reinterpret_cast<uint32_t *>(&p2);
+        pk.w = *reinterpret_cast<uint32_t *>(&p3);
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j)
-        if (rows[j] >= 0)
-          reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(x_perm) + (size_t)rows[j] * d)[c] = pk;
-    } else {
+        for (int j = 0; j < kMaxK; ++j)
+          if (rows[j] >= 0)
+            reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(x_perm) + (size_t)rows[j] * d)[c] = pk;
+      } else {
 #pragma unroll
-      for (int j = 0; j < kMaxK; ++j)
-        if (rows[j] >= 0) {
-          float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(x_perm) + (size_t)rows[j] * d);
-          dst[2 * c] = u;
-          dst[2 * c + 1] = v;
-        }
+        for (int j = 0; j < kMaxK; ++j)
+          if (rows[j] >= 0) {
+            float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(x_perm) + (size_t)rows[j] * d);
+            dst[2 * c] = u;
+            dst[2 * c + 1] = v;
+          }
+      }
     }
   }
 }
@@ -283,37 +311,41 @@ int dispatch_tokens_per_block(int T) {
 
 int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
   if (a.n > SCAN_NT * SCAN_PER) return MOE_EINVAL;
+  if (a.T > 0 && a.x && (!a.x_perm || a.d % 8)) return MOE_EINVAL;
   const int tpb = dispatch_tokens_per_block(a.T);
   const int B = (int)ceil_div(a.T, tpb);
-  const size_t sh = sizeof(int) * a.n;
   if (B > 0) {
+    const size_t sh = sizeof(int) * ((size_t)a.n + (size_t)tpb * a.k);
     MOE_TRY(launch("dispatch_hist", dispatch_hist_kernel, dim3(B), dim3(NT), sh, st, a.idx, a.T,
-                   a.k, a.n, tpb, a.hist, a.status));
-    MOE_TRY(launch("dispatch_scan_cols", dispatch_scan_cols_kernel,
-                   dim3((unsigned)ceil_div(a.n, 32)), dim3(32, SC), 0, st, (const int *)a.hist, B,
-                   a.n, a.base, a.counts));
-  } else {
-    cudaMemsetAsync(a.counts, 0, sizeof(int) * a.n, st);
+                   a.k, a.n, tpb, a.hist, a.row_of, a.ticket, a.status));
+  } else if (cudaMemsetAsync(a.ticket, 0, sizeof(int), st) != cudaSuccess) {
+    return MOE_ECUDA;
   }
+  PlanOut o;
+  o.C = a.C;
+  o.offsets = a.offsets;
+  o.ucoff = a.ucoff;
+  o.seg_mblk = a.seg_mblk;
+  o.seg_tiles = a.seg_tiles;
+  o.mblk_rows = a.mblk_rows;
+  o.tile_rows = a.tile_rows;
+  o.tab1 = a.tab1;
+  o.tab2 = a.tab2;
+  o.nblk1 = a.nblk1;
+  o.nblk2 = a.nblk2;
+  MOE_TRY(launch("dispatch_scan", dispatch_scan_kernel, dim3((unsigned)ceil_div(a.n, 32)),
+                 dim3(SCAN_NT), 0, st, (const int *)a.hist, B, a.n, a.base, a.counts, a.ticket, o));
+  if (B == 0) return MOE_OK;
+  const dim3 grid((unsigned)ceil_div(a.T, NT / 32));
   const long long C = a.C;
-  MOE_TRY(launch("dispatch_offsets", dispatch_offsets_kernel, dim3(1), dim3(SCAN_NT), 0, st,
-                 (const int *)a.counts, a.n, C, a.offsets, a.ucoff, a.seg_mblk, a.mblk_rows,
-                 a.seg_tiles, a.tile_rows, a.tab1, a.nblk1, a.tab2, a.nblk2));
-  if (B > 0)
-    MOE_TRY(launch("dispatch_rank", dispatch_rank_kernel, dim3(B), dim3(128), sh, st, a.idx,
-                   a.gate, a.T, a.k, a.n, tpb, C, (const int *)a.base, (const int *)a.offsets,
-                   (const int *)a.ucoff, a.row_of, a.perm_token, a.perm_slot, a.gate_sorted));
-  return MOE_OK;
-}
-
-int launch_gather(const float *x, const int *row_of, int T, int k, int d, int bf16, void *x_perm,
-                  cudaStream_t st) {
-  dim3 grid((unsigned)ceil_div(T, NT / 32));
-  if (bf16)
-    return launch("dispatch_gather", dispatch_gather_kernel<true>, grid, dim3(NT), 0, st, x,
-                  row_of, T, k, d, x_perm);
-  return launch("dispatch_gather", dispatch_gather_kernel<false>, grid, dim3(NT), 0, st, x, row_of,
-                T, k, d, x_perm);
+  auto place = [&](auto kern) {
+    return launch("dispatch_place", kern, grid, dim3(NT), 0, st, a.idx, a.gate, a.T, a.k, a.n, tpb,
+                  C, (const int *)a.base, (const int *)a.offsets, (const int *)a.ucoff, a.row_of,
+                  a.perm_token, a.perm_slot, a.gate_sorted, a.x, a.d, a.x_perm);
+  };
+  if (!a.x) return place(dispatch_place_kernel<false, false>);
+  if (a.x_bf16) return place(dispatch_place_kernel<true, true>);
+  return place(dispatch_place_kernel<true, false>);
 }
 
 int launch_expert_plan(const int *offsets, int n, int *mprefix, int4 *tab1, int nblk1, int4 *tab2,

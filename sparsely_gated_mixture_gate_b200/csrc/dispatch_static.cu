@@ -67,9 +67,9 @@ extern "C" int moe_dispatch_noalloc(const moe_config *cfg, const float *x, const
   auto al16 = [](const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (c.T > 0 && x && (!al16(x) || !al16(x_perm))) return MOE_EINVAL;
 
-  // scratch: hist [B][n], base [B][n], uncapped offsets [n+1]
+  // scratch: hist [B][n], base [B][n], uncapped offsets [n+1], the scan's ticket
   const int64_t B = ceil_div(c.T, dispatch_tokens_per_block(c.T));
-  const int64_t need = 2 * B * (int64_t)c.n + c.n + 1;
+  const int64_t need = 2 * B * (int64_t)c.n + c.n + 2;
   if (need > kScratchInts) return MOE_EWORKSPACE;  // beyond the fixed array
 
   int *scratch = nullptr;
@@ -94,13 +94,15 @@ extern "C" int moe_dispatch_noalloc(const moe_config *cfg, const float *x, const
   da.hist = scratch;
   da.base = scratch + B * c.n;
   da.ucoff = scratch + 2 * B * c.n;
+  da.ticket = scratch + 2 * B * c.n + c.n + 1;
+  da.x = x;
+  da.x_perm = x_perm;
+  da.d = c.d;
+  da.x_bf16 = c.expert_dtype == MOE_BF16;
   da.counts = counts;
   da.offsets = offsets;
   da.perm_token = perm_token;
   da.row_of = row_of;
   da.status = status;
-  MOE_TRY(launch_dispatch(da, st));
-  if (x && c.T > 0)
-    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, c.expert_dtype == MOE_BF16, x_perm, st));
-  return MOE_OK;
+  return launch_dispatch(da, st);
 }

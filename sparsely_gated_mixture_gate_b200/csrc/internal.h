@@ -118,11 +118,13 @@ struct DispatchArgs {
   int tile_rows;
   int4 *tab1, *tab2;       // expert GEMM tile tables (see ExpertArgs), or nullptr
   int nblk1, nblk2;
+  int *ticket;             // one int of scratch (last-block election of the scan)
+  const float *x;          // [T][d] or nullptr: with it x rows are copied to x_perm
+  void *x_perm;            // [kept rows][d], bf16 (x_bf16) or fp32
+  int d, x_bf16;
   int *status;
 };
 int launch_dispatch(const DispatchArgs &a, cudaStream_t st);
-int launch_gather(const float *x, const int *row_of, int T, int k, int d, int bf16, void *x_perm,
-                  cudaStream_t st);
 // Expert GEMM plan from offsets: mprefix[n+1] = exclusive scan of
 // ceil(M_e / kExpertBM); tab1 / tab2: one int4 per tile of the two GEMMs
 // (nblk1 / nblk2 N-blocks): {expert, first row, valid rows, N-block}, tiles

@@ -14,11 +14,33 @@
 
 namespace moe {
 
+// ---------------------------------------------------------------- side stream
+namespace {
+// moe_forward runs the balance statistics (the reduction of the smoothed Load,
+// Importance and the losses) on a second stream beside the dispatch -> experts
+// -> combine chain: they feed only the loss outputs.  Fork and join are
+// events, so the whole call stays ordered on the caller's stream.  One stream
+// and its events per device and host thread, so concurrent callers on other
+// threads never wait on one another's events.
+struct Side {
+  cudaStream_t s = nullptr;
+  cudaEvent_t fork_gate = nullptr, fork_dispatch = nullptr, join = nullptr;
+};
+thread_local std::vector<Side> t_side;  // by device
+
+bool is_side_stream(cudaStream_t st) {
+  for (const auto &sd : t_side)
+    if (sd.s && sd.s == st) return true;
+  return false;
+}
+}  // namespace
+
 // ---------------------------------------------------------------- tracing
 namespace {
 struct TraceRec {
   const char *name;
   cudaEvent_t a, b;
+  bool side;  // launched on the side stream: its time overlaps the main chain
 };
 struct TraceAgg {
   std::string name;
@@ -48,14 +70,15 @@ void trace_collect() {
     cudaEventSynchronize(r.b);
     cudaEventElapsedTime(&ms, r.a, r.b);
     bool found = false;
+    const std::string name = r.side ? std::string(r.name) + " [side stream]" : std::string(r.name);
     for (auto &g : g_agg)
-      if (g.name == r.name) {
+      if (g.name == name) {
         g.launches += 1;
         g.ms += ms;
         found = true;
         break;
       }
-    if (!found) g_agg.push_back({r.name, 1, (double)ms});
+    if (!found) g_agg.push_back({name, 1, (double)ms});
     g_pool.push_back(r.a);
     g_pool.push_back(r.b);
   }
@@ -65,7 +88,7 @@ void trace_collect() {
 
 void trace_begin(const char *name, cudaStream_t st, int *slot) {
   if (!g_trace) return;
-  TraceRec r{name, pooled_event(), pooled_event()};
+  TraceRec r{name, pooled_event(), pooled_event(), is_side_stream(st)};
   cudaEventRecord(r.a, st);
   g_pending.push_back(r);
   *slot = (int)g_pending.size() - 1;
@@ -104,7 +127,7 @@ struct Layout {
   size_t c, s, load_part, psum_part, prob_sum;
   size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
-  size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch;
+  size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch, ticket;
   size_t mprefix, tab1, tab2, x_perm, hid, y_perm;
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
@@ -177,6 +200,7 @@ Layout make_layout(const moe_config &c) {
   L.row_of = bp.take(4 * S);
   L.gate_sorted = bp.take(4 * S);
   L.counts_scratch = bp.take(4 * n);
+  L.ticket = bp.take(4);
   L.mprefix = bp.take(4 * (n + 1));
   {
     const size_t mb_upper = (size_t)ceil_div((int64_t)S, kExpertBM) + n;
@@ -239,10 +263,39 @@ int common_checks(const moe_config *cfg, void *ws, size_t ws_bytes, int32_t *sta
   return check_device();
 }
 
+// ---------------------------------------------------------------- side stream
+int side_stream(Side **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ECUDA;
+  if ((int)t_side.size() <= dev) t_side.resize(dev + 1);
+  Side &sd = t_side[dev];
+  if (!sd.s) {
+    cudaStream_t s = nullptr;
+    cudaEvent_t e[3] = {nullptr, nullptr, nullptr};
+    if (cudaStreamCreateWithFlags(&s, cudaStreamNonBlocking) != cudaSuccess) return MOE_ECUDA;
+    for (auto &ev : e)
+      if (cudaEventCreateWithFlags(&ev, cudaEventDisableTiming) != cudaSuccess) return MOE_ECUDA;
+    sd.fork_gate = e[0];
+    sd.fork_dispatch = e[1];
+    sd.join = e[2];
+    sd.s = s;
+  }
+  *out = &sd;
+  return MOE_OK;
+}
+
+// work queued on `to` after this waits for everything queued on `from` so far
+int stream_after(cudaStream_t to, cudaStream_t from, cudaEvent_t ev) {
+  if (cudaEventRecord(ev, from) != cudaSuccess) return MOE_ECUDA;
+  if (cudaStreamWaitEvent(to, ev, 0) != cudaSuccess) return MOE_ECUDA;
+  return MOE_OK;
+}
+
 // ---------------------------------------------------------------- stage drivers
+// side: when given, the flat gate's Load (and Switch P) reductions go there
 int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gate_params &gp,
              int *idx, float *gate, float *load, float *prob_sum, void *ws, int *status,
-             cudaStream_t st) {
+             cudaStream_t st, const Side *side = nullptr) {
   if (c.T == 0) {
     if (cudaMemsetAsync(load, 0, 4 * (size_t)c.n, st) != cudaSuccess) return MOE_ECUDA;
     if (prob_sum && cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess)
@@ -294,12 +347,17 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
     const bool sw = c.router == MOE_ROUTER_SWITCH;
     r.psum_part = sw ? at<float>(ws, L.psum_part) : nullptr;
     MOE_TRY(launch_route(r, L.tiles1, st));
-    MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, c.n, load, st));
+    cudaStream_t rs = st;
+    if (side) {
+      MOE_TRY(stream_after(side->s, st, side->fork_gate));
+      rs = side->s;
+    }
+    MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, c.n, load, rs));
     if (sw) {
       float *ps = prob_sum ? prob_sum : at<float>(ws, L.prob_sum);
-      MOE_TRY(launch_route_reduce(r.psum_part, nullptr, 1, L.tiles1, c.n, ps, st));
+      MOE_TRY(launch_route_reduce(r.psum_part, nullptr, 1, L.tiles1, c.n, ps, rs));
     } else if (prob_sum) {
-      if (cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess) return MOE_ECUDA;
+      if (cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, rs) != cudaSuccess) return MOE_ECUDA;
     }
     return MOE_OK;
   }
@@ -324,6 +382,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   da.C = INT64_MAX;
   da.hist = at<int>(ws, L.g_hist);
   da.base = at<int>(ws, L.g_base);
+  da.ticket = at<int>(ws, L.ticket);
   da.counts = at<int>(ws, L.g_counts);
   da.offsets = at<int>(ws, L.g_offsets);
   da.ucoff = at<int>(ws, L.g_ucoff);
@@ -380,10 +439,17 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   return MOE_OK;
 }
 
+// x / x_perm: when x is given its rows are copied into their expert rows
 int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const float *gate,
-                 int64_t C, int *counts, int *offsets, int *perm_token, int *row_of, void *ws,
-                 int *status, cudaStream_t st, bool plan_experts = false) {
+                 int64_t C, int *counts, int *offsets, int *perm_token, int *row_of,
+                 const float *x, void *x_perm, void *ws, int *status, cudaStream_t st,
+                 bool plan_experts = false) {
   DispatchArgs da{};
+  da.ticket = at<int>(ws, L.ticket);
+  da.x = x;
+  da.x_perm = x_perm;
+  da.d = c.d;
+  da.x_bf16 = c.expert_dtype == MOE_BF16;
   da.idx = idx;
   da.T = c.T;
   da.k = c.k;
@@ -436,9 +502,11 @@ int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const 
 }
 
 bool gate_params_ok(const moe_config &c, const moe_gate_params *gp) {
+  // the gate GEMM copies weight rows in 16-byte pieces
   if (!gp || !gp->W_g || !aligned(gp->W_g, 16)) return false;
-  if (c.noise && !gp->W_noise) return false;
-  if (c.hier_a > 0 && (!gp->W_g2 || (c.noise && !gp->W_noise2))) return false;
+  if (c.noise && (!gp->W_noise || !aligned(gp->W_noise, 16))) return false;
+  if (c.hier_a > 0 && (!gp->W_g2 || !aligned(gp->W_g2, 16))) return false;
+  if (c.hier_a > 0 && c.noise && (!gp->W_noise2 || !aligned(gp->W_noise2, 16))) return false;
   return true;
 }
 
@@ -528,11 +596,8 @@ int moe_dispatch(const moe_config *cfg, const float *x, const int32_t *topk_idx,
   if (c.T > 0 && (x == nullptr) != (x_perm == nullptr)) return MOE_EINVAL;
   if (c.T > 0 && x && (!aligned(x, 16) || !aligned(x_perm, 16))) return MOE_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  MOE_TRY(run_dispatch(c, L, topk_idx, nullptr, capacity_of(c), counts, offsets, perm_token, row_of,
-                       ws, status, st));
-  if (x && c.T > 0)
-    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, c.expert_dtype == MOE_BF16, x_perm, st));
-  return MOE_OK;
+  return run_dispatch(c, L, topk_idx, nullptr, capacity_of(c), counts, offsets, perm_token,
+                      row_of, x, x_perm, ws, status, st);
 }
 
 int moe_expert_ffn(const moe_config *cfg, const void *x_perm, const int32_t *offsets,
@@ -578,8 +643,8 @@ int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx, const flo
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   // gates sorted by expert (stable), from a capacity-free dispatch into scratch
   MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, INT64_MAX, at<int>(ws, L.counts_scratch),
-                       at<int>(ws, L.offsets), at<int>(ws, L.perm_token), at<int>(ws, L.row_of), ws,
-                       status, st));
+                       at<int>(ws, L.offsets), at<int>(ws, L.perm_token), at<int>(ws, L.row_of),
+                       nullptr, nullptr, ws, status, st));
   MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
                             st));
   return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, capacity_of(c), c.router,
@@ -606,20 +671,25 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   void *x_perm = at<void>(ws, L.x_perm);
   void *y_perm = at<void>(ws, L.y_perm);
 
-  MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st));
+  Side *side = nullptr;
+  MOE_TRY(side_stream(&side));
+  MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st, side));
   const bool tc = c.expert_dtype == MOE_BF16;
   MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, C, counts, offsets, at<int>(ws, L.perm_token),
-                       row_of, ws, status, st, tc));
+                       row_of, x, x_perm, ws, status, st, tc));
+  // balance statistics beside the expert chain; they read only the gate's and
+  // the dispatch's outputs
+  MOE_TRY(stream_after(side->s, st, side->fork_dispatch));
+  MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
+                            side->s));
+  MOE_TRY(launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, C, c.router,
+                        c.w_importance, c.w_load, c.alpha_aux, losses, side->s));
   if (c.T > 0) {
-    MOE_TRY(launch_gather(x, row_of, c.T, c.k, c.d, tc, x_perm, st));
     MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));
     MOE_TRY(launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
                            c.overflow_passthrough, c.T, c.k, c.d, y, st));
   }
-  MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
-                            st));
-  return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, C, c.router,
-                       c.w_importance, c.w_load, c.alpha_aux, losses, st);
+  return stream_after(st, side->s, side->join);
 }
 
 int moe_trace_enable(int on) {
