@@ -99,6 +99,40 @@ __device__ __forceinline__ long long block_exclusive_scan(long long v) {
   return res;
 }
 
+// Four block-wide exclusive scans at once (one set of barriers): v[i] is
+// replaced by the sum of v[i] over all threads with a lower index.
+__device__ __forceinline__ void block_exclusive_scan4(long long (&v)[4]) {
+  __shared__ long long warp_tot[4][32];
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int nwarps = (int)(blockDim.x >> 5);
+  long long inc[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    inc[i] = v[i];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long o = __shfl_up_sync(0xffffffffu, inc[i], off);
+      if (lane >= off) inc[i] += o;
+    }
+    if (lane == 31) warp_tot[i][w] = inc[i];
+  }
+  __syncthreads();
+  if (w < 4) {  // warp i scans the warp totals of value i
+    const long long t = lane < nwarps ? warp_tot[w][lane] : 0;
+    long long ti = t;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const long long o = __shfl_up_sync(0xffffffffu, ti, off);
+      if (lane >= off) ti += o;
+    }
+    warp_tot[w][lane] = ti - t;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i) v[i] = warp_tot[i][w] + inc[i] - v[i];
+  __syncthreads();  // warp_tot is reused by the next call
+}
+
 constexpr int SCAN_NT = 1024, SCAN_PER = 8;  // n <= 8192
 
 // One expert's tiles of a grouped GEMM: N-block major, M-block minor.
@@ -143,10 +177,9 @@ __device__ void write_plan(const int *counts, int n, const PlanOut &o) {
     values(e0 + j, raw, kept, mb, tl);
     sk += kept; sr += raw; sm += mb; st += tl;
   }
-  long long p = block_exclusive_scan(sk);
-  long long q = block_exclusive_scan(sr);
-  long long pm = block_exclusive_scan(sm);
-  long long pt = block_exclusive_scan(st);
+  long long sc[4] = {sk, sr, sm, st};
+  block_exclusive_scan4(sc);
+  long long p = sc[0], q = sc[1], pm = sc[2], pt = sc[3];
   for (int j = 0; j < per; ++j) {
     const int e = e0 + j;
     long long raw, kept, mb, tl;
@@ -225,6 +258,14 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
+  // the token's first x chunk is requested before the rank lookups below
+  const float4 *xr = COPY ? reinterpret_cast<const float4 *>(x + (size_t)t * d) : nullptr;
+  const int nchunk = d >> 3;  // 8 elements per chunk
+  float4 u0 = make_float4(0.f, 0.f, 0.f, 0.f), v0 = u0;
+  if (COPY && lane < nchunk) {
+    u0 = __ldg(xr + 2 * lane);
+    v0 = __ldg(xr + 2 * lane + 1);
+  }
   int myrow = -1;
   if (lane < k) {
     const int64_t p = (int64_t)t * k + lane;
@@ -248,10 +289,9 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
       const int v = __shfl_sync(0xffffffffu, myrow, j);
       rows[j] = j < k ? v : -1;
     }
-    const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)t * d);
-    const int nchunk = d >> 3;  // 8 elements per chunk
     for (int c = lane; c < nchunk; c += 32) {
-      const float4 u = __ldg(xr + 2 * c), v = __ldg(xr + 2 * c + 1);
+      const float4 u = c == lane ? u0 : __ldg(xr + 2 * c);
+      const float4 v = c == lane ? v0 : __ldg(xr + 2 * c + 1);
       if (BF16) {
         __nv_bfloat162 p0 = __floats2bfloat162_rn(u.x, u.y), p1 = __floats2bfloat162_rn(u.z, u.w);
         __nv_bfloat162 p2 = __floats2bfloat162_rn(v.x, v.y), p3 = __floats2bfloat162_rn(v.z, v.w);
