@@ -16,8 +16,10 @@
 //   warps 2-9  epilogue: two warps per 32-lane quarter of tensor memory, one
 //           per 128-column half; tcgen05.ld of the fp32 accumulator 64
 //           columns at a time, bias (prefetched into registers before the
-//           wait, broadcast by shuffles), ReLU, bf16, masked stores of the
-//           expert's valid rows
+//           wait, broadcast by shuffles), ReLU, bf16; the warp's 32 x 64 block
+//           goes through its own 4 KiB of shared memory (XOR-swizzled 16-byte
+//           chunks) so that every store instruction writes four whole 128-byte
+//           row segments, masked to the expert's valid rows
 // Two accumulators of 256 columns (all 512 TMEM columns) let the epilogue of
 // one tile overlap the main loop of the next.  Tiles are ordered expert by
 // expert, N-block by N-block, M-block fastest, so the M-blocks that share a
@@ -42,7 +44,9 @@ constexpr int NUM_EPI = 256;                 // epilogue threads (warps 2-9)
 constexpr int NUM_THREADS = 64 + NUM_EPI;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int BAR_BYTES = 256;
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+constexpr int EPI_STAGE_BYTES = 32 * 128;    // per epilogue warp: 32 rows x 64 bf16
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES + (NUM_EPI / 32) * EPI_STAGE_BYTES;
+static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 // instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
@@ -78,6 +82,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   auto tempty = [&](int c) { return bar0 + 8u * (2 * STAGES + 2 + c); };
   const uint32_t drain = bar0 + 8u * (2 * STAGES + 4);
   const uint32_t sbase = smem_u32(smem);
+  // epilogue warps' output staging, 4 KiB each, after the barriers
+  uint8_t *const stage_epi_all = smem + STAGES * STAGE_BYTES + BAR_BYTES;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -169,6 +175,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     // ------------------------------------------------ epilogue
     const int q = warp & 3;                 // TMEM lanes 32q .. 32q+31 belong to this warp
     const int half = (warp - 2) >> 2;       // columns [128*half, 128*half + 128) of the tile
+    uint8_t *const stage_epi = stage_epi_all + (warp - 2) * EPI_STAGE_BYTES;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
@@ -182,9 +189,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const int col = nbk * BN + half * 128 + u * 32 + lane;
         breg[u] = (a.bias && col < a.N) ? __ldg(a.bias + (size_t)e * a.N + col) : 0.f;
       }
-      const int r_in = q * 32 + lane;
-      const bool row_ok = r_in < ti.z;
-      __nv_bfloat16 *drow = a.D + (size_t)(ti.y + r_in) * a.N;
+      // this warp's rows are q*32 .. q*32+31 of the tile; the row of lane l is
+      // staged, the stores go out four rows at a time (rows rr, columns cc*8)
+      __nv_bfloat16 *const dtile = a.D + (size_t)(ti.y + q * 32) * a.N;
+      const int rows_here = ti.z - q * 32;  // valid rows of this warp (may be <= 0)
+      const int rr = lane >> 3, cc = lane & 7;
       // every lane waits; the outcome is made warp-uniform so that the
       // .sync.aligned tensor-memory loads below always see the full warp
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
@@ -212,17 +221,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
           pk[j] = *reinterpret_cast<uint32_t *>(&h);
         }
-        if (row_ok && col0 < a.N) {
-          if (col0 + 64 <= a.N) {
-            uint4 *dst = reinterpret_cast<uint4 *>(drow + col0);
+        if (col0 < a.N && rows_here > 0) {
+          // lane l's row, chunk u (8 columns) at chunk slot u ^ (l & 7)
+          uint8_t *row_st = stage_epi + lane * 128;
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          } else {
-            for (int j = 0; j < 64 && col0 + j < a.N; ++j)
-              reinterpret_cast<uint16_t *>(drow)[col0 + j] =
-                  (uint16_t)((pk[j >> 1] >> (16 * (j & 1))) & 0xFFFFu);
+          for (int u = 0; u < 8; ++u)
+            *reinterpret_cast<uint4 *>(row_st + ((u ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const int r = i * 4 + rr;  // row inside the warp's block
+            const uint4 v4 = *reinterpret_cast<const uint4 *>(stage_epi + r * 128 + ((cc ^ (r & 7)) << 4));
+            if (r < rows_here && col0 + cc * 8 < a.N)
+              *reinterpret_cast<uint4 *>(dtile + (size_t)r * a.N + col0 + cc * 8) = v4;
           }
+          __syncwarp();  // the block is reused by the next chunk
         }
       }
       tc_fence_before();
