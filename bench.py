@@ -133,7 +133,7 @@ def src_sha(name: str) -> str:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-KERNEL_SRC = {"expert_gemm1_tcgen05": "expert_tc.cu", "expert_gemm2_tcgen05": "expert_tc.cu",
+KERNEL_SRC = {"expert_ffn_tcgen05": "expert_tc.cu",
               "gate_gemm_fp32": "gate_gemm.cu", "route_topk": "route.cu", "combine": "combine.cu",
               "dispatch_place": "dispatch.cu", "dispatch_hist": "dispatch.cu"}
 
@@ -158,10 +158,11 @@ def kernel_work(w, name: str, S_kept: int):
     S = T * k
     ng = w.hier_a if w.hier_a else n
     esz = 2 if w.expert_bf16 else 4
-    if name == "expert_gemm1_tcgen05":
-        return "tensor", 2.0 * S_kept * d * f, n * f * d * esz + S_kept * d * esz + S_kept * f * esz
-    if name == "expert_gemm2_tcgen05":
-        return "tensor", 2.0 * S_kept * d * f, n * d * f * esz + S_kept * f * esz + S_kept * d * esz
+    if name == "expert_ffn_tcgen05":
+        # both layers in one persistent launch: every weight once, x_perm in,
+        # hid out and back in, y_perm out
+        return "tensor", 4.0 * S_kept * d * f, \
+            n * 2 * d * f * esz + S_kept * d * esz + 2 * S_kept * f * esz + S_kept * d * esz
     if name == "gate_gemm_fp32":
         return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
     if name == "gate_gemm_tf32x3":
@@ -351,7 +352,7 @@ def run_ours(args, w, world, rank, local):
     roof["traffic"] = ncu_traffic(dom, w.name)
 
     ffn_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in per_kernel
-                 if k.startswith("expert_gemm"))
+                 if k.startswith("expert_ffn_tcgen05"))
     ffn_flops = 4.0 * S_kept * w.d * w.f
     route_names = [k for k in main_chain if k.startswith(("route", "dispatch", "combine"))]
     route_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in route_names)

@@ -135,13 +135,15 @@ __device__ __forceinline__ void block_exclusive_scan4(long long (&v)[4]) {
 
 constexpr int SCAN_NT = 1024, SCAN_PER = 8;  // n <= 8192
 
-// One expert's tiles of a grouped GEMM: N-block major, M-block minor.
+// One expert's tiles of a grouped GEMM: N-block major, M-block minor; the
+// last field packs the N-block (8 bits) and the global M-block index.
 __device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_base, int mbe,
                                             int row_base, int rows) {
   for (int nbk = 0; nbk < nblk; ++nbk)
     for (int mb = 0; mb < mbe; ++mb)
       tab[(size_t)(mb_base * nblk + nbk * mbe + mb)] =
-          make_int4(e, row_base + mb * kExpertBM, min(kExpertBM, rows - mb * kExpertBM), nbk);
+          make_int4(e, row_base + mb * kExpertBM, min(kExpertBM, rows - mb * kExpertBM),
+                    nbk | ((mb_base + mb) << 8));
 }
 
 struct PlanOut {
@@ -150,6 +152,7 @@ struct PlanOut {
   int mblk_rows, tile_rows;
   int4 *tab1, *tab2;
   int nblk1, nblk2;
+  int *mdone;  // with the tables: per-M-block counters of the expert GEMM, zeroed
 };
 
 // offsets[e] = sum_{e'<e} min(count, C); ucoff: the same without the cap;
@@ -161,6 +164,7 @@ __device__ void write_plan(const int *counts, int n, const PlanOut &o) {
   const int mblk_rows = o.mblk_rows, tile_rows = o.tile_rows;
   int4 *tab1 = o.tab1, *tab2 = o.tab2;
   const int nblk1 = o.nblk1, nblk2 = o.nblk2;
+  int *mdone = o.mdone;
   // each thread takes a contiguous run of per <= SCAN_PER experts, so that
   // small n still spreads over the whole block
   const int per = (n + SCAN_NT - 1) / SCAN_NT;
@@ -192,6 +196,8 @@ __device__ void write_plan(const int *counts, int n, const PlanOut &o) {
       if (tab1) {  // expert GEMM tile tables
         write_tiles(tab1, nblk1, e, (int)pm, (int)mb, (int)p, (int)kept);
         write_tiles(tab2, nblk2, e, (int)pm, (int)mb, (int)p, (int)kept);
+        for (long long j = 0; j < mb; ++j) mdone[pm + j] = 0;
+        if (e == n - 1) mdone[pm + mb] = 0;  // the count over all M-blocks
       }
     }
     p += kept;
@@ -221,18 +227,32 @@ __global__ void __launch_bounds__(SCAN_NT) dispatch_scan_kernel(const int *hist,
   const int e = blockIdx.x * 32 + tx;
   const int chunk = (B + SC - 1) / SC;
   const int b0 = min(B, r * chunk), b1 = min(B, b0 + chunk);
+  // the range is read in batches of 8 independent loads (the sums are exact
+  // integer sums, so batching changes nothing)
+  constexpr int VB = 8;
   int s = 0;
   if (e < n)
-    for (int b = b0; b < b1; ++b) s += hist[(size_t)b * n + e];
+    for (int b = b0; b < b1; b += VB) {
+      int h[VB];
+#pragma unroll
+      for (int j = 0; j < VB; ++j) h[j] = b + j < b1 ? hist[(size_t)(b + j) * n + e] : 0;
+#pragma unroll
+      for (int j = 0; j < VB; ++j) s += h[j];
+    }
   tot[r][tx] = s;
   __syncthreads();
   int run = 0;
   for (int q = 0; q < r; ++q) run += tot[q][tx];
   if (e < n) {
-    for (int b = b0; b < b1; ++b) {
-      const int h = hist[(size_t)b * n + e];
-      base[(size_t)b * n + e] = run;
-      run += h;
+    for (int b = b0; b < b1; b += VB) {
+      int h[VB];
+#pragma unroll
+      for (int j = 0; j < VB; ++j) h[j] = b + j < b1 ? hist[(size_t)(b + j) * n + e] : 0;
+#pragma unroll
+      for (int j = 0; j < VB; ++j) {
+        if (b + j < b1) base[(size_t)(b + j) * n + e] = run;
+        run += h[j];
+      }
     }
     if (r == SC - 1) counts[e] = run;
   }
@@ -319,7 +339,7 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
 
 __global__ void __launch_bounds__(SCAN_NT) expert_plan_kernel(const int *offsets, int n,
                                                               int *mprefix, int4 *tab1, int nblk1,
-                                                              int4 *tab2, int nblk2) {
+                                                              int4 *tab2, int nblk2, int *mdone) {
   const int per = (n + SCAN_NT - 1) / SCAN_NT;
   const int e0 = threadIdx.x * per;
   auto rows = [&](int e) -> long long { return e < n ? (long long)(offsets[e + 1] - offsets[e]) : 0; };
@@ -333,6 +353,8 @@ __global__ void __launch_bounds__(SCAN_NT) expert_plan_kernel(const int *offsets
       mprefix[e] = (int)p;
       write_tiles(tab1, nblk1, e, (int)p, (int)mb, offsets[e], (int)m);
       write_tiles(tab2, nblk2, e, (int)p, (int)mb, offsets[e], (int)m);
+      for (long long j = 0; j < mb; ++j) mdone[p + j] = 0;
+      if (e == n - 1) mdone[p + mb] = 0;  // the count over all M-blocks
     }
     p += mb;
     if (e == n - 1) mprefix[n] = (int)p;
@@ -373,6 +395,7 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
   o.tab2 = a.tab2;
   o.nblk1 = a.nblk1;
   o.nblk2 = a.nblk2;
+  o.mdone = a.mdone;
   MOE_TRY(launch("dispatch_scan", dispatch_scan_kernel, dim3((unsigned)ceil_div(a.n, 32)),
                  dim3(SCAN_NT), 0, st, (const int *)a.hist, B, a.n, a.base, a.counts, a.ticket, o));
   if (B == 0) return MOE_OK;
@@ -389,10 +412,10 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
 }
 
 int launch_expert_plan(const int *offsets, int n, int *mprefix, int4 *tab1, int nblk1, int4 *tab2,
-                       int nblk2, cudaStream_t st) {
+                       int nblk2, int *mdone, cudaStream_t st) {
   if (n > SCAN_NT * SCAN_PER) return MOE_EINVAL;
   return launch("expert_plan", expert_plan_kernel, dim3(1), dim3(SCAN_NT), 0, st, offsets, n,
-                mprefix, tab1, nblk1, tab2, nblk2);
+                mprefix, tab1, nblk1, tab2, nblk2, mdone);
 }
 
 }  // namespace moe

@@ -8,7 +8,14 @@
 //   GEMM2: y_perm = hid_e W2_e^T + b2_e            (bf16 out)
 // Both are "grouped" GEMMs with a ragged M per expert and K-major operands.
 //
-// One persistent kernel, one CTA per SM, 320 threads:
+// One persistent kernel runs both, one CTA per SM, 320 threads.  Every CTA
+// takes its share of GEMM1's tiles and then of GEMM2's, so GEMM2 starts on
+// the SMs that finish GEMM1 first; a GEMM2 tile of M-block m waits (bounded)
+// until the epilogues of all GEMM1 tiles of m have published their rows of
+// hid (a counter per M-block, and one for all of GEMM1: once a CTA has seen
+// all of GEMM1 published, its later GEMM2 tiles need no check).  The launch
+// is cooperative, so every CTA is resident and no wait can depend on a CTA
+// that has not started.
 //   warp 0  TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte
 //           swizzle), 4 stages, mbarrier transaction counts
 //   warp 1  MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128,
@@ -26,10 +33,10 @@
 // weight tile run at the same time and the weights stream from HBM once.
 // No cluster multicast anywhere.
 //
-// Every mbarrier wait is bounded (about two seconds of %globaltimer); a wait
-// that runs out sets MOE_STATUS_TIMEOUT, raises an abort flag seen by the
-// other roles, drains the copies and MMAs this CTA issued (again bounded),
-// frees its tensor memory and returns.
+// Every wait is bounded (about two seconds of %globaltimer); a wait that runs
+// out sets MOE_STATUS_TIMEOUT, raises an abort flag seen by the other roles,
+// drains the copies and MMAs this CTA issued (again bounded), frees its
+// tensor memory and returns.
 #include "tc_common.cuh"
 
 namespace moe {
@@ -41,11 +48,12 @@ constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
 constexpr int NUM_EPI = 256;                 // epilogue threads (warps 2-9)
+constexpr int NUM_EPI_WARPS = NUM_EPI / 32;
 constexpr int NUM_THREADS = 64 + NUM_EPI;
 constexpr uint32_t TMEM_COLS = 2 * BN;
 constexpr int BAR_BYTES = 256;
 constexpr int EPI_STAGE_BYTES = 32 * 128;    // per epilogue warp: 32 rows x 64 bf16
-constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES + (NUM_EPI / 32) * EPI_STAGE_BYTES;
+constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES + NUM_EPI_WARPS * EPI_STAGE_BYTES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
@@ -55,19 +63,48 @@ constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
 
-struct TcArgs {
-  const int4 *tiles;     // per tile: {expert, first row, valid rows, N-block}
-  const int *mprefix;    // [n+1]; mprefix[n] * nblk tiles in total
-  int n, N, K, nblk;
+struct GemmArgs {
+  const int4 *tiles;     // per tile: {expert, first row, valid rows, N-block | M-block << 8}
+  int N, K, nblk;
   const float *bias;     // [n][N] or nullptr
   __nv_bfloat16 *D;      // [S][N]
   int relu;
+};
+
+struct FfnArgs {
+  GemmArgs g[2];         // GEMM1, GEMM2
+  const int *mprefix;    // [n+1]; mprefix[n] M-blocks
+  int n;
+  int *mdone;            // [M-blocks + 1] GEMM1 epilogue warps finished, per M-block; the
+                         // last entry counts them over all of GEMM1
   int *status;
 };
 
+__device__ __forceinline__ int ld_acquire(const int *p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+// bounded wait until *p >= target (acquire at GPU scope)
+__device__ __noinline__ bool wait_count(const int *p, int target, volatile int *abort_flag,
+                                        unsigned long long limit_ns) {
+  if (ld_acquire(p) >= target) return true;
+  const unsigned long long t0 = globaltimer();
+  for (uint32_t it = 1;; ++it) {
+    __nanosleep(64);
+    if (ld_acquire(p) >= target) return true;
+    if ((it & 15u) == 0u) {
+      if (*abort_flag) return false;
+      if (globaltimer() - t0 > limit_ns) return false;
+    }
+  }
+}
+
 __global__ void __launch_bounds__(NUM_THREADS, 1)
-    expert_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                       const __grid_constant__ CUtensorMap tmB, TcArgs a) {
+    expert_ffn_kernel(const __grid_constant__ CUtensorMap tmA1,
+                      const __grid_constant__ CUtensorMap tmB1,
+                      const __grid_constant__ CUtensorMap tmA2,
+                      const __grid_constant__ CUtensorMap tmB2, FfnArgs a) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -105,8 +142,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int total = __ldg(a.mprefix + a.n) * a.nblk;
-  const int nkb = (a.K + BK - 1) / BK;
+  const int mtotal = __ldg(a.mprefix + a.n);
+  const int T1 = mtotal * a.g[0].nblk, total = T1 + mtotal * a.g[1].nblk;
+  const int ready = NUM_EPI_WARPS * a.g[0].nblk;  // arrivals that complete an M-block of hid
   bool failed = false;
 
   if (warp == 0 && lane == 0) {
@@ -115,23 +153,40 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0;
     int issued[STAGES];
     for (int s = 0; s < STAGES; ++s) issued[s] = -1;
-    int4 cur = blockIdx.x < total ? __ldg(a.tiles + blockIdx.x) : make_int4(0, 0, 0, 0);
+    bool g1_all = false;  // all of GEMM1's hid seen published (acquire + proxy fence done)
+    auto entry = [&](int t) {
+      return t < total ? __ldg(a.g[t >= T1].tiles + (t >= T1 ? t - T1 : t)) : make_int4(0, 0, 0, 0);
+    };
+    int4 ti = entry(blockIdx.x);
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      // the next tile's entry is fetched while this tile's loads go out
-      const int nxt = tile + gridDim.x;
-      const int4 next = nxt < total ? __ldg(a.tiles + nxt) : cur;
-      const int row0 = cur.y;
-      const int brow = cur.x * a.N + cur.w * BN;
-      cur = next;
+      const int which = tile >= T1;
+      const GemmArgs &g = a.g[which];
+      const int4 next = entry(tile + gridDim.x);  // fetched while this tile's loads go out
+      if (which && !g1_all) {
+        // hid rows of this M-block: every GEMM1 epilogue warp of it has
+        // published them; then order the TMA reads after that observation
+        if (ld_acquire(a.mdone + mtotal) >= NUM_EPI_WARPS * T1) {
+          g1_all = true;
+        } else if (!wait_count(a.mdone + (ti.w >> 8), ready, abort_flag, kWaitNs)) {
+          failed = true;
+          break;
+        }
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+      }
+      const CUtensorMap *mA = which ? &tmA2 : &tmA1;
+      const CUtensorMap *mB = which ? &tmB2 : &tmB1;
+      const int nkb = (g.K + BK - 1) / BK;
+      const int brow = ti.x * g.N + (ti.w & 0xFF) * BN;
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
         const uint32_t sa = sbase + stage * STAGE_BYTES;
         mbar_expect_tx(full(stage), STAGE_BYTES);
-        tma_load_2d(sa, &tmA, full(stage), kb * BK, row0);
-        tma_load_2d(sa + A_BYTES, &tmB, full(stage), kb * BK, brow);
+        tma_load_2d(sa, mA, full(stage), kb * BK, ti.y);
+        tma_load_2d(sa + A_BYTES, mB, full(stage), kb * BK, brow);
         issued[stage] = (int)phase;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
+      ti = next;
     }
     if (failed || *abort_flag) {
       *abort_flag = 1;
@@ -145,6 +200,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0, acc_phase = 0;
     bool issued_any = false;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
+      const int nkb = (a.g[tile >= T1].K + BK - 1) / BK;
       if (!mbar_wait(tempty(acc), acc_phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -176,24 +232,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int q = warp & 3;                 // TMEM lanes 32q .. 32q+31 belong to this warp
     const int half = (warp - 2) >> 2;       // columns [128*half, 128*half + 128) of the tile
     uint8_t *const stage_epi = stage_epi_all + (warp - 2) * EPI_STAGE_BYTES;
+    const int rr = lane >> 3, cc = lane & 7;
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      const int4 ti = __ldg(a.tiles + tile);
-      const int e = ti.x, nbk = ti.w;
+      const int which = tile >= T1;
+      const GemmArgs &g = a.g[which];
+      const int4 ti = __ldg(g.tiles + (which ? tile - T1 : tile));
+      const int e = ti.x, nbk = ti.w & 0xFF;
       // bias of this warp's 128 columns, lane l holding columns l, l+32, ...;
       // loaded before the wait so the latency hides behind the main loop
       float breg[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int col = nbk * BN + half * 128 + u * 32 + lane;
-        breg[u] = (a.bias && col < a.N) ? __ldg(a.bias + (size_t)e * a.N + col) : 0.f;
+        breg[u] = (g.bias && col < g.N) ? __ldg(g.bias + (size_t)e * g.N + col) : 0.f;
       }
       // this warp's rows are q*32 .. q*32+31 of the tile; the row of lane l is
       // staged, the stores go out four rows at a time (rows rr, columns cc*8)
-      __nv_bfloat16 *const dtile = a.D + (size_t)(ti.y + q * 32) * a.N;
+      __nv_bfloat16 *const dtile = g.D + (size_t)(ti.y + q * 32) * g.N;
       const int rows_here = ti.z - q * 32;  // valid rows of this warp (may be <= 0)
-      const int rr = lane >> 3, cc = lane & 7;
       // every lane waits; the outcome is made warp-uniform so that the
       // .sync.aligned tensor-memory loads below always see the full warp
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
@@ -205,8 +263,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t v[64];
         tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cl), v);
         const int col0 = nbk * BN + cl;
-        // conversion by the whole warp (the shuffles need every lane), stores
-        // only for valid rows and columns
+        // conversion by the whole warp (the shuffles need every lane)
         uint32_t pk[32];
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
@@ -214,14 +271,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const float b1 = __shfl_sync(0xffffffffu, breg[2 * c + (j >> 4)], (2 * j + 1) & 31);
           float x0 = __uint_as_float(v[2 * j]) + b0;
           float x1 = __uint_as_float(v[2 * j + 1]) + b1;
-          if (a.relu) {
+          if (g.relu) {
             x0 = fmaxf(x0, 0.f);
             x1 = fmaxf(x1, 0.f);
           }
           __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
           pk[j] = *reinterpret_cast<uint32_t *>(&h);
         }
-        if (col0 < a.N && rows_here > 0) {
+        if (col0 < g.N && rows_here > 0) {
           // lane l's row, chunk u (8 columns) at chunk slot u ^ (l & 7)
           uint8_t *row_st = stage_epi + lane * 128;
 #pragma unroll
@@ -233,8 +290,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 8; ++i) {
             const int r = i * 4 + rr;  // row inside the warp's block
             const uint4 v4 = *reinterpret_cast<const uint4 *>(stage_epi + r * 128 + ((cc ^ (r & 7)) << 4));
-            if (r < rows_here && col0 + cc * 8 < a.N)
-              *reinterpret_cast<uint4 *>(dtile + (size_t)r * a.N + col0 + cc * 8) = v4;
+            if (r < rows_here && col0 + cc * 8 < g.N)
+              *reinterpret_cast<uint4 *>(dtile + (size_t)r * g.N + col0 + cc * 8) = v4;
           }
           __syncwarp();  // the block is reused by the next chunk
         }
@@ -242,6 +299,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       tc_fence_before();
       mbar_arrive(tempty(acc));
       if (++acc == 2) { acc = 0; acc_phase ^= 1u; }
+      if (!which) {
+        // publish this warp's rows of hid to the GEMM2 tiles of the M-block:
+        // the stores before the release, visible to the async proxy (TMA)
+        asm volatile("fence.proxy.async.global;" ::: "memory");
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) {
+          atomicAdd(a.mdone + (ti.w >> 8), 1);
+          atomicAdd(a.mdone + mtotal, 1);
+        }
+      }
     }
     if (failed) *abort_flag = 1;
   }
@@ -255,36 +323,20 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
-// ---------------------------------------------------------------- host side
-int run_gemm(const void *A, int S, int K, const void *B, int n, int N, const float *bias, void *D,
-             int relu, const int4 *tiles, const int *mprefix, int *status, cudaStream_t st,
-             const char *name) {
-  CUtensorMap ta, tb;
-  MOE_TRY(tc::make_map_2d(&ta, A, 2, (uint64_t)K, (uint64_t)S, BM));
-  MOE_TRY(tc::make_map_2d(&tb, B, 2, (uint64_t)K, (uint64_t)n * N, BN));
-  TcArgs a;
-  a.tiles = tiles;
-  a.mprefix = mprefix;
-  a.n = n;
-  a.N = N;
-  a.K = K;
-  a.nblk = (N + BN - 1) / BN;
-  a.bias = bias;
-  a.D = static_cast<__nv_bfloat16 *>(D);
-  a.relu = relu;
-  a.status = status;
-  const int64_t upper = (ceil_div(S, BM) + n) * (int64_t)a.nblk;
-  const int grid = (int)(upper < num_sms() ? upper : num_sms());
-  static int attr_dev = -1;
+int ffn_ctas() {
+  static int cached_dev = -1, cached = 0;
   int dev = 0;
   cudaGetDevice(&dev);
-  if (attr_dev != dev) {
-    if (cudaFuncSetAttribute(expert_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return MOE_ECUDA;
-    attr_dev = dev;
+  if (dev != cached_dev) {
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ffn_kernel, NUM_THREADS,
+                                                      SMEM_BYTES) != cudaSuccess ||
+        per_sm < 1)
+      return 0;
+    cached = per_sm * num_sms();
+    cached_dev = dev;
   }
-  return launch(name, expert_gemm_kernel, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st, ta, tb, a);
+  return cached;
 }
 
 }  // namespace
@@ -293,14 +345,54 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   if (a.S == 0) return MOE_OK;
   static_assert(BN == kExpertBN, "tile tables assume the GEMM's N-block width");
   const int nblk1 = (a.f + BN - 1) / BN, nblk2 = (a.d + BN - 1) / BN;
+  if (nblk1 > 256 || nblk2 > 256) return MOE_EINVAL;  // N-block fits the tile table's 8 bits
   if (!a.plan_ready)
     MOE_TRY(launch_expert_plan(a.offsets, a.n, const_cast<int *>(a.mprefix), a.tab1, nblk1, a.tab2,
-                               nblk2, st));
-  MOE_TRY(run_gemm(a.x_perm, a.S, a.d, a.W1, a.n, a.f, a.b1, a.hid, 1, a.tab1, a.mprefix, a.status,
-                   st, "expert_gemm1_tcgen05"));
-  MOE_TRY(run_gemm(a.hid, a.S, a.f, a.W2, a.n, a.d, a.b2, a.y_perm, 0, a.tab2, a.mprefix, a.status,
-                   st, "expert_gemm2_tcgen05"));
-  return MOE_OK;
+                               nblk2, a.mdone, st));
+  static int attr_dev = -1;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (attr_dev != dev) {
+    if (cudaFuncSetAttribute(expert_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess)
+      return MOE_ECUDA;
+    attr_dev = dev;
+  }
+  CUtensorMap a1, b1, a2, b2;
+  MOE_TRY(tc::make_map_2d(&a1, a.x_perm, 2, (uint64_t)a.d, (uint64_t)a.S, BM));
+  MOE_TRY(tc::make_map_2d(&b1, a.W1, 2, (uint64_t)a.d, (uint64_t)a.n * a.f, BN));
+  MOE_TRY(tc::make_map_2d(&a2, a.hid, 2, (uint64_t)a.f, (uint64_t)a.S, BM));
+  MOE_TRY(tc::make_map_2d(&b2, a.W2, 2, (uint64_t)a.f, (uint64_t)a.n * a.d, BN));
+  FfnArgs f;
+  f.g[0] = GemmArgs{a.tab1, a.f, a.d, nblk1, a.b1, static_cast<__nv_bfloat16 *>(a.hid), 1};
+  f.g[1] = GemmArgs{a.tab2, a.d, a.f, nblk2, a.b2, static_cast<__nv_bfloat16 *>(a.y_perm), 0};
+  f.mprefix = a.mprefix;
+  f.n = a.n;
+  f.mdone = a.mdone;
+  f.status = a.status;
+  const int64_t upper = (ceil_div(a.S, BM) + a.n) * (int64_t)(nblk1 + nblk2);
+  const int ctas = ffn_ctas();
+  if (ctas < 1) return MOE_ECUDA;
+  const int grid = (int)(upper < ctas ? upper : ctas);
+
+  // cooperative: all CTAs resident at once (a GEMM2 tile waits on other
+  // CTAs' GEMM1 tiles)
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(NUM_THREADS);
+  cfg.dynamicSmemBytes = SMEM_BYTES;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int slot = -1;
+  trace_begin("expert_ffn_tcgen05", st, &slot);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, expert_ffn_kernel, a1, b1, a2, b2, f);
+  trace_end(slot, st);
+  count_launch();
+  return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
 }
 
 }  // namespace moe

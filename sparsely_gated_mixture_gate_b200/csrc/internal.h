@@ -118,6 +118,7 @@ struct DispatchArgs {
   int tile_rows;
   int4 *tab1, *tab2;       // expert GEMM tile tables (see ExpertArgs), or nullptr
   int nblk1, nblk2;
+  int *mdone;              // with the tables: per-M-block counters, zeroed
   int *ticket;             // one int of scratch (last-block election of the scan)
   const float *x;          // [T][d] or nullptr: with it x rows are copied to x_perm
   void *x_perm;            // [kept rows][d], bf16 (x_bf16) or fp32
@@ -127,10 +128,12 @@ struct DispatchArgs {
 int launch_dispatch(const DispatchArgs &a, cudaStream_t st);
 // Expert GEMM plan from offsets: mprefix[n+1] = exclusive scan of
 // ceil(M_e / kExpertBM); tab1 / tab2: one int4 per tile of the two GEMMs
-// (nblk1 / nblk2 N-blocks): {expert, first row, valid rows, N-block}, tiles
-// of an expert N-block major, M-block minor.
+// (nblk1 / nblk2 N-blocks): {expert, first row, valid rows, N-block | global
+// M-block << 8}, tiles of an expert N-block major, M-block minor; mdone[m] = 0
+// for every M-block and mdone[mprefix[n]] = 0 (the expert kernel's GEMM1 ->
+// GEMM2 counters).
 int launch_expert_plan(const int *offsets, int n, int *mprefix, int4 *tab1, int nblk1, int4 *tab2,
-                       int nblk2, cudaStream_t st);
+                       int nblk2, int *mdone, cudaStream_t st);
 constexpr int kExpertBN = 256;
 
 struct ExpertArgs {
@@ -138,6 +141,7 @@ struct ExpertArgs {
   const int *offsets;      // [n+1]
   const int *mprefix;      // [n+1] exclusive scan of ceil(M_e / kExpertBM)
   int4 *tab1, *tab2;       // tile tables of GEMM1 / GEMM2
+  int *mdone;              // [M-blocks + 1] GEMM1 -> GEMM2 counters (zeroed by the plan)
   int plan_ready;          // 1: mprefix and the tables were written by the dispatch
   int n, d, f, S;
   const void *W1, *W2;

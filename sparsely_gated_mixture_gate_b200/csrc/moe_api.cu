@@ -128,7 +128,7 @@ struct Layout {
   size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch, ticket;
-  size_t mprefix, tab1, tab2, x_perm, hid, y_perm;
+  size_t mprefix, tab1, tab2, mdone, x_perm, hid, y_perm;
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
@@ -206,6 +206,7 @@ Layout make_layout(const moe_config &c) {
     const size_t mb_upper = (size_t)ceil_div((int64_t)S, kExpertBM) + n;
     L.tab1 = bp.take(16 * mb_upper * (size_t)ceil_div(c.f, kExpertBN));
     L.tab2 = bp.take(16 * mb_upper * (size_t)ceil_div(c.d, kExpertBN));
+    L.mdone = bp.take(4 * (mb_upper + 1));
   }
   L.x_perm = bp.take(esz * S * (size_t)c.d);
   L.hid = bp.take(esz * S * (size_t)c.f);
@@ -472,6 +473,7 @@ int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const flo
     da.tab2 = at<int4>(ws, L.tab2);
     da.nblk1 = (int)ceil_div(c.f, kExpertBN);
     da.nblk2 = (int)ceil_div(c.d, kExpertBN);
+    da.mdone = at<int>(ws, L.mdone);
   }
   da.status = status;
   return launch_dispatch(da, st);
@@ -486,6 +488,7 @@ int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const 
   e.mprefix = at<int>(ws, L.mprefix);
   e.tab1 = at<int4>(ws, L.tab1);
   e.tab2 = at<int4>(ws, L.tab2);
+  e.mdone = at<int>(ws, L.mdone);
   e.plan_ready = plan_ready;
   e.n = c.n;
   e.d = c.d;
