@@ -160,9 +160,9 @@ def kernel_work(w, name: str, S_kept: int):
     esz = 2 if w.expert_bf16 else 4
     if name == "expert_ffn_tcgen05":
         # both layers in one persistent launch: every weight once, x_perm in,
-        # hid out and back in, y_perm out
-        return "tensor", 4.0 * S_kept * d * f, \
-            n * 2 * d * f * esz + S_kept * d * esz + 2 * S_kept * f * esz + S_kept * d * esz
+        # y_perm out (the hidden layer's round trip through memory is this
+        # implementation's choice, not counted as algorithmic traffic)
+        return "tensor", 4.0 * S_kept * d * f, n * 2 * d * f * esz + 2 * S_kept * d * esz
     if name == "gate_gemm_fp32":
         return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
     if name == "gate_gemm_tf32x3":
