@@ -250,6 +250,38 @@ def test_expert_ffn_lm_size_sampled(orc):
         assert rel_fro(got[r], want) < 3e-2, (r, e)
 
 
+SKEWED = [
+    # one expert holds almost every row: its GEMM2 tiles land on CTAs that have
+    # no GEMM1 tiles and wait for the counters of M-blocks computed elsewhere
+    (256, 1024, [4000, 0, 3, 0]),
+    # GEMM2 with more N-blocks than GEMM1, ragged tails
+    (768, 256, [1, 2000, 0, 900, 5]),
+]
+
+
+@pytest.mark.parametrize("d,f,counts", SKEWED)
+def test_expert_ffn_skewed_sampled(orc, d, f, counts):
+    xp, W1, b1, W2, b2, offsets = _expert_case(d, f, counts, True, seed=5)
+    n, S = len(counts), sum(counts)
+    cfg = M.Config(T=S, d=d, n=n, k=1, f=f)
+    out = M.expert_ffn(cfg, xp.to(DEV), offsets.to(DEV),
+                       dict(W1=W1.to(DEV), b1=b1.to(DEV), W2=W2.to(DEV), b2=b2.to(DEV)))
+    torch.cuda.synchronize()
+    assert M.status_bits(out["status"]) == 0
+    got = out["y_perm"].float().cpu().numpy()
+    off = offsets.numpy()
+    rng = np.random.default_rng(1)
+    rows = set(rng.integers(0, S, 120).tolist())
+    for e in range(n):  # first and last row of every expert and of every 128-row block
+        for r0 in range(int(off[e]), int(off[e + 1]), 128):
+            rows |= {r0, min(r0 + 127, int(off[e + 1]) - 1)}
+    for r in sorted(rows):
+        e = int(np.searchsorted(off, r, side="right") - 1)
+        want = orc.expert_row(xp[r].float().numpy(), _bits(W1[e]), b1[e].numpy(), _bits(W2[e]),
+                              b2[e].numpy(), bf16=True)
+        assert rel_fro(got[r], want) < 3e-2, (r, e)
+
+
 # ------------------------------------------------------------------ whole layer
 def run_layer(w, inp):
     cfg = M.Config.from_workload(w)
