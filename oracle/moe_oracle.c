@@ -174,7 +174,7 @@ void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
                   uint32_t token, uint32_t gate_id, const float *x,
                   const float *Wg, const float *bg, const float *Wn,
                   double *c, double *s, float *H, int *order, double *gates,
-                  double *p)
+                  double *p, const float *sel_bias)
 {
   for (int i = 0; i < n; ++i) { c[i] = 0.0; s[i] = 0.0; }
   for (int j = 0; j < d; ++j) {
@@ -191,7 +191,9 @@ void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
       H[i] = (float)(c[i] + eps * s[i]);
     } else {
       s[i] = 0.0;
-      H[i] = (float)c[i];
+      /* router 2 ranks the routing score c + b ([MoE-deep] §6.3: the bias
+       * enters the selection only) */
+      H[i] = (float)(router == 2 && sel_bias ? c[i] + (double)sel_bias[i] : c[i]);
     }
   }
 
@@ -211,6 +213,15 @@ void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
       if (p) p[i] = pi;
       if (i == order[0]) gates[0] = pi;
     }
+    return;
+  }
+
+  if (router == 2) {
+    /* [MoE-deep] §6.2: s_i = Sigmoid(h_i) of the logits without the bias,
+     * g_i = s_i / sum of s_j over the kept k */
+    double den = 0.0;
+    for (int j = 0; j < k; ++j) den += 1.0 / (1.0 + exp(-c[order[j]]));
+    for (int j = 0; j < k; ++j) gates[j] = (1.0 / (1.0 + exp(-c[order[j]]))) / den;
     return;
   }
 
@@ -359,8 +370,9 @@ static float min_gap(const float *H, const int *order, int n, int k)
 static int valid_cfg(const orc_cfg *c)
 {
   if (c->T < 0 || c->d < 1 || c->f < 1 || c->n < 1 || c->k < 1 || c->k > c->n) return 0;
-  if (c->router != 0 && c->router != 1) return 0;
+  if (c->router != 0 && c->router != 1 && c->router != 2) return 0;
   if (c->router == 1 && (c->k != 1 || c->noise || c->hier_a)) return 0;
+  if (c->router == 2 && (c->noise || c->hier_a)) return 0;
   if (c->hier_a) {
     if (c->hier_b < 1 || c->hier_a * c->hier_b != c->n) return 0;
     if (c->hier_k1 < 1 || c->hier_k1 > c->hier_a) return 0;
@@ -425,7 +437,7 @@ int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tok
       const int tok = tokens ? tokens[t] : t;
       const float *xt = in->x + (size_t)tok * d;
       orc_gate_row(d, n, k, cfg->router, cfg->noise, cfg->seed, (uint32_t)tok, 0u,
-                   xt, in->Wg, in->bg, in->Wn, c, s, H, order, g1, pr);
+                   xt, in->Wg, in->bg, in->Wn, c, s, H, order, g1, pr, in->sel_bias);
       for (int j = 0; j < k; ++j) {
         topk_idx[(size_t)t * k + j] = order[j];
         topk_gate[(size_t)t * k + j] = g1[j];
@@ -445,7 +457,7 @@ int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tok
       const int tok = tokens ? tokens[t] : t;
       const float *xt = in->x + (size_t)tok * d;
       orc_gate_row(d, a, k1, 0, cfg->noise, cfg->seed, (uint32_t)tok, 0u, xt,
-                   in->Wg, in->bg, in->Wn, c, s, H, order, g1, NULL);
+                   in->Wg, in->bg, in->Wn, c, s, H, order, g1, NULL, NULL);
       float gap = min_gap(H, order, a, k1);
       orc_load_row(a, k1, cfg->noise, c, s, H, P);
       for (int i = 0; i < a; ++i) load_p[i] += P[i];
@@ -457,7 +469,7 @@ int orc_gate_tokens(const orc_cfg *cfg, const orc_inputs *in, const int32_t *tok
         const float *Wn2 = in->Wn2 ? in->Wn2 + (size_t)gi * d * b : NULL;
         const float *bg2 = in->bg2 ? in->bg2 + (size_t)gi * b : NULL;
         orc_gate_row(d, b, k2, 0, cfg->noise, cfg->seed, (uint32_t)tok, (uint32_t)(1 + gi),
-                     xt, Wg2, bg2, Wn2, c, s, H, order, g2, NULL);
+                     xt, Wg2, bg2, Wn2, c, s, H, order, g2, NULL, NULL);
         float gap2 = min_gap(H, order, b, k2);
         if (gap2 < gap) gap = gap2;
         orc_load_row(b, k2, cfg->noise, c, s, H, P);
@@ -552,8 +564,23 @@ void orc_balance(int n, int T, int k, const int32_t *topk_idx, const double *top
  * dispatch, each kept expert applied to the token directly, gate-weighted
  * sum, pass-through of fully dropped tokens, balancing statistics.  Losses
  * as in orc_balance. */
+/* [MoE-deep] §6.3: the bias of an overloaded expert goes down by gamma, that
+ * of an underloaded one up by gamma.  Our reading of over / under: more / fewer
+ * slots than the average T*k/n (compared exactly: counts*n against T*k); an
+ * expert exactly at the average keeps its bias. */
+void orc_sel_bias_update(int n, int T, int k, const int32_t *counts, float gamma, float *bias)
+{
+  const int64_t total = (int64_t)T * k;
+  for (int i = 0; i < n; ++i) {
+    const int64_t scaled = (int64_t)counts[i] * n;
+    if (scaled > total) bias[i] = bias[i] - gamma;
+    else if (scaled < total) bias[i] = bias[i] + gamma;
+  }
+}
+
 int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
 {
+  if (cfg->shared_expert && (!in->W1s || !in->W2s)) return -1;
   if (orc_gate_batch(cfg, in, out->topk_idx, out->topk_gate, out->load, out->prob_sum,
                      out->near_tie) != 0)
     return -1;
@@ -588,6 +615,15 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
     }
     if (kept_slots == 0 && k > 0 && cfg->passthrough)
       for (int q = 0; q < d; ++q) yt[q] = (double)in->x[(size_t)t * d + q];
+    if (cfg->shared_expert) {
+      /* [MoE-deep] §5.2 / §6.2: y = E_shared(x) + sum_j g_j E_j(x); one
+       * shared expert with weight 1 (DeepSeek-V3's form).  Our reading: a
+       * token whose routed slots all overflowed keeps its shared-expert term
+       * (the pass-through replaces only the routed sum). */
+      orc_expert_row(d, f, cfg->expert_bf16, in->x + (size_t)t * d, in->W1s, in->b1s, in->W2s,
+                     in->b2s, ye);
+      for (int q = 0; q < d; ++q) yt[q] += ye[q];
+    }
   }
 
   orc_balance(n, T, k, out->topk_idx, out->topk_gate, out->counts, out->load, out->prob_sum, C,

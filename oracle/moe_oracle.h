@@ -21,8 +21,11 @@
  *                1701.06538), section "方法（與關鍵公式）": "Noisy Top-K 門控" and
  *                "負載平衡損失".
  *  [MoE-intro]   "MoE (Mixture-of-Experts) 算法介绍" (wkbse.com), "工作流程".
- *  [MoE-deep]    "MoE 稀疏架构深度解析" (tufusi.com), §3.1 核心架构 and
- *                §3.2 负载均衡问题.
+ *  [MoE-deep]    "MoE 稀疏架构深度解析" (tufusi.com), §3.1 核心架构,
+ *                §3.2 负载均衡问题, §5.2 DeepSeekMoE 的细粒度设计 (shared
+ *                expert), §6.2 DeepSeek-V3 的 MoE 配置 (sigmoid scores
+ *                normalised over the top K), §6.3 Auxiliary-Loss-Free 负载均衡
+ *                (selection bias and its update).
  *  [Philox]      Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as easy
  *                as 1, 2, 3", SC'11 (Philox4x32-10).
  *  [Box-Muller]  Box & Muller, "A note on the generation of random normal
@@ -49,13 +52,16 @@ extern "C" {
 typedef struct {
   int T, d, n, k, f;
   int hier_a, hier_b, hier_k1, hier_k2;
-  int router;               /* 0: noisy top-k softmax gate; 1: Switch top-1 router */
+  int router;               /* 0: noisy top-k softmax gate; 1: Switch top-1 router;
+                               2: sigmoid scores, top k of score + selection bias,
+                               gates normalised over the kept k (no noise) */
   int noise;                /* 1: add StandardNormal * Softplus(x W_noise)        */
   uint64_t seed;
   double capacity_factor;   /* <= 0: no capacity limit                           */
   int passthrough;          /* 1: a token whose every slot overflowed gets y = x  */
   int expert_bf16;          /* 1: expert weights and activations are bf16         */
   double w_importance, w_load, alpha;
+  int shared_expert;        /* 1: y also gets one always-active expert, weight 1 */
 } orc_cfg;
 
 /* ---- noise ------------------------------------------------------------ */
@@ -73,14 +79,22 @@ int64_t orc_capacity(int T, int k, int n, double capacity_factor);
 /* ---- gate, one token (one row of the batch) ---------------------------- */
 /* x[d]; Wg, Wn: [d][n] row-major; bg: [n] or NULL; Wn may be NULL when noise
  * is off.  Writes c[n] = (x Wg)+bg, s[n] = Softplus(x Wn) (0 if noise off),
- * H[n] (fp32), order[n] = indices sorted by (H desc, index asc), gates[k]
- * (softmax over the kept k for router 0; the full-softmax probability of the
- * argmax for router 1, k must be 1) and, for router 1, p[n] (may be NULL). */
+ * H[n] (fp32: the score KeepTopK ranks; for router 2 it is c + sel_bias),
+ * order[n] = indices sorted by (H desc, index asc), gates[k] (softmax over
+ * the kept k for router 0; the full-softmax probability of the argmax for
+ * router 1, k must be 1; for router 2 Sigmoid(c_i) over the sum of
+ * Sigmoid(c_j) of the kept k) and, for router 1, p[n] (may be NULL).
+ * sel_bias [n] (router 2 only) may be NULL. */
 void orc_gate_row(int d, int n, int k, int router, int noise, uint64_t seed,
                   uint32_t token, uint32_t gate_id, const float *x,
                   const float *Wg, const float *bg, const float *Wn,
                   double *c, double *s, float *H, int *order, double *gates,
-                  double *p);
+                  double *p, const float *sel_bias);
+
+/* Selection-bias update of router 2 ([MoE-deep] §6.3): an expert that took
+ * more than the average T*k/n slots (counts before capacity) gets
+ * bias -= gamma, one that took fewer gets bias += gamma, in fp32. */
+void orc_sel_bias_update(int n, int T, int k, const int32_t *counts, float gamma, float *bias);
 
 /* P(x,i) of the smoothed load estimator for every i, from one token's c, s
  * and H (as written by orc_gate_row). */
@@ -108,6 +122,9 @@ typedef struct {
   const float *Wg2, *bg2, *Wn2;  /* hierarchical secondary gates: [a][d][b], [a][b], [a][d][b] */
   const void *W1; const float *b1;   /* [n][f][d], [n][f] */
   const void *W2; const float *b2;   /* [n][d][f], [n][d] */
+  const float *sel_bias;             /* [n] selection bias of router 2, or NULL (0) */
+  const void *W1s; const float *b1s; /* shared expert: [f][d], [f] */
+  const void *W2s; const float *b2s; /* [d][f], [d] */
 } orc_inputs;
 
 typedef struct {

@@ -37,6 +37,7 @@ class OrcCfg(C.Structure):
         ("router", C.c_int), ("noise", C.c_int), ("seed", C.c_uint64),
         ("capacity_factor", C.c_double), ("passthrough", C.c_int), ("expert_bf16", C.c_int),
         ("w_importance", C.c_double), ("w_load", C.c_double), ("alpha", C.c_double),
+        ("shared_expert", C.c_int),
     ]
 
 
@@ -45,6 +46,8 @@ class OrcInputs(C.Structure):
         ("x", C.c_void_p), ("Wg", C.c_void_p), ("bg", C.c_void_p), ("Wn", C.c_void_p),
         ("Wg2", C.c_void_p), ("bg2", C.c_void_p), ("Wn2", C.c_void_p),
         ("W1", C.c_void_p), ("b1", C.c_void_p), ("W2", C.c_void_p), ("b2", C.c_void_p),
+        ("sel_bias", C.c_void_p),
+        ("W1s", C.c_void_p), ("b1s", C.c_void_p), ("W2s", C.c_void_p), ("b2s", C.c_void_p),
     ]
 
 
@@ -79,7 +82,8 @@ def lib():
         L.orc_capacity.argtypes = [i32, i32, i32, f64]
         L.orc_capacity.restype = C.c_int64
         L.orc_gate_row.argtypes = [i32, i32, i32, i32, i32, C.c_uint64, u32, u32,
-                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+                                   vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.orc_sel_bias_update.argtypes = [i32, i32, i32, vp, C.c_float, vp]
         L.orc_load_row.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.orc_dispatch.argtypes = [i32, i32, i32, C.c_int64, vp, vp, vp, vp, vp, vp, vp]
         L.orc_expert_row.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -145,17 +149,27 @@ def capacity(T: int, k: int, n: int, cf: float) -> int:
 
 
 # ---------------------------------------------------------------- gate
-def gate_row(x, Wg, k, *, bg=None, Wn=None, router=0, noise=True, seed=0, token=0, gate_id=0):
+def gate_row(x, Wg, k, *, bg=None, Wn=None, router=0, noise=True, seed=0, token=0, gate_id=0,
+             sel_bias=None):
     x = _c(x, np.float32)
     Wg = _c(Wg, np.float32)
     d, n = Wg.shape
     bg = _c(bg, np.float32)
     Wn = _c(Wn, np.float32) if noise else None
+    sb = _c(sel_bias, np.float32)
     c = np.zeros(n); s = np.zeros(n); H = np.zeros(n, np.float32)
     order = np.zeros(n, np.int32); gates = np.zeros(k); p = np.zeros(n)
     lib().orc_gate_row(d, n, k, router, int(bool(noise)), seed, token, gate_id, _p(x), _p(Wg),
-                       _p(bg), _p(Wn), _p(c), _p(s), _p(H), _p(order), _p(gates), _p(p))
+                       _p(bg), _p(Wn), _p(c), _p(s), _p(H), _p(order), _p(gates), _p(p), _p(sb))
     return dict(c=c, s=s, H=H, order=order, gates=gates, idx=order[:k].copy(), p=p)
+
+
+def sel_bias_update(counts, T: int, k: int, gamma: float, bias) -> np.ndarray:
+    """Router 2's selection-bias update; returns the new bias (fp32)."""
+    counts = _c(counts, np.int32)
+    b = np.array(bias, dtype=np.float32, copy=True)
+    lib().orc_sel_bias_update(counts.size, T, k, _p(counts), gamma, _p(b))
+    return b
 
 
 def load_row(c, s, H, k, noise=True) -> np.ndarray:
@@ -196,13 +210,14 @@ def expert_row(x, W1, b1, W2, b2, bf16: bool) -> np.ndarray:
 
 # ---------------------------------------------------------------- forward
 _CFG_KEYS = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router", "noise",
-             "seed", "capacity_factor", "passthrough", "expert_bf16", "w_importance", "w_load", "alpha")
+             "seed", "capacity_factor", "passthrough", "expert_bf16", "w_importance", "w_load", "alpha",
+             "shared_expert")
 
 
 def make_cfg(**kw) -> OrcCfg:
     base = dict(hier_a=0, hier_b=0, hier_k1=0, hier_k2=0, router=0, noise=1, seed=0,
                 capacity_factor=0.0, passthrough=0, expert_bf16=0, w_importance=0.1,
-                w_load=0.1, alpha=0.01)
+                w_load=0.1, alpha=0.01, shared_expert=0)
     base.update({k: v for k, v in kw.items() if k in _CFG_KEYS})
     return OrcCfg(**{k: base[k] for k in _CFG_KEYS})
 
@@ -212,7 +227,9 @@ def _inputs(oc, inp):
     keep = {}
     for name, dt in (("x", np.float32), ("Wg", np.float32), ("bg", np.float32), ("Wn", np.float32),
                      ("Wg2", np.float32), ("bg2", np.float32), ("Wn2", np.float32),
-                     ("W1", wdt), ("b1", np.float32), ("W2", wdt), ("b2", np.float32)):
+                     ("W1", wdt), ("b1", np.float32), ("W2", wdt), ("b2", np.float32),
+                     ("sel_bias", np.float32), ("W1s", wdt), ("b1s", np.float32), ("W2s", wdt),
+                     ("b2s", np.float32)):
         keep[name] = _c(inp.get(name), dt)
     return keep, OrcInputs(**{name: _p(a) for name, a in keep.items()})
 
@@ -272,8 +289,9 @@ def balance(n, topk_idx, topk_gate, counts, load, prob_sum=None, C=2**63 - 1, ro
 
 def forward(cfg: dict, inp: dict) -> dict:
     """Run the whole layer.  ``cfg`` holds the fields of ``OrcCfg``; ``inp``
-    holds numpy arrays x, Wg, bg, Wn, Wg2, bg2, Wn2, W1, b1, W2, b2 (bf16
-    expert weights as uint16 bit patterns)."""
+    holds numpy arrays x, Wg, bg, Wn, Wg2, bg2, Wn2, W1, b1, W2, b2, and for
+    router 2 / a shared expert sel_bias, W1s, b1s, W2s, b2s (bf16 expert
+    weights as uint16 bit patterns)."""
     oc = make_cfg(**cfg)
     T, d, n, k = oc.T, oc.d, oc.n, oc.k
     keep, ins = _inputs(oc, inp)
