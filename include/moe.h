@@ -70,7 +70,7 @@ enum {
   MOE_EDEVICE = -4      /* no usable sm_100 device                        */
 };
 
-enum { MOE_ROUTER_NOISY_TOPK = 0, MOE_ROUTER_SWITCH = 1 };
+enum { MOE_ROUTER_NOISY_TOPK = 0, MOE_ROUTER_SWITCH = 1, MOE_ROUTER_SIGMOID = 2 };
 enum { MOE_F32 = 0, MOE_BF16 = 1 };
 /* How the gate's fp32 projections x W_g, x W_noise are computed:
  * MOE_GATE_FP32   fp32 fused multiply-adds on the CUDA cores;
@@ -92,9 +92,17 @@ enum {
  *   Hierarchical layer ([SGMoE-note] "分层 MoE"): hier_a > 0 groups of hier_b
  *   experts each; the primary gate keeps hier_k1 groups, each group's gate
  *   keeps hier_k2 of its experts; then n = hier_a*hier_b, k = hier_k1*hier_k2.
- *   router: MOE_ROUTER_NOISY_TOPK ([SGMoE-xyz] "Noisy Top-K 門控") or
+ *   router: MOE_ROUTER_NOISY_TOPK ([SGMoE-xyz] "Noisy Top-K 門控"),
  *   MOE_ROUTER_SWITCH ([MoE-deep] §3.1: softmax over all experts, top-1, gate
- *   = the winner's probability, no noise).
+ *   = the winner's probability, no noise) or MOE_ROUTER_SIGMOID ([MoE-deep]
+ *   §6.2, §6.3: the k largest routing scores h_i + b_i are kept, b being the
+ *   selection bias (moe_gate_params.sel_bias, moe_sel_bias_update); the gates
+ *   are Sigmoid(h_i) / sum of Sigmoid(h_j) over the kept j, without the bias;
+ *   no noise, flat only).  h = x W_g + b_g as for the other routers.
+ *   shared_expert: 1 adds one always-active expert to every token, weight 1
+ *   ([MoE-deep] §5.2, §6.2: y = E_shared(x) + sum_j g_j E_j(x)); a token whose
+ *   routed slots all overflowed keeps it (pass-through replaces only the
+ *   routed sum).  Only moe_forward evaluates it.
  *   noise: 1 adds StandardNormal() * Softplus(x W_noise); the deviate for
  *   (seed, token t, expert i, gate g) comes from Philox4x32-10 with key
  *   (seed lo, seed hi) and counter (t, i/4, g, 0): words 0,1 give the cosine
@@ -120,25 +128,33 @@ typedef struct moe_config {
   int32_t overflow_passthrough;
   float w_importance, w_load, alpha_aux;
   int32_t gate_precision;     /* MOE_GATE_FP32 or MOE_GATE_TF32X3 */
+  int32_t shared_expert;      /* 0 or 1 */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
  * clean-logit bias, may be NULL).  Hierarchical layer: the same three for the
  * primary gate over hier_a groups, plus the secondary gates W_g2, W_noise2
  * [hier_a][d][hier_b] and b_g2 [hier_a][hier_b] (may be NULL).  W_noise /
- * W_noise2 may be NULL when noise == 0. */
+ * W_noise2 may be NULL when noise == 0.  sel_bias [n]: the selection bias of
+ * MOE_ROUTER_SIGMOID (NULL: zero; ignored by the other routers). */
 typedef struct moe_gate_params {
   const float *W_g, *b_g, *W_noise;
   const float *W_g2, *b_g2, *W_noise2;
+  const float *sel_bias;
 } moe_gate_params;
 
 /* Expert parameters: W1 [n][f][d], W2 [n][d][f] of expert_dtype; b1 [n][f],
- * b2 [n][d] fp32 or NULL. */
+ * b2 [n][d] fp32 or NULL.  With shared_expert: the shared expert's W1s [f][d],
+ * W2s [d][f] (expert_dtype), b1s [f], b2s [d] (fp32 or NULL); else unused. */
 typedef struct moe_expert_params {
   const void *W1;
   const float *b1;
   const void *W2;
   const float *b2;
+  const void *W1s;
+  const float *b1s;
+  const void *W2s;
+  const float *b2s;
 } moe_expert_params;
 
 /* Text for a return code. */
@@ -146,7 +162,8 @@ MOE_API const char *moe_strerror(int code);
 
 /* Validates cfg.  MOE_OK or MOE_EINVAL.  Limits: T >= 0, 1 <= k <= min(n,8),
  * 1 <= n <= 8192, d, f multiples of 8, d <= 16384, f <= 65536; Switch router:
- * k = 1, no noise, n <= 4096, flat only. */
+ * k = 1, no noise, n <= 4096, flat only; sigmoid router: no noise, flat only;
+ * shared_expert 0 or 1. */
 MOE_API int moe_validate(const moe_config *cfg);
 
 /* Expert capacity C = ceil(T*k*capacity_factor/n), or INT64_MAX when
@@ -246,7 +263,7 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm, const float *
  *   [0] L_importance = w_importance * CV(Importance)^2
  *   [1] L_load       = w_load * CV(load)^2
  *   [2] N * sum_i f_i P_i  (Switch: f_i = counts_i / T before the capacity
- *       cut, P_i = prob_sum_i / T); 0 for the noisy gate
+ *       cut, P_i = prob_sum_i / T); 0 for the noisy and sigmoid routers
  *   [3] alpha_aux * [2]
  *   [4] dropped slots / (T*k),   [5] CV(Importance)^2,   [6] CV(load)^2,
  *   [7] dropped slots
@@ -259,12 +276,22 @@ MOE_API int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx,
                        float *losses, void *ws, size_t ws_bytes, int32_t *status,
                        moe_stream_t stream);
 
+/* Selection-bias update of MOE_ROUTER_SIGMOID ([MoE-deep] §6.3): with
+ * counts [n] from a dispatch of T tokens (before the capacity cut), an expert
+ * that took more than the average T*k/n slots gets sel_bias -= gamma, one that
+ * took fewer gets sel_bias += gamma (fp32), one exactly at the average keeps
+ * its bias; the comparison is exact (counts*n against T*k).  sel_bias [n] is
+ * read and written in place on the stream.  Errors: MOE_EINVAL for NULL
+ * pointers or an invalid cfg. */
+MOE_API int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
+                                float *sel_bias, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- fused */
 
-/* The whole layer on one stream: gate, dispatch, experts, combine and the
- * balancing statistics, every intermediate in ws.  Outputs as the step calls
- * above: y [T][d], topk_idx, topk_gate [T][k], importance, load [n],
- * counts [n], losses [8]. */
+/* The whole layer on one stream: gate, dispatch, experts (and the shared
+ * expert when cfg->shared_expert), combine and the balancing statistics,
+ * every intermediate in ws.  Outputs as the step calls above: y [T][d],
+ * topk_idx, topk_gate [T][k], importance, load [n], counts [n], losses [8]. */
 MOE_API int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
                 const moe_expert_params *ep, float *y, int32_t *topk_idx,
                 float *topk_gate, float *importance, float *load, int32_t *counts,

@@ -17,7 +17,7 @@ STATUS_NONFINITE, STATUS_BAD_INDEX, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 EXPORTS = ("moe_strerror", "moe_validate", "moe_capacity", "moe_workspace_size", "moe_gate",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_balance_losses", "moe_forward",
            "moe_trace_enable", "moe_trace_reset", "moe_trace_count", "moe_trace_get",
-           "moe_launch_count", "moe_dispatch_noalloc")
+           "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update")
 
 
 class moe_config(C.Structure):
@@ -27,17 +27,19 @@ class moe_config(C.Structure):
         ("router", C.c_int32), ("noise", C.c_int32), ("expert_dtype", C.c_int32),
         ("seed", C.c_uint64), ("capacity_factor", C.c_double), ("overflow_passthrough", C.c_int32),
         ("w_importance", C.c_float), ("w_load", C.c_float), ("alpha_aux", C.c_float),
-        ("gate_precision", C.c_int32),
+        ("gate_precision", C.c_int32), ("shared_expert", C.c_int32),
     ]
 
 
 class moe_gate_params(C.Structure):
     _fields_ = [("W_g", C.c_void_p), ("b_g", C.c_void_p), ("W_noise", C.c_void_p),
-                ("W_g2", C.c_void_p), ("b_g2", C.c_void_p), ("W_noise2", C.c_void_p)]
+                ("W_g2", C.c_void_p), ("b_g2", C.c_void_p), ("W_noise2", C.c_void_p),
+                ("sel_bias", C.c_void_p)]
 
 
 class moe_expert_params(C.Structure):
-    _fields_ = [("W1", C.c_void_p), ("b1", C.c_void_p), ("W2", C.c_void_p), ("b2", C.c_void_p)]
+    _fields_ = [("W1", C.c_void_p), ("b1", C.c_void_p), ("W2", C.c_void_p), ("b2", C.c_void_p),
+                ("W1s", C.c_void_p), ("b1s", C.c_void_p), ("W2s", C.c_void_p), ("b2s", C.c_void_p)]
 
 
 _lib = None
@@ -62,6 +64,7 @@ def load():
     L.moe_gate.argtypes = [cfgp, vp, C.POINTER(moe_gate_params), vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_dispatch.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_dispatch_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+    L.moe_sel_bias_update.argtypes = [cfgp, vp, C.c_float, vp, vp]
     L.moe_expert_ffn.argtypes = [cfgp, vp, vp, C.POINTER(moe_expert_params), vp, vp, sz, vp, vp]
     L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_balance_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]

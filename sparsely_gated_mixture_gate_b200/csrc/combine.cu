@@ -1,7 +1,9 @@
 // combine.cu -- y = sum_i G(x)_i E_i(x) ([SGMoE-note] "Sparsely-Gated MoE 层架构")
 // over each token's kept slots, in slot order, fp32 accumulation.  A dropped
 // slot adds nothing; a token with no kept slot passes through the residual
-// ([MoE-deep] §3.2) when pass-through is on (y = x), else gets 0.
+// ([MoE-deep] §3.2) when pass-through is on (y = x), else gets 0.  With a
+// shared expert ([MoE-deep] §5.2) its row E_shared(x) is the first term of
+// every token's sum (and is added to the pass-through x).
 // One warp per token, 8 features per lane per step: the 16-byte loads of all
 // the token's expert rows are issued before the sums, two 16-byte stores of y.
 #include "internal.h"
@@ -17,7 +19,8 @@ __global__ void __launch_bounds__(NT) combine_kernel(const void *__restrict__ yp
                                                       const float *__restrict__ gate,
                                                       const int *__restrict__ row_of,
                                                       const float *__restrict__ x, int passthrough,
-                                                      int T, int k, int d, float *__restrict__ y) {
+                                                      int T, int k, int d, float *__restrict__ y,
+                                                      const void *__restrict__ ys) {
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
@@ -32,6 +35,28 @@ __global__ void __launch_bounds__(NT) combine_kernel(const void *__restrict__ yp
   }
   float4 *yr = reinterpret_cast<float4 *>(y + (size_t)t * d);
   const int nchunk = d >> 3;
+  // the shared expert's 8 features of chunk c of this token (0 without one)
+  auto shared8 = [&](int c, float (&s)[8]) {
+    if (!ys) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) s[u] = 0.f;
+    } else if (BF16) {
+      const uint4 pk = __ldg(reinterpret_cast<const uint4 *>(
+                                 static_cast<const __nv_bfloat16 *>(ys) + (size_t)t * d) + c);
+      const uint32_t w4[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[u]));
+        s[2 * u] = f2.x;
+        s[2 * u + 1] = f2.y;
+      }
+    } else {
+      const float4 *src = reinterpret_cast<const float4 *>(static_cast<const float *>(ys) + (size_t)t * d);
+      const float4 u = __ldg(src + 2 * c), v = __ldg(src + 2 * c + 1);
+      s[0] = u.x; s[1] = u.y; s[2] = u.z; s[3] = u.w;
+      s[4] = v.x; s[5] = v.y; s[6] = v.z; s[7] = v.w;
+    }
+  };
   if (!any) {
     const float4 *xr = reinterpret_cast<const float4 *>(x + (size_t)t * d);
     for (int c = lane; c < nchunk; c += 32) {
@@ -40,12 +65,19 @@ __global__ void __launch_bounds__(NT) combine_kernel(const void *__restrict__ yp
         u = __ldg(xr + 2 * c);
         v = __ldg(xr + 2 * c + 1);
       }
+      if (ys) {
+        float s[8];
+        shared8(c, s);
+        u.x += s[0]; u.y += s[1]; u.z += s[2]; u.w += s[3];
+        v.x += s[4]; v.y += s[5]; v.z += s[6]; v.w += s[7];
+      }
       yr[2 * c] = u;
       yr[2 * c + 1] = v;
     }
     return;
   }
-#pragma unroll 2
+  constexpr int UNR = KM <= 4 ? 2 : 1;  // two chunks in flight while registers allow
+#pragma unroll UNR
   for (int c = lane; c < nchunk; c += 32) {
     // every kept slot's 8 features first (independent loads), then the sum
     float f[KM][8];
@@ -71,7 +103,8 @@ __global__ void __launch_bounds__(NT) combine_kernel(const void *__restrict__ yp
         f[j][4] = v.x; f[j][5] = v.y; f[j][6] = v.z; f[j][7] = v.w;
       }
     }
-    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    float acc[8];
+    shared8(c, acc);
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
       if (rows[j] < 0) continue;
@@ -87,11 +120,11 @@ __global__ void __launch_bounds__(NT) combine_kernel(const void *__restrict__ yp
 
 int launch_combine(const void *y_perm, int bf16, const float *gate, const int *row_of,
                    const float *x, int passthrough, int T, int k, int d, float *y,
-                   cudaStream_t st) {
+                   const void *y_shared, cudaStream_t st) {
   dim3 grid((unsigned)ceil_div(T, NT / 32));
   auto go = [&](auto kern) {
     return launch("combine", kern, grid, dim3(NT), 0, st, y_perm, gate, row_of, x, passthrough, T,
-                  k, d, y);
+                  k, d, y, y_shared);
   };
   if (k > kMaxK) return MOE_EINVAL;
   if (bf16) {

@@ -19,8 +19,8 @@
 //                      and the expert GEMM tile tables
 //   3. dispatch_place  one warp per token: rank = base[b][e] + block rank ->
 //                      row_of, perm_token, sorted gates; optionally the token's
-//                      x row copied (and cast) into its expert rows, 16-byte
-//                      stores
+//                      x row copied (and cast) into its expert rows, and into
+//                      row t of the shared expert's input, 16-byte stores
 // No step depends on scheduling order, so the permutation is deterministic.
 #include <limits.h>
 
@@ -274,7 +274,12 @@ template <bool COPY, bool BF16>
 __global__ void __launch_bounds__(NT) dispatch_place_kernel(
     const int *idx, const float *gate, int T, int k, int n, int tpb, long long C,
     const int *base, const int *offsets, const int *ucoff, int *row_of, int *perm_token,
-    int *perm_slot, float *gate_sorted, const float *x, int d, void *x_perm) {
+    int *perm_slot, float *gate_sorted, const float *x, int d, void *x_perm, void *x_shared,
+    int *shared_off) {
+  if (shared_off && blockIdx.x == 0 && threadIdx.x == 0) {
+    shared_off[0] = 0;
+    shared_off[1] = T;
+  }
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
@@ -324,6 +329,8 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
         for (int j = 0; j < kMaxK; ++j)
           if (rows[j] >= 0)
             reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(x_perm) + (size_t)rows[j] * d)[c] = pk;
+        if (x_shared)
+          reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(x_shared) + (size_t)t * d)[c] = pk;
       } else {
 #pragma unroll
         for (int j = 0; j < kMaxK; ++j)
@@ -332,6 +339,11 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
             dst[2 * c] = u;
             dst[2 * c + 1] = v;
           }
+        if (x_shared) {
+          float4 *dst = reinterpret_cast<float4 *>(static_cast<float *>(x_shared) + (size_t)t * d);
+          dst[2 * c] = u;
+          dst[2 * c + 1] = v;
+        }
       }
     }
   }
@@ -404,7 +416,8 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
   auto place = [&](auto kern) {
     return launch("dispatch_place", kern, grid, dim3(NT), 0, st, a.idx, a.gate, a.T, a.k, a.n, tpb,
                   C, (const int *)a.base, (const int *)a.offsets, (const int *)a.ucoff, a.row_of,
-                  a.perm_token, a.perm_slot, a.gate_sorted, a.x, a.d, a.x_perm);
+                  a.perm_token, a.perm_slot, a.gate_sorted, a.x, a.d, a.x_perm, a.x_shared,
+                  a.shared_off);
   };
   if (!a.x) return place(dispatch_place_kernel<false, false>);
   if (a.x_bf16) return place(dispatch_place_kernel<true, true>);

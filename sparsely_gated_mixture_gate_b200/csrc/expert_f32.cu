@@ -64,7 +64,7 @@ int launch_expert_f32(const ExpertArgs &a, cudaStream_t st) {
                              (int)smem) != cudaSuccess)
       return MOE_EINVAL;
   }
-  return launch("expert_ffn_fp32", expert_f32_kernel, dim3(a.S), dim3(NT), smem, st,
+  return launch(a.name ? a.name : "expert_ffn_fp32", expert_f32_kernel, dim3(a.S), dim3(NT), smem, st,
                 static_cast<const float *>(a.x_perm), a.offsets, a.n, a.d, a.f,
                 static_cast<const float *>(a.W1), a.b1, static_cast<const float *>(a.W2), a.b2,
                 static_cast<float *>(a.y_perm));

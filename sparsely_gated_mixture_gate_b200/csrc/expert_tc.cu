@@ -388,7 +388,7 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int slot = -1;
-  trace_begin("expert_ffn_tcgen05", st, &slot);
+  trace_begin(a.name ? a.name : "expert_ffn_tcgen05", st, &slot);
   const cudaError_t e = cudaLaunchKernelEx(&cfg, expert_ffn_kernel, a1, b1, a2, b2, f);
   trace_end(slot, st);
   count_launch();

@@ -89,6 +89,7 @@ struct RouteArgs {
   int k1;
   float *load_part;        // [tiles][nb]
   float *psum_part;        // [tiles][nb] or nullptr
+  const float *sel_bias;   // sigmoid router: [nb] selection bias, or nullptr
   int *status;
 };
 int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st);
@@ -122,6 +123,8 @@ struct DispatchArgs {
   int *ticket;             // one int of scratch (last-block election of the scan)
   const float *x;          // [T][d] or nullptr: with it x rows are copied to x_perm
   void *x_perm;            // [kept rows][d], bf16 (x_bf16) or fp32
+  void *x_shared;          // [T][d] or nullptr: every x row again, in token order
+  int *shared_off;         // with x_shared: {0, T}, the shared expert's row offsets
   int d, x_bf16;
   int *status;
 };
@@ -143,6 +146,7 @@ struct ExpertArgs {
   int4 *tab1, *tab2;       // tile tables of GEMM1 / GEMM2
   int *mdone;              // [M-blocks + 1] GEMM1 -> GEMM2 counters (zeroed by the plan)
   int plan_ready;          // 1: mprefix and the tables were written by the dispatch
+  const char *name;        // trace name, or nullptr for the default
   int n, d, f, S;
   const void *W1, *W2;
   const float *b1, *b2;
@@ -153,9 +157,13 @@ struct ExpertArgs {
 int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st);
 int launch_expert_f32(const ExpertArgs &a, cudaStream_t st);
 
+// y_shared [T][d] (expert dtype) or nullptr: the shared expert's rows, added
+// to every token before its routed slots
 int launch_combine(const void *y_perm, int bf16, const float *gate, const int *row_of,
                    const float *x, int passthrough, int T, int k, int d, float *y,
-                   cudaStream_t st);
+                   const void *y_shared, cudaStream_t st);
+int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, float *bias,
+                           cudaStream_t st);
 
 int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
                       cudaStream_t st);

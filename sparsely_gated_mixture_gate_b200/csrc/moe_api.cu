@@ -129,6 +129,7 @@ struct Layout {
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch, ticket;
   size_t mprefix, tab1, tab2, mdone, x_perm, hid, y_perm;
+  size_t x_shared, y_shared, shared_off;  // shared expert: input and output rows, {0, T}
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
@@ -211,6 +212,13 @@ Layout make_layout(const moe_config &c) {
   L.x_perm = bp.take(esz * S * (size_t)c.d);
   L.hid = bp.take(esz * S * (size_t)c.f);
   L.y_perm = bp.take(esz * S * (size_t)c.d);
+  if (c.shared_expert) {
+    L.x_shared = bp.take(esz * (size_t)T * c.d);
+    L.y_shared = bp.take(esz * (size_t)T * c.d);
+    L.shared_off = bp.take(8);
+  } else {
+    L.x_shared = L.y_shared = L.shared_off = 0;
+  }
   if (c.gate_precision == MOE_GATE_TF32X3) {
     const size_t rows = hier ? (T > R2 ? T : R2) : T;
     const size_t nw = (size_t)(c.noise ? 2 : 1);
@@ -339,6 +347,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.G = 1;
   r.RT = L.RT1;
   r.load_part = at<float>(ws, L.load_part);
+  r.sel_bias = (!hier && c.router == MOE_ROUTER_SIGMOID) ? gp.sel_bias : nullptr;
   r.status = status;
   if (!hier) {
     r.k = c.k;
@@ -444,8 +453,10 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
 int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const float *gate,
                  int64_t C, int *counts, int *offsets, int *perm_token, int *row_of,
                  const float *x, void *x_perm, void *ws, int *status, cudaStream_t st,
-                 bool plan_experts = false) {
+                 bool plan_experts = false, void *x_shared = nullptr, int *shared_off = nullptr) {
   DispatchArgs da{};
+  da.x_shared = x_shared;
+  da.shared_off = shared_off;
   da.ticket = at<int>(ws, L.ticket);
   da.x = x;
   da.x_perm = x_perm;
@@ -481,8 +492,9 @@ int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const flo
 
 int run_experts(const moe_config &c, const Layout &L, const void *x_perm, const int *offsets,
                 const moe_expert_params &ep, void *y_perm, void *ws, int *status,
-                cudaStream_t st, int plan_ready = 0) {
+                cudaStream_t st, int plan_ready = 0, const char *name = nullptr) {
   ExpertArgs e{};
+  e.name = name;
   e.x_perm = x_perm;
   e.offsets = offsets;
   e.mprefix = at<int>(ws, L.mprefix);
@@ -510,11 +522,18 @@ bool gate_params_ok(const moe_config &c, const moe_gate_params *gp) {
   if (c.noise && (!gp->W_noise || !aligned(gp->W_noise, 16))) return false;
   if (c.hier_a > 0 && (!gp->W_g2 || !aligned(gp->W_g2, 16))) return false;
   if (c.hier_a > 0 && c.noise && (!gp->W_noise2 || !aligned(gp->W_noise2, 16))) return false;
+  // the routing kernel reads the selection bias in 16-byte pieces
+  if (c.router == MOE_ROUTER_SIGMOID && gp->sel_bias && !aligned(gp->sel_bias, 16)) return false;
   return true;
 }
 
 bool expert_params_ok(const moe_expert_params *ep) {
   return ep && ep->W1 && ep->W2 && aligned(ep->W1, 16) && aligned(ep->W2, 16);
+}
+
+bool shared_params_ok(const moe_config &c, const moe_expert_params *ep) {
+  return !c.shared_expert ||
+         (ep->W1s && ep->W2s && aligned(ep->W1s, 16) && aligned(ep->W2s, 16));
 }
 
 }  // namespace
@@ -542,7 +561,11 @@ int moe_validate(const moe_config *c) {
     return MOE_EINVAL;
   if (c->d < 8 || c->d % 8 || c->d > 16384 || c->f < 8 || c->f % 8 || c->f > 65536)
     return MOE_EINVAL;
-  if (c->router != MOE_ROUTER_NOISY_TOPK && c->router != MOE_ROUTER_SWITCH) return MOE_EINVAL;
+  if (c->router != MOE_ROUTER_NOISY_TOPK && c->router != MOE_ROUTER_SWITCH &&
+      c->router != MOE_ROUTER_SIGMOID)
+    return MOE_EINVAL;
+  if (c->router == MOE_ROUTER_SIGMOID && (c->noise || c->hier_a)) return MOE_EINVAL;
+  if (c->shared_expert != 0 && c->shared_expert != 1) return MOE_EINVAL;
   if (c->noise != 0 && c->noise != 1) return MOE_EINVAL;
   if (c->expert_dtype != MOE_F32 && c->expert_dtype != MOE_BF16) return MOE_EINVAL;
   if (c->overflow_passthrough != 0 && c->overflow_passthrough != 1) return MOE_EINVAL;
@@ -629,7 +652,7 @@ int moe_combine(const moe_config *cfg, const void *y_perm, const float *topk_gat
   if (c.T > 0 && c.overflow_passthrough && (!x || !aligned(x, 16))) return MOE_EINVAL;
   MOE_TRY(check_device());
   return launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
-                        c.overflow_passthrough, c.T, c.k, c.d, y,
+                        c.overflow_passthrough, c.T, c.k, c.d, y, nullptr,
                         reinterpret_cast<cudaStream_t>(stream));
 }
 
@@ -664,7 +687,8 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   if (!importance || !load || !counts || !losses) return MOE_EINVAL;
   if (c.T > 0 && (!x || !y || !topk_idx || !topk_gate || !aligned(x, 16) || !aligned(y, 16)))
     return MOE_EINVAL;
-  if (!gate_params_ok(c, gp) || !expert_params_ok(ep)) return MOE_EINVAL;
+  if (!gate_params_ok(c, gp) || !expert_params_ok(ep) || !shared_params_ok(c, ep))
+    return MOE_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const bool sw = c.router == MOE_ROUTER_SWITCH;
   float *prob_sum = sw ? at<float>(ws, L.prob_sum) : nullptr;
@@ -678,8 +702,11 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   MOE_TRY(side_stream(&side));
   MOE_TRY(run_gate(c, L, x, *gp, topk_idx, topk_gate, load, prob_sum, ws, status, st, side));
   const bool tc = c.expert_dtype == MOE_BF16;
+  void *x_shared = c.shared_expert ? at<void>(ws, L.x_shared) : nullptr;
+  void *y_shared = c.shared_expert ? at<void>(ws, L.y_shared) : nullptr;
+  int *shared_off = c.shared_expert ? at<int>(ws, L.shared_off) : nullptr;
   MOE_TRY(run_dispatch(c, L, topk_idx, topk_gate, C, counts, offsets, at<int>(ws, L.perm_token),
-                       row_of, x, x_perm, ws, status, st, tc));
+                       row_of, x, x_perm, ws, status, st, tc, x_shared, shared_off));
   // balance statistics beside the expert chain; they read only the gate's and
   // the dispatch's outputs
   MOE_TRY(stream_after(side->s, st, side->fork_dispatch));
@@ -689,10 +716,30 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
                         c.w_importance, c.w_load, c.alpha_aux, losses, side->s));
   if (c.T > 0) {
     MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));
+    if (c.shared_expert) {
+      // every token through the shared expert: one expert, rows 0..T-1 in
+      // token order; the routed launch is done with the tile tables and the
+      // hidden-layer rows by now, so they are reused
+      moe_config cs = c;
+      cs.n = 1;
+      cs.k = 1;
+      moe_expert_params es{ep->W1s, ep->b1s, ep->W2s, ep->b2s, nullptr, nullptr, nullptr, nullptr};
+      MOE_TRY(run_experts(cs, L, x_shared, shared_off, es, y_shared, ws, status, st, 0,
+                          tc ? "shared_expert_ffn_tcgen05" : "shared_expert_ffn_fp32"));
+    }
     MOE_TRY(launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
-                           c.overflow_passthrough, c.T, c.k, c.d, y, st));
+                           c.overflow_passthrough, c.T, c.k, c.d, y, y_shared, st));
   }
   return stream_after(st, side->s, side->join);
+}
+
+int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
+                        float *sel_bias, moe_stream_t stream) {
+  MOE_TRY(moe_validate(cfg));
+  if (!counts || !sel_bias) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_sel_bias_update(counts, cfg->n, cfg->T, cfg->k, gamma, sel_bias,
+                                reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_trace_enable(int on) {

@@ -8,6 +8,8 @@
 //     kth_excluding is the (k+1)-th largest H when i is kept, the k-th otherwise
 //   Switch router ([MoE-deep] §3.1): p = softmax(c) over all experts, the row
 //   goes to argmax p with gate p_argmax; sum_t p_i is accumulated too.
+//   Sigmoid router ([MoE-deep] §6.2, §6.3): H_i = c_i + b_i with the selection
+//   bias b, top-k of H, gates Sigmoid(c_i) / sum of Sigmoid(c_j) over the kept.
 // Pass 1, one warp per row: each lane scans column quads 4m .. 4m+3 (16-byte
 // loads, one Philox call per quad), keeps a sorted top-(k+1) list in
 // registers, and the warp merges the 32 lists with shuffles; the row's kept
@@ -141,7 +143,18 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
           }
         }
         float h[4] = {cv[0], cv[1], cv[2], cv[3]};
-        if (a.noise) {
+        if (a.sel_bias) {  // sigmoid router: the bias enters the routing score only
+          float bv[4];
+          if (vec4) {
+            const float4 b4 = *reinterpret_cast<const float4 *>(a.sel_bias + i0);
+            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) bv[j] = i0 + j < nb ? a.sel_bias[i0 + j] : 0.f;
+          }
+#pragma unroll
+          for (int j = 0; j < 4; ++j) h[j] = cv[j] + bv[j];
+        } else if (a.noise) {
           const uint4 wd =
               philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, gate_id, 0u), key0, key1);
           float z[4];
@@ -200,10 +213,24 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
         }
       }
 
-      // gates: softmax over the kept k (Switch: the winner's full-softmax p)
+      // gates: softmax over the kept k (Switch: the winner's full-softmax p;
+      // sigmoid router: Sigmoid(c) of the kept, normalised over them)
       float gate_j = 0.f;
       int idx_j = 0;
-      {
+      if (a.router == MOE_ROUTER_SIGMOID) {
+        float sg[KM], den = 0.f;
+#pragma unroll
+        for (int j = 0; j < KM; ++j) {
+          sg[j] = S[j].i < nb ? 1.f / (1.f + expf(-crow[S[j].i])) : 0.f;
+          den += sg[j];
+        }
+#pragma unroll
+        for (int j = 0; j < KM; ++j)
+          if (j == lane) {
+            idx_j = S[j].i;
+            gate_j = sg[j] / den;
+          }
+      } else {
         float den = 0.f;
 #pragma unroll
         for (int j = 0; j < KM; ++j) den += expf(S[j].v - S[0].v);

@@ -89,7 +89,25 @@ __global__ void __launch_bounds__(LNT) losses_kernel(const float *importance, co
   }
 }
 
+// Selection-bias update of the sigmoid router ([MoE-deep] §6.3): overloaded
+// experts (more than T*k/n slots, compared exactly as counts*n > T*k) lose
+// gamma, underloaded ones gain it, fp32.
+__global__ void sel_bias_update_kernel(const int *counts, int n, long long total, float gamma,
+                                       float *bias) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n) return;
+  const long long scaled = (long long)counts[i] * n;
+  if (scaled > total) bias[i] = bias[i] - gamma;
+  else if (scaled < total) bias[i] = bias[i] + gamma;
+}
+
 }  // namespace
+
+int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, float *bias,
+                           cudaStream_t st) {
+  return launch("sel_bias_update", sel_bias_update_kernel, dim3((unsigned)ceil_div(n, 256)),
+                dim3(256), 0, st, counts, n, (long long)T * k, gamma, bias);
+}
 
 int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
                       cudaStream_t st) {

@@ -48,6 +48,7 @@ class Config:
     w_load: float = 0.1
     alpha: float = 0.01
     gate_precision: int = 0   # 0: fp32 multiply-adds, 1: tensor cores, 3-pass TF32 split
+    shared_expert: int = 0    # 1: one always-active expert (W1s, b1s, W2s, b2s) in forward
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -64,7 +65,7 @@ class Config:
                           seed=self.seed, capacity_factor=float(self.capacity_factor),
                           overflow_passthrough=self.passthrough, w_importance=self.w_importance,
                           w_load=self.w_load, alpha_aux=self.alpha,
-                          gate_precision=self.gate_precision)
+                          gate_precision=self.gate_precision, shared_expert=self.shared_expert)
 
     @property
     def expert_dtype(self):
@@ -130,12 +131,15 @@ def workspace(cfg: Config, device) -> torch.Tensor:
 def gate_params(params: dict) -> moe_gate_params:
     return moe_gate_params(W_g=_ptr(params.get("Wg")), b_g=_ptr(params.get("bg")),
                            W_noise=_ptr(params.get("Wn")), W_g2=_ptr(params.get("Wg2")),
-                           b_g2=_ptr(params.get("bg2")), W_noise2=_ptr(params.get("Wn2")))
+                           b_g2=_ptr(params.get("bg2")), W_noise2=_ptr(params.get("Wn2")),
+                           sel_bias=_ptr(params.get("sel_bias")))
 
 
 def expert_params(params: dict) -> moe_expert_params:
     return moe_expert_params(W1=_ptr(params.get("W1")), b1=_ptr(params.get("b1")),
-                             W2=_ptr(params.get("W2")), b2=_ptr(params.get("b2")))
+                             W2=_ptr(params.get("W2")), b2=_ptr(params.get("b2")),
+                             W1s=_ptr(params.get("W1s")), b1s=_ptr(params.get("b1s")),
+                             W2s=_ptr(params.get("W2s")), b2s=_ptr(params.get("b2s")))
 
 
 def _check_params(cfg: Config, p: dict, dev, gate=True, experts=True):
@@ -144,6 +148,8 @@ def _check_params(cfg: Config, p: dict, dev, gate=True, experts=True):
         _need(p.get("Wg"), "Wg", torch.float32, (cfg.d, gn), dev)
         _need(p.get("Wn"), "Wn", torch.float32, (cfg.d, gn), dev, optional=not cfg.noise)
         _need(p.get("bg"), "bg", torch.float32, (gn,), dev, optional=True)
+        if cfg.router == 2:
+            _need(p.get("sel_bias"), "sel_bias", torch.float32, (cfg.n,), dev, optional=True)
         if cfg.hier_a:
             sh = (cfg.hier_a, cfg.d, cfg.hier_b)
             _need(p.get("Wg2"), "Wg2", torch.float32, sh, dev)
@@ -154,6 +160,11 @@ def _check_params(cfg: Config, p: dict, dev, gate=True, experts=True):
         _need(p.get("W2"), "W2", cfg.expert_dtype, (cfg.n, cfg.d, cfg.f), dev)
         _need(p.get("b1"), "b1", torch.float32, (cfg.n, cfg.f), dev, optional=True)
         _need(p.get("b2"), "b2", torch.float32, (cfg.n, cfg.d), dev, optional=True)
+        if cfg.shared_expert:
+            _need(p.get("W1s"), "W1s", cfg.expert_dtype, (cfg.f, cfg.d), dev)
+            _need(p.get("W2s"), "W2s", cfg.expert_dtype, (cfg.d, cfg.f), dev)
+            _need(p.get("b1s"), "b1s", torch.float32, (cfg.f,), dev, optional=True)
+            _need(p.get("b2s"), "b2s", torch.float32, (cfg.d,), dev, optional=True)
 
 
 def new_status(device) -> torch.Tensor:
@@ -353,6 +364,18 @@ def forward(cfg: Config, x: torch.Tensor, params: dict) -> dict:
 
 
 # ---------------------------------------------------------------- tracing
+def sel_bias_update(cfg: Config, counts: torch.Tensor, gamma: float, sel_bias: torch.Tensor):
+    """The sigmoid router's selection-bias update, in place on the current
+    stream: experts with more than T*k/n of the slots in counts lose gamma,
+    those with fewer gain it."""
+    _need(counts, "counts", torch.int32, (cfg.n,), sel_bias.device)
+    _need(sel_bias, "sel_bias", torch.float32, (cfg.n,), counts.device)
+    c = cfg.c()
+    _check(_lib.load().moe_sel_bias_update(C.byref(c), _ptr(counts), float(gamma), _ptr(sel_bias),
+                                           _stream()), "moe_sel_bias_update")
+    return sel_bias
+
+
 def trace_enable(on: bool = True):
     _lib.load().moe_trace_enable(int(bool(on)))
 

@@ -38,7 +38,7 @@ class Workload:
     hier_b: int = 0
     hier_k1: int = 0
     hier_k2: int = 0
-    router: int = 0             # 0 noisy top-k gate, 1 Switch top-1 router
+    router: int = 0             # 0 noisy top-k gate, 1 Switch top-1 router, 2 sigmoid router
     noise: int = 1
     expert_bf16: int = 1
     capacity_factor: float = 0.0
@@ -51,6 +51,8 @@ class Workload:
     w_load: float = 0.1
     alpha: float = 0.01
     gate_precision: int = 0     # library option; the oracle is always fp64
+    shared_expert: int = 0      # 1: one always-active expert added to every token
+    sel_bias_std: float = 0.0   # sigmoid router: spread of the selection bias
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -63,7 +65,7 @@ class Workload:
     def cfg(self) -> dict:
         keys = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router",
                 "noise", "expert_bf16", "capacity_factor", "passthrough", "seed",
-                "w_importance", "w_load", "alpha")
+                "w_importance", "w_load", "alpha", "shared_expert")
         return {k: getattr(self, k) for k in keys}
 
 
@@ -85,6 +87,15 @@ VARIANTS = {
     "tiny-bias": WORKLOADS["tiny-flat"].with_(name="tiny-bias", bias_var=0.1, logit_bias_var=0.1),
     # a skewed Switch router so that the capacity limit actually drops tokens
     "switch-skew": WORKLOADS["switch-top1"].with_(name="switch-skew", logit_bias_var=0.5),
+    # sigmoid router with a selection bias and a shared expert ("MoE 稀疏架构深度
+    # 解析" §5.2, §6.2, §6.3), DeepSeek-V3's shape scaled to the lm-flat layer:
+    # 256 routed experts, top 8 of them, experts half as wide, one shared expert
+    "deepseek-tiny": Workload("deepseek-tiny", T=64, d=32, n=16, k=4, f=64, router=2, noise=0,
+                              shared_expert=1, sel_bias_std=0.5, bias_var=0.1),
+    "deepseek-tiny-f32": Workload("deepseek-tiny-f32", T=64, d=32, n=16, k=4, f=64, router=2,
+                                  noise=0, shared_expert=1, sel_bias_std=0.5, expert_bf16=0),
+    "deepseek-flat": Workload("deepseek-flat", T=8192, d=512, n=256, k=8, f=512, router=2,
+                              noise=0, shared_expert=1, sel_bias_std=0.1, x_unit_rows=True),
 }
 
 
@@ -139,6 +150,8 @@ def make_inputs(w: Workload, device="cpu", T: Optional[int] = None, seed: Option
         out["Wg2"] = _randn((w.hier_a, d, w.hier_b), gstd, device, s, 5)
         out["Wn2"] = _randn((w.hier_a, d, w.hier_b), gstd, device, s, 6) if w.noise else None
         out["bg2"] = None
+    out["sel_bias"] = (_randn((gn,), w.sel_bias_std, device, s, 12)
+                       if w.router == 2 and w.sel_bias_std > 0 else None)
     if experts:
         edt = torch.bfloat16 if w.expert_bf16 else torch.float32
         out["W1"] = _randn_chunked(n, f, d, 1.0 / math.sqrt(d), device, s, 7, edt)
@@ -149,6 +162,12 @@ def make_inputs(w: Workload, device="cpu", T: Optional[int] = None, seed: Option
         else:
             out["b1"] = torch.zeros(n, f, device=device)
             out["b2"] = torch.zeros(n, d, device=device)
+        if w.shared_expert:
+            out["W1s"] = _randn_chunked(1, f, d, 1.0 / math.sqrt(d), device, s, 13, edt)[0]
+            out["W2s"] = _randn_chunked(1, d, f, 1.0 / math.sqrt(f), device, s, 14, edt)[0]
+            sv = math.sqrt(w.bias_var) if w.bias_var > 0 else 0.0
+            out["b1s"] = _randn((f,), sv, device, s, 15) if sv else torch.zeros(f, device=device)
+            out["b2s"] = _randn((d,), sv, device, s, 16) if sv else torch.zeros(d, device=device)
     return out
 
 

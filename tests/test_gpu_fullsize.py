@@ -60,10 +60,13 @@ def _expert_sum(orc, w, inp, t, idx_row, gate_row, kept):
                                           bf16=bool(w.expert_bf16))
     if not any(kept) and w.passthrough:
         y = x.astype(np.float64)
+    if w.shared_expert:  # the always-active expert, weight 1
+        y = y + orc.expert_row(x, _bits(inp["W1s"]), inp["b1s"].cpu().numpy(), _bits(inp["W2s"]),
+                               inp["b2s"].cpu().numpy(), bf16=bool(w.expert_bf16))
     return y
 
 
-CASES = ["lm-flat", "many-expert", "hierarchical", "switch-top1", "switch-skew"]
+CASES = ["lm-flat", "many-expert", "hierarchical", "switch-top1", "switch-skew", "deepseek-flat"]
 
 
 @pytest.mark.parametrize("gp", [pytest.param(0, id="fp32fma"), pytest.param(1, id="tf32x3")])
@@ -86,7 +89,7 @@ def test_fullsize(orc, name, gp):
     # ---- properties at any size
     assert counts.sum() == T * k
     assert np.array_equal(np.bincount(idx.ravel(), minlength=n), counts)
-    if w.router == 0:
+    if w.router in (0, 2):
         assert np.allclose(gate.sum(1), 1.0, atol=2e-6 * k)
     assert out["importance"].sum().item() == pytest.approx(float(gate.sum()), rel=1e-5)
     load = out["load"].numpy()
@@ -97,7 +100,7 @@ def test_fullsize(orc, name, gp):
     C = orc.capacity(T, k, n, w.capacity_factor)
     assert losses[7] == np.maximum(counts.astype(np.int64) - C, 0).sum()
 
-    gate_keys = ["x", "Wg", "bg", "Wn", "Wg2", "bg2", "Wn2"]
+    gate_keys = ["x", "Wg", "bg", "Wn", "Wg2", "bg2", "Wn2", "sel_bias"]
     ginp = _host(inp, gate_keys)
     toks = _sample(T)
 

@@ -73,6 +73,13 @@ SMALL = {
     "one-token": W["lm-flat"].with_(T=1, n=16, k=2, d=64, f=64),
     "bf16-narrow": W["lm-flat"].with_(T=100, n=5, k=2, d=40, f=24),
     "hier-nonoise": W["hierarchical"].with_(T=256, d=64, n=8 * 16, hier_a=8, hier_b=16, f=128, noise=0),
+    # sigmoid router with selection bias and shared expert, and its parts
+    "deepseek-tiny": V["deepseek-tiny"],
+    "deepseek-tiny-f32": V["deepseek-tiny-f32"],
+    "deepseek-noshared": V["deepseek-tiny"].with_(shared_expert=0),
+    "deepseek-512": V["deepseek-flat"].with_(T=512),
+    "shared-noisy": W["lm-flat"].with_(T=200, n=32, k=2, d=64, f=64, shared_expert=1),
+    "shared-passthrough": V["switch-skew"].with_(T=1024, d=128, n=16, f=128, shared_expert=1),
 }
 
 
@@ -308,6 +315,22 @@ def test_forward_matches_oracle(orc, name, gp):
     tol = 2e-2 if w.expert_bf16 else 1e-4
     err = rel_fro(out["y"].numpy(), ref["y"])
     assert err < tol, err
+
+
+@pytest.mark.parametrize("n,T,k", [(256, 8192, 8), (7, 1000, 3), (1, 5, 1), (300, 0, 2)])
+def test_sel_bias_update_matches_oracle(orc, n, T, k):
+    rng = np.random.default_rng(n + T)
+    counts = rng.integers(0, 2 * max(T * k // max(n, 1), 1) + 1, n).astype(np.int32)
+    if n > 1:
+        counts[0] = (T * k) // n if (T * k) % n == 0 else counts[0]  # one exactly at the average
+    bias = rng.normal(0, 1, n).astype(np.float32)
+    gamma = 1e-3
+    want = orc.sel_bias_update(counts, T, k, gamma, bias)
+    cfg = M.Config(T=T, d=8, n=n, k=k, f=8, router=2, noise=0)
+    b = torch.from_numpy(bias.copy()).to(DEV)
+    M.sel_bias_update(cfg, torch.from_numpy(counts).to(DEV), gamma, b)
+    torch.cuda.synchronize()
+    assert np.array_equal(b.cpu().numpy().view(np.uint32), want.view(np.uint32))
 
 
 def test_forward_is_deterministic():
