@@ -163,6 +163,9 @@ def kernel_work(w, name: str, S_kept: int):
         # y_perm out (the hidden layer's round trip through memory is this
         # implementation's choice, not counted as algorithmic traffic)
         return "tensor", 4.0 * S_kept * d * f, n * 2 * d * f * esz + 2 * S_kept * d * esz
+    if name == "shared_expert_ffn_tcgen05":
+        # one expert on all T tokens: its weights once, x rows in, rows out
+        return "tensor", 4.0 * T * d * f, 2 * d * f * esz + 2 * T * d * esz
     if name == "gate_gemm_fp32":
         return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
     if name == "gate_gemm_tf32x3":
@@ -467,7 +470,8 @@ def main():
         raise SystemExit("--warmup must be at least 3")
 
     from sparsely_gated_mixture_gate_b200 import synth
-    w = synth.WORKLOADS[args.workload].with_(gate_precision=1 if args.gate == "tf32x3" else 0)
+    w = (synth.WORKLOADS.get(args.workload) or synth.VARIANTS[args.workload]).with_(
+        gate_precision=1 if args.gate == "tf32x3" else 0)
     world, rank, local = dist_info()
 
     if args.impl == "reference":

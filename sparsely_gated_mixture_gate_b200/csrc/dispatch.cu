@@ -275,10 +275,27 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
     const int *idx, const float *gate, int T, int k, int n, int tpb, long long C,
     const int *base, const int *offsets, const int *ucoff, int *row_of, int *perm_token,
     int *perm_slot, float *gate_sorted, const float *x, int d, void *x_perm, void *x_shared,
-    int *shared_off) {
-  if (shared_off && blockIdx.x == 0 && threadIdx.x == 0) {
-    shared_off[0] = 0;
-    shared_off[1] = T;
+    int *shared_off, int *shared_mprefix, int4 *shared_tab1, int4 *shared_tab2, int *shared_mdone,
+    int nblk1, int nblk2) {
+  if (shared_off && blockIdx.x == 0) {
+    // the shared expert: rows 0..T-1 in token order, its tile tables and
+    // counters (one expert, mbe M-blocks; see write_tiles)
+    const int mbe = (T + kExpertBM - 1) / kExpertBM;
+    if (threadIdx.x == 0) {
+      shared_off[0] = 0;
+      shared_off[1] = T;
+      shared_mprefix[0] = 0;
+      shared_mprefix[1] = mbe;
+    }
+    for (int i = threadIdx.x; i < mbe * nblk1; i += NT) {
+      const int nbk = i / mbe, mb = i - nbk * mbe;
+      shared_tab1[i] = make_int4(0, mb * kExpertBM, min(kExpertBM, T - mb * kExpertBM), nbk | (mb << 8));
+    }
+    for (int i = threadIdx.x; i < mbe * nblk2; i += NT) {
+      const int nbk = i / mbe, mb = i - nbk * mbe;
+      shared_tab2[i] = make_int4(0, mb * kExpertBM, min(kExpertBM, T - mb * kExpertBM), nbk | (mb << 8));
+    }
+    for (int i = threadIdx.x; i <= mbe; i += NT) shared_mdone[i] = 0;
   }
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
@@ -417,7 +434,8 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
     return launch("dispatch_place", kern, grid, dim3(NT), 0, st, a.idx, a.gate, a.T, a.k, a.n, tpb,
                   C, (const int *)a.base, (const int *)a.offsets, (const int *)a.ucoff, a.row_of,
                   a.perm_token, a.perm_slot, a.gate_sorted, a.x, a.d, a.x_perm, a.x_shared,
-                  a.shared_off);
+                  a.shared_off, a.shared_mprefix, a.shared_tab1, a.shared_tab2, a.shared_mdone,
+                  a.nblk1, a.nblk2);
   };
   if (!a.x) return place(dispatch_place_kernel<false, false>);
   if (a.x_bf16) return place(dispatch_place_kernel<true, true>);

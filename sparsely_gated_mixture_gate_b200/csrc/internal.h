@@ -125,6 +125,11 @@ struct DispatchArgs {
   void *x_perm;            // [kept rows][d], bf16 (x_bf16) or fp32
   void *x_shared;          // [T][d] or nullptr: every x row again, in token order
   int *shared_off;         // with x_shared: {0, T}, the shared expert's row offsets
+  // with x_shared: the shared expert's GEMM plan (one expert of T rows), as
+  // launch_expert_plan would write it
+  int *shared_mprefix;     // [2]
+  int4 *shared_tab1, *shared_tab2;
+  int *shared_mdone;       // [ceil(T / kExpertBM) + 1]
   int d, x_bf16;
   int *status;
 };

@@ -130,6 +130,7 @@ struct Layout {
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch, ticket;
   size_t mprefix, tab1, tab2, mdone, x_perm, hid, y_perm;
   size_t x_shared, y_shared, shared_off;  // shared expert: input and output rows, {0, T}
+  size_t shared_mprefix, shared_tab1, shared_tab2, shared_mdone;  // and its GEMM plan
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
@@ -216,8 +217,14 @@ Layout make_layout(const moe_config &c) {
     L.x_shared = bp.take(esz * (size_t)T * c.d);
     L.y_shared = bp.take(esz * (size_t)T * c.d);
     L.shared_off = bp.take(8);
+    const size_t mbe = (size_t)ceil_div((int64_t)T, kExpertBM);
+    L.shared_mprefix = bp.take(8);
+    L.shared_tab1 = bp.take(16 * mbe * (size_t)ceil_div(c.f, kExpertBN));
+    L.shared_tab2 = bp.take(16 * mbe * (size_t)ceil_div(c.d, kExpertBN));
+    L.shared_mdone = bp.take(4 * (mbe + 1));
   } else {
     L.x_shared = L.y_shared = L.shared_off = 0;
+    L.shared_mprefix = L.shared_tab1 = L.shared_tab2 = L.shared_mdone = 0;
   }
   if (c.gate_precision == MOE_GATE_TF32X3) {
     const size_t rows = hier ? (T > R2 ? T : R2) : T;
@@ -457,6 +464,14 @@ int run_dispatch(const moe_config &c, const Layout &L, const int *idx, const flo
   DispatchArgs da{};
   da.x_shared = x_shared;
   da.shared_off = shared_off;
+  if (shared_off) {
+    da.shared_mprefix = at<int>(ws, L.shared_mprefix);
+    da.shared_tab1 = at<int4>(ws, L.shared_tab1);
+    da.shared_tab2 = at<int4>(ws, L.shared_tab2);
+    da.shared_mdone = at<int>(ws, L.shared_mdone);
+    da.nblk1 = (int)ceil_div(c.f, kExpertBN);
+    da.nblk2 = (int)ceil_div(c.d, kExpertBN);
+  }
   da.ticket = at<int>(ws, L.ticket);
   da.x = x;
   da.x_perm = x_perm;
@@ -718,14 +733,29 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
     MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));
     if (c.shared_expert) {
       // every token through the shared expert: one expert, rows 0..T-1 in
-      // token order; the routed launch is done with the tile tables and the
-      // hidden-layer rows by now, so they are reused
-      moe_config cs = c;
-      cs.n = 1;
-      cs.k = 1;
-      moe_expert_params es{ep->W1s, ep->b1s, ep->W2s, ep->b2s, nullptr, nullptr, nullptr, nullptr};
-      MOE_TRY(run_experts(cs, L, x_shared, shared_off, es, y_shared, ws, status, st, 0,
-                          tc ? "shared_expert_ffn_tcgen05" : "shared_expert_ffn_fp32"));
+      // token order, its plan written by the dispatch; the routed launch is
+      // done with the hidden-layer rows by now, so they are reused
+      ExpertArgs e{};
+      e.name = tc ? "shared_expert_ffn_tcgen05" : "shared_expert_ffn_fp32";
+      e.x_perm = x_shared;
+      e.offsets = shared_off;
+      e.mprefix = at<int>(ws, L.shared_mprefix);
+      e.tab1 = at<int4>(ws, L.shared_tab1);
+      e.tab2 = at<int4>(ws, L.shared_tab2);
+      e.mdone = at<int>(ws, L.shared_mdone);
+      e.plan_ready = 1;
+      e.n = 1;
+      e.d = c.d;
+      e.f = c.f;
+      e.S = c.T;
+      e.W1 = ep->W1s;
+      e.W2 = ep->W2s;
+      e.b1 = ep->b1s;
+      e.b2 = ep->b2s;
+      e.hid = at<void>(ws, L.hid);
+      e.y_perm = y_shared;
+      e.status = status;
+      MOE_TRY(tc ? launch_expert_bf16(e, st) : launch_expert_f32(e, st));
     }
     MOE_TRY(launch_combine(y_perm, c.expert_dtype == MOE_BF16, topk_gate, row_of, x,
                            c.overflow_passthrough, c.T, c.k, c.d, y, y_shared, st));
