@@ -578,6 +578,38 @@ void orc_sel_bias_update(int n, int T, int k, const int32_t *counts, float gamma
   }
 }
 
+int orc_router_stats(const orc_cfg *cfg, const orc_inputs *in, double *zsum, double *hsum)
+{
+  if (!valid_cfg(cfg)) return -1;
+  const int d = cfg->d, ng = cfg->hier_a > 0 ? cfg->hier_a : cfg->n;
+  double *c = (double *)malloc(sizeof(double) * (size_t)ng);
+  double z = 0.0, h = 0.0;
+  for (int t = 0; t < cfg->T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    for (int i = 0; i < ng; ++i) c[i] = in->bg ? (double)in->bg[i] : 0.0;
+    for (int j = 0; j < d; ++j)
+      for (int i = 0; i < ng; ++i) c[i] += (double)xt[j] * (double)in->Wg[(size_t)j * ng + i];
+    double m = c[0];
+    for (int i = 0; i < ng; ++i) {
+      z += c[i] * c[i];
+      if (c[i] > m) m = c[i];
+    }
+    /* entropy of p = softmax(c): -sum p_i log p_i with log p_i = c_i - m - log S */
+    double S = 0.0;
+    for (int i = 0; i < ng; ++i) S += exp(c[i] - m);
+    double ent = 0.0;
+    for (int i = 0; i < ng; ++i) {
+      double p = exp(c[i] - m) / S;
+      if (p > 0.0) ent -= p * (c[i] - m - log(S));
+    }
+    h += ent;
+  }
+  free(c);
+  *zsum = z;
+  *hsum = h;
+  return 0;
+}
+
 int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
 {
   if (cfg->shared_expert && (!in->W1s || !in->W2s)) return -1;
@@ -629,6 +661,13 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
   orc_balance(n, T, k, out->topk_idx, out->topk_gate, out->counts, out->load, out->prob_sum, C,
               cfg->router, cfg->w_importance, cfg->w_load, cfg->alpha, out->importance,
               out->losses);
+  out->losses[8] = out->losses[9] = 0.0;
+  if (cfg->router_stats && T > 0) {
+    double zs, hs;
+    orc_router_stats(cfg, in, &zs, &hs);
+    out->losses[8] = zs / T;
+    out->losses[9] = hs / T;
+  }
   free(ye); free(offsets); free(perm_token); free(perm_slot);
   return 0;
 }

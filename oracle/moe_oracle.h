@@ -20,7 +20,9 @@
  *  [SGMoE-xyz]   "極大規模神經網路：稀疏門控專家混合層" (xyznot.com, arXiv
  *                1701.06538), section "方法（與關鍵公式）": "Noisy Top-K 門控" and
  *                "負載平衡損失".
- *  [MoE-intro]   "MoE (Mixture-of-Experts) 算法介绍" (wkbse.com), "工作流程".
+ *  [MoE-intro]   "MoE (Mixture-of-Experts) 算法介绍" (wkbse.com), "工作流程";
+ *                "第三部分：MoE 的训练挑战与解决方案" (router z-loss, gate
+ *                entropy loss).
  *  [MoE-deep]    "MoE 稀疏架构深度解析" (tufusi.com), §3.1 核心架构,
  *                §3.2 负载均衡问题, §5.2 DeepSeekMoE 的细粒度设计 (shared
  *                expert), §6.2 DeepSeek-V3 的 MoE 配置 (sigmoid scores
@@ -62,6 +64,7 @@ typedef struct {
   int expert_bf16;          /* 1: expert weights and activations are bf16         */
   double w_importance, w_load, alpha;
   int shared_expert;        /* 1: y also gets one always-active expert, weight 1 */
+  int router_stats;         /* 1: losses[8], [9] get the router z-loss and entropy */
 } orc_cfg;
 
 /* ---- noise ------------------------------------------------------------ */
@@ -136,7 +139,7 @@ typedef struct {
   double *prob_sum;     /* [n]   sum over tokens of the router softmax (router 1) */
   int32_t *counts;      /* [n]                                      */
   int32_t *row_of;      /* [T][k]                                   */
-  double *losses;       /* [8]   see orc_forward                    */
+  double *losses;       /* [10]  see orc_forward                    */
   float *near_tie;      /* [T]   H_(k) - H_(k+1) of the deciding gate, or NULL */
 } orc_outputs;
 
@@ -161,7 +164,16 @@ void orc_balance(int n, int T, int k, const int32_t *topk_idx, const double *top
                  int64_t C, int router, double w_importance, double w_load, double alpha,
                  double *importance, double *losses);
 
-/* Returns 0 on success, -1 on an invalid configuration. */
+/* Router statistics of the flat (or primary) gate, [MoE-intro] 第三部分:
+ * *zsum = sum over tokens of the squared L2 norm of the clean logits
+ * h = x W_g + b_g ("Router Z-loss" penalises the L2 norm of the logits before
+ * the softmax); *hsum = sum over tokens of the entropy of softmax(h) over all
+ * experts (the "gate entropy loss" rewards a high entropy).  0 or -1. */
+int orc_router_stats(const orc_cfg *cfg, const orc_inputs *in, double *zsum, double *hsum);
+
+/* Returns 0 on success, -1 on an invalid configuration.  losses [10]: [0..7]
+ * as orc_balance; with router_stats, [8] = zsum / T and [9] = hsum / T of
+ * orc_router_stats (else 0). */
 int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
 
 #ifdef __cplusplus

@@ -37,7 +37,7 @@ class OrcCfg(C.Structure):
         ("router", C.c_int), ("noise", C.c_int), ("seed", C.c_uint64),
         ("capacity_factor", C.c_double), ("passthrough", C.c_int), ("expert_bf16", C.c_int),
         ("w_importance", C.c_double), ("w_load", C.c_double), ("alpha", C.c_double),
-        ("shared_expert", C.c_int),
+        ("shared_expert", C.c_int), ("router_stats", C.c_int),
     ]
 
 
@@ -84,6 +84,8 @@ def lib():
         L.orc_gate_row.argtypes = [i32, i32, i32, i32, i32, C.c_uint64, u32, u32,
                                    vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.orc_sel_bias_update.argtypes = [i32, i32, i32, vp, C.c_float, vp]
+        L.orc_router_stats.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, vp]
+        L.orc_router_stats.restype = i32
         L.orc_load_row.argtypes = [i32, i32, i32, vp, vp, vp, vp]
         L.orc_dispatch.argtypes = [i32, i32, i32, C.c_int64, vp, vp, vp, vp, vp, vp, vp]
         L.orc_expert_row.argtypes = [i32, i32, i32, vp, vp, vp, vp, vp, vp]
@@ -211,13 +213,13 @@ def expert_row(x, W1, b1, W2, b2, bf16: bool) -> np.ndarray:
 # ---------------------------------------------------------------- forward
 _CFG_KEYS = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router", "noise",
              "seed", "capacity_factor", "passthrough", "expert_bf16", "w_importance", "w_load", "alpha",
-             "shared_expert")
+             "shared_expert", "router_stats")
 
 
 def make_cfg(**kw) -> OrcCfg:
     base = dict(hier_a=0, hier_b=0, hier_k1=0, hier_k2=0, router=0, noise=1, seed=0,
                 capacity_factor=0.0, passthrough=0, expert_bf16=0, w_importance=0.1,
-                w_load=0.1, alpha=0.01, shared_expert=0)
+                w_load=0.1, alpha=0.01, shared_expert=0, router_stats=0)
     base.update({k: v for k, v in kw.items() if k in _CFG_KEYS})
     return OrcCfg(**{k: base[k] for k in _CFG_KEYS})
 
@@ -266,6 +268,17 @@ def gate_tokens(cfg: dict, inp: dict, tokens) -> dict:
     return out
 
 
+def router_stats(cfg: dict, inp: dict):
+    """(sum of squared logit norms, sum of softmax entropies) over the tokens
+    of the flat / primary gate."""
+    oc = make_cfg(**cfg)
+    keep, ins = _inputs(oc, inp)
+    z = C.c_double(); h = C.c_double()
+    if lib().orc_router_stats(C.byref(oc), C.byref(ins), C.byref(z), C.byref(h)) != 0:
+        raise ValueError(f"oracle rejected the configuration {cfg}")
+    return z.value, h.value
+
+
 def combine(Y, gate, row_of, x=None, passthrough=False) -> np.ndarray:
     Y = _c(Y, np.float64); gate = _c(gate, np.float64); row_of = _c(row_of, np.int32)
     T, k = row_of.shape
@@ -298,7 +311,7 @@ def forward(cfg: dict, inp: dict) -> dict:
     out = dict(y=np.zeros((T, d)), topk_idx=np.zeros((T, k), np.int32), topk_gate=np.zeros((T, k)),
                importance=np.zeros(n), load=np.zeros(n), prob_sum=np.zeros(n),
                counts=np.zeros(n, np.int32), row_of=np.zeros((T, k), np.int32),
-               losses=np.zeros(8), near_tie=np.zeros(T, np.float32))
+               losses=np.zeros(10), near_tie=np.zeros(T, np.float32))
     outs = OrcOutputs(**{name: _p(a) for name, a in out.items()})
     rc = lib().orc_forward(C.byref(oc), C.byref(ins), C.byref(outs))
     if rc != 0:
