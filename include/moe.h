@@ -103,6 +103,9 @@ enum {
  *   ([MoE-deep] §5.2, §6.2: y = E_shared(x) + sum_j g_j E_j(x)); a token whose
  *   routed slots all overflowed keeps it (pass-through replaces only the
  *   routed sum).  Only moe_forward evaluates it.
+ *   router_stats: 1 makes moe_forward report the router z-loss and the gate
+ *   entropy ([MoE-intro] "第三部分：MoE 的训练挑战与解决方案") in losses[8], [9]
+ *   over the flat (or primary) gate's clean logits h = x W_g + b_g.
  *   noise: 1 adds StandardNormal() * Softplus(x W_noise); the deviate for
  *   (seed, token t, expert i, gate g) comes from Philox4x32-10 with key
  *   (seed lo, seed hi) and counter (t, i/4, g, 0): words 0,1 give the cosine
@@ -129,6 +132,7 @@ typedef struct moe_config {
   float w_importance, w_load, alpha_aux;
   int32_t gate_precision;     /* MOE_GATE_FP32 or MOE_GATE_TF32X3 */
   int32_t shared_expert;      /* 0 or 1 */
+  int32_t router_stats;       /* 1: moe_forward reports losses[8], [9] */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
@@ -259,7 +263,7 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm, const float *
 
 /* Balancing statistics ([SGMoE-xyz] "負載平衡損失"; [MoE-deep] §3.2).
  * importance [n]: Importance(X)_i = sum_x G(x)_i.
- * losses [8]:
+ * losses [10]:
  *   [0] L_importance = w_importance * CV(Importance)^2
  *   [1] L_load       = w_load * CV(load)^2
  *   [2] N * sum_i f_i P_i  (Switch: f_i = counts_i / T before the capacity
@@ -267,6 +271,13 @@ MOE_API int moe_combine(const moe_config *cfg, const void *y_perm, const float *
  *   [3] alpha_aux * [2]
  *   [4] dropped slots / (T*k),   [5] CV(Importance)^2,   [6] CV(load)^2,
  *   [7] dropped slots
+ *   [8] router z-loss: mean over tokens of |h|^2, the squared L2 norm of the
+ *       clean logits (our reading of "penalise the L2 norm of the logits
+ *       before the softmax"); [9] mean over tokens of the entropy of
+ *       softmax(h) over all experts (a statistic; the "gate entropy loss"
+ *       rewards it, so its weight is negative).  Both come from moe_forward
+ *       with router_stats = 1 and are 0 otherwise (moe_balance_losses always
+ *       writes 0 there).
  * CV^2 is the population variance over the squared mean (0 for a zero
  * mean), evaluated in fp64.  counts and load come from moe_dispatch /
  * moe_gate; prob_sum may be NULL for the noisy gate. */
@@ -291,7 +302,7 @@ MOE_API int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, fl
 /* The whole layer on one stream: gate, dispatch, experts (and the shared
  * expert when cfg->shared_expert), combine and the balancing statistics,
  * every intermediate in ws.  Outputs as the step calls above: y [T][d],
- * topk_idx, topk_gate [T][k], importance, load [n], counts [n], losses [8]. */
+ * topk_idx, topk_gate [T][k], importance, load [n], counts [n], losses [10]. */
 MOE_API int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
                 const moe_expert_params *ep, float *y, int32_t *topk_idx,
                 float *topk_gate, float *importance, float *load, int32_t *counts,

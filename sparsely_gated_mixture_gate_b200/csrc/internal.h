@@ -90,6 +90,8 @@ struct RouteArgs {
   float *load_part;        // [tiles][nb]
   float *psum_part;        // [tiles][nb] or nullptr
   const float *sel_bias;   // sigmoid router: [nb] selection bias, or nullptr
+  float *stats_part;       // [tiles][2] or nullptr: per tile, sum over rows of |c|^2
+                           // and of the entropy of softmax(c)
   int *status;
 };
 int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st);
@@ -172,8 +174,11 @@ int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, 
 
 int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
                       cudaStream_t st);
+// rstats [2] or nullptr: the router statistics' sums over tokens (losses[8],
+// [9] become their means; 0 without them)
 int launch_losses(const float *importance, const float *load, const int *counts,
                   const float *prob_sum, int n, int T, int k, int64_t C, int router,
-                  float w_imp, float w_load, float alpha, float *losses, cudaStream_t st);
+                  float w_imp, float w_load, float alpha, const float *rstats, float *losses,
+                  cudaStream_t st);
 
 }  // namespace moe

@@ -125,6 +125,7 @@ namespace {
 
 struct Layout {
   size_t c, s, load_part, psum_part, prob_sum;
+  size_t stats_part, rstats;  // router statistics: per-tile sums, their totals
   size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
   size_t hist, base, ucoff, offsets, perm_token, row_of, gate_sorted, counts_scratch, ticket;
@@ -171,6 +172,8 @@ Layout make_layout(const moe_config &c) {
   L.load_part = bp.take(4 * (lp1 > lp2 ? lp1 : lp2));
   L.psum_part = bp.take(c.router == MOE_ROUTER_SWITCH ? 4 * (size_t)L.tiles1 * n : 0);
   L.prob_sum = bp.take(4 * n);
+  L.stats_part = bp.take(c.router_stats ? 8 * (size_t)L.tiles1 : 0);
+  L.rstats = bp.take(c.router_stats ? 8 : 0);
   L.B = (int)ceil_div(c.T, dispatch_tokens_per_block(c.T));
   if (hier) {
     const size_t a = (size_t)c.hier_a, k1 = (size_t)c.hier_k1;
@@ -355,6 +358,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.RT = L.RT1;
   r.load_part = at<float>(ws, L.load_part);
   r.sel_bias = (!hier && c.router == MOE_ROUTER_SIGMOID) ? gp.sel_bias : nullptr;
+  r.stats_part = c.router_stats ? at<float>(ws, L.stats_part) : nullptr;  // flat / primary rows
   r.status = status;
   if (!hier) {
     r.k = c.k;
@@ -370,6 +374,8 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
       rs = side->s;
     }
     MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, c.n, load, rs));
+    if (r.stats_part)
+      MOE_TRY(launch_route_reduce(r.stats_part, nullptr, 1, L.tiles1, 2, at<float>(ws, L.rstats), rs));
     if (sw) {
       float *ps = prob_sum ? prob_sum : at<float>(ws, L.prob_sum);
       MOE_TRY(launch_route_reduce(r.psum_part, nullptr, 1, L.tiles1, c.n, ps, rs));
@@ -389,6 +395,8 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.K = k1;
   MOE_TRY(launch_route(r, L.tiles1, st));
   MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, a, at<float>(ws, L.load_p), st));
+  if (r.stats_part)
+    MOE_TRY(launch_route_reduce(r.stats_part, nullptr, 1, L.tiles1, 2, at<float>(ws, L.rstats), st));
 
   // ---- tokens grouped by their kept groups (stable), tile prefixes per group
   DispatchArgs da{};
@@ -428,6 +436,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   MOE_TRY(gate_gemm(g2, (int)ceil_div(R2, kGateBM) + a));
 
   RouteArgs r2 = r;
+  r2.stats_part = nullptr;  // the statistics cover the primary gate only
   r2.R = R2;
   r2.nb = b;
   r2.k = k2;
@@ -581,6 +590,7 @@ int moe_validate(const moe_config *c) {
     return MOE_EINVAL;
   if (c->router == MOE_ROUTER_SIGMOID && (c->noise || c->hier_a)) return MOE_EINVAL;
   if (c->shared_expert != 0 && c->shared_expert != 1) return MOE_EINVAL;
+  if (c->router_stats != 0 && c->router_stats != 1) return MOE_EINVAL;
   if (c->noise != 0 && c->noise != 1) return MOE_EINVAL;
   if (c->expert_dtype != MOE_F32 && c->expert_dtype != MOE_BF16) return MOE_EINVAL;
   if (c->overflow_passthrough != 0 && c->overflow_passthrough != 1) return MOE_EINVAL;
@@ -689,7 +699,7 @@ int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx, const flo
   MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
                             st));
   return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, capacity_of(c), c.router,
-                       c.w_importance, c.w_load, c.alpha_aux, losses, st);
+                       c.w_importance, c.w_load, c.alpha_aux, nullptr, losses, st);
 }
 
 int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
@@ -728,7 +738,8 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
   MOE_TRY(launch_importance(at<float>(ws, L.gate_sorted), at<int>(ws, L.ucoff), c.n, importance,
                             side->s));
   MOE_TRY(launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, C, c.router,
-                        c.w_importance, c.w_load, c.alpha_aux, losses, side->s));
+                        c.w_importance, c.w_load, c.alpha_aux,
+                        c.router_stats ? at<float>(ws, L.rstats) : nullptr, losses, side->s));
   if (c.T > 0) {
     MOE_TRY(run_experts(c, L, x_perm, offsets, *ep, y_perm, ws, status, st, tc ? 1 : 0));
     if (c.shared_expert) {

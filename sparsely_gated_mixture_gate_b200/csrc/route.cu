@@ -10,6 +10,8 @@
 //   goes to argmax p with gate p_argmax; sum_t p_i is accumulated too.
 //   Sigmoid router ([MoE-deep] §6.2, §6.3): H_i = c_i + b_i with the selection
 //   bias b, top-k of H, gates Sigmoid(c_i) / sum of Sigmoid(c_j) over the kept.
+//   Router statistics ([MoE-intro] 第三部分, optional): per row |c|^2 and the
+//   entropy of softmax(c), summed over the tile's rows in a fixed order.
 // Pass 1, one warp per row: each lane scans column quads 4m .. 4m+3 (16-byte
 // loads, one Philox call per quad), keeps a sorted top-(k+1) list in
 // registers, and the warp merges the 32 lists with shuffles; the row's kept
@@ -56,7 +58,8 @@ __device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
 
 // K1 = k + 1; MAXQ = column quads per thread (nb <= MAXQ * 4 * 256); SW =
 // Switch router (probability sums kept).
-template <int K1, int MAXQ, bool SW>
+// ST = router statistics (stats_part written).
+template <int K1, int MAXQ, bool SW, bool ST>
 __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
   constexpr int KM = K1 - 1;  // k
   constexpr int PQ = SW ? MAXQ : 1;
@@ -109,6 +112,8 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) pacc[u][j] = 0.f;
 
+  constexpr bool stats = ST;
+  float rz = 0.f, rh = 0.f;  // lane 0: this warp's rows' |c|^2 and entropies
   const int nwords = (nb + 31) >> 5;
   for (int rb = row0; rb < row_end; rb += NW) {
     // ================= pass 1: routing of row rb + w (warp per row)
@@ -263,6 +268,42 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
         sm_s[w][0] = M;
         sm_s[w][1] = SE;
       }
+      if (stats) {
+        // router statistics of the row, a second pass over its clean logits
+        // (cache hits): sum c^2 and an online softmax with S = sum e^(c-m),
+        // Q = sum e^(c-m) (c-m), the entropy being log S - Q/S
+        float zs = 0.f, sm = -INFINITY, ss = 0.f, sq = 0.f;
+        for (int i = lane; i < nb; i += 32) {
+          const float v = crow[i];
+          zs = fmaf(v, v, zs);
+          if (v > sm) {  // rescale to the new maximum
+            const float r = ss > 0.f ? expf(sm - v) : 0.f;
+            sq = ss > 0.f ? r * (sq + ss * (sm - v)) : 0.f;
+            ss *= r;
+            sm = v;
+          }
+          const float e = expf(v - sm);
+          ss += e;
+          sq = fmaf(e, v - sm, sq);
+        }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+          zs += __shfl_xor_sync(0xffffffffu, zs, off);
+          const float om = __shfl_xor_sync(0xffffffffu, sm, off);
+          const float os = __shfl_xor_sync(0xffffffffu, ss, off);
+          const float oq = __shfl_xor_sync(0xffffffffu, sq, off);
+          const float m2 = fmaxf(sm, om);
+          const float r1 = ss > 0.f ? expf(sm - m2) : 0.f, r2 = os > 0.f ? expf(om - m2) : 0.f;
+          sq = (ss > 0.f ? r1 * (sq + ss * (sm - m2)) : 0.f) +
+               (os > 0.f ? r2 * (oq + os * (om - m2)) : 0.f);
+          ss = ss * r1 + os * r2;
+          sm = m2;
+        }
+        if (lane == 0) {
+          rz += zs;
+          rh += logf(ss) - sq / ss;
+        }
+      }
     }
     __syncthreads();
 
@@ -316,6 +357,25 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
     __syncthreads();  // the next block of rows reuses kept_s / thr_s / sm_s
   }
   if (bad && a.status) atomicOr(a.status, MOE_STATUS_NONFINITE);
+
+  if (stats) {  // the tile's statistics: warps added in warp order
+    __shared__ float st_s[NW][2];
+    if (lane == 0) {
+      st_s[w][0] = rz;
+      st_s[w][1] = rh;
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      float z = 0.f, hh = 0.f;
+#pragma unroll
+      for (int q = 0; q < NW; ++q) {
+        z += st_s[q][0];
+        hh += st_s[q][1];
+      }
+      a.stats_part[(size_t)tile * 2] = z;
+      a.stats_part[(size_t)tile * 2 + 1] = hh;
+    }
+  }
 
   // ---- the tile's column sums: row groups added in group order
   float *outp = a.load_part + (size_t)tile * nb;
@@ -399,13 +459,16 @@ int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st) {
     return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), 0, st, a);
   };
   const bool wide = a.nb > 4 * 4 * NW * 32;  // more than 4096 columns
+  const bool st_on = a.stats_part != nullptr;
   if (a.router == MOE_ROUTER_SWITCH) {
     if (a.k != 1 || wide) return MOE_EINVAL;
-    return go(route_kernel<2, 4, true>);
+    return st_on ? go(route_kernel<2, 4, true, true>) : go(route_kernel<2, 4, true, false>);
   }
-#define MOE_ROUTE_CASE(K1)                                                      \
-  case K1:                                                                      \
-    return wide ? go(route_kernel<K1, 8, false>) : go(route_kernel<K1, 4, false>);
+#define MOE_ROUTE_CASE(K1)                                                                   \
+  case K1:                                                                                   \
+    if (st_on)                                                                               \
+      return wide ? go(route_kernel<K1, 8, false, true>) : go(route_kernel<K1, 4, false, true>); \
+    return wide ? go(route_kernel<K1, 8, false, false>) : go(route_kernel<K1, 4, false, false>);
   switch (a.k + 1) {
     MOE_ROUTE_CASE(2)
     MOE_ROUTE_CASE(3)

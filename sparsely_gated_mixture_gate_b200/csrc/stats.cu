@@ -63,7 +63,7 @@ __global__ void __launch_bounds__(LNT) losses_kernel(const float *importance, co
                                                      const int *counts, const float *prob_sum,
                                                      int n, int T, int k, long long C, int router,
                                                      float w_imp, float w_load, float alpha,
-                                                     float *losses) {
+                                                     const float *rstats, float *losses) {
   __shared__ double sh[LNT / 32];
   const double cv_imp = cv2(importance, n, sh);
   const double cv_load = cv2(load, n, sh);
@@ -86,6 +86,9 @@ __global__ void __launch_bounds__(LNT) losses_kernel(const float *importance, co
     losses[5] = (float)cv_imp;
     losses[6] = (float)cv_load;
     losses[7] = (float)dropped;
+    // router statistics: means over tokens of |c|^2 and of the softmax entropy
+    losses[8] = rstats && T > 0 ? (float)((double)rstats[0] / T) : 0.f;
+    losses[9] = rstats && T > 0 ? (float)((double)rstats[1] / T) : 0.f;
   }
 }
 
@@ -117,9 +120,10 @@ int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *
 
 int launch_losses(const float *importance, const float *load, const int *counts,
                   const float *prob_sum, int n, int T, int k, int64_t C, int router, float w_imp,
-                  float w_load, float alpha, float *losses, cudaStream_t st) {
+                  float w_load, float alpha, const float *rstats, float *losses, cudaStream_t st) {
   return launch("balance_losses", losses_kernel, dim3(1), dim3(LNT), 0, st, importance, load,
-                counts, prob_sum, n, T, k, (long long)C, router, w_imp, w_load, alpha, losses);
+                counts, prob_sum, n, T, k, (long long)C, router, w_imp, w_load, alpha, rstats,
+                losses);
 }
 
 }  // namespace moe

@@ -49,6 +49,7 @@ class Config:
     alpha: float = 0.01
     gate_precision: int = 0   # 0: fp32 multiply-adds, 1: tensor cores, 3-pass TF32 split
     shared_expert: int = 0    # 1: one always-active expert (W1s, b1s, W2s, b2s) in forward
+    router_stats: int = 0     # 1: forward reports the router z-loss and entropy (losses[8:10])
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -65,7 +66,8 @@ class Config:
                           seed=self.seed, capacity_factor=float(self.capacity_factor),
                           overflow_passthrough=self.passthrough, w_importance=self.w_importance,
                           w_load=self.w_load, alpha_aux=self.alpha,
-                          gate_precision=self.gate_precision, shared_expert=self.shared_expert)
+                          gate_precision=self.gate_precision, shared_expert=self.shared_expert,
+                          router_stats=self.router_stats)
 
     @property
     def expert_dtype(self):
@@ -250,7 +252,7 @@ def combine(cfg: Config, y_perm: torch.Tensor, topk_gate: torch.Tensor, row_of: 
 def balance_losses(cfg: Config, topk_idx, topk_gate, counts, load, prob_sum=None, ws=None, status=None):
     dev = topk_idx.device
     importance = torch.empty(cfg.n, dtype=torch.float32, device=dev)
-    losses = torch.empty(8, dtype=torch.float32, device=dev)
+    losses = torch.empty(10, dtype=torch.float32, device=dev)
     ws = workspace(cfg, dev) if ws is None else ws
     status = new_status(dev) if status is None else status
     c = cfg.c()
@@ -285,7 +287,7 @@ class MoELayer:
         self.importance = torch.empty(n, dtype=torch.float32, device=dev)
         self.load = torch.empty(n, dtype=torch.float32, device=dev)
         self.counts = torch.empty(n, dtype=torch.int32, device=dev)
-        self.losses = torch.empty(8, dtype=torch.float32, device=dev)
+        self.losses = torch.empty(10, dtype=torch.float32, device=dev)
 
     def forward_(self, x: torch.Tensor, stream=None, y: Optional[torch.Tensor] = None,
                  losses: Optional[torch.Tensor] = None):

@@ -53,6 +53,7 @@ class Workload:
     gate_precision: int = 0     # library option; the oracle is always fp64
     shared_expert: int = 0      # 1: one always-active expert added to every token
     sel_bias_std: float = 0.0   # sigmoid router: spread of the selection bias
+    router_stats: int = 0       # 1: the router z-loss and entropy are reported too
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -65,7 +66,7 @@ class Workload:
     def cfg(self) -> dict:
         keys = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router",
                 "noise", "expert_bf16", "capacity_factor", "passthrough", "seed",
-                "w_importance", "w_load", "alpha", "shared_expert")
+                "w_importance", "w_load", "alpha", "shared_expert", "router_stats")
         return {k: getattr(self, k) for k in keys}
 
 

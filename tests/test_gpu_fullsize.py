@@ -138,7 +138,7 @@ def test_fullsize(orc, name, gp):
         imp = out["importance"].numpy()
         assert np.allclose(imp[~touched], imp_ref[~touched], rtol=1e-5, atol=1e-6)
         if near == 0:
-            assert np.allclose(losses, losses_ref, rtol=1e-5, atol=1e-7)
+            assert np.allclose(losses[:8], losses_ref, rtol=1e-5, atol=1e-7)
 
     # ---- the layer output of the sampled tokens
     kept_all = None
