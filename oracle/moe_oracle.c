@@ -671,3 +671,296 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out)
   free(ye); free(offsets); free(perm_token); free(perm_slot);
   return 0;
 }
+
+/* ======================================================================= */
+/* Backward pass                                                            */
+/* ======================================================================= */
+/*
+ * The pages give no backward formulas; they say which paths carry a
+ * gradient.  The kept gates are a smooth function of the logits, so the
+ * gradient reaches the gate network through them ([SGMoE-xyz] 常見問題);
+ * KeepTopK gives the experts it drops none ([SGMoE-note] 缺点与局限性); the
+ * noise lets the load loss reach the gate through Phi ([SGMoE-note] Noisy
+ * Top-K Gating).  orc_backward is the chain rule of orc_forward, taken in the
+ * reverse order of its steps: combine, experts, dispatch, gate.
+ *
+ * Mixed precision (expert_bf16): the kernels keep every expert-side
+ * activation gradient in bf16 and accumulate in fp32, so the oracle rounds
+ * where they store: the gradient reaching an expert row, g * dy (the product
+ * taken in fp32, as g is an fp32 output of the gate); the hidden-layer
+ * gradient after the ReLU mask; the input-row gradient of each expert.  The
+ * combine's gate gradient uses the expert output rounded to bf16, the value
+ * the combine summed.  Everything else is fp64.
+ */
+
+void orc_cv2_grad(const double *v, int n, double *g)
+{
+  /* CV^2 = var / mean^2 with var = sum (v_i - mean)^2 / n:
+   * d var / d v_i = 2 (v_i - mean) / n, d mean / d v_i = 1 / n, so
+   * d CV^2 / d v_i = 2 / (n mean^2) * ((v_i - mean) - var / mean). */
+  double sum = 0.0;
+  for (int i = 0; i < n; ++i) sum += v[i];
+  double mean = n > 0 ? sum / (double)n : 0.0;
+  if (mean == 0.0) {
+    for (int i = 0; i < n; ++i) g[i] = 0.0;
+    return;
+  }
+  double ss = 0.0;
+  for (int i = 0; i < n; ++i) ss += (v[i] - mean) * (v[i] - mean);
+  double var = ss / (double)n;
+  for (int i = 0; i < n; ++i)
+    g[i] = 2.0 / ((double)n * mean * mean) * ((v[i] - mean) - var / mean);
+}
+
+static double wval(const void *W, int bf16, size_t i)
+{
+  return bf16 ? bf16_bits_to_double(((const uint16_t *)W)[i]) : (double)((const float *)W)[i];
+}
+
+static double rnd(int bf16, double v)
+{
+  return bf16 ? (double)orc_bf16_round((float)v) : v;
+}
+
+/* One expert on one row, forward and backward.  dyr: the gradient reaching
+ * the layer output row; gate: the weight of this expert's output in it (1 for
+ * the shared expert).  Adds to dW1 [f][d], db1 [f], dW2 [d][f], db2 [d] and
+ * dxr [d]; returns <dyr, E(x)> (the gradient of the gate). */
+static double expert_row_bwd(int d, int f, int bf16, const float *x, const void *W1,
+                             const float *b1, const void *W2, const float *b2, double gate,
+                             const float *dyr, double *dW1, double *db1, double *dW2, double *db2,
+                             double *dxr)
+{
+  double *xv = (double *)malloc(sizeof(double) * (size_t)d);
+  double *h = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dh = (double *)malloc(sizeof(double) * (size_t)f);
+  double *dyp = (double *)malloc(sizeof(double) * (size_t)d);
+  for (int q = 0; q < d; ++q) xv[q] = rnd(bf16, (double)x[q]);
+  /* forward: h = ReLU(W1 x + b1), E = W2 h + b2 */
+  for (int j = 0; j < f; ++j) {
+    double a = b1 ? (double)b1[j] : 0.0;
+    for (int q = 0; q < d; ++q) a += wval(W1, bf16, (size_t)j * d + q) * xv[q];
+    h[j] = rnd(bf16, a > 0.0 ? a : 0.0);
+  }
+  double dgate = 0.0;
+  for (int q = 0; q < d; ++q) {
+    double e = b2 ? (double)b2[q] : 0.0;
+    for (int j = 0; j < f; ++j) e += wval(W2, bf16, (size_t)q * f + j) * h[j];
+    dgate += (double)dyr[q] * rnd(bf16, e);
+  }
+  /* dE = gate * dy */
+  for (int q = 0; q < d; ++q)
+    dyp[q] = bf16 ? (double)orc_bf16_round((float)gate * dyr[q]) : gate * (double)dyr[q];
+  /* E = W2 h + b2: dW2 += dE h^T, db2 += dE, dh = W2^T dE */
+  for (int q = 0; q < d; ++q) {
+    if (db2) db2[q] += dyp[q];
+    for (int j = 0; j < f; ++j) dW2[(size_t)q * f + j] += dyp[q] * h[j];
+  }
+  for (int j = 0; j < f; ++j) {
+    double acc = 0.0;
+    for (int q = 0; q < d; ++q) acc += wval(W2, bf16, (size_t)q * f + j) * dyp[q];
+    /* ReLU passes the gradient where its output is positive */
+    dh[j] = rnd(bf16, h[j] > 0.0 ? acc : 0.0);
+  }
+  /* a = W1 x + b1: dW1 += dh x^T, db1 += dh, dx = W1^T dh */
+  for (int j = 0; j < f; ++j) {
+    if (db1) db1[j] += dh[j];
+    for (int q = 0; q < d; ++q) dW1[(size_t)j * d + q] += dh[j] * xv[q];
+  }
+  for (int q = 0; q < d; ++q) {
+    double acc = 0.0;
+    for (int j = 0; j < f; ++j) acc += wval(W1, bf16, (size_t)j * d + q) * dh[j];
+    dxr[q] += rnd(bf16, acc);
+  }
+  free(xv); free(h); free(dh); free(dyp);
+  return dgate;
+}
+
+int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g)
+{
+  if (!valid_cfg(cfg) || cfg->hier_a) return -1;
+  if (cfg->shared_expert && (!in->W1s || !in->W2s)) return -1;
+  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f, bf16 = cfg->expert_bf16;
+  const int noise = cfg->noise;
+  const size_t esz = bf16 ? 2 : 4;
+  const size_t S = (size_t)T * k;
+
+  /* ---- forward state: routing, dispatch, importance, load */
+  int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  double *gate = (double *)malloc(sizeof(double) * (S ? S : 1));
+  double *load = (double *)malloc(sizeof(double) * (size_t)n);
+  double *psum = (double *)malloc(sizeof(double) * (size_t)n);
+  double *imp = (double *)calloc((size_t)n, sizeof(double));
+  int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+  int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
+  int32_t *ptok = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  int32_t *pslot = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  int32_t *row_of = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  orc_gate_batch(cfg, in, idx, gate, load, psum, NULL);
+  const int64_t C = orc_capacity(T, k, n, cfg->capacity_factor);
+  orc_dispatch(T, k, n, C, idx, counts, offsets, ptok, pslot, row_of, NULL);
+  for (size_t p = 0; p < S; ++p) imp[idx[p]] += gate[p];
+
+  /* ---- the losses' gradients with respect to Importance and Load */
+  double *lam_imp = (double *)malloc(sizeof(double) * (size_t)n);
+  double *lam_load = (double *)malloc(sizeof(double) * (size_t)n);
+  orc_cv2_grad(imp, n, lam_imp);
+  orc_cv2_grad(load, n, lam_load);
+  for (int i = 0; i < n; ++i) {
+    lam_imp[i] *= cfg->w_importance;
+    lam_load[i] *= cfg->w_load;
+  }
+
+  /* ---- zero the outputs */
+#define ZERO(ptr, cnt) do { if (ptr) memset((ptr), 0, sizeof(double) * (size_t)(cnt)); } while (0)
+  ZERO(g->dx, (size_t)T * d);
+  ZERO(g->dWg, (size_t)d * n); ZERO(g->dbg, n); ZERO(g->dWn, (size_t)d * n);
+  ZERO(g->dW1, (size_t)n * f * d); ZERO(g->db1, (size_t)n * f);
+  ZERO(g->dW2, (size_t)n * d * f); ZERO(g->db2, (size_t)n * d);
+  ZERO(g->dW1s, (size_t)f * d); ZERO(g->db1s, f); ZERO(g->dW2s, (size_t)d * f); ZERO(g->db2s, d);
+  ZERO(g->dgate, S); ZERO(g->dlogits, (size_t)T * n); ZERO(g->dnoise, (size_t)T * n);
+#undef ZERO
+  double *dW1 = g->dW1 ? g->dW1 : (double *)calloc((size_t)n * f * d, sizeof(double));
+  double *dW2 = g->dW2 ? g->dW2 : (double *)calloc((size_t)n * d * f, sizeof(double));
+  double *dW1s = NULL, *dW2s = NULL;
+  if (cfg->shared_expert) {
+    dW1s = g->dW1s ? g->dW1s : (double *)calloc((size_t)f * d, sizeof(double));
+    dW2s = g->dW2s ? g->dW2s : (double *)calloc((size_t)d * f, sizeof(double));
+  }
+  double *dx = g->dx;
+
+  /* ---- combine and experts: y_t = sum_j g_tj E_{e_tj}(x_t) (+ E_shared(x_t)) */
+  double *dgate = (double *)calloc(S ? S : 1, sizeof(double));
+  for (int t = 0; t < T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    const float *dyt = dy + (size_t)t * d;
+    double *dxt = dx + (size_t)t * d;
+    int kept = 0;
+    for (int j = 0; j < k; ++j) {
+      size_t pj = (size_t)t * k + j;
+      if (row_of[pj] < 0) continue; /* dropped: contributes nothing */
+      kept++;
+      int e = idx[pj];
+      dgate[pj] = expert_row_bwd(
+          d, f, bf16, xt, (const char *)in->W1 + (size_t)e * f * d * esz,
+          in->b1 ? in->b1 + (size_t)e * f : NULL, (const char *)in->W2 + (size_t)e * d * f * esz,
+          in->b2 ? in->b2 + (size_t)e * d : NULL, gate[pj], dyt, dW1 + (size_t)e * f * d,
+          g->db1 ? g->db1 + (size_t)e * f : NULL, dW2 + (size_t)e * d * f,
+          g->db2 ? g->db2 + (size_t)e * d : NULL, dxt);
+    }
+    if (kept == 0 && cfg->passthrough)
+      for (int q = 0; q < d; ++q) dxt[q] += (double)dyt[q]; /* y = x */
+    if (cfg->shared_expert)
+      expert_row_bwd(d, f, bf16, xt, in->W1s, in->b1s, in->W2s, in->b2s, 1.0, dyt, dW1s, g->db1s,
+                     dW2s, g->db2s, dxt);
+  }
+  if (g->dgate) memcpy(g->dgate, dgate, sizeof(double) * S);
+
+  /* ---- gate */
+  double *c = (double *)malloc(sizeof(double) * (size_t)n);
+  double *s = (double *)malloc(sizeof(double) * (size_t)n);
+  double *pr = (double *)malloc(sizeof(double) * (size_t)n);
+  double *gk = (double *)malloc(sizeof(double) * (size_t)k);
+  double *dG = (double *)malloc(sizeof(double) * (size_t)k);
+  double *dc = (double *)malloc(sizeof(double) * (size_t)n);
+  double *ds = (double *)malloc(sizeof(double) * (size_t)n);
+  double *dH = (double *)malloc(sizeof(double) * (size_t)n);
+  double *zp = (double *)malloc(sizeof(double) * (size_t)n);
+  float *H = (float *)malloc(sizeof(float) * (size_t)n);
+  int *order = (int *)malloc(sizeof(int) * (size_t)n);
+  int *rank = (int *)malloc(sizeof(int) * (size_t)n);
+  for (int t = 0; t < T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    orc_gate_row(d, n, k, cfg->router, noise, cfg->seed, (uint32_t)t, 0u, xt, in->Wg, in->bg,
+                 in->Wn, c, s, H, order, gk, pr, in->sel_bias);
+    for (int r = 0; r < n; ++r) rank[order[r]] = r;
+    for (int i = 0; i < n; ++i) dc[i] = ds[i] = dH[i] = 0.0;
+    /* dL/dG of each kept gate: from the combine, and from Importance (the sum
+     * of the gates, dropped slots included) */
+    for (int j = 0; j < k; ++j) dG[j] = dgate[(size_t)t * k + j] + lam_imp[order[j]];
+
+    if (cfg->router == 0) {
+      /* G = Softmax over the kept k of H: dH_i = G_i (dG_i - sum_l G_l dG_l) */
+      double sum = 0.0;
+      for (int j = 0; j < k; ++j) sum += gk[j] * dG[j];
+      for (int j = 0; j < k; ++j) dH[order[j]] = gk[j] * (dG[j] - sum);
+    } else if (cfg->router == 1) {
+      /* gate = p_argmax of p = softmax(c); the auxiliary loss
+       * alpha N sum_i f_i P_i has dP_i/dp_ti = 1/T with f_i fixed */
+      double *dp = dH; /* reuse: router 1 has no H gradient of its own */
+      for (int i = 0; i < n; ++i)
+        dp[i] = T > 0 ? cfg->alpha * (double)n * ((double)counts[i] / (double)T) / (double)T : 0.0;
+      dp[order[0]] += dG[0];
+      double sum = 0.0;
+      for (int i = 0; i < n; ++i) sum += pr[i] * dp[i];
+      for (int i = 0; i < n; ++i) dc[i] += pr[i] * (dp[i] - sum);
+      for (int i = 0; i < n; ++i) dH[i] = 0.0;
+    } else {
+      /* router 2: g_j = sigma(c_j) / S, S = sum over the kept of sigma:
+       * d sigma_m = (dG_m - sum_j g_j dG_j) / S, d c = d sigma * sigma (1 - sigma) */
+      double Ssum = 0.0, sum = 0.0;
+      for (int j = 0; j < k; ++j) Ssum += 1.0 / (1.0 + exp(-c[order[j]]));
+      for (int j = 0; j < k; ++j) sum += gk[j] * dG[j];
+      for (int j = 0; j < k; ++j) {
+        double sg = 1.0 / (1.0 + exp(-c[order[j]]));
+        dc[order[j]] += (dG[j] - sum) / Ssum * sg * (1.0 - sg);
+      }
+    }
+
+    if (noise && cfg->w_load != 0.0) {
+      /* P(x,i) = Phi((c_i - thr_i) / s_i), thr_i = H of the (k+1)-th ranked
+       * expert when i is kept, else of the k-th; Load_i = sum_t P(x_t,i) */
+      const int jk = order[k - 1], jk1 = k < n ? order[k] : -1;
+      for (int i = 0; i < n; ++i) {
+        const int jt = rank[i] < k ? jk1 : jk;
+        if (jt < 0 || s[i] == 0.0) continue; /* P is constant there */
+        const double u = (c[i] - (double)H[jt]) / s[i];
+        const double dens = exp(-0.5 * u * u) / sqrt(2.0 * acos(-1.0));
+        const double a = lam_load[i] * dens / s[i];
+        dc[i] += a;
+        ds[i] -= a * u;
+        dH[jt] -= a;
+      }
+    }
+    /* H = c + eps * s (noise), H = c otherwise (router 2's bias has no gradient) */
+    for (int i = 0; i < n; ++i) {
+      dc[i] += dH[i];
+      if (noise) ds[i] += dH[i] * orc_noise(cfg->seed, (uint32_t)t, (uint32_t)i, 0u);
+    }
+    /* s = Softplus(z), z = x W_noise: dz = ds * Sigmoid(z) */
+    if (noise) {
+      for (int i = 0; i < n; ++i) zp[i] = 0.0;
+      for (int q = 0; q < d; ++q)
+        for (int i = 0; i < n; ++i) zp[i] += (double)xt[q] * (double)in->Wn[(size_t)q * n + i];
+      for (int i = 0; i < n; ++i) ds[i] *= 1.0 / (1.0 + exp(-zp[i]));
+    }
+    if (g->dlogits) memcpy(g->dlogits + (size_t)t * n, dc, sizeof(double) * (size_t)n);
+    if (g->dnoise && noise) memcpy(g->dnoise + (size_t)t * n, ds, sizeof(double) * (size_t)n);
+    /* c = x W_g + b_g, z = x W_noise */
+    double *dxt = dx + (size_t)t * d;
+    for (int q = 0; q < d; ++q) {
+      double acc = 0.0;
+      for (int i = 0; i < n; ++i) {
+        acc += in->Wg[(size_t)q * n + i] * dc[i];
+        if (g->dWg) g->dWg[(size_t)q * n + i] += (double)xt[q] * dc[i];
+        if (noise) {
+          acc += in->Wn[(size_t)q * n + i] * ds[i];
+          if (g->dWn) g->dWn[(size_t)q * n + i] += (double)xt[q] * ds[i];
+        }
+      }
+      dxt[q] += acc;
+    }
+    if (g->dbg)
+      for (int i = 0; i < n; ++i) g->dbg[i] += dc[i];
+  }
+
+  if (!g->dW1) free(dW1);
+  if (!g->dW2) free(dW2);
+  if (cfg->shared_expert && !g->dW1s) free(dW1s);
+  if (cfg->shared_expert && !g->dW2s) free(dW2s);
+  free(c); free(s); free(pr); free(gk); free(dG); free(dc); free(ds); free(dH); free(zp);
+  free(H); free(order); free(rank); free(dgate);
+  free(idx); free(gate); free(load); free(psum); free(imp); free(counts); free(offsets);
+  free(ptok); free(pslot); free(row_of); free(lam_imp); free(lam_load);
+  return 0;
+}

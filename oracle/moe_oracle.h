@@ -176,6 +176,30 @@ int orc_router_stats(const orc_cfg *cfg, const orc_inputs *in, double *zsum, dou
  * orc_router_stats (else 0). */
 int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
 
+/* ---- backward pass ------------------------------------------------------ */
+/* Gradients of
+ *   L = sum_t <dy_t, y_t> + losses[0] + losses[1] + losses[3]
+ * (an upstream gradient dy[T][d] of the layer output plus the weighted
+ * balancing losses of orc_forward) with respect to x and every parameter;
+ * flat layers only (hier_a == 0).  With expert_bf16 the rounding points of a
+ * mixed-precision backward are taken (see orc_backward).  Any pointer other
+ * than dx and the routed experts' may be NULL (not written). */
+typedef struct {
+  double *dx;                                 /* [T][d]                      */
+  double *dWg, *dbg, *dWn;                    /* [d][n], [n], [d][n] (noise) */
+  double *dW1, *db1, *dW2, *db2;              /* [n][f][d], [n][f], [n][d][f], [n][d] */
+  double *dW1s, *db1s, *dW2s, *db2s;          /* shared expert: [f][d], [f], [d][f], [d] */
+  double *dgate;                              /* [T][k] dL / d topk_gate      */
+  double *dlogits;                            /* [T][n] dL / d (x W_g + b_g)  */
+  double *dnoise;                             /* [T][n] dL / d (x W_noise)    */
+} orc_grads;
+
+/* d CV(v)^2 / d v_i of orc_cv2 (0 where the mean is 0). */
+void orc_cv2_grad(const double *v, int n, double *g);
+
+/* 0, or -1 for a configuration the backward does not cover. */
+int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g);
+
 #ifdef __cplusplus
 }
 #endif

@@ -60,6 +60,12 @@ class OrcOutputs(C.Structure):
     ]
 
 
+class OrcGrads(C.Structure):
+    _fields_ = [(name, C.c_void_p) for name in (
+        "dx", "dWg", "dbg", "dWn", "dW1", "db1", "dW2", "db2", "dW1s", "db1s", "dW2s", "db2s",
+        "dgate", "dlogits", "dnoise")]
+
+
 def lib():
     global _lib
     if _lib is None:
@@ -99,6 +105,9 @@ def lib():
                                   vp, vp]
         L.orc_forward.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), C.POINTER(OrcOutputs)]
         L.orc_forward.restype = i32
+        L.orc_cv2_grad.argtypes = [vp, i32, vp]
+        L.orc_backward.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, C.POINTER(OrcGrads)]
+        L.orc_backward.restype = i32
         _lib = L
     return _lib
 
@@ -316,4 +325,33 @@ def forward(cfg: dict, inp: dict) -> dict:
     rc = lib().orc_forward(C.byref(oc), C.byref(ins), C.byref(outs))
     if rc != 0:
         raise ValueError(f"oracle rejected the configuration {cfg}")
+    return out
+
+
+# ---------------------------------------------------------------- backward
+def cv2_grad(v) -> np.ndarray:
+    a = _c(v, np.float64)
+    g = np.zeros(a.size)
+    lib().orc_cv2_grad(_p(a), a.size, _p(g))
+    return g
+
+
+def backward(cfg: dict, inp: dict, dy) -> dict:
+    """Gradients of L = sum(dy * y) + losses[0] + losses[1] + losses[3] of
+    ``forward(cfg, inp)`` with respect to x and every parameter (flat layers);
+    also dL/d topk_gate ("dgate"), dL/d clean logits ("dlogits") and dL/d
+    (x W_noise) ("dnoise")."""
+    oc = make_cfg(**cfg)
+    T, d, n, k, f = oc.T, oc.d, oc.n, oc.k, oc.f
+    keep, ins = _inputs(oc, inp)
+    dy = _c(dy, np.float32)
+    out = dict(dx=np.zeros((T, d)), dWg=np.zeros((d, n)), dbg=np.zeros(n), dWn=np.zeros((d, n)),
+               dW1=np.zeros((n, f, d)), db1=np.zeros((n, f)), dW2=np.zeros((n, d, f)),
+               db2=np.zeros((n, d)), dgate=np.zeros((T, k)), dlogits=np.zeros((T, n)),
+               dnoise=np.zeros((T, n)))
+    if oc.shared_expert:
+        out.update(dW1s=np.zeros((f, d)), db1s=np.zeros(f), dW2s=np.zeros((d, f)), db2s=np.zeros(d))
+    g = OrcGrads(**{name: _p(a) for name, a in out.items()})
+    if lib().orc_backward(C.byref(oc), C.byref(ins), _p(dy), C.byref(g)) != 0:
+        raise ValueError(f"oracle backward rejected the configuration {cfg}")
     return out

@@ -1,0 +1,233 @@
+"""Pins of the oracle's backward pass.
+
+The forward pass is pinned elsewhere (pages' worked examples, closed forms,
+library routines, brute force); here the gradients are pinned to it by
+central finite differences of
+
+    L = sum(dy * y) + losses[0] + losses[1] + losses[3]
+
+with fp32 experts (the bf16 path's roundings make L piecewise constant at the
+scale of a difference step).  The pages say which paths carry a gradient: the
+kept gates are smooth in the logits ("極大規模神經網路：稀疏門控專家混合層",
+常見問題), dropped experts get none (reading note, 缺点与局限性), and the noise
+lets the load loss reach the gate through Phi (reading note, Noisy Top-K
+Gating).  A step that flips a top-k choice or a capacity drop makes L jump;
+such entries are detected (routing compared at both ends) and skipped.
+
+Closed forms pin the CV^2 derivative, and torch autograd of a plain MLP (a
+library derivative, n = k = 1 so that the layer is one expert) pins the
+expert backward.  The bf16 rounding points are pinned against the fp32
+gradient of the same bf16-representable weights."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import oracle as O
+
+LOSS_IDX = (0, 1, 3)
+
+
+def _loss(cfg, inp, dy):
+    out = O.forward(cfg, inp)
+    return float(np.sum(dy * out["y"]) + sum(out["losses"][i] for i in LOSS_IDX)), out
+
+
+def _inputs(rng, T, d, n, f, *, noise=True, router=0, shared=False, bias=True):
+    inp = dict(
+        x=rng.normal(0, 1, (T, d)).astype(np.float32),
+        Wg=rng.normal(0, 0.7, (d, n)).astype(np.float32),
+        bg=rng.normal(0, 0.3, n).astype(np.float32) if bias else None,
+        Wn=rng.normal(0, 0.4, (d, n)).astype(np.float32) if noise else None,
+        W1=(rng.normal(0, 1, (n, f, d)) / math.sqrt(d)).astype(np.float32),
+        b1=rng.normal(0, 0.2, (n, f)).astype(np.float32),
+        W2=(rng.normal(0, 1, (n, d, f)) / math.sqrt(f)).astype(np.float32),
+        b2=rng.normal(0, 0.2, (n, d)).astype(np.float32),
+    )
+    if router == 2:
+        inp["sel_bias"] = rng.normal(0, 0.5, n).astype(np.float32)
+    if shared:
+        inp.update(W1s=(rng.normal(0, 1, (f, d)) / math.sqrt(d)).astype(np.float32),
+                   b1s=rng.normal(0, 0.2, f).astype(np.float32),
+                   W2s=(rng.normal(0, 1, (d, f)) / math.sqrt(f)).astype(np.float32),
+                   b2s=rng.normal(0, 0.2, d).astype(np.float32))
+    return inp
+
+
+GRAD_OF = dict(x="dx", Wg="dWg", bg="dbg", Wn="dWn", W1="dW1", b1="db1", W2="dW2", b2="db2",
+               W1s="dW1s", b1s="db1s", W2s="dW2s", b2s="db2s")
+
+
+def _check_fd(cfg, inp, dy, names, rng, per=10, step=2e-3, rtol=2e-3):
+    g = O.backward(cfg, inp, dy)
+    _, base = _loss(cfg, inp, dy)
+    checked = skipped = 0
+    for name in names:
+        arr = inp[name]
+        an = g[GRAD_OF[name]]
+        scale = float(np.abs(an).max()) + 1e-12
+        flat = rng.choice(arr.size, size=min(per, arr.size), replace=False)
+        for i in flat:
+            pos = np.unravel_index(int(i), arr.shape)
+            v0 = arr[pos]
+            h = np.float32(step * max(1.0, abs(float(v0))))
+            vp, vm = np.float32(v0 + h), np.float32(v0 - h)
+            arr[pos] = vp
+            lp, op = _loss(cfg, inp, dy)
+            arr[pos] = vm
+            lm, om = _loss(cfg, inp, dy)
+            arr[pos] = v0
+            same = all(np.array_equal(o["topk_idx"], base["topk_idx"]) and
+                       np.array_equal(o["row_of"], base["row_of"]) for o in (op, om))
+            if not same:
+                skipped += 1
+                continue
+            fd = (lp - lm) / (float(vp) - float(vm))
+            assert abs(fd - an[pos]) <= rtol * (abs(an[pos]) + 0.05 * scale) + 1e-9, \
+                (name, pos, fd, an[pos], scale)
+            checked += 1
+    assert checked >= 0.8 * (checked + skipped), (checked, skipped)
+    return g
+
+
+def test_cv2_grad_closed_form_and_differences():
+    # [1, 2, 3]: mean 2, var 2/3, CV^2 = 1/6; dCV^2/dv = (v - 2 - 1/3) / 6
+    assert O.cv2_grad([1, 2, 3]) == pytest.approx([-2 / 9, -1 / 18, 1 / 9], abs=1e-15)
+    rng = np.random.default_rng(0)
+    v = rng.uniform(0.5, 3, 9)
+    g = O.cv2_grad(v)
+    for i in range(v.size):
+        e = np.zeros_like(v); e[i] = 1e-6
+        fd = (O.cv2(v + e) - O.cv2(v - e)) / 2e-6
+        assert g[i] == pytest.approx(fd, rel=1e-6, abs=1e-9)
+    # a scale change leaves CV^2 alone: the gradient is orthogonal to v
+    assert float(np.dot(g, v)) == pytest.approx(0.0, abs=1e-12)
+    assert np.all(O.cv2_grad(np.zeros(4)) == 0)
+
+
+def test_noisy_topk_with_capacity_and_passthrough():
+    rng = np.random.default_rng(11)
+    T, d, n, k, f = 14, 6, 5, 2, 8
+    inp = _inputs(rng, T, d, n, f)
+    cfg = dict(T=T, d=d, n=n, k=k, f=f, router=0, noise=1, seed=5, capacity_factor=0.8,
+               passthrough=1, w_importance=0.4, w_load=0.6)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    out = O.forward(cfg, inp)
+    assert (out["row_of"] < 0).any()  # the capacity limit drops slots
+    g = _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "Wn", "W1", "b1", "W2", "b2"], rng)
+    # the load loss reaches the noise weights
+    assert np.abs(g["dWn"]).max() > 0
+
+
+def test_load_loss_alone_reaches_gate_through_phi():
+    # dy = 0 and no importance weight: the only gradient is the load loss's
+    rng = np.random.default_rng(4)
+    T, d, n, k, f = 10, 5, 6, 2, 8
+    inp = _inputs(rng, T, d, n, f)
+    cfg = dict(T=T, d=d, n=n, k=k, f=f, router=0, noise=1, seed=1, w_importance=0.0, w_load=1.0)
+    dy = np.zeros((T, d), np.float32)
+    g = _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "Wn"], rng)
+    assert np.abs(g["dW1"]).max() == 0 and np.abs(g["dW2"]).max() == 0
+    assert np.abs(g["dbg"]).max() > 0
+
+
+def test_noise_free_gate_and_k_equals_n():
+    rng = np.random.default_rng(5)
+    T, d, n, k, f = 9, 5, 4, 2, 8
+    inp = _inputs(rng, T, d, n, f, noise=False)
+    cfg = dict(T=T, d=d, n=n, k=k, f=f, router=0, noise=0, w_importance=0.5, w_load=0.5)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "W1", "b2"], rng)
+    # k = n: every expert kept, the gate is the full softmax, kth_excluding of
+    # a kept expert does not exist (P = 1): still differentiable
+    inp = _inputs(rng, T, d, n, f)
+    cfg = dict(T=T, d=d, n=n, k=n, f=f, router=0, noise=1, seed=3, w_importance=0.5, w_load=0.5)
+    _check_fd(cfg, inp, dy, ["x", "Wg", "Wn", "W2"], rng)
+
+
+def test_switch_router_with_aux_loss_and_capacity():
+    rng = np.random.default_rng(8)
+    T, d, n, f = 16, 6, 4, 8
+    inp = _inputs(rng, T, d, n, f, noise=False, router=1)
+    cfg = dict(T=T, d=d, n=n, k=1, f=f, router=1, noise=0, capacity_factor=1.0, passthrough=1,
+               w_importance=0.3, w_load=0.0, alpha=0.7)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    assert (O.forward(cfg, inp)["row_of"] < 0).any()
+    _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "W1", "b1", "W2"], rng)
+
+
+def test_sigmoid_router_with_bias_and_shared_expert():
+    rng = np.random.default_rng(9)
+    T, d, n, k, f = 12, 6, 6, 3, 8
+    inp = _inputs(rng, T, d, n, f, noise=False, router=2, shared=True)
+    cfg = dict(T=T, d=d, n=n, k=k, f=f, router=2, noise=0, shared_expert=1, w_importance=0.2,
+               w_load=0.0)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "W1", "W2", "W1s", "b1s", "W2s", "b2s"], rng)
+
+
+def test_single_expert_matches_torch_autograd():
+    """n = k = 1: the layer is y = E(x) (gate 1 for any logit), so the
+    expert gradients are those of a plain MLP, taken by torch autograd."""
+    rng = np.random.default_rng(2)
+    T, d, f = 7, 5, 9
+    inp = _inputs(rng, T, d, 1, f, noise=False)
+    cfg = dict(T=T, d=d, n=1, k=1, f=f, router=0, noise=0, w_importance=0.0, w_load=0.0)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    g = O.backward(cfg, inp, dy)
+    x = torch.tensor(inp["x"], dtype=torch.float64, requires_grad=True)
+    W1 = torch.tensor(inp["W1"][0], dtype=torch.float64, requires_grad=True)
+    b1 = torch.tensor(inp["b1"][0], dtype=torch.float64, requires_grad=True)
+    W2 = torch.tensor(inp["W2"][0], dtype=torch.float64, requires_grad=True)
+    b2 = torch.tensor(inp["b2"][0], dtype=torch.float64, requires_grad=True)
+    y = torch.nn.functional.linear(torch.relu(torch.nn.functional.linear(x, W1, b1)), W2, b2)
+    (y * torch.tensor(dy, dtype=torch.float64)).sum().backward()
+    for a, b in ((g["dx"], x), (g["dW1"][0], W1), (g["db1"][0], b1), (g["dW2"][0], W2),
+                 (g["db2"][0], b2)):
+        assert np.allclose(a, b.grad.numpy(), rtol=1e-12, atol=1e-12)
+    # one kept expert: the gate is identically 1, no gradient reaches W_g
+    assert np.abs(g["dWg"]).max() < 1e-12
+
+
+def _to_bf16_bits(a):
+    t = torch.tensor(a, dtype=torch.float32).to(torch.bfloat16)
+    return t.view(torch.int16).numpy().view(np.uint16), t.float().numpy()
+
+
+def test_bf16_rounding_points_track_fp32_gradient():
+    """The mixed-precision backward rounds only activation gradients to bf16:
+    with bf16-representable weights it stays within bf16 error of the fp32
+    backward, and exactly equal where nothing is rounded (the gate's dlogits
+    for dy = 0)."""
+    rng = np.random.default_rng(6)
+    T, d, n, k, f = 16, 16, 4, 2, 32
+    inp = _inputs(rng, T, d, n, f)
+    inp["x"] = _to_bf16_bits(inp["x"])[1]
+    b = dict(inp)
+    for w in ("W1", "W2"):
+        bits, vals = _to_bf16_bits(inp[w])
+        b[w] = bits
+        inp[w] = vals
+    cfg = dict(T=T, d=d, n=n, k=k, f=f, router=0, noise=1, seed=2, w_importance=0.3, w_load=0.3)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    g32 = O.backward(cfg, inp, dy)
+    g16 = O.backward(dict(cfg, expert_bf16=1), b, dy)
+    for key in ("dx", "dW1", "db1", "dW2", "db2", "dgate", "dlogits", "dWg"):
+        ref = g32[key]
+        err = np.abs(g16[key] - ref).max() / (np.abs(ref).max() + 1e-30)
+        assert err < 2e-2, (key, err)
+        assert err > 0 or key in ("dWg",), key  # something was rounded
+    z = np.zeros_like(dy)
+    assert np.array_equal(O.backward(cfg, inp, z)["dlogits"],
+                          O.backward(dict(cfg, expert_bf16=1), b, z)["dlogits"])
+
+
+def test_hierarchical_rejected():
+    with pytest.raises(ValueError):
+        O.backward(dict(T=2, d=4, n=4, k=1, f=8, hier_a=2, hier_b=2, hier_k1=1, hier_k2=1),
+                   dict(x=np.zeros((2, 4), np.float32), Wg=np.zeros((4, 2), np.float32),
+                        Wn=np.zeros((4, 2), np.float32), Wg2=np.zeros((2, 4, 2), np.float32),
+                        Wn2=np.zeros((2, 4, 2), np.float32), W1=np.zeros((4, 8, 4), np.float32),
+                        W2=np.zeros((4, 4, 8), np.float32)),
+                   np.zeros((2, 4), np.float32))
