@@ -133,6 +133,8 @@ typedef struct moe_config {
   int32_t gate_precision;     /* MOE_GATE_FP32 or MOE_GATE_TF32X3 */
   int32_t shared_expert;      /* 0 or 1 */
   int32_t router_stats;       /* 1: moe_forward reports losses[8], [9] */
+  int32_t backward;           /* 1: the workspace also serves moe_backward and
+                                 moe_forward keeps what it needs (0 or 1) */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
@@ -308,6 +310,49 @@ MOE_API int moe_forward(const moe_config *cfg, const float *x, const moe_gate_pa
                 float *topk_gate, float *importance, float *load, int32_t *counts,
                 float *losses, void *ws, size_t ws_bytes, int32_t *status,
                 moe_stream_t stream);
+
+/* ---------------------------------------------------------------- backward */
+
+/* Gradients written by moe_backward, fp32, caller-owned device memory in the
+ * layouts of the parameters.  Any pointer may be NULL (that gradient is not
+ * written) except dW1 and dW2; dW_noise is ignored without noise, the shared
+ * expert's without a shared expert.  dgate [T][k] and dlogits [T][n] are
+ * optional intermediate results: dL/d topk_gate and dL/d(x W_g + b_g). */
+typedef struct moe_grads {
+  float *dW_g, *db_g, *dW_noise;        /* [d][n], [n], [d][n] */
+  float *dW1, *db1, *dW2, *db2;         /* [n][f][d], [n][f], [n][d][f], [n][d] */
+  float *dW1s, *db1s, *dW2s, *db2s;     /* [f][d], [f], [d][f], [d] */
+  float *dgate, *dlogits;               /* [T][k], [T][n] */
+} moe_grads;
+
+/* Backward pass of a flat layer with bf16 experts.  The pages give no
+ * backward formulas; they fix which paths carry a gradient: the kept gates
+ * are a smooth function of the logits ([SGMoE-xyz] "常見問題"), KeepTopK
+ * gives the experts it drops none ([SGMoE-note] "缺点与局限性"), and the
+ * noise lets the load loss reach the gate through Phi ([SGMoE-note] "Noisy
+ * Top-K Gating").  Computes the gradients of
+ *   L = sum(dy * y) + losses[0] + losses[1] + losses[3]
+ * (dy [T][d] fp32, the upstream gradient of moe_forward's y, plus the
+ * weighted balancing losses) with respect to x (dx [T][d], fp32, written) and
+ * every parameter (grads).  Mixed precision: the gradients reaching the
+ * expert rows (g * dy), the hidden layer and the expert inputs are kept in
+ * bf16 as the forward keeps its activations; accumulation is fp32; the gate
+ * is fp32 throughout.  The selection bias of MOE_ROUTER_SIGMOID gets no
+ * gradient (it enters only the choice of experts).
+ *
+ * Preconditions: cfg->backward == 1 and ws is the workspace of the preceding
+ * moe_forward with the same cfg, x and parameters, whose outputs topk_idx,
+ * topk_gate, importance, load and counts are passed back here; both calls
+ * on the same stream, in that order.  ws is read and overwritten.
+ * Errors: MOE_EINVAL for a hierarchical layer, fp32 experts, cfg->backward
+ * != 1, NULL required pointers or misaligned ones (x, dy, dx 16-byte
+ * aligned); MOE_EWORKSPACE; MOE_ECUDA.  Device-side timeouts are OR-ed into
+ * *status (MOE_STATUS_TIMEOUT). */
+MOE_API int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
+                         const moe_expert_params *ep, const float *dy, const int32_t *topk_idx,
+                         const float *topk_gate, const float *importance, const float *load,
+                         const int32_t *counts, float *dx, const moe_grads *grads, void *ws,
+                         size_t ws_bytes, int32_t *status, moe_stream_t stream);
 
 /* ---------------------------------------------------------------- tracing */
 

@@ -17,7 +17,7 @@ STATUS_NONFINITE, STATUS_BAD_INDEX, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 EXPORTS = ("moe_strerror", "moe_validate", "moe_capacity", "moe_workspace_size", "moe_gate",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_balance_losses", "moe_forward",
            "moe_trace_enable", "moe_trace_reset", "moe_trace_count", "moe_trace_get",
-           "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update")
+           "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update", "moe_backward")
 
 
 class moe_config(C.Structure):
@@ -28,6 +28,7 @@ class moe_config(C.Structure):
         ("seed", C.c_uint64), ("capacity_factor", C.c_double), ("overflow_passthrough", C.c_int32),
         ("w_importance", C.c_float), ("w_load", C.c_float), ("alpha_aux", C.c_float),
         ("gate_precision", C.c_int32), ("shared_expert", C.c_int32), ("router_stats", C.c_int32),
+        ("backward", C.c_int32),
     ]
 
 
@@ -40,6 +41,12 @@ class moe_gate_params(C.Structure):
 class moe_expert_params(C.Structure):
     _fields_ = [("W1", C.c_void_p), ("b1", C.c_void_p), ("W2", C.c_void_p), ("b2", C.c_void_p),
                 ("W1s", C.c_void_p), ("b1s", C.c_void_p), ("W2s", C.c_void_p), ("b2s", C.c_void_p)]
+
+
+class moe_grads(C.Structure):
+    _fields_ = [(name, C.c_void_p) for name in (
+        "dW_g", "db_g", "dW_noise", "dW1", "db1", "dW2", "db2", "dW1s", "db1s", "dW2s", "db2s",
+        "dgate", "dlogits")]
 
 
 _lib = None
@@ -70,6 +77,8 @@ def load():
     L.moe_balance_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_forward.argtypes = [cfgp, vp, C.POINTER(moe_gate_params), C.POINTER(moe_expert_params),
                               vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
+    L.moe_backward.argtypes = [cfgp, vp, C.POINTER(moe_gate_params), C.POINTER(moe_expert_params),
+                               vp, vp, vp, vp, vp, vp, vp, C.POINTER(moe_grads), vp, sz, vp, vp]
     L.moe_trace_enable.argtypes = [i32]
     L.moe_trace_get.argtypes = [i32, C.POINTER(C.c_char_p), C.POINTER(C.c_int), C.POINTER(C.c_double)]
     L.moe_launch_count.restype = C.c_longlong

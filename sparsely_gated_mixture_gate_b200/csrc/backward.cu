@@ -1,0 +1,507 @@
+// backward.cu -- the memory-bound kernels of the layer's backward pass.
+//
+// The pages give no backward formulas; they say which paths carry a
+// gradient: the kept gates are smooth in the logits ([SGMoE-xyz] 常見問題),
+// KeepTopK gives the experts it drops none ([SGMoE-note] 缺点与局限性), and
+// the noise lets the load loss reach the gate through Phi ([SGMoE-note]
+// Noisy Top-K Gating).  What follows is the chain rule of the forward pass in
+// reverse order, for the loss
+//   L = sum(dy * y) + w_importance CV(Importance)^2 + w_load CV(Load)^2
+//       + alpha * N sum_i f_i P_i (Switch)
+//   bwd_coef        dL/dImportance_i, dL/dLoad_i (through CV^2) and the Switch
+//                   loss's dL/dp_ti (one block, fp64)
+//   combine_bwd     per token and kept slot: dy_perm[row] = bf16(g * dy_t),
+//                   dgate = <dy_t, y_perm[row]>; the shared expert's rows get dy
+//   bias_grad       db of every expert: column sums of its rows of dy_perm and
+//                   dhid, in a fixed order
+//   dx_gather       dx_t = sum over kept slots of dx_perm[row] (+ dy_t for a
+//                   passed-through token, + the shared expert's row)
+//   gate_bwd        per token: dL/dc (clean logits) and dL/dz (noise logits,
+//                   z = x W_noise) through the softmax over the kept, the
+//                   importance and load losses (Phi' and kth_excluding), the
+//                   noise (eps recomputed from Philox) and Softplus
+//   colsum          column sums of a row-major matrix in row blocks (db_g)
+#include "internal.h"
+#include "philox.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int CT = 1024;
+
+__device__ double block_sum_d(double v, double *sh) {
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  if (lane == 0) sh[w] = v;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    double r = 0.0;
+    for (int i = 0; i < CT / 32; ++i) r += sh[i];
+    sh[CT / 32] = r;
+  }
+  __syncthreads();
+  const double r = sh[CT / 32];
+  __syncthreads();
+  return r;
+}
+
+// d CV(v)^2 / d v_i = 2 / (n mean^2) * ((v_i - mean) - var / mean), times w
+// (0 where the mean is 0, as CV^2 is defined 0 there)
+__device__ void cv2_grad(const float *v, int n, float w, float *out, double *sh) {
+  double s = 0.0;
+  for (int i = threadIdx.x; i < n; i += CT) s += (double)v[i];
+  const double mean = block_sum_d(s, sh) / (double)n;
+  double q = 0.0;
+  for (int i = threadIdx.x; i < n; i += CT) {
+    const double dv = (double)v[i] - mean;
+    q += dv * dv;
+  }
+  const double var = block_sum_d(q, sh) / (double)n;
+  for (int i = threadIdx.x; i < n; i += CT) {
+    double g = 0.0;
+    if (mean != 0.0 && w != 0.f)
+      g = (double)w * 2.0 / ((double)n * mean * mean) * (((double)v[i] - mean) - var / mean);
+    out[i] = (float)g;
+  }
+}
+
+__global__ void __launch_bounds__(CT) bwd_coef_kernel(const float *importance, const float *load,
+                                                      const int *counts, int n, int T, float w_imp,
+                                                      float w_load, float alpha, int router,
+                                                      int noise, float *lam_imp, float *lam_load,
+                                                      float *sw_coef) {
+  __shared__ double sh[CT / 32 + 1];
+  cv2_grad(importance, n, w_imp, lam_imp, sh);
+  // without noise Load is the count of selections: no gradient
+  cv2_grad(load, n, noise ? w_load : 0.f, lam_load, sh);
+  for (int i = threadIdx.x; i < n; i += CT) {
+    // Switch: alpha N sum_i f_i P_i, P_i = sum_t p_ti / T, f_i fixed
+    const double c = router == MOE_ROUTER_SWITCH && T > 0
+                         ? (double)alpha * (double)n * ((double)counts[i] / (double)T) / (double)T
+                         : 0.0;
+    sw_coef[i] = (float)c;
+  }
+}
+
+// ---------------------------------------------------------------- combine_bwd
+constexpr int NT = 256;
+
+__device__ __forceinline__ void bf16x8_to_f32(const uint4 pk, float (&f)[8]) {
+  const uint32_t w4[4] = {pk.x, pk.y, pk.z, pk.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 f2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&w4[u]));
+    f[2 * u] = f2.x;
+    f[2 * u + 1] = f2.y;
+  }
+}
+__device__ __forceinline__ uint4 f32x8_to_bf16(const float (&f)[8]) {
+  uint32_t w[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    __nv_bfloat162 h = __floats2bfloat162_rn(f[2 * u], f[2 * u + 1]);
+    w[u] = *reinterpret_cast<uint32_t *>(&h);
+  }
+  return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// one warp per token, 8 features per lane per step
+template <int KM>
+__global__ void __launch_bounds__(NT) combine_bwd_kernel(
+    const float *__restrict__ dy, const float *__restrict__ gate, const int *__restrict__ row_of,
+    const __nv_bfloat16 *__restrict__ y_perm, int T, int k, int d,
+    __nv_bfloat16 *__restrict__ dy_perm, float *__restrict__ dgate,
+    __nv_bfloat16 *__restrict__ dy_shared) {
+  const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  int rows[KM];
+  float g[KM], acc[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    rows[j] = j < k ? __ldg(row_of + (size_t)t * k + j) : -1;
+    g[j] = j < k ? __ldg(gate + (size_t)t * k + j) : 0.f;
+    acc[j] = 0.f;
+  }
+  const float4 *dyr = reinterpret_cast<const float4 *>(dy + (size_t)t * d);
+  for (int c = lane; c < (d >> 3); c += 32) {
+    float v[8];
+    {
+      const float4 u = __ldg(dyr + 2 * c), w = __ldg(dyr + 2 * c + 1);
+      v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+      v[4] = w.x; v[5] = w.y; v[6] = w.z; v[7] = w.w;
+    }
+    if (dy_shared)
+      reinterpret_cast<uint4 *>(dy_shared + (size_t)t * d)[c] = f32x8_to_bf16(v);
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (rows[j] < 0) continue;
+      float yv[8], o[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(y_perm + (size_t)rows[j] * d) + c), yv);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        acc[j] = fmaf(v[u], yv[u], acc[j]);
+        o[u] = g[j] * v[u];
+      }
+      reinterpret_cast<uint4 *>(dy_perm + (size_t)rows[j] * d)[c] = f32x8_to_bf16(o);
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xffffffffu, acc[j], off);
+  }
+  if (lane == 0)
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (j < k) dgate[(size_t)t * k + j] = acc[j];  // 0 for a dropped slot
+}
+
+// ---------------------------------------------------------------- dx_gather
+template <int KM>
+__global__ void __launch_bounds__(NT) dx_gather_kernel(
+    const __nv_bfloat16 *__restrict__ dx_perm, const int *__restrict__ row_of,
+    const float *__restrict__ dy, int passthrough, int T, int k, int d,
+    const __nv_bfloat16 *__restrict__ dx_shared, float *__restrict__ dx) {
+  const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  int rows[KM];
+  bool any = false;
+#pragma unroll
+  for (int j = 0; j < KM; ++j) {
+    rows[j] = j < k ? __ldg(row_of + (size_t)t * k + j) : -1;
+    any |= rows[j] >= 0;
+  }
+  const bool pass = passthrough && !any;
+  float4 *out = reinterpret_cast<float4 *>(dx + (size_t)t * d);
+  for (int c = lane; c < (d >> 3); c += 32) {
+    float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      if (rows[j] < 0) continue;
+      float v[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(dx_perm + (size_t)rows[j] * d) + c), v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] += v[u];
+    }
+    if (pass) {  // y = x for a token whose every slot overflowed
+      const float4 *dyr = reinterpret_cast<const float4 *>(dy + (size_t)t * d);
+      const float4 u = __ldg(dyr + 2 * c), w = __ldg(dyr + 2 * c + 1);
+      a[0] += u.x; a[1] += u.y; a[2] += u.z; a[3] += u.w;
+      a[4] += w.x; a[5] += w.y; a[6] += w.z; a[7] += w.w;
+    }
+    if (dx_shared) {
+      float v[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(dx_shared + (size_t)t * d) + c), v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] += v[u];
+    }
+    out[2 * c] = make_float4(a[0], a[1], a[2], a[3]);
+    out[2 * c + 1] = make_float4(a[4], a[5], a[6], a[7]);
+  }
+}
+
+// ---------------------------------------------------------------- bias_grad
+// grid.y: expert; grid.x: 256-column blocks of dy_perm (N = d) then of dhid
+// (N = f).  Thread (row group rg of 8, column group cg of 32) sums 8 columns
+// over rows rg, rg+8, ...; the 8 row groups are then added in order.
+__global__ void __launch_bounds__(256) bias_grad_kernel(
+    const __nv_bfloat16 *__restrict__ dy_perm, const __nv_bfloat16 *__restrict__ dhid,
+    const int *__restrict__ offsets, int d, int f, float *__restrict__ db2,
+    float *__restrict__ db1) {
+  __shared__ float part[8][256];
+  const int e = blockIdx.y;
+  const int cb2 = (d + 255) / 256;
+  const bool first = (int)blockIdx.x < cb2;
+  const int N = first ? d : f;
+  const int cb = first ? blockIdx.x : blockIdx.x - cb2;
+  const __nv_bfloat16 *src = first ? dy_perm : dhid;
+  float *const dsel = first ? db2 : db1;
+  if (!dsel) return;  // that bias gradient is not wanted
+  float *dst = dsel + (size_t)e * N;
+  const int cg = threadIdx.x & 31, rg = threadIdx.x >> 5;
+  const int c0 = cb * 256 + cg * 8;
+  const int r0 = offsets[e], r1 = offsets[e + 1];
+  float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  if (c0 < N) {
+    for (int r = r0 + rg; r < r1; r += 8) {
+      float v[8];
+      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(src + (size_t)r * N + c0)), v);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) a[u] += v[u];
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < 8; ++u) part[rg][cg * 8 + u] = a[u];
+  __syncthreads();
+  const int col = cb * 256 + threadIdx.x;
+  if (col < N) {
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) s += part[q][threadIdx.x];
+    dst[col] = s;
+  }
+}
+
+// ---------------------------------------------------------------- gate_bwd
+constexpr int GW = 8;  // warps (rows) per block
+
+// one warp per token row of the flat gate
+template <int KM>
+__global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
+  const int t = blockIdx.x * GW + (threadIdx.x >> 5);
+  if (t >= a.T) return;
+  const int lane = threadIdx.x & 31;
+  const int n = a.n, k = a.k;
+  const float *crow = a.c + (size_t)t * n;
+  const float *srow = a.s + (size_t)t * n;
+  float *dcrow = a.dc + (size_t)t * n;
+  float *dzrow = a.dz ? a.dz + (size_t)t * n : nullptr;
+
+  // the kept slots, larger H first (every lane holds all of them)
+  int ids[KM];
+  float gs[KM], dG[KM];
+  {
+    int id = 0;
+    float gv = 0.f, dv = 0.f;
+    if (lane < k) {
+      id = a.idx[(size_t)t * k + lane];
+      gv = a.gate[(size_t)t * k + lane];
+      dv = a.dgate[(size_t)t * k + lane] + a.lam_imp[id];  // combine + importance
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      ids[j] = __shfl_sync(0xffffffffu, id, j);
+      gs[j] = __shfl_sync(0xffffffffu, gv, j);
+      dG[j] = __shfl_sync(0xffffffffu, dv, j);
+    }
+  }
+  float gdg = 0.f;  // sum_j g_j dG_j
+#pragma unroll
+  for (int j = 0; j < KM; ++j)
+    if (j < k) gdg = fmaf(gs[j], dG[j], gdg);
+
+  if (a.router == MOE_ROUTER_SWITCH) {
+    // gate = p_argmax, p = softmax(c): dp_i = sw_i + [i = e_0] dG_0,
+    // dc_i = p_i (dp_i - sum_l p_l dp_l)
+    float mx = -INFINITY, se = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float v = crow[i];
+      const float m2 = fmaxf(mx, v);
+      se = se * expf(mx - m2) + expf(v - m2);
+      mx = m2;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float om = __shfl_xor_sync(0xffffffffu, mx, off);
+      const float os = __shfl_xor_sync(0xffffffffu, se, off);
+      const float m2 = fmaxf(mx, om);
+      const float a1 = mx == -INFINITY ? 0.f : se * expf(mx - m2);
+      const float a2 = om == -INFINITY ? 0.f : os * expf(om - m2);
+      mx = m2;
+      se = a1 + a2;
+    }
+    float pd = 0.f;
+    for (int i = lane; i < n; i += 32) {
+      const float p = expf(crow[i] - mx) / se;
+      pd = fmaf(p, a.sw_coef[i] + (i == ids[0] ? dG[0] : 0.f), pd);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) pd += __shfl_xor_sync(0xffffffffu, pd, off);
+    for (int i = lane; i < n; i += 32) {
+      const float p = expf(crow[i] - mx) / se;
+      dcrow[i] = p * (a.sw_coef[i] + (i == ids[0] ? dG[0] : 0.f) - pd);
+    }
+    return;
+  }
+
+  if (a.router == MOE_ROUTER_SIGMOID) {
+    // g_j = sigma(c_j) / S over the kept: dc_m = (dG_m - sum g dG) / S sigma_m (1 - sigma_m)
+    float sg[KM], S = 0.f;
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      sg[j] = j < k ? 1.f / (1.f + expf(-crow[ids[j]])) : 0.f;
+      S += sg[j];
+    }
+    for (int i = lane; i < n; i += 32) {
+      float v = 0.f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j < k && ids[j] == i) v = (dG[j] - gdg) / S * sg[j] * (1.f - sg[j]);
+      dcrow[i] = v;
+    }
+    return;
+  }
+
+  // ---- noisy top-k softmax gate: dH_i = G_i (dG_i - sum_l G_l dG_l) on the kept
+  float dHk[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) dHk[j] = gs[j] * (dG[j] - gdg);
+
+  // load loss: P_i = Phi(u_i), u_i = (c_i - thr_i) / s_i; thr_i is H of the
+  // (k+1)-th ranked expert jk1 when i is kept, of the k-th (jk) otherwise
+  const bool loadg = a.noise && a.has_load;
+  float thr_kept = -INFINITY, thr_out = -INFINITY;
+  int jk1 = -1, jkk = 0;  // the (k+1)-th and the k-th ranked expert
+#pragma unroll
+  for (int j = 0; j < KM; ++j)
+    if (j == k - 1) jkk = ids[j];
+  if (loadg) {
+    const int4 q = a.kth[t];
+    thr_kept = __int_as_float(q.x);
+    jk1 = thr_kept == -INFINITY ? -1 : q.y;
+    thr_out = __int_as_float(q.z);
+  }
+  auto kept_slot = [&](int i) {
+    int js = -1;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (j < k && ids[j] == i) js = j;
+    return js;
+  };
+  // A_kept / A_out: sum of lam_load_i phi(u_i) / s_i over kept / not kept i
+  float A_kept = 0.f, A_out = 0.f;
+  if (loadg) {
+    for (int i = lane; i < n; i += 32) {
+      const bool kept = kept_slot(i) >= 0;
+      const float thr = kept ? thr_kept : thr_out;
+      const float sv = srow[i];
+      if (thr == -INFINITY || sv == 0.f) continue;  // P constant there
+      const float u = (crow[i] - thr) / sv;
+      const float av = a.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
+      if (kept) A_kept += av; else A_out += av;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      A_kept += __shfl_xor_sync(0xffffffffu, A_kept, off);
+      A_out += __shfl_xor_sync(0xffffffffu, A_out, off);
+    }
+  }
+  const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
+  for (int m = lane; 4 * m < n; m += 32) {
+    float eps[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.noise) {
+      const uint4 wd = philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, 0u, 0u), key0, key1);
+      box_muller2(wd.x, wd.y, eps[0], eps[1]);
+      box_muller2(wd.z, wd.w, eps[2], eps[3]);
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const int i = 4 * m + j4;
+      if (i >= n) break;
+      const int js = kept_slot(i);
+      float dH = 0.f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j == js) dH = dHk[j];
+      float dc = 0.f, ds = 0.f;
+      const float sv = a.noise ? srow[i] : 0.f;
+      if (loadg) {
+        if (i == jk1) dH -= A_kept;
+        if (i == jkk) dH -= A_out;
+        const float thr = js >= 0 ? thr_kept : thr_out;
+        if (thr != -INFINITY && sv != 0.f) {
+          const float u = (crow[i] - thr) / sv;
+          const float av = a.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
+          dc += av;
+          ds -= av * u;
+        }
+      }
+      dc += dH;  // H = c + eps s
+      dcrow[i] = dc;
+      if (dzrow) {
+        ds = fmaf(dH, eps[j4], ds);
+        // s = Softplus(z): dz = ds Sigmoid(z), Sigmoid(z) = 1 - e^-s
+        dzrow[i] = ds * -expm1f(-sv);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------- colsum
+// part[blockIdx.y][j] = sum of rows [blockIdx.y * rows_per, ...) of column j
+__global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ X, int R, int N,
+                                                     int rows_per, float *__restrict__ part) {
+  const int j = blockIdx.x * 256 + threadIdx.x;
+  if (j >= N) return;
+  const int r0 = blockIdx.y * rows_per, r1 = min(r0 + rows_per, R);
+  float s = 0.f;
+  for (int r = r0; r < r1; ++r) s += X[(size_t)r * N + j];
+  part[(size_t)blockIdx.y * N + j] = s;
+}
+
+}  // namespace
+
+int launch_bwd_coef(const float *importance, const float *load, const int *counts, int n, int T,
+                    float w_imp, float w_load, float alpha, int router, int noise, float *lam_imp,
+                    float *lam_load, float *sw_coef, cudaStream_t st) {
+  return launch("bwd_coef", bwd_coef_kernel, dim3(1), dim3(CT), 0, st, importance, load, counts,
+                n, T, w_imp, w_load, alpha, router, noise, lam_imp, lam_load, sw_coef);
+}
+
+int launch_combine_bwd(const float *dy, const float *gate, const int *row_of, const void *y_perm,
+                       int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
+                       cudaStream_t st) {
+  if (k > kMaxK) return MOE_EINVAL;
+  const dim3 grid((unsigned)ceil_div(T, NT / 32));
+  auto go = [&](auto kern) {
+    return launch("combine_bwd", kern, grid, dim3(NT), 0, st, dy, gate, row_of,
+                  static_cast<const __nv_bfloat16 *>(y_perm), T, k, d,
+                  static_cast<__nv_bfloat16 *>(dy_perm), dgate,
+                  static_cast<__nv_bfloat16 *>(dy_shared));
+  };
+  if (k <= 1) return go(combine_bwd_kernel<1>);
+  if (k <= 2) return go(combine_bwd_kernel<2>);
+  if (k <= 4) return go(combine_bwd_kernel<4>);
+  return go(combine_bwd_kernel<8>);
+}
+
+int launch_dx_gather(const void *dx_perm, const int *row_of, const float *dy, int passthrough,
+                     int T, int k, int d, const void *dx_shared, float *dx, cudaStream_t st) {
+  if (k > kMaxK) return MOE_EINVAL;
+  const dim3 grid((unsigned)ceil_div(T, NT / 32));
+  auto go = [&](auto kern) {
+    return launch("dx_gather", kern, grid, dim3(NT), 0, st,
+                  static_cast<const __nv_bfloat16 *>(dx_perm), row_of, dy, passthrough, T, k, d,
+                  static_cast<const __nv_bfloat16 *>(dx_shared), dx);
+  };
+  if (k <= 1) return go(dx_gather_kernel<1>);
+  if (k <= 2) return go(dx_gather_kernel<2>);
+  if (k <= 4) return go(dx_gather_kernel<4>);
+  return go(dx_gather_kernel<8>);
+}
+
+int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,
+                     int f, float *db2, float *db1, const char *name, cudaStream_t st) {
+  const dim3 grid((unsigned)(ceil_div(d, 256) + ceil_div(f, 256)), (unsigned)n);
+  return launch(name ? name : "bias_grad", bias_grad_kernel, grid, dim3(256), 0, st,
+                static_cast<const __nv_bfloat16 *>(dy_perm),
+                static_cast<const __nv_bfloat16 *>(dhid), offsets, d, f, db2, db1);
+}
+
+int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st) {
+  if (a.k > kMaxK) return MOE_EINVAL;
+  const dim3 grid((unsigned)ceil_div(a.T, GW));
+  auto go = [&](auto kern) { return launch("gate_bwd", kern, grid, dim3(GW * 32), 0, st, a); };
+  if (a.k <= 1) return go(gate_bwd_kernel<1>);
+  if (a.k <= 2) return go(gate_bwd_kernel<2>);
+  if (a.k <= 4) return go(gate_bwd_kernel<4>);
+  return go(gate_bwd_kernel<8>);
+}
+
+int colsum_parts(int R) { return R <= 0 ? 0 : (int)ceil_div(R, 256) < 64 ? (int)ceil_div(R, 256) : 64; }
+
+int launch_colsum(const float *X, int R, int N, float *part, float *out, cudaStream_t st) {
+  const int parts = colsum_parts(R);
+  if (parts == 0) {
+    return cudaMemsetAsync(out, 0, 4 * (size_t)N, st) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+  }
+  const int rows_per = (int)ceil_div(R, parts);
+  MOE_TRY(launch("colsum", colsum_kernel, dim3((unsigned)ceil_div(N, 256), (unsigned)parts),
+                 dim3(256), 0, st, X, R, N, rows_per, part));
+  return launch_route_reduce(part, nullptr, 1, parts, N, out, st);
+}
+
+}  // namespace moe

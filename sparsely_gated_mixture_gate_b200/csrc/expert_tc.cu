@@ -7,6 +7,11 @@
 //   GEMM1: hid    = ReLU(x_perm_e W1_e^T + b1_e)   (bf16 out)
 //   GEMM2: y_perm = hid_e W2_e^T + b2_e            (bf16 out)
 // Both are "grouped" GEMMs with a ragged M per expert and K-major operands.
+// The backward pass's activation gradients have the same two-step shape:
+//   GEMM1': dhid    = (dy_perm_e W2_e) * [hid > 0]  (bf16 out; ReLU mask)
+//   GEMM2': dx_perm = dhid_e W1_e                   (bf16 out)
+// with the same tiles (N = f, then N = d); their B operands are the weights
+// as stored, i.e. MN-major (N contiguous), loaded as four 64-column boxes.
 //
 // One persistent kernel runs both, one CTA per SM, 320 threads.  Every CTA
 // takes its share of GEMM1's tiles and then of GEMM2's, so GEMM2 starts on
@@ -62,6 +67,8 @@ constexpr unsigned long long kWaitNs = 2000000000ull;
 // 17-22, M>>4 at bits 24-28.
 constexpr uint32_t IDESC = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) |
                            ((uint32_t)(BM >> 4) << 24);
+constexpr uint32_t IDESC_BMN = IDESC | (1u << 16);  // B MN-major (bit 16)
+constexpr int BOX_MN = 64 * BK * 2;                  // one 64-column box of an MN-major tile
 
 struct GemmArgs {
   const int4 *tiles;     // per tile: {expert, first row, valid rows, N-block | M-block << 8}
@@ -69,6 +76,7 @@ struct GemmArgs {
   const float *bias;     // [n][N] or nullptr
   __nv_bfloat16 *D;      // [S][N]
   int relu;
+  const __nv_bfloat16 *mask;  // [S][N] or nullptr: D = acc where mask > 0, else 0
 };
 
 struct FfnArgs {
@@ -100,6 +108,8 @@ __device__ __noinline__ bool wait_count(const int *p, int target, volatile int *
   }
 }
 
+// BMN: B operands MN-major (the backward pass's activation gradients)
+template <bool BMN>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     expert_ffn_kernel(const __grid_constant__ CUtensorMap tmA1,
                       const __grid_constant__ CUtensorMap tmB1,
@@ -176,13 +186,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const CUtensorMap *mA = which ? &tmA2 : &tmA1;
       const CUtensorMap *mB = which ? &tmB2 : &tmB1;
       const int nkb = (g.K + BK - 1) / BK;
-      const int brow = ti.x * g.N + (ti.w & 0xFF) * BN;
+      const int brow = ti.x * g.N + (ti.w & 0xFF) * BN;  // K-major B: first weight row
+      const int bcol = (ti.w & 0xFF) * BN;                // MN-major B: first column
       for (int kb = 0; kb < nkb; ++kb) {
         if (!mbar_wait(empty(stage), phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
         const uint32_t sa = sbase + stage * STAGE_BYTES;
         mbar_expect_tx(full(stage), STAGE_BYTES);
         tma_load_2d(sa, mA, full(stage), kb * BK, ti.y);
-        tma_load_2d(sa + A_BYTES, mB, full(stage), kb * BK, brow);
+        if (BMN) {
+          // rows ti.x*K + kb*BK .. +63 of the [n*K][N] weights, four 64-column boxes
+#pragma unroll
+          for (int i = 0; i < BN / 64; ++i)
+            tma_load_2d(sa + A_BYTES + i * BOX_MN, mB, full(stage), bcol + 64 * i,
+                        ti.x * g.K + kb * BK);
+        } else {
+          tma_load_2d(sa + A_BYTES, mB, full(stage), kb * BK, brow);
+        }
         issued[stage] = (int)phase;
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
       }
@@ -209,9 +228,14 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         tc_fence_after();
         const uint32_t sa = sbase + stage * STAGE_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / 16; ++kk)
-          tc_mma_f16(d_tmem, sw128_desc(sa + kk * 32), sw128_desc(sa + A_BYTES + kk * 32), IDESC,
+        for (int kk = 0; kk < BK / 16; ++kk) {
+          // K-major: the 16-wide K step is 32 bytes into each 128-byte row;
+          // MN-major: 16 rows of 128 bytes further on
+          const uint64_t bdesc = BMN ? sw128_mn_desc(sa + A_BYTES + kk * 2048, BOX_MN)
+                                     : sw128_desc(sa + A_BYTES + kk * 32);
+          tc_mma_f16(d_tmem, sw128_desc(sa + kk * 32), bdesc, BMN ? IDESC_BMN : IDESC,
                      (kb | kk) != 0);
+        }
         issued_any = true;
         tc_commit(empty(stage));
         if (++stage == STAGES) { stage = 0; phase ^= 1u; }
@@ -263,6 +287,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t v[64];
         tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cl), v);
         const int col0 = nbk * BN + cl;
+        // ReLU mask of the backward pass: this lane's row of hid, 64 columns
+        uint32_t mk[32];
+        if (BMN && g.mask) {
+          const bool in = lane < rows_here && col0 < g.N;
+          const uint4 *mrow = reinterpret_cast<const uint4 *>(
+              g.mask + (size_t)(ti.y + q * 32 + (in ? lane : 0)) * g.N + (in ? col0 : 0));
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const uint4 m4 = in && col0 + 8 * u < g.N ? __ldg(mrow + u) : make_uint4(0u, 0u, 0u, 0u);
+            mk[4 * u] = m4.x; mk[4 * u + 1] = m4.y; mk[4 * u + 2] = m4.z; mk[4 * u + 3] = m4.w;
+          }
+        }
         // conversion by the whole warp (the shuffles need every lane)
         uint32_t pk[32];
 #pragma unroll
@@ -274,6 +310,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           if (g.relu) {
             x0 = fmaxf(x0, 0.f);
             x1 = fmaxf(x1, 0.f);
+          }
+          if (BMN && g.mask) {  // bf16 pair: positive iff sign clear and not zero
+            const uint32_t m2 = mk[j];
+            if ((m2 & 0x8000u) || !(m2 & 0x7FFFu)) x0 = 0.f;
+            if ((m2 & 0x80000000u) || !(m2 & 0x7FFF0000u)) x1 = 0.f;
           }
           __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
           pk[j] = *reinterpret_cast<uint32_t *>(&h);
@@ -329,7 +370,7 @@ int ffn_ctas() {
   cudaGetDevice(&dev);
   if (dev != cached_dev) {
     int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ffn_kernel, NUM_THREADS,
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ffn_kernel<false>, NUM_THREADS,
                                                       SMEM_BYTES) != cudaSuccess ||
         per_sm < 1)
       return 0;
@@ -353,19 +394,34 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (attr_dev != dev) {
-    if (cudaFuncSetAttribute(expert_ffn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(expert_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             SMEM_BYTES) != cudaSuccess ||
+        cudaFuncSetAttribute(expert_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES) != cudaSuccess)
       return MOE_ECUDA;
     attr_dev = dev;
   }
+  const bool bwd = a.backward != 0;
   CUtensorMap a1, b1, a2, b2;
-  MOE_TRY(tc::make_map_2d(&a1, a.x_perm, 2, (uint64_t)a.d, (uint64_t)a.S, BM));
-  MOE_TRY(tc::make_map_2d(&b1, a.W1, 2, (uint64_t)a.d, (uint64_t)a.n * a.f, BN));
-  MOE_TRY(tc::make_map_2d(&a2, a.hid, 2, (uint64_t)a.f, (uint64_t)a.S, BM));
-  MOE_TRY(tc::make_map_2d(&b2, a.W2, 2, (uint64_t)a.f, (uint64_t)a.n * a.d, BN));
   FfnArgs f;
-  f.g[0] = GemmArgs{a.tab1, a.f, a.d, nblk1, a.b1, static_cast<__nv_bfloat16 *>(a.hid), 1};
-  f.g[1] = GemmArgs{a.tab2, a.d, a.f, nblk2, a.b2, static_cast<__nv_bfloat16 *>(a.y_perm), 0};
+  MOE_TRY(tc::make_map_2d(&a1, a.x_perm, 2, (uint64_t)a.d, (uint64_t)a.S, BM));
+  MOE_TRY(tc::make_map_2d(&a2, a.hid, 2, (uint64_t)a.f, (uint64_t)a.S, BM));
+  if (!bwd) {
+    MOE_TRY(tc::make_map_2d(&b1, a.W1, 2, (uint64_t)a.d, (uint64_t)a.n * a.f, BN));
+    MOE_TRY(tc::make_map_2d(&b2, a.W2, 2, (uint64_t)a.f, (uint64_t)a.n * a.d, BN));
+    f.g[0] = GemmArgs{a.tab1, a.f, a.d, nblk1, a.b1, static_cast<__nv_bfloat16 *>(a.hid), 1, nullptr};
+    f.g[1] = GemmArgs{a.tab2, a.d, a.f, nblk2, a.b2, static_cast<__nv_bfloat16 *>(a.y_perm), 0,
+                      nullptr};
+  } else {
+    // dhid = (dy_perm W2_e) * [hid > 0]: B(n, k) = W2[e][k][n], rows e*d + k of [n*d][f];
+    // dx_perm = dhid W1_e: B(n, k) = W1[e][k][n], rows e*f + k of [n*f][d]
+    MOE_TRY(tc::make_map_2d(&b1, a.W2, 2, (uint64_t)a.f, (uint64_t)a.n * a.d, BK));
+    MOE_TRY(tc::make_map_2d(&b2, a.W1, 2, (uint64_t)a.d, (uint64_t)a.n * a.f, BK));
+    f.g[0] = GemmArgs{a.tab1, a.f, a.d, nblk1, nullptr, static_cast<__nv_bfloat16 *>(a.hid), 0,
+                      static_cast<const __nv_bfloat16 *>(a.mask)};
+    f.g[1] = GemmArgs{a.tab2, a.d, a.f, nblk2, nullptr, static_cast<__nv_bfloat16 *>(a.y_perm), 0,
+                      nullptr};
+  }
   f.mprefix = a.mprefix;
   f.n = a.n;
   f.mdone = a.mdone;
@@ -388,8 +444,9 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int slot = -1;
-  trace_begin(a.name ? a.name : "expert_ffn_tcgen05", st, &slot);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, expert_ffn_kernel, a1, b1, a2, b2, f);
+  trace_begin(a.name ? a.name : (bwd ? "expert_bwd_tcgen05" : "expert_ffn_tcgen05"), st, &slot);
+  const cudaError_t e = bwd ? cudaLaunchKernelEx(&cfg, expert_ffn_kernel<true>, a1, b1, a2, b2, f)
+                            : cudaLaunchKernelEx(&cfg, expert_ffn_kernel<false>, a1, b1, a2, b2, f);
   trace_end(slot, st);
   count_launch();
   return e == cudaSuccess ? MOE_OK : MOE_ECUDA;

@@ -92,6 +92,8 @@ struct RouteArgs {
   const float *sel_bias;   // sigmoid router: [nb] selection bias, or nullptr
   float *stats_part;       // [tiles][2] or nullptr: per tile, sum over rows of |c|^2
                            // and of the entropy of softmax(c)
+  int4 *kth;               // [R] or nullptr: per row {H of the (k+1)-th ranked, its id,
+                           // H of the k-th, its id} (H bits as int; -inf / INT_MAX if absent)
   int *status;
 };
 int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st);
@@ -160,6 +162,11 @@ struct ExpertArgs {
   void *hid;               // [S][f]
   void *y_perm;            // [S][d]
   int *status;
+  // backward (activation gradients, bf16 only): x_perm = dy_perm [S][d],
+  // hid = dhid [S][f] (written, then read), y_perm = dx_perm [S][d],
+  // mask = the forward's hid [S][f]; W1, W2 the forward's weights; no biases
+  int backward;
+  const void *mask;
 };
 int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st);
 int launch_expert_f32(const ExpertArgs &a, cudaStream_t st);
@@ -171,6 +178,61 @@ int launch_combine(const void *y_perm, int bf16, const float *gate, const int *r
                    const void *y_shared, cudaStream_t st);
 int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, float *bias,
                            cudaStream_t st);
+
+// ---- backward pass (backward.cu, wgrad_tc.cu, grad_gemm.cu)
+struct GateBwdArgs {
+  int T, n, k;
+  const float *c, *s;          // [T][n] clean logits, Softplus(x W_noise) of the forward
+  const int *idx;              // [T][k] kept experts, larger H first
+  const float *gate, *dgate;   // [T][k] gates and dL/dgate
+  const float *lam_imp, *lam_load, *sw_coef;  // [n] (bwd_coef)
+  const int4 *kth;             // [T] {H of the (k+1)-th, its id, H of the k-th, its id}
+  unsigned long long seed;
+  int router, noise, has_load;
+  float *dc, *dz;              // [T][n] outputs (dz: noise only)
+};
+int launch_bwd_coef(const float *importance, const float *load, const int *counts, int n, int T,
+                    float w_imp, float w_load, float alpha, int router, int noise, float *lam_imp,
+                    float *lam_load, float *sw_coef, cudaStream_t st);
+int launch_combine_bwd(const float *dy, const float *gate, const int *row_of, const void *y_perm,
+                       int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
+                       cudaStream_t st);
+int launch_dx_gather(const void *dx_perm, const int *row_of, const float *dy, int passthrough,
+                     int T, int k, int d, const void *dx_shared, float *dx, cudaStream_t st);
+int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,
+                     int f, float *db2, float *db1, const char *name, cudaStream_t st);
+int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st);
+int colsum_parts(int R);
+int launch_colsum(const float *X, int R, int N, float *part, float *out, cudaStream_t st);
+// weight gradients of the experts on the tensor cores, per expert e with rows
+// offsets[e] .. offsets[e+1]-1: dW2_e = dy_perm_e^T hid_e ([d][f]) and
+// dW1_e = dhid_e^T x_perm_e ([f][d]), fp32
+struct WgradArgs {
+  const void *dy_perm, *hid, *dhid, *x_perm;  // [S][d], [S][f], [S][f], [S][d] bf16
+  const int *offsets;                         // [n+1]
+  int n, d, f, S;
+  float *dW1, *dW2;
+  int *status;
+  const char *name;
+};
+int launch_wgrad_bf16(const WgradArgs &a, cudaStream_t st);
+// C[M][N] = sum_k A(m,k) B(k,n) (+ C when accumulate), fp32; A(m,k) =
+// A[m*lda+k] or, with at, A[k*lda+m]; B(k,n) = B[k*ldb+n] or, with bt,
+// B[n*ldb+k].  part: split-K scratch of splits*M*N floats (nullptr: no split).
+struct SgemmArgs {
+  int M, N, K;
+  const float *A;
+  int lda, at;
+  const float *B;
+  int ldb, bt;
+  float *C;
+  int ldc, accumulate;
+  float *part;
+  int splits;
+  const char *name;
+};
+int launch_sgemm(const SgemmArgs &a, cudaStream_t st);
+int sgemm_splits(int M, int N, int K);
 
 int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
                       cudaStream_t st);

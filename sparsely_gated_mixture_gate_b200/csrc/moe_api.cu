@@ -133,6 +133,10 @@ struct Layout {
   size_t x_shared, y_shared, shared_off;  // shared expert: input and output rows, {0, T}
   size_t shared_mprefix, shared_tab1, shared_tab2, shared_mdone;  // and its GEMM plan
   size_t xhi, xlo, whi, wlo;  // three-pass TF32 gate operands
+  // backward pass (cfg.backward): the forward's extra state, then scratch
+  size_t kth, hid_shared;
+  size_t dy_perm, dhid, dx_perm, dy_shared, dhid_shared, dx_shared, dgate, lam_imp, lam_load,
+      sw_coef, dc, dz, colsum_part, sgemm_part;
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
 };
@@ -240,6 +244,30 @@ Layout make_layout(const moe_config &c) {
     L.wlo = bp.take(4 * wrows * (size_t)c.d);
   } else {
     L.xhi = L.xlo = L.whi = L.wlo = 0;
+  }
+  L.kth = L.hid_shared = L.dy_perm = L.dhid = L.dx_perm = L.dy_shared = L.dhid_shared =
+      L.dx_shared = L.dgate = L.lam_imp = L.lam_load = L.sw_coef = L.dc = L.dz = L.colsum_part =
+          L.sgemm_part = 0;
+  if (c.backward) {
+    L.kth = bp.take(16 * T);
+    L.hid_shared = bp.take(c.shared_expert ? esz * T * (size_t)c.f : 0);
+    L.dy_perm = bp.take(esz * S * (size_t)c.d);
+    L.dhid = bp.take(esz * S * (size_t)c.f);
+    L.dx_perm = bp.take(esz * S * (size_t)c.d);
+    if (c.shared_expert) {
+      L.dy_shared = bp.take(esz * T * (size_t)c.d);
+      L.dhid_shared = bp.take(esz * T * (size_t)c.f);
+      L.dx_shared = bp.take(esz * T * (size_t)c.d);
+    }
+    L.dgate = bp.take(4 * S);
+    L.lam_imp = bp.take(4 * n);
+    L.lam_load = bp.take(4 * n);
+    L.sw_coef = bp.take(4 * n);
+    L.dc = bp.take(4 * T * n);
+    L.dz = bp.take(c.noise ? 4 * T * n : 0);
+    L.colsum_part = bp.take(4 * (size_t)colsum_parts(c.T) * n);
+    const size_t sp = (size_t)sgemm_splits(c.d, c.n, c.T);
+    L.sgemm_part = bp.take(sp > 1 ? 4 * sp * (size_t)c.d * n : 0);
   }
   L.total = bp.off;
   return L;
@@ -359,6 +387,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.load_part = at<float>(ws, L.load_part);
   r.sel_bias = (!hier && c.router == MOE_ROUTER_SIGMOID) ? gp.sel_bias : nullptr;
   r.stats_part = c.router_stats ? at<float>(ws, L.stats_part) : nullptr;  // flat / primary rows
+  r.kth = (c.backward && !hier) ? at<int4>(ws, L.kth) : nullptr;
   r.status = status;
   if (!hier) {
     r.k = c.k;
@@ -591,6 +620,7 @@ int moe_validate(const moe_config *c) {
   if (c->router == MOE_ROUTER_SIGMOID && (c->noise || c->hier_a)) return MOE_EINVAL;
   if (c->shared_expert != 0 && c->shared_expert != 1) return MOE_EINVAL;
   if (c->router_stats != 0 && c->router_stats != 1) return MOE_EINVAL;
+  if (c->backward != 0 && c->backward != 1) return MOE_EINVAL;
   if (c->noise != 0 && c->noise != 1) return MOE_EINVAL;
   if (c->expert_dtype != MOE_F32 && c->expert_dtype != MOE_BF16) return MOE_EINVAL;
   if (c->overflow_passthrough != 0 && c->overflow_passthrough != 1) return MOE_EINVAL;
@@ -763,7 +793,8 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
       e.W2 = ep->W2s;
       e.b1 = ep->b1s;
       e.b2 = ep->b2s;
-      e.hid = at<void>(ws, L.hid);
+      // the backward pass needs both hidden layers: the shared one then has its own rows
+      e.hid = at<void>(ws, c.backward ? L.hid_shared : L.hid);
       e.y_perm = y_shared;
       e.status = status;
       MOE_TRY(tc ? launch_expert_bf16(e, st) : launch_expert_f32(e, st));
@@ -772,6 +803,201 @@ int moe_forward(const moe_config *cfg, const float *x, const moe_gate_params *gp
                            c.overflow_passthrough, c.T, c.k, c.d, y, y_shared, st));
   }
   return stream_after(st, side->s, side->join);
+}
+
+int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *gp,
+                 const moe_expert_params *ep, const float *dy, const int32_t *topk_idx,
+                 const float *topk_gate, const float *importance, const float *load,
+                 const int32_t *counts, float *dx, const moe_grads *gr, void *ws,
+                 size_t ws_bytes, int32_t *status, moe_stream_t stream) {
+  Layout L;
+  MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
+  const moe_config &c = *cfg;
+  if (!c.backward || c.hier_a > 0 || c.expert_dtype != MOE_BF16) return MOE_EINVAL;
+  if (!gr || !gr->dW1 || !gr->dW2 || !importance || !load || !counts) return MOE_EINVAL;
+  if (!aligned(gr->dW1, 16) || !aligned(gr->dW2, 16)) return MOE_EINVAL;
+  if (c.T > 0 && (!x || !dy || !dx || !topk_idx || !topk_gate || !aligned(x, 16) ||
+                  !aligned(dy, 16) || !aligned(dx, 16)))
+    return MOE_EINVAL;
+  if (!gate_params_ok(c, gp) || !expert_params_ok(ep) || !shared_params_ok(c, ep))
+    return MOE_EINVAL;
+  if (c.shared_expert && (!gr->dW1s || !gr->dW2s || !aligned(gr->dW1s, 16) ||
+                          !aligned(gr->dW2s, 16)))
+    return MOE_EINVAL;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int T = c.T, d = c.d, n = c.n, k = c.k, f = c.f;
+  const size_t S = (size_t)T * k;
+  auto zero = [&](float *p, size_t cnt) -> int {
+    if (!p || cnt == 0) return MOE_OK;
+    return cudaMemsetAsync(p, 0, 4 * cnt, st) == cudaSuccess ? MOE_OK : MOE_ECUDA;
+  };
+  if (T == 0) {  // no tokens: every gradient is zero
+    MOE_TRY(zero(gr->dW_g, (size_t)d * n));
+    MOE_TRY(zero(gr->db_g, n));
+    if (c.noise) MOE_TRY(zero(gr->dW_noise, (size_t)d * n));
+    MOE_TRY(zero(gr->dW1, (size_t)n * f * d));
+    MOE_TRY(zero(gr->db1, (size_t)n * f));
+    MOE_TRY(zero(gr->dW2, (size_t)n * d * f));
+    MOE_TRY(zero(gr->db2, (size_t)n * d));
+    if (c.shared_expert) {
+      MOE_TRY(zero(gr->dW1s, (size_t)f * d));
+      MOE_TRY(zero(gr->db1s, f));
+      MOE_TRY(zero(gr->dW2s, (size_t)d * f));
+      MOE_TRY(zero(gr->db2s, d));
+    }
+    return MOE_OK;
+  }
+  const int *offsets = at<int>(ws, L.offsets);
+  const int *row_of = at<int>(ws, L.row_of);
+  void *dy_perm = at<void>(ws, L.dy_perm), *dhid = at<void>(ws, L.dhid);
+  void *dx_perm = at<void>(ws, L.dx_perm);
+  void *dy_sh = c.shared_expert ? at<void>(ws, L.dy_shared) : nullptr;
+  void *dhid_sh = c.shared_expert ? at<void>(ws, L.dhid_shared) : nullptr;
+  void *dx_sh = c.shared_expert ? at<void>(ws, L.dx_shared) : nullptr;
+  float *dgate = at<float>(ws, L.dgate);
+  float *lam_imp = at<float>(ws, L.lam_imp), *lam_load = at<float>(ws, L.lam_load);
+  float *sw_coef = at<float>(ws, L.sw_coef);
+  float *dc = at<float>(ws, L.dc), *dz = c.noise ? at<float>(ws, L.dz) : nullptr;
+
+  // ---- balancing losses -> dL/dImportance, dL/dLoad, Switch dL/dp
+  MOE_TRY(launch_bwd_coef(importance, load, counts, n, T, c.w_importance, c.w_load, c.alpha_aux,
+                          c.router, c.noise, lam_imp, lam_load, sw_coef, st));
+  // ---- combine: dy_perm rows, dL/dgate, the shared expert's rows
+  MOE_TRY(launch_combine_bwd(dy, topk_gate, row_of, at<void>(ws, L.y_perm), T, k, d, dy_perm,
+                             dgate, dy_sh, st));
+  // ---- experts: dhid = (dy_perm W2) * [hid > 0], dx_perm = dhid W1 (the forward's tiles)
+  const int64_t mb_upper = ceil_div((int64_t)S, kExpertBM) + n;
+  if (cudaMemsetAsync(at<int>(ws, L.mdone), 0, 4 * (size_t)(mb_upper + 1), st) != cudaSuccess)
+    return MOE_ECUDA;
+  ExpertArgs e{};
+  e.backward = 1;
+  e.x_perm = dy_perm;
+  e.offsets = offsets;
+  e.mprefix = at<int>(ws, L.mprefix);
+  e.tab1 = at<int4>(ws, L.tab1);
+  e.tab2 = at<int4>(ws, L.tab2);
+  e.mdone = at<int>(ws, L.mdone);
+  e.plan_ready = 1;
+  e.n = n;
+  e.d = d;
+  e.f = f;
+  e.S = (int)S;
+  e.W1 = ep->W1;
+  e.W2 = ep->W2;
+  e.hid = dhid;
+  e.y_perm = dx_perm;
+  e.mask = at<void>(ws, L.hid);
+  e.status = status;
+  MOE_TRY(launch_expert_bf16(e, st));
+  WgradArgs w{};
+  w.dy_perm = dy_perm;
+  w.hid = at<void>(ws, L.hid);
+  w.dhid = dhid;
+  w.x_perm = at<void>(ws, L.x_perm);
+  w.offsets = offsets;
+  w.n = n;
+  w.d = d;
+  w.f = f;
+  w.S = (int)S;
+  w.dW1 = gr->dW1;
+  w.dW2 = gr->dW2;
+  w.status = status;
+  MOE_TRY(launch_wgrad_bf16(w, st));
+  MOE_TRY(launch_bias_grad(dy_perm, dhid, offsets, n, d, f, gr->db2, gr->db1, nullptr, st));
+  if (c.shared_expert) {
+    const int64_t mbe = ceil_div((int64_t)T, kExpertBM);
+    if (cudaMemsetAsync(at<int>(ws, L.shared_mdone), 0, 4 * (size_t)(mbe + 1), st) != cudaSuccess)
+      return MOE_ECUDA;
+    ExpertArgs es = e;
+    es.name = "shared_expert_bwd_tcgen05";
+    es.x_perm = dy_sh;
+    es.offsets = at<int>(ws, L.shared_off);
+    es.mprefix = at<int>(ws, L.shared_mprefix);
+    es.tab1 = at<int4>(ws, L.shared_tab1);
+    es.tab2 = at<int4>(ws, L.shared_tab2);
+    es.mdone = at<int>(ws, L.shared_mdone);
+    es.n = 1;
+    es.S = T;
+    es.W1 = ep->W1s;
+    es.W2 = ep->W2s;
+    es.hid = dhid_sh;
+    es.y_perm = dx_sh;
+    es.mask = at<void>(ws, L.hid_shared);
+    MOE_TRY(launch_expert_bf16(es, st));
+    WgradArgs ws2 = w;
+    ws2.name = "shared_wgrad_tcgen05";
+    ws2.dy_perm = dy_sh;
+    ws2.hid = at<void>(ws, L.hid_shared);
+    ws2.dhid = dhid_sh;
+    ws2.x_perm = at<void>(ws, L.x_shared);
+    ws2.offsets = at<int>(ws, L.shared_off);
+    ws2.n = 1;
+    ws2.S = T;
+    ws2.dW1 = gr->dW1s;
+    ws2.dW2 = gr->dW2s;
+    MOE_TRY(launch_wgrad_bf16(ws2, st));
+    MOE_TRY(launch_bias_grad(dy_sh, dhid_sh, at<int>(ws, L.shared_off), 1, d, f, gr->db2s,
+                             gr->db1s, "shared_bias_grad", st));
+  }
+  // ---- dispatch: dx = sum of the token's expert rows (+ pass-through, + shared)
+  MOE_TRY(launch_dx_gather(dx_perm, row_of, dy, c.overflow_passthrough, T, k, d, dx_sh, dx, st));
+  // ---- gate: dL/dc, dL/dz per token, then the fp32 contractions
+  GateBwdArgs g{};
+  g.T = T;
+  g.n = n;
+  g.k = k;
+  g.c = at<float>(ws, L.c);
+  g.s = at<float>(ws, L.s);
+  g.idx = topk_idx;
+  g.gate = topk_gate;
+  g.dgate = dgate;
+  g.lam_imp = lam_imp;
+  g.lam_load = lam_load;
+  g.sw_coef = sw_coef;
+  g.kth = at<int4>(ws, L.kth);
+  g.seed = c.seed;
+  g.router = c.router;
+  g.noise = c.noise;
+  g.has_load = c.noise && c.w_load != 0.f;
+  g.dc = dc;
+  g.dz = dz;
+  MOE_TRY(launch_gate_bwd(g, st));
+  if (gr->db_g) MOE_TRY(launch_colsum(dc, T, n, at<float>(ws, L.colsum_part), gr->db_g, st));
+  float *sp = at<float>(ws, L.sgemm_part);
+  const int splits = sgemm_splits(d, n, T);
+  for (int q = 0; q < (c.noise ? 2 : 1); ++q) {
+    const float *G = q ? dz : dc;
+    const float *W = q ? gp->W_noise : gp->W_g;
+    float *dW = q ? gr->dW_noise : gr->dW_g;
+    if (dW) {  // dW = x^T G: M = d, N = n, K = T
+      SgemmArgs a{};
+      a.M = d; a.N = n; a.K = T;
+      a.A = x; a.lda = d; a.at = 1;
+      a.B = G; a.ldb = n; a.bt = 0;
+      a.C = dW; a.ldc = n; a.accumulate = 0;
+      a.part = splits > 1 ? sp : nullptr;
+      a.splits = splits;
+      a.name = "gate_wgrad_fp32";
+      MOE_TRY(launch_sgemm(a, st));
+    }
+    // dx += G W^T: M = T, N = d, K = n; B(k, q) = W[q][k]
+    SgemmArgs a{};
+    a.M = T; a.N = d; a.K = n;
+    a.A = G; a.lda = n; a.at = 0;
+    a.B = W; a.ldb = n; a.bt = 1;
+    a.C = dx; a.ldc = d; a.accumulate = 1;
+    a.part = nullptr;
+    a.splits = 1;
+    a.name = "gate_dgrad_fp32";
+    MOE_TRY(launch_sgemm(a, st));
+  }
+  if (gr->dgate &&
+      cudaMemcpyAsync(gr->dgate, dgate, 4 * S, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ECUDA;
+  if (gr->dlogits && cudaMemcpyAsync(gr->dlogits, dc, 4 * (size_t)T * n,
+                                     cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+    return MOE_ECUDA;
+  return MOE_OK;
 }
 
 int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,

@@ -265,6 +265,9 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
           if (S[j].i >= 0 && S[j].i < nb) kept_s[w][S[j].i >> 5] |= 1u << (S[j].i & 31);
         thr_s[w][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
         thr_s[w][1] = S[K1 - 2].v;
+        if (a.kth)  // kept for the backward pass's load gradient
+          a.kth[row] = make_int4(__float_as_int(S[K1 - 1].v), S[K1 - 1].i,
+                                 __float_as_int(S[K1 - 2].v), S[K1 - 2].i);
         sm_s[w][0] = M;
         sm_s[w][1] = SE;
       }
@@ -459,7 +462,7 @@ int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st) {
     return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), 0, st, a);
   };
   const bool wide = a.nb > 4 * 4 * NW * 32;  // more than 4096 columns
-  const bool st_on = a.stats_part != nullptr;
+  const bool st_on = a.stats_part != nullptr || a.kth != nullptr;  // the EX instances
   if (a.router == MOE_ROUTER_SWITCH) {
     if (a.k != 1 || wide) return MOE_EINVAL;
     return st_on ? go(route_kernel<2, 4, true, true>) : go(route_kernel<2, 4, true, false>);

@@ -50,6 +50,7 @@ class Config:
     gate_precision: int = 0   # 0: fp32 multiply-adds, 1: tensor cores, 3-pass TF32 split
     shared_expert: int = 0    # 1: one always-active expert (W1s, b1s, W2s, b2s) in forward
     router_stats: int = 0     # 1: forward reports the router z-loss and entropy (losses[8:10])
+    backward: int = 0         # 1: the layer also runs the backward pass (workspace, saved state)
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -67,7 +68,7 @@ class Config:
                           overflow_passthrough=self.passthrough, w_importance=self.w_importance,
                           w_load=self.w_load, alpha_aux=self.alpha,
                           gate_precision=self.gate_precision, shared_expert=self.shared_expert,
-                          router_stats=self.router_stats)
+                          router_stats=self.router_stats, backward=self.backward)
 
     @property
     def expert_dtype(self):
@@ -303,6 +304,47 @@ class MoELayer:
                                        _ptr(losses), _ptr(self.ws), self.ws.numel(),
                                        _ptr(self.status), st), "moe_forward")
         return y
+
+    def grads(self, intermediates: bool = False) -> dict:
+        """Gradient buffers of this layer (allocated on first use), fp32 in
+        the parameters' layouts; with intermediates also dgate [T][k] and
+        dlogits [T][n]."""
+        if not hasattr(self, "_grads"):
+            cfg, dev = self.cfg, self.device
+            z = lambda *shape: torch.zeros(*shape, dtype=torch.float32, device=dev)
+            g = dict(dx=z(cfg.T, cfg.d), dWg=z(cfg.d, cfg.n), dbg=z(cfg.n),
+                     dW1=z(cfg.n, cfg.f, cfg.d), db1=z(cfg.n, cfg.f), dW2=z(cfg.n, cfg.d, cfg.f),
+                     db2=z(cfg.n, cfg.d))
+            if cfg.noise:
+                g["dWn"] = z(cfg.d, cfg.n)
+            if cfg.shared_expert:
+                g.update(dW1s=z(cfg.f, cfg.d), db1s=z(cfg.f), dW2s=z(cfg.d, cfg.f), db2s=z(cfg.d))
+            if intermediates:
+                g.update(dgate=z(cfg.T, cfg.k), dlogits=z(cfg.T, cfg.n))
+            self._grads = g
+            self._mg = _lib.moe_grads(
+                dW_g=_ptr(g["dWg"]), db_g=_ptr(g["dbg"]), dW_noise=_ptr(g.get("dWn")),
+                dW1=_ptr(g["dW1"]), db1=_ptr(g["db1"]), dW2=_ptr(g["dW2"]), db2=_ptr(g["db2"]),
+                dW1s=_ptr(g.get("dW1s")), db1s=_ptr(g.get("db1s")), dW2s=_ptr(g.get("dW2s")),
+                db2s=_ptr(g.get("db2s")), dgate=_ptr(g.get("dgate")), dlogits=_ptr(g.get("dlogits")))
+        return self._grads
+
+    def backward_(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
+        """Gradients of sum(dy * y) + the weighted balancing losses of the last
+        forward_ (same x) into the buffers of grads(); asynchronous."""
+        if not self.cfg.backward:
+            raise MoEError("the layer was built without backward=1")
+        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        _need(dy, "dy", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        g = self.grads()
+        st = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+        _check(_lib.load().moe_backward(C.byref(self._c), _ptr(x), C.byref(self._gp),
+                                        C.byref(self._ep), _ptr(dy), _ptr(self.topk_idx),
+                                        _ptr(self.topk_gate), _ptr(self.importance),
+                                        _ptr(self.load), _ptr(self.counts), _ptr(g["dx"]),
+                                        C.byref(self._mg), _ptr(self.ws), self.ws.numel(),
+                                        _ptr(self.status), st), "moe_backward")
+        return g
 
     def outputs(self) -> dict:
         return dict(y=self.y, topk_idx=self.topk_idx, topk_gate=self.topk_gate,

@@ -172,6 +172,14 @@ def make_inputs(w: Workload, device="cpu", T: Optional[int] = None, seed: Option
     return out
 
 
+def make_dy(w: Workload, device="cpu", T: Optional[int] = None, seed: Optional[int] = None):
+    """Upstream gradient of the layer output for the backward pass: [T][d]
+    standard normal (the first T rows are the same for any T)."""
+    s = w.seed if seed is None else seed
+    T = w.T if T is None else T
+    return _randn((w.T, w.d), 1.0, device, s, 17)[:T].contiguous()
+
+
 def random_routing(T: int, k: int, n: int, device="cpu", seed: int = 0, skew: float = 0.0,
                    invalid_frac: float = 0.0) -> torch.Tensor:
     """Synthetic expert choices [T][k] for stand-alone dispatch tests: k

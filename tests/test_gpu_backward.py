@@ -1,0 +1,162 @@
+"""GPU parity of the backward pass (moe_backward through the C ABI) against
+the oracle's backward in its bf16 mode, on the same seeded inputs.
+
+The oracle takes the kernels' rounding points (bf16 expert-row gradients,
+hidden-layer gradient and input-row gradients; fp32 gates), so what remains
+is fp32-versus-fp64 accumulation order and the odd bf16 rounding that lands
+on the other side of a tie: every gradient within 1e-2 relative Frobenius
+of the oracle's (bf16 carries 8 bits), the gate gradient dL/dgate within
+5e-3.  Cases whose routing has near ties (k-th and (k+1)-th logits closer
+than 1e-5) are skipped: a flipped choice changes the whole token."""
+import dataclasses
+
+import numpy as np
+import pytest
+import torch
+
+from sparsely_gated_mixture_gate_b200 import build, synth
+from sparsely_gated_mixture_gate_b200 import moe as M
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+TIE = 1e-5
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    build.build()
+
+
+def to_dev(inp):
+    return {k: (v.to(DEV) if v is not None else None) for k, v in inp.items()}
+
+
+def np_inputs(inp):
+    out = {}
+    for k, v in inp.items():
+        if v is None:
+            out[k] = None
+        elif v.dtype == torch.bfloat16:
+            out[k] = synth.bf16_bits(v)
+        else:
+            out[k] = v.detach().cpu().numpy()
+    return out
+
+
+def rel_fro(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+
+
+W = synth.WORKLOADS
+V = synth.VARIANTS
+LOSSES = dict(w_importance=0.3, w_load=0.4)
+CASES = {
+    # noisy top-k, ragged d and f (not multiples of 64), capacity drops and pass-through
+    "noisy-ragged-capacity": W["lm-flat"].with_(T=300, n=24, k=2, d=200, f=136, capacity_factor=1.0,
+                                                passthrough=1, bias_var=0.1, logit_bias_var=0.1,
+                                                **LOSSES),
+    # the lm-flat layer's shape on 512 tokens: about 8 rows per expert, so nearly every
+    # weight-gradient K loop ends in a partial 16-row step
+    "lm-flat-512": W["lm-flat"].with_(T=512, **LOSSES),
+    "noise-free": W["lm-flat"].with_(T=256, n=16, k=2, d=64, f=64, noise=0, **LOSSES),
+    "k1-noisy": W["lm-flat"].with_(T=333, n=8, k=1, d=64, f=192, **LOSSES),
+    "kn-equal": W["tiny-flat"].with_(T=65, n=3, k=3, d=16, f=24, expert_bf16=1, **LOSSES),
+    "empty-experts": W["lm-flat"].with_(T=40, n=64, k=1, d=64, f=64, **LOSSES),
+    "many-rows": W["lm-flat"].with_(T=2048, n=4, k=2, d=128, f=256, **LOSSES),
+    "switch-capacity": V["switch-skew"].with_(T=1024, d=128, n=16, f=128, alpha=0.5,
+                                              w_importance=0.3),
+    "sigmoid-shared": V["deepseek-tiny"].with_(w_importance=0.3),
+    "sigmoid-shared-256": V["deepseek-flat"].with_(T=256, d=128, n=32, k=4, f=128,
+                                                   w_importance=0.3),
+    "shared-noisy-passthrough": W["lm-flat"].with_(T=200, n=32, k=2, d=64, f=64, shared_expert=1,
+                                                   capacity_factor=0.5, passthrough=1, **LOSSES),
+}
+
+GRAD_KEYS = [("dx", "dx"), ("dWg", "dWg"), ("dbg", "dbg"), ("dWn", "dWn"), ("dW1", "dW1"),
+             ("db1", "db1"), ("dW2", "dW2"), ("db2", "db2"), ("dW1s", "dW1s"), ("db1s", "db1s"),
+             ("dW2s", "dW2s"), ("db2s", "db2s"), ("dlogits", "dlogits")]
+
+
+def run_backward(w, inp, dy):
+    cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
+    dinp = to_dev(inp)
+    layer = M.MoELayer(cfg, dinp, torch.device(DEV))
+    x = dinp["x"]
+    layer.forward_(x)
+    layer.grads(intermediates=True)
+    g = layer.backward_(x, dy.to(DEV))
+    torch.cuda.synchronize()
+    out = {k: v.cpu().numpy() for k, v in g.items()}
+    fwd = {k: v.cpu() for k, v in layer.outputs().items()}
+    return out, fwd
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_backward_matches_oracle(orc, name):
+    w = CASES[name]
+    inp = synth.make_inputs(w)
+    dy = synth.make_dy(w)
+    got, fwd = run_backward(w, inp, dy)
+    assert M.status_bits(fwd["status"]) == 0
+    ref_f = orc.forward(w.cfg(), np_inputs(inp))
+    nt = int((ref_f["near_tie"] < TIE).sum())
+    if nt:
+        pytest.skip(f"{nt} near-tie tokens")
+    assert np.array_equal(fwd["topk_idx"].numpy(), ref_f["topk_idx"])
+    assert np.array_equal(fwd["counts"].numpy(), ref_f["counts"])
+    ref = orc.backward(w.cfg(), np_inputs(inp), dy.numpy())
+    assert rel_fro(got["dgate"], ref["dgate"]) < 5e-3
+    for gk, rk in GRAD_KEYS:
+        if gk not in got or rk not in ref:
+            continue
+        if not np.any(ref[rk]) and not np.any(got[gk]):
+            continue
+        err = rel_fro(got[gk], ref[rk])
+        assert err < 1e-2, (gk, err)
+    # experts that received no rows get exactly zero weight gradients
+    empty = np.flatnonzero(ref_f["counts"] == 0)
+    assert not np.any(got["dW1"][empty]) and not np.any(got["dW2"][empty])
+
+
+def test_backward_is_deterministic():
+    w = CASES["noisy-ragged-capacity"]
+    inp = synth.make_inputs(w)
+    dy = synth.make_dy(w)
+    a, _ = run_backward(w, inp, dy)
+    b, _ = run_backward(w, inp, dy)
+    for k in a:
+        assert np.array_equal(a[k].view(np.uint32), b[k].view(np.uint32)), k
+
+
+def test_backward_zero_tokens():
+    w = CASES["noise-free"].with_(T=0)
+    inp = synth.make_inputs(w)
+    cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
+    layer = M.MoELayer(cfg, to_dev(inp), torch.device(DEV))
+    x = torch.zeros(0, w.d, device=DEV)
+    layer.forward_(x)
+    g = layer.grads()
+    for v in g.values():
+        v.fill_(7.0)
+    layer.backward_(x, torch.zeros(0, w.d, device=DEV))
+    torch.cuda.synchronize()
+    for k, v in g.items():
+        if k != "dx":
+            assert torch.all(v == 0), k
+
+
+def test_backward_requires_flag_and_bf16():
+    w = CASES["noise-free"]
+    inp = to_dev(synth.make_inputs(w))
+    layer = M.MoELayer(M.Config.from_workload(w), inp, torch.device(DEV))
+    with pytest.raises(M.MoEError):
+        layer.backward_(inp["x"], torch.zeros_like(inp["x"]))
+    w32 = w.with_(expert_bf16=0)
+    inp32 = to_dev(synth.make_inputs(w32))
+    cfg32 = dataclasses.replace(M.Config.from_workload(w32), backward=1)
+    layer32 = M.MoELayer(cfg32, inp32, torch.device(DEV))
+    layer32.forward_(inp32["x"])
+    with pytest.raises(M.MoEError):
+        layer32.backward_(inp32["x"], torch.zeros_like(inp32["x"]))
