@@ -17,10 +17,15 @@ its own launches), the expert-FFN TFLOP/s and routing GB/s of the metric,
 clocks sampled during the timed region, the count of library kernel launches,
 and the oracle's CPU baseline on a bounded sample.  ``--impl reference`` times
 the oracle itself (the reference arm of this comparison).
+
+``--backward``: one step is the forward pass followed by the backward pass
+(``moe_backward``: dx and every parameter's gradient for an upstream gradient
+dy plus the weighted balancing losses); the metric is then training tokens/s.
 """
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -36,6 +41,7 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 METRIC = "MoE-layer fwd tokens/s; expert-FFN TFLOP/s vs bf16 peak; routing HBM GB/s"
+METRIC_TRAIN = "MoE-layer training tokens/s (forward + backward, all gradients)"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
                   "sm_max_mhz": 1965.0}
@@ -135,7 +141,11 @@ def src_sha(name: str) -> str:
 
 KERNEL_SRC = {"expert_ffn_tcgen05": "expert_tc.cu",
               "gate_gemm_fp32": "gate_gemm.cu", "route_topk": "route.cu", "combine": "combine.cu",
-              "dispatch_place": "dispatch.cu", "dispatch_hist": "dispatch.cu"}
+              "dispatch_place": "dispatch.cu", "dispatch_hist": "dispatch.cu",
+              "expert_bwd_tcgen05": "expert_tc.cu", "wgrad_tcgen05": "wgrad_tc.cu",
+              "gate_wgrad_fp32": "grad_gemm.cu", "gate_dgrad_fp32": "grad_gemm.cu",
+              "combine_bwd": "backward.cu", "dx_gather": "backward.cu", "gate_bwd": "backward.cu",
+              "bias_grad": "backward.cu"}
 
 
 def ncu_traffic(kernel: str, workload: str):
@@ -175,6 +185,25 @@ def kernel_work(w, name: str, S_kept: int):
     if name == "expert_ffn_fp32":
         # both layers of every expert on its rows, fp32 weights streamed once
         return "hbm", 4.0 * S_kept * d * f, n * 2 * d * f * 4 + S_kept * d * 4 * 2
+    # ---- backward pass
+    if name == "expert_bwd_tcgen05":
+        # dhid = (dy_perm W2) * mask, dx_perm = dhid W1: both weights once, dy_perm and the
+        # forward's hid in, dhid (needed again by the weight gradients) and dx_perm out
+        return "tensor", 4.0 * S_kept * d * f, \
+            n * 2 * d * f * esz + S_kept * (2 * d + 2 * f) * esz
+    if name == "wgrad_tcgen05":
+        # dW2 = dy_perm^T hid, dW1 = dhid^T x_perm per expert: four activations in, fp32 out
+        return "tensor", 4.0 * S_kept * d * f, S_kept * 2 * (d + f) * esz + n * 2 * d * f * 4
+    if name == "combine_bwd":
+        return "hbm", 0.0, T * d * 4 + 2 * S_kept * d * esz + 12 * T * k
+    if name == "dx_gather":
+        return "hbm", 0.0, S_kept * d * esz + T * d * 4 + 4 * T * k
+    if name == "bias_grad":
+        return "hbm", 0.0, S_kept * (d + f) * esz + n * (d + f) * 4
+    if name == "gate_bwd":
+        return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) * 2 + 16 * T * k + 16 * T
+    if name in ("gate_wgrad_fp32", "gate_dgrad_fp32"):
+        return "alu", 2.0 * T * d * ng, 4 * (T * d + d * ng + T * ng)
     if name == "route_topk":
         return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
     if name == "combine":
@@ -202,14 +231,22 @@ def run_ours(args, w, world, rank, local):
     if rank:
         inp["x"] = synth.make_inputs(w.with_(seed=rank), device=dev, experts=False)["x"]
     cfg = M.Config.from_workload(w)
+    if args.backward:
+        cfg = dataclasses.replace(cfg, backward=1)
     layer = M.MoELayer(cfg, inp, dev)
     x = inp["x"]
+    dy = synth.make_dy(w.with_(seed=w.seed + rank), device=dev) if args.backward else None
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    def step():
+        layer.forward_(x)
+        if dy is not None:
+            layer.backward_(x, dy)
+
     for _ in range(args.warmup):
         flush.fill_(1.0)
-        layer.forward_(x)
+        step()
     torch.cuda.synchronize()
     st = M.status_bits(layer.status)
     if st:
@@ -229,7 +266,7 @@ def run_ours(args, w, world, rank, local):
     for i in range(args.steps):
         flush.fill_(float(i))
         starts[i].record(stream)
-        layer.forward_(x)
+        step()
         ends[i].record(stream)
     torch.cuda.synchronize()
     if world > 1:
@@ -249,7 +286,7 @@ def run_ours(args, w, world, rank, local):
     torch.cuda.synchronize()
     for i in range(t_steps):
         flush.fill_(float(i))
-        layer.forward_(x)
+        step()
     torch.cuda.synchronize()
     M.trace_enable(False)
     per_kernel = M.trace_read()
@@ -261,24 +298,58 @@ def run_ours(args, w, world, rank, local):
     xh = x.cpu().pin_memory()
     yh = [torch.empty(w.T, w.d, dtype=torch.float32).pin_memory() for _ in range(2)]
     lh = [torch.empty(layer.losses.numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
-    layer.forward_host_batches([xh] * 3, [yh[i & 1] for i in range(3)], [lh[i & 1] for i in range(3)])
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    d2h = layer.forward_host_batches([xh] * e_steps, [yh[i & 1] for i in range(e_steps)],
-                                     [lh[i & 1] for i in range(e_steps)])
-    stream.wait_stream(d2h)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    if dy is None:
+        layer.forward_host_batches([xh] * 3, [yh[i & 1] for i in range(3)],
+                                   [lh[i & 1] for i in range(3)])
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        d2h = layer.forward_host_batches([xh] * e_steps, [yh[i & 1] for i in range(e_steps)],
+                                         [lh[i & 1] for i in range(e_steps)])
+        stream.wait_stream(d2h)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        h2d_bytes, d2h_bytes = w.T * w.d * 4, w.T * w.d * 4 + 4 * layer.losses.numel()
+    else:
+        # training step from host memory: x and dy in, y, the losses and dx out
+        # (the parameter gradients stay on the device for the optimizer)
+        dyh = dy.cpu().pin_memory()
+        dxh = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
+        xd, dyd = torch.empty_like(x), torch.empty_like(dy)
+        dx = layer.grads()["dx"]
+
+        def host_step(i):
+            xd.copy_(xh, non_blocking=True)
+            dyd.copy_(dyh, non_blocking=True)
+            layer.forward_(xd)
+            layer.backward_(xd, dyd)
+            yh[i & 1].copy_(layer.y, non_blocking=True)
+            lh[i & 1].copy_(layer.losses, non_blocking=True)
+            dxh.copy_(dx, non_blocking=True)
+
+        for i in range(3):
+            host_step(i)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e_steps):
+            host_step(i)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        h2d_bytes = 2 * w.T * w.d * 4
+        d2h_bytes = 2 * w.T * w.d * 4 + 4 * layer.losses.numel()
     e_ms, e_value = aggregate(e0.elapsed_time(e1), w.T, e_steps, world)
     st = M.status_bits(layer.status)
 
     # ---- the other gate mode on the same weights (short run, reported apart)
     alt = None
-    if args.alt_gate and world == 1:
+    if args.alt_gate and world == 1 and dy is None:
         other = 0 if w.gate_precision else 1
         alt_layer = M.MoELayer(M.Config.from_workload(w.with_(gate_precision=other)), inp, dev)
         for _ in range(3):
@@ -362,11 +433,13 @@ def run_ours(args, w, world, rank, local):
     route_bytes = sum(kernel_work(w, k, S_kept)[2] for k in route_names)
 
     line = {
-        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "metric": METRIC_TRAIN if dy is not None else METRIC, "value": round(value, 1),
+        "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32",
         "data": "synthetic (seeded; random-init weights of the workload's shapes)",
-        "config": {"workload": w.name, "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k,
+        "config": {"workload": w.name + (" (forward + backward)" if dy is not None else ""),
+                   "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k,
                    "d_ff": w.f, "hier": [w.hier_a, w.hier_b] if w.hier_a else None,
                    "router": "switch-top1" if w.router else "noisy-top-k",
                    "gate": "3-pass TF32 on tensor cores (fp32-level)" if w.gate_precision
@@ -381,10 +454,12 @@ def run_ours(args, w, world, rank, local):
         "kernels": kstats,
         "kernel_timing": f"second pass of {t_steps} steps, CUDA events around every library launch",
         "gpu_launches": int(launches),
-        "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": w.T * w.d * 4,
-                "d2h_bytes_per_step": w.T * w.d * 4 + 4 * layer.losses.numel(), "steps": e_steps,
-                "how": "pinned host x in, y and losses out every step; copies of neighbouring "
-                       "steps overlap compute on two copy streams"},
+        "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
+                "d2h_bytes_per_step": d2h_bytes, "steps": e_steps,
+                "how": ("pinned host x in, y and losses out every step; copies of neighbouring "
+                        "steps overlap compute on two copy streams") if dy is None else
+                       ("pinned host x and dy in, y, losses and dx out every step, on the "
+                        "compute stream (parameter gradients stay on the device)")},
         "clocks": clk,
         "alt_gate_mode": alt,
         "wall_s": round(wall, 3),
@@ -402,46 +477,62 @@ def oracle_sample_inputs(w, T_s):
             for k, v in inp.items()}
 
 
-def time_oracle(w, T_s, reps=1):
+def oracle_step(w, T_s, backward=False):
+    """One oracle step on the first T_s tokens: the forward pass, and with
+    backward the backward pass too (as a function of no arguments)."""
     from oracle import oracle as orc
     orc.build()
     npin = oracle_sample_inputs(w, T_s)
     cfg = dict(w.cfg(), T=T_s)
+    if not backward:
+        return lambda: orc.forward(cfg, npin)
+    from sparsely_gated_mixture_gate_b200 import synth
+    dy = synth.make_dy(w, T=T_s).numpy()
+
+    def both():
+        orc.forward(cfg, npin)
+        orc.backward(cfg, npin, dy)
+    return both
+
+
+def time_oracle(w, T_s, reps=1, backward=False):
+    fn = oracle_step(w, T_s, backward)
     t0 = time.perf_counter()
     for _ in range(reps):
-        orc.forward(cfg, npin)
+        fn()
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, budget_s=12.0):
+def cpu_baseline(w, budget_s=12.0, backward=False):
     """The oracle (single-threaded C, as it stands) on the first tokens of the
     workload: calibrate on 8 tokens, then run a sample of about budget_s."""
-    t8 = time_oracle(w, 8)
+    t8 = time_oracle(w, 8, backward=backward)
     T_s = int(max(8, min(w.T, budget_s / max(t8 / 8, 1e-6))))
-    t = time_oracle(w, T_s)
+    t = time_oracle(w, T_s, backward=backward)
+    what = "forward + backward" if backward else "forward"
     return {"value": round(T_s / t, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
-            "sample": f"first {T_s} tokens of {w.name} as one batch (same weights), {t:.1f} s"}
+            "sample": f"{what} of the first {T_s} tokens of {w.name} as one batch "
+                      f"(same weights), {t:.1f} s"}
 
 
 def run_reference(args, w):
     """The reference arm: the oracle itself, each step a bounded sample of the
     workload sized so the whole run stays within about two minutes."""
-    t8 = time_oracle(w, 8)
+    t8 = time_oracle(w, 8, backward=args.backward)
     per_tok = max(t8 / 8, 1e-6)
     budget = 90.0 / max(args.steps + args.warmup, 1)
     T_s = int(max(1, min(w.T, budget / per_tok)))
-    from oracle import oracle as orc
-    npin = oracle_sample_inputs(w, T_s)
-    cfg = dict(w.cfg(), T=T_s)
+    fn = oracle_step(w, T_s, args.backward)
     for _ in range(args.warmup):
-        orc.forward(cfg, npin)
+        fn()
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        orc.forward(cfg, npin)
+        fn()
     t = time.perf_counter() - t0
     value = T_s * args.steps / t
     sample = f"first {T_s} tokens of {w.name} per step (same weights)"
-    return {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+    return {"impl": "reference", "metric": METRIC_TRAIN if args.backward else METRIC,
+            "value": round(value, 3), "unit": "tokens/s",
             "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": round(t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -463,6 +554,8 @@ def main():
     ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
                     help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward", action="store_true",
+                    help="time forward + backward (training step) instead of the forward pass")
     ap.add_argument("--no-alt-gate", dest="alt_gate", action="store_false",
                     help="skip the short run of the other gate mode")
     args = ap.parse_args()
@@ -488,7 +581,7 @@ def main():
         line = run_ours(args, w, world, rank, local)
         if rank == 0 and line is not None:
             if world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(w)
+                line["cpu_baseline"] = cpu_baseline(w, backward=args.backward)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

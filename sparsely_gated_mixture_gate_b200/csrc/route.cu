@@ -58,8 +58,10 @@ __device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
 
 // K1 = k + 1; MAXQ = column quads per thread (nb <= MAXQ * 4 * 256); SW =
 // Switch router (probability sums kept).
-// ST = router statistics (stats_part written).
-template <int K1, int MAXQ, bool SW, bool ST>
+// EX = extra outputs compiled in: the router statistics (stats_part) and the
+// rows' thresholds for the backward pass (kth), each only when its pointer is
+// set.
+template <int K1, int MAXQ, bool SW, bool EX>
 __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
   constexpr int KM = K1 - 1;  // k
   constexpr int PQ = SW ? MAXQ : 1;
@@ -112,7 +114,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
 #pragma unroll
     for (int j = 0; j < 4; ++j) pacc[u][j] = 0.f;
 
-  constexpr bool stats = ST;
+  const bool stats = EX && a.stats_part != nullptr;
   float rz = 0.f, rh = 0.f;  // lane 0: this warp's rows' |c|^2 and entropies
   const int nwords = (nb + 31) >> 5;
   for (int rb = row0; rb < row_end; rb += NW) {
@@ -265,7 +267,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
           if (S[j].i >= 0 && S[j].i < nb) kept_s[w][S[j].i >> 5] |= 1u << (S[j].i & 31);
         thr_s[w][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
         thr_s[w][1] = S[K1 - 2].v;
-        if (a.kth)  // kept for the backward pass's load gradient
+        if (EX && a.kth)  // kept for the backward pass's load gradient
           a.kth[row] = make_int4(__float_as_int(S[K1 - 1].v), S[K1 - 1].i,
                                  __float_as_int(S[K1 - 2].v), S[K1 - 2].i);
         sm_s[w][0] = M;
