@@ -203,7 +203,9 @@ def kernel_work(w, name: str, S_kept: int):
     if name == "gate_bwd":
         return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) * 2 + 16 * T * k + 16 * T
     if name in ("gate_wgrad_fp32", "gate_dgrad_fp32"):
-        return "alu", 2.0 * T * d * ng, 4 * (T * d + d * ng + T * ng)
+        # one launch carries the clean and the noise products (two with noise)
+        nprod = 2 if w.noise else 1
+        return "alu", nprod * 2.0 * T * d * ng, 4 * (T * d + nprod * (d * ng + T * ng))
     if name == "route_topk":
         return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
     if name == "combine":

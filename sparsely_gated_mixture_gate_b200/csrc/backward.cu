@@ -27,7 +27,7 @@
 namespace moe {
 namespace {
 
-constexpr int CT = 1024;
+constexpr int CT = 256;
 
 __device__ double block_sum_d(double v, double *sh) {
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -226,6 +226,7 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(
   const int r0 = offsets[e], r1 = offsets[e + 1];
   float a[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
   if (c0 < N) {
+#pragma unroll 4
     for (int r = r0 + rg; r < r1; r += 8) {
       float v[8];
       bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(src + (size_t)r * N + c0)), v);
@@ -428,7 +429,8 @@ __global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ X
   if (j >= N) return;
   const int r0 = blockIdx.y * rows_per, r1 = min(r0 + rows_per, R);
   float s = 0.f;
-  for (int r = r0; r < r1; ++r) s += X[(size_t)r * N + j];
+#pragma unroll 4
+  for (int r = r0; r < r1; ++r) s += __ldg(X + (size_t)r * N + j);
   part[(size_t)blockIdx.y * N + j] = s;
 }
 
@@ -491,10 +493,17 @@ int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st) {
   return go(gate_bwd_kernel<8>);
 }
 
-int colsum_parts(int R) { return R <= 0 ? 0 : (int)ceil_div(R, 256) < 64 ? (int)ceil_div(R, 256) : 64; }
+// row blocks of at least 16 rows, about two blocks per SM over all column blocks
+int colsum_parts(int R, int N) {
+  if (R <= 0) return 0;
+  const int cb = (int)ceil_div(N, 256);
+  const int want = (int)ceil_div(2 * num_sms(), cb);
+  const int most = (int)ceil_div(R, 16);
+  return want < most ? (want > 0 ? want : 1) : most;
+}
 
 int launch_colsum(const float *X, int R, int N, float *part, float *out, cudaStream_t st) {
-  const int parts = colsum_parts(R);
+  const int parts = colsum_parts(R, N);
   if (parts == 0) {
     return cudaMemsetAsync(out, 0, 4 * (size_t)N, st) == cudaSuccess ? MOE_OK : MOE_ECUDA;
   }

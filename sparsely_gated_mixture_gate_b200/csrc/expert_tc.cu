@@ -276,6 +276,22 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       // staged, the stores go out four rows at a time (rows rr, columns cc*8)
       __nv_bfloat16 *const dtile = g.D + (size_t)(ti.y + q * 32) * g.N;
       const int rows_here = ti.z - q * 32;  // valid rows of this warp (may be <= 0)
+      // ReLU mask of the backward pass: this lane's row of hid, 64 columns of
+      // chunk c; chunk 0's is loaded before the wait, chunk 1's while chunk 0
+      // is stored
+      uint32_t mk[32];
+      auto load_mask = [&](int c) {
+        const int col0 = nbk * BN + half * 128 + c * 64;
+        const bool in = lane < rows_here && col0 < g.N;
+        const uint4 *mrow = reinterpret_cast<const uint4 *>(
+            g.mask + (size_t)(ti.y + q * 32 + (in ? lane : 0)) * g.N + (in ? col0 : 0));
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const uint4 m4 = in && col0 + 8 * u < g.N ? __ldg(mrow + u) : make_uint4(0u, 0u, 0u, 0u);
+          mk[4 * u] = m4.x; mk[4 * u + 1] = m4.y; mk[4 * u + 2] = m4.z; mk[4 * u + 3] = m4.w;
+        }
+      };
+      if (BMN && g.mask) load_mask(0);
       // every lane waits; the outcome is made warp-uniform so that the
       // .sync.aligned tensor-memory loads below always see the full warp
       const bool ok = __all_sync(0xffffffffu, mbar_wait(tfull(acc), acc_phase, abort_flag, kWaitNs));
@@ -287,18 +303,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         uint32_t v[64];
         tmem_ld64(tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * BN + cl), v);
         const int col0 = nbk * BN + cl;
-        // ReLU mask of the backward pass: this lane's row of hid, 64 columns
-        uint32_t mk[32];
-        if (BMN && g.mask) {
-          const bool in = lane < rows_here && col0 < g.N;
-          const uint4 *mrow = reinterpret_cast<const uint4 *>(
-              g.mask + (size_t)(ti.y + q * 32 + (in ? lane : 0)) * g.N + (in ? col0 : 0));
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const uint4 m4 = in && col0 + 8 * u < g.N ? __ldg(mrow + u) : make_uint4(0u, 0u, 0u, 0u);
-            mk[4 * u] = m4.x; mk[4 * u + 1] = m4.y; mk[4 * u + 2] = m4.z; mk[4 * u + 3] = m4.w;
-          }
-        }
         // conversion by the whole warp (the shuffles need every lane)
         uint32_t pk[32];
 #pragma unroll
@@ -319,6 +323,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
           pk[j] = *reinterpret_cast<uint32_t *>(&h);
         }
+        if (BMN && g.mask && c == 0) load_mask(1);
         if (col0 < g.N && rows_here > 0) {
           // lane l's row, chunk u (8 columns) at chunk slot u ^ (l & 7)
           uint8_t *row_st = stage_epi + lane * 128;

@@ -2,72 +2,113 @@
 //
 // The gate stays in fp32 ([SGMoE-note] 缺点与局限性: the layer diverges when
 // trained in bf16), so its gradients are fp32 contractions:
-//   dW_g = x^T dc, dW_noise = x^T dz        (M = d, N = n, K = T)
-//   dx  += dc W_g^T + dz W_noise^T          (M = T, N = d, K = n)
-// One kernel for both shapes: C[M][N] = sum_k A(m,k) B(k,n), A and B read
-// row- or column-major, 128x128 tiles of 256 threads (8x8 outputs each),
-// 8-deep K slices staged through double-buffered shared memory.  When M x N
-// is small next to the machine (the weight gradients: K = T is the long
-// side) the K range is split across CTAs into a scratch buffer, and a second
-// kernel adds the splits in order, so the result does not depend on timing.
+//   dW_g = x^T dc, dW_noise = x^T dz        (M = d, N = n, K = T; one launch,
+//                                            two problems sharing A)
+//   dx  += dc W_g^T + dz W_noise^T          (M = T, N = d, K = n; one launch,
+//                                            the two products summed)
+// One kernel for all of them: C[M][N] = sum over pairs p of sum_k A_p(m,k)
+// B_p(k,n), A read row- or column-major, B likewise.  128 x 128 tiles, 16-deep
+// K slices, 256 threads with 8 x 8 outputs each held as four 4 x 4 quadrants
+// (rows ty*4 and 64+ty*4, columns tx*4 and 64+tx*4) so that the shared-memory
+// reads of a warp are broadcasts or conflict free; 16-byte global loads where
+// the layout allows, double-buffered shared memory.  When M x N is small next
+// to the machine (the weight gradients: K = T is the long side) the K range
+// is split across CTAs into a scratch buffer and a second kernel adds the
+// splits in order, so the result does not depend on timing.
 #include "internal.h"
 
 namespace moe {
 namespace {
 
-constexpr int BM = 128, BN = 128, BK = 8, NT = 256;
-
-// element (r, c) of an R x Cc view of a matrix stored row-major with leading
-// dimension ld, or transposed (stored Cc x R)
-template <bool TR>
-__device__ __forceinline__ float ld_elem(const float *__restrict__ p, int ld, int r, int c) {
-  return TR ? __ldg(p + (size_t)c * ld + r) : __ldg(p + (size_t)r * ld + c);
-}
+constexpr int BM = 128, BN = 128, BK = 16, NT = 256;
 
 template <bool AT, bool BT>
-__global__ void __launch_bounds__(NT) sgemm_kernel(SgemmArgs a) {
+__global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
   __shared__ __align__(16) float As[2][BK][BM + 4];
   __shared__ __align__(16) float Bs[2][BK][BN + 4];
   const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
   const int splits = a.part ? a.splits : 1;
-  const int kc = (a.K + splits - 1) / splits;
-  const int kbeg = blockIdx.z * kc, kend = min(a.K, kbeg + kc);
+  const int prob = a.nprob > 1 ? (int)blockIdx.z / splits : 0;
+  const int split = (int)blockIdx.z % splits;
+  // split length a multiple of the slice, so every 16-byte load stays aligned
+  const int kc = (a.K + splits - 1) / splits + BK - 1 & ~(BK - 1);
+  const int kbeg = split * kc, kend = min(a.K, kbeg + kc);
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  // 16-byte loads need 4 consecutive in-range elements along the contiguous
+  // dimension and a leading dimension that keeps them aligned
+  const bool va = (a.lda & 3) == 0, vb = (a.ldb & 3) == 0;
 
-  // loader mapping: 256 threads x 4 elements = a 128 x 8 slice.  Stored
-  // [M][K] (A not transposed): thread -> (row tid>>1, 4 columns (tid&1)*4);
-  // stored [K][M]: thread -> (k-row tid>>5, 4 columns (tid&31)*4).
-  float ra[4], rb[4];
-  auto load_a = [&](int k0) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      int m, kk;
-      if (!AT) { m = m0 + (tid >> 1); kk = k0 + (tid & 1) * 4 + u; }
-      else { m = m0 + (tid & 31) * 4 + u; kk = k0 + (tid >> 5); }
-      ra[u] = (m < a.M && kk < kend) ? (AT ? ld_elem<true>(a.A, a.lda, m, kk)
-                                          : ld_elem<false>(a.A, a.lda, m, kk))
-                                     : 0.f;
+  // loader of A (128 x 16 slice): stored [M][K]: thread -> rows tid/4 (+64),
+  // k quad (tid&3)*4; stored [K][M]: k rows tid/32 (+8), m quad (tid&31)*4
+  auto load_a = [&](const float *A, int k0, int h) -> float4 {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!AT) {
+      const int m = m0 + (tid >> 2) + 64 * h, kk = k0 + (tid & 3) * 4;
+      if (m >= a.M) return v;
+      const float *p = A + (size_t)m * a.lda + kk;
+      if (va && kk + 3 < kend) return __ldg(reinterpret_cast<const float4 *>(p));
+      v.x = kk + 0 < kend ? __ldg(p + 0) : 0.f;
+      v.y = kk + 1 < kend ? __ldg(p + 1) : 0.f;
+      v.z = kk + 2 < kend ? __ldg(p + 2) : 0.f;
+      v.w = kk + 3 < kend ? __ldg(p + 3) : 0.f;
+    } else {
+      const int kk = k0 + (tid >> 5) + 8 * h, m = m0 + (tid & 31) * 4;
+      if (kk >= kend) return v;
+      const float *p = A + (size_t)kk * a.lda + m;
+      if (va && m + 3 < a.M) return __ldg(reinterpret_cast<const float4 *>(p));
+      v.x = m + 0 < a.M ? __ldg(p + 0) : 0.f;
+      v.y = m + 1 < a.M ? __ldg(p + 1) : 0.f;
+      v.z = m + 2 < a.M ? __ldg(p + 2) : 0.f;
+      v.w = m + 3 < a.M ? __ldg(p + 3) : 0.f;
     }
+    return v;
   };
-  auto load_b = [&](int k0) {
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      int nn, kk;
-      if (BT) { nn = n0 + (tid >> 1); kk = k0 + (tid & 1) * 4 + u; }
-      else { nn = n0 + (tid & 31) * 4 + u; kk = k0 + (tid >> 5); }
-      // B(k, n): stored [K][N] (row k), or [N][K] with bt
-      rb[u] = (nn < a.N && kk < kend) ? (BT ? __ldg(a.B + (size_t)nn * a.ldb + kk)
-                                            : __ldg(a.B + (size_t)kk * a.ldb + nn))
-                                      : 0.f;
+  // loader of B (16 x 128 slice): stored [K][N]: k rows tid/32 (+8), n quad
+  // (tid&31)*4; stored [N][K]: n rows tid/4 (+64), k quad (tid&3)*4
+  auto load_b = [&](const float *B, int k0, int h) -> float4 {
+    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (!BT) {
+      const int kk = k0 + (tid >> 5) + 8 * h, nn = n0 + (tid & 31) * 4;
+      if (kk >= kend) return v;
+      const float *p = B + (size_t)kk * a.ldb + nn;
+      if (vb && nn + 3 < a.N) return __ldg(reinterpret_cast<const float4 *>(p));
+      v.x = nn + 0 < a.N ? __ldg(p + 0) : 0.f;
+      v.y = nn + 1 < a.N ? __ldg(p + 1) : 0.f;
+      v.z = nn + 2 < a.N ? __ldg(p + 2) : 0.f;
+      v.w = nn + 3 < a.N ? __ldg(p + 3) : 0.f;
+    } else {
+      const int nn = n0 + (tid >> 2) + 64 * h, kk = k0 + (tid & 3) * 4;
+      if (nn >= a.N) return v;
+      const float *p = B + (size_t)nn * a.ldb + kk;
+      if (vb && kk + 3 < kend) return __ldg(reinterpret_cast<const float4 *>(p));
+      v.x = kk + 0 < kend ? __ldg(p + 0) : 0.f;
+      v.y = kk + 1 < kend ? __ldg(p + 1) : 0.f;
+      v.z = kk + 2 < kend ? __ldg(p + 2) : 0.f;
+      v.w = kk + 3 < kend ? __ldg(p + 3) : 0.f;
     }
+    return v;
   };
-  auto store = [&](int buf) {
+  auto store = [&](int buf, const float4 (&av)[2], const float4 (&bv)[2]) {
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      if (!AT) As[buf][(tid & 1) * 4 + u][tid >> 1] = ra[u];
-      else As[buf][tid >> 5][(tid & 31) * 4 + u] = ra[u];
-      if (BT) Bs[buf][(tid & 1) * 4 + u][tid >> 1] = rb[u];
-      else Bs[buf][tid >> 5][(tid & 31) * 4 + u] = rb[u];
+    for (int h = 0; h < 2; ++h) {
+      if (!AT) {
+        const int r = (tid >> 2) + 64 * h, q = (tid & 3) * 4;
+        As[buf][q + 0][r] = av[h].x;
+        As[buf][q + 1][r] = av[h].y;
+        As[buf][q + 2][r] = av[h].z;
+        As[buf][q + 3][r] = av[h].w;
+      } else {
+        *reinterpret_cast<float4 *>(&As[buf][(tid >> 5) + 8 * h][(tid & 31) * 4]) = av[h];
+      }
+      if (!BT) {
+        *reinterpret_cast<float4 *>(&Bs[buf][(tid >> 5) + 8 * h][(tid & 31) * 4]) = bv[h];
+      } else {
+        const int r = (tid >> 2) + 64 * h, q = (tid & 3) * 4;
+        Bs[buf][q + 0][r] = bv[h].x;
+        Bs[buf][q + 1][r] = bv[h].y;
+        Bs[buf][q + 2][r] = bv[h].z;
+        Bs[buf][q + 3][r] = bv[h].w;
+      }
     }
   };
 
@@ -77,75 +118,100 @@ __global__ void __launch_bounds__(NT) sgemm_kernel(SgemmArgs a) {
 #pragma unroll
     for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
 
-  int buf = 0;
-  if (kbeg < kend) {
-    load_a(kbeg);
-    load_b(kbeg);
-    store(0);
+  // the pairs whose products are summed: pair 1 only with ksum
+  const int npair = a.ksum ? 2 : 1;
+  for (int p = 0; p < npair; ++p) {
+    const int pi = a.ksum ? p : prob;
+    // (selected, not indexed: a runtime index would copy the arguments to local memory)
+    const float *A = pi ? a.A[1] : a.A[0], *B = pi ? a.B[1] : a.B[0];
+    if (kbeg >= kend) break;
+    float4 av[2] = {load_a(A, kbeg, 0), load_a(A, kbeg, 1)};
+    float4 bv[2] = {load_b(B, kbeg, 0), load_b(B, kbeg, 1)};
+    __syncthreads();  // the previous pair's last slice has been read
+    store(0, av, bv);
     __syncthreads();
+    int buf = 0;
     for (int k0 = kbeg; k0 < kend; k0 += BK) {
       const bool more = k0 + BK < kend;
-      if (more) {  // next slice into registers while this one is used
-        load_a(k0 + BK);
-        load_b(k0 + BK);
+      if (more) {  // the next slice into registers while this one is used
+        av[0] = load_a(A, k0 + BK, 0);
+        av[1] = load_a(A, k0 + BK, 1);
+        bv[0] = load_b(B, k0 + BK, 0);
+        bv[1] = load_b(B, k0 + BK, 1);
       }
 #pragma unroll
       for (int kk = 0; kk < BK; ++kk) {
-        const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 8]);
-        const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 8 + 4]);
-        const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 8]);
-        const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 8 + 4]);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
+        const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
+        const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
+        const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
+        const float av8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+        const float bv8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av8[i], bv8[j], acc[i][j]);
       }
       if (more) {
-        store(buf ^ 1);
+        store(buf ^ 1, av, bv);
         __syncthreads();
         buf ^= 1;
       }
     }
   }
 
-  // rows ty*8.., columns tx*8..
+  // output rows ty*4+i (i<4) and 64+ty*4+i-4, columns tx*4+j and 64+tx*4+j-4
+  float *const C = prob ? a.C[1] : a.C[0];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    const int m = m0 + ty * 8 + i;
-    if (m >= a.M) break;
+    const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
+    if (m >= a.M) continue;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int nn = n0 + tx * 8 + j;
-      if (nn >= a.N) break;
+    for (int h = 0; h < 2; ++h) {
+      const int nn = n0 + h * 64 + tx * 4;
+      const float4 v = make_float4(acc[i][4 * h], acc[i][4 * h + 1], acc[i][4 * h + 2],
+                                   acc[i][4 * h + 3]);
       if (a.part) {
-        a.part[((size_t)blockIdx.z * a.M + m) * a.N + nn] = acc[i][j];
+        float *dst = a.part + (((size_t)prob * splits + split) * a.M + m) * a.N + nn;
+        if ((a.N & 3) == 0 && nn + 3 < a.N) {
+          *reinterpret_cast<float4 *>(dst) = v;
+        } else {
+          const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            if (nn + j < a.N) dst[j] = vv[j];
+        }
       } else {
-        float *c = a.C + (size_t)m * a.ldc + nn;
-        *c = a.accumulate ? *c + acc[i][j] : acc[i][j];
+        float *dst = C + (size_t)m * a.ldc + nn;
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (nn + j < a.N) dst[j] = a.accumulate ? dst[j] + vv[j] : vv[j];
       }
     }
   }
 }
 
-// C = sum over the splits in order (+ C)
+// C_p = sum over the splits of problem p in order (+ C_p)
 __global__ void __launch_bounds__(256) split_sum_kernel(const float *__restrict__ part, int splits,
-                                                        int M, int N, float *C, int ldc,
-                                                        int accumulate) {
+                                                        int M, int N, float *C0, float *C1,
+                                                        int ldc, int accumulate) {
+  const size_t MN = (size_t)M * N;
   const size_t i = (size_t)blockIdx.x * 256 + threadIdx.x;
-  if (i >= (size_t)M * N) return;
+  const int prob = blockIdx.y;
+  if (i >= MN) return;
+  const float *pp = part + (size_t)prob * splits * MN;
   float s = 0.f;
-  for (int z = 0; z < splits; ++z) s += part[(size_t)z * M * N + i];
+  for (int z = 0; z < splits; ++z) s += pp[(size_t)z * MN + i];
   const int m = (int)(i / N), nn = (int)(i % N);
-  float *c = C + (size_t)m * ldc + nn;
+  float *c = (prob ? C1 : C0) + (size_t)m * ldc + nn;
   *c = accumulate ? *c + s : s;
 }
 
 }  // namespace
 
-int sgemm_splits(int M, int N, int K) {
-  const int tiles = (int)(ceil_div(M, BM) * ceil_div(N, BN));
+int sgemm_splits(int M, int N, int K, int nprob) {
+  const int tiles = (int)(ceil_div(M, BM) * ceil_div(N, BN)) * (nprob > 1 ? nprob : 1);
   const int want = 2 * num_sms();
   if (tiles >= want / 2 || K < 8 * BK) return 1;
   int s = want / tiles;
@@ -157,9 +223,12 @@ int sgemm_splits(int M, int N, int K) {
 int launch_sgemm(const SgemmArgs &a, cudaStream_t st) {
   if (a.M <= 0 || a.N <= 0) return MOE_OK;
   SgemmArgs b = a;
+  if (b.nprob < 1) b.nprob = 1;
+  if (b.ksum) b.nprob = 1;
   if (b.splits <= 1) b.part = nullptr;
   const int splits = b.part ? b.splits : 1;
-  const dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ceil_div(a.M, BM), (unsigned)splits);
+  const dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ceil_div(a.M, BM),
+                  (unsigned)(splits * b.nprob));
   const char *name = a.name ? a.name : "gate_grad_gemm";
   int rc;
   if (!a.at && !a.bt) rc = launch(name, sgemm_kernel<false, false>, grid, dim3(NT), 0, st, b);
@@ -168,8 +237,9 @@ int launch_sgemm(const SgemmArgs &a, cudaStream_t st) {
   else rc = launch(name, sgemm_kernel<true, true>, grid, dim3(NT), 0, st, b);
   if (rc != MOE_OK || !b.part) return rc;
   const size_t total = (size_t)a.M * a.N;
-  return launch("gate_grad_split_sum", split_sum_kernel, dim3((unsigned)ceil_div((int64_t)total, 256)),
-                dim3(256), 0, st, (const float *)b.part, splits, a.M, a.N, a.C, a.ldc,
+  return launch("gate_grad_split_sum", split_sum_kernel,
+                dim3((unsigned)ceil_div((int64_t)total, 256), (unsigned)b.nprob), dim3(256), 0, st,
+                (const float *)b.part, splits, a.M, a.N, b.C[0], b.C[b.nprob > 1 ? 1 : 0], a.ldc,
                 a.accumulate);
 }
 

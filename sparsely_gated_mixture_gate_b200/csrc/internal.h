@@ -202,7 +202,7 @@ int launch_dx_gather(const void *dx_perm, const int *row_of, const float *dy, in
 int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,
                      int f, float *db2, float *db1, const char *name, cudaStream_t st);
 int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st);
-int colsum_parts(int R);
+int colsum_parts(int R, int N);
 int launch_colsum(const float *X, int R, int N, float *part, float *out, cudaStream_t st);
 // weight gradients of the experts on the tensor cores, per expert e with rows
 // offsets[e] .. offsets[e+1]-1: dW2_e = dy_perm_e^T hid_e ([d][f]) and
@@ -218,21 +218,22 @@ struct WgradArgs {
 int launch_wgrad_bf16(const WgradArgs &a, cudaStream_t st);
 // C[M][N] = sum_k A(m,k) B(k,n) (+ C when accumulate), fp32; A(m,k) =
 // A[m*lda+k] or, with at, A[k*lda+m]; B(k,n) = B[k*ldb+n] or, with bt,
-// B[n*ldb+k].  part: split-K scratch of splits*M*N floats (nullptr: no split).
+// B[n*ldb+k].  nprob = 2: two problems in one launch, C[p] = A[p] B[p];
+// ksum: one problem, C[0] = A[0] B[0] + A[1] B[1].  part: split-K scratch of
+// nprob*splits*M*N floats (nullptr: no split).  A, B 16-byte aligned.
 struct SgemmArgs {
   int M, N, K;
-  const float *A;
-  int lda, at;
-  const float *B;
-  int ldb, bt;
-  float *C;
-  int ldc, accumulate;
+  const float *A[2];
+  const float *B[2];
+  float *C[2];
+  int lda, ldb, ldc, at, bt;
+  int nprob, ksum, accumulate;
   float *part;
   int splits;
   const char *name;
 };
 int launch_sgemm(const SgemmArgs &a, cudaStream_t st);
-int sgemm_splits(int M, int N, int K);
+int sgemm_splits(int M, int N, int K, int nprob);  // split-K factor for nprob problems of M x N
 
 int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *importance,
                       cudaStream_t st);

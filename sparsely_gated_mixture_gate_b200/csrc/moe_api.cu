@@ -265,9 +265,10 @@ Layout make_layout(const moe_config &c) {
     L.sw_coef = bp.take(4 * n);
     L.dc = bp.take(4 * T * n);
     L.dz = bp.take(c.noise ? 4 * T * n : 0);
-    L.colsum_part = bp.take(4 * (size_t)colsum_parts(c.T) * n);
-    const size_t sp = (size_t)sgemm_splits(c.d, c.n, c.T);
-    L.sgemm_part = bp.take(sp > 1 ? 4 * sp * (size_t)c.d * n : 0);
+    L.colsum_part = bp.take(4 * (size_t)colsum_parts(c.T, c.n) * n);
+    const size_t np = c.noise ? 2 : 1;  // dW_g, and dW_noise beside it
+    const size_t sp = (size_t)sgemm_splits(c.d, c.n, c.T, (int)np);
+    L.sgemm_part = bp.take(sp > 1 ? 4 * np * sp * (size_t)c.d * n : 0);
   }
   L.total = bp.off;
   return L;
@@ -859,9 +860,13 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   float *sw_coef = at<float>(ws, L.sw_coef);
   float *dc = at<float>(ws, L.dc), *dz = c.noise ? at<float>(ws, L.dz) : nullptr;
 
-  // ---- balancing losses -> dL/dImportance, dL/dLoad, Switch dL/dp
+  // ---- balancing losses -> dL/dImportance, dL/dLoad, Switch dL/dp: one
+  // block on the side stream, needed only by the gate's backward
+  Side *side = nullptr;
+  MOE_TRY(side_stream(&side));
+  MOE_TRY(stream_after(side->s, st, side->fork_gate));
   MOE_TRY(launch_bwd_coef(importance, load, counts, n, T, c.w_importance, c.w_load, c.alpha_aux,
-                          c.router, c.noise, lam_imp, lam_load, sw_coef, st));
+                          c.router, c.noise, lam_imp, lam_load, sw_coef, side->s));
   // ---- combine: dy_perm rows, dL/dgate, the shared expert's rows
   MOE_TRY(launch_combine_bwd(dy, topk_gate, row_of, at<void>(ws, L.y_perm), T, k, d, dy_perm,
                              dgate, dy_sh, st));
@@ -961,32 +966,43 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   g.has_load = c.noise && c.w_load != 0.f;
   g.dc = dc;
   g.dz = dz;
+  MOE_TRY(stream_after(st, side->s, side->join));  // the loss coefficients
   MOE_TRY(launch_gate_bwd(g, st));
   if (gr->db_g) MOE_TRY(launch_colsum(dc, T, n, at<float>(ws, L.colsum_part), gr->db_g, st));
   float *sp = at<float>(ws, L.sgemm_part);
-  const int splits = sgemm_splits(d, n, T);
-  for (int q = 0; q < (c.noise ? 2 : 1); ++q) {
-    const float *G = q ? dz : dc;
-    const float *W = q ? gp->W_noise : gp->W_g;
-    float *dW = q ? gr->dW_noise : gr->dW_g;
-    if (dW) {  // dW = x^T G: M = d, N = n, K = T
-      SgemmArgs a{};
-      a.M = d; a.N = n; a.K = T;
-      a.A = x; a.lda = d; a.at = 1;
-      a.B = G; a.ldb = n; a.bt = 0;
-      a.C = dW; a.ldc = n; a.accumulate = 0;
-      a.part = splits > 1 ? sp : nullptr;
-      a.splits = splits;
-      a.name = "gate_wgrad_fp32";
-      MOE_TRY(launch_sgemm(a, st));
+  const bool want_n = c.noise && gr->dW_noise;
+  // the split count the workspace was sized for (two problems with noise)
+  const int splits = sgemm_splits(d, n, T, c.noise ? 2 : 1);
+  if (gr->dW_g || want_n) {
+    // dW_g = x^T dc and dW_noise = x^T dz: M = d, N = n, K = T, A shared
+    SgemmArgs a{};
+    a.M = d; a.N = n; a.K = T;
+    a.A[0] = a.A[1] = x; a.lda = d; a.at = 1;
+    a.ldb = n; a.bt = 0; a.ldc = n;
+    if (gr->dW_g && want_n) {
+      a.B[0] = dc; a.C[0] = gr->dW_g;
+      a.B[1] = dz; a.C[1] = gr->dW_noise;
+      a.nprob = 2;
+    } else {
+      a.B[0] = gr->dW_g ? dc : dz;
+      a.C[0] = gr->dW_g ? gr->dW_g : gr->dW_noise;
+      a.nprob = 1;
     }
-    // dx += G W^T: M = T, N = d, K = n; B(k, q) = W[q][k]
+    a.part = splits > 1 ? sp : nullptr;
+    a.splits = splits;
+    a.name = "gate_wgrad_fp32";
+    MOE_TRY(launch_sgemm(a, st));
+  }
+  {
+    // dx += dc W_g^T (+ dz W_noise^T): M = T, N = d, K = n; B(k, q) = W[q][k]
     SgemmArgs a{};
     a.M = T; a.N = d; a.K = n;
-    a.A = G; a.lda = n; a.at = 0;
-    a.B = W; a.ldb = n; a.bt = 1;
-    a.C = dx; a.ldc = d; a.accumulate = 1;
-    a.part = nullptr;
+    a.A[0] = dc; a.A[1] = dz; a.lda = n; a.at = 0;
+    a.B[0] = gp->W_g; a.B[1] = gp->W_noise; a.ldb = n; a.bt = 1;
+    a.C[0] = a.C[1] = dx; a.ldc = d;
+    a.nprob = 1;
+    a.ksum = c.noise ? 1 : 0;
+    a.accumulate = 1;
     a.splits = 1;
     a.name = "gate_dgrad_fp32";
     MOE_TRY(launch_sgemm(a, st));
