@@ -31,7 +31,8 @@
 //           wait, broadcast by shuffles), ReLU, bf16; the warp's 32 x 64 block
 //           goes through its own 4 KiB of shared memory (XOR-swizzled 16-byte
 //           chunks) so that every store instruction writes four whole 128-byte
-//           row segments, masked to the expert's valid rows
+//           row segments, masked to the expert's valid rows; the hidden layer's
+//           stores carry an evict-last L2 policy (GEMM2 reads it back)
 // Two accumulators of 256 columns (all 512 TMEM columns) let the epilogue of
 // one tile overlap the main loop of the next.  Tiles are ordered expert by
 // expert, N-block by N-block, M-block fastest, so the M-blocks that share a
@@ -257,6 +258,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     const int half = (warp - 2) >> 2;       // columns [128*half, 128*half + 128) of the tile
     uint8_t *const stage_epi = stage_epi_all + (warp - 2) * EPI_STAGE_BYTES;
     const int rr = lane >> 3, cc = lane & 7;
+    // the hidden layer is stored with an evict-last L2 policy: GEMM2 reads it
+    // back while the weights stream through L2 (measured: 2% faster)
+    const uint64_t hpol = l2_evict_last_policy();
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
@@ -336,8 +340,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           for (int i = 0; i < 8; ++i) {
             const int r = i * 4 + rr;  // row inside the warp's block
             const uint4 v4 = *reinterpret_cast<const uint4 *>(stage_epi + r * 128 + ((cc ^ (r & 7)) << 4));
-            if (r < rows_here && col0 + cc * 8 < g.N)
-              *reinterpret_cast<uint4 *>(dtile + (size_t)r * g.N + col0 + cc * 8) = v4;
+            if (r < rows_here && col0 + cc * 8 < g.N) {
+              __nv_bfloat16 *dst = dtile + (size_t)r * g.N + col0 + cc * 8;
+              if (!which) st_global_l2_hint(dst, v4, hpol);  // hidden layer: read back soon
+              else *reinterpret_cast<uint4 *>(dst) = v4;
+            }
           }
           __syncwarp();  // the block is reused by the next chunk
         }
