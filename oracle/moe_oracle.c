@@ -776,6 +776,19 @@ static double expert_row_bwd(int d, int f, int bf16, const float *x, const void 
   return dgate;
 }
 
+void orc_expert_backward(int d, int f, int bf16, int nrows, const float *x_rows, const double *g,
+                         const float *dy_rows, const void *W1, const float *b1, const void *W2,
+                         const float *b2, double *dW1, double *db1, double *dW2, double *db2,
+                         double *dgate, double *dx_rows)
+{
+  for (int r = 0; r < nrows; ++r) {
+    double *dxr = dx_rows + (size_t)r * d;
+    for (int q = 0; q < d; ++q) dxr[q] = 0.0;
+    dgate[r] = expert_row_bwd(d, f, bf16, x_rows + (size_t)r * d, W1, b1, W2, b2, g[r],
+                              dy_rows + (size_t)r * d, dW1, db1, dW2, db2, dxr);
+  }
+}
+
 int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g)
 {
   if (!valid_cfg(cfg) || cfg->hier_a) return -1;

@@ -200,6 +200,17 @@ void orc_cv2_grad(const double *v, int n, double *g);
 /* 0, or -1 for a configuration the backward does not cover. */
 int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g);
 
+/* One expert's part of the backward over nrows rows (the steps orc_backward
+ * takes for each kept slot): row r is a token's input x_rows[r][d], the gate
+ * g[r] of this expert in that token's output and the upstream gradient
+ * dy_rows[r][d].  Adds to dW1 [f][d], db1 [f], dW2 [d][f], db2 [d] (db1, db2
+ * may be NULL) and writes dgate[r] = <dy_r, E(x_r)> and dx_rows[r][d], the
+ * expert's part of the input gradient. */
+void orc_expert_backward(int d, int f, int bf16, int nrows, const float *x_rows, const double *g,
+                         const float *dy_rows, const void *W1, const float *b1, const void *W2,
+                         const float *b2, double *dW1, double *db1, double *dW2, double *db2,
+                         double *dgate, double *dx_rows);
+
 #ifdef __cplusplus
 }
 #endif

@@ -108,6 +108,8 @@ def lib():
         L.orc_cv2_grad.argtypes = [vp, i32, vp]
         L.orc_backward.argtypes = [C.POINTER(OrcCfg), C.POINTER(OrcInputs), vp, C.POINTER(OrcGrads)]
         L.orc_backward.restype = i32
+        L.orc_expert_backward.argtypes = [i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp]
         _lib = L
     return _lib
 
@@ -354,4 +356,23 @@ def backward(cfg: dict, inp: dict, dy) -> dict:
     g = OrcGrads(**{name: _p(a) for name, a in out.items()})
     if lib().orc_backward(C.byref(oc), C.byref(ins), _p(dy), C.byref(g)) != 0:
         raise ValueError(f"oracle backward rejected the configuration {cfg}")
+    return out
+
+
+def expert_backward(x_rows, g, dy_rows, W1, b1, W2, b2, bf16: bool) -> dict:
+    """One expert's part of the backward over the given rows (see
+    orc_expert_backward): its weight and bias gradients, dL/dgate per row and
+    its part of dx per row.  bf16 weights as uint16 bit patterns."""
+    x_rows = _c(x_rows, np.float32); dy_rows = _c(dy_rows, np.float32)
+    g = _c(g, np.float64)
+    wdt = np.uint16 if bf16 else np.float32
+    W1 = _c(W1, wdt); W2 = _c(W2, wdt)
+    f, d = W1.shape
+    b1 = _c(b1, np.float32); b2 = _c(b2, np.float32)
+    R = x_rows.shape[0]
+    out = dict(dW1=np.zeros((f, d)), db1=np.zeros(f), dW2=np.zeros((d, f)), db2=np.zeros(d),
+               dgate=np.zeros(R), dx=np.zeros((R, d)))
+    lib().orc_expert_backward(d, f, int(bool(bf16)), R, _p(x_rows), _p(g), _p(dy_rows), _p(W1),
+                              _p(b1), _p(W2), _p(b2), _p(out["dW1"]), _p(out["db1"]),
+                              _p(out["dW2"]), _p(out["db2"]), _p(out["dgate"]), _p(out["dx"]))
     return out

@@ -165,3 +165,55 @@ def test_fullsize(orc, name, gp):
         assert err < 2e-2, (t, err)
         checked += 1
     assert checked >= len(toks) // 2
+
+
+# ------------------------------------------------------------------ backward
+@pytest.mark.parametrize("name", ["lm-flat", "deepseek-flat"])
+def test_fullsize_backward(orc, name):
+    """The training step the bench times (forward + moe_backward) at full size.
+    The oracle routes the whole batch (its own gate), then computes the
+    weight and bias gradients of sampled experts from the rows it routed to
+    them and dL/dgate of their tokens; the gate's gradients depend on
+    whole-batch sums and are covered by the small parity cases."""
+    import dataclasses
+    w = synth.WORKLOADS.get(name) or synth.VARIANTS[name]
+    inp = synth.make_inputs(w, device=DEV)
+    dy = synth.make_dy(w, device=DEV)
+    cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
+    layer = M.MoELayer(cfg, inp, DEV)
+    layer.forward_(inp["x"])
+    layer.grads(intermediates=True)
+    g = layer.backward_(inp["x"], dy)
+    torch.cuda.synchronize()
+    assert M.status_bits(layer.status) == 0
+    host = _host(inp, ["x", "Wg", "bg", "Wn", "sel_bias"])
+    ref = orc.gate_batch(w.cfg(), host)
+    tie = ref["near_tie"] < TIE
+    idx = layer.topk_idx.cpu().numpy()
+    assert np.array_equal(idx[~tie], ref["topk_idx"][~tie])
+    x = host["x"]
+    dyh = dy.cpu().numpy()
+    dgate = g["dgate"].cpu().numpy()
+    counts = np.bincount(ref["topk_idx"].ravel(), minlength=w.n)
+    rng = np.random.default_rng(3)
+    experts = sorted({int(np.argmax(counts)), int(np.argmin(counts))} |
+                     set(rng.integers(0, w.n, 4).tolist()))
+    checked = 0
+    for e in experts:
+        slots = np.argwhere(ref["topk_idx"] == e)  # (token, slot), token order
+        if tie[slots[:, 0]].any():
+            continue  # a near tie could move a row in or out of this expert
+        toks = slots[:, 0]
+        gates = ref["topk_gate"][slots[:, 0], slots[:, 1]]
+        r = orc.expert_backward(x[toks], gates, dyh[toks], _bits(inp["W1"][e]),
+                                inp["b1"][e].cpu().numpy(), _bits(inp["W2"][e]),
+                                inp["b2"][e].cpu().numpy(), bf16=True)
+        for key in ("dW1", "db1", "dW2", "db2"):
+            got = g[key][e].cpu().numpy()
+            if not np.any(r[key]) and not np.any(got):
+                continue
+            assert _rel(got, r[key]) < 1e-2, (name, e, key, _rel(got, r[key]))
+        if len(toks):
+            assert _rel(dgate[slots[:, 0], slots[:, 1]], r["dgate"]) < 5e-3, (name, e)
+        checked += 1
+    assert checked >= 3

@@ -231,3 +231,33 @@ def test_hierarchical_rejected():
                         Wn2=np.zeros((2, 4, 2), np.float32), W1=np.zeros((4, 8, 4), np.float32),
                         W2=np.zeros((4, 4, 8), np.float32)),
                    np.zeros((2, 4), np.float32))
+
+
+def test_expert_backward_is_the_layer_backward_of_one_expert():
+    """The per-expert entry point, applied to the rows the layer routed to each
+    expert with their gates, gives the layer backward's dW1..db2 and dgate
+    (the whole-layer backward is pinned above)."""
+    rng = np.random.default_rng(12)
+    T, d, n, k, f = 20, 8, 4, 2, 16
+    inp = _inputs(rng, T, d, n, f)
+    for bf16 in (0, 1):
+        cfg = dict(T=T, d=d, n=n, k=k, f=f, router=0, noise=1, seed=4, capacity_factor=0.8,
+                   expert_bf16=bf16)
+        e_inp = dict(inp)
+        if bf16:
+            for w in ("W1", "W2"):
+                e_inp[w] = _to_bf16_bits(inp[w])[0]
+        dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+        out = O.forward(cfg, e_inp)
+        g = O.backward(cfg, e_inp, dy)
+        for e in range(n):
+            rows = [(t, j) for t in range(T) for j in range(k)
+                    if out["topk_idx"][t, j] == e and out["row_of"][t, j] >= 0]
+            toks = np.array([t for t, _ in rows], np.int64)
+            gates = np.array([out["topk_gate"][t, j] for t, j in rows])
+            r = O.expert_backward(inp["x"][toks], gates, dy[toks], e_inp["W1"][e], inp["b1"][e],
+                                  e_inp["W2"][e], inp["b2"][e], bf16=bool(bf16))
+            for key in ("dW1", "db1", "dW2", "db2"):
+                assert np.allclose(r[key], g[key][e], rtol=1e-12, atol=1e-12), (bf16, e, key)
+            for (t, j), dg in zip(rows, r["dgate"]):
+                assert dg == pytest.approx(g["dgate"][t, j], rel=1e-12, abs=1e-12)
