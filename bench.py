@@ -316,32 +316,26 @@ def run_ours(args, w, world, rank, local):
         torch.cuda.synchronize()
         h2d_bytes, d2h_bytes = w.T * w.d * 4, w.T * w.d * 4 + 4 * layer.losses.numel()
     else:
-        # training step from host memory: x and dy in, y, the losses and dx out
-        # (the parameter gradients stay on the device for the optimizer)
+        # training steps from host memory: x and dy in, y, the losses and dx
+        # out every step (the parameter gradients stay on the device for the
+        # optimizer); copies of neighbouring steps overlap compute
         dyh = dy.cpu().pin_memory()
-        dxh = torch.empty(w.T, w.d, dtype=torch.float32).pin_memory()
-        xd, dyd = torch.empty_like(x), torch.empty_like(dy)
-        dx = layer.grads()["dx"]
+        dxh = [torch.empty(w.T, w.d, dtype=torch.float32).pin_memory() for _ in range(2)]
 
-        def host_step(i):
-            xd.copy_(xh, non_blocking=True)
-            dyd.copy_(dyh, non_blocking=True)
-            layer.forward_(xd)
-            layer.backward_(xd, dyd)
-            yh[i & 1].copy_(layer.y, non_blocking=True)
-            lh[i & 1].copy_(layer.losses, non_blocking=True)
-            dxh.copy_(dx, non_blocking=True)
+        def host_steps(m):
+            return layer.train_host_batches([xh] * m, [dyh] * m, [yh[i & 1] for i in range(m)],
+                                            [lh[i & 1] for i in range(m)],
+                                            [dxh[i & 1] for i in range(m)])
 
-        for i in range(3):
-            host_step(i)
+        host_steps(3)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(e_steps):
-            host_step(i)
+        d2h = host_steps(e_steps)
+        stream.wait_stream(d2h)
         e1.record(stream)
         torch.cuda.synchronize()
         h2d_bytes = 2 * w.T * w.d * 4
@@ -460,8 +454,9 @@ def run_ours(args, w, world, rank, local):
                 "d2h_bytes_per_step": d2h_bytes, "steps": e_steps,
                 "how": ("pinned host x in, y and losses out every step; copies of neighbouring "
                         "steps overlap compute on two copy streams") if dy is None else
-                       ("pinned host x and dy in, y, losses and dx out every step, on the "
-                        "compute stream (parameter gradients stay on the device)")},
+                       ("pinned host x and dy in, y, losses and dx out every step; copies of "
+                        "neighbouring steps overlap compute on two copy streams (parameter "
+                        "gradients stay on the device)")},
         "clocks": clk,
         "alt_gate_mode": alt,
         "wall_s": round(wall, 3),

@@ -421,6 +421,149 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
   }
 }
 
+// The noisy top-k gate's backward with the row in registers: lane l holds
+// column quads l, l+32, ... (NQ of them, n <= 128 NQ, n a multiple of 4),
+// loaded once with 16-byte loads, so both passes run from registers.  Same
+// arithmetic, in the same order per element, as gate_bwd_kernel.
+template <int KM, int NQ>
+__global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
+  const int t = blockIdx.x * GW + (threadIdx.x >> 5);
+  if (t >= a.T) return;
+  const int lane = threadIdx.x & 31;
+  const int n = a.n, k = a.k;
+  const float4 *crow = reinterpret_cast<const float4 *>(a.c + (size_t)t * n);
+  const float4 *srow = reinterpret_cast<const float4 *>(a.s + (size_t)t * n);
+  float cv[NQ][4], sv[NQ][4];
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int m = lane + 32 * q;
+    float4 c4 = make_float4(0.f, 0.f, 0.f, 0.f), s4 = c4;
+    if (4 * m < n) {
+      c4 = __ldg(crow + m);
+      if (a.noise) s4 = __ldg(srow + m);
+    }
+    cv[q][0] = c4.x; cv[q][1] = c4.y; cv[q][2] = c4.z; cv[q][3] = c4.w;
+    sv[q][0] = s4.x; sv[q][1] = s4.y; sv[q][2] = s4.z; sv[q][3] = s4.w;
+  }
+  int ids[KM];
+  float gs[KM], dG[KM];
+  {
+    int id = 0;
+    float gv = 0.f, dv = 0.f;
+    if (lane < k) {
+      id = a.idx[(size_t)t * k + lane];
+      gv = a.gate[(size_t)t * k + lane];
+      dv = a.dgate[(size_t)t * k + lane] + a.lam_imp[id];  // combine + importance
+    }
+#pragma unroll
+    for (int j = 0; j < KM; ++j) {
+      ids[j] = __shfl_sync(0xffffffffu, id, j);
+      gs[j] = __shfl_sync(0xffffffffu, gv, j);
+      dG[j] = __shfl_sync(0xffffffffu, dv, j);
+    }
+  }
+  float gdg = 0.f;
+#pragma unroll
+  for (int j = 0; j < KM; ++j)
+    if (j < k) gdg = fmaf(gs[j], dG[j], gdg);
+  float dHk[KM];
+#pragma unroll
+  for (int j = 0; j < KM; ++j) dHk[j] = gs[j] * (dG[j] - gdg);
+  int jkk = 0;
+#pragma unroll
+  for (int j = 0; j < KM; ++j)
+    if (j == k - 1) jkk = ids[j];
+  const bool loadg = a.noise && a.has_load;
+  float thr_kept = -INFINITY, thr_out = -INFINITY;
+  int jk1 = -1;
+  if (loadg) {
+    const int4 q = a.kth[t];
+    thr_kept = __int_as_float(q.x);
+    jk1 = thr_kept == -INFINITY ? -1 : q.y;
+    thr_out = __int_as_float(q.z);
+  }
+  auto kept_slot = [&](int i) {
+    int js = -1;
+#pragma unroll
+    for (int j = 0; j < KM; ++j)
+      if (j < k && ids[j] == i) js = j;
+    return js;
+  };
+  // load term per element: av = lam_load_i phi(u_i) / s_i, u_i = (c_i - thr_i) / s_i
+  float av[NQ][4], uv[NQ][4];
+  float A_kept = 0.f, A_out = 0.f;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int i0 = 4 * (lane + 32 * q);
+    float lam4[4] = {0.f, 0.f, 0.f, 0.f};
+    if (loadg && i0 < n) {
+      const float4 l4 = __ldg(reinterpret_cast<const float4 *>(a.lam_load) + lane + 32 * q);
+      lam4[0] = l4.x; lam4[1] = l4.y; lam4[2] = l4.z; lam4[3] = l4.w;
+    }
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const int i = i0 + j4;
+      av[q][j4] = 0.f;
+      uv[q][j4] = 0.f;
+      if (!loadg || i >= n) continue;
+      const bool kept = kept_slot(i) >= 0;
+      const float thr = kept ? thr_kept : thr_out;
+      const float svv = sv[q][j4];
+      if (thr == -INFINITY || svv == 0.f) continue;  // P constant there
+      const float u = (cv[q][j4] - thr) / svv;
+      const float v = lam4[j4] * (0.3989422804014327f * expf(-0.5f * u * u)) / svv;
+      av[q][j4] = v;
+      uv[q][j4] = u;
+      if (kept) A_kept += v; else A_out += v;
+    }
+  }
+  if (loadg) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      A_kept += __shfl_xor_sync(0xffffffffu, A_kept, off);
+      A_out += __shfl_xor_sync(0xffffffffu, A_out, off);
+    }
+  }
+  const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
+  float4 *dcrow = reinterpret_cast<float4 *>(a.dc + (size_t)t * n);
+  float4 *dzrow = a.dz ? reinterpret_cast<float4 *>(a.dz + (size_t)t * n) : nullptr;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int m = lane + 32 * q;
+    if (4 * m >= n) break;
+    float eps[4] = {0.f, 0.f, 0.f, 0.f};
+    if (a.noise) {
+      const uint4 wd = philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, 0u, 0u), key0, key1);
+      box_muller2(wd.x, wd.y, eps[0], eps[1]);
+      box_muller2(wd.z, wd.w, eps[2], eps[3]);
+    }
+    float dc4[4], dz4[4];
+#pragma unroll
+    for (int j4 = 0; j4 < 4; ++j4) {
+      const int i = 4 * m + j4;
+      const int js = kept_slot(i);
+      float dH = 0.f;
+#pragma unroll
+      for (int j = 0; j < KM; ++j)
+        if (j == js) dH = dHk[j];
+      float dc = 0.f, ds = 0.f;
+      if (loadg) {
+        if (i == jk1) dH -= A_kept;
+        if (i == jkk) dH -= A_out;
+        dc += av[q][j4];
+        ds -= av[q][j4] * uv[q][j4];
+      }
+      dc += dH;  // H = c + eps s
+      dc4[j4] = dc;
+      ds = fmaf(dH, eps[j4], ds);
+      // s = Softplus(z): dz = ds Sigmoid(z), Sigmoid(z) = 1 - e^-s
+      dz4[j4] = ds * -expm1f(-sv[q][j4]);
+    }
+    dcrow[m] = make_float4(dc4[0], dc4[1], dc4[2], dc4[3]);
+    if (dzrow) dzrow[m] = make_float4(dz4[0], dz4[1], dz4[2], dz4[3]);
+  }
+}
+
 // ---------------------------------------------------------------- colsum
 // part[blockIdx.y][j] = sum of rows [blockIdx.y * rows_per, ...) of column j
 __global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ X, int R, int N,
@@ -487,6 +630,20 @@ int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st) {
   if (a.k > kMaxK) return MOE_EINVAL;
   const dim3 grid((unsigned)ceil_div(a.T, GW));
   auto go = [&](auto kern) { return launch("gate_bwd", kern, grid, dim3(GW * 32), 0, st, a); };
+  if (a.router == MOE_ROUTER_NOISY_TOPK && (a.n & 3) == 0 && a.n <= 4 * 32 * 8) {
+    // the row in registers: quads per lane 1, 2, 4 or 8
+    const int nq = (a.n + 127) / 128;
+#define MOE_GBWD_REG(KMV)                                                      \
+    if (nq <= 1) return go(gate_bwd_reg_kernel<KMV, 1>);                       \
+    if (nq <= 2) return go(gate_bwd_reg_kernel<KMV, 2>);                       \
+    if (nq <= 4) return go(gate_bwd_reg_kernel<KMV, 4>);                       \
+    return go(gate_bwd_reg_kernel<KMV, 8>);
+    if (a.k <= 1) { MOE_GBWD_REG(1) }
+    if (a.k <= 2) { MOE_GBWD_REG(2) }
+    if (a.k <= 4) { MOE_GBWD_REG(4) }
+    MOE_GBWD_REG(8)
+#undef MOE_GBWD_REG
+  }
   if (a.k <= 1) return go(gate_bwd_kernel<1>);
   if (a.k <= 2) return go(gate_bwd_kernel<2>);
   if (a.k <= 4) return go(gate_bwd_kernel<4>);

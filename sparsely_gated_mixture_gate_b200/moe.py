@@ -329,22 +329,70 @@ class MoELayer:
                 db2s=_ptr(g.get("db2s")), dgate=_ptr(g.get("dgate")), dlogits=_ptr(g.get("dlogits")))
         return self._grads
 
-    def backward_(self, x: torch.Tensor, dy: torch.Tensor, stream=None) -> dict:
+    def backward_(self, x: torch.Tensor, dy: torch.Tensor, stream=None,
+                  dx: Optional[torch.Tensor] = None) -> dict:
         """Gradients of sum(dy * y) + the weighted balancing losses of the last
-        forward_ (same x) into the buffers of grads(); asynchronous."""
+        forward_ (same x) into the buffers of grads() (dx into the given
+        buffer when one is passed); asynchronous."""
         if not self.cfg.backward:
             raise MoEError("the layer was built without backward=1")
         _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
         _need(dy, "dy", torch.float32, (self.cfg.T, self.cfg.d), self.device)
         g = self.grads()
+        dx = g["dx"] if dx is None else dx
+        _need(dx, "dx", torch.float32, (self.cfg.T, self.cfg.d), self.device)
         st = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
         _check(_lib.load().moe_backward(C.byref(self._c), _ptr(x), C.byref(self._gp),
                                         C.byref(self._ep), _ptr(dy), _ptr(self.topk_idx),
                                         _ptr(self.topk_gate), _ptr(self.importance),
-                                        _ptr(self.load), _ptr(self.counts), _ptr(g["dx"]),
+                                        _ptr(self.load), _ptr(self.counts), _ptr(dx),
                                         C.byref(self._mg), _ptr(self.ws), self.ws.numel(),
                                         _ptr(self.status), st), "moe_backward")
         return g
+
+    def train_host_batches(self, x_hosts, dy_hosts, y_hosts, losses_hosts, dx_hosts):
+        """Training steps (forward + backward) over batches in pinned host
+        memory, pipelined like forward_host_batches: x and dy of batch i+1 go
+        to the device and y, the losses and dx of batch i-1 come back on their
+        own streams while batch i runs on the current stream.  The parameter
+        gradients stay on the device (those of the last batch).  Returns the
+        device-to-host stream after queuing; the caller synchronises."""
+        if not hasattr(self, "_tpipe"):
+            dev = self.device
+            e = lambda: [torch.empty_like(self.y) for _ in range(2)]
+            self._tpipe = dict(h2d=torch.cuda.Stream(device=dev), d2h=torch.cuda.Stream(device=dev),
+                               x=e(), dy=e(), y=e(), dx=e(),
+                               losses=[torch.empty_like(self.losses) for _ in range(2)])
+        P = self._tpipe
+        comp = torch.cuda.current_stream(self.device)
+        in_free = [None, None]    # event: device x / dy buffer b may be overwritten
+        out_free = [None, None]   # event: device y / losses / dx buffer b has been copied out
+        for i, (xh, dyh, yh, lh, dxh) in enumerate(zip(x_hosts, dy_hosts, y_hosts, losses_hosts,
+                                                       dx_hosts)):
+            b = i & 1
+            with torch.cuda.stream(P["h2d"]):
+                if in_free[b] is not None:
+                    P["h2d"].wait_event(in_free[b])
+                P["x"][b].copy_(xh, non_blocking=True)
+                P["dy"][b].copy_(dyh, non_blocking=True)
+                ready = torch.cuda.Event()
+                ready.record(P["h2d"])
+            comp.wait_event(ready)
+            if out_free[b] is not None:
+                comp.wait_event(out_free[b])
+            self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
+            self.backward_(P["x"][b], P["dy"][b], stream=comp, dx=P["dx"][b])
+            done = torch.cuda.Event()
+            done.record(comp)
+            in_free[b] = done
+            with torch.cuda.stream(P["d2h"]):
+                P["d2h"].wait_event(done)
+                yh.copy_(P["y"][b], non_blocking=True)
+                lh.copy_(P["losses"][b], non_blocking=True)
+                dxh.copy_(P["dx"][b], non_blocking=True)
+                out_free[b] = torch.cuda.Event()
+                out_free[b].record(P["d2h"])
+        return P["d2h"]
 
     def outputs(self) -> dict:
         return dict(y=self.y, topk_idx=self.topk_idx, topk_gate=self.topk_gate,

@@ -160,3 +160,32 @@ def test_backward_requires_flag_and_bf16():
     layer32.forward_(inp32["x"])
     with pytest.raises(M.MoEError):
         layer32.backward_(inp32["x"], torch.zeros_like(inp32["x"]))
+
+
+def test_train_host_batches_matches_device_path():
+    """The pipelined host-memory training path gives the same y, losses and dx,
+    bit for bit, as forward_ + backward_ on device tensors, batch by batch."""
+    w = CASES["noise-free"]
+    inp = to_dev(synth.make_inputs(w))
+    cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
+    layer = M.MoELayer(cfg, inp, torch.device(DEV))
+    xs = [synth.make_inputs(w.with_(seed=s), experts=False)["x"] for s in (1, 2, 3)]
+    dys = [synth.make_dy(w.with_(seed=s)) for s in (4, 5, 6)]
+    want = []
+    for x, dy in zip(xs, dys):
+        xd, dyd = x.to(DEV), dy.to(DEV)
+        layer.forward_(xd)
+        g = layer.backward_(xd, dyd)
+        torch.cuda.synchronize()
+        want.append((layer.y.cpu().clone(), layer.losses.cpu().clone(), g["dx"].cpu().clone()))
+    pin = lambda t: t.contiguous().pin_memory()
+    yh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
+    lh = [torch.empty(layer.losses.numel()).pin_memory() for _ in xs]
+    dxh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
+    d2h = layer.train_host_batches([pin(x) for x in xs], [pin(d) for d in dys], yh, lh, dxh)
+    d2h.synchronize()
+    torch.cuda.synchronize()
+    for i, (y, l, dx) in enumerate(want):
+        assert torch.equal(yh[i], y), i
+        assert torch.equal(lh[i], l), i
+        assert torch.equal(dxh[i], dx), i
