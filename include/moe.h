@@ -325,7 +325,7 @@ typedef struct moe_grads {
   float *dgate, *dlogits;               /* [T][k], [T][n] */
 } moe_grads;
 
-/* Backward pass of a flat layer with bf16 experts.  The pages give no
+/* Backward pass of a flat layer.  The pages give no
  * backward formulas; they fix which paths carry a gradient: the kept gates
  * are a smooth function of the logits ([SGMoE-xyz] "常見問題"), KeepTopK
  * gives the experts it drops none ([SGMoE-note] "缺点与局限性"), and the
@@ -334,18 +334,17 @@ typedef struct moe_grads {
  *   L = sum(dy * y) + losses[0] + losses[1] + losses[3]
  * (dy [T][d] fp32, the upstream gradient of moe_forward's y, plus the
  * weighted balancing losses) with respect to x (dx [T][d], fp32, written) and
- * every parameter (grads).  Mixed precision: the gradients reaching the
- * expert rows (g * dy), the hidden layer and the expert inputs are kept in
- * bf16 as the forward keeps its activations; accumulation is fp32; the gate
- * is fp32 throughout.  The selection bias of MOE_ROUTER_SIGMOID gets no
+ * every parameter (grads).  With bf16 experts (mixed precision) the gradients
+ * reaching the expert rows (g * dy), the hidden layer and the expert inputs
+ * are kept in bf16 as the forward keeps its activations, accumulation is
+ * fp32; with fp32 experts everything is fp32.  The gate is fp32 throughout.  The selection bias of MOE_ROUTER_SIGMOID gets no
  * gradient (it enters only the choice of experts).
  *
  * Preconditions: cfg->backward == 1 and ws is the workspace of the preceding
  * moe_forward with the same cfg, x and parameters, whose outputs topk_idx,
  * topk_gate, importance, load and counts are passed back here; both calls
  * on the same stream, in that order.  ws is read and overwritten.
- * Errors: MOE_EINVAL for a hierarchical layer, fp32 experts, cfg->backward
- * != 1, NULL required pointers or misaligned ones (x, dy, dx 16-byte
+ * Errors: MOE_EINVAL for a hierarchical layer, cfg->backward != 1, NULL required pointers or misaligned ones (x, dy, dx 16-byte
  * aligned); MOE_EWORKSPACE; MOE_ECUDA.  Device-side timeouts are OR-ed into
  * *status (MOE_STATUS_TIMEOUT). */
 MOE_API int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *gp,

@@ -106,13 +106,38 @@ __device__ __forceinline__ uint4 f32x8_to_bf16(const float (&f)[8]) {
   return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-// one warp per token, 8 features per lane per step
-template <int KM>
+// expert rows: 8 features as bf16 (16 bytes) or fp32 (32 bytes)
+template <bool BF16>
+__device__ __forceinline__ void load8(const void *base, size_t row, int d, int c, float (&f)[8]) {
+  if (BF16) {
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(static_cast<const __nv_bfloat16 *>(base) +
+                                                         row * d) + c), f);
+  } else {
+    const float4 *p = reinterpret_cast<const float4 *>(static_cast<const float *>(base) + row * d);
+    const float4 u = __ldg(p + 2 * c), v = __ldg(p + 2 * c + 1);
+    f[0] = u.x; f[1] = u.y; f[2] = u.z; f[3] = u.w;
+    f[4] = v.x; f[5] = v.y; f[6] = v.z; f[7] = v.w;
+  }
+}
+template <bool BF16>
+__device__ __forceinline__ void store8(void *base, size_t row, int d, int c, const float (&f)[8]) {
+  if (BF16) {
+    reinterpret_cast<uint4 *>(static_cast<__nv_bfloat16 *>(base) + row * d)[c] = f32x8_to_bf16(f);
+  } else {
+    float4 *p = reinterpret_cast<float4 *>(static_cast<float *>(base) + row * d);
+    p[2 * c] = make_float4(f[0], f[1], f[2], f[3]);
+    p[2 * c + 1] = make_float4(f[4], f[5], f[6], f[7]);
+  }
+}
+
+// one warp per token, 8 features per lane per step; BF16: the experts' rows
+// are bf16 (the gradient reaching them is rounded to bf16 like their
+// activations), else fp32
+template <int KM, bool BF16>
 __global__ void __launch_bounds__(NT) combine_bwd_kernel(
     const float *__restrict__ dy, const float *__restrict__ gate, const int *__restrict__ row_of,
-    const __nv_bfloat16 *__restrict__ y_perm, int T, int k, int d,
-    __nv_bfloat16 *__restrict__ dy_perm, float *__restrict__ dgate,
-    __nv_bfloat16 *__restrict__ dy_shared) {
+    const void *__restrict__ y_perm, int T, int k, int d, void *__restrict__ dy_perm,
+    float *__restrict__ dgate, void *__restrict__ dy_shared) {
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
@@ -132,19 +157,18 @@ __global__ void __launch_bounds__(NT) combine_bwd_kernel(
       v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
       v[4] = w.x; v[5] = w.y; v[6] = w.z; v[7] = w.w;
     }
-    if (dy_shared)
-      reinterpret_cast<uint4 *>(dy_shared + (size_t)t * d)[c] = f32x8_to_bf16(v);
+    if (dy_shared) store8<BF16>(dy_shared, (size_t)t, d, c, v);
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
       if (rows[j] < 0) continue;
       float yv[8], o[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(y_perm + (size_t)rows[j] * d) + c), yv);
+      load8<BF16>(y_perm, (size_t)rows[j], d, c, yv);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         acc[j] = fmaf(v[u], yv[u], acc[j]);
         o[u] = g[j] * v[u];
       }
-      reinterpret_cast<uint4 *>(dy_perm + (size_t)rows[j] * d)[c] = f32x8_to_bf16(o);
+      store8<BF16>(dy_perm, (size_t)rows[j], d, c, o);
     }
   }
 #pragma unroll
@@ -159,11 +183,11 @@ __global__ void __launch_bounds__(NT) combine_bwd_kernel(
 }
 
 // ---------------------------------------------------------------- dx_gather
-template <int KM>
+template <int KM, bool BF16>
 __global__ void __launch_bounds__(NT) dx_gather_kernel(
-    const __nv_bfloat16 *__restrict__ dx_perm, const int *__restrict__ row_of,
+    const void *__restrict__ dx_perm, const int *__restrict__ row_of,
     const float *__restrict__ dy, int passthrough, int T, int k, int d,
-    const __nv_bfloat16 *__restrict__ dx_shared, float *__restrict__ dx) {
+    const void *__restrict__ dx_shared, float *__restrict__ dx) {
   const int t = blockIdx.x * (NT / 32) + (threadIdx.x >> 5);
   if (t >= T) return;
   const int lane = threadIdx.x & 31;
@@ -182,7 +206,7 @@ __global__ void __launch_bounds__(NT) dx_gather_kernel(
     for (int j = 0; j < KM; ++j) {
       if (rows[j] < 0) continue;
       float v[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(dx_perm + (size_t)rows[j] * d) + c), v);
+      load8<BF16>(dx_perm, (size_t)rows[j], d, c, v);
 #pragma unroll
       for (int u = 0; u < 8; ++u) a[u] += v[u];
     }
@@ -194,7 +218,7 @@ __global__ void __launch_bounds__(NT) dx_gather_kernel(
     }
     if (dx_shared) {
       float v[8];
-      bf16x8_to_f32(__ldg(reinterpret_cast<const uint4 *>(dx_shared + (size_t)t * d) + c), v);
+      load8<BF16>(dx_shared, (size_t)t, d, c, v);
 #pragma unroll
       for (int u = 0; u < 8; ++u) a[u] += v[u];
     }
@@ -243,6 +267,77 @@ __global__ void __launch_bounds__(256) bias_grad_kernel(
 #pragma unroll
     for (int q = 0; q < 8; ++q) s += part[q][threadIdx.x];
     dst[col] = s;
+  }
+}
+
+// ---------------------------------------------------------------- expert_bwd_f32
+// fp32 experts: one block per expert walks the expert's rows in order.  Per
+// row it recomputes the hidden layer exactly as the forward's fp32 kernel
+// does (warp per unit, lanes over the input, the same shuffle reduction), then
+//   dh = (W2^T dy_perm) * [h > 0],  dx_perm = W1^T dh,
+//   dW2 += dy_perm h^T, dW1 += dh x^T, db2 += dy_perm, db1 += dh,
+// accumulated in place: the block owns its expert's gradients (each element
+// always updated by the same thread), so the result does not depend on timing.
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__global__ void __launch_bounds__(256) expert_bwd_f32_kernel(
+    const float *__restrict__ x_perm, const float *__restrict__ dy_perm,
+    const int *__restrict__ offsets, int d, int f, const float *__restrict__ W1,
+    const float *__restrict__ b1, const float *__restrict__ W2, float *__restrict__ dx_perm,
+    float *__restrict__ dW1, float *__restrict__ db1, float *__restrict__ dW2,
+    float *__restrict__ db2) {
+  extern __shared__ float sh[];
+  float *xs = sh, *gs = sh + d, *hs = sh + 2 * d, *dh = sh + 2 * d + f;
+  const int e = blockIdx.x, tid = threadIdx.x, w = tid >> 5, lane = tid & 31;
+  constexpr int NTB = 256, NWB = NTB / 32;
+  const float *W1e = W1 + (size_t)e * f * d, *W2e = W2 + (size_t)e * d * f;
+  float *dW1e = dW1 + (size_t)e * f * d, *dW2e = dW2 + (size_t)e * d * f;
+  float *db1e = db1 ? db1 + (size_t)e * f : nullptr, *db2e = db2 ? db2 + (size_t)e * d : nullptr;
+  for (int i = tid; i < f * d; i += NTB) {
+    dW1e[i] = 0.f;
+    dW2e[i] = 0.f;
+  }
+  for (int j = tid; j < f; j += NTB)
+    if (db1e) db1e[j] = 0.f;
+  for (int q = tid; q < d; q += NTB)
+    if (db2e) db2e[q] = 0.f;
+  const int r0 = offsets[e], r1 = offsets[e + 1];
+  for (int r = r0; r < r1; ++r) {
+    for (int q = tid; q < d; q += NTB) {
+      xs[q] = x_perm[(size_t)r * d + q];
+      gs[q] = dy_perm[(size_t)r * d + q];
+    }
+    __syncthreads();
+    for (int j = w; j < f; j += NWB) {  // the forward's hidden unit j
+      const float *wr = W1e + (size_t)j * d;
+      float acc = 0.f;
+      for (int q = lane; q < d; q += 32) acc = fmaf(xs[q], wr[q], acc);
+      acc = warp_sum_f(acc);
+      if (lane == 0) hs[j] = fmaxf(acc + (b1 ? b1[(size_t)e * f + j] : 0.f), 0.f);
+    }
+    __syncthreads();
+    for (int j = tid; j < f; j += NTB) {
+      float acc = 0.f;
+      for (int q = 0; q < d; ++q) acc = fmaf(W2e[(size_t)q * f + j], gs[q], acc);
+      dh[j] = hs[j] > 0.f ? acc : 0.f;  // ReLU passes the gradient where it is positive
+    }
+    __syncthreads();
+    for (int q = tid; q < d; q += NTB) {
+      float acc = 0.f;
+      for (int j = 0; j < f; ++j) acc = fmaf(W1e[(size_t)j * d + q], dh[j], acc);
+      dx_perm[(size_t)r * d + q] = acc;
+    }
+    for (int i = tid; i < d * f; i += NTB) dW2e[i] = fmaf(gs[i / f], hs[i % f], dW2e[i]);
+    for (int i = tid; i < f * d; i += NTB) dW1e[i] = fmaf(dh[i / d], xs[i % d], dW1e[i]);
+    if (db2e)
+      for (int q = tid; q < d; q += NTB) db2e[q] += gs[q];
+    if (db1e)
+      for (int j = tid; j < f; j += NTB) db1e[j] += dh[j];
+    __syncthreads();  // xs, gs, hs, dh are rewritten by the next row
   }
 }
 
@@ -587,35 +682,59 @@ int launch_bwd_coef(const float *importance, const float *load, const int *count
 }
 
 int launch_combine_bwd(const float *dy, const float *gate, const int *row_of, const void *y_perm,
-                       int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
+                       int bf16, int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
                        cudaStream_t st) {
   if (k > kMaxK) return MOE_EINVAL;
   const dim3 grid((unsigned)ceil_div(T, NT / 32));
   auto go = [&](auto kern) {
-    return launch("combine_bwd", kern, grid, dim3(NT), 0, st, dy, gate, row_of,
-                  static_cast<const __nv_bfloat16 *>(y_perm), T, k, d,
-                  static_cast<__nv_bfloat16 *>(dy_perm), dgate,
-                  static_cast<__nv_bfloat16 *>(dy_shared));
+    return launch("combine_bwd", kern, grid, dim3(NT), 0, st, dy, gate, row_of, y_perm, T, k, d,
+                  dy_perm, dgate, dy_shared);
   };
-  if (k <= 1) return go(combine_bwd_kernel<1>);
-  if (k <= 2) return go(combine_bwd_kernel<2>);
-  if (k <= 4) return go(combine_bwd_kernel<4>);
-  return go(combine_bwd_kernel<8>);
+  if (bf16) {
+    if (k <= 1) return go(combine_bwd_kernel<1, true>);
+    if (k <= 2) return go(combine_bwd_kernel<2, true>);
+    if (k <= 4) return go(combine_bwd_kernel<4, true>);
+    return go(combine_bwd_kernel<8, true>);
+  }
+  if (k <= 1) return go(combine_bwd_kernel<1, false>);
+  if (k <= 2) return go(combine_bwd_kernel<2, false>);
+  if (k <= 4) return go(combine_bwd_kernel<4, false>);
+  return go(combine_bwd_kernel<8, false>);
 }
 
-int launch_dx_gather(const void *dx_perm, const int *row_of, const float *dy, int passthrough,
-                     int T, int k, int d, const void *dx_shared, float *dx, cudaStream_t st) {
+int launch_expert_bwd_f32(const float *x_perm, const float *dy_perm, const int *offsets, int n,
+                          int d, int f, const float *W1, const float *b1, const float *W2,
+                          float *dx_perm, float *dW1, float *db1, float *dW2, float *db2,
+                          const char *name, cudaStream_t st) {
+  const size_t smem = sizeof(float) * (size_t)(2 * d + 2 * f);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(expert_bwd_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem) != cudaSuccess)
+    return MOE_EINVAL;
+  return launch(name ? name : "expert_bwd_fp32", expert_bwd_f32_kernel, dim3((unsigned)n),
+                dim3(256), smem, st, x_perm, dy_perm, offsets, d, f, W1, b1, W2, dx_perm, dW1, db1,
+                dW2, db2);
+}
+
+int launch_dx_gather(const void *dx_perm, int bf16, const int *row_of, const float *dy,
+                     int passthrough, int T, int k, int d, const void *dx_shared, float *dx,
+                     cudaStream_t st) {
   if (k > kMaxK) return MOE_EINVAL;
   const dim3 grid((unsigned)ceil_div(T, NT / 32));
   auto go = [&](auto kern) {
-    return launch("dx_gather", kern, grid, dim3(NT), 0, st,
-                  static_cast<const __nv_bfloat16 *>(dx_perm), row_of, dy, passthrough, T, k, d,
-                  static_cast<const __nv_bfloat16 *>(dx_shared), dx);
+    return launch("dx_gather", kern, grid, dim3(NT), 0, st, dx_perm, row_of, dy, passthrough, T,
+                  k, d, dx_shared, dx);
   };
-  if (k <= 1) return go(dx_gather_kernel<1>);
-  if (k <= 2) return go(dx_gather_kernel<2>);
-  if (k <= 4) return go(dx_gather_kernel<4>);
-  return go(dx_gather_kernel<8>);
+  if (bf16) {
+    if (k <= 1) return go(dx_gather_kernel<1, true>);
+    if (k <= 2) return go(dx_gather_kernel<2, true>);
+    if (k <= 4) return go(dx_gather_kernel<4, true>);
+    return go(dx_gather_kernel<8, true>);
+  }
+  if (k <= 1) return go(dx_gather_kernel<1, false>);
+  if (k <= 2) return go(dx_gather_kernel<2, false>);
+  if (k <= 4) return go(dx_gather_kernel<4, false>);
+  return go(dx_gather_kernel<8, false>);
 }
 
 int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,

@@ -194,11 +194,20 @@ struct GateBwdArgs {
 int launch_bwd_coef(const float *importance, const float *load, const int *counts, int n, int T,
                     float w_imp, float w_load, float alpha, int router, int noise, float *lam_imp,
                     float *lam_load, float *sw_coef, cudaStream_t st);
+// bf16: the expert rows (y_perm, dy_perm, dy_shared / dx_perm, dx_shared)
+// are bf16, else fp32
 int launch_combine_bwd(const float *dy, const float *gate, const int *row_of, const void *y_perm,
-                       int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
+                       int bf16, int T, int k, int d, void *dy_perm, float *dgate, void *dy_shared,
                        cudaStream_t st);
-int launch_dx_gather(const void *dx_perm, const int *row_of, const float *dy, int passthrough,
-                     int T, int k, int d, const void *dx_shared, float *dx, cudaStream_t st);
+int launch_dx_gather(const void *dx_perm, int bf16, const int *row_of, const float *dy,
+                     int passthrough, int T, int k, int d, const void *dx_shared, float *dx,
+                     cudaStream_t st);
+// fp32 experts' backward: block per expert, gradients written whole (zeroed
+// first); db1, db2 may be nullptr
+int launch_expert_bwd_f32(const float *x_perm, const float *dy_perm, const int *offsets, int n,
+                          int d, int f, const float *W1, const float *b1, const float *W2,
+                          float *dx_perm, float *dW1, float *db1, float *dW2, float *db2,
+                          const char *name, cudaStream_t st);
 int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,
                      int f, float *db2, float *db1, const char *name, cudaStream_t st);
 int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st);

@@ -814,7 +814,7 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   Layout L;
   MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
   const moe_config &c = *cfg;
-  if (!c.backward || c.hier_a > 0 || c.expert_dtype != MOE_BF16) return MOE_EINVAL;
+  if (!c.backward || c.hier_a > 0) return MOE_EINVAL;
   if (!gr || !gr->dW1 || !gr->dW2 || !importance || !load || !counts) return MOE_EINVAL;
   if (!aligned(gr->dW1, 16) || !aligned(gr->dW2, 16)) return MOE_EINVAL;
   if (c.T > 0 && (!x || !dy || !dx || !topk_idx || !topk_gate || !aligned(x, 16) ||
@@ -868,8 +868,23 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   MOE_TRY(launch_bwd_coef(importance, load, counts, n, T, c.w_importance, c.w_load, c.alpha_aux,
                           c.router, c.noise, lam_imp, lam_load, sw_coef, side->s));
   // ---- combine: dy_perm rows, dL/dgate, the shared expert's rows
-  MOE_TRY(launch_combine_bwd(dy, topk_gate, row_of, at<void>(ws, L.y_perm), T, k, d, dy_perm,
+  const bool tc = c.expert_dtype == MOE_BF16;
+  MOE_TRY(launch_combine_bwd(dy, topk_gate, row_of, at<void>(ws, L.y_perm), tc, T, k, d, dy_perm,
                              dgate, dy_sh, st));
+  if (!tc) {
+    // fp32 experts: per expert, its rows in order, gradients accumulated in place
+    MOE_TRY(launch_expert_bwd_f32(at<float>(ws, L.x_perm), static_cast<const float *>(dy_perm),
+                                  offsets, n, d, f, static_cast<const float *>(ep->W1), ep->b1,
+                                  static_cast<const float *>(ep->W2),
+                                  static_cast<float *>(dx_perm), gr->dW1, gr->db1, gr->dW2,
+                                  gr->db2, nullptr, st));
+    if (c.shared_expert)
+      MOE_TRY(launch_expert_bwd_f32(
+          at<float>(ws, L.x_shared), static_cast<const float *>(dy_sh), at<int>(ws, L.shared_off),
+          1, d, f, static_cast<const float *>(ep->W1s), ep->b1s,
+          static_cast<const float *>(ep->W2s), static_cast<float *>(dx_sh), gr->dW1s, gr->db1s,
+          gr->dW2s, gr->db2s, "shared_expert_bwd_fp32", st));
+  } else {
   // ---- experts: dhid = (dy_perm W2) * [hid > 0], dx_perm = dhid W1 (the forward's tiles)
   const int64_t mb_upper = ceil_div((int64_t)S, kExpertBM) + n;
   if (cudaMemsetAsync(at<int>(ws, L.mdone), 0, 4 * (size_t)(mb_upper + 1), st) != cudaSuccess)
@@ -944,8 +959,10 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
     MOE_TRY(launch_bias_grad(dy_sh, dhid_sh, at<int>(ws, L.shared_off), 1, d, f, gr->db2s,
                              gr->db1s, "shared_bias_grad", st));
   }
+  }  // bf16 experts
   // ---- dispatch: dx = sum of the token's expert rows (+ pass-through, + shared)
-  MOE_TRY(launch_dx_gather(dx_perm, row_of, dy, c.overflow_passthrough, T, k, d, dx_sh, dx, st));
+  MOE_TRY(launch_dx_gather(dx_perm, tc, row_of, dy, c.overflow_passthrough, T, k, d, dx_sh, dx,
+                           st));
   // ---- gate: dL/dc, dL/dz per token, then the fp32 contractions
   GateBwdArgs g{};
   g.T = T;

@@ -6,7 +6,7 @@ hidden-layer gradient and input-row gradients; fp32 gates), so what remains
 is fp32-versus-fp64 accumulation order and the odd bf16 rounding that lands
 on the other side of a tie: every gradient within 1e-2 relative Frobenius
 of the oracle's (bf16 carries 8 bits), the gate gradient dL/dgate within
-5e-3.  Cases whose routing has near ties (k-th and (k+1)-th logits closer
+5e-3.  With fp32 experts nothing is rounded: 1e-4 for all.  Cases whose routing has near ties (k-th and (k+1)-th logits closer
 than 1e-5) are skipped: a flipped choice changes the whole token."""
 import dataclasses
 
@@ -72,6 +72,11 @@ CASES = {
                                                    w_importance=0.3),
     "shared-noisy-passthrough": W["lm-flat"].with_(T=200, n=32, k=2, d=64, f=64, shared_expert=1,
                                                    capacity_factor=0.5, passthrough=1, **LOSSES),
+    # fp32 experts (everything fp32: 1e-4)
+    "f32-tiny": W["tiny-flat"].with_(**LOSSES),
+    "f32-capacity": W["tiny-flat"].with_(T=200, n=6, k=2, d=40, f=24, capacity_factor=0.7,
+                                         passthrough=1, bias_var=0.1, **LOSSES),
+    "f32-sigmoid-shared": V["deepseek-tiny-f32"].with_(w_importance=0.3),
 }
 
 GRAD_KEYS = [("dx", "dx"), ("dWg", "dWg"), ("dbg", "dbg"), ("dWn", "dWn"), ("dW1", "dW1"),
@@ -107,14 +112,15 @@ def test_backward_matches_oracle(orc, name):
     assert np.array_equal(fwd["topk_idx"].numpy(), ref_f["topk_idx"])
     assert np.array_equal(fwd["counts"].numpy(), ref_f["counts"])
     ref = orc.backward(w.cfg(), np_inputs(inp), dy.numpy())
-    assert rel_fro(got["dgate"], ref["dgate"]) < 5e-3
+    tol, tol_g = (1e-2, 5e-3) if w.expert_bf16 else (1e-4, 1e-4)
+    assert rel_fro(got["dgate"], ref["dgate"]) < tol_g
     for gk, rk in GRAD_KEYS:
         if gk not in got or rk not in ref:
             continue
         if not np.any(ref[rk]) and not np.any(got[gk]):
             continue
         err = rel_fro(got[gk], ref[rk])
-        assert err < 1e-2, (gk, err)
+        assert err < tol, (gk, err)
     # experts that received no rows get exactly zero weight gradients
     empty = np.flatnonzero(ref_f["counts"] == 0)
     assert not np.any(got["dW1"][empty]) and not np.any(got["dW2"][empty])
@@ -147,19 +153,23 @@ def test_backward_zero_tokens():
             assert torch.all(v == 0), k
 
 
-def test_backward_requires_flag_and_bf16():
+def test_backward_requires_flag():
     w = CASES["noise-free"]
     inp = to_dev(synth.make_inputs(w))
     layer = M.MoELayer(M.Config.from_workload(w), inp, torch.device(DEV))
     with pytest.raises(M.MoEError):
         layer.backward_(inp["x"], torch.zeros_like(inp["x"]))
-    w32 = w.with_(expert_bf16=0)
-    inp32 = to_dev(synth.make_inputs(w32))
-    cfg32 = dataclasses.replace(M.Config.from_workload(w32), backward=1)
-    layer32 = M.MoELayer(cfg32, inp32, torch.device(DEV))
-    layer32.forward_(inp32["x"])
-    with pytest.raises(M.MoEError):
-        layer32.backward_(inp32["x"], torch.zeros_like(inp32["x"]))
+    # the C ABI refuses too (the flag sizes the workspace and keeps the state)
+    from sparsely_gated_mixture_gate_b200 import _lib
+    import ctypes as C
+    g = layer.grads()
+    rc = _lib.load().moe_backward(C.byref(layer._c), M._ptr(inp["x"]), C.byref(layer._gp),
+                                  C.byref(layer._ep), M._ptr(inp["x"]), M._ptr(layer.topk_idx),
+                                  M._ptr(layer.topk_gate), M._ptr(layer.importance),
+                                  M._ptr(layer.load), M._ptr(layer.counts), M._ptr(g["dx"]),
+                                  C.byref(layer._mg), M._ptr(layer.ws), layer.ws.numel(),
+                                  M._ptr(layer.status), None)
+    assert rc == _lib.MOE_EINVAL
 
 
 def test_train_host_batches_matches_device_path():
