@@ -72,6 +72,9 @@ CASES = {
                                                    w_importance=0.3),
     "shared-noisy-passthrough": W["lm-flat"].with_(T=200, n=32, k=2, d=64, f=64, shared_expert=1,
                                                    capacity_factor=0.5, passthrough=1, **LOSSES),
+    # the largest slot count, and a gate wider than the register path (n > 1024)
+    "k8-n64": W["lm-flat"].with_(T=200, n=64, k=8, d=64, f=64, **LOSSES),
+    "wide-n2000": W["lm-flat"].with_(T=128, n=2000, k=2, d=64, f=32, **LOSSES),
     # fp32 experts (everything fp32: 1e-4)
     "f32-tiny": W["tiny-flat"].with_(**LOSSES),
     "f32-capacity": W["tiny-flat"].with_(T=200, n=6, k=2, d=40, f=24, capacity_factor=0.7,
