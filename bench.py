@@ -4,7 +4,9 @@
 
 One step = one full forward pass (gate, dispatch, experts, combine, balancing
 statistics) of one batch of the workload through the fused C-ABI call
-``moe_forward``.  Inputs are resident in HBM; L2 is flushed (256 MiB write)
+``moe_forward``, its launches replayed from a CUDA graph captured from that
+call (``MoELayer.forward_graph_``; ``--no-graph`` times direct calls).  Inputs
+are resident in HBM; L2 is flushed (256 MiB write)
 before every timed step, and every step is timed on the device with CUDA
 events on the launching stream; the total is the max over ranks.  With N > 1
 (launched by torchrun) every rank runs its own independent batch on its own
@@ -241,10 +243,25 @@ def run_ours(args, w, world, rank, local):
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
+    # the forward pass's launches are replayed from a CUDA graph (one host call
+    # per step; the same kernels on the same buffers) unless --no-graph
+    use_graph = not args.no_graph and dy is None
+
     def step():
+        if use_graph:
+            layer.forward_graph_(x)
+            return
         layer.forward_(x)
         if dy is not None:
             layer.backward_(x, dy)
+
+    # kernels per step, counted on one direct call (a graph replay launches the
+    # same kernels without passing through the library's launch counter)
+    l0 = M.launch_count()
+    layer.forward_(x)
+    if dy is not None:
+        layer.backward_(x, dy)
+    per_step_launches = M.launch_count() - l0
 
     for _ in range(args.warmup):
         flush.fill_(1.0)
@@ -274,7 +291,7 @@ def run_ours(args, w, world, rank, local):
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - wall0
-    launches = M.launch_count() - launches0
+    launches = per_step_launches * args.steps if use_graph else M.launch_count() - launches0
     clk = clocks.stop()
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
     ms, value = aggregate(total_ms, w.T, args.steps, world)
@@ -442,6 +459,8 @@ def run_ours(args, w, world, rank, local):
                    else "fp32 multiply-adds",
                    "capacity_factor": w.capacity_factor or None,
                    "l2": "flushed before every timed step (256 MiB write)",
+                   "launch": ("one CUDA graph replay per step (captured from moe_forward)"
+                              if use_graph else "direct C-ABI calls"),
                    "parallelism": f"replicas x{world}"},
         "expert_ffn_tflops": round(ffn_flops / (ffn_ms / 1e3) / 1e12, 2) if ffn_ms else None,
         "expert_ffn_frac_bf16_peak": round(ffn_flops / (ffn_ms / 1e3) / 1e12 / sustained, 4) if ffn_ms else None,
@@ -450,6 +469,7 @@ def run_ours(args, w, world, rank, local):
         "kernels": kstats,
         "kernel_timing": f"second pass of {t_steps} steps, CUDA events around every library launch",
         "gpu_launches": int(launches),
+        "gpu_launches_per_step": int(per_step_launches),
         "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "steps": e_steps,
                 "how": ("pinned host x in, y and losses out every step; copies of neighbouring "
@@ -551,6 +571,8 @@ def main():
     ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
                     help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time direct library calls instead of a CUDA graph replay of the forward")
     ap.add_argument("--backward", action="store_true",
                     help="time forward + backward (training step) instead of the forward pass")
     ap.add_argument("--no-alt-gate", dest="alt_gate", action="store_false",

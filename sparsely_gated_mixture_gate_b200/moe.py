@@ -305,6 +305,33 @@ class MoELayer:
                                        _ptr(self.status), st), "moe_forward")
         return y
 
+    def forward_graph_(self, x: torch.Tensor) -> torch.Tensor:
+        """forward_ replayed from a CUDA graph on the current stream.  The
+        graph is captured on the first call for this x buffer (its address is
+        baked in: later calls must pass the same tensor, whose contents may
+        change between calls); the library's launches, the side stream's fork
+        and join and its memsets are all captured, so a replay runs the same
+        kernels on the same buffers with one host call."""
+        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        if getattr(self, "_graph_x", None) != x.data_ptr():
+            self._graph = None
+            cap = torch.cuda.Stream(device=self.device)
+            cap.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(cap):
+                self.forward_(x, stream=cap)  # one-time set-up outside the capture
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                self.forward_(x, stream=cap)
+            torch.cuda.current_stream(self.device).wait_stream(cap)
+            self._graph, self._graph_x = g, x.data_ptr()
+        self._graph.replay()
+        return self.y
+
+    def release_graph(self):
+        """Drop the captured forward graph."""
+        self._graph = None
+        self._graph_x = None
+
     def grads(self, intermediates: bool = False) -> dict:
         """Gradient buffers of this layer (allocated on first use), fp32 in
         the parameters' layouts; with intermediates also dgate [T][k] and

@@ -418,3 +418,31 @@ def test_pipelined_host_batches_match_device_calls():
         torch.cuda.synchronize()
         assert torch.equal(ys[i], layer.y.cpu()), i
         assert torch.equal(ls[i], layer.losses.cpu()), i
+
+
+def test_forward_graph_replay_matches_direct():
+    """The CUDA-graph replay of moe_forward (MoELayer.forward_graph_) gives the
+    direct call's outputs bit for bit, and follows new contents of the same
+    input buffer."""
+    for name in ("lm-flat-512", "deepseek-tiny", "switch-skew-small"):
+        w = SMALL[name]
+        inp = synth.make_inputs(w)
+        dinp = to_dev(inp)
+        layer = M.MoELayer(M.Config.from_workload(w), dinp, torch.device(DEV))
+        x = dinp["x"]
+        x2 = synth.make_inputs(w.with_(seed=w.seed + 7), experts=False)["x"].to(DEV)
+        outs = []
+        for src in (x.clone(), x2):
+            x.copy_(src)
+            layer.forward_(x)
+            torch.cuda.synchronize()
+            want = {k: v.clone() for k, v in layer.outputs().items()}
+            layer.y.zero_()
+            layer.forward_graph_(x)
+            torch.cuda.synchronize()
+            got = layer.outputs()
+            for k in ("y", "topk_idx", "topk_gate", "importance", "load", "counts", "losses"):
+                assert torch.equal(got[k], want[k]), (name, k)
+            outs.append(want["y"])
+        assert not torch.equal(outs[0], outs[1])
+        layer.release_graph()
