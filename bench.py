@@ -365,9 +365,10 @@ def run_ours(args, w, world, rank, local):
     if args.alt_gate and world == 1 and dy is None:
         other = 0 if w.gate_precision else 1
         alt_layer = M.MoELayer(M.Config.from_workload(w.with_(gate_precision=other)), inp, dev)
+        alt_step = alt_layer.forward_graph_ if use_graph else alt_layer.forward_
         for _ in range(3):
             flush.fill_(1.0)
-            alt_layer.forward_(x)
+            alt_step(x)
         torch.cuda.synchronize()
         a_steps = max(3, min(args.steps, 300))
         as_ = [torch.cuda.Event(enable_timing=True) for _ in range(a_steps)]
@@ -375,13 +376,14 @@ def run_ours(args, w, world, rank, local):
         for i in range(a_steps):
             flush.fill_(float(i))
             as_[i].record(stream)
-            alt_layer.forward_(x)
+            alt_step(x)
             ae_[i].record(stream)
         torch.cuda.synchronize()
         a_ms = sum(p.elapsed_time(q) for p, q in zip(as_, ae_))
         alt = {"gate": "tf32x3" if other else "fp32", "value": round(w.T * a_steps / (a_ms / 1e3), 1),
                "ms_per_step": round(a_ms / a_steps, 5), "steps": a_steps,
                "device_status": M.status_bits(alt_layer.status)}
+        alt_layer.release_graph()
         del alt_layer
 
     if rank != 0:
