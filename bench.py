@@ -247,20 +247,21 @@ def run_ours(args, w, world, rank, local):
     # per step; the same kernels on the same buffers) unless --no-graph
     use_graph = not args.no_graph and dy is None
 
-    def step():
-        if use_graph:
-            layer.forward_graph_(x)
-            return
+    def direct_step():
         layer.forward_(x)
         if dy is not None:
             layer.backward_(x, dy)
 
+    def step():
+        if use_graph:
+            layer.forward_graph_(x)
+        else:
+            direct_step()
+
     # kernels per step, counted on one direct call (a graph replay launches the
     # same kernels without passing through the library's launch counter)
     l0 = M.launch_count()
-    layer.forward_(x)
-    if dy is not None:
-        layer.backward_(x, dy)
+    direct_step()
     per_step_launches = M.launch_count() - l0
 
     for _ in range(args.warmup):
@@ -298,14 +299,15 @@ def run_ours(args, w, world, rank, local):
 
     # ---- second timed pass for the roofline: CUDA events recorded by the
     # library around each of its launches, on the launching stream (the
-    # events add a little time per launch, so this pass is not the value)
+    # events add a little time per launch, so this pass is not the value;
+    # direct calls, so it times every kernel without the graph's tighter gaps)
     t_steps = max(3, min(args.steps, 300))
     M.trace_reset()
     M.trace_enable(True)
     torch.cuda.synchronize()
     for i in range(t_steps):
         flush.fill_(float(i))
-        step()
+        direct_step()  # the library's events need its own launches, not a graph replay
     torch.cuda.synchronize()
     M.trace_enable(False)
     per_kernel = M.trace_read()
