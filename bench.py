@@ -245,7 +245,7 @@ def run_ours(args, w, world, rank, local):
 
     # the forward pass's launches are replayed from a CUDA graph (one host call
     # per step; the same kernels on the same buffers) unless --no-graph
-    use_graph = not args.no_graph and dy is None
+    use_graph = not args.no_graph
 
     def direct_step():
         layer.forward_(x)
@@ -253,10 +253,12 @@ def run_ours(args, w, world, rank, local):
             layer.backward_(x, dy)
 
     def step():
-        if use_graph:
+        if not use_graph:
+            direct_step()
+        elif dy is None:
             layer.forward_graph_(x)
         else:
-            direct_step()
+            layer.train_graph_(x, dy)
 
     # kernels per step, counted on one direct call (a graph replay launches the
     # same kernels without passing through the library's launch counter)
@@ -463,7 +465,8 @@ def run_ours(args, w, world, rank, local):
                    else "fp32 multiply-adds",
                    "capacity_factor": w.capacity_factor or None,
                    "l2": "flushed before every timed step (256 MiB write)",
-                   "launch": ("one CUDA graph replay per step (captured from moe_forward)"
+                   "launch": (("one CUDA graph replay per step (captured from moe_forward"
+                               + (" and moe_backward)" if dy is not None else ")"))
                               if use_graph else "direct C-ABI calls"),
                    "parallelism": f"replicas x{world}"},
         "expert_ffn_tflops": round(ffn_flops / (ffn_ms / 1e3) / 1e12, 2) if ffn_ms else None,

@@ -327,10 +327,36 @@ class MoELayer:
         self._graph.replay()
         return self.y
 
+    def train_graph_(self, x: torch.Tensor, dy: torch.Tensor) -> dict:
+        """forward_ then backward_ replayed from one CUDA graph on the current
+        stream, captured on the first call for these x and dy buffers (same
+        tensors on later calls; their contents may change)."""
+        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        _need(dy, "dy", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        key = (x.data_ptr(), dy.data_ptr())
+        if getattr(self, "_tgraph_key", None) != key:
+            self._tgraph = None
+            self.grads()
+            cap = torch.cuda.Stream(device=self.device)
+            cap.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(cap):
+                self.forward_(x, stream=cap)  # one-time set-up outside the capture
+                self.backward_(x, dy, stream=cap)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
+                self.forward_(x, stream=cap)
+                self.backward_(x, dy, stream=cap)
+            torch.cuda.current_stream(self.device).wait_stream(cap)
+            self._tgraph, self._tgraph_key = g, key
+        self._tgraph.replay()
+        return self._grads
+
     def release_graph(self):
-        """Drop the captured forward graph."""
+        """Drop the captured graphs."""
         self._graph = None
         self._graph_x = None
+        self._tgraph = None
+        self._tgraph_key = None
 
     def grads(self, intermediates: bool = False) -> dict:
         """Gradient buffers of this layer (allocated on first use), fp32 in

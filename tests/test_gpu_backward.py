@@ -202,3 +202,28 @@ def test_train_host_batches_matches_device_path():
         assert torch.equal(yh[i], y), i
         assert torch.equal(lh[i], l), i
         assert torch.equal(dxh[i], dx), i
+
+
+def test_train_graph_replay_matches_direct():
+    """forward + backward replayed from one CUDA graph (MoELayer.train_graph_)
+    give the direct calls' outputs and gradients bit for bit."""
+    w = CASES["noisy-ragged-capacity"]
+    inp = to_dev(synth.make_inputs(w))
+    cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
+    layer = M.MoELayer(cfg, inp, torch.device(DEV))
+    x = inp["x"]
+    dy = synth.make_dy(w).to(DEV)
+    layer.forward_(x)
+    g = layer.backward_(x, dy)
+    torch.cuda.synchronize()
+    want = {k: v.clone() for k, v in g.items()}
+    want_y = layer.y.clone()
+    for v in g.values():
+        v.zero_()
+    layer.y.zero_()
+    layer.train_graph_(x, dy)
+    torch.cuda.synchronize()
+    assert torch.equal(layer.y, want_y)
+    for k, v in layer.grads().items():
+        assert torch.equal(v, want[k]), k
+    layer.release_graph()
