@@ -83,6 +83,7 @@ BAD = [
     dict(hier_a=4, hier_b=2, hier_k1=5, hier_k2=1, n=8, k=5),
     dict(passthrough=2), dict(capacity_factor=float("nan")),
     dict(raw_expert_dtype=3), dict(raw_gate_precision=2),
+    dict(raw_backward=2), dict(raw_shared_expert=2), dict(raw_router_stats=-1),
 ]
 
 
@@ -135,3 +136,24 @@ def test_calls_fail_cleanly_without_gpu(lib):
     import torch
     if not torch.cuda.is_available():
         assert rc == _lib.MOE_EDEVICE
+
+
+def test_backward_workspace_and_refusals_without_gpu(lib):
+    """backward = 1 adds the backward's scratch to the workspace; the entry
+    point checks its arguments on the host before anything touches a device."""
+    cfg = M.Config(T=64, d=32, n=8, k=2, f=64)
+    import dataclasses
+    bwd = dataclasses.replace(cfg, backward=1)
+    assert M.workspace_size(bwd) > M.workspace_size(cfg)
+    assert M.workspace_size(dataclasses.replace(bwd, shared_expert=1)) > M.workspace_size(bwd)
+    c = cfg.c()
+    g = _lib.moe_grads()
+    # no backward flag -> EINVAL (before any device work; a NULL workspace is
+    # refused first, either way not MOE_OK)
+    rc = lib.moe_backward(C.byref(c), None, None, None, None, None, None, None, None, None, None,
+                          C.byref(g), None, 0, None, None)
+    assert rc in (_lib.MOE_EINVAL, _lib.MOE_EWORKSPACE, _lib.MOE_EDEVICE)
+    cb = bwd.c()
+    rc = lib.moe_backward(C.byref(cb), None, None, None, None, None, None, None, None, None, None,
+                          None, None, 0, None, None)
+    assert rc != _lib.MOE_OK
