@@ -1,4 +1,5 @@
-// backward.cu -- the memory-bound kernels of the layer's backward pass.
+// backward.cu -- the layer's backward pass apart from the tensor-core GEMMs
+// (expert_tc.cu, wgrad_tc.cu) and the gate's fp32 GEMMs (grad_gemm.cu).
 //
 // The pages give no backward formulas; they say which paths carry a
 // gradient: the kept gates are smooth in the logits ([SGMoE-xyz] 常見問題),
@@ -14,12 +15,15 @@
 //                   dgate = <dy_t, y_perm[row]>; the shared expert's rows get dy
 //   bias_grad       db of every expert: column sums of its rows of dy_perm and
 //                   dhid, in a fixed order
+//   expert_bwd_f32  fp32 experts: block per expert over its rows, the hidden
+//                   layer recomputed, dW1, dW2, db1, db2 accumulated in place
 //   dx_gather       dx_t = sum over kept slots of dx_perm[row] (+ dy_t for a
 //                   passed-through token, + the shared expert's row)
 //   gate_bwd        per token: dL/dc (clean logits) and dL/dz (noise logits,
 //                   z = x W_noise) through the softmax over the kept, the
 //                   importance and load losses (Phi' and kth_excluding), the
-//                   noise (eps recomputed from Philox) and Softplus
+//                   noise (eps recomputed from Philox) and Softplus; for the
+//                   noisy gate up to 1024 experts the row sits in registers
 //   colsum          column sums of a row-major matrix in row blocks (db_g)
 #include "internal.h"
 #include "philox.cuh"
