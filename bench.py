@@ -323,7 +323,7 @@ def run_ours(args, w, world, rank, local):
     lh = [torch.empty(layer.losses.numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
     if dy is None:
         layer.forward_host_batches([xh] * 3, [yh[i & 1] for i in range(3)],
-                                   [lh[i & 1] for i in range(3)])
+                                   [lh[i & 1] for i in range(3)], graph=use_graph)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
@@ -331,7 +331,7 @@ def run_ours(args, w, world, rank, local):
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         d2h = layer.forward_host_batches([xh] * e_steps, [yh[i & 1] for i in range(e_steps)],
-                                         [lh[i & 1] for i in range(e_steps)])
+                                         [lh[i & 1] for i in range(e_steps)], graph=use_graph)
         stream.wait_stream(d2h)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -346,7 +346,7 @@ def run_ours(args, w, world, rank, local):
         def host_steps(m):
             return layer.train_host_batches([xh] * m, [dyh] * m, [yh[i & 1] for i in range(m)],
                                             [lh[i & 1] for i in range(m)],
-                                            [dxh[i & 1] for i in range(m)])
+                                            [dxh[i & 1] for i in range(m)], graph=use_graph)
 
         host_steps(3)
         torch.cuda.synchronize()
@@ -480,7 +480,9 @@ def run_ours(args, w, world, rank, local):
         "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
                 "d2h_bytes_per_step": d2h_bytes, "steps": e_steps,
                 "how": ("pinned host x in, y and losses out every step; copies of neighbouring "
-                        "steps overlap compute on two copy streams") if dy is None else
+                        "steps overlap compute on two copy streams"
+                        + ("; each step's forward replayed from a CUDA graph" if use_graph else ""))
+                       if dy is None else
                        ("pinned host x and dy in, y, losses and dx out every step; copies of "
                         "neighbouring steps overlap compute on two copy streams (parameter "
                         "gradients stay on the device)")},

@@ -305,58 +305,64 @@ class MoELayer:
                                        _ptr(self.status), st), "moe_forward")
         return y
 
-    def forward_graph_(self, x: torch.Tensor) -> torch.Tensor:
-        """forward_ replayed from a CUDA graph on the current stream.  The
-        graph is captured on the first call for this x buffer (its address is
-        baked in: later calls must pass the same tensor, whose contents may
-        change between calls); the library's launches, the side stream's fork
-        and join and its memsets are all captured, so a replay runs the same
-        kernels on the same buffers with one host call."""
-        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
-        if getattr(self, "_graph_x", None) != x.data_ptr():
-            self._graph = None
+    def _graph(self, key, record):
+        """The CUDA graph captured for these buffers (key), captured on first
+        use: record() issues the calls on the given stream, once outside the
+        capture (one-time set-up) and once inside it."""
+        graphs = self.__dict__.setdefault("_graphs", {})
+        g = graphs.get(key)
+        if g is None:
             cap = torch.cuda.Stream(device=self.device)
             cap.wait_stream(torch.cuda.current_stream(self.device))
             with torch.cuda.stream(cap):
-                self.forward_(x, stream=cap)  # one-time set-up outside the capture
+                record(cap)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
-                self.forward_(x, stream=cap)
+                record(cap)
             torch.cuda.current_stream(self.device).wait_stream(cap)
-            self._graph, self._graph_x = g, x.data_ptr()
-        self._graph.replay()
-        return self.y
+            graphs[key] = g
+        return g
 
-    def train_graph_(self, x: torch.Tensor, dy: torch.Tensor) -> dict:
+    def forward_graph_(self, x: torch.Tensor, y: Optional[torch.Tensor] = None,
+                       losses: Optional[torch.Tensor] = None) -> torch.Tensor:
+        """forward_ replayed from a CUDA graph on the current stream.  A graph
+        is captured on the first call for each set of buffers (x, y, losses;
+        their addresses are baked in, their contents may change between
+        calls); the library's launches, the side stream's fork and join and
+        its memsets are all captured, so a replay runs the same kernels on the
+        same buffers with one host call."""
+        _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
+        y = self.y if y is None else y
+        losses = self.losses if losses is None else losses
+        g = self._graph(("fwd", x.data_ptr(), y.data_ptr(), losses.data_ptr()),
+                        lambda st: self.forward_(x, stream=st, y=y, losses=losses))
+        g.replay()
+        return y
+
+    def train_graph_(self, x: torch.Tensor, dy: torch.Tensor, y: Optional[torch.Tensor] = None,
+                     losses: Optional[torch.Tensor] = None,
+                     dx: Optional[torch.Tensor] = None) -> dict:
         """forward_ then backward_ replayed from one CUDA graph on the current
-        stream, captured on the first call for these x and dy buffers (same
-        tensors on later calls; their contents may change)."""
+        stream, captured on the first call for each set of buffers (x, dy, y,
+        losses, dx)."""
         _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
         _need(dy, "dy", torch.float32, (self.cfg.T, self.cfg.d), self.device)
-        key = (x.data_ptr(), dy.data_ptr())
-        if getattr(self, "_tgraph_key", None) != key:
-            self._tgraph = None
-            self.grads()
-            cap = torch.cuda.Stream(device=self.device)
-            cap.wait_stream(torch.cuda.current_stream(self.device))
-            with torch.cuda.stream(cap):
-                self.forward_(x, stream=cap)  # one-time set-up outside the capture
-                self.backward_(x, dy, stream=cap)
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
-                self.forward_(x, stream=cap)
-                self.backward_(x, dy, stream=cap)
-            torch.cuda.current_stream(self.device).wait_stream(cap)
-            self._tgraph, self._tgraph_key = g, key
-        self._tgraph.replay()
-        return self._grads
+        grads = self.grads()
+        y = self.y if y is None else y
+        losses = self.losses if losses is None else losses
+        dx = grads["dx"] if dx is None else dx
+
+        def record(st):
+            self.forward_(x, stream=st, y=y, losses=losses)
+            self.backward_(x, dy, stream=st, dx=dx)
+        g = self._graph(("train", x.data_ptr(), dy.data_ptr(), y.data_ptr(), losses.data_ptr(),
+                         dx.data_ptr()), record)
+        g.replay()
+        return grads
 
     def release_graph(self):
         """Drop the captured graphs."""
-        self._graph = None
-        self._graph_x = None
-        self._tgraph = None
-        self._tgraph_key = None
+        self.__dict__["_graphs"] = {}
 
     def grads(self, intermediates: bool = False) -> dict:
         """Gradient buffers of this layer (allocated on first use), fp32 in
@@ -403,11 +409,13 @@ class MoELayer:
                                         _ptr(self.status), st), "moe_backward")
         return g
 
-    def train_host_batches(self, x_hosts, dy_hosts, y_hosts, losses_hosts, dx_hosts):
+    def train_host_batches(self, x_hosts, dy_hosts, y_hosts, losses_hosts, dx_hosts,
+                           graph: bool = False):
         """Training steps (forward + backward) over batches in pinned host
         memory, pipelined like forward_host_batches: x and dy of batch i+1 go
         to the device and y, the losses and dx of batch i-1 come back on their
-        own streams while batch i runs on the current stream.  The parameter
+        own streams while batch i runs on the current stream (with graph each
+        buffer set's step is replayed from a CUDA graph).  The parameter
         gradients stay on the device (those of the last batch).  Returns the
         device-to-host stream after queuing; the caller synchronises."""
         if not hasattr(self, "_tpipe"):
@@ -433,8 +441,12 @@ class MoELayer:
             comp.wait_event(ready)
             if out_free[b] is not None:
                 comp.wait_event(out_free[b])
-            self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
-            self.backward_(P["x"][b], P["dy"][b], stream=comp, dx=P["dx"][b])
+            if graph:
+                self.train_graph_(P["x"][b], P["dy"][b], y=P["y"][b], losses=P["losses"][b],
+                                  dx=P["dx"][b])
+            else:
+                self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
+                self.backward_(P["x"][b], P["dy"][b], stream=comp, dx=P["dx"][b])
             done = torch.cuda.Event()
             done.record(comp)
             in_free[b] = done
@@ -461,11 +473,12 @@ class MoELayer:
         y_host.copy_(self.y, non_blocking=True)
         losses_host.copy_(self.losses, non_blocking=True)
 
-    def forward_host_batches(self, x_hosts, y_hosts, losses_hosts):
+    def forward_host_batches(self, x_hosts, y_hosts, losses_hosts, graph: bool = False):
         """End-to-end calls over a sequence of batches in pinned host memory,
         pipelined: the copy of batch i+1 to the device and the copy of batch
         i-1's y and losses to the host run on their own streams while batch i
-        runs on the current stream (double-buffered device copies).  Returns
+        runs on the current stream (double-buffered device copies; with graph
+        each buffer set's forward is replayed from a CUDA graph).  Returns
         after queuing; the caller synchronises."""
         if not hasattr(self, "_pipe"):
             dev = self.device
@@ -489,7 +502,10 @@ class MoELayer:
             comp.wait_event(x_ready)
             if y_free[b] is not None:
                 comp.wait_event(y_free[b])
-            self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
+            if graph:
+                self.forward_graph_(P["x"][b], y=P["y"][b], losses=P["losses"][b])
+            else:
+                self.forward_(P["x"][b], stream=comp, y=P["y"][b], losses=P["losses"][b])
             done = torch.cuda.Event()
             done.record(comp)
             x_free[b] = done

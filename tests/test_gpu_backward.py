@@ -175,9 +175,11 @@ def test_backward_requires_flag():
     assert rc == _lib.MOE_EINVAL
 
 
-def test_train_host_batches_matches_device_path():
-    """The pipelined host-memory training path gives the same y, losses and dx,
-    bit for bit, as forward_ + backward_ on device tensors, batch by batch."""
+@pytest.mark.parametrize("graph", [False, True])
+def test_train_host_batches_matches_device_path(graph):
+    """The pipelined host-memory training path (direct calls, or one CUDA
+    graph per buffer set) gives the same y, losses and dx, bit for bit, as
+    forward_ + backward_ on device tensors, batch by batch."""
     w = CASES["noise-free"]
     inp = to_dev(synth.make_inputs(w))
     cfg = dataclasses.replace(M.Config.from_workload(w), backward=1)
@@ -195,7 +197,8 @@ def test_train_host_batches_matches_device_path():
     yh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
     lh = [torch.empty(layer.losses.numel()).pin_memory() for _ in xs]
     dxh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
-    d2h = layer.train_host_batches([pin(x) for x in xs], [pin(d) for d in dys], yh, lh, dxh)
+    d2h = layer.train_host_batches([pin(x) for x in xs], [pin(d) for d in dys], yh, lh, dxh,
+                                   graph=graph)
     d2h.synchronize()
     torch.cuda.synchronize()
     for i, (y, l, dx) in enumerate(want):

@@ -446,3 +446,26 @@ def test_forward_graph_replay_matches_direct():
             outs.append(want["y"])
         assert not torch.equal(outs[0], outs[1])
         layer.release_graph()
+
+
+def test_forward_host_batches_with_graphs_matches_direct():
+    """The pipelined host path with a CUDA graph per buffer set gives each
+    batch's y and losses bit for bit as direct device calls."""
+    w = SMALL["lm-flat-512"]
+    dinp = to_dev(synth.make_inputs(w))
+    layer = M.MoELayer(M.Config.from_workload(w), dinp, torch.device(DEV))
+    xs = [synth.make_inputs(w.with_(seed=s), experts=False)["x"] for s in (11, 12, 13)]
+    want = []
+    for x in xs:
+        layer.forward_(x.to(DEV))
+        torch.cuda.synchronize()
+        want.append((layer.y.cpu().clone(), layer.losses.cpu().clone()))
+    yh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
+    lh = [torch.empty(layer.losses.numel()).pin_memory() for _ in xs]
+    d2h = layer.forward_host_batches([x.contiguous().pin_memory() for x in xs], yh, lh, graph=True)
+    d2h.synchronize()
+    torch.cuda.synchronize()
+    for i, (y, l) in enumerate(want):
+        assert torch.equal(yh[i], y), i
+        assert torch.equal(lh[i], l), i
+    layer.release_graph()
