@@ -935,6 +935,25 @@ int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_
         dH[jt] -= a;
       }
     }
+    /* router z-loss w_z mean_t |c_t|^2 and gate entropy -w_entropy mean_t
+     * H(softmax(c_t)) ([MoE-intro] 第三部分): d|c|^2/dc_i = 2 c_i;
+     * dH/dc_i = -p_i (log p_i + H) for p = softmax(c) */
+    if (T > 0 && (cfg->w_z != 0.0 || cfg->w_entropy != 0.0)) {
+      double m = c[0];
+      for (int i = 1; i < n; ++i) if (c[i] > m) m = c[i];
+      double Ssum = 0.0;
+      for (int i = 0; i < n; ++i) Ssum += exp(c[i] - m);
+      const double logS = log(Ssum);
+      double ent = 0.0;
+      for (int i = 0; i < n; ++i) {
+        const double lp = c[i] - m - logS;
+        ent -= exp(lp) * lp;
+      }
+      for (int i = 0; i < n; ++i) {
+        const double lp = c[i] - m - logS;
+        dc[i] += (cfg->w_z * 2.0 * c[i] + cfg->w_entropy * exp(lp) * (lp + ent)) / (double)T;
+      }
+    }
     /* H = c + eps * s (noise), H = c otherwise (router 2's bias has no gradient) */
     for (int i = 0; i < n; ++i) {
       dc[i] += dH[i];

@@ -65,6 +65,8 @@ typedef struct {
   double w_importance, w_load, alpha;
   int shared_expert;        /* 1: y also gets one always-active expert, weight 1 */
   int router_stats;         /* 1: losses[8], [9] get the router z-loss and entropy */
+  double w_z, w_entropy;    /* weights of the z-loss and of the entropy in the
+                               backward's loss (orc_backward) */
 } orc_cfg;
 
 /* ---- noise ------------------------------------------------------------ */
@@ -179,6 +181,7 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
 /* ---- backward pass ------------------------------------------------------ */
 /* Gradients of
  *   L = sum_t <dy_t, y_t> + losses[0] + losses[1] + losses[3]
+ *       + w_z * losses[8] - w_entropy * losses[9]
  * (an upstream gradient dy[T][d] of the layer output plus the weighted
  * balancing losses of orc_forward) with respect to x and every parameter;
  * flat layers only (hier_a == 0).  With expert_bf16 the rounding points of a

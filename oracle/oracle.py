@@ -38,6 +38,7 @@ class OrcCfg(C.Structure):
         ("capacity_factor", C.c_double), ("passthrough", C.c_int), ("expert_bf16", C.c_int),
         ("w_importance", C.c_double), ("w_load", C.c_double), ("alpha", C.c_double),
         ("shared_expert", C.c_int), ("router_stats", C.c_int),
+        ("w_z", C.c_double), ("w_entropy", C.c_double),
     ]
 
 
@@ -224,13 +225,13 @@ def expert_row(x, W1, b1, W2, b2, bf16: bool) -> np.ndarray:
 # ---------------------------------------------------------------- forward
 _CFG_KEYS = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router", "noise",
              "seed", "capacity_factor", "passthrough", "expert_bf16", "w_importance", "w_load", "alpha",
-             "shared_expert", "router_stats")
+             "shared_expert", "router_stats", "w_z", "w_entropy")
 
 
 def make_cfg(**kw) -> OrcCfg:
     base = dict(hier_a=0, hier_b=0, hier_k1=0, hier_k2=0, router=0, noise=1, seed=0,
                 capacity_factor=0.0, passthrough=0, expert_bf16=0, w_importance=0.1,
-                w_load=0.1, alpha=0.01, shared_expert=0, router_stats=0)
+                w_load=0.1, alpha=0.01, shared_expert=0, router_stats=0, w_z=0.0, w_entropy=0.0)
     base.update({k: v for k, v in kw.items() if k in _CFG_KEYS})
     return OrcCfg(**{k: base[k] for k in _CFG_KEYS})
 
@@ -339,7 +340,8 @@ def cv2_grad(v) -> np.ndarray:
 
 
 def backward(cfg: dict, inp: dict, dy) -> dict:
-    """Gradients of L = sum(dy * y) + losses[0] + losses[1] + losses[3] of
+    """Gradients of L = sum(dy * y) + losses[0] + losses[1] + losses[3]
+    + w_z losses[8] - w_entropy losses[9] of
     ``forward(cfg, inp)`` with respect to x and every parameter (flat layers);
     also dL/d topk_gate ("dgate"), dL/d clean logits ("dlogits") and dL/d
     (x W_noise) ("dnoise")."""

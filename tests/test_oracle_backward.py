@@ -261,3 +261,47 @@ def test_expert_backward_is_the_layer_backward_of_one_expert():
                 assert np.allclose(r[key], g[key][e], rtol=1e-12, atol=1e-12), (bf16, e, key)
             for (t, j), dg in zip(rows, r["dgate"]):
                 assert dg == pytest.approx(g["dgate"][t, j], rel=1e-12, abs=1e-12)
+
+
+@pytest.mark.parametrize("router", [0, 1, 2])
+def test_zloss_and_entropy_terms(router):
+    """With weights on the router z-loss and the gate entropy the backward's
+    loss is L + w_z losses[8] - w_entropy losses[9]: central differences of the
+    forward (router_stats on) pin their gradients, alone (dy = 0, no other
+    loss) and together with everything else."""
+    rng = np.random.default_rng(30 + router)
+    T, d, n, f = 10, 5, 5, 8
+    k = 1 if router == 1 else 2
+    inp = _inputs(rng, T, d, n, f, noise=(router == 0), router=router)
+    base = dict(T=T, d=d, n=n, k=k, f=f, router=router, noise=int(router == 0), seed=2,
+                router_stats=1, w_z=0.7, w_entropy=1.3)
+
+    def loss(cfg, inp, dy):
+        out = O.forward(cfg, inp)
+        return float(np.sum(dy * out["y"]) + out["losses"][0] + out["losses"][1] +
+                     out["losses"][3] + cfg["w_z"] * out["losses"][8] -
+                     cfg["w_entropy"] * out["losses"][9]), out
+
+    for cfg, dy in ((dict(base, w_importance=0.0, w_load=0.0, alpha=0.0),
+                     np.zeros((T, d), np.float32)),
+                    (dict(base, w_importance=0.3, w_load=0.4, alpha=0.5),
+                     rng.normal(0, 1, (T, d)).astype(np.float32))):
+        g = O.backward(cfg, inp, dy)
+        _, ref_out = loss(cfg, inp, dy)
+        for name in ("Wg", "bg", "x"):
+            arr = inp[name]
+            an = g[GRAD_OF[name]]
+            scale = float(np.abs(an).max()) + 1e-12
+            for i in rng.choice(arr.size, size=min(8, arr.size), replace=False):
+                pos = np.unravel_index(int(i), arr.shape)
+                v0 = arr[pos]
+                h = np.float32(2e-3 * max(1.0, abs(float(v0))))
+                arr[pos] = np.float32(v0 + h); lp, op = loss(cfg, inp, dy)
+                arr[pos] = np.float32(v0 - h); lm, om = loss(cfg, inp, dy)
+                arr[pos] = v0
+                if not (np.array_equal(op["topk_idx"], ref_out["topk_idx"]) and
+                        np.array_equal(om["topk_idx"], ref_out["topk_idx"])):
+                    continue
+                fd = (lp - lm) / (float(np.float32(v0 + h)) - float(np.float32(v0 - h)))
+                assert abs(fd - an[pos]) <= 2e-3 * (abs(an[pos]) + 0.05 * scale) + 1e-9, \
+                    (router, name, pos, fd, an[pos])
