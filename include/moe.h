@@ -135,6 +135,8 @@ typedef struct moe_config {
   int32_t router_stats;       /* 1: moe_forward reports losses[8], [9] */
   int32_t backward;           /* 1: the workspace also serves moe_backward and
                                  moe_forward keeps what it needs (0 or 1) */
+  float w_z, w_entropy;       /* weights of the router z-loss and of the gate
+                                 entropy in moe_backward's loss (0: none) */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
@@ -332,8 +334,12 @@ typedef struct moe_grads {
  * noise lets the load loss reach the gate through Phi ([SGMoE-note] "Noisy
  * Top-K Gating").  Computes the gradients of
  *   L = sum(dy * y) + losses[0] + losses[1] + losses[3]
+ *       + w_z * losses[8] - w_entropy * losses[9]
  * (dy [T][d] fp32, the upstream gradient of moe_forward's y, plus the
- * weighted balancing losses) with respect to x (dx [T][d], fp32, written) and
+ * weighted balancing losses; the router z-loss mean_t |h_t|^2 and the gate
+ * entropy mean_t H(softmax(h_t)) of [MoE-intro] "第三部分" enter with the
+ * weights w_z and -w_entropy, so a positive w_entropy rewards entropy) with
+ * respect to x (dx [T][d], fp32, written) and
  * every parameter (grads).  With bf16 experts (mixed precision) the gradients
  * reaching the expert rows (g * dy), the hidden layer and the expert inputs
  * are kept in bf16 as the forward keeps its activations, accumulation is

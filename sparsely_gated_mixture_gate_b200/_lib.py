@@ -28,7 +28,7 @@ class moe_config(C.Structure):
         ("seed", C.c_uint64), ("capacity_factor", C.c_double), ("overflow_passthrough", C.c_int32),
         ("w_importance", C.c_float), ("w_load", C.c_float), ("alpha_aux", C.c_float),
         ("gate_precision", C.c_int32), ("shared_expert", C.c_int32), ("router_stats", C.c_int32),
-        ("backward", C.c_int32),
+        ("backward", C.c_int32), ("w_z", C.c_float), ("w_entropy", C.c_float),
     ]
 
 

@@ -24,6 +24,7 @@
 //                   importance and load losses (Phi' and kth_excluding), the
 //                   noise (eps recomputed from Philox) and Softplus; for the
 //                   noisy gate up to 1024 experts the row sits in registers
+//   gate_stats_bwd  the router z-loss and gate entropy terms added to dL/dc
 //   colsum          column sums of a row-major matrix in row blocks (db_g)
 #include "internal.h"
 #include "philox.cuh"
@@ -663,6 +664,52 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
   }
 }
 
+// ---------------------------------------------------------------- gate_stats_bwd
+// The router z-loss w_z mean_t |c_t|^2 and the gate entropy term
+// -w_entropy mean_t H(softmax(c_t)) ([MoE-intro] 第三部分): per token (warp),
+// an online pass for m = max c, S = sum e^(c-m), Q = sum e^(c-m) (c-m)
+// (H = log S - Q/S), then dc_i += (w_z 2 c_i + w_entropy p_i (log p_i + H)) / T,
+// since dH/dc_i = -p_i (log p_i + H).
+__global__ void __launch_bounds__(GW * 32) gate_stats_bwd_kernel(const float *__restrict__ c,
+                                                                  int T, int n, float w_z,
+                                                                  float w_e, float *dc) {
+  const int t = blockIdx.x * GW + (threadIdx.x >> 5);
+  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  const float *crow = c + (size_t)t * n;
+  float m = -INFINITY, S = 0.f, Q = 0.f;
+  for (int i = lane; i < n; i += 32) {
+    const float v = crow[i];
+    if (v > m) {  // rescale to the new maximum
+      const float r = S > 0.f ? expf(m - v) : 0.f;
+      Q = S > 0.f ? r * (Q + S * (m - v)) : 0.f;
+      S *= r;
+      m = v;
+    }
+    const float e = expf(v - m);
+    S += e;
+    Q = fmaf(e, v - m, Q);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) {
+    const float om = __shfl_xor_sync(0xffffffffu, m, off);
+    const float os = __shfl_xor_sync(0xffffffffu, S, off);
+    const float oq = __shfl_xor_sync(0xffffffffu, Q, off);
+    const float m2 = fmaxf(m, om);
+    const float r1 = S > 0.f ? expf(m - m2) : 0.f, r2 = os > 0.f ? expf(om - m2) : 0.f;
+    Q = (S > 0.f ? r1 * (Q + S * (m - m2)) : 0.f) + (os > 0.f ? r2 * (oq + os * (om - m2)) : 0.f);
+    S = S * r1 + os * r2;
+    m = m2;
+  }
+  const float logS = logf(S), H = logS - Q / S, invT = 1.f / (float)T;
+  float *drow = dc + (size_t)t * n;
+  for (int i = lane; i < n; i += 32) {
+    const float v = crow[i];
+    const float lp = v - m - logS;
+    drow[i] += (w_z * 2.f * v + w_e * expf(lp) * (lp + H)) * invT;
+  }
+}
+
 // ---------------------------------------------------------------- colsum
 // part[blockIdx.y][j] = sum of rows [blockIdx.y * rows_per, ...) of column j
 __global__ void __launch_bounds__(256) colsum_kernel(const float *__restrict__ X, int R, int N,
@@ -774,6 +821,12 @@ int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st) {
 }
 
 // row blocks of at least 16 rows, about two blocks per SM over all column blocks
+int launch_gate_stats_bwd(const float *c, int T, int n, float w_z, float w_entropy, float *dc,
+                          cudaStream_t st) {
+  return launch("gate_stats_bwd", gate_stats_bwd_kernel, dim3((unsigned)ceil_div(T, GW)),
+                dim3(GW * 32), 0, st, c, T, n, w_z, w_entropy, dc);
+}
+
 int colsum_parts(int R, int N) {
   if (R <= 0) return 0;
   const int cb = (int)ceil_div(N, 256);

@@ -211,6 +211,9 @@ int launch_expert_bwd_f32(const float *x_perm, const float *dy_perm, const int *
 int launch_bias_grad(const void *dy_perm, const void *dhid, const int *offsets, int n, int d,
                      int f, float *db2, float *db1, const char *name, cudaStream_t st);
 int launch_gate_bwd(const GateBwdArgs &a, cudaStream_t st);
+// dc[t][i] += (w_z 2 c_i + w_entropy p_i (log p_i + H_t)) / T, p = softmax(c_t)
+int launch_gate_stats_bwd(const float *c, int T, int n, float w_z, float w_entropy, float *dc,
+                          cudaStream_t st);
 int colsum_parts(int R, int N);
 int launch_colsum(const float *X, int R, int N, float *part, float *out, cudaStream_t st);
 // weight gradients of the experts on the tensor cores, per expert e with rows

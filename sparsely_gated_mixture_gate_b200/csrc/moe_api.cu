@@ -622,6 +622,7 @@ int moe_validate(const moe_config *c) {
   if (c->shared_expert != 0 && c->shared_expert != 1) return MOE_EINVAL;
   if (c->router_stats != 0 && c->router_stats != 1) return MOE_EINVAL;
   if (c->backward != 0 && c->backward != 1) return MOE_EINVAL;
+  if (!(c->w_z == c->w_z) || !(c->w_entropy == c->w_entropy)) return MOE_EINVAL;  // NaN
   if (c->noise != 0 && c->noise != 1) return MOE_EINVAL;
   if (c->expert_dtype != MOE_F32 && c->expert_dtype != MOE_BF16) return MOE_EINVAL;
   if (c->overflow_passthrough != 0 && c->overflow_passthrough != 1) return MOE_EINVAL;
@@ -985,6 +986,8 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   g.dz = dz;
   MOE_TRY(stream_after(st, side->s, side->join));  // the loss coefficients
   MOE_TRY(launch_gate_bwd(g, st));
+  if (c.w_z != 0.f || c.w_entropy != 0.f)  // router z-loss and gate entropy terms
+    MOE_TRY(launch_gate_stats_bwd(at<float>(ws, L.c), T, n, c.w_z, c.w_entropy, dc, st));
   if (gr->db_g) MOE_TRY(launch_colsum(dc, T, n, at<float>(ws, L.colsum_part), gr->db_g, st));
   float *sp = at<float>(ws, L.sgemm_part);
   const bool want_n = c.noise && gr->dW_noise;

@@ -51,6 +51,8 @@ class Config:
     shared_expert: int = 0    # 1: one always-active expert (W1s, b1s, W2s, b2s) in forward
     router_stats: int = 0     # 1: forward reports the router z-loss and entropy (losses[8:10])
     backward: int = 0         # 1: the layer also runs the backward pass (workspace, saved state)
+    w_z: float = 0.0          # backward: weight of the router z-loss (losses[8])
+    w_entropy: float = 0.0    # backward: weight rewarding the gate entropy (-losses[9])
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -68,7 +70,8 @@ class Config:
                           overflow_passthrough=self.passthrough, w_importance=self.w_importance,
                           w_load=self.w_load, alpha_aux=self.alpha,
                           gate_precision=self.gate_precision, shared_expert=self.shared_expert,
-                          router_stats=self.router_stats, backward=self.backward)
+                          router_stats=self.router_stats, backward=self.backward,
+                          w_z=self.w_z, w_entropy=self.w_entropy)
 
     @property
     def expert_dtype(self):

@@ -54,6 +54,8 @@ class Workload:
     shared_expert: int = 0      # 1: one always-active expert added to every token
     sel_bias_std: float = 0.0   # sigmoid router: spread of the selection bias
     router_stats: int = 0       # 1: the router z-loss and entropy are reported too
+    w_z: float = 0.0            # backward: weights of the z-loss and of the entropy
+    w_entropy: float = 0.0
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -66,7 +68,8 @@ class Workload:
     def cfg(self) -> dict:
         keys = ("T", "d", "n", "k", "f", "hier_a", "hier_b", "hier_k1", "hier_k2", "router",
                 "noise", "expert_bf16", "capacity_factor", "passthrough", "seed",
-                "w_importance", "w_load", "alpha", "shared_expert", "router_stats")
+                "w_importance", "w_load", "alpha", "shared_expert", "router_stats", "w_z",
+                "w_entropy")
         return {k: getattr(self, k) for k in keys}
 
 

@@ -75,6 +75,12 @@ CASES = {
     # the largest slot count, and a gate wider than the register path (n > 1024)
     "k8-n64": W["lm-flat"].with_(T=200, n=64, k=8, d=64, f=64, **LOSSES),
     "wide-n2000": W["lm-flat"].with_(T=128, n=2000, k=2, d=64, f=32, **LOSSES),
+    # the router z-loss and gate entropy as weighted loss terms, on each router
+    "zloss-entropy-noisy": W["lm-flat"].with_(T=300, n=24, k=2, d=64, f=64, router_stats=1,
+                                              w_z=0.5, w_entropy=0.8, **LOSSES),
+    "zloss-entropy-switch": V["switch-skew"].with_(T=512, d=64, n=16, f=64, alpha=0.5,
+                                                   w_importance=0.3, w_z=0.5, w_entropy=0.8),
+    "zloss-entropy-sigmoid": V["deepseek-tiny"].with_(w_importance=0.3, w_z=0.5, w_entropy=0.8),
     # fp32 experts (everything fp32: 1e-4)
     "f32-tiny": W["tiny-flat"].with_(**LOSSES),
     "f32-capacity": W["tiny-flat"].with_(T=200, n=6, k=2, d=40, f=24, capacity_factor=0.7,
