@@ -1,6 +1,6 @@
 /*
  * moe_oracle.c -- plain single-threaded CPU oracle of the Sparsely-Gated MoE
- * layer forward pass.  TEST INFRASTRUCTURE ONLY (see moe_oracle.h): it is
+ * layer's forward and backward passes.  TEST INFRASTRUCTURE ONLY (see moe_oracle.h): it is
  * loaded by tests, the smoke check and the bench's CPU-baseline leg, never by
  * the product path.  Loops are written in the order of the formulas they
  * follow; no blocking, fusion or reordering beyond that.

@@ -1,6 +1,6 @@
 /*
- * moe_oracle.h -- plain single-threaded CPU oracle for the forward pass of the
- * Sparsely-Gated Mixture-of-Experts layer.
+ * moe_oracle.h -- plain single-threaded CPU oracle for the forward and backward
+ * passes of the Sparsely-Gated Mixture-of-Experts layer.
  *
  * TEST INFRASTRUCTURE ONLY.  This code exists to check the CUDA path; it is
  * never part of the product path.  Only tests/, the smoke check and the
@@ -8,8 +8,9 @@
  * helper with the CUDA library: every formula below is written out again from
  * the pages it cites.
  *
- * Arithmetic: fp64 accumulation everywhere.  Two results are deliberately
- * taken in fp32 because an integer decision hangs on them and the kernel takes
+ * Arithmetic: fp64 accumulation everywhere (the backward's bf16 mode rounds
+ * where the mixed-precision kernels store, see orc_backward).  Two results are
+ * deliberately taken in fp32 because an integer decision hangs on them and the kernel takes
  * that decision in fp32: the gate logits H used for KeepTopK / argmax.
  *
  * Sources (page title, section):
