@@ -10,8 +10,9 @@
  *
  * Arithmetic: fp64 accumulation everywhere (the backward's bf16 mode rounds
  * where the mixed-precision kernels store, see orc_backward).  Two results are
- * deliberately taken in fp32 because an integer decision hangs on them and the kernel takes
- * that decision in fp32: the gate logits H used for KeepTopK / argmax.
+ * deliberately taken in fp32 because an integer decision hangs on them and
+ * the kernel takes that decision in fp32: the gate logits H used for
+ * KeepTopK / argmax.
  *
  * Sources (page title, section):
  *  [SGMoE-note]  "Outrageously Large Neural Networks: The Sparsely-Gated
