@@ -1,28 +1,36 @@
 """Benchmark of the Sparsely-Gated MoE layer forward pass on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload lm-flat] [--impl ours|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload hierarchical]
+                    [--impl ours|reference] [--backward] [--no-per-config]
 
 One step = one full forward pass (gate, dispatch, experts, combine, balancing
 statistics) of one batch of the workload through the fused C-ABI call
 ``moe_forward``, its launches replayed from a CUDA graph captured from that
-call (``MoELayer.forward_graph_``; ``--no-graph`` times direct calls).  Inputs
-are resident in HBM; L2 is flushed (256 MiB write)
-before every timed step, and every step is timed on the device with CUDA
-events on the launching stream; the total is the max over ranks.  With N > 1
-(launched by torchrun) every rank runs its own independent batch on its own
-GPU (replicas, weak scaling; the layer has no cross-batch exchange).
+call (``MoELayer.forward_graph_``; ``--no-graph`` times direct calls).  The
+default workload is the hierarchical layer (65536 tokens, 64 groups x 128
+experts, 8.6 B expert parameters), the largest that fits one GPU.  Inputs
+are resident in HBM; L2 is flushed (256 MiB write) before every timed step,
+and every step is timed on the device with CUDA events on the launching
+stream; the total is the max over ranks.  The gate's noise is redrawn every
+step (the layer advances its noise key on the device).  With N > 1 (launched
+by torchrun) every rank runs its own independent batch on its own GPU
+(replicas, weak scaling; the layer has no cross-batch exchange).
 
 The JSON line also carries: e2e (same metric through the Python/C-ABI call
 with pinned host buffers, copies inside the timed region), the roofline of the
-dominant kernel (per-kernel CUDA-event times recorded by the library around
-its own launches), the expert-FFN TFLOP/s and routing GB/s of the metric,
-clocks sampled during the timed region, the count of library kernel launches,
-and the oracle's CPU baseline on a bounded sample.  ``--impl reference`` times
-the oracle itself (the reference arm of this comparison).
+dominant kernel and of every kernel (per-kernel CUDA-event times recorded by
+the library around its own launches, against the algorithmic work per step:
+expert weight bytes or FLOPs, gate FP32 FLOPs, routing bytes), the FP32 FMA
+peak measured in the same run, the expert-FFN TFLOP/s and routing GB/s of the
+metric, clocks sampled during the timed region, the count of library kernel
+launches, the oracle's CPU baseline on a bounded sample, and ``per_config``:
+a short run of each of the five workloads.  ``--impl reference`` times the
+oracle itself (the reference arm of this comparison).
 
 ``--backward``: one step is the forward pass followed by the backward pass
 (``moe_backward``: dx and every parameter's gradient for an upstream gradient
-dy plus the weighted balancing losses); the metric is then training tokens/s.
+dy plus the weighted balancing losses); the metric is then training tokens/s
+(default workload lm-flat: the backward pass covers flat layers).
 """
 from __future__ import annotations
 
@@ -165,36 +173,46 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 def kernel_work(w, name: str, S_kept: int):
-    """Algorithmic work of one launch: (bound, flops, bytes)."""
+    """Algorithmic work of all of one step's launches of a kernel, in the
+    units of the layer's measurement table: (bound, flops, bytes).
+
+    The expert FFN streams every expert's two weight matrices once: its
+    bytes are the weight bytes n*2*d*f*esz (the activations it reads and
+    writes are counted by the dispatch and the combine); its FLOPs are
+    4*S*d*f.  The fp32 gate GEMM is counted in FLOPs (primary and secondary
+    gates of the hierarchical layer together), the routing, dispatch and
+    combine kernels in the bytes they must move."""
     T, d, n, k, f = w.T, w.d, w.n, w.k, w.f
     S = T * k
-    ng = w.hier_a if w.hier_a else n
     esz = 2 if w.expert_bf16 else 4
+    npj = 2 if w.noise else 1          # projections: clean (+ noise)
+    if w.hier_a:
+        k1 = w.hier_k1
+        gate_flops = 2.0 * T * d * w.hier_a * npj + 2.0 * T * k1 * d * w.hier_b * npj
+        gate_cols = T * w.hier_a + T * k1 * w.hier_b        # (row, column) pairs of c and s
+        route_extra = 8 * T * k1 + 8 * T * k
+        place_extra = 28 * T * k1                              # the group pass moves indices only
+    else:
+        gate_flops = 2.0 * T * d * n * npj
+        gate_cols = T * n
+        route_extra = 8 * T * k
+        place_extra = 0
     if name == "expert_ffn_tcgen05":
-        # both layers in one persistent launch: every weight once, x_perm in,
-        # y_perm out (the hidden layer's round trip through memory is this
-        # implementation's choice, not counted as algorithmic traffic)
-        return "tensor", 4.0 * S_kept * d * f, n * 2 * d * f * esz + 2 * S_kept * d * esz
+        return "tensor", 4.0 * S_kept * d * f, n * 2 * d * f * esz
     if name == "shared_expert_ffn_tcgen05":
-        # one expert on all T tokens: its weights once, x rows in, rows out
-        return "tensor", 4.0 * T * d * f, 2 * d * f * esz + 2 * T * d * esz
+        return "tensor", 4.0 * T * d * f, 2 * d * f * esz
     if name == "gate_gemm_fp32":
-        return "alu", 2.0 * T * d * ng * (2 if w.noise else 1), 4 * (T * d + d * ng * 2 + 2 * T * ng)
+        return "alu", gate_flops, 4 * (T * d + 4 * gate_cols)
     if name == "gate_gemm_tf32x3":
         # the fp32-equivalent contraction; three tf32 MMAs carry it
-        return "tensor_tf32x3", 2.0 * T * d * ng * (2 if w.noise else 1), \
-            4 * (2 * T * d + 2 * d * ng * 2 + 2 * T * ng)
+        return "tensor_tf32x3", gate_flops, 4 * (2 * T * d + 4 * gate_cols)
     if name == "expert_ffn_fp32":
-        # both layers of every expert on its rows, fp32 weights streamed once
-        return "hbm", 4.0 * S_kept * d * f, n * 2 * d * f * 4 + S_kept * d * 4 * 2
+        return "hbm", 4.0 * S_kept * d * f, n * 2 * d * f * 4
     # ---- backward pass
     if name == "expert_bwd_tcgen05":
-        # dhid = (dy_perm W2) * mask, dx_perm = dhid W1: both weights once, dy_perm and the
-        # forward's hid in, dhid (needed again by the weight gradients) and dx_perm out
         return "tensor", 4.0 * S_kept * d * f, \
             n * 2 * d * f * esz + S_kept * (2 * d + 2 * f) * esz
     if name == "wgrad_tcgen05":
-        # dW2 = dy_perm^T hid, dW1 = dhid^T x_perm per expert: four activations in, fp32 out
         return "tensor", 4.0 * S_kept * d * f, S_kept * 2 * (d + f) * esz + n * 2 * d * f * 4
     if name == "combine_bwd":
         return "hbm", 0.0, T * d * 4 + 2 * S_kept * d * esz + 12 * T * k
@@ -203,24 +221,65 @@ def kernel_work(w, name: str, S_kept: int):
     if name == "bias_grad":
         return "hbm", 0.0, S_kept * (d + f) * esz + n * (d + f) * 4
     if name == "gate_bwd":
-        return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) * 2 + 16 * T * k + 16 * T
+        return "hbm", 0.0, 4 * T * n * npj * 2 + 16 * T * k + 16 * T
     if name in ("gate_wgrad_fp32", "gate_dgrad_fp32"):
-        # one launch carries the clean and the noise products (two with noise)
-        nprod = 2 if w.noise else 1
-        return "alu", nprod * 2.0 * T * d * ng, 4 * (T * d + nprod * (d * ng + T * ng))
+        return "alu", npj * 2.0 * T * d * n, 4 * (T * d + npj * (d * n + T * n))
     if name == "route_topk":
-        return "hbm", 0.0, 4 * T * ng * (2 if w.noise else 1) + 8 * T * k
+        return "hbm", 0.0, 4 * gate_cols * npj + route_extra
     if name == "combine":
         return "hbm", 0.0, S_kept * d * esz + T * d * 4 + 8 * T * k
     if name == "dispatch_place":
         # x read, kept rows written; per pair: id, gate, block rank and base
         # read, row and sorted gate written; per kept row its token
-        return "hbm", 0.0, T * d * 4 + S_kept * d * esz + 24 * S + 4 * S_kept
+        return "hbm", 0.0, T * d * 4 + S_kept * d * esz + 24 * S + 4 * S_kept + place_extra
     return None, 0.0, 0.0
 
 
+def fp32_fma_peak(dev, pk):
+    """The FP32 FMA throughput of this GPU, measured: scalar fma.rn.f32 and
+    packed fma.rn.f32x2 probe kernels (8 blocks of 256 threads per SM,
+    16 independent chains per thread), best of three runs each, CUDA events
+    on the launching stream.  Falls back to SMs x 128 lanes x 2 x max clock."""
+    import ctypes as C
+
+    import torch
+
+    from sparsely_gated_mixture_gate_b200 import _lib
+    derived = SMS * FP32_LANES * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+    try:
+        L = _lib.load()
+        sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        blocks, iters = sms * 8, 4096
+        out = torch.empty(blocks * 256, dtype=torch.float32, device=dev)
+        st = torch.cuda.current_stream()
+        res = {}
+        for packed in (0, 1):
+            best = 0.0
+            for rep in range(4):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(st)
+                rc = L.moe_fma_probe(C.c_void_p(out.data_ptr()), blocks, iters, packed,
+                                     C.c_void_p(st.cuda_stream))
+                e1.record(st)
+                torch.cuda.synchronize()
+                if rc != 0:
+                    raise RuntimeError(f"moe_fma_probe: {rc}")
+                if rep:  # the first run warms up
+                    best = max(best, blocks * 256.0 * iters * 256.0 / (e0.elapsed_time(e1) / 1e3) / 1e12)
+            res["f32x2" if packed else "f32"] = round(best, 2)
+        return {"tflops": max(res.values()), "source": "measured (FMA probe in this run)", **res,
+                "derived": round(derived, 1)}
+    except Exception as e:  # pragma: no cover - reported, not hidden
+        return {"tflops": derived, "source": f"derived (probe failed: {e})", "derived": round(derived, 1)}
+
+
 # ------------------------------------------------------------------ arms
-def run_ours(args, w, world, rank, local):
+def run_ours(args, w, world, rank, local, steps=None, warmup=None, alt_gate=None, fp32_peak=None,
+             cpu_sample=False):
+    """One workload through the fused forward (or the training step): the
+    device-timed value, the per-kernel trace, e2e, the roofline of the
+    dominant kernel; with cpu_sample also the oracle's CPU baseline on a
+    sample of the same inputs."""
     import torch
     import torch.distributed as dist
 
@@ -230,6 +289,9 @@ def run_ours(args, w, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     pk = peaks()
+    steps = args.steps if steps is None else steps
+    warmup = args.warmup if warmup is None else warmup
+    alt_gate = args.alt_gate if alt_gate is None else alt_gate
     # every rank: its own batch (x seeded by rank), the same weights
     inp = synth.make_inputs(w, device=dev)
     if rank:
@@ -266,7 +328,7 @@ def run_ours(args, w, world, rank, local):
     direct_step()
     per_step_launches = M.launch_count() - l0
 
-    for _ in range(args.warmup):
+    for _ in range(warmup):
         flush.fill_(1.0)
         step()
     torch.cuda.synchronize()
@@ -278,14 +340,14 @@ def run_ours(args, w, world, rank, local):
     # ---- timed region: K device-timed steps (no per-kernel events inside)
     clocks = ClockSampler(local)
     time.sleep(0.3)
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     launches0 = M.launch_count()
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
-    for i in range(args.steps):
+    for i in range(steps):
         flush.fill_(float(i))
         starts[i].record(stream)
         step()
@@ -294,16 +356,16 @@ def run_ours(args, w, world, rank, local):
     if world > 1:
         dist.barrier()
     wall = time.perf_counter() - wall0
-    launches = per_step_launches * args.steps if use_graph else M.launch_count() - launches0
+    launches = per_step_launches * steps if use_graph else M.launch_count() - launches0
     clk = clocks.stop()
     total_ms = sum(s.elapsed_time(e) for s, e in zip(starts, ends))
-    ms, value = aggregate(total_ms, w.T, args.steps, world)
+    ms, value = aggregate(total_ms, w.T, steps, world)
 
     # ---- second timed pass for the roofline: CUDA events recorded by the
     # library around each of its launches, on the launching stream (the
     # events add a little time per launch, so this pass is not the value;
     # direct calls, so it times every kernel without the graph's tighter gaps)
-    t_steps = max(3, min(args.steps, 300))
+    t_steps = max(3, min(steps, 300))
     M.trace_reset()
     M.trace_enable(True)
     torch.cuda.synchronize()
@@ -317,7 +379,7 @@ def run_ours(args, w, world, rank, local):
     # ---- e2e: host buffers, copies inside the timed region.  Every step
     # copies its batch from pinned host memory and its y and losses back;
     # consecutive steps overlap copies with compute on separate streams.
-    e_steps = max(3, min(args.steps, 200))
+    e_steps = max(3, min(steps, 200))
     xh = x.cpu().pin_memory()
     yh = [torch.empty(w.T, w.d, dtype=torch.float32).pin_memory() for _ in range(2)]
     lh = [torch.empty(layer.losses.numel(), dtype=torch.float32).pin_memory() for _ in range(2)]
@@ -366,7 +428,7 @@ def run_ours(args, w, world, rank, local):
 
     # ---- the other gate mode on the same weights (short run, reported apart)
     alt = None
-    if args.alt_gate and world == 1 and dy is None:
+    if alt_gate and world == 1 and dy is None:
         other = 0 if w.gate_precision else 1
         alt_layer = M.MoELayer(M.Config.from_workload(w.with_(gate_precision=other)), inp, dev)
         alt_step = alt_layer.forward_graph_ if use_graph else alt_layer.forward_
@@ -374,7 +436,7 @@ def run_ours(args, w, world, rank, local):
             flush.fill_(1.0)
             alt_step(x)
         torch.cuda.synchronize()
-        a_steps = max(3, min(args.steps, 300))
+        a_steps = max(3, min(steps, 300))
         as_ = [torch.cuda.Event(enable_timing=True) for _ in range(a_steps)]
         ae_ = [torch.cuda.Event(enable_timing=True) for _ in range(a_steps)]
         for i in range(a_steps):
@@ -390,91 +452,111 @@ def run_ours(args, w, world, rank, local):
         alt_layer.release_graph()
         del alt_layer
 
+    cpu = None
+    if cpu_sample and rank == 0 and world == 1:
+        cpu = cpu_baseline(w, inp=inp, backward=dy is not None)
+    layer.release_graph()
     if rank != 0:
         return None
 
-    # ---- roofline of the dominant kernel and the metric's two side figures
+    # ---- per kernel: the step's launches of each kernel against its
+    # algorithmic work per step (see kernel_work)
+    burst = pk["bf16_tflops"]
+    if fp32_peak is None:
+        fp32_peak = fp32_fma_peak(dev, pk)
     kstats = {}
     # launches on the library's side stream run beside the main chain; their
     # event spans include waits for SMs the main chain holds, so they take no
     # share of the step and cannot be the dominant kernel
     main_chain = {k: v for k, v in per_kernel.items() if not k.endswith("[side stream]")}
     main_ms = max(sum(r["ms"] for r in main_chain.values()), 1e-9)
-    for name, rec in per_kernel.items():
-        per_launch_ms = rec["ms"] / max(rec["launches"], 1)
+
+    def roof_of(name):
         bound, flops, nbytes = kernel_work(w, name, S_kept)
-        e = {"launches": rec["launches"], "ms_per_launch": round(per_launch_ms, 5)}
+        step_ms = per_kernel[name]["ms"] / t_steps
+        if bound == "tensor":
+            ai = flops / max(nbytes, 1)
+            ridge = burst * 1e12 / (pk["hbm_gbs"] * 1e9)
+            if ai < ridge:  # the weights stream from HBM: bandwidth bound
+                r = {"bound": "hbm", "achieved": nbytes / (step_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                     "unit": "GB/s", "work": "expert weight bytes streamed"}
+            else:
+                r = {"bound": "tensor", "achieved": flops / (step_ms / 1e3) / 1e12, "peak": burst,
+                     "unit": "TFLOP/s", "work": "expert FLOPs (bf16)"}
+        elif bound == "tensor_tf32x3":
+            # tf32 dense peak = bf16 peak / 2 (nominal ratio); three MMAs per product
+            r = {"bound": "tensor", "achieved": 3 * flops / (step_ms / 1e3) / 1e12, "peak": burst / 2.0,
+                 "unit": "TFLOP/s (tf32, 3 MMAs per fp32 product)", "work": "gate FLOPs"}
+        elif bound == "alu":
+            r = {"bound": "alu", "achieved": flops / (step_ms / 1e3) / 1e12,
+                 "peak": round(fp32_peak["tflops"], 2), "unit": "TFLOP/s", "work": "gate FLOPs (fp32)"}
+        elif bound == "hbm":
+            r = {"bound": "hbm", "achieved": nbytes / (step_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
+                 "unit": "GB/s", "work": "bytes moved"}
+        else:
+            return None
+        r["achieved"] = round(r["achieved"], 2)
+        r["frac"] = round(r["achieved"] / r["peak"], 4)
+        return r
+
+    for name, rec in per_kernel.items():
+        e = {"launches_per_step": round(rec["launches"] / t_steps, 2),
+             "ms_per_step": round(rec["ms"] / t_steps, 5)}
         if name in main_chain:
             e["share"] = round(rec["ms"] / main_ms, 4)
+            r = roof_of(name)
+            if r:
+                e["roofline"] = {k2: r[k2] for k2 in ("bound", "achieved", "unit", "frac")}
         else:
             e["overlapped"] = True
-        if bound:
-            e["gbs"] = round(nbytes / (per_launch_ms / 1e3) / 1e9, 1)
-            if flops:
-                e["tflops"] = round(flops / (per_launch_ms / 1e3) / 1e12, 2)
         kstats[name] = e
     dom = max(main_chain, key=lambda k: main_chain[k]["ms"])
-    bound, flops, nbytes = kernel_work(w, dom, S_kept)
-    dom_ms = per_kernel[dom]["ms"] / per_kernel[dom]["launches"]
-    sustained = pk.get("bf16_tflops_sustained", pk["bf16_tflops"])
-    if bound == "tensor":
-        ai = flops / nbytes
-        ridge = sustained * 1e12 / (pk["hbm_gbs"] * 1e9)
-        if ai < ridge:  # the weights stream from HBM: bandwidth bound
-            roof = {"bound": "hbm", "achieved": nbytes / (dom_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
-                    "unit": "GB/s"}
-        else:
-            roof = {"bound": "tensor", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": sustained,
-                    "unit": "TFLOP/s"}
-    elif bound == "tensor_tf32x3":
-        # tf32 dense peak = bf16 peak / 2 (nominal ratio); three MMAs per product
-        tf32_peak = sustained / 2.0
-        roof = {"bound": "tensor", "achieved": 3 * flops / (dom_ms / 1e3) / 1e12, "peak": tf32_peak,
-                "unit": "TFLOP/s (tf32, 3 MMAs per fp32 product)"}
-    elif bound == "alu":
-        fp32_peak = SMS * FP32_LANES * 2 * pk.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
-        roof = {"bound": "alu", "achieved": flops / (dom_ms / 1e3) / 1e12, "peak": round(fp32_peak, 1),
-                "unit": "TFLOP/s"}
-    else:
-        roof = {"bound": "hbm", "achieved": nbytes / (dom_ms / 1e3) / 1e9, "peak": pk["hbm_gbs"],
-                "unit": "GB/s"}
-    roof["achieved"] = round(roof["achieved"], 2)
-    roof["frac"] = round(roof["achieved"] / roof["peak"], 4)
+    roof = roof_of(dom) or {"bound": None, "achieved": None, "peak": None, "unit": None, "frac": None}
     roof["kernel"] = dom
-    roof["peak_source"] = pk["source"]
-    roof["traffic"] = ncu_traffic(dom, w.name)
+    roof["peak_source"] = fp32_peak["source"] if roof["bound"] == "alu" else \
+        (pk["source"] + (" (burst)" if roof["bound"] == "tensor" else ""))
+    trf = ncu_traffic(dom, w.name)
+    roof["traffic"] = trf
+    if trf is not None and roof["bound"] == "hbm":
+        # the capture's DRAM bytes per launch against the algorithmic bytes of one launch
+        lps = per_kernel[dom]["launches"] / t_steps
+        roof["traffic_over_algorithmic"] = round(trf * lps / kernel_work(w, dom, S_kept)[2], 3)
 
-    ffn_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in per_kernel
-                 if k.startswith("expert_ffn_tcgen05"))
+    ffn_ms = sum(per_kernel[k]["ms"] / t_steps for k in per_kernel if k.startswith("expert_ffn_tcgen05"))
     ffn_flops = 4.0 * S_kept * w.d * w.f
     route_names = [k for k in main_chain if k.startswith(("route", "dispatch", "combine"))]
-    route_ms = sum(per_kernel[k]["ms"] / per_kernel[k]["launches"] for k in route_names)
+    route_ms = sum(per_kernel[k]["ms"] / t_steps for k in route_names)
     route_bytes = sum(kernel_work(w, k, S_kept)[2] for k in route_names)
 
     line = {
         "metric": METRIC_TRAIN if dy is not None else METRIC, "value": round(value, 1),
         "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms / args.steps, 5),
+        "steps": steps, "warmup": warmup, "ms_per_step": round(ms / steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16/fp32",
         "data": "synthetic (seeded; random-init weights of the workload's shapes)",
         "config": {"workload": w.name + (" (forward + backward)" if dy is not None else ""),
                    "T": w.T, "d_model": w.d, "experts": w.n, "k": w.k,
                    "d_ff": w.f, "hier": [w.hier_a, w.hier_b] if w.hier_a else None,
-                   "router": "switch-top1" if w.router else "noisy-top-k",
+                   "router": {0: "noisy-top-k", 1: "switch-top1", 2: "sigmoid"}[w.router],
                    "gate": "3-pass TF32 on tensor cores (fp32-level)" if w.gate_precision
                    else "fp32 multiply-adds",
                    "capacity_factor": w.capacity_factor or None,
                    "l2": "flushed before every timed step (256 MiB write)",
+                   "noise": "redrawn every step (noise key advanced on the device)" if w.noise else None,
                    "launch": (("one CUDA graph replay per step (captured from moe_forward"
                                + (" and moe_backward)" if dy is not None else ")"))
                               if use_graph else "direct C-ABI calls"),
                    "parallelism": f"replicas x{world}"},
         "expert_ffn_tflops": round(ffn_flops / (ffn_ms / 1e3) / 1e12, 2) if ffn_ms else None,
-        "expert_ffn_frac_bf16_peak": round(ffn_flops / (ffn_ms / 1e3) / 1e12 / sustained, 4) if ffn_ms else None,
+        "expert_ffn_frac_bf16_peak": round(ffn_flops / (ffn_ms / 1e3) / 1e12 / burst, 4) if ffn_ms else None,
         "routing_hbm_gbs": round(route_bytes / (route_ms / 1e3) / 1e9, 1) if route_ms else None,
+        "routing_frac_hbm": round(route_bytes / (route_ms / 1e3) / 1e9 / pk["hbm_gbs"], 4)
+        if route_ms else None,
         "roofline": roof,
+        "fp32_fma_peak": fp32_peak,
         "kernels": kstats,
-        "kernel_timing": f"second pass of {t_steps} steps, CUDA events around every library launch",
+        "kernel_timing": f"second pass of {t_steps} steps, CUDA events around every library launch; "
+                         "work and time per step",
         "gpu_launches": int(launches),
         "gpu_launches_per_step": int(per_step_launches),
         "e2e": {"value": round(e_value, 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d_bytes,
@@ -491,24 +573,72 @@ def run_ours(args, w, world, rank, local):
         "wall_s": round(wall, 3),
         "device_status": st,
     }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
     return line
 
 
-def oracle_sample_inputs(w, T_s):
+def per_config_summary(line):
+    """The per-workload figures kept in the headline line's per_config."""
+    roof = line["roofline"]
+    out = {"value": line["value"], "unit": "tokens/s", "ms_per_step": line["ms_per_step"],
+           "e2e_value": line["e2e"]["value"], "steps": line["steps"],
+           "dominant": {k: roof.get(k) for k in ("kernel", "bound", "achieved", "peak", "unit", "frac")},
+           "expert_ffn_tflops": line["expert_ffn_tflops"],
+           "expert_ffn_frac_bf16_peak": line["expert_ffn_frac_bf16_peak"],
+           "routing_frac_hbm": line["routing_frac_hbm"], "clocks": line["clocks"],
+           "device_status": line["device_status"]}
+    ks = {}
+    for name in ("gate_gemm_fp32", "route_topk", "dispatch_place", "combine", "expert_ffn_tcgen05"):
+        if name in line["kernels"] and "roofline" in line["kernels"][name]:
+            r = line["kernels"][name]["roofline"]
+            ks[name] = {"ms_per_step": line["kernels"][name]["ms_per_step"],
+                        "share": line["kernels"][name].get("share"), "achieved": r["achieved"],
+                        "unit": r["unit"], "frac": r["frac"]}
+    out["kernels"] = ks
+    return out
+
+
+def oracle_sample_inputs(w, T_s, inp=None):
+    """The oracle's inputs for the first T_s tokens of the workload, as numpy
+    arrays (bf16 weights as uint16 bit patterns).  The expert weight arrays
+    keep their full [n][...] shapes but only the experts that the sample's
+    tokens reach (found by the oracle's own gate, untimed) are filled: the
+    arrays start as lazily zeroed pages, so the 8192-expert layer does not
+    need its 17 GB of weights in host memory.  inp: the workload's tensors
+    already made (on any device); else they are made here, on the GPU when
+    there is one (the same generator the GPU path uses)."""
+    import numpy as np
     import torch
 
+    from oracle import oracle as orc
     from sparsely_gated_mixture_gate_b200 import synth
-    inp = synth.make_inputs(w, T=T_s)
-    return {k: (None if v is None else (synth.bf16_bits(v) if v.dtype == torch.bfloat16 else v.numpy()))
-            for k, v in inp.items()}
+    if inp is None:
+        inp = synth.make_inputs(w, device="cuda" if torch.cuda.is_available() else "cpu")
+
+    def host(t):
+        if t is None:
+            return None
+        return synth.bf16_bits(t) if t.dtype == torch.bfloat16 else t.detach().cpu().numpy()
+
+    expert_keys = ("W1", "W2", "b1", "b2")
+    out = {key: host(v[:T_s] if key == "x" else v) for key, v in inp.items() if key not in expert_keys}
+    used = np.unique(orc.gate_batch(dict(w.cfg(), T=T_s), out)["topk_idx"])
+    for key in expert_keys:
+        v = inp[key]
+        arr = np.zeros(tuple(v.shape), np.uint16 if v.dtype == torch.bfloat16 else np.float32)
+        if used.size:
+            arr[used] = host(v.index_select(0, torch.from_numpy(used.astype(np.int64)).to(v.device)))
+        out[key] = arr
+    return out
 
 
-def oracle_step(w, T_s, backward=False):
+def oracle_step(w, T_s, backward=False, inp=None):
     """One oracle step on the first T_s tokens: the forward pass, and with
     backward the backward pass too (as a function of no arguments)."""
     from oracle import oracle as orc
     orc.build()
-    npin = oracle_sample_inputs(w, T_s)
+    npin = oracle_sample_inputs(w, T_s, inp)
     cfg = dict(w.cfg(), T=T_s)
     if not backward:
         return lambda: orc.forward(cfg, npin)
@@ -521,20 +651,20 @@ def oracle_step(w, T_s, backward=False):
     return both
 
 
-def time_oracle(w, T_s, reps=1, backward=False):
-    fn = oracle_step(w, T_s, backward)
+def time_oracle(w, T_s, reps=1, backward=False, inp=None):
+    fn = oracle_step(w, T_s, backward, inp)
     t0 = time.perf_counter()
     for _ in range(reps):
         fn()
     return time.perf_counter() - t0
 
 
-def cpu_baseline(w, budget_s=12.0, backward=False):
+def cpu_baseline(w, budget_s=12.0, backward=False, inp=None):
     """The oracle (single-threaded C, as it stands) on the first tokens of the
     workload: calibrate on 8 tokens, then run a sample of about budget_s."""
-    t8 = time_oracle(w, 8, backward=backward)
+    t8 = time_oracle(w, 8, backward=backward, inp=inp)
     T_s = int(max(8, min(w.T, budget_s / max(t8 / 8, 1e-6))))
-    t = time_oracle(w, T_s, backward=backward)
+    t = time_oracle(w, T_s, backward=backward, inp=inp)
     what = "forward + backward" if backward else "forward"
     return {"value": round(T_s / t, 2), "unit": "tokens/s", "cores": 1, "kind": "oracle",
             "sample": f"{what} of the first {T_s} tokens of {w.name} as one batch "
@@ -570,31 +700,92 @@ def run_reference(args, w):
                     "d2h_bytes_per_step": 0}}
 
 
+def run_stage(args, w):
+    """One stage of the layer through its own C-ABI call, timed alone on a
+    workload's shapes (optionally with fewer tokens, so that a profiler
+    capture stays small): gate (moe_gate), dispatch (moe_dispatch on the
+    gate's routing), experts (moe_expert_ffn on a dispatched batch), combine
+    (moe_combine).  Prints the mean device time per call; not a bench line."""
+    import torch
+
+    from sparsely_gated_mixture_gate_b200 import moe as M
+    from sparsely_gated_mixture_gate_b200 import synth
+    if args.tokens:
+        w = w.with_(T=args.tokens)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = synth.make_inputs(w, device=dev, experts=args.stage == "experts")
+    cfg = M.Config.from_workload(w)
+    ws = M.workspace(cfg, dev)
+    status = M.new_status(dev)
+    x = inp["x"]
+    if args.stage == "gate":
+        def step():
+            return M.gate(cfg, x, inp, ws=ws, status=status)
+    else:
+        g = M.gate(cfg, x, inp, ws=ws, status=status)
+        d = M.dispatch(cfg, x, g["topk_idx"], ws=ws, status=status)
+        if args.stage == "dispatch":
+            def step():
+                return M.dispatch(cfg, x, g["topk_idx"], ws=ws, status=status)
+        elif args.stage == "experts":
+            def step():
+                return M.expert_ffn(cfg, d["x_perm"], d["offsets"], inp, ws=ws, status=status)
+        else:
+            y_perm = d["x_perm"]  # any expert-row buffer of the right shape
+
+            def step():
+                return M.combine(cfg, y_perm, g["topk_gate"], d["row_of"], x, status=status)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st = torch.cuda.current_stream()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    return {"stage": args.stage, "workload": w.name, "T": w.T, "gate": args.gate,
+            "ms_per_call": e0.elapsed_time(e1) / args.steps, "calls": args.steps,
+            "device_status": M.status_bits(status)}
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=2000)
-    ap.add_argument("--warmup", type=int, default=20)
-    ap.add_argument("--workload", default="lm-flat")
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=None,
+                    help="default: hierarchical (the largest single-GPU workload); lm-flat with "
+                         "--backward (the backward pass covers flat layers)")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
                     help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", dest="per_config", action="store_false",
+                    help="skip the short runs of the other workloads (per_config)")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct library calls instead of a CUDA graph replay of the forward")
     ap.add_argument("--backward", action="store_true",
                     help="time forward + backward (training step) instead of the forward pass")
     ap.add_argument("--no-alt-gate", dest="alt_gate", action="store_false",
                     help="skip the short run of the other gate mode")
+    ap.add_argument("--stage", default=None, choices=["gate", "dispatch", "experts", "combine"],
+                    help="time one stage's C-ABI call alone (for profiler captures); no bench line")
+    ap.add_argument("--tokens", type=int, default=None, help="with --stage: tokens of the batch")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be at least 3")
 
     from sparsely_gated_mixture_gate_b200 import synth
-    w = (synth.WORKLOADS.get(args.workload) or synth.VARIANTS[args.workload]).with_(
+    name = args.workload or ("lm-flat" if args.backward else "hierarchical")
+    w = (synth.WORKLOADS.get(name) or synth.VARIANTS[name]).with_(
         gate_precision=1 if args.gate == "tf32x3" else 0)
     world, rank, local = dist_info()
 
+    if args.stage:
+        print(json.dumps(run_stage(args, w)), flush=True)
+        return
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args, w)), flush=True)
@@ -602,14 +793,26 @@ def main():
 
     import datetime
 
+    import torch
     import torch.distributed as dist
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     try:
-        line = run_ours(args, w, world, rank, local)
+        cpu = world == 1 and not args.no_cpu_baseline
+        line = run_ours(args, w, world, rank, local, cpu_sample=cpu)
+        if rank == 0 and line is not None and world == 1 and args.per_config and not args.backward:
+            # the five workloads, each a short run of its own (the headline's own figures reused)
+            per = {}
+            for other, wo in synth.WORKLOADS.items():
+                if other == w.name and not w.gate_precision:
+                    per[other] = per_config_summary(line)
+                    continue
+                torch.cuda.empty_cache()
+                o = run_ours(args, wo, world, rank, local, steps=min(args.steps, 20), warmup=3,
+                             alt_gate=False, fp32_peak=line["fp32_fma_peak"])
+                per[other] = per_config_summary(o)
+            line["per_config"] = per
         if rank == 0 and line is not None:
-            if world == 1 and not args.no_cpu_baseline:
-                line["cpu_baseline"] = cpu_baseline(w, backward=args.backward)
             print(json.dumps(line), flush=True)
     finally:
         if world > 1:

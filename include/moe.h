@@ -137,6 +137,12 @@ typedef struct moe_config {
                                  moe_forward keeps what it needs (0 or 1) */
   float w_z, w_entropy;       /* weights of the router z-loss and of the gate
                                  entropy in moe_backward's loss (0: none) */
+  int64_t token_base;         /* index of the first token in the noise counter:
+                                 0 for a whole batch; a data-parallel shard of a
+                                 batch passes its first token's index in the batch,
+                                 so that its tokens draw the noise they would draw
+                                 in the whole batch (0 <= token_base,
+                                 token_base + T <= 2^32) */
 } moe_config;
 
 /* Gate parameters.  Flat layer: W_g, W_noise [d][n], b_g [n] (per-expert
@@ -144,11 +150,19 @@ typedef struct moe_config {
  * primary gate over hier_a groups, plus the secondary gates W_g2, W_noise2
  * [hier_a][d][hier_b] and b_g2 [hier_a][hier_b] (may be NULL).  W_noise /
  * W_noise2 may be NULL when noise == 0.  sel_bias [n]: the selection bias of
- * MOE_ROUTER_SIGMOID (NULL: zero; ignored by the other routers). */
+ * MOE_ROUTER_SIGMOID (NULL: zero; ignored by the other routers).
+ * seed_dev: NULL, or one uint64 in device memory (8-byte aligned) that then
+ * replaces cfg->seed as the noise key: the routing kernel and moe_backward's
+ * gate backward read it when they run, so a captured CUDA graph draws the
+ * noise of whatever the word holds at each replay.  The pages' noisy gate
+ * draws a new StandardNormal() every time it runs ([SGMoE-xyz] "Noisy Top-K
+ * 門控"); a caller advances the word once per step with moe_noise_step and
+ * leaves it alone between a forward and its backward. */
 typedef struct moe_gate_params {
   const float *W_g, *b_g, *W_noise;
   const float *W_g2, *b_g2, *W_noise2;
   const float *sel_bias;
+  const uint64_t *seed_dev;
 } moe_gate_params;
 
 /* Expert parameters: W1 [n][f][d], W2 [n][d][f] of expert_dtype; b1 [n][f],
@@ -301,6 +315,13 @@ MOE_API int moe_balance_losses(const moe_config *cfg, const int32_t *topk_idx,
 MOE_API int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,
                                 float *sel_bias, moe_stream_t stream);
 
+/* Adds 1 to the device word *seed_dev (see moe_gate_params.seed_dev) in
+ * stream order, so that the next moe_forward / moe_gate on the stream draws
+ * fresh noise ([SGMoE-xyz] "Noisy Top-K 門控": a new StandardNormal() per
+ * evaluation).  One single-thread kernel; capturable in a CUDA graph.
+ * Errors: MOE_EINVAL for a NULL or misaligned pointer, MOE_ECUDA. */
+MOE_API int moe_noise_step(uint64_t *seed_dev, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- fused */
 
 /* The whole layer on one stream: gate, dispatch, experts (and the shared
@@ -358,6 +379,32 @@ MOE_API int moe_backward(const moe_config *cfg, const float *x, const moe_gate_p
                          const float *topk_gate, const float *importance, const float *load,
                          const int32_t *counts, float *dx, const moe_grads *grads, void *ws,
                          size_t ws_bytes, int32_t *status, moe_stream_t stream);
+
+/* ---------------------------------------------------------------- measurement */
+
+/* FP32 FMA throughput probe (a measurement helper; the pages have no
+ * counterpart).  Launches `blocks` blocks of 256 threads; every thread runs
+ * 16 independent fp32 FMA chains for iters x 8 steps, i.e. 256 FLOP per
+ * thread per iteration, blocks * 256 * iters * 256 FLOP in all, and writes
+ * one float per thread to out[blocks * 256] (device memory).  packed = 0
+ * issues scalar fma.rn.f32, packed = 1 the two-wide fma.rn.f32x2.  Timing it
+ * with CUDA events gives the FP32 FMA peak that bounds the fp32 gate GEMM.
+ * Errors: MOE_EINVAL (NULL out, blocks or iters < 1), MOE_ECUDA. */
+MOE_API int moe_fma_probe(float *out, int blocks, int iters, int packed, moe_stream_t stream);
+
+/* Test hook for the expert kernel's bounded cross-CTA wait (failure
+ * detection; the pages have no counterpart).  In the fused expert kernel a
+ * GEMM2 tile waits for the GEMM1 tiles of its 128-row M-block to publish
+ * their hidden rows; the wait gives up after a limit (default 2 s), sets
+ * MOE_STATUS_TIMEOUT in *status, and the kernel drains its copies and MMAs
+ * (bounded), frees its tensor memory and returns, leaving the context
+ * usable.  moe_test_expert_wait(limit_ns, withhold_mblock) sets, for the
+ * expert launches that follow in this process, that limit (0: back to the
+ * default) and one M-block whose GEMM1 tiles skip their publish
+ * (withhold_mblock = -1: none), so that the wait for it can only end by its
+ * limit; the outputs of such a call are void.  Process-wide, not for
+ * concurrent use; reset with (0, -1).  Always MOE_OK. */
+MOE_API int moe_test_expert_wait(unsigned long long limit_ns, int withhold_mblock);
 
 /* ---------------------------------------------------------------- tracing */
 

@@ -17,7 +17,8 @@ STATUS_NONFINITE, STATUS_BAD_INDEX, STATUS_TIMEOUT, STATUS_OVERFLOW = 1, 2, 4, 8
 EXPORTS = ("moe_strerror", "moe_validate", "moe_capacity", "moe_workspace_size", "moe_gate",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_balance_losses", "moe_forward",
            "moe_trace_enable", "moe_trace_reset", "moe_trace_count", "moe_trace_get",
-           "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update", "moe_backward")
+           "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update", "moe_backward",
+           "moe_noise_step", "moe_fma_probe", "moe_test_expert_wait")
 
 
 class moe_config(C.Structure):
@@ -29,13 +30,14 @@ class moe_config(C.Structure):
         ("w_importance", C.c_float), ("w_load", C.c_float), ("alpha_aux", C.c_float),
         ("gate_precision", C.c_int32), ("shared_expert", C.c_int32), ("router_stats", C.c_int32),
         ("backward", C.c_int32), ("w_z", C.c_float), ("w_entropy", C.c_float),
+        ("token_base", C.c_int64),
     ]
 
 
 class moe_gate_params(C.Structure):
     _fields_ = [("W_g", C.c_void_p), ("b_g", C.c_void_p), ("W_noise", C.c_void_p),
                 ("W_g2", C.c_void_p), ("b_g2", C.c_void_p), ("W_noise2", C.c_void_p),
-                ("sel_bias", C.c_void_p)]
+                ("sel_bias", C.c_void_p), ("seed_dev", C.c_void_p)]
 
 
 class moe_expert_params(C.Structure):
@@ -72,6 +74,9 @@ def load():
     L.moe_dispatch.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]
     L.moe_dispatch_noalloc.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_sel_bias_update.argtypes = [cfgp, vp, C.c_float, vp, vp]
+    L.moe_noise_step.argtypes = [vp, vp]
+    L.moe_fma_probe.argtypes = [vp, i32, i32, i32, vp]
+    L.moe_test_expert_wait.argtypes = [C.c_ulonglong, i32]
     L.moe_expert_ffn.argtypes = [cfgp, vp, vp, C.POINTER(moe_expert_params), vp, vp, sz, vp, vp]
     L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_balance_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]

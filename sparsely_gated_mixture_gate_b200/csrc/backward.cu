@@ -480,11 +480,13 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
       A_out += __shfl_xor_sync(0xffffffffu, A_out, off);
     }
   }
-  const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
+  const unsigned long long seed = a.seed_dev ? __ldg(a.seed_dev) : a.seed;
+  const uint32_t key0 = (uint32_t)(seed & 0xffffffffu), key1 = (uint32_t)(seed >> 32);
   for (int m = lane; 4 * m < n; m += 32) {
     float eps[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.noise) {
-      const uint4 wd = philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, 0u, 0u), key0, key1);
+      const uint4 wd =
+          philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, 0u, 0u), key0, key1);
       box_muller2(wd.x, wd.y, eps[0], eps[1]);
       box_muller2(wd.z, wd.w, eps[2], eps[3]);
     }
@@ -624,7 +626,8 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
       A_out += __shfl_xor_sync(0xffffffffu, A_out, off);
     }
   }
-  const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
+  const unsigned long long seed = a.seed_dev ? __ldg(a.seed_dev) : a.seed;
+  const uint32_t key0 = (uint32_t)(seed & 0xffffffffu), key1 = (uint32_t)(seed >> 32);
   float4 *dcrow = reinterpret_cast<float4 *>(a.dc + (size_t)t * n);
   float4 *dzrow = a.dz ? reinterpret_cast<float4 *>(a.dz + (size_t)t * n) : nullptr;
 #pragma unroll
@@ -633,7 +636,8 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
     if (4 * m >= n) break;
     float eps[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.noise) {
-      const uint4 wd = philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, 0u, 0u), key0, key1);
+      const uint4 wd =
+          philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, 0u, 0u), key0, key1);
       box_muller2(wd.x, wd.y, eps[0], eps[1]);
       box_muller2(wd.z, wd.w, eps[2], eps[3]);
     }

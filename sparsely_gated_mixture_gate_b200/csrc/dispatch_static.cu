@@ -31,7 +31,6 @@ namespace {
 constexpr int64_t kScratchInts = MOE_DISPATCH_NOALLOC_SCRATCH_INTS;
 static __device__ __align__(256) int g_dispatch_scratch[kScratchInts];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 int *g_scratch_ptr[kMaxDevices] = {};
 
@@ -72,15 +71,11 @@ extern "C" int moe_dispatch_noalloc(const moe_config *cfg, const float *x, const
   const int64_t need = 2 * B * (int64_t)c.n + c.n + 2;
   if (need > kScratchInts) return MOE_EWORKSPACE;  // beyond the fixed array
 
+  // the device first: on anything but an sm_100 part the library's module has
+  // no image, so the symbol lookup would fail with a CUDA error instead
+  MOE_TRY(check_device());
   int *scratch = nullptr;
-  const int rc = scratch_on_current_device(&scratch);
-  if (rc != MOE_OK) return rc;
-  int major = 0, minor = 0, dev = 0;
-  cudaGetDevice(&dev);
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-      major != 10 || minor != 0)
-    return MOE_EDEVICE;
+  MOE_TRY(scratch_on_current_device(&scratch));
 
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   DispatchArgs da{};

@@ -43,6 +43,8 @@
 // out sets MOE_STATUS_TIMEOUT, raises an abort flag seen by the other roles,
 // drains the copies and MMAs this CTA issued (again bounded), frees its
 // tensor memory and returns.
+#include <atomic>
+
 #include "tc_common.cuh"
 
 namespace moe {
@@ -87,6 +89,8 @@ struct FfnArgs {
   int *mdone;            // [M-blocks + 1] GEMM1 epilogue warps finished, per M-block; the
                          // last entry counts them over all of GEMM1
   int *status;
+  unsigned long long xwait_ns;  // limit of a GEMM2 tile's wait for its M-block of hid
+  int withhold_mblk;     // test hook: this M-block's GEMM1 tiles never publish (-1: none)
 };
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         // published them; then order the TMA reads after that observation
         if (ld_acquire(a.mdone + mtotal) >= NUM_EPI_WARPS * T1) {
           g1_all = true;
-        } else if (!wait_count(a.mdone + (ti.w >> 8), ready, abort_flag, kWaitNs)) {
+        } else if (!wait_count(a.mdone + (ti.w >> 8), ready, abort_flag, a.xwait_ns)) {
           failed = true;
           break;
         }
@@ -358,7 +362,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         asm volatile("fence.proxy.async.global;" ::: "memory");
         __threadfence();
         __syncwarp();
-        if (lane == 0) {
+        if (lane == 0 && (ti.w >> 8) != a.withhold_mblk) {
           atomicAdd(a.mdone + (ti.w >> 8), 1);
           atomicAdd(a.mdone + mtotal, 1);
         }
@@ -376,20 +380,27 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   }
 }
 
+// the wait limit of a GEMM2 tile for its M-block of hid and the test hook
+// (moe_test_expert_wait); the defaults: kWaitNs, nothing withheld
+std::atomic<unsigned long long> g_xwait_ns{kWaitNs};
+std::atomic<int> g_withhold{-1};
+unsigned long long expert_wait_limit_ns() { return g_xwait_ns.load(std::memory_order_relaxed); }
+int expert_withheld_mblock() { return g_withhold.load(std::memory_order_relaxed); }
+
 int ffn_ctas() {
-  static int cached_dev = -1, cached = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev != cached_dev) {
-    int per_sm = 0;
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ffn_kernel<false>, NUM_THREADS,
-                                                      SMEM_BYTES) != cudaSuccess ||
-        per_sm < 1)
-      return 0;
-    cached = per_sm * num_sms();
-    cached_dev = dev;
-  }
-  return cached;
+  static PerDevice ctas;
+  int v = 0;
+  if (ctas.get([](int, int *out) {
+        int per_sm = 0;
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, expert_ffn_kernel<false>,
+                                                          NUM_THREADS, SMEM_BYTES) != cudaSuccess ||
+            per_sm < 1)
+          return MOE_ECUDA;
+        *out = per_sm * num_sms();
+        return MOE_OK;
+      }, &v) != MOE_OK)
+    return 0;
+  return v;
 }
 
 }  // namespace
@@ -402,17 +413,16 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   if (!a.plan_ready)
     MOE_TRY(launch_expert_plan(a.offsets, a.n, const_cast<int *>(a.mprefix), a.tab1, nblk1, a.tab2,
                                nblk2, a.mdone, st));
-  static int attr_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_dev != dev) {
-    if (cudaFuncSetAttribute(expert_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess ||
-        cudaFuncSetAttribute(expert_ffn_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return MOE_ECUDA;
-    attr_dev = dev;
-  }
+  static PerDevice attrs;
+  MOE_TRY(attrs.get([](int, int *) {
+    return cudaFuncSetAttribute(expert_ffn_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES) == cudaSuccess &&
+                   cudaFuncSetAttribute(expert_ffn_kernel<true>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        SMEM_BYTES) == cudaSuccess
+               ? MOE_OK
+               : MOE_ECUDA;
+  }));
   const bool bwd = a.backward != 0;
   CUtensorMap a1, b1, a2, b2;
   FfnArgs f;
@@ -438,6 +448,8 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   f.n = a.n;
   f.mdone = a.mdone;
   f.status = a.status;
+  f.xwait_ns = expert_wait_limit_ns();
+  f.withhold_mblk = expert_withheld_mblock();
   const int64_t upper = (ceil_div(a.S, BM) + a.n) * (int64_t)(nblk1 + nblk2);
   const int ctas = ffn_ctas();
   if (ctas < 1) return MOE_ECUDA;
@@ -462,6 +474,11 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   trace_end(slot, st);
   count_launch();
   return e == cudaSuccess ? MOE_OK : MOE_ECUDA;
+}
+
+void set_expert_wait(unsigned long long limit_ns, int withhold_mblock) {
+  g_xwait_ns.store(limit_ns ? limit_ns : kWaitNs, std::memory_order_relaxed);
+  g_withhold.store(withhold_mblock >= 0 ? withhold_mblock : -1, std::memory_order_relaxed);
 }
 
 }  // namespace moe

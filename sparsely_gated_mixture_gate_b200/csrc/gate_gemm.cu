@@ -8,8 +8,10 @@
 // One kernel serves the flat gate, the primary gate and the grouped
 // secondary gates of the hierarchical layer: rows can be gathered from x
 // through row_token, and rows are split into groups (ragged M) that each use
-// their own weights.  The output columns [0,nb) of W_g and of W_noise are
-// separate N-tiles (blockIdx.y), so one launch computes both c and s.
+// their own weights.  The N dimension runs over the columns of W_g followed
+// by those of W_noise (2 nb columns with noise), tiled in 128-column pieces
+// (blockIdx.y), so one launch computes both c and s and a narrow gate (the
+// hierarchical layer's primary gate has nb = 64) fills whole tiles.
 //
 // Tile: 128 x 128 x 16, 256 threads, 8x8 outputs per thread held as two 4x4
 // quadrants (rows ty*4, 64+ty*4; cols tx*4, 64+tx*4) so the shared-memory
@@ -50,12 +52,12 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     row_end = a.R;
     if (row0 >= row_end) return;
   }
-  const int ntn = (a.nb + BN - 1) / BN;
-  const int which = blockIdx.y / ntn;          // 0: W_g -> c, 1: W_noise -> s
-  const int col0 = (blockIdx.y % ntn) * BN;
-  const float *B = (which ? a.Wn : a.Wg) + (size_t)g * a.d * a.nb;
   const int nb = a.nb;
-  const bool vecB = (nb & 3) == 0;
+  const int ncol = a.noise ? 2 * nb : nb;      // columns of [W_g | W_noise]
+  const int col0 = blockIdx.y * BN;            // first column of this tile
+  const float *Bg = a.Wg + (size_t)g * a.d * nb;
+  const float *Bn = a.noise ? a.Wn + (size_t)g * a.d * nb : nullptr;
+  const bool vecB = (nb & 3) == 0;             // a column quad never straddles the two
 
   const int tid = threadIdx.x;
   // A loader: rows ar and ar + 64 (ar = tid/4), k quad aq = (tid&3)*4
@@ -79,17 +81,20 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     if (k0 + aq >= a.d) return make_float4(0.f, 0.f, 0.f, 0.f);
     return __ldg(reinterpret_cast<const float4 *>(Arow[h] + k0 + aq));
   };
+  // element (kr, column vc) of [W_g | W_noise]
+  auto b_elem = [&](int kr, int vc) -> float {
+    if (vc >= ncol) return 0.f;
+    return vc < nb ? __ldg(Bg + (size_t)kr * nb + vc) : __ldg(Bn + (size_t)kr * nb + (vc - nb));
+  };
   auto load_b = [&](int k0, int h) -> float4 {
     const int kr = k0 + bk + 8 * h;
     if (kr >= a.d) return make_float4(0.f, 0.f, 0.f, 0.f);
-    const float *p = B + (size_t)kr * nb + bcol;
-    if (vecB && bcol + 3 < nb) return __ldg(reinterpret_cast<const float4 *>(p));
-    float4 v;
-    v.x = bcol + 0 < nb ? __ldg(p + 0) : 0.f;
-    v.y = bcol + 1 < nb ? __ldg(p + 1) : 0.f;
-    v.z = bcol + 2 < nb ? __ldg(p + 2) : 0.f;
-    v.w = bcol + 3 < nb ? __ldg(p + 3) : 0.f;
-    return v;
+    if (vecB && bcol + 3 < ncol) {
+      const float *p = bcol < nb ? Bg + (size_t)kr * nb + bcol : Bn + (size_t)kr * nb + (bcol - nb);
+      return __ldg(reinterpret_cast<const float4 *>(p));
+    }
+    return make_float4(b_elem(kr, bcol), b_elem(kr, bcol + 1), b_elem(kr, bcol + 2),
+                       b_elem(kr, bcol + 3));
   };
   auto store_tiles = [&](int buf, const float4 (&av)[2], const float4 (&bv)[2]) {
 #pragma unroll
@@ -142,15 +147,13 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     __syncthreads();
   }
 
-  // ---- epilogue
-  float *out = which ? a.s : a.c;
-  const float *bias = (which == 0 && a.bias) ? a.bias + (size_t)g * nb : nullptr;
+  // ---- epilogue: columns [0, nb) are c (+ bias), [nb, 2 nb) are s = Softplus
+  const float *bias = a.bias ? a.bias + (size_t)g * nb : nullptr;
   bool bad = false;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int row = row0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + (i - 4));
     if (row >= row_end) continue;
-    float *orow = out + (size_t)row * nb;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int col = col0 + h * 64 + tx * 4;
@@ -158,20 +161,26 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         float z = acc[i][h * 4 + j];
-        const int cc = col + j;
-        if (cc < nb) {
-          if (which) z = softplus_f(z);
-          else if (bias) z += bias[cc];
+        const int vc = col + j;
+        if (vc < nb) {
+          if (bias) z += bias[vc];
+          bad |= !isfinite(z);
+        } else if (vc < ncol) {
+          z = softplus_f(z);
+          bad |= !isfinite(z);
         }
-        bad |= !isfinite(z);
         v[j] = z;
       }
-      if (vecB && col + 3 < nb) {
-        *reinterpret_cast<float4 *>(orow + col) = make_float4(v[0], v[1], v[2], v[3]);
+      if (vecB && col + 3 < ncol) {
+        float *dst = col < nb ? a.c + (size_t)row * nb + col : a.s + (size_t)row * nb + (col - nb);
+        *reinterpret_cast<float4 *>(dst) = make_float4(v[0], v[1], v[2], v[3]);
       } else {
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          if (col + j < nb) orow[col + j] = v[j];
+        for (int j = 0; j < 4; ++j) {
+          const int vc = col + j;
+          if (vc < nb) a.c[(size_t)row * nb + vc] = v[j];
+          else if (vc < ncol) a.s[(size_t)row * nb + (vc - nb)] = v[j];
+        }
       }
     }
   }
@@ -181,8 +190,8 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
 }  // namespace
 
 int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st) {
-  const int ntn = (a.nb + BN - 1) / BN;
-  dim3 grid(mblk_upper, ntn * (a.noise ? 2 : 1));
+  const int ncol = a.noise ? 2 * a.nb : a.nb;
+  dim3 grid(mblk_upper, (ncol + BN - 1) / BN);
   return launch("gate_gemm_fp32", gate_gemm_kernel, grid, dim3(NT), 0, st, a);
 }
 

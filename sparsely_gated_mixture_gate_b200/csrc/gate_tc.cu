@@ -365,15 +365,13 @@ int launch_gate_tf32x3(const GateGemmArgs &a, int mblk_upper, float *xhi, float 
   t.status = a.status;
   const int64_t upper = (int64_t)mblk_upper * t.nblk;
   const int grid = (int)std::min<int64_t>(upper, num_sms());
-  static int attr_dev = -1;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_dev != dev) {
-    if (cudaFuncSetAttribute(gate_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             SMEM_BYTES) != cudaSuccess)
-      return MOE_ECUDA;
-    attr_dev = dev;
-  }
+  static PerDevice attrs;
+  MOE_TRY(attrs.get([](int, int *) {
+    return cudaFuncSetAttribute(gate_tf32x3_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                SMEM_BYTES) == cudaSuccess
+               ? MOE_OK
+               : MOE_ECUDA;
+  }));
   if (grid <= 0) return MOE_OK;
   return launch("gate_gemm_tf32x3", gate_tf32x3_kernel, dim3(grid), dim3(NUM_THREADS), SMEM_BYTES, st,
                 ahi, alo, bhi, blo, t);

@@ -7,6 +7,8 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <mutex>
+
 #include "../../include/moe.h"
 
 namespace moe {
@@ -37,6 +39,39 @@ int launch(const char *name, Kernel kernel, dim3 grid, dim3 block, size_t smem, 
     int _rc = (expr);            \
     if (_rc != MOE_OK) return _rc; \
   } while (0)
+
+// A value worked out once per device (a kernel attribute set, an occupancy,
+// a device check) and shared by every host thread: get() runs make(dev, &v)
+// for the current device the first time, under a lock, and returns the
+// stored value afterwards.  A failed make() stores nothing.
+constexpr int kMaxDevices = 64;
+class PerDevice {
+ public:
+  template <class F>
+  int get(F make, int *out = nullptr) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return MOE_EDEVICE;
+    std::lock_guard<std::mutex> lock(mu_);
+    if (!done_[dev]) {
+      int v = 0;
+      const int rc = make(dev, &v);
+      if (rc != MOE_OK) return rc;
+      val_[dev] = v;
+      done_[dev] = true;
+    }
+    if (out) *out = val_[dev];
+    return MOE_OK;
+  }
+
+ private:
+  std::mutex mu_;
+  bool done_[kMaxDevices] = {};
+  int val_[kMaxDevices] = {};
+};
+
+// MOE_OK when the current device is an sm_100 part (the library's only
+// target), else MOE_EDEVICE; checked once per device.
+int check_device();
 
 int num_sms();
 
@@ -75,6 +110,8 @@ struct RouteArgs {
   const float *c, *s;      // [R][nb]
   int R, nb, k, router, noise;
   uint64_t seed;
+  const unsigned long long *seed_dev;  // when set, the noise key is read here at run time
+  uint32_t token_base;     // added to the token index in the noise counter
   const int *row_token;    // [R] or nullptr
   const int *row_slot;     // [R] primary slot of the row (secondary gate), or nullptr
   const int *seg_off;      // [G+1] or nullptr
@@ -169,6 +206,9 @@ struct ExpertArgs {
   const void *mask;
 };
 int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st);
+// moe_test_expert_wait: the GEMM2 tiles' wait limit (0: the default) and an
+// M-block whose GEMM1 tiles do not publish (-1: none), for later launches
+void set_expert_wait(unsigned long long limit_ns, int withhold_mblock);
 int launch_expert_f32(const ExpertArgs &a, cudaStream_t st);
 
 // y_shared [T][d] (expert dtype) or nullptr: the shared expert's rows, added
@@ -176,6 +216,10 @@ int launch_expert_f32(const ExpertArgs &a, cudaStream_t st);
 int launch_combine(const void *y_perm, int bf16, const float *gate, const int *row_of,
                    const float *x, int passthrough, int T, int k, int d, float *y,
                    const void *y_shared, cudaStream_t st);
+// FP32 FMA throughput probe: blocks x 256 threads, 256 FLOP per thread per iteration
+int launch_fma_probe(float *out, int blocks, int iters, int packed, cudaStream_t st);
+// *seed += 1 (one thread)
+int launch_noise_step(unsigned long long *seed, cudaStream_t st);
 int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, float *bias,
                            cudaStream_t st);
 
@@ -188,6 +232,8 @@ struct GateBwdArgs {
   const float *lam_imp, *lam_load, *sw_coef;  // [n] (bwd_coef)
   const int4 *kth;             // [T] {H of the (k+1)-th, its id, H of the k-th, its id}
   unsigned long long seed;
+  const unsigned long long *seed_dev;  // when set, the noise key is read here at run time
+  uint32_t token_base;         // added to the token index in the noise counter
   int router, noise, has_load;
   float *dc, *dz;              // [T][n] outputs (dz: noise only)
 };

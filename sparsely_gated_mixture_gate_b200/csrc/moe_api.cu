@@ -99,16 +99,27 @@ void trace_end(int slot, cudaStream_t st) {
 void count_launch() { ++g_launches; }
 
 int num_sms() {
-  static int cached_dev = -1, cached = 148;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev != cached_dev) {
-    int v = 0;
-    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-      cached = v;
-    cached_dev = dev;
-  }
-  return cached;
+  static PerDevice sms;
+  int v = 148;
+  sms.get([](int dev, int *out) {
+    int c = 0;
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || c < 1)
+      return MOE_EDEVICE;
+    *out = c;
+    return MOE_OK;
+  }, &v);
+  return v;
+}
+
+int check_device() {
+  static PerDevice checked;
+  return checked.get([](int dev, int *) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return MOE_EDEVICE;
+    return (major == 10 && minor == 0) ? MOE_OK : MOE_EDEVICE;  // built for sm_100a only
+  });
 }
 
 int route_rows_per_tile(int R) {
@@ -286,19 +297,6 @@ int64_t capacity_of(const moe_config &c) {
   return (int64_t)ceil((double)c.T * (double)c.k * c.capacity_factor / (double)c.n);
 }
 
-int check_device() {
-  static int checked_dev = -1;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_EDEVICE;
-  if (dev == checked_dev) return MOE_OK;
-  int major = 0, minor = 0;
-  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-    return MOE_EDEVICE;
-  if (major != 10 || minor != 0) return MOE_EDEVICE;  // built for sm_100a only
-  checked_dev = dev;
-  return MOE_OK;
-}
 
 int common_checks(const moe_config *cfg, void *ws, size_t ws_bytes, int32_t *status,
                   Layout *L) {
@@ -383,6 +381,8 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.router = c.router;
   r.noise = c.noise;
   r.seed = c.seed;
+  r.token_base = (uint32_t)c.token_base;
+  r.seed_dev = reinterpret_cast<const unsigned long long *>(gp.seed_dev);
   r.G = 1;
   r.RT = L.RT1;
   r.load_part = at<float>(ws, L.load_part);
@@ -578,6 +578,7 @@ bool gate_params_ok(const moe_config &c, const moe_gate_params *gp) {
   if (c.hier_a > 0 && c.noise && (!gp->W_noise2 || !aligned(gp->W_noise2, 16))) return false;
   // the routing kernel reads the selection bias in 16-byte pieces
   if (c.router == MOE_ROUTER_SIGMOID && gp->sel_bias && !aligned(gp->sel_bias, 16)) return false;
+  if (gp->seed_dev && !aligned(gp->seed_dev, 8)) return false;
   return true;
 }
 
@@ -637,6 +638,7 @@ int moe_validate(const moe_config *c) {
     if (c->hier_k1 * c->hier_k2 != c->k) return MOE_EINVAL;
   }
   if ((int64_t)c->T * c->k > INT_MAX / 2) return MOE_EINVAL;
+  if (c->token_base < 0 || c->token_base + (int64_t)c->T > (int64_t)1 << 32) return MOE_EINVAL;
   return MOE_OK;
 }
 
@@ -979,6 +981,8 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   g.sw_coef = sw_coef;
   g.kth = at<int4>(ws, L.kth);
   g.seed = c.seed;
+  g.token_base = (uint32_t)c.token_base;
+  g.seed_dev = reinterpret_cast<const unsigned long long *>(gp->seed_dev);
   g.router = c.router;
   g.noise = c.noise;
   g.has_load = c.noise && c.w_load != 0.f;
@@ -1034,6 +1038,24 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
                                      cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ECUDA;
   return MOE_OK;
+}
+
+int moe_fma_probe(float *out, int blocks, int iters, int packed, moe_stream_t stream) {
+  if (!out || blocks < 1 || iters < 1) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_fma_probe(out, blocks, iters, packed ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_test_expert_wait(unsigned long long limit_ns, int withhold_mblock) {
+  set_expert_wait(limit_ns, withhold_mblock);
+  return MOE_OK;
+}
+
+int moe_noise_step(uint64_t *seed_dev, moe_stream_t stream) {
+  if (!seed_dev || !aligned(seed_dev, 8)) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_noise_step(reinterpret_cast<unsigned long long *>(seed_dev),
+                           reinterpret_cast<cudaStream_t>(stream));
 }
 
 int moe_sel_bias_update(const moe_config *cfg, const int32_t *counts, float gamma,

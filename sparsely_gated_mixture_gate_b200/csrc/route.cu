@@ -94,7 +94,8 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
   const int k = a.k;
   const bool vec4 = (nb & 3) == 0;  // rows start 16-byte aligned
   constexpr bool sw = SW;
-  const uint32_t key0 = (uint32_t)(a.seed & 0xffffffffu), key1 = (uint32_t)(a.seed >> 32);
+  const uint64_t seed = a.seed_dev ? (uint64_t)__ldg(a.seed_dev) : a.seed;
+  const uint32_t key0 = (uint32_t)(seed & 0xffffffffu), key1 = (uint32_t)(seed >> 32);
   const uint32_t gate_id = a.secondary ? (uint32_t)(1 + g) : 0u;
   bool bad = false;
 
@@ -163,7 +164,7 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
           for (int j = 0; j < 4; ++j) h[j] = cv[j] + bv[j];
         } else if (a.noise) {
           const uint4 wd =
-              philox4x32_10(make_uint4((uint32_t)t, (uint32_t)m, gate_id, 0u), key0, key1);
+              philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, gate_id, 0u), key0, key1);
           float z[4];
           box_muller2(wd.x, wd.y, z[0], z[1]);
           box_muller2(wd.z, wd.w, z[2], z[3]);

@@ -104,7 +104,15 @@ __global__ void sel_bias_update_kernel(const int *counts, int n, long long total
   else if (scaled < total) bias[i] = bias[i] + gamma;
 }
 
+// The next noise key: one add in stream order, so a captured graph that
+// starts with it draws new noise at every replay.
+__global__ void noise_step_kernel(unsigned long long *seed) { *seed += 1ull; }
+
 }  // namespace
+
+int launch_noise_step(unsigned long long *seed, cudaStream_t st) {
+  return launch("noise_step", noise_step_kernel, dim3(1), dim3(1), 0, st, seed);
+}
 
 int launch_sel_bias_update(const int *counts, int n, int T, int k, float gamma, float *bias,
                            cudaStream_t st) {

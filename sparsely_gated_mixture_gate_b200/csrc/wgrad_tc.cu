@@ -292,10 +292,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
 int launch_wgrad_bf16(const WgradArgs &a, cudaStream_t st) {
   if (a.n == 0) return MOE_OK;
-  static int attr_dev = -1, ctas = 0;
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (attr_dev != dev) {
+  static PerDevice setup;  // the kernel's shared-memory attribute, then its resident CTAs
+  int ctas = 0;
+  MOE_TRY(setup.get([](int, int *out) {
     if (cudaFuncSetAttribute(wgrad_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              SMEM_BYTES) != cudaSuccess)
       return MOE_ECUDA;
@@ -304,9 +303,9 @@ int launch_wgrad_bf16(const WgradArgs &a, cudaStream_t st) {
                                                       SMEM_BYTES) != cudaSuccess ||
         per_sm < 1)
       return MOE_ECUDA;
-    ctas = per_sm * num_sms();
-    attr_dev = dev;
-  }
+    *out = per_sm * num_sms();
+    return MOE_OK;
+  }, &ctas));
   // rows beyond S read as zero; every box is 64 columns x 64 rows
   const uint64_t S = (uint64_t)(a.S > 0 ? a.S : 1);
   CUtensorMap mA0, mB0, mA1, mB1;

@@ -53,6 +53,7 @@ class Config:
     backward: int = 0         # 1: the layer also runs the backward pass (workspace, saved state)
     w_z: float = 0.0          # backward: weight of the router z-loss (losses[8])
     w_entropy: float = 0.0    # backward: weight rewarding the gate entropy (-losses[9])
+    token_base: int = 0       # first token's index in the noise counter (a shard of a batch)
 
     @classmethod
     def from_workload(cls, w, T: Optional[int] = None) -> "Config":
@@ -71,7 +72,7 @@ class Config:
                           w_load=self.w_load, alpha_aux=self.alpha,
                           gate_precision=self.gate_precision, shared_expert=self.shared_expert,
                           router_stats=self.router_stats, backward=self.backward,
-                          w_z=self.w_z, w_entropy=self.w_entropy)
+                          w_z=self.w_z, w_entropy=self.w_entropy, token_base=self.token_base)
 
     @property
     def expert_dtype(self):
@@ -134,11 +135,17 @@ def workspace(cfg: Config, device) -> torch.Tensor:
     return torch.empty(max(workspace_size(cfg), 256), dtype=torch.uint8, device=device)
 
 
-def gate_params(params: dict) -> moe_gate_params:
+def gate_params(params: dict, seed_dev: Optional[torch.Tensor] = None) -> moe_gate_params:
     return moe_gate_params(W_g=_ptr(params.get("Wg")), b_g=_ptr(params.get("bg")),
                            W_noise=_ptr(params.get("Wn")), W_g2=_ptr(params.get("Wg2")),
                            b_g2=_ptr(params.get("bg2")), W_noise2=_ptr(params.get("Wn2")),
-                           sel_bias=_ptr(params.get("sel_bias")))
+                           sel_bias=_ptr(params.get("sel_bias")), seed_dev=_ptr(seed_dev))
+
+
+def noise_step(seed_dev: torch.Tensor):
+    """Advance the device noise key by one on the current stream."""
+    _need(seed_dev, "seed_dev", torch.int64, (1,))
+    _check(_lib.load().moe_noise_step(_ptr(seed_dev), _stream()), "moe_noise_step")
 
 
 def expert_params(params: dict) -> moe_expert_params:
@@ -270,9 +277,16 @@ def balance_losses(cfg: Config, topk_idx, topk_gate, counts, load, prob_sum=None
 # ---------------------------------------------------------------- fused layer
 class MoELayer:
     """Parameters plus pre-allocated workspace and outputs for repeated calls
-    of the fused ``moe_forward`` on one device."""
+    of the fused ``moe_forward`` on one device.
 
-    def __init__(self, cfg: Config, params: dict, device=None):
+    Noise: the noisy gate draws a new StandardNormal() every time it runs.
+    The layer keeps its noise key in a device word that every forward step
+    (direct or replayed from a CUDA graph) first advances by one, so step s
+    of the layer draws with key cfg.seed + s, and a backward step uses the key
+    of the forward before it.  noise_seed_(v) makes the next step draw with
+    key v.  With resample_noise=False every step draws with cfg.seed."""
+
+    def __init__(self, cfg: Config, params: dict, device=None, resample_noise: bool = True):
         self.cfg = cfg
         self.params = params
         dev = _dev(device) if device is not None else params["Wg"].device
@@ -280,7 +294,11 @@ class MoELayer:
         _check_params(cfg, params, dev)
         _lib.load()
         self._c = cfg.c()
-        self._gp = gate_params(params)
+        self.resample_noise = bool(resample_noise) and bool(cfg.noise)
+        # the key the last step used (the next step adds one first); uint64 bits in an int64
+        self.seed_dev = torch.empty(1, dtype=torch.int64, device=dev)
+        self.noise_seed_(cfg.seed)
+        self._gp = gate_params(params, self.seed_dev)
         self._ep = expert_params(params)
         self.ws = workspace(cfg, dev)
         self.status = new_status(dev)
@@ -293,14 +311,24 @@ class MoELayer:
         self.counts = torch.empty(n, dtype=torch.int32, device=dev)
         self.losses = torch.empty(10, dtype=torch.float32, device=dev)
 
+    def noise_seed_(self, seed: int):
+        """The next forward step draws its noise with key ``seed`` (stream
+        ordered: a device write on the current stream)."""
+        first = (seed - 1) if self.resample_noise else seed
+        first &= (1 << 64) - 1
+        self.seed_dev.fill_(first - (1 << 64) if first >= (1 << 63) else first)
+
     def forward_(self, x: torch.Tensor, stream=None, y: Optional[torch.Tensor] = None,
                  losses: Optional[torch.Tensor] = None):
         """Run the layer on device-resident x; outputs land in this object's
-        buffers, or in y / losses when given (asynchronous on the stream)."""
+        buffers, or in y / losses when given (asynchronous on the stream).
+        Advances the noise key first (see the class notes)."""
         _need(x, "x", torch.float32, (self.cfg.T, self.cfg.d), self.device)
         y = self.y if y is None else y
         losses = self.losses if losses is None else losses
         st = C.c_void_p(stream.cuda_stream) if stream is not None else _stream()
+        if self.resample_noise:
+            _check(_lib.load().moe_noise_step(_ptr(self.seed_dev), st), "moe_noise_step")
         _check(_lib.load().moe_forward(C.byref(self._c), _ptr(x), C.byref(self._gp), C.byref(self._ep),
                                        _ptr(y), _ptr(self.topk_idx), _ptr(self.topk_gate),
                                        _ptr(self.importance), _ptr(self.load), _ptr(self.counts),
@@ -318,10 +346,15 @@ class MoELayer:
             cap = torch.cuda.Stream(device=self.device)
             cap.wait_stream(torch.cuda.current_stream(self.device))
             with torch.cuda.stream(cap):
+                seed = self.seed_dev.clone()
                 record(cap)
             g = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g, stream=cap, capture_error_mode="thread_local"):
                 record(cap)
+            with torch.cuda.stream(cap):
+                # the set-up call consumed a noise key: put it back, so the
+                # replay that follows draws what a direct call would have
+                self.seed_dev.copy_(seed)
             torch.cuda.current_stream(self.device).wait_stream(cap)
             graphs[key] = g
         return g

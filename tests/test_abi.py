@@ -45,10 +45,11 @@ def test_struct_layout_matches_c(tmp_path):
 #include <stddef.h>
 #include "{HEADER}"
 int main(void) {{
-  printf("%zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config), offsetof(moe_config, seed),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config), offsetof(moe_config, seed),
          offsetof(moe_config, capacity_factor), offsetof(moe_config, gate_precision),
          sizeof(moe_gate_params), sizeof(moe_expert_params),
-         offsetof(moe_config, alpha_aux));
+         offsetof(moe_config, alpha_aux), offsetof(moe_config, token_base),
+         offsetof(moe_gate_params, seed_dev));
   return 0;
 }}
 ''')
@@ -58,7 +59,8 @@ int main(void) {{
     want = [C.sizeof(_lib.moe_config), _lib.moe_config.seed.offset,
             _lib.moe_config.capacity_factor.offset, _lib.moe_config.gate_precision.offset,
             C.sizeof(_lib.moe_gate_params), C.sizeof(_lib.moe_expert_params),
-            _lib.moe_config.alpha_aux.offset]
+            _lib.moe_config.alpha_aux.offset, _lib.moe_config.token_base.offset,
+            _lib.moe_gate_params.seed_dev.offset]
     assert vals == want
 
 
@@ -84,6 +86,7 @@ BAD = [
     dict(passthrough=2), dict(capacity_factor=float("nan")),
     dict(raw_expert_dtype=3), dict(raw_gate_precision=2),
     dict(raw_backward=2), dict(raw_shared_expert=2), dict(raw_router_stats=-1),
+    dict(token_base=-1), dict(token_base=(1 << 32) - 63),
 ]
 
 
@@ -157,3 +160,36 @@ def test_backward_workspace_and_refusals_without_gpu(lib):
     rc = lib.moe_backward(C.byref(cb), None, None, None, None, None, None, None, None, None, None,
                           None, None, 0, None, None)
     assert rc != _lib.MOE_OK
+
+
+def test_noise_step_and_probe_refuse_bad_arguments(lib):
+    """moe_noise_step wants an 8-byte aligned word, moe_fma_probe a buffer
+    and positive sizes: both refuse on the host, before any device work."""
+    assert lib.moe_noise_step(None, None) == _lib.MOE_EINVAL
+    buf = (C.c_uint64 * 2)()
+    assert lib.moe_noise_step(C.c_void_p(C.addressof(buf) + 4), None) == _lib.MOE_EINVAL
+    assert lib.moe_fma_probe(None, 1, 1, 0, None) == _lib.MOE_EINVAL
+    assert lib.moe_fma_probe(C.c_void_p(C.addressof(buf)), 0, 1, 0, None) == _lib.MOE_EINVAL
+    assert lib.moe_fma_probe(C.c_void_p(C.addressof(buf)), 1, 0, 1, None) == _lib.MOE_EINVAL
+    import torch
+    if not torch.cuda.is_available():
+        assert lib.moe_noise_step(C.c_void_p(C.addressof(buf)), None) == _lib.MOE_EDEVICE
+
+
+def test_gate_params_seed_word_must_be_aligned(lib):
+    """A misaligned seed word in moe_gate_params is an argument error."""
+    cfg = M.Config(T=64, d=32, n=8, k=2, f=64, expert_bf16=0)
+    c = cfg.c()
+    buf = (C.c_byte * 65536)()
+    base = C.addressof(buf) + (-C.addressof(buf)) % 256
+    fake = C.c_void_p(base)
+    gp = _lib.moe_gate_params(W_g=fake, W_noise=fake, seed_dev=C.c_void_p(base + 4))
+    ws = C.c_void_p(base)
+    rc = lib.moe_gate(C.byref(c), fake, C.byref(gp), fake, fake, fake, None, ws, 0, fake, None)
+    assert rc in (_lib.MOE_EINVAL, _lib.MOE_EWORKSPACE)
+    need = C.c_size_t(0)
+    assert lib.moe_workspace_size(C.byref(c), C.byref(need)) == _lib.MOE_OK
+    if need.value <= 65536 - 256:
+        rc = lib.moe_gate(C.byref(c), fake, C.byref(gp), fake, fake, fake, None, ws, need.value,
+                          fake, None)
+        assert rc == _lib.MOE_EINVAL

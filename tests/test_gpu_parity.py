@@ -1,22 +1,24 @@
 """GPU parity: every stage of the CUDA path (through the C ABI) against the
 oracle, element by element, on the same seeded inputs.
 
-Tolerances: expert ids and the permutation bit-exact (tokens whose k-th and
-(k+1)-th logits are closer than 1e-5 are counted and left out of the id and
-gate comparison); gates, load, importance and losses fp32 within 1e-5
-relative; layer output within 1e-4 relative Frobenius for fp32 experts and
-2e-2 for bf16 experts.
+Tolerances: expert ids and the permutation bit-exact; gates, load,
+importance and losses fp32 within 1e-5 relative; layer output within 1e-4
+relative Frobenius for fp32 experts and 2e-2 for bf16 experts.  A token whose
+kept logits come closer than 1e-5 (a near tie) is excluded together with
+every expert it reaches on either side, and nothing is skipped: the rest of
+the batch is compared (see parity_util).
 """
 import numpy as np
 import pytest
 import torch
 
+from parity_util import (TIE, assert_rel, check_routing, check_stats, rel_fro, touched_experts,
+                         y_rows_to_compare)
 from sparsely_gated_mixture_gate_b200 import build, synth
 from sparsely_gated_mixture_gate_b200 import moe as M
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
-TIE = 1e-5
 
 
 @pytest.fixture(scope="module", autouse=True)
@@ -38,21 +40,6 @@ def np_inputs(inp):
         else:
             out[k] = v.detach().cpu().numpy()
     return out
-
-
-def rel_fro(a, b):
-    a = np.asarray(a, np.float64)
-    b = np.asarray(b, np.float64)
-    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
-
-
-def assert_rel(got, want, rtol, atol=0.0, what=""):
-    got = np.asarray(got, np.float64)
-    want = np.asarray(want, np.float64)
-    err = np.abs(got - want)
-    bad = err > atol + rtol * np.abs(want)
-    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} off; worst {err.max():.3e} " \
-                          f"at {np.unravel_index(np.argmax(err), err.shape)}"
 
 
 # ------------------------------------------------------------------ workloads
@@ -89,16 +76,6 @@ SMALL = {
 }
 
 
-def check_routing(out_idx, out_gate, ref, what):
-    tie = ref["near_tie"] < TIE
-    ok = ~tie
-    idx = out_idx.cpu().numpy()
-    g = out_gate.cpu().numpy()
-    assert np.array_equal(idx[ok], ref["topk_idx"][ok]), f"{what}: expert ids differ"
-    assert_rel(g[ok], ref["topk_gate"][ok], 1e-5, 1e-7, f"{what} gates")
-    return int(tie.sum())
-
-
 GP = [pytest.param(0, id="fp32fma"), pytest.param(1, id="tf32x3")]
 
 
@@ -112,9 +89,13 @@ def test_gate_matches_oracle(orc, name, gp):
     torch.cuda.synchronize()
     assert M.status_bits(out["status"]) == 0
     ref = orc.gate_batch(w.cfg(), np_inputs(inp))
-    nt = check_routing(out["topk_idx"], out["topk_gate"], ref, name)
-    if nt == 0:
-        assert_rel(out["load"].cpu().numpy(), ref["load"], 1e-5, 1e-6 * w.T, f"{name} load")
+    idx = out["topk_idx"].cpu().numpy()
+    tie = check_routing(idx, out["topk_gate"].cpu().numpy(), ref, name)
+    u = ~touched_experts(w, tie, idx, ref["topk_idx"])
+    load = out["load"].cpu().numpy()
+    assert_rel(load[u], ref["load"][u], 1e-5, 1e-6 * w.T, f"{name} load")
+    if w.noise and not w.hier_a:  # a near-tie swap moves the smoothed load by O(gap)
+        assert_rel(load, ref["load"], 1e-5, 1e-6 * w.T, f"{name} load (all experts)")
     if w.router == 1:
         assert_rel(out["prob_sum"].cpu().numpy(), ref["prob_sum"], 1e-5, 1e-7 * w.T, f"{name} prob_sum")
 
@@ -311,15 +292,17 @@ def test_forward_matches_oracle(orc, name, gp):
     out = run_layer(w, inp)
     assert M.status_bits(out["status"]) == 0
     ref = orc.forward(w.cfg(), np_inputs(inp))
-    nt = check_routing(out["topk_idx"], out["topk_gate"], ref, name)
+    o = {key: v.numpy() for key, v in out.items()}
+    nt, nx = check_stats(orc, w, o, ref, name)
+    tie = ref["near_tie"] < TIE
+    touched = touched_experts(w, tie, o["topk_idx"], ref["topk_idx"])
+    rows = y_rows_to_compare(w, tie, touched, o["topk_idx"], ref["topk_idx"])
     if nt:
-        pytest.skip(f"{nt} near-tie tokens: whole-batch statistics not comparable")
-    assert np.array_equal(out["counts"].numpy(), ref["counts"])
-    assert_rel(out["load"].numpy(), ref["load"], 1e-5, 1e-6 * w.T, "load")
-    assert_rel(out["importance"].numpy(), ref["importance"], 1e-5, 1e-6, "importance")
-    assert_rel(out["losses"].numpy(), ref["losses"], 1e-5, 1e-7, "losses")
+        print(f"{name}: {nt} near-tie tokens, {nx} experts excluded, {rows.sum()} of {w.T} rows of y")
+    if w.T:
+        assert rows.sum() >= w.T // 2
     tol = 2e-2 if w.expert_bf16 else 1e-4
-    err = rel_fro(out["y"].numpy(), ref["y"])
+    err = rel_fro(o["y"][rows], ref["y"][rows])
     assert err < tol, err
 
 
@@ -414,6 +397,7 @@ def test_pipelined_host_batches_match_device_calls():
     layer.forward_host_batches(xs, ys, ls)
     torch.cuda.synchronize()
     for i in range(5):
+        layer.noise_seed_(w.seed + i)  # batch i drew its noise with key seed + i
         layer.forward_(xs[i].to(DEV))
         torch.cuda.synchronize()
         assert torch.equal(ys[i], layer.y.cpu()), i
@@ -432,12 +416,14 @@ def test_forward_graph_replay_matches_direct():
         x = dinp["x"]
         x2 = synth.make_inputs(w.with_(seed=w.seed + 7), experts=False)["x"].to(DEV)
         outs = []
-        for src in (x.clone(), x2):
+        for step, src in enumerate((x.clone(), x2)):
             x.copy_(src)
+            layer.noise_seed_(w.seed + step)
             layer.forward_(x)
             torch.cuda.synchronize()
             want = {k: v.clone() for k, v in layer.outputs().items()}
             layer.y.zero_()
+            layer.noise_seed_(w.seed + step)
             layer.forward_graph_(x)
             torch.cuda.synchronize()
             got = layer.outputs()
@@ -462,6 +448,7 @@ def test_forward_host_batches_with_graphs_matches_direct():
         want.append((layer.y.cpu().clone(), layer.losses.cpu().clone()))
     yh = [torch.empty(w.T, w.d).pin_memory() for _ in xs]
     lh = [torch.empty(layer.losses.numel()).pin_memory() for _ in xs]
+    layer.noise_seed_(w.seed)  # the same keys as the direct calls above
     d2h = layer.forward_host_batches([x.contiguous().pin_memory() for x in xs], yh, lh, graph=True)
     d2h.synchronize()
     torch.cuda.synchronize()
@@ -469,3 +456,59 @@ def test_forward_host_batches_with_graphs_matches_direct():
         assert torch.equal(yh[i], y), i
         assert torch.equal(lh[i], l), i
     layer.release_graph()
+
+
+def test_noise_is_redrawn_every_step(orc):
+    """The noisy gate draws new noise every time it runs ("極大規模神經網路：
+    稀疏門控專家混合層", Noisy Top-K 門控): step s of a layer uses noise key
+    seed + s, whether the step is a direct call or a CUDA graph replay, and
+    equals, bit for bit, a fresh layer configured with that seed; the oracle
+    with that seed gives the same routing."""
+    w = SMALL["lm-flat-512"]
+    inp = synth.make_inputs(w)
+    dinp = to_dev(inp)
+    layer = M.MoELayer(M.Config.from_workload(w), dinp, torch.device(DEV))
+    x = dinp["x"]
+    keys = ("y", "topk_idx", "topk_gate", "importance", "load", "counts", "losses")
+    steps = []
+    for call in (layer.forward_, layer.forward_graph_, layer.forward_graph_, layer.forward_):
+        call(x)
+        torch.cuda.synchronize()
+        steps.append({k: v.cpu().clone() for k, v in layer.outputs().items()})
+    layer.release_graph()
+    for s, got in enumerate(steps):
+        fresh = run_layer(w.with_(seed=w.seed + s), inp)
+        for k in keys:
+            assert torch.equal(got[k], fresh[k]), (s, k)
+    assert not torch.equal(steps[1]["topk_gate"], steps[2]["topk_gate"])
+    assert not torch.equal(steps[1]["load"], steps[2]["load"])
+    ref = orc.gate_batch(w.with_(seed=w.seed + 2).cfg(), np_inputs(synth.make_inputs(w, experts=False)))
+    check_routing(steps[2]["topk_idx"].numpy(), steps[2]["topk_gate"].numpy(), ref, "step 2")
+    # with resampling off every step draws with cfg.seed
+    fixed = M.MoELayer(M.Config.from_workload(w), dinp, torch.device(DEV), resample_noise=False)
+    fixed.forward_(x)
+    fixed.forward_(x)
+    torch.cuda.synchronize()
+    assert torch.equal(fixed.y.cpu(), steps[0]["y"])
+
+
+@pytest.mark.parametrize("name", ["lm-flat-512", "hier-small"])
+def test_shard_with_token_base_draws_the_batch_noise(name):
+    """A data-parallel shard of a batch (its tokens, token_base = the index
+    of its first token) routes exactly as those tokens do in the whole batch:
+    the noise counter runs over the batch's token indices."""
+    import dataclasses
+    w = SMALL[name]
+    inp = to_dev(synth.make_inputs(w, experts=False))
+    x = inp["x"]
+    whole = M.gate(M.Config.from_workload(w), x, inp)
+    h = w.T // 2 + 3
+    cfg = dataclasses.replace(M.Config.from_workload(w.with_(T=w.T - h)), token_base=h)
+    part = M.gate(cfg, x[h:].contiguous(), inp)
+    torch.cuda.synchronize()
+    assert torch.equal(part["topk_idx"], whole["topk_idx"][h:])
+    assert torch.equal(part["topk_gate"], whole["topk_gate"][h:])
+    # and without the base the shard draws other noise
+    other = M.gate(M.Config.from_workload(w.with_(T=w.T - h)), x[h:].contiguous(), inp)
+    torch.cuda.synchronize()
+    assert not torch.equal(other["topk_gate"], whole["topk_gate"][h:])

@@ -83,7 +83,30 @@ def test_noalloc_dispatch_matches_workspace_dispatch_twice():
 
 
 @pytest.mark.gpu
+@pytest.mark.parametrize("n,T_max", [(256, 524032), (4096, 4064)])
+def test_noalloc_dispatch_size_limit_is_exact(n, T_max):
+    """The documented limits: T_max tokens fit the fixed array (and give
+    moe_dispatch's results), T_max + 1 is refused before any device work."""
+    build.build()
+    L = _lib.load()
+    cfg = M.Config(T=T_max, d=8, n=n, k=4, f=8)
+    idx = synth.random_routing(T_max, 4, n, device=DEV, skew=0.5, seed=n)
+    x = torch.randn(T_max, 8, device=DEV)
+    a, b = _run_both(L, cfg, x, idx)
+    _same(a, b, int(a["offsets"][-1]))
+    c = M.Config(T=T_max + 1, d=8, n=n, k=4, f=8).c()
+    dummy = torch.zeros(16, dtype=torch.int32, device=DEV)
+    p = _p(dummy)
+    rc = L.moe_dispatch_noalloc(C.byref(c), None, p, p, p, p, p, None, p,
+                                C.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert rc == _lib.MOE_EWORKSPACE
+    torch.cuda.synchronize()
+    assert int(dummy.abs().sum()) == 0
+
+
+@pytest.mark.gpu
 def test_noalloc_dispatch_rejects_sizes_beyond_its_array():
+    build.build()
     L = _lib.load()
     cfg = M.Config(T=65536, d=512, n=4096, k=4, f=1024)
     c = cfg.c()
