@@ -334,6 +334,35 @@ MOE_API int moe_forward(const moe_config *cfg, const float *x, const moe_gate_pa
                 float *losses, void *ws, size_t ws_bytes, int32_t *status,
                 moe_stream_t stream);
 
+/* ---------------------------------------------------------------- expert parallel */
+
+/* Row gather for the expert-parallel layer ([MoE-deep] §7.1: each token's
+ * rows travel to the device of their expert and back).  dst row i = src row
+ * index[i], i < rows, each row row_bytes long (a positive multiple of 16);
+ * src holds src_rows rows.  An index outside [0, src_rows) gives a zero row
+ * and sets MOE_STATUS_BAD_INDEX.  src, dst: device memory, 16-byte aligned,
+ * not overlapping; index [rows] int32 device memory.  Used to regroup rows
+ * received from every rank by local expert before moe_expert_ffn, and (with
+ * the inverse index) to put the results back in the exchange's order.
+ * Errors: MOE_EINVAL (NULL or misaligned pointers, a bad row_bytes, negative
+ * sizes), MOE_EDEVICE, MOE_ECUDA. */
+MOE_API int moe_gather_rows(const void *src, const int32_t *index, void *dst, int64_t rows,
+                            int64_t row_bytes, int64_t src_rows, int32_t *status,
+                            moe_stream_t stream);
+
+/* The balancing losses of a batch split over data-parallel shards, from its
+ * totals ([SGMoE-xyz] "負載平衡損失"; [MoE-deep] §3.2): importance, load,
+ * counts and (Switch) prob_sum [n] are the sums over all shards' tokens,
+ * dropped [1] the sum of the slots each shard's own capacity cut dropped;
+ * cfg->T is the whole batch's token count.  losses[0..7] as moe_balance_losses
+ * (losses[4] = dropped / (T*k), losses[7] = dropped), losses[8], [9] = 0.
+ * Errors: MOE_EINVAL (invalid cfg, NULL pointers; prob_sum for Switch),
+ * MOE_EDEVICE, MOE_ECUDA. */
+MOE_API int moe_balance_from_totals(const moe_config *cfg, const float *importance,
+                                    const float *load, const int32_t *counts,
+                                    const float *prob_sum, const float *dropped, float *losses,
+                                    int32_t *status, moe_stream_t stream);
+
 /* ---------------------------------------------------------------- backward */
 
 /* Gradients written by moe_backward, fp32, caller-owned device memory in the

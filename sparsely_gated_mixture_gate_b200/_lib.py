@@ -18,7 +18,8 @@ EXPORTS = ("moe_strerror", "moe_validate", "moe_capacity", "moe_workspace_size",
            "moe_dispatch", "moe_expert_ffn", "moe_combine", "moe_balance_losses", "moe_forward",
            "moe_trace_enable", "moe_trace_reset", "moe_trace_count", "moe_trace_get",
            "moe_launch_count", "moe_dispatch_noalloc", "moe_sel_bias_update", "moe_backward",
-           "moe_noise_step", "moe_fma_probe", "moe_test_expert_wait")
+           "moe_noise_step", "moe_fma_probe", "moe_test_expert_wait", "moe_gather_rows",
+           "moe_balance_from_totals")
 
 
 class moe_config(C.Structure):
@@ -77,6 +78,9 @@ def load():
     L.moe_noise_step.argtypes = [vp, vp]
     L.moe_fma_probe.argtypes = [vp, i32, i32, i32, vp]
     L.moe_test_expert_wait.argtypes = [C.c_ulonglong, i32]
+    i64 = C.c_int64
+    L.moe_gather_rows.argtypes = [vp, vp, vp, i64, i64, i64, vp, vp]
+    L.moe_balance_from_totals.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_expert_ffn.argtypes = [cfgp, vp, vp, C.POINTER(moe_expert_params), vp, vp, sz, vp, vp]
     L.moe_combine.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp]
     L.moe_balance_losses.argtypes = [cfgp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp, vp]

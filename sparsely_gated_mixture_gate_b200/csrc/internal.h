@@ -297,9 +297,14 @@ int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *
                       cudaStream_t st);
 // rstats [2] or nullptr: the router statistics' sums over tokens (losses[8],
 // [9] become their means; 0 without them)
+// dropped (optional): the dropped slots counted elsewhere, instead of counts vs C
 int launch_losses(const float *importance, const float *load, const int *counts,
                   const float *prob_sum, int n, int T, int k, int64_t C, int router,
                   float w_imp, float w_load, float alpha, const float *rstats, float *losses,
-                  cudaStream_t st);
+                  cudaStream_t st, const float *dropped = nullptr);
+// dst[i] = src[index[i]] for rows of row_bytes (a multiple of 16); an index
+// outside [0, src_rows) gives a zero row and MOE_STATUS_BAD_INDEX
+int launch_gather_rows(const void *src, const int *index, void *dst, int64_t rows,
+                       int64_t row_bytes, int64_t src_rows, int *status, cudaStream_t st);
 
 }  // namespace moe

@@ -1046,6 +1046,30 @@ int moe_fma_probe(float *out, int blocks, int iters, int packed, moe_stream_t st
   return launch_fma_probe(out, blocks, iters, packed ? 1 : 0, reinterpret_cast<cudaStream_t>(stream));
 }
 
+int moe_gather_rows(const void *src, const int32_t *index, void *dst, int64_t rows,
+                    int64_t row_bytes, int64_t src_rows, int32_t *status, moe_stream_t stream) {
+  if (rows < 0 || src_rows < 0 || row_bytes <= 0 || row_bytes % 16) return MOE_EINVAL;
+  if (rows > 0 && (!src || !index || !dst || !aligned(src, 16) || !aligned(dst, 16)))
+    return MOE_EINVAL;
+  if (!status) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_gather_rows(src, index, dst, rows, row_bytes, src_rows, status,
+                            reinterpret_cast<cudaStream_t>(stream));
+}
+
+int moe_balance_from_totals(const moe_config *cfg, const float *importance, const float *load,
+                            const int32_t *counts, const float *prob_sum, const float *dropped,
+                            float *losses, int32_t *status, moe_stream_t stream) {
+  MOE_TRY(moe_validate(cfg));
+  const moe_config &c = *cfg;
+  if (!importance || !load || !counts || !dropped || !losses || !status) return MOE_EINVAL;
+  if (c.router == MOE_ROUTER_SWITCH && !prob_sum) return MOE_EINVAL;
+  MOE_TRY(check_device());
+  return launch_losses(importance, load, counts, prob_sum, c.n, c.T, c.k, INT64_MAX, c.router,
+                       c.w_importance, c.w_load, c.alpha_aux, nullptr, losses,
+                       reinterpret_cast<cudaStream_t>(stream), dropped);
+}
+
 int moe_test_expert_wait(unsigned long long limit_ns, int withhold_mblock) {
   set_expert_wait(limit_ns, withhold_mblock);
   return MOE_OK;

@@ -63,7 +63,8 @@ __global__ void __launch_bounds__(LNT) losses_kernel(const float *importance, co
                                                      const int *counts, const float *prob_sum,
                                                      int n, int T, int k, long long C, int router,
                                                      float w_imp, float w_load, float alpha,
-                                                     const float *rstats, float *losses) {
+                                                     const float *rstats, const float *dropped_in,
+                                                     float *losses) {
   __shared__ double sh[LNT / 32];
   const double cv_imp = cv2(importance, n, sh);
   const double cv_load = cv2(load, n, sh);
@@ -75,7 +76,9 @@ __global__ void __launch_bounds__(LNT) losses_kernel(const float *importance, co
       aux_part += ((double)c / (double)T) * ((double)prob_sum[i] / (double)T);
   }
   const double aux = block_sum(aux_part, sh) * (double)n;
-  const double dropped = block_sum(drop_part, sh);
+  // with dropped_in the dropped slots were counted elsewhere (the shards of
+  // an expert-parallel batch each cut at their own capacity)
+  const double dropped = dropped_in ? (double)*dropped_in : block_sum(drop_part, sh);
   if (threadIdx.x == 0) {
     const double S = (double)T * (double)k;
     losses[0] = (float)((double)w_imp * cv_imp);
@@ -128,10 +131,11 @@ int launch_importance(const float *gate_sorted, const int *ucoff, int n, float *
 
 int launch_losses(const float *importance, const float *load, const int *counts,
                   const float *prob_sum, int n, int T, int k, int64_t C, int router, float w_imp,
-                  float w_load, float alpha, const float *rstats, float *losses, cudaStream_t st) {
+                  float w_load, float alpha, const float *rstats, float *losses, cudaStream_t st,
+                  const float *dropped) {
   return launch("balance_losses", losses_kernel, dim3(1), dim3(LNT), 0, st, importance, load,
                 counts, prob_sum, n, T, k, (long long)C, router, w_imp, w_load, alpha, rstats,
-                losses);
+                dropped, losses);
 }
 
 }  // namespace moe

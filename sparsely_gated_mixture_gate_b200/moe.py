@@ -8,6 +8,7 @@ from __future__ import annotations
 
 import ctypes as C
 import dataclasses
+import math
 from typing import Optional
 
 import torch
@@ -272,6 +273,38 @@ def balance_losses(cfg: Config, topk_idx, topk_gate, counts, load, prob_sum=None
                                           _ptr(ws), ws.numel(), _ptr(status), _stream()),
            "moe_balance_losses")
     return dict(importance=importance, losses=losses, status=status)
+
+
+def gather_rows(src: torch.Tensor, index: torch.Tensor, src_rows: Optional[int] = None,
+                out: Optional[torch.Tensor] = None, status=None) -> torch.Tensor:
+    """out[i] = src[index[i]] (whole rows, through moe_gather_rows); an index
+    outside [0, src_rows) gives a zero row and the BAD_INDEX status bit."""
+    _need(index, "index", torch.int32, None, src.device)
+    rows = index.numel()
+    if not src.is_cuda or not src.is_contiguous():
+        raise MoEError("src must be a contiguous CUDA tensor")
+    row_shape = tuple(src.shape[1:])
+    if out is None:
+        out = torch.empty((rows,) + row_shape, dtype=src.dtype, device=src.device)
+    row_bytes = math.prod(row_shape) * src.element_size()
+    status = new_status(src.device) if status is None else status
+    _check(_lib.load().moe_gather_rows(_ptr(src), _ptr(index), _ptr(out), rows, row_bytes,
+                                       src.shape[0] if src_rows is None else src_rows,
+                                       _ptr(status), _stream()), "moe_gather_rows")
+    return out
+
+
+def balance_from_totals(cfg: Config, importance, load, counts, prob_sum, dropped, status=None):
+    """The losses [10] of a batch from its totals over data-parallel shards
+    (moe_balance_from_totals; cfg.T is the whole batch)."""
+    dev = importance.device
+    losses = torch.empty(10, dtype=torch.float32, device=dev)
+    status = new_status(dev) if status is None else status
+    c = cfg.c()
+    _check(_lib.load().moe_balance_from_totals(C.byref(c), _ptr(importance), _ptr(load), _ptr(counts),
+                                               _ptr(prob_sum), _ptr(dropped), _ptr(losses),
+                                               _ptr(status), _stream()), "moe_balance_from_totals")
+    return losses
 
 
 # ---------------------------------------------------------------- fused layer

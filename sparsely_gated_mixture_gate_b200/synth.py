@@ -100,6 +100,10 @@ VARIANTS = {
                                   noise=0, shared_expert=1, sel_bias_std=0.5, expert_bf16=0),
     "deepseek-flat": Workload("deepseek-flat", T=8192, d=512, n=256, k=8, f=512, router=2,
                               noise=0, shared_expert=1, sel_bias_std=0.1, x_unit_rows=True),
+    # the hierarchical layer with 8 of its 64 groups and the same ~32 rows per
+    # expert: 2.1 GB of expert weights instead of 17.2 GB, for profiler captures
+    "hierarchical-a8": WORKLOADS["hierarchical"].with_(name="hierarchical-a8", T=8192, n=8 * 128,
+                                                       hier_a=8),
 }
 
 
