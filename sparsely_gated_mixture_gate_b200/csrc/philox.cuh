@@ -17,19 +17,14 @@
 
 namespace moe {
 
-// Each round's two products are taken as one 32 x 32 -> 64-bit multiply each
-// (both halves at once), and round r's key is k + r * (Weyl constant), a
-// function of the key alone, so a caller's loop can keep the ten round keys
-// instead of bumping the key every round.
 __device__ __forceinline__ uint4 philox4x32_10(uint4 ctr, uint32_t k0, uint32_t k1) {
 #pragma unroll
   for (int round = 0; round < 10; ++round) {
-    const uint64_t p0 = (uint64_t)0xD2511F53u * ctr.x;
-    const uint64_t p1 = (uint64_t)0xCD9E8D57u * ctr.z;
-    const uint32_t rk0 = k0 + (uint32_t)round * 0x9E3779B9u;
-    const uint32_t rk1 = k1 + (uint32_t)round * 0xBB67AE85u;
-    ctr = make_uint4((uint32_t)(p1 >> 32) ^ ctr.y ^ rk0, (uint32_t)p1,
-                     (uint32_t)(p0 >> 32) ^ ctr.w ^ rk1, (uint32_t)p0);
+    const uint32_t hi0 = __umulhi(0xD2511F53u, ctr.x), lo0 = 0xD2511F53u * ctr.x;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, ctr.z), lo1 = 0xCD9E8D57u * ctr.z;
+    ctr = make_uint4(hi1 ^ ctr.y ^ k0, lo1, hi0 ^ ctr.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
   }
   return ctr;
 }
