@@ -789,9 +789,260 @@ void orc_expert_backward(int d, int f, int bf16, int nrows, const float *x_rows,
   }
 }
 
+/* One noisy top-k softmax level of a gate ([SGMoE-xyz] "Noisy Top-K 門控"),
+ * backward: H = c + eps s, G = Softmax over the kept k of H, s = Softplus(z),
+ * z = x W_noise.  In: the row's c, s, H and order (orc_gate_row), its kept
+ * gates gk and dL/dG of them (dG), the load-loss coefficient of each column
+ * (lam_load, NULL without a load term), the noise stream's (token, gate id).
+ * Out: dc [m] (dL/dc) and dz [m] (dL/dz, noise only); scratch dH [m], rank [m].
+ * The load term differentiates P(x,i) = Phi((c_i - thr_i) / s_i) in c_i, s_i
+ * and in the H of the expert that fixes thr_i, as in orc_backward. */
+static void level_bwd(int m, int k, int noise, uint64_t seed, uint32_t tok, uint32_t gate_id,
+                      const float *xt, int d, const float *Wn, const double *c, const double *s,
+                      const float *H, const int *order, const double *gk, const double *dG,
+                      const double *lam_load, double *dc, double *dz, double *dH, int *rank)
+{
+  for (int r = 0; r < m; ++r) rank[order[r]] = r;
+  for (int i = 0; i < m; ++i) dc[i] = dz[i] = dH[i] = 0.0;
+  double sum = 0.0;
+  for (int j = 0; j < k; ++j) sum += gk[j] * dG[j];
+  for (int j = 0; j < k; ++j) dH[order[j]] = gk[j] * (dG[j] - sum);
+  if (noise && lam_load) {
+    const int jk = order[k - 1], jk1 = k < m ? order[k] : -1;
+    for (int i = 0; i < m; ++i) {
+      const int jt = rank[i] < k ? jk1 : jk;
+      if (jt < 0 || s[i] == 0.0) continue;
+      const double u = (c[i] - (double)H[jt]) / s[i];
+      const double a = lam_load[i] * exp(-0.5 * u * u) / sqrt(2.0 * acos(-1.0)) / s[i];
+      dc[i] += a;
+      dz[i] -= a * u;
+      dH[jt] -= a;
+    }
+  }
+  for (int i = 0; i < m; ++i) {
+    dc[i] += dH[i];
+    if (noise) dz[i] += dH[i] * orc_noise(seed, tok, (uint32_t)i, gate_id);
+  }
+  if (noise)
+    for (int i = 0; i < m; ++i) {
+      double z = 0.0;
+      for (int q = 0; q < d; ++q) z += (double)xt[q] * (double)Wn[(size_t)q * m + i];
+      dz[i] *= 1.0 / (1.0 + exp(-z));
+    }
+}
+
+/* The backward of a gate level's projections c = x W + bias, z = x W_noise
+ * (W, W_noise [d][m]): adds x dc^T to dW, dc to db, x dz^T to dWn and
+ * W dc + W_noise dz to dxt. */
+static void level_proj_bwd(int d, int m, int noise, const float *xt, const float *W, const float *Wn,
+                           const double *dc, const double *dz, double *dW, double *db, double *dWn,
+                           double *dxt)
+{
+  for (int q = 0; q < d; ++q) {
+    double acc = 0.0;
+    for (int i = 0; i < m; ++i) {
+      acc += W[(size_t)q * m + i] * dc[i];
+      if (dW) dW[(size_t)q * m + i] += (double)xt[q] * dc[i];
+      if (noise) {
+        acc += Wn[(size_t)q * m + i] * dz[i];
+        if (dWn) dWn[(size_t)q * m + i] += (double)xt[q] * dz[i];
+      }
+    }
+    dxt[q] += acc;
+  }
+  if (db)
+    for (int i = 0; i < m; ++i) db[i] += dc[i];
+}
+
+/* The hierarchical layer ([SGMoE-note] "分层 MoE"): token t's slot ps*k2+ss
+ * is expert gi*b + j, gi the ps-th kept group of the primary gate and j the
+ * ss-th kept expert of gi's gate, with gate G_p(x)_gi G_gi(x)_j.  Importance
+ * sums the slot gates; Load(gi*b+j) = Load_p(X)_gi Load_gi(X_gi)_j / |X_gi|,
+ * the forward's reading, |X_gi| a count (no gradient): so the load loss
+ * reaches the primary level through lam_p(gi) = sum_j lamL(gi*b+j)
+ * Load_gi_j / |X_gi| and group gi's level through lam_s(gi, j) =
+ * lamL(gi*b+j) Load_p_gi / |X_gi|.  Each level's chain rule is that of the
+ * flat gate (level_bwd); the experts and the combine are the flat layer's. */
+static int orc_backward_hier(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g)
+{
+  const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f, bf16 = cfg->expert_bf16;
+  const int a = cfg->hier_a, b = cfg->hier_b, k1 = cfg->hier_k1, k2 = cfg->hier_k2;
+  const int noise = cfg->noise;
+  const size_t esz = bf16 ? 2 : 4;
+  const size_t S = (size_t)T * k;
+  const int mx = a > b ? a : b;
+
+  int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  double *gate = (double *)malloc(sizeof(double) * (S ? S : 1));
+  double *load = (double *)malloc(sizeof(double) * (size_t)n);
+  double *psum = (double *)malloc(sizeof(double) * (size_t)n);
+  double *imp = (double *)calloc((size_t)n, sizeof(double));
+  int32_t *counts = (int32_t *)malloc(sizeof(int32_t) * (size_t)n);
+  int32_t *offsets = (int32_t *)malloc(sizeof(int32_t) * (size_t)(n + 1));
+  int32_t *ptok = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  int32_t *pslot = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  int32_t *row_of = (int32_t *)malloc(sizeof(int32_t) * (S ? S : 1));
+  orc_gate_batch(cfg, in, idx, gate, load, psum, NULL);
+  const int64_t C = orc_capacity(T, k, n, cfg->capacity_factor);
+  orc_dispatch(T, k, n, C, idx, counts, offsets, ptok, pslot, row_of, NULL);
+  for (size_t p = 0; p < S; ++p) imp[idx[p]] += gate[p];
+
+  /* the two levels' loads and the group sizes (as the forward sums them) */
+  double *cp = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *sp = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *cs = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *ss = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *P = (double *)malloc(sizeof(double) * (size_t)mx);
+  float *Hp = (float *)malloc(sizeof(float) * (size_t)mx);
+  float *Hs = (float *)malloc(sizeof(float) * (size_t)mx);
+  int *op = (int *)malloc(sizeof(int) * (size_t)mx);
+  int *os = (int *)malloc(sizeof(int) * (size_t)mx);
+  double *g1 = (double *)malloc(sizeof(double) * (size_t)(k1 + 1));
+  double *g2 = (double *)malloc(sizeof(double) * (size_t)(k2 + 1));
+  double *load_p = (double *)calloc((size_t)a, sizeof(double));
+  double *load_s = (double *)calloc((size_t)a * b, sizeof(double));
+  int64_t *cnt = (int64_t *)calloc((size_t)a, sizeof(int64_t));
+  for (int t = 0; t < T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    orc_gate_row(d, a, k1, 0, noise, cfg->seed, (uint32_t)t, 0u, xt, in->Wg, in->bg, in->Wn, cp, sp,
+                 Hp, op, g1, NULL, NULL);
+    orc_load_row(a, k1, noise, cp, sp, Hp, P);
+    for (int i = 0; i < a; ++i) load_p[i] += P[i];
+    for (int ps = 0; ps < k1; ++ps) {
+      const int gi = op[ps];
+      cnt[gi]++;
+      orc_gate_row(d, b, k2, 0, noise, cfg->seed, (uint32_t)t, (uint32_t)(1 + gi), xt,
+                   in->Wg2 + (size_t)gi * d * b, in->bg2 ? in->bg2 + (size_t)gi * b : NULL,
+                   in->Wn2 ? in->Wn2 + (size_t)gi * d * b : NULL, cs, ss, Hs, os, g2, NULL, NULL);
+      orc_load_row(b, k2, noise, cs, ss, Hs, P);
+      for (int j = 0; j < b; ++j) load_s[(size_t)gi * b + j] += P[j];
+    }
+  }
+
+  double *lam_imp = (double *)malloc(sizeof(double) * (size_t)n);
+  double *lam_load = (double *)malloc(sizeof(double) * (size_t)n);
+  orc_cv2_grad(imp, n, lam_imp);
+  orc_cv2_grad(load, n, lam_load);
+  for (int i = 0; i < n; ++i) {
+    lam_imp[i] *= cfg->w_importance;
+    lam_load[i] *= cfg->w_load;
+  }
+  const int load_term = noise && cfg->w_load != 0.0;
+  double *lam_p = (double *)calloc((size_t)a, sizeof(double));
+  double *lam_s = (double *)calloc((size_t)a * b, sizeof(double));
+  for (int i = 0; i < a; ++i) {
+    if (cnt[i] == 0) continue;
+    for (int j = 0; j < b; ++j) {
+      lam_p[i] += lam_load[(size_t)i * b + j] * load_s[(size_t)i * b + j] / (double)cnt[i];
+      lam_s[(size_t)i * b + j] = lam_load[(size_t)i * b + j] * load_p[i] / (double)cnt[i];
+    }
+  }
+
+#define ZERO(ptr, cnt_) do { if (ptr) memset((ptr), 0, sizeof(double) * (size_t)(cnt_)); } while (0)
+  ZERO(g->dx, (size_t)T * d);
+  ZERO(g->dWg, (size_t)d * a); ZERO(g->dbg, a); ZERO(g->dWn, (size_t)d * a);
+  ZERO(g->dWg2, (size_t)a * d * b); ZERO(g->dbg2, (size_t)a * b); ZERO(g->dWn2, (size_t)a * d * b);
+  ZERO(g->dW1, (size_t)n * f * d); ZERO(g->db1, (size_t)n * f);
+  ZERO(g->dW2, (size_t)n * d * f); ZERO(g->db2, (size_t)n * d);
+  ZERO(g->dgate, S);
+#undef ZERO
+  double *dW1 = g->dW1 ? g->dW1 : (double *)calloc((size_t)n * f * d, sizeof(double));
+  double *dW2 = g->dW2 ? g->dW2 : (double *)calloc((size_t)n * d * f, sizeof(double));
+  double *dx = g->dx;
+
+  /* ---- combine and experts, as in the flat layer */
+  double *dgate = (double *)calloc(S ? S : 1, sizeof(double));
+  for (int t = 0; t < T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    const float *dyt = dy + (size_t)t * d;
+    double *dxt = dx + (size_t)t * d;
+    int kept = 0;
+    for (int j = 0; j < k; ++j) {
+      size_t pj = (size_t)t * k + j;
+      if (row_of[pj] < 0) continue;
+      kept++;
+      int e = idx[pj];
+      dgate[pj] = expert_row_bwd(
+          d, f, bf16, xt, (const char *)in->W1 + (size_t)e * f * d * esz,
+          in->b1 ? in->b1 + (size_t)e * f : NULL, (const char *)in->W2 + (size_t)e * d * f * esz,
+          in->b2 ? in->b2 + (size_t)e * d : NULL, gate[pj], dyt, dW1 + (size_t)e * f * d,
+          g->db1 ? g->db1 + (size_t)e * f : NULL, dW2 + (size_t)e * d * f,
+          g->db2 ? g->db2 + (size_t)e * d : NULL, dxt);
+    }
+    if (kept == 0 && cfg->passthrough)
+      for (int q = 0; q < d; ++q) dxt[q] += (double)dyt[q];
+  }
+  if (g->dgate) memcpy(g->dgate, dgate, sizeof(double) * S);
+
+  /* ---- the two gate levels */
+  double *dG1 = (double *)malloc(sizeof(double) * (size_t)k1);
+  double *dG2 = (double *)malloc(sizeof(double) * (size_t)k2);
+  double *dc = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *dz = (double *)malloc(sizeof(double) * (size_t)mx);
+  double *dH = (double *)malloc(sizeof(double) * (size_t)mx);
+  int *rank = (int *)malloc(sizeof(int) * (size_t)mx);
+  for (int t = 0; t < T; ++t) {
+    const float *xt = in->x + (size_t)t * d;
+    double *dxt = dx + (size_t)t * d;
+    orc_gate_row(d, a, k1, 0, noise, cfg->seed, (uint32_t)t, 0u, xt, in->Wg, in->bg, in->Wn, cp, sp,
+                 Hp, op, g1, NULL, NULL);
+    for (int ps = 0; ps < k1; ++ps) dG1[ps] = 0.0;
+    for (int ps = 0; ps < k1; ++ps) {
+      const int gi = op[ps];
+      const float *Wg2 = in->Wg2 + (size_t)gi * d * b;
+      const float *Wn2 = in->Wn2 ? in->Wn2 + (size_t)gi * d * b : NULL;
+      orc_gate_row(d, b, k2, 0, noise, cfg->seed, (uint32_t)t, (uint32_t)(1 + gi), xt, Wg2,
+                   in->bg2 ? in->bg2 + (size_t)gi * b : NULL, Wn2, cs, ss, Hs, os, g2, NULL, NULL);
+      /* slot gate G_p G_s: dL/dG_s = dL/dslot G_p, dL/dG_p = sum_ss dL/dslot G_s */
+      for (int s2 = 0; s2 < k2; ++s2) {
+        const size_t slot = (size_t)t * k + (size_t)ps * k2 + s2;
+        const double dslot = dgate[slot] + lam_imp[(size_t)gi * b + os[s2]];
+        dG1[ps] += dslot * g2[s2];
+        dG2[s2] = dslot * g1[ps];
+      }
+      level_bwd(b, k2, noise, cfg->seed, (uint32_t)t, (uint32_t)(1 + gi), xt, d, Wn2, cs, ss, Hs, os,
+                g2, dG2, load_term ? lam_s + (size_t)gi * b : NULL, dc, dz, dH, rank);
+      level_proj_bwd(d, b, noise, xt, Wg2, Wn2, dc, dz, g->dWg2 ? g->dWg2 + (size_t)gi * d * b : NULL,
+                     g->dbg2 ? g->dbg2 + (size_t)gi * b : NULL,
+                     g->dWn2 ? g->dWn2 + (size_t)gi * d * b : NULL, dxt);
+    }
+    level_bwd(a, k1, noise, cfg->seed, (uint32_t)t, 0u, xt, d, in->Wn, cp, sp, Hp, op, g1, dG1,
+              load_term ? lam_p : NULL, dc, dz, dH, rank);
+    /* router z-loss and entropy of the primary gate's clean logits, as flat */
+    if (T > 0 && (cfg->w_z != 0.0 || cfg->w_entropy != 0.0)) {
+      double m = cp[0];
+      for (int i = 1; i < a; ++i) if (cp[i] > m) m = cp[i];
+      double Ssum = 0.0;
+      for (int i = 0; i < a; ++i) Ssum += exp(cp[i] - m);
+      const double logS = log(Ssum);
+      double ent = 0.0;
+      for (int i = 0; i < a; ++i) {
+        const double lp = cp[i] - m - logS;
+        ent -= exp(lp) * lp;
+      }
+      for (int i = 0; i < a; ++i) {
+        const double lp = cp[i] - m - logS;
+        dc[i] += (cfg->w_z * 2.0 * cp[i] + cfg->w_entropy * exp(lp) * (lp + ent)) / (double)T;
+      }
+    }
+    level_proj_bwd(d, a, noise, xt, in->Wg, in->Wn, dc, dz, g->dWg, g->dbg, g->dWn, dxt);
+  }
+
+  if (!g->dW1) free(dW1);
+  if (!g->dW2) free(dW2);
+  free(dG1); free(dG2); free(dc); free(dz); free(dH); free(rank);
+  free(cp); free(sp); free(cs); free(ss); free(P); free(Hp); free(Hs); free(op); free(os);
+  free(g1); free(g2); free(load_p); free(load_s); free(cnt); free(lam_p); free(lam_s);
+  free(lam_imp); free(lam_load); free(dgate);
+  free(idx); free(gate); free(load); free(psum); free(imp); free(counts); free(offsets);
+  free(ptok); free(pslot); free(row_of);
+  return 0;
+}
+
 int orc_backward(const orc_cfg *cfg, const orc_inputs *in, const float *dy, orc_grads *g)
 {
-  if (!valid_cfg(cfg) || cfg->hier_a) return -1;
+  if (!valid_cfg(cfg)) return -1;
+  if (cfg->hier_a) return cfg->shared_expert ? -1 : orc_backward_hier(cfg, in, dy, g);
   if (cfg->shared_expert && (!in->W1s || !in->W2s)) return -1;
   const int T = cfg->T, d = cfg->d, n = cfg->n, k = cfg->k, f = cfg->f, bf16 = cfg->expert_bf16;
   const int noise = cfg->noise;

@@ -185,10 +185,13 @@ int orc_forward(const orc_cfg *cfg, const orc_inputs *in, orc_outputs *out);
  *   L = sum_t <dy_t, y_t> + losses[0] + losses[1] + losses[3]
  *       + w_z * losses[8] - w_entropy * losses[9]
  * (an upstream gradient dy[T][d] of the layer output plus the weighted
- * balancing losses of orc_forward) with respect to x and every parameter;
- * flat layers only (hier_a == 0).  With expert_bf16 the rounding points of a
- * mixed-precision backward are taken (see orc_backward).  Any pointer other
- * than dx and the routed experts' may be NULL (not written). */
+ * balancing losses of orc_forward) with respect to x and every parameter.
+ * For a hierarchical layer dWg, dbg, dWn are the primary gate's ([d][a],
+ * [a], [d][a]), dWg2, dbg2, dWn2 the secondary gates' ([a][d][b], [a][b],
+ * [a][d][b]), and dlogits / dnoise are not written.  With expert_bf16 the
+ * rounding points of a mixed-precision backward are taken (see
+ * orc_backward).  Any pointer other than dx and the routed experts' may be
+ * NULL (not written). */
 typedef struct {
   double *dx;                                 /* [T][d]                      */
   double *dWg, *dbg, *dWn;                    /* [d][n], [n], [d][n] (noise) */
@@ -197,6 +200,7 @@ typedef struct {
   double *dgate;                              /* [T][k] dL / d topk_gate      */
   double *dlogits;                            /* [T][n] dL / d (x W_g + b_g)  */
   double *dnoise;                             /* [T][n] dL / d (x W_noise)    */
+  double *dWg2, *dbg2, *dWn2;                 /* hierarchical: [a][d][b], [a][b], [a][d][b] */
 } orc_grads;
 
 /* d CV(v)^2 / d v_i of orc_cv2 (0 where the mean is 0). */

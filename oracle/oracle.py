@@ -64,7 +64,7 @@ class OrcOutputs(C.Structure):
 class OrcGrads(C.Structure):
     _fields_ = [(name, C.c_void_p) for name in (
         "dx", "dWg", "dbg", "dWn", "dW1", "db1", "dW2", "db2", "dW1s", "db1s", "dW2s", "db2s",
-        "dgate", "dlogits", "dnoise")]
+        "dgate", "dlogits", "dnoise", "dWg2", "dbg2", "dWn2")]
 
 
 def lib():
@@ -342,17 +342,22 @@ def cv2_grad(v) -> np.ndarray:
 def backward(cfg: dict, inp: dict, dy) -> dict:
     """Gradients of L = sum(dy * y) + losses[0] + losses[1] + losses[3]
     + w_z losses[8] - w_entropy losses[9] of
-    ``forward(cfg, inp)`` with respect to x and every parameter (flat layers);
-    also dL/d topk_gate ("dgate"), dL/d clean logits ("dlogits") and dL/d
-    (x W_noise) ("dnoise")."""
+    ``forward(cfg, inp)`` with respect to x and every parameter; also dL/d
+    topk_gate ("dgate") and, for flat layers, dL/d clean logits ("dlogits")
+    and dL/d (x W_noise) ("dnoise").  Hierarchical layers: dWg, dbg, dWn are
+    the primary gate's, dWg2, dbg2, dWn2 the secondary gates'."""
     oc = make_cfg(**cfg)
     T, d, n, k, f = oc.T, oc.d, oc.n, oc.k, oc.f
     keep, ins = _inputs(oc, inp)
     dy = _c(dy, np.float32)
-    out = dict(dx=np.zeros((T, d)), dWg=np.zeros((d, n)), dbg=np.zeros(n), dWn=np.zeros((d, n)),
+    gn = oc.hier_a if oc.hier_a else n   # width of the flat or primary gate
+    out = dict(dx=np.zeros((T, d)), dWg=np.zeros((d, gn)), dbg=np.zeros(gn), dWn=np.zeros((d, gn)),
                dW1=np.zeros((n, f, d)), db1=np.zeros((n, f)), dW2=np.zeros((n, d, f)),
                db2=np.zeros((n, d)), dgate=np.zeros((T, k)), dlogits=np.zeros((T, n)),
                dnoise=np.zeros((T, n)))
+    if oc.hier_a:
+        a_, b_ = oc.hier_a, oc.hier_b
+        out.update(dWg2=np.zeros((a_, d, b_)), dbg2=np.zeros((a_, b_)), dWn2=np.zeros((a_, d, b_)))
     if oc.shared_expert:
         out.update(dW1s=np.zeros((f, d)), db1s=np.zeros(f), dW2s=np.zeros((d, f)), db2s=np.zeros(d))
     g = OrcGrads(**{name: _p(a) for name, a in out.items()})

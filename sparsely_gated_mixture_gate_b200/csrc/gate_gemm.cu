@@ -190,6 +190,7 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
 }  // namespace
 
 int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st) {
+  if (gate_gemm_cutlass_applies(a)) return launch_gate_gemm_cutlass(a, st);
   const int ncol = a.noise ? 2 * a.nb : a.nb;
   dim3 grid(mblk_upper, (ncol + BN - 1) / BN);
   return launch("gate_gemm_fp32", gate_gemm_kernel, grid, dim3(NT), 0, st, a);

@@ -340,8 +340,10 @@ def test_forward_zero_tokens():
     assert torch.all(out["losses"] == 0)
 
 
-def test_nonfinite_input_sets_status():
-    w = SMALL["lm-flat-512"]
+@pytest.mark.parametrize("w", [SMALL["lm-flat-512"], W["many-expert"].with_(T=64, d=64, f=64),
+                               W["many-expert"].with_(T=64, d=64, f=64, noise=0)],
+                         ids=["lm-flat-512", "n4096", "n4096-nonoise"])
+def test_nonfinite_input_sets_status(w):
     inp = synth.make_inputs(w)
     inp["x"][5, 3] = float("nan")
     out = run_layer(w, inp)

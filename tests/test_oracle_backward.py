@@ -223,13 +223,17 @@ def test_bf16_rounding_points_track_fp32_gradient():
                           O.backward(dict(cfg, expert_bf16=1), b, z)["dlogits"])
 
 
-def test_hierarchical_rejected():
+def test_hierarchical_with_a_shared_expert_rejected():
+    """The hierarchical layer's backward covers routed experts only (the pages'
+    hierarchical layer has no shared expert)."""
     with pytest.raises(ValueError):
-        O.backward(dict(T=2, d=4, n=4, k=1, f=8, hier_a=2, hier_b=2, hier_k1=1, hier_k2=1),
+        O.backward(dict(T=2, d=4, n=4, k=1, f=8, hier_a=2, hier_b=2, hier_k1=1, hier_k2=1,
+                        shared_expert=1),
                    dict(x=np.zeros((2, 4), np.float32), Wg=np.zeros((4, 2), np.float32),
                         Wn=np.zeros((4, 2), np.float32), Wg2=np.zeros((2, 4, 2), np.float32),
                         Wn2=np.zeros((2, 4, 2), np.float32), W1=np.zeros((4, 8, 4), np.float32),
-                        W2=np.zeros((4, 4, 8), np.float32)),
+                        W2=np.zeros((4, 4, 8), np.float32), W1s=np.zeros((8, 4), np.float32),
+                        W2s=np.zeros((4, 8), np.float32)),
                    np.zeros((2, 4), np.float32))
 
 
@@ -305,3 +309,92 @@ def test_zloss_and_entropy_terms(router):
                 fd = (lp - lm) / (float(np.float32(v0 + h)) - float(np.float32(v0 - h)))
                 assert abs(fd - an[pos]) <= 2e-3 * (abs(an[pos]) + 0.05 * scale) + 1e-9, \
                     (router, name, pos, fd, an[pos])
+
+
+# ------------------------------------------------------------------ hierarchical layer
+GRAD_OF.update(Wg2="dWg2", bg2="dbg2", Wn2="dWn2")
+
+
+def _hier_inputs(rng, T, d, a, b, f, *, noise=True):
+    n = a * b
+    inp = _inputs(rng, T, d, a, f, noise=noise)           # the primary gate over a groups
+    inp.update(
+        Wg2=rng.normal(0, 0.7, (a, d, b)).astype(np.float32),
+        bg2=rng.normal(0, 0.3, (a, b)).astype(np.float32),
+        Wn2=rng.normal(0, 0.4, (a, d, b)).astype(np.float32) if noise else None,
+        W1=(rng.normal(0, 1, (n, f, d)) / math.sqrt(d)).astype(np.float32),
+        b1=rng.normal(0, 0.2, (n, f)).astype(np.float32),
+        W2=(rng.normal(0, 1, (n, d, f)) / math.sqrt(f)).astype(np.float32),
+        b2=rng.normal(0, 0.2, (n, d)).astype(np.float32))
+    return inp
+
+
+def _hier_cfg(T, d, a, b, f, **kw):
+    return dict(T=T, d=d, n=a * b, k=4, f=f, hier_a=a, hier_b=b, hier_k1=2, hier_k2=2, **kw)
+
+
+def test_hierarchical_noisy_with_capacity_and_passthrough():
+    """Both gate levels, the product-form load and the experts ("Outrageously
+    Large Neural Networks" reading note, 分层 MoE): every gradient against
+    central differences of the forward loss, capacity drops included."""
+    rng = np.random.default_rng(21)
+    T, d, a, b, f = 14, 5, 3, 4, 6
+    inp = _hier_inputs(rng, T, d, a, b, f)
+    cfg = _hier_cfg(T, d, a, b, f, router=0, noise=1, seed=3, capacity_factor=0.9, passthrough=1,
+                    w_importance=0.5, w_load=0.7)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+    assert (O.forward(cfg, inp)["row_of"] < 0).any()
+    g = _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "Wn", "Wg2", "bg2", "Wn2", "W1", "b1", "W2", "b2"],
+                  rng, per=8)
+    assert np.abs(g["dWn2"]).max() > 0 and np.abs(g["dbg2"]).max() > 0
+
+
+def test_hierarchical_load_loss_reaches_both_levels():
+    """dy = 0, no importance weight: the only gradient is the load loss of
+    Load(i b + j) = Load_p_i Load_i_j / |X_i|, reaching the primary gate and
+    each group's gate through Phi."""
+    rng = np.random.default_rng(22)
+    T, d, a, b, f = 12, 4, 3, 3, 4
+    inp = _hier_inputs(rng, T, d, a, b, f)
+    cfg = _hier_cfg(T, d, a, b, f, router=0, noise=1, seed=9, w_importance=0.0, w_load=1.0)
+    dy = np.zeros((T, d), np.float32)
+    g = _check_fd(cfg, inp, dy, ["x", "Wg", "bg", "Wn", "Wg2", "bg2", "Wn2"], rng, per=8)
+    assert np.abs(g["dW1"]).max() == 0
+    assert np.abs(g["dbg"]).max() > 0 and np.abs(g["dbg2"]).max() > 0
+
+
+def test_hierarchical_noise_free_and_router_statistics():
+    rng = np.random.default_rng(23)
+    T, d, a, b, f = 10, 5, 4, 3, 6
+    inp = _hier_inputs(rng, T, d, a, b, f, noise=False)
+    cfg = _hier_cfg(T, d, a, b, f, router=0, noise=0, w_importance=0.6, w_load=0.4, router_stats=1,
+                    w_z=0.05, w_entropy=0.2)
+    dy = rng.normal(0, 1, (T, d)).astype(np.float32)
+
+    def loss(cfg_, inp_, dy_):
+        out = O.forward(cfg_, inp_)
+        L = float(np.sum(dy_ * out["y"]) + sum(out["losses"][i] for i in LOSS_IDX)
+                   + cfg_["w_z"] * out["losses"][8] - cfg_["w_entropy"] * out["losses"][9])
+        return L, out
+    g = O.backward(cfg, inp, dy)
+    _, base = loss(cfg, inp, dy)
+    checked = 0
+    for name in ("x", "Wg", "bg", "Wg2", "bg2"):
+        arr = inp[name]
+        for i in rng.choice(arr.size, size=min(6, arr.size), replace=False):
+            pos = np.unravel_index(int(i), arr.shape)
+            v0 = arr[pos]
+            h = np.float32(2e-3 * max(1.0, abs(float(v0))))
+            arr[pos] = v0 + h
+            lp, op = loss(cfg, inp, dy)
+            arr[pos] = v0 - h
+            lm, om = loss(cfg, inp, dy)
+            arr[pos] = v0
+            if not all(np.array_equal(o["topk_idx"], base["topk_idx"]) for o in (op, om)):
+                continue
+            fd = (lp - lm) / (float(np.float32(v0 + h)) - float(np.float32(v0 - h)))
+            an = g[GRAD_OF[name]][pos]
+            assert abs(fd - an) <= 2e-3 * (abs(an) + 0.05 * np.abs(g[GRAD_OF[name]]).max()) + 1e-9, \
+                (name, pos, fd, an)
+            checked += 1
+    assert checked >= 20
