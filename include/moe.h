@@ -371,13 +371,17 @@ MOE_API int moe_balance_from_totals(const moe_config *cfg, const float *importan
  * expert's without a shared expert.  dgate [T][k] and dlogits [T][n] are
  * optional intermediate results: dL/d topk_gate and dL/d(x W_g + b_g). */
 typedef struct moe_grads {
-  float *dW_g, *db_g, *dW_noise;        /* [d][n], [n], [d][n] */
+  float *dW_g, *db_g, *dW_noise;        /* [d][n], [n], [d][n]; hierarchical: the primary
+                                           gate's [d][hier_a], [hier_a], [d][hier_a] */
   float *dW1, *db1, *dW2, *db2;         /* [n][f][d], [n][f], [n][d][f], [n][d] */
   float *dW1s, *db1s, *dW2s, *db2s;     /* [f][d], [f], [d][f], [d] */
-  float *dgate, *dlogits;               /* [T][k], [T][n] */
+  float *dgate, *dlogits;               /* [T][k], [T][n] (dlogits: flat layers only) */
+  float *dW_g2, *db_g2, *dW_noise2;     /* hierarchical: the secondary gates'
+                                           [hier_a][d][hier_b], [hier_a][hier_b],
+                                           [hier_a][d][hier_b] */
 } moe_grads;
 
-/* Backward pass of a flat layer.  The pages give no
+/* Backward pass of the layer (flat or hierarchical).  The pages give no
  * backward formulas; they fix which paths carry a gradient: the kept gates
  * are a smooth function of the logits ([SGMoE-xyz] "常見問題"), KeepTopK
  * gives the experts it drops none ([SGMoE-note] "缺点与局限性"), and the
@@ -400,7 +404,15 @@ typedef struct moe_grads {
  * moe_forward with the same cfg, x and parameters, whose outputs topk_idx,
  * topk_gate, importance, load and counts are passed back here; both calls
  * on the same stream, in that order.  ws is read and overwritten.
- * Errors: MOE_EINVAL for a hierarchical layer, cfg->backward != 1, NULL required pointers or misaligned ones (x, dy, dx 16-byte
+ * Hierarchical layer ([SGMoE-note] "分层 MoE"): the slot gate G_p(x)_g G_g(x)_j
+ * passes dL/dG_p = sum over its slots of dL/dslot G_g and dL/dG_g = dL/dslot
+ * G_p to the two levels; Load(g*b+j) = Load_p_g Load_g_j / |X_g| (the
+ * forward's reading, |X_g| a count) sends the load loss to both levels; each
+ * level's gate then takes the flat gate's chain rule, a secondary row with
+ * its own noise stream (gate 1 + g).  grads->dW_g, db_g, dW_noise are the
+ * primary gate's, dW_g2, db_g2, dW_noise2 the secondary gates'; dlogits is
+ * not written.  No shared expert with a hierarchical layer.
+ * Errors: MOE_EINVAL for cfg->backward != 1, a hierarchical layer with a shared expert, NULL required pointers or misaligned ones (x, dy, dx 16-byte
  * aligned); MOE_EWORKSPACE; MOE_ECUDA.  Device-side timeouts are OR-ed into
  * *status (MOE_STATUS_TIMEOUT). */
 MOE_API int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *gp,

@@ -49,7 +49,7 @@ class moe_expert_params(C.Structure):
 class moe_grads(C.Structure):
     _fields_ = [(name, C.c_void_p) for name in (
         "dW_g", "db_g", "dW_noise", "dW1", "db1", "dW2", "db2", "dW1s", "db1s", "dW2s", "db2s",
-        "dgate", "dlogits")]
+        "dgate", "dlogits", "dW_g2", "db_g2", "dW_noise2")]
 
 
 _lib = None

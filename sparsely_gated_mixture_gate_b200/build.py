@@ -15,7 +15,7 @@ LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["moe_api.cu", "gate_gemm.cu", "route.cu", "dispatch.cu", "expert_tc.cu",
            "expert_f32.cu", "combine.cu", "stats.cu", "dispatch_static.cu", "tc_common.cu", "gate_tc.cu",
            "backward.cu", "grad_gemm.cu", "wgrad_tc.cu", "fma_probe.cu", "ep.cu",
-           "gate_cutlass.cu"]
+           "gate_cutlass.cu", "backward_hier.cu"]
 HEADERS = ["internal.h", "philox.cuh", "tc_common.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",

@@ -350,12 +350,33 @@ __global__ void __launch_bounds__(256) expert_bwd_f32_kernel(
 constexpr int GW = 8;  // warps (rows) per block
 
 // one warp per token row of the flat gate
+// the row's token (noise counter), its noise stream and its load coefficients:
+// token rows use gate id 0; a secondary gate's row uses 1 + its group
+struct RowCtx {
+  uint32_t tok, gate_id;
+  const float *lam_load;
+};
+__device__ __forceinline__ RowCtx row_ctx(const GateBwdArgs &a, int t) {
+  RowCtx r{(uint32_t)(a.row_token ? a.row_token[t] : t) + a.token_base, 0u, a.lam_load};
+  if (a.seg_off) {
+    int lo = 0, hi = a.G - 1;  // largest g with seg_off[g] <= t
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (a.seg_off[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    r.gate_id = 1u + (uint32_t)lo;
+    r.lam_load = a.lam_load ? a.lam_load + (size_t)lo * a.n : nullptr;
+  }
+  return r;
+}
+
 template <int KM>
 __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
   const int t = blockIdx.x * GW + (threadIdx.x >> 5);
   if (t >= a.T) return;
   const int lane = threadIdx.x & 31;
   const int n = a.n, k = a.k;
+  const RowCtx rc = row_ctx(a, t);
   const float *crow = a.c + (size_t)t * n;
   const float *srow = a.s + (size_t)t * n;
   float *dcrow = a.dc + (size_t)t * n;
@@ -370,7 +391,9 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
     if (lane < k) {
       id = a.idx[(size_t)t * k + lane];
       gv = a.gate[(size_t)t * k + lane];
-      dv = a.dgate[(size_t)t * k + lane] + a.lam_imp[id];  // combine + importance
+      // + the importance term (an id out of range, only after non-finite
+      // logits, which the forward reports, reads nothing)
+      dv = a.dgate[(size_t)t * k + lane] + (a.lam_imp && id >= 0 && id < n ? a.lam_imp[id] : 0.f);
     }
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
@@ -471,7 +494,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
       const float sv = srow[i];
       if (thr == -INFINITY || sv == 0.f) continue;  // P constant there
       const float u = (crow[i] - thr) / sv;
-      const float av = a.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
+      const float av = rc.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
       if (kept) A_kept += av; else A_out += av;
     }
 #pragma unroll
@@ -486,7 +509,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
     float eps[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.noise) {
       const uint4 wd =
-          philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, 0u, 0u), key0, key1);
+          philox4x32_10(make_uint4(rc.tok, (uint32_t)m, rc.gate_id, 0u), key0, key1);
       box_muller2(wd.x, wd.y, eps[0], eps[1]);
       box_muller2(wd.z, wd.w, eps[2], eps[3]);
     }
@@ -507,7 +530,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_kernel(GateBwdArgs a) {
         const float thr = js >= 0 ? thr_kept : thr_out;
         if (thr != -INFINITY && sv != 0.f) {
           const float u = (crow[i] - thr) / sv;
-          const float av = a.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
+          const float av = rc.lam_load[i] * (0.3989422804014327f * expf(-0.5f * u * u)) / sv;
           dc += av;
           ds -= av * u;
         }
@@ -533,6 +556,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
   if (t >= a.T) return;
   const int lane = threadIdx.x & 31;
   const int n = a.n, k = a.k;
+  const RowCtx rc = row_ctx(a, t);
   const float4 *crow = reinterpret_cast<const float4 *>(a.c + (size_t)t * n);
   const float4 *srow = reinterpret_cast<const float4 *>(a.s + (size_t)t * n);
   float cv[NQ][4], sv[NQ][4];
@@ -555,7 +579,9 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
     if (lane < k) {
       id = a.idx[(size_t)t * k + lane];
       gv = a.gate[(size_t)t * k + lane];
-      dv = a.dgate[(size_t)t * k + lane] + a.lam_imp[id];  // combine + importance
+      // + the importance term (an id out of range, only after non-finite
+      // logits, which the forward reports, reads nothing)
+      dv = a.dgate[(size_t)t * k + lane] + (a.lam_imp && id >= 0 && id < n ? a.lam_imp[id] : 0.f);
     }
 #pragma unroll
     for (int j = 0; j < KM; ++j) {
@@ -599,7 +625,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
     const int i0 = 4 * (lane + 32 * q);
     float lam4[4] = {0.f, 0.f, 0.f, 0.f};
     if (loadg && i0 < n) {
-      const float4 l4 = __ldg(reinterpret_cast<const float4 *>(a.lam_load) + lane + 32 * q);
+      const float4 l4 = __ldg(reinterpret_cast<const float4 *>(rc.lam_load) + lane + 32 * q);
       lam4[0] = l4.x; lam4[1] = l4.y; lam4[2] = l4.z; lam4[3] = l4.w;
     }
 #pragma unroll
@@ -637,7 +663,7 @@ __global__ void __launch_bounds__(GW * 32) gate_bwd_reg_kernel(GateBwdArgs a) {
     float eps[4] = {0.f, 0.f, 0.f, 0.f};
     if (a.noise) {
       const uint4 wd =
-          philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, 0u, 0u), key0, key1);
+          philox4x32_10(make_uint4(rc.tok, (uint32_t)m, rc.gate_id, 0u), key0, key1);
       box_muller2(wd.x, wd.y, eps[0], eps[1]);
       box_muller2(wd.z, wd.w, eps[2], eps[3]);
     }

@@ -136,6 +136,8 @@ struct RouteArgs {
                            // and of the entropy of softmax(c)
   int4 *kth;               // [R] or nullptr: per row {H of the (k+1)-th ranked, its id,
                            // H of the k-th, its id} (H bits as int; -inf / INT_MAX if absent)
+  float *gate_raw;         // [R][k] or nullptr: the row's own gates (the secondary gate's,
+  int *idx_raw;            // before the primary factor) and kept ids, by row (backward)
   int *status;
 };
 int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st);
@@ -241,7 +243,27 @@ struct GateBwdArgs {
   uint32_t token_base;         // added to the token index in the noise counter
   int router, noise, has_load;
   float *dc, *dz;              // [T][n] outputs (dz: noise only)
+  // rows of a hierarchical layer's secondary gates (T = their count): the
+  // token of every row (noise counter) and the first row of every group
+  // (seg_off [G+1]: noise stream 1 + group, lam_load + group * n); both
+  // nullptr for token rows.  lam_imp may be nullptr (folded into dgate).
+  const int *row_token, *seg_off;
+  int G;
 };
+// hierarchical backward (backward_hier.cu)
+int launch_hier_coef(const float *lam_load, const float *load_p, const float *load2,
+                     const int *cnt, int a, int b, float *lam_p, float *lam_s, cudaStream_t st);
+int launch_hier_split(int T, int k1, int k2, int K, int n, const float *pgate,
+                      const int *grow, const int *topk_idx, const float *dgate,
+                      const float *gate2, const float *lam_imp, float *dgp, float *dgs,
+                      cudaStream_t st);
+int launch_hier_gate_wgrad(const float *x, int d, const int *row_token, const int *seg_off, int a,
+                           int b, const float *dc2, const float *dz2, float *dWg2, float *dWn2,
+                           float *dbg2, cudaStream_t st);
+int launch_hier_gate_dgrad(const float *dc2, const float *dz2, const float *Wg2, const float *Wn2,
+                           const int *seg_off, const int *seg_mblk, int mblk_upper, int a, int d,
+                           int b, float *dxs, int T, int k1, const int *grow, float *dx,
+                           cudaStream_t st);
 int launch_bwd_coef(const float *importance, const float *load, const int *counts, int n, int T,
                     float w_imp, float w_load, float alpha, int router, int noise, float *lam_imp,
                     float *lam_load, float *sw_coef, cudaStream_t st);

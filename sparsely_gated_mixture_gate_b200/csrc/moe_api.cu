@@ -135,7 +135,7 @@ int route_rows_per_tile(int R) {
 namespace {
 
 struct Layout {
-  size_t c, s, load_part, psum_part, prob_sum;
+  size_t c, s, c2, s2, load_part, psum_part, prob_sum;
   size_t stats_part, rstats;  // router statistics: per-tile sums, their totals
   size_t pidx, pgate, load_p, g_hist, g_base, g_counts, g_offsets, g_ucoff, g_perm_token,
       g_perm_slot, g_row_of, g_mblk, g_tiles, load2_part, load2;
@@ -148,6 +148,10 @@ struct Layout {
   size_t kth, hid_shared;
   size_t dy_perm, dhid, dx_perm, dy_shared, dhid_shared, dx_shared, dgate, lam_imp, lam_load,
       sw_coef, dc, dz, colsum_part, sgemm_part;
+  // hierarchical backward: the secondary rows' thresholds, own gates and ids,
+  // the two levels' gate gradients and load coefficients, the secondary
+  // logits' gradients, and each secondary row's part of dx
+  size_t kth2, gate2, idx2, dgp, dgs, lam_p, lam_s, dc2, dz2, dxs;
   size_t total;
   int RT1, tiles1, RT2, tiles2_upper, B;
 };
@@ -180,9 +184,12 @@ Layout make_layout(const moe_config &c) {
     L.RT2 = 0;
     L.tiles2_upper = 0;
   }
-  const size_t cs = T * ng > R2 * (size_t)c.hier_b ? T * ng : R2 * (size_t)c.hier_b;
-  L.c = bp.take(4 * cs);
-  L.s = bp.take(4 * cs);
+  // the flat / primary gate's logits; a hierarchical layer's secondary gates
+  // have their own (the backward reads both levels)
+  L.c = bp.take(4 * T * ng);
+  L.s = bp.take(4 * T * ng);
+  L.c2 = hier ? bp.take(4 * R2 * (size_t)c.hier_b) : 0;
+  L.s2 = hier ? bp.take(4 * R2 * (size_t)c.hier_b) : 0;
   const size_t lp1 = (size_t)L.tiles1 * ng, lp2 = (size_t)L.tiles2_upper * (size_t)c.hier_b;
   L.load_part = bp.take(4 * (lp1 > lp2 ? lp1 : lp2));
   L.psum_part = bp.take(c.router == MOE_ROUTER_SWITCH ? 4 * (size_t)L.tiles1 * n : 0);
@@ -259,6 +266,7 @@ Layout make_layout(const moe_config &c) {
   L.kth = L.hid_shared = L.dy_perm = L.dhid = L.dx_perm = L.dy_shared = L.dhid_shared =
       L.dx_shared = L.dgate = L.lam_imp = L.lam_load = L.sw_coef = L.dc = L.dz = L.colsum_part =
           L.sgemm_part = 0;
+  L.kth2 = L.gate2 = L.idx2 = L.dgp = L.dgs = L.lam_p = L.lam_s = L.dc2 = L.dz2 = L.dxs = 0;
   if (c.backward) {
     L.kth = bp.take(16 * T);
     L.hid_shared = bp.take(c.shared_expert ? esz * T * (size_t)c.f : 0);
@@ -274,12 +282,26 @@ Layout make_layout(const moe_config &c) {
     L.lam_imp = bp.take(4 * n);
     L.lam_load = bp.take(4 * n);
     L.sw_coef = bp.take(4 * n);
-    L.dc = bp.take(4 * T * n);
-    L.dz = bp.take(c.noise ? 4 * T * n : 0);
-    L.colsum_part = bp.take(4 * (size_t)colsum_parts(c.T, c.n) * n);
+    L.dc = bp.take(4 * T * ng);
+    L.dz = bp.take(c.noise ? 4 * T * ng : 0);
+    L.colsum_part = bp.take(4 * (size_t)colsum_parts(c.T, (int)ng) * ng);
     const size_t np = c.noise ? 2 : 1;  // dW_g, and dW_noise beside it
-    const size_t sp = (size_t)sgemm_splits(c.d, c.n, c.T, (int)np);
-    L.sgemm_part = bp.take(sp > 1 ? 4 * np * sp * (size_t)c.d * n : 0);
+    const size_t sp = (size_t)sgemm_splits(c.d, (int)ng, c.T, (int)np);
+    L.sgemm_part = bp.take(sp > 1 ? 4 * np * sp * (size_t)c.d * ng : 0);
+    if (hier) {
+      const size_t a = (size_t)c.hier_a, b = (size_t)c.hier_b;
+      const size_t k1 = (size_t)c.hier_k1, k2 = (size_t)c.hier_k2;
+      L.kth2 = bp.take(16 * R2);
+      L.gate2 = bp.take(4 * R2 * k2);
+      L.idx2 = bp.take(4 * R2 * k2);
+      L.dgp = bp.take(4 * T * k1);
+      L.dgs = bp.take(4 * R2 * k2);
+      L.lam_p = bp.take(4 * a);
+      L.lam_s = bp.take(4 * a * b);
+      L.dc2 = bp.take(4 * R2 * b);
+      L.dz2 = bp.take(c.noise ? 4 * R2 * b : 0);
+      L.dxs = bp.take(4 * R2 * (size_t)c.d);
+    }
   }
   L.total = bp.off;
   return L;
@@ -388,7 +410,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.load_part = at<float>(ws, L.load_part);
   r.sel_bias = (!hier && c.router == MOE_ROUTER_SIGMOID) ? gp.sel_bias : nullptr;
   r.stats_part = c.router_stats ? at<float>(ws, L.stats_part) : nullptr;  // flat / primary rows
-  r.kth = (c.backward && !hier) ? at<int4>(ws, L.kth) : nullptr;
+  r.kth = c.backward ? at<int4>(ws, L.kth) : nullptr;  // flat / primary rows
   r.status = status;
   if (!hier) {
     r.k = c.k;
@@ -454,6 +476,8 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   // ---- secondary gates: grouped fp32 GEMM over each group's tokens
   const int R2 = c.T * k1;
   GateGemmArgs g2 = g;
+  g2.c = at<float>(ws, L.c2);
+  g2.s = at<float>(ws, L.s2);
   g2.row_token = da.perm_token;
   g2.seg_off = da.offsets;
   g2.seg_mblk = da.seg_mblk;
@@ -467,6 +491,11 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
 
   RouteArgs r2 = r;
   r2.stats_part = nullptr;  // the statistics cover the primary gate only
+  r2.c = g2.c;
+  r2.s = g2.s;
+  r2.kth = c.backward ? at<int4>(ws, L.kth2) : nullptr;
+  r2.gate_raw = c.backward ? at<float>(ws, L.gate2) : nullptr;
+  r2.idx_raw = c.backward ? at<int>(ws, L.idx2) : nullptr;
   r2.R = R2;
   r2.nb = b;
   r2.k = k2;
@@ -817,7 +846,8 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   Layout L;
   MOE_TRY(common_checks(cfg, ws, ws_bytes, status, &L));
   const moe_config &c = *cfg;
-  if (!c.backward || c.hier_a > 0) return MOE_EINVAL;
+  const bool hier = c.hier_a > 0;
+  if (!c.backward || (hier && c.shared_expert)) return MOE_EINVAL;
   if (!gr || !gr->dW1 || !gr->dW2 || !importance || !load || !counts) return MOE_EINVAL;
   if (!aligned(gr->dW1, 16) || !aligned(gr->dW2, 16)) return MOE_EINVAL;
   if (c.T > 0 && (!x || !dy || !dx || !topk_idx || !topk_gate || !aligned(x, 16) ||
@@ -830,15 +860,22 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
     return MOE_EINVAL;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   const int T = c.T, d = c.d, n = c.n, k = c.k, f = c.f;
+  const int ng = hier ? c.hier_a : n;  // width of the flat / primary gate
   const size_t S = (size_t)T * k;
   auto zero = [&](float *p, size_t cnt) -> int {
     if (!p || cnt == 0) return MOE_OK;
     return cudaMemsetAsync(p, 0, 4 * cnt, st) == cudaSuccess ? MOE_OK : MOE_ECUDA;
   };
   if (T == 0) {  // no tokens: every gradient is zero
-    MOE_TRY(zero(gr->dW_g, (size_t)d * n));
-    MOE_TRY(zero(gr->db_g, n));
-    if (c.noise) MOE_TRY(zero(gr->dW_noise, (size_t)d * n));
+    MOE_TRY(zero(gr->dW_g, (size_t)d * ng));
+    MOE_TRY(zero(gr->db_g, ng));
+    if (c.noise) MOE_TRY(zero(gr->dW_noise, (size_t)d * ng));
+    if (hier) {
+      const size_t ab = (size_t)c.hier_a * c.hier_b;
+      MOE_TRY(zero(gr->dW_g2, ab * d));
+      MOE_TRY(zero(gr->db_g2, ab));
+      if (c.noise) MOE_TRY(zero(gr->dW_noise2, ab * d));
+    }
     MOE_TRY(zero(gr->dW1, (size_t)n * f * d));
     MOE_TRY(zero(gr->db1, (size_t)n * f));
     MOE_TRY(zero(gr->dW2, (size_t)n * d * f));
@@ -966,10 +1003,10 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   // ---- dispatch: dx = sum of the token's expert rows (+ pass-through, + shared)
   MOE_TRY(launch_dx_gather(dx_perm, tc, row_of, dy, c.overflow_passthrough, T, k, d, dx_sh, dx,
                            st));
-  // ---- gate: dL/dc, dL/dz per token, then the fp32 contractions
+  // ---- gate: dL/dc, dL/dz per row, then the fp32 contractions
   GateBwdArgs g{};
   g.T = T;
-  g.n = n;
+  g.n = ng;
   g.k = k;
   g.c = at<float>(ws, L.c);
   g.s = at<float>(ws, L.s);
@@ -989,20 +1026,60 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
   g.dc = dc;
   g.dz = dz;
   MOE_TRY(stream_after(st, side->s, side->join));  // the loss coefficients
-  MOE_TRY(launch_gate_bwd(g, st));
+  if (hier) {
+    // [SGMoE-note] "分层 MoE": the slot gradients split into the two levels,
+    // the load coefficients too, then each level is a flat gate's backward
+    const int a = c.hier_a, b = c.hier_b, k1 = c.hier_k1, k2 = c.hier_k2, R2 = T * k1;
+    float *lam_p = at<float>(ws, L.lam_p), *lam_s = at<float>(ws, L.lam_s);
+    float *dgp = at<float>(ws, L.dgp), *dgs = at<float>(ws, L.dgs);
+    const int *grow = at<int>(ws, L.g_row_of);
+    if (g.has_load)
+      MOE_TRY(launch_hier_coef(lam_load, at<float>(ws, L.load_p), at<float>(ws, L.load2),
+                               at<int>(ws, L.g_counts), a, b, lam_p, lam_s, st));
+    MOE_TRY(launch_hier_split(T, k1, k2, k, n, at<float>(ws, L.pgate), grow,
+                              topk_idx, dgate, at<float>(ws, L.gate2), lam_imp, dgp, dgs, st));
+    g.k = k1;  // the primary gate over the groups
+    g.idx = at<int>(ws, L.pidx);
+    g.gate = at<float>(ws, L.pgate);
+    g.dgate = dgp;
+    g.lam_imp = nullptr;  // folded into dgp
+    g.lam_load = lam_p;
+    MOE_TRY(launch_gate_bwd(g, st));
+    GateBwdArgs g2 = g;  // the secondary gates, one row per (token, kept group)
+    g2.T = R2;
+    g2.n = b;
+    g2.k = k2;
+    g2.c = at<float>(ws, L.c2);
+    g2.s = at<float>(ws, L.s2);
+    g2.idx = at<int>(ws, L.idx2);
+    g2.gate = at<float>(ws, L.gate2);
+    g2.dgate = dgs;
+    g2.lam_load = lam_s;
+    g2.kth = at<int4>(ws, L.kth2);
+    g2.row_token = at<int>(ws, L.g_perm_token);
+    g2.seg_off = at<int>(ws, L.g_offsets);
+    g2.G = a;
+    g2.dc = at<float>(ws, L.dc2);
+    g2.dz = c.noise ? at<float>(ws, L.dz2) : nullptr;
+    MOE_TRY(launch_gate_bwd(g2, st));
+    MOE_TRY(launch_hier_gate_wgrad(x, d, g2.row_token, g2.seg_off, a, b, g2.dc, g2.dz, gr->dW_g2,
+                                   c.noise ? gr->dW_noise2 : nullptr, gr->db_g2, st));
+  } else {
+    MOE_TRY(launch_gate_bwd(g, st));
+  }
   if (c.w_z != 0.f || c.w_entropy != 0.f)  // router z-loss and gate entropy terms
-    MOE_TRY(launch_gate_stats_bwd(at<float>(ws, L.c), T, n, c.w_z, c.w_entropy, dc, st));
-  if (gr->db_g) MOE_TRY(launch_colsum(dc, T, n, at<float>(ws, L.colsum_part), gr->db_g, st));
+    MOE_TRY(launch_gate_stats_bwd(at<float>(ws, L.c), T, ng, c.w_z, c.w_entropy, dc, st));
+  if (gr->db_g) MOE_TRY(launch_colsum(dc, T, ng, at<float>(ws, L.colsum_part), gr->db_g, st));
   float *sp = at<float>(ws, L.sgemm_part);
   const bool want_n = c.noise && gr->dW_noise;
   // the split count the workspace was sized for (two problems with noise)
-  const int splits = sgemm_splits(d, n, T, c.noise ? 2 : 1);
+  const int splits = sgemm_splits(d, ng, T, c.noise ? 2 : 1);
   if (gr->dW_g || want_n) {
-    // dW_g = x^T dc and dW_noise = x^T dz: M = d, N = n, K = T, A shared
+    // dW_g = x^T dc and dW_noise = x^T dz: M = d, N = ng, K = T, A shared
     SgemmArgs a{};
-    a.M = d; a.N = n; a.K = T;
+    a.M = d; a.N = ng; a.K = T;
     a.A[0] = a.A[1] = x; a.lda = d; a.at = 1;
-    a.ldb = n; a.bt = 0; a.ldc = n;
+    a.ldb = ng; a.bt = 0; a.ldc = ng;
     if (gr->dW_g && want_n) {
       a.B[0] = dc; a.C[0] = gr->dW_g;
       a.B[1] = dz; a.C[1] = gr->dW_noise;
@@ -1018,11 +1095,11 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
     MOE_TRY(launch_sgemm(a, st));
   }
   {
-    // dx += dc W_g^T (+ dz W_noise^T): M = T, N = d, K = n; B(k, q) = W[q][k]
+    // dx += dc W_g^T (+ dz W_noise^T): M = T, N = d, K = ng; B(k, q) = W[q][k]
     SgemmArgs a{};
-    a.M = T; a.N = d; a.K = n;
-    a.A[0] = dc; a.A[1] = dz; a.lda = n; a.at = 0;
-    a.B[0] = gp->W_g; a.B[1] = gp->W_noise; a.ldb = n; a.bt = 1;
+    a.M = T; a.N = d; a.K = ng;
+    a.A[0] = dc; a.A[1] = dz; a.lda = ng; a.at = 0;
+    a.B[0] = gp->W_g; a.B[1] = gp->W_noise; a.ldb = ng; a.bt = 1;
     a.C[0] = a.C[1] = dx; a.ldc = d;
     a.nprob = 1;
     a.ksum = c.noise ? 1 : 0;
@@ -1031,11 +1108,18 @@ int moe_backward(const moe_config *cfg, const float *x, const moe_gate_params *g
     a.name = "gate_dgrad_fp32";
     MOE_TRY(launch_sgemm(a, st));
   }
+  if (hier) {  // dx += the secondary gates' part, row by row, then per token in order
+    const int a = c.hier_a, b = c.hier_b, k1 = c.hier_k1, R2 = T * k1;
+    MOE_TRY(launch_hier_gate_dgrad(at<float>(ws, L.dc2), c.noise ? at<float>(ws, L.dz2) : nullptr,
+                                   gp->W_g2, gp->W_noise2, at<int>(ws, L.g_offsets),
+                                   at<int>(ws, L.g_mblk), (int)ceil_div(R2, kGateBM) + a, a, d, b,
+                                   at<float>(ws, L.dxs), T, k1, at<int>(ws, L.g_row_of), dx, st));
+  }
   if (gr->dgate &&
       cudaMemcpyAsync(gr->dgate, dgate, 4 * S, cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ECUDA;
-  if (gr->dlogits && cudaMemcpyAsync(gr->dlogits, dc, 4 * (size_t)T * n,
-                                     cudaMemcpyDeviceToDevice, st) != cudaSuccess)
+  if (!hier && gr->dlogits && cudaMemcpyAsync(gr->dlogits, dc, 4 * (size_t)T * n,
+                                              cudaMemcpyDeviceToDevice, st) != cudaSuccess)
     return MOE_ECUDA;
   return MOE_OK;
 }

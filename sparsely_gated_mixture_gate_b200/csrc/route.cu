@@ -249,6 +249,10 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
             gate_j = sw ? expf(crow[S[0].i] - M) / SE : expf(S[j].v - S[0].v) / den;
           }
       }
+      if (EX && a.gate_raw && lane < k) {  // kept for the backward pass, by row
+        a.gate_raw[(size_t)row * k + lane] = gate_j;
+        a.idx_raw[(size_t)row * k + lane] = idx_j;
+      }
       if (lane < k) {
         int slot = lane;
         float gmul = 1.f;
@@ -465,7 +469,7 @@ int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st) {
     return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), 0, st, a);
   };
   const bool wide = a.nb > 4 * 4 * NW * 32;  // more than 4096 columns
-  const bool st_on = a.stats_part != nullptr || a.kth != nullptr;  // the EX instances
+  const bool st_on = a.stats_part != nullptr || a.kth != nullptr || a.gate_raw != nullptr;
   if (a.router == MOE_ROUTER_SWITCH) {
     if (a.k != 1 || wide) return MOE_EINVAL;
     return st_on ? go(route_kernel<2, 4, true, true>) : go(route_kernel<2, 4, true, false>);

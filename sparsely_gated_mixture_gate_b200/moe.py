@@ -435,26 +435,35 @@ class MoELayer:
 
     def grads(self, intermediates: bool = False) -> dict:
         """Gradient buffers of this layer (allocated on first use), fp32 in
-        the parameters' layouts; with intermediates also dgate [T][k] and
-        dlogits [T][n]."""
+        the parameters' layouts; with intermediates also dgate [T][k] and,
+        for a flat layer, dlogits [T][n].  A hierarchical layer's dWg, dbg, dWn
+        are the primary gate's, dWg2, dbg2, dWn2 the secondary gates'."""
         if not hasattr(self, "_grads"):
             cfg, dev = self.cfg, self.device
             z = lambda *shape: torch.zeros(*shape, dtype=torch.float32, device=dev)
-            g = dict(dx=z(cfg.T, cfg.d), dWg=z(cfg.d, cfg.n), dbg=z(cfg.n),
+            gn = cfg.hier_a if cfg.hier_a else cfg.n
+            g = dict(dx=z(cfg.T, cfg.d), dWg=z(cfg.d, gn), dbg=z(gn),
                      dW1=z(cfg.n, cfg.f, cfg.d), db1=z(cfg.n, cfg.f), dW2=z(cfg.n, cfg.d, cfg.f),
                      db2=z(cfg.n, cfg.d))
             if cfg.noise:
-                g["dWn"] = z(cfg.d, cfg.n)
+                g["dWn"] = z(cfg.d, gn)
+            if cfg.hier_a:
+                g.update(dWg2=z(cfg.hier_a, cfg.d, cfg.hier_b), dbg2=z(cfg.hier_a, cfg.hier_b))
+                if cfg.noise:
+                    g["dWn2"] = z(cfg.hier_a, cfg.d, cfg.hier_b)
             if cfg.shared_expert:
                 g.update(dW1s=z(cfg.f, cfg.d), db1s=z(cfg.f), dW2s=z(cfg.d, cfg.f), db2s=z(cfg.d))
             if intermediates:
-                g.update(dgate=z(cfg.T, cfg.k), dlogits=z(cfg.T, cfg.n))
+                g["dgate"] = z(cfg.T, cfg.k)
+                if not cfg.hier_a:
+                    g["dlogits"] = z(cfg.T, cfg.n)
             self._grads = g
             self._mg = _lib.moe_grads(
                 dW_g=_ptr(g["dWg"]), db_g=_ptr(g["dbg"]), dW_noise=_ptr(g.get("dWn")),
                 dW1=_ptr(g["dW1"]), db1=_ptr(g["db1"]), dW2=_ptr(g["dW2"]), db2=_ptr(g["db2"]),
                 dW1s=_ptr(g.get("dW1s")), db1s=_ptr(g.get("db1s")), dW2s=_ptr(g.get("dW2s")),
-                db2s=_ptr(g.get("db2s")), dgate=_ptr(g.get("dgate")), dlogits=_ptr(g.get("dlogits")))
+                db2s=_ptr(g.get("db2s")), dgate=_ptr(g.get("dgate")), dlogits=_ptr(g.get("dlogits")),
+                dW_g2=_ptr(g.get("dWg2")), db_g2=_ptr(g.get("dbg2")), dW_noise2=_ptr(g.get("dWn2")))
         return self._grads
 
     def backward_(self, x: torch.Tensor, dy: torch.Tensor, stream=None,

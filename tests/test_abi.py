@@ -45,11 +45,11 @@ def test_struct_layout_matches_c(tmp_path):
 #include <stddef.h>
 #include "{HEADER}"
 int main(void) {{
-  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config), offsetof(moe_config, seed),
+  printf("%zu %zu %zu %zu %zu %zu %zu %zu %zu %zu %zu\\n", sizeof(moe_config), offsetof(moe_config, seed),
          offsetof(moe_config, capacity_factor), offsetof(moe_config, gate_precision),
          sizeof(moe_gate_params), sizeof(moe_expert_params),
          offsetof(moe_config, alpha_aux), offsetof(moe_config, token_base),
-         offsetof(moe_gate_params, seed_dev));
+         offsetof(moe_gate_params, seed_dev), sizeof(moe_grads), offsetof(moe_grads, dW_g2));
   return 0;
 }}
 ''')
@@ -60,7 +60,8 @@ int main(void) {{
             _lib.moe_config.capacity_factor.offset, _lib.moe_config.gate_precision.offset,
             C.sizeof(_lib.moe_gate_params), C.sizeof(_lib.moe_expert_params),
             _lib.moe_config.alpha_aux.offset, _lib.moe_config.token_base.offset,
-            _lib.moe_gate_params.seed_dev.offset]
+            _lib.moe_gate_params.seed_dev.offset, C.sizeof(_lib.moe_grads),
+            _lib.moe_grads.dW_g2.offset]
     assert vals == want
 
 

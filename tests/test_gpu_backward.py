@@ -86,11 +86,23 @@ CASES = {
     "f32-capacity": W["tiny-flat"].with_(T=200, n=6, k=2, d=40, f=24, capacity_factor=0.7,
                                          passthrough=1, bias_var=0.1, **LOSSES),
     "f32-sigmoid-shared": V["deepseek-tiny-f32"].with_(w_importance=0.3),
+    # the hierarchical layer: both gate levels, the product-form load
+    "hier-noisy": W["hierarchical"].with_(T=256, d=64, n=8 * 16, hier_a=8, hier_b=16, f=64,
+                                          **LOSSES),
+    "hier-capacity-ragged": W["hierarchical"].with_(T=300, d=40, n=4 * 8, hier_a=4, hier_b=8, f=24,
+                                                    capacity_factor=1.0, passthrough=1,
+                                                    logit_bias_var=0.2, **LOSSES),
+    "hier-nonoise-zloss": W["hierarchical"].with_(T=200, d=64, n=8 * 16, hier_a=8, hier_b=16, f=64,
+                                                  noise=0, router_stats=1, w_z=0.5, w_entropy=0.8,
+                                                  **LOSSES),
+    "hier-f32": W["hierarchical"].with_(T=64, d=32, n=4 * 4, hier_a=4, hier_b=4, f=32,
+                                        expert_bf16=0, **LOSSES),
 }
 
 GRAD_KEYS = [("dx", "dx"), ("dWg", "dWg"), ("dbg", "dbg"), ("dWn", "dWn"), ("dW1", "dW1"),
              ("db1", "db1"), ("dW2", "dW2"), ("db2", "db2"), ("dW1s", "dW1s"), ("db1s", "db1s"),
-             ("dW2s", "dW2s"), ("db2s", "db2s"), ("dlogits", "dlogits")]
+             ("dW2s", "dW2s"), ("db2s", "db2s"), ("dlogits", "dlogits"), ("dWg2", "dWg2"),
+             ("dbg2", "dbg2"), ("dWn2", "dWn2")]
 
 
 def run_backward(w, inp, dy):

@@ -211,7 +211,7 @@ def _guard_layer(layer, cfg):
 def test_forward_and_backward_stay_inside_their_buffers(name):
     w = GUARD_CASES[name]
     inp = {k: (v.to(DEV) if v is not None else None) for k, v in synth.make_inputs(w).items()}
-    backward = not w.hier_a  # the backward pass covers flat layers
+    backward = True
     cfg = dataclasses.replace(M.Config.from_workload(w), backward=int(backward))
     plain = M.MoELayer(cfg, inp, torch.device(DEV))
     plain.forward_(inp["x"])
@@ -231,7 +231,8 @@ def test_forward_and_backward_stay_inside_their_buffers(name):
     layer._mg = _lib.moe_grads(
         dW_g=_p(gg["dWg"]), db_g=_p(gg["dbg"]), dW_noise=_p(gg.get("dWn")), dW1=_p(gg["dW1"]),
         db1=_p(gg["db1"]), dW2=_p(gg["dW2"]), db2=_p(gg["db2"]), dW1s=_p(gg.get("dW1s")),
-        db1s=_p(gg.get("db1s")), dW2s=_p(gg.get("dW2s")), db2s=_p(gg.get("db2s")))
+        db1s=_p(gg.get("db1s")), dW2s=_p(gg.get("dW2s")), db2s=_p(gg.get("db2s")),
+        dW_g2=_p(gg.get("dWg2")), db_g2=_p(gg.get("dbg2")), dW_noise2=_p(gg.get("dWn2")))
     layer.backward_(inp["x"], dy)
     _check(G)
     _check(grads)
