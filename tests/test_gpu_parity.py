@@ -514,3 +514,25 @@ def test_shard_with_token_base_draws_the_batch_noise(name):
     other = M.gate(M.Config.from_workload(w.with_(T=w.T - h)), x[h:].contiguous(), inp)
     torch.cuda.synchronize()
     assert not torch.equal(other["topk_gate"], whole["topk_gate"][h:])
+
+
+def test_wide_gate_paths_route_alike():
+    """Flat gates of 2048 or more columns take the CUTLASS SIMT mainloop,
+    narrower ones the library's own SIMT kernel; both compute each logit as
+    the same fp32 FMA chain over d in order with the same epilogue rounding.
+    Run the same 2044 experts through both: at 2048 columns the four extra
+    experts carry a bias of -1e30 (never kept, never a threshold), so the
+    routing, the gates and the smoothed Load of the 2044 must agree exactly."""
+    w = W["many-expert"].with_(T=1000, d=256, n=2048, k=4)
+    inp = to_dev(synth.make_inputs(w, experts=False))
+    inp["bg"][2044:] = -1e30
+    narrow = {k: (v[..., :2044].contiguous() if k in ("Wg", "Wn", "bg") else v)
+              for k, v in inp.items()}
+    wide = M.gate(M.Config.from_workload(w), inp["x"], inp)
+    own = M.gate(M.Config.from_workload(w.with_(n=2044)), inp["x"], narrow)
+    torch.cuda.synchronize()
+    assert M.status_bits(wide["status"]) == 0 and M.status_bits(own["status"]) == 0
+    assert int(wide["topk_idx"].max()) < 2044
+    assert torch.equal(wide["topk_idx"], own["topk_idx"])
+    assert torch.equal(wide["topk_gate"], own["topk_gate"])
+    assert torch.equal(wide["load"][:2044], own["load"])
