@@ -16,7 +16,7 @@ SOURCES = ["moe_api.cu", "gate_gemm.cu", "route.cu", "dispatch.cu", "expert_tc.c
            "expert_f32.cu", "combine.cu", "stats.cu", "dispatch_static.cu", "tc_common.cu", "gate_tc.cu",
            "backward.cu", "grad_gemm.cu", "wgrad_tc.cu", "fma_probe.cu", "ep.cu",
            "gate_cutlass.cu", "backward_hier.cu"]
-HEADERS = ["internal.h", "philox.cuh", "tc_common.cuh"]
+HEADERS = ["internal.h", "philox.cuh", "tc_common.cuh", "route_common.cuh", "phi.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr"]

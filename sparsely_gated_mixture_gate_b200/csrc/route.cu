@@ -13,9 +13,16 @@
 //   Router statistics ([MoE-intro] 第三部分, optional): per row |c|^2 and the
 //   entropy of softmax(c), summed over the tile's rows in a fixed order.
 // Pass 1, one warp per row: each lane scans column quads 4m .. 4m+3 (16-byte
-// loads, one Philox call per quad), keeps a sorted top-(k+1) list in
-// registers, and the warp merges the 32 lists with shuffles; the row's kept
-// ids and its two thresholds go to shared memory.  Pass 2, one thread per
+// loads, one Philox call per quad) and keeps a sorted list of its k + 1 best
+// columns (ranked by H, then the lower column index); the warp merges the 32
+// lists with shuffles.  Rows of 512 columns or more rank quads instead, by
+// their largest H (then the lower quad index), which inserts a quarter as
+// often: the top k + 1 columns lie in the k + 1 best quads (a quad ranked
+// before the quad of a top column holds a column ranked before that column,
+// and there are fewer than k + 1 of those), so the warp evaluates the 4 (k +
+// 1) columns of those quads again (the same arithmetic, bitwise the same H)
+// and merges them into the row's top k + 1.  The row's kept ids and its two
+// thresholds go to shared memory.  Pass 2, one thread per
 // column quad: the thread walks the tile's rows in order and sums P (and the
 // Switch probabilities) in registers, then writes the tile's column sums;
 // route_reduce adds the tiles in a fixed order, so the load is bitwise
@@ -24,34 +31,82 @@
 #include <limits.h>
 
 #include "internal.h"
+#include "phi.cuh"
 #include "philox.cuh"
+#include "route_common.cuh"
 
 namespace moe {
 namespace {
 
 constexpr int NW = 8;  // warps per routing block
 
-struct Cand {
-  float v;
-  int i;
-};
-
-// a ranks before b: larger value first, equal values -> lower index first.
-// NaN never ranks before anything.
-__device__ __forceinline__ bool before(float av, int ai, float bv, int bi) {
-  return av > bv || (av == bv && ai < bi);
+// H of the columns of quad m (4m .. 4m+3) of a row: c, plus the selection
+// bias (sigmoid router) or eps * s (noise on); columns past nb get c = -inf.
+__device__ __forceinline__ void quad_h(const RouteArgs &a, const float *crow, const float *srow,
+                                       int m, int nb, bool vec4, uint32_t ctr0, uint32_t gate_id,
+                                       uint32_t key0, uint32_t key1, float (&cv)[4],
+                                       float (&sv)[4], float (&h)[4]) {
+  const int i0 = 4 * m;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) sv[j] = 0.f;
+  if (vec4) {
+    const float4 c4 = *reinterpret_cast<const float4 *>(crow + i0);
+    cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
+    if (a.noise) {
+      const float4 s4 = *reinterpret_cast<const float4 *>(srow + i0);
+      sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      cv[j] = i0 + j < nb ? crow[i0 + j] : -INFINITY;
+      if (a.noise) sv[j] = i0 + j < nb ? srow[i0 + j] : 0.f;
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j) h[j] = cv[j];
+  if (a.sel_bias) {  // sigmoid router: the bias enters the routing score only
+    float bv[4];
+    if (vec4) {
+      const float4 b4 = *reinterpret_cast<const float4 *>(a.sel_bias + i0);
+      bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
+    } else {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) bv[j] = i0 + j < nb ? a.sel_bias[i0 + j] : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = cv[j] + bv[j];
+  } else if (a.noise) {
+    const uint4 wd = philox4x32_10(make_uint4(ctr0, (uint32_t)m, gate_id, 0u), key0, key1);
+    float z[4];
+    box_muller2(wd.x, wd.y, z[0], z[1]);
+    box_muller2(wd.z, wd.w, z[2], z[3]);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) h[j] = fmaf(z[j], sv[j], cv[j]);
+  }
 }
 
-template <int K1>
-__device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
-  if (!before(v, i, L[K1 - 1].v, L[K1 - 1].i)) return;
+// K1 rounds of a warp-wide arg-max over the heads of the lanes' sorted lists;
+// the owner pops its head.  S gets the warp's K1 first entries, in order.
+template <int K1, int LN>
+__device__ __forceinline__ void warp_merge(Cand (&L)[LN], Cand (&S)[K1]) {
 #pragma unroll
-  for (int j = K1 - 1; j >= 0; --j) {
-    const bool gt = before(v, i, L[j].v, L[j].i);
-    const bool gt_prev = (j > 0) ? before(v, i, L[j - 1].v, L[j - 1].i) : false;
-    if (gt) {
-      if (gt_prev) L[j] = L[j - 1];
-      else { L[j].v = v; L[j].i = i; }
+  for (int r = 0; r < K1; ++r) {
+    float bv = L[0].v;
+    int bi = L[0].i;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+    }
+    S[r].v = bv;
+    S[r].i = bi;
+    if (L[0].i == bi && bi != INT_MAX) {
+#pragma unroll
+      for (int j = 0; j < LN - 1; ++j) L[j] = L[j + 1];
+      L[LN - 1].v = -INFINITY;
+      L[LN - 1].i = INT_MAX;
     }
   }
 }
@@ -62,7 +117,7 @@ __device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
 // rows' thresholds for the backward pass (kth), each only when its pointer is
 // set.
 template <int K1, int MAXQ, bool SW, bool EX>
-__global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
+__global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kernel(RouteArgs a) {
   constexpr int KM = K1 - 1;  // k
   constexpr int PQ = SW ? MAXQ : 1;
   __shared__ uint32_t kept_s[NW][MAXQ * NW * 32 * 4 / 32];  // kept columns of each row, one bit each
@@ -133,77 +188,53 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
       for (int j = 0; j < K1; ++j) { L[j].v = -INFINITY; L[j].i = INT_MAX; }
       float mx = -INFINITY, se = 0.f;  // online softmax of c (Switch)
 
+      const uint32_t ctr0 = (uint32_t)t + a.token_base;
+      const bool by_quad = nb >= 512;  // at least four quads per lane
       for (int m = lane; 4 * m < nb; m += 32) {
         const int i0 = 4 * m;
-        float cv[4], sv[4] = {0.f, 0.f, 0.f, 0.f};
-        if (vec4) {
-          const float4 c4 = *reinterpret_cast<const float4 *>(crow + i0);
-          cv[0] = c4.x; cv[1] = c4.y; cv[2] = c4.z; cv[3] = c4.w;
-          if (a.noise) {
-            const float4 s4 = *reinterpret_cast<const float4 *>(srow + i0);
-            sv[0] = s4.x; sv[1] = s4.y; sv[2] = s4.z; sv[3] = s4.w;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            cv[j] = i0 + j < nb ? crow[i0 + j] : -INFINITY;
-            if (a.noise) sv[j] = i0 + j < nb ? srow[i0 + j] : 0.f;
-          }
-        }
-        float h[4] = {cv[0], cv[1], cv[2], cv[3]};
-        if (a.sel_bias) {  // sigmoid router: the bias enters the routing score only
-          float bv[4];
-          if (vec4) {
-            const float4 b4 = *reinterpret_cast<const float4 *>(a.sel_bias + i0);
-            bv[0] = b4.x; bv[1] = b4.y; bv[2] = b4.z; bv[3] = b4.w;
-          } else {
-#pragma unroll
-            for (int j = 0; j < 4; ++j) bv[j] = i0 + j < nb ? a.sel_bias[i0 + j] : 0.f;
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) h[j] = cv[j] + bv[j];
-        } else if (a.noise) {
-          const uint4 wd =
-              philox4x32_10(make_uint4((uint32_t)t + a.token_base, (uint32_t)m, gate_id, 0u), key0, key1);
-          float z[4];
-          box_muller2(wd.x, wd.y, z[0], z[1]);
-          box_muller2(wd.z, wd.w, z[2], z[3]);
-#pragma unroll
-          for (int j = 0; j < 4; ++j) h[j] = fmaf(z[j], sv[j], cv[j]);
-        }
+        float cv[4], sv[4], h[4];
+        quad_h(a, crow, srow, m, nb, vec4, ctr0, gate_id, key0, key1, cv, sv, h);
+        float qm = -INFINITY;  // the quad's largest H (NaN never ranks)
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           if (i0 + j >= nb) break;
           bad |= !isfinite(h[j]);
-          insert<K1>(L, h[j], i0 + j);
+          if (by_quad) qm = fmaxf(qm, h[j]);
+          else insert<K1>(L, h[j], i0 + j);
           if (sw) {
             const float m2 = fmaxf(mx, cv[j]);
             se = se * expf(mx - m2) + expf(cv[j] - m2);
             mx = m2;
           }
         }
+        if (by_quad) insert<K1>(L, qm, m);
       }
 
-      // warp merge: K1 rounds of a warp-wide arg-max with the same order
+      // the row's k + 1 best quads, then their columns again: each lane holds
+      // (at most) two of the 4 (k + 1) columns, and the warp merges them
       Cand S[K1];
+      if (!by_quad) {
+        warp_merge<K1, K1>(L, S);
+      } else {
+      Cand Q[K1];
+      warp_merge<K1, K1>(L, Q);
+      Cand C2[2];
 #pragma unroll
-      for (int r = 0; r < K1; ++r) {
-        float bv = L[0].v;
-        int bi = L[0].i;
+      for (int j = 0; j < 2; ++j) { C2[j].v = -INFINITY; C2[j].i = INT_MAX; }
 #pragma unroll
-        for (int off = 16; off > 0; off >>= 1) {
-          const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
-          const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-          if (before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
+      for (int l0 = 0; l0 < 4 * K1; l0 += 32) {
+        const int l = l0 + lane, r = l >> 2, q = l & 3;
+        int m = INT_MAX;
+#pragma unroll
+        for (int rr = 0; rr < K1; ++rr)
+          if (rr == r) m = Q[rr].i;
+        if (l < 4 * K1 && m != INT_MAX && 4 * m + q < nb) {
+          float cv[4], sv[4], h[4];
+          quad_h(a, crow, srow, m, nb, vec4, ctr0, gate_id, key0, key1, cv, sv, h);
+          insert<2>(C2, q == 0 ? h[0] : q == 1 ? h[1] : q == 2 ? h[2] : h[3], 4 * m + q);
         }
-        S[r].v = bv;
-        S[r].i = bi;
-        if (L[0].i == bi && bi != INT_MAX) {  // the owner pops its head
-#pragma unroll
-          for (int j = 0; j < K1 - 1; ++j) L[j] = L[j + 1];
-          L[K1 - 1].v = -INFINITY;
-          L[K1 - 1].i = INT_MAX;
-        }
+      }
+      warp_merge<K1, 2>(C2, S);
       }
 
       float M = 0.f, SE = 1.f;
@@ -353,10 +384,11 @@ __global__ void __launch_bounds__(NW * 32) route_kernel(RouteArgs a) {
             if (!a.noise) {
               P = kept ? 1.f : 0.f;
             } else {
+              // thr = -inf (no (k+1)-th) gives z = +inf and P = 1; s = 0 gives
+              // z = +-inf (P = 1 or 0) or, when c = thr, 0 / 0: P = 1/2
               const float thr = kept ? thr_kept : thr_out;
-              if (thr == -INFINITY) P = 1.f;
-              else if (sv[j] == 0.f) P = cv[j] > thr ? 1.f : (cv[j] < thr ? 0.f : 0.5f);
-              else P = normcdff(__fdividef(cv[j] - thr, sv[j]));
+              const float z = __fdividef(cv[j] - thr, sv[j]);
+              P = z == z ? phi_cdf(z) : 0.5f;
             }
             acc[u][j] += P;
             if (SW) pacc[u < PQ ? u : 0][j] += expf(cv[j] - sm_s[r][0]) / sm_s[r][1];
