@@ -220,10 +220,17 @@ def kernel_work(w, name: str, S_kept: int):
         return "hbm", 0.0, S_kept * d * esz + T * d * 4 + 4 * T * k
     if name == "bias_grad":
         return "hbm", 0.0, S_kept * (d + f) * esz + n * (d + f) * 4
+    ng = w.hier_a if w.hier_a else n   # the flat (or primary) gate's width
     if name == "gate_bwd":
-        return "hbm", 0.0, 4 * T * n * npj * 2 + 16 * T * k + 16 * T
+        # c, s read and dc, dz written per (row, column): the flat / primary
+        # gate's T rows and, hierarchical, the T k1 secondary rows of width b
+        return "hbm", 0.0, 4 * gate_cols * npj * 2 + 16 * T * k + 16 * T
     if name in ("gate_wgrad_fp32", "gate_dgrad_fp32"):
-        return "alu", npj * 2.0 * T * d * n, 4 * (T * d + npj * (d * n + T * n))
+        return "alu", npj * 2.0 * T * d * ng, 4 * (T * d + npj * (d * ng + T * ng))
+    if w.hier_a and name in ("hier_gate_wgrad", "hier_gate_dgrad"):
+        # the secondary gates' contractions over the T k1 gathered rows
+        R2, b = T * w.hier_k1, w.hier_b
+        return "alu", npj * 2.0 * R2 * d * b, 4 * (R2 * d + npj * (w.hier_a * d * b + R2 * b))
     if name == "route_topk":
         return "hbm", 0.0, 4 * gate_cols * npj + route_extra
     if name == "combine":

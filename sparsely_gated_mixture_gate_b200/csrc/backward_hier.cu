@@ -13,8 +13,9 @@
 // after which each level is a flat noisy top-k gate (gate_bwd, with the
 // secondary rows' tokens, noise streams 1 + g and coefficients lam_s(g, .)),
 // and the secondary gates' projections, one per group and gathered rows,
-// take these contractions (fp32, every output summed by one thread in row
-// order, so the results are bitwise reproducible):
+// take these contractions (fp32; grad_gemm.cu's kernel in its grouped mode,
+// every output one fused multiply-add chain in row or column order, so the
+// results are bitwise reproducible):
 //   dW_g2[g] = sum over g's rows r of x[token(r)] (x) dc2[r]   (and dW_noise2)
 //   db_g2[g] = sum over g's rows of dc2[r]
 //   dx[t]   += sum_ps (dc2[r] W_g2[g]^T + dz2[r] W_noise2[g]^T), r = row of (t, ps)
@@ -78,140 +79,46 @@ __global__ void hier_split_kernel(int T, int k1, int k2, int K, int n, const flo
   dgp[u] = acc;
 }
 
-// dW[g] [d][b] = sum over the group's rows of x[token(r)] (x) D[r]; blockIdx.z
-// picks the projection (0: dc2 -> dW_g2, 1: dz2 -> dW_noise2)
-constexpr int WT = 64, WR = 32;
-__global__ void __launch_bounds__(NT) hier_wgrad_kernel(const float *__restrict__ x, int d,
-                                                        const int *__restrict__ row_token,
-                                                        const int *__restrict__ seg_off, int b,
-                                                        const float *__restrict__ D0,
-                                                        const float *__restrict__ D1, float *dW0,
-                                                        float *dW1) {
-  __shared__ float Xs[WR][WT + 4];
-  __shared__ float Ds[WR][WT + 4];
-  const int g = blockIdx.x, q0 = blockIdx.y * WT, j0 = blockIdx.z % ((b + WT - 1) / WT) * WT;
-  const int proj = blockIdx.z / ((b + WT - 1) / WT);
-  const float *D = proj ? D1 : D0;
-  float *dW = (proj ? dW1 : dW0) + (size_t)g * d * b;
-  const int r_beg = seg_off[g], r_end = seg_off[g + 1];
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int r0 = r_beg; r0 < r_end; r0 += WR) {
-    for (int e = threadIdx.x; e < WR * WT; e += NT) {
-      const int rr = e / WT, cc = e % WT, r = r0 + rr;
-      const bool ok = r < r_end;
-      Xs[rr][cc] = ok && q0 + cc < d ? __ldg(x + (size_t)row_token[r] * d + q0 + cc) : 0.f;
-      Ds[rr][cc] = ok && j0 + cc < b ? __ldg(D + (size_t)r * b + j0 + cc) : 0.f;
-    }
-    __syncthreads();
-    const int nr = min(WR, r_end - r0);
-    for (int rr = 0; rr < nr; ++rr) {
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(Xs[rr][ty * 4 + i], Ds[rr][tx * 4 + j], acc[i][j]);
-    }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int q = q0 + ty * 4 + i;
-    if (q >= d) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int jj = j0 + tx * 4 + j;
-      if (jj < b) dW[(size_t)q * b + jj] = acc[i][j];
-    }
-  }
-}
-
-// db[g][j] = sum over the group's rows of D[r][j], rows in order
-__global__ void hier_colsum_kernel(const int *seg_off, int b, const float *D, float *db) {
-  const int g = blockIdx.x, j = blockIdx.y * blockDim.x + threadIdx.x;
-  if (j >= b) return;
+// db[g][j] = sum over the group's rows of D[r][j]: 8 row lanes per column
+// (lane l adds rows l, l + 8, ... in order), then the lanes in order
+constexpr int CL = 8, CC = 32;  // row lanes x columns per block
+__global__ void __launch_bounds__(CL * CC) hier_colsum_kernel(const int *seg_off, int b,
+                                                              const float *D, float *db) {
+  __shared__ float part[CL][CC + 1];
+  const int g = blockIdx.x, c = threadIdx.x % CC, l = threadIdx.x / CC;
+  const int j = blockIdx.y * CC + c;
+  const int r0 = seg_off[g], r1 = seg_off[g + 1];
   float s = 0.f;
-  for (int r = seg_off[g]; r < seg_off[g + 1]; ++r) s += D[(size_t)r * b + j];
-  db[(size_t)g * b + j] = s;
-}
-
-// dxs[r][q] = sum_j dc2[r][j] W_g2[g][q][j] + sum_j dz2[r][j] W_noise2[g][q][j]
-// over 128-row tiles of one group (seg_mblk: the groups' tile prefix)
-constexpr int DM = kGateBM, DQ = 64, DK = 16;  // the groups' 128-row tiles (seg_mblk)
-__global__ void __launch_bounds__(NT) hier_dgrad_kernel(const float *__restrict__ dc2,
-                                                        const float *__restrict__ dz2,
-                                                        const float *__restrict__ Wg2,
-                                                        const float *__restrict__ Wn2,
-                                                        const int *seg_off, const int *seg_mblk,
-                                                        int G, int d, int b, float *dxs) {
-  __shared__ float Dsh[DM][DK + 1];
-  __shared__ float Wsh[DK][DQ + 4];
-  const int mblk = blockIdx.x;
-  if (mblk >= seg_mblk[G]) return;
-  int lo = 0, hi = G - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (seg_mblk[mid] <= mblk) lo = mid; else hi = mid - 1;
-  }
-  const int g = lo;
-  const int row0 = seg_off[g] + (mblk - seg_mblk[g]) * DM, row_end = seg_off[g + 1];
-  const int q0 = blockIdx.y * DQ;
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  float acc[8][4];
+  if (j < b)
+    for (int r = r0 + l; r < r1; r += CL) s += __ldg(D + (size_t)r * b + j);
+  part[l][c] = s;
+  __syncthreads();
+  if (l == 0 && j < b) {
+    float t = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-  for (int proj = 0; proj < (dz2 ? 2 : 1); ++proj) {
-    const float *D = proj ? dz2 : dc2;
-    const float *W = (proj ? Wn2 : Wg2) + (size_t)g * d * b;
-    for (int j0 = 0; j0 < b; j0 += DK) {
-      for (int e = threadIdx.x; e < DM * DK; e += NT) {
-        const int rr = e / DK, kk = e % DK, r = row0 + rr;
-        Dsh[rr][kk] = r < row_end && j0 + kk < b ? __ldg(D + (size_t)r * b + j0 + kk) : 0.f;
-      }
-      for (int e = threadIdx.x; e < DK * DQ; e += NT) {
-        const int qq = e / DK, kk = e % DK;
-        Wsh[kk][qq] = q0 + qq < d && j0 + kk < b ? __ldg(W + (size_t)(q0 + qq) * b + j0 + kk) : 0.f;
-      }
-      __syncthreads();
-#pragma unroll
-      for (int kk = 0; kk < DK; ++kk)
-#pragma unroll
-        for (int i = 0; i < 8; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(Dsh[ty * 8 + i][kk], Wsh[kk][tx * 4 + j], acc[i][j]);
-      __syncthreads();
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int r = row0 + ty * 8 + i;
-    if (r >= row_end) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int q = q0 + tx * 4 + j;
-      if (q < d) dxs[(size_t)r * d + q] = acc[i][j];
-    }
+    for (int q = 0; q < CL; ++q) t += part[q][c];
+    db[(size_t)g * b + j] = t;
   }
 }
 
-// dx[t][q] += sum over the kept groups ps of dxs[row of (t, ps)][q], ps in order
+// dx[t][q] += sum over the kept groups ps of dxs[row of (t, ps)][q], ps in
+// order; four columns per thread (d is a multiple of 8)
 __global__ void hier_dx_sum_kernel(int T, int k1, int d, const int *grow, const float *dxs,
                                    float *dx) {
-  const int64_t total = (int64_t)T * d;
+  const int d4 = d >> 2;
+  const int64_t total = (int64_t)T * d4;
   for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
        e += (int64_t)gridDim.x * blockDim.x) {
-    const int t = (int)(e / d), q = (int)(e % d);
-    float s = dx[e];
+    const int t = (int)(e / d4), q4 = (int)(e % d4);
+    float4 s = reinterpret_cast<float4 *>(dx)[e];
     for (int ps = 0; ps < k1; ++ps) {
       const int r = grow[(size_t)t * k1 + ps];  // -1: unplaced (non-finite logits)
-      if (r >= 0 && r < T * k1) s += dxs[(size_t)r * d + q];
+      if (r >= 0 && r < T * k1) {
+        const float4 v = __ldg(reinterpret_cast<const float4 *>(dxs + (size_t)r * d) + q4);
+        s.x += v.x; s.y += v.y; s.z += v.z; s.w += v.w;
+      }
     }
-    dx[e] = s;
+    reinterpret_cast<float4 *>(dx)[e] = s;
   }
 }
 
@@ -235,20 +142,37 @@ int launch_hier_split(int T, int k1, int k2, int K, int n, const float *pgate,
 int launch_hier_gate_wgrad(const float *x, int d, const int *row_token, const int *seg_off, int a,
                            int b, const float *dc2, const float *dz2, float *dWg2, float *dWn2,
                            float *dbg2, cudaStream_t st) {
-  const int nj = (int)ceil_div(b, WT);
   if (dWg2 || dWn2) {
-    // both projections in one launch when both are asked for
+    // dW[g] = X_g^T D_g: M = d, N = b, K = the group's rows (x rows gathered
+    // by token); both projections in one launch when both are asked for
+    SgemmArgs s{};
+    s.M = d;
+    s.N = b;
+    s.K = 0;
+    s.A[0] = s.A[1] = x;
+    s.lda = d;
+    s.at = 1;
+    s.ldb = b;
+    s.bt = 0;
+    s.ldc = b;
     const bool two = dWg2 && dWn2 && dz2;
-    const float *D0 = dWg2 ? dc2 : dz2;
-    float *W0 = dWg2 ? dWg2 : dWn2;
-    MOE_TRY(launch("hier_gate_wgrad", hier_wgrad_kernel,
-                   dim3((unsigned)a, (unsigned)ceil_div(d, WT), (unsigned)(nj * (two ? 2 : 1))),
-                   dim3(NT), 0, st, x, d, row_token, seg_off, b, D0, two ? dz2 : D0, W0,
-                   two ? dWn2 : W0));
+    s.B[0] = dWg2 ? dc2 : dz2;
+    s.C[0] = dWg2 ? dWg2 : dWn2;
+    s.B[1] = two ? dz2 : s.B[0];
+    s.C[1] = two ? dWn2 : s.C[0];
+    s.nprob = two ? 2 : 1;
+    s.splits = 1;
+    s.seg_off = seg_off;
+    s.a_row = row_token;
+    s.G = a;
+    s.seg_k = 1;
+    s.sC = (int64_t)d * b;
+    s.name = "hier_gate_wgrad";
+    MOE_TRY(launch_sgemm(s, st));
   }
   if (dbg2)
-    MOE_TRY(launch("hier_colsum", hier_colsum_kernel, dim3((unsigned)a, (unsigned)ceil_div(b, NT)),
-                   dim3(NT), 0, st, seg_off, b, dc2, dbg2));
+    MOE_TRY(launch("hier_colsum", hier_colsum_kernel, dim3((unsigned)a, (unsigned)ceil_div(b, CC)),
+                   dim3(CL * CC), 0, st, seg_off, b, dc2, dbg2));
   return MOE_OK;
 }
 
@@ -256,10 +180,34 @@ int launch_hier_gate_dgrad(const float *dc2, const float *dz2, const float *Wg2,
                            const int *seg_off, const int *seg_mblk, int mblk_upper, int a, int d,
                            int b, float *dxs, int T, int k1, const int *grow, float *dx,
                            cudaStream_t st) {
-  MOE_TRY(launch("hier_gate_dgrad", hier_dgrad_kernel,
-                 dim3((unsigned)mblk_upper, (unsigned)ceil_div(d, DQ)), dim3(NT), 0, st, dc2, dz2,
-                 Wg2, Wn2, seg_off, seg_mblk, a, d, b, dxs));
-  const int64_t total = (int64_t)T * d;
+  // dxs[rows of g] = dc2 W_g2[g]^T (+ dz2 W_noise2[g]^T): M = the group's rows,
+  // N = d, K = b; B(k, n) = W[g][n][k]
+  SgemmArgs s{};
+  s.M = T * k1;
+  s.N = d;
+  s.K = b;
+  s.A[0] = dc2;
+  s.A[1] = dz2;
+  s.lda = b;
+  s.at = 0;
+  s.B[0] = Wg2;
+  s.B[1] = Wn2;
+  s.ldb = b;
+  s.bt = 1;
+  s.C[0] = s.C[1] = dxs;
+  s.ldc = d;
+  s.nprob = 1;
+  s.ksum = dz2 ? 1 : 0;
+  s.splits = 1;
+  s.seg_off = seg_off;
+  s.seg_mblk = seg_mblk;
+  s.G = a;
+  s.seg_k = 0;
+  s.mblk_upper = mblk_upper;
+  s.sB = (int64_t)d * b;
+  s.name = "hier_gate_dgrad";
+  MOE_TRY(launch_sgemm(s, st));
+  const int64_t total = (int64_t)T * (d / 4);
   const int grid = (int)std::min<int64_t>(ceil_div(total, NT), 8 * (int64_t)num_sms());
   return launch("hier_dx_sum", hier_dx_sum_kernel, dim3((unsigned)(grid > 0 ? grid : 1)), dim3(NT),
                 0, st, T, k1, d, grow, dxs, dx);

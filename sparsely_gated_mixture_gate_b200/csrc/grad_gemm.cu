@@ -15,24 +15,60 @@
 // to the machine (the weight gradients: K = T is the long side) the K range
 // is split across CTAs into a scratch buffer and a second kernel adds the
 // splits in order, so the result does not depend on timing.
+// A grouped mode serves the hierarchical layer's secondary gates: one launch
+// over the groups' row segments, along K (the weight gradients, A's rows
+// gathered by token) or along M (the input gradient, one weight pair per group).
 #include "internal.h"
 
 namespace moe {
 namespace {
 
 constexpr int BM = 128, BN = 128, BK = 16, NT = 256;
+static_assert(BM == kGateBM, "grouped M tiles come from the gate's 128-row tile prefix");
 
-template <bool AT, bool BT>
+// GR: the grouped mode (compiled separately so that the plain instances keep
+// their registers)
+template <bool AT, bool BT, bool GR>
 __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
   __shared__ __align__(16) float As[2][BK][BM + 4];
   __shared__ __align__(16) float Bs[2][BK][BN + 4];
-  const int m0 = blockIdx.y * BM, n0 = blockIdx.x * BN;
+  int m0 = blockIdx.y * BM;
+  const int n0 = blockIdx.x * BN;
   const int splits = a.part ? a.splits : 1;
-  const int prob = a.nprob > 1 ? (int)blockIdx.z / splits : 0;
+  int prob = a.nprob > 1 ? (int)blockIdx.z / splits : 0;
   const int split = (int)blockIdx.z % splits;
   // split length a multiple of the slice, so every 16-byte load stays aligned
   const int kc = (a.K + splits - 1) / splits + BK - 1 & ~(BK - 1);
-  const int kbeg = split * kc, kend = min(a.K, kbeg + kc);
+  int kbeg = split * kc, kend = min(a.K, kbeg + kc);
+  int Mx = a.M;                   // rows of this problem
+  const int *arow = nullptr;      // A's rows (stored [K][M]) gathered through it
+  int64_t offA = 0, offB = 0, offC = 0;
+  if (GR) {
+    if (a.seg_k) {  // blockIdx.z = group * nprob + problem
+      const int g = (int)blockIdx.z / a.nprob;
+      prob = (int)blockIdx.z % a.nprob;
+      const int r0 = a.seg_off[g];
+      kbeg = 0;
+      kend = a.seg_off[g + 1] - r0;
+      arow = a.a_row + r0;
+      offB = (int64_t)r0 * a.ldb;
+      offC = (int64_t)g * a.sC;
+    } else {  // blockIdx.y = the M tile over all groups
+      const int t = (int)blockIdx.y;
+      if (t >= a.seg_mblk[a.G]) return;
+      int lo = 0, hi = a.G - 1;  // largest g with seg_mblk[g] <= t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.seg_mblk[mid] <= t) lo = mid; else hi = mid - 1;
+      }
+      const int r0 = a.seg_off[lo];
+      m0 = (t - a.seg_mblk[lo]) * BM;
+      Mx = a.seg_off[lo + 1] - r0;
+      offA = (int64_t)r0 * a.lda;
+      offB = (int64_t)lo * a.sB;
+      offC = (int64_t)r0 * a.ldc;
+    }
+  }
   const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
   // 16-byte loads need 4 consecutive in-range elements along the contiguous
   // dimension and a leading dimension that keeps them aligned
@@ -44,7 +80,7 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (!AT) {
       const int m = m0 + (tid >> 2) + 64 * h, kk = k0 + (tid & 3) * 4;
-      if (m >= a.M) return v;
+      if (m >= Mx) return v;
       const float *p = A + (size_t)m * a.lda + kk;
       if (va && kk + 3 < kend) return __ldg(reinterpret_cast<const float4 *>(p));
       v.x = kk + 0 < kend ? __ldg(p + 0) : 0.f;
@@ -54,12 +90,12 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
     } else {
       const int kk = k0 + (tid >> 5) + 8 * h, m = m0 + (tid & 31) * 4;
       if (kk >= kend) return v;
-      const float *p = A + (size_t)kk * a.lda + m;
-      if (va && m + 3 < a.M) return __ldg(reinterpret_cast<const float4 *>(p));
-      v.x = m + 0 < a.M ? __ldg(p + 0) : 0.f;
-      v.y = m + 1 < a.M ? __ldg(p + 1) : 0.f;
-      v.z = m + 2 < a.M ? __ldg(p + 2) : 0.f;
-      v.w = m + 3 < a.M ? __ldg(p + 3) : 0.f;
+      const float *p = A + (size_t)(GR && arow ? __ldg(arow + kk) : kk) * a.lda + m;
+      if (va && m + 3 < Mx) return __ldg(reinterpret_cast<const float4 *>(p));
+      v.x = m + 0 < Mx ? __ldg(p + 0) : 0.f;
+      v.y = m + 1 < Mx ? __ldg(p + 1) : 0.f;
+      v.z = m + 2 < Mx ? __ldg(p + 2) : 0.f;
+      v.w = m + 3 < Mx ? __ldg(p + 3) : 0.f;
     }
     return v;
   };
@@ -123,7 +159,7 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
   for (int p = 0; p < npair; ++p) {
     const int pi = a.ksum ? p : prob;
     // (selected, not indexed: a runtime index would copy the arguments to local memory)
-    const float *A = pi ? a.A[1] : a.A[0], *B = pi ? a.B[1] : a.B[0];
+    const float *A = (pi ? a.A[1] : a.A[0]) + offA, *B = (pi ? a.B[1] : a.B[0]) + offB;
     if (kbeg >= kend) break;
     float4 av[2] = {load_a(A, kbeg, 0), load_a(A, kbeg, 1)};
     float4 bv[2] = {load_b(B, kbeg, 0), load_b(B, kbeg, 1)};
@@ -161,11 +197,11 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
   }
 
   // output rows ty*4+i (i<4) and 64+ty*4+i-4, columns tx*4+j and 64+tx*4+j-4
-  float *const C = prob ? a.C[1] : a.C[0];
+  float *const C = (prob ? a.C[1] : a.C[0]) + offC;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     const int m = m0 + (i < 4 ? ty * 4 + i : 64 + ty * 4 + i - 4);
-    if (m >= a.M) continue;
+    if (m >= Mx) continue;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int nn = n0 + h * 64 + tx * 4;
@@ -225,16 +261,29 @@ int launch_sgemm(const SgemmArgs &a, cudaStream_t st) {
   SgemmArgs b = a;
   if (b.nprob < 1) b.nprob = 1;
   if (b.ksum) b.nprob = 1;
-  if (b.splits <= 1) b.part = nullptr;
+  if (b.splits <= 1 || b.seg_off) b.part = nullptr;
   const int splits = b.part ? b.splits : 1;
-  const dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ceil_div(a.M, BM),
-                  (unsigned)(splits * b.nprob));
+  dim3 grid((unsigned)ceil_div(a.N, BN), (unsigned)ceil_div(a.M, BM), (unsigned)(splits * b.nprob));
+  if (b.seg_off) {
+    if (b.G <= 0) return MOE_OK;
+    if (b.seg_k) grid.z = (unsigned)(b.G * b.nprob);
+    else grid.y = (unsigned)b.mblk_upper;  // M = the rows of each group
+  }
   const char *name = a.name ? a.name : "gate_grad_gemm";
   int rc;
-  if (!a.at && !a.bt) rc = launch(name, sgemm_kernel<false, false>, grid, dim3(NT), 0, st, b);
-  else if (a.at && !a.bt) rc = launch(name, sgemm_kernel<true, false>, grid, dim3(NT), 0, st, b);
-  else if (!a.at && a.bt) rc = launch(name, sgemm_kernel<false, true>, grid, dim3(NT), 0, st, b);
-  else rc = launch(name, sgemm_kernel<true, true>, grid, dim3(NT), 0, st, b);
+  if (b.seg_off) {  // the two grouped shapes in use: K-grouped x^T D and M-grouped D W^T
+    if (a.at && !a.bt) rc = launch(name, sgemm_kernel<true, false, true>, grid, dim3(NT), 0, st, b);
+    else if (!a.at && a.bt) rc = launch(name, sgemm_kernel<false, true, true>, grid, dim3(NT), 0, st, b);
+    else return MOE_EINVAL;
+  } else if (!a.at && !a.bt) {
+    rc = launch(name, sgemm_kernel<false, false, false>, grid, dim3(NT), 0, st, b);
+  } else if (a.at && !a.bt) {
+    rc = launch(name, sgemm_kernel<true, false, false>, grid, dim3(NT), 0, st, b);
+  } else if (!a.at && a.bt) {
+    rc = launch(name, sgemm_kernel<false, true, false>, grid, dim3(NT), 0, st, b);
+  } else {
+    rc = launch(name, sgemm_kernel<true, true, false>, grid, dim3(NT), 0, st, b);
+  }
   if (rc != MOE_OK || !b.part) return rc;
   const size_t total = (size_t)a.M * a.N;
   return launch("gate_grad_split_sum", split_sum_kernel,

@@ -316,6 +316,15 @@ struct SgemmArgs {
   float *part;
   int splits;
   const char *name;
+  // Grouped (seg_off set, no split-K): G problems over row segments
+  // [seg_off[g], seg_off[g+1]).  seg_k = 1: the segment is the K range (A
+  // stored [K][M] with its rows gathered through a_row, B's rows the
+  // segment's), C_g = C + g * sC.  seg_k = 0: the segment is the M range (M
+  // tiles found through seg_mblk, the exclusive scan of ceil(rows / 128)), A's
+  // and C's rows the segment's, B_g = B + g * sB.
+  const int *seg_off, *seg_mblk, *a_row;
+  int G, seg_k, mblk_upper;
+  int64_t sB, sC;
 };
 int launch_sgemm(const SgemmArgs &a, cudaStream_t st);
 int sgemm_splits(int M, int N, int K, int nprob);  // split-K factor for nprob problems of M x N
