@@ -12,7 +12,8 @@
 //   bias b, top-k of H, gates Sigmoid(c_i) / sum of Sigmoid(c_j) over the kept.
 //   Router statistics ([MoE-intro] 第三部分, optional): per row |c|^2 and the
 //   entropy of softmax(c), summed over the tile's rows in a fixed order.
-// Pass 1, one warp per row: each lane scans column quads 4m .. 4m+3 (16-byte
+// Pass 1, one warp per row (rows of at most 128 or 64 columns: two or four
+// rows per warp, 16 or 8 lanes each): each lane scans column quads 4m .. 4m+3 (16-byte
 // loads, one Philox call per quad) and keeps a sorted list of its k + 1 best
 // columns (ranked by H, then the lower column index); the warp merges the 32
 // lists with shuffles.  Rows of 512 columns or more rank quads instead, by
@@ -86,16 +87,19 @@ __device__ __forceinline__ void quad_h(const RouteArgs &a, const float *crow, co
   }
 }
 
-// K1 rounds of a warp-wide arg-max over the heads of the lanes' sorted lists;
-// the owner pops its head.  S gets the warp's K1 first entries, in order.
+// K1 rounds of an arg-max over the heads of the sorted lists of each aligned
+// group of lpr lanes (32, 16 or 8: one row each); the owner pops its head.  S
+// gets the group's K1 first entries, in order.  Every lane of the warp takes
+// part.
 template <int K1, int LN>
-__device__ __forceinline__ void warp_merge(Cand (&L)[LN], Cand (&S)[K1]) {
+__device__ __forceinline__ void warp_merge(Cand (&L)[LN], Cand (&S)[K1], int lpr) {
 #pragma unroll
   for (int r = 0; r < K1; ++r) {
     float bv = L[0].v;
     int bi = L[0].i;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
+      if (off >= lpr) continue;
       const float ov = __shfl_xor_sync(0xffffffffu, bv, off);
       const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
       if (before(ov, oi, bv, bi)) { bv = ov; bi = oi; }
@@ -116,13 +120,18 @@ __device__ __forceinline__ void warp_merge(Cand (&L)[LN], Cand (&S)[K1]) {
 // EX = extra outputs compiled in: the router statistics (stats_part) and the
 // rows' thresholds for the backward pass (kth), each only when its pointer is
 // set.
-template <int K1, int MAXQ, bool SW, bool EX>
+// NARROW: rows of at most 128 columns and tiles of at least 16 rows, several
+// rows per warp in pass 1 (a separate instance, so that one row per warp pays
+// nothing for it).
+template <int K1, int MAXQ, bool SW, bool EX, bool NARROW>
 __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kernel(RouteArgs a) {
   constexpr int KM = K1 - 1;  // k
   constexpr int PQ = SW ? MAXQ : 1;
-  __shared__ uint32_t kept_s[NW][MAXQ * NW * 32 * 4 / 32];  // kept columns of each row, one bit each
-  __shared__ float thr_s[NW][2];   // (k+1)-th largest, k-th largest
-  __shared__ float sm_s[NW][2];    // Switch: max and sum of exp of the clean logits
+  // per row of a round: kept columns (one bit each, nwords words a row), the
+  // (k+1)-th and k-th largest H, the Switch softmax's max and sum
+  __shared__ uint32_t kept_s[NW * MAXQ * 32];
+  __shared__ float thr_s[NW * 4][2];
+  __shared__ float sm_s[NW * 4][2];
   __shared__ float4 red_s[NW * 32];
   __shared__ float4 redp_s[NW * 32];
   const int nb = a.nb;
@@ -154,10 +163,15 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
   const uint32_t gate_id = a.secondary ? (uint32_t)(1 + g) : 0u;
   bool bad = false;
 
+  // pass 1: rows per warp and lanes per row; NR rows per round
+  const bool by_quad = nb >= 512;  // rank quads: at least four quads per lane
+  const int RPW = !NARROW ? 1 : (nb <= 64 && a.RT >= 4 * NW) ? 4 : 2;
+  const int LPR = 32 / RPW, sub = lane / LPR, sl = lane % LPR;
+  const int NR = NW * RPW;
   // pass-2 thread layout: thread per column quad; with fewer quads than
-  // threads, RG groups of threads split the rows of each block
+  // threads, RG groups of threads split the rows of each round
   const int nq = (nb + 3) >> 2;
-  const int RG = nq >= NW * 32 ? 1 : min((NW * 32) / nq, NW);
+  const int RG = nq >= NW * 32 ? 1 : min((NW * 32) / nq, NR);
   const int rg = nq >= NW * 32 ? 0 : (int)threadIdx.x / nq;
   const int nqpass = (nq + NW * 32 - 1) / (NW * 32);  // quads per thread when RG == 1
   float acc[MAXQ][4], pacc[PQ][4];
@@ -171,17 +185,19 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
     for (int j = 0; j < 4; ++j) pacc[u][j] = 0.f;
 
   const bool stats = EX && a.stats_part != nullptr;
-  float rz = 0.f, rh = 0.f;  // lane 0: this warp's rows' |c|^2 and entropies
+  float rz = 0.f, rh = 0.f;  // lanes sl = 0: their rows' |c|^2 and entropies
   const int nwords = (nb + 31) >> 5;
-  for (int rb = row0; rb < row_end; rb += NW) {
-    // ================= pass 1: routing of row rb + w (warp per row)
-    const int row = rb + w;
-    for (int q = lane; q < nwords; q += 32) kept_s[w][q] = 0u;  // read by the last pass 2
+  for (int rb = row0; rb < row_end; rb += NR) {
+    // ================= pass 1: routing of row rb + rloc (LPR lanes per row)
+    const int rloc = w * RPW + sub, row = rb + rloc;
+    const bool live = row < row_end;
+    for (int q = lane; q < RPW * nwords; q += 32) kept_s[w * RPW * nwords + q] = 0u;  // read by pass 2
     __syncwarp();
-    if (row < row_end) {
-      const int t = a.row_token ? a.row_token[row] : row;
-      const float *crow = a.c + (size_t)row * nb;
-      const float *srow = a.s + (size_t)row * nb;
+    {
+      const int nbe = live ? nb : 0;  // a row past the tile's end scans nothing
+      const int t = live ? (a.row_token ? a.row_token[row] : row) : 0;
+      const float *crow = a.c + (size_t)(live ? row : row0) * nb;
+      const float *srow = a.s + (size_t)(live ? row : row0) * nb;
 
       Cand L[K1];
 #pragma unroll
@@ -189,8 +205,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
       float mx = -INFINITY, se = 0.f;  // online softmax of c (Switch)
 
       const uint32_t ctr0 = (uint32_t)t + a.token_base;
-      const bool by_quad = nb >= 512;  // at least four quads per lane
-      for (int m = lane; 4 * m < nb; m += 32) {
+      for (int m = sl; 4 * m < nbe; m += LPR) {
         const int i0 = 4 * m;
         float cv[4], sv[4], h[4];
         quad_h(a, crow, srow, m, nb, vec4, ctr0, gate_id, key0, key1, cv, sv, h);
@@ -214,10 +229,10 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
       // (at most) two of the 4 (k + 1) columns, and the warp merges them
       Cand S[K1];
       if (!by_quad) {
-        warp_merge<K1, K1>(L, S);
-      } else {
+        warp_merge<K1, K1>(L, S, LPR);
+      } else {  // one row per warp here
       Cand Q[K1];
-      warp_merge<K1, K1>(L, Q);
+      warp_merge<K1, K1>(L, Q, 32);
       Cand C2[2];
 #pragma unroll
       for (int j = 0; j < 2; ++j) { C2[j].v = -INFINITY; C2[j].i = INT_MAX; }
@@ -228,13 +243,13 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
 #pragma unroll
         for (int rr = 0; rr < K1; ++rr)
           if (rr == r) m = Q[rr].i;
-        if (l < 4 * K1 && m != INT_MAX && 4 * m + q < nb) {
+        if (live && l < 4 * K1 && m != INT_MAX && 4 * m + q < nb) {
           float cv[4], sv[4], h[4];
           quad_h(a, crow, srow, m, nb, vec4, ctr0, gate_id, key0, key1, cv, sv, h);
           insert<2>(C2, q == 0 ? h[0] : q == 1 ? h[1] : q == 2 ? h[2] : h[3], 4 * m + q);
         }
       }
-      warp_merge<K1, 2>(C2, S);
+      warp_merge<K1, 2>(C2, S, 32);
       }
 
       float M = 0.f, SE = 1.f;
@@ -242,6 +257,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
         M = mx; SE = se;
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
+          if (off >= LPR) continue;
           const float om = __shfl_xor_sync(0xffffffffu, M, off);
           const float os = __shfl_xor_sync(0xffffffffu, SE, off);
           const float m2 = fmaxf(M, om);
@@ -260,12 +276,12 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
         float sg[KM], den = 0.f;
 #pragma unroll
         for (int j = 0; j < KM; ++j) {
-          sg[j] = S[j].i < nb ? 1.f / (1.f + expf(-crow[S[j].i])) : 0.f;
+          sg[j] = live && S[j].i < nb ? 1.f / (1.f + expf(-crow[S[j].i])) : 0.f;
           den += sg[j];
         }
 #pragma unroll
         for (int j = 0; j < KM; ++j)
-          if (j == lane) {
+          if (j == sl) {
             idx_j = S[j].i;
             gate_j = sg[j] / den;
           }
@@ -275,46 +291,48 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
         for (int j = 0; j < KM; ++j) den += expf(S[j].v - S[0].v);
 #pragma unroll
         for (int j = 0; j < KM; ++j)
-          if (j == lane) {
+          if (j == sl) {
             idx_j = S[j].i;
-            gate_j = sw ? expf(crow[S[0].i] - M) / SE : expf(S[j].v - S[0].v) / den;
+            gate_j = sw ? (live && S[0].i < nb ? expf(crow[S[0].i] - M) / SE : 0.f)
+                        : expf(S[j].v - S[0].v) / den;
           }
       }
-      if (EX && a.gate_raw && lane < k) {  // kept for the backward pass, by row
-        a.gate_raw[(size_t)row * k + lane] = gate_j;
-        a.idx_raw[(size_t)row * k + lane] = idx_j;
+      if (EX && a.gate_raw && live && sl < k) {  // kept for the backward pass, by row
+        a.gate_raw[(size_t)row * k + sl] = gate_j;
+        a.idx_raw[(size_t)row * k + sl] = idx_j;
       }
-      if (lane < k) {
-        int slot = lane;
+      if (live && sl < k) {
+        int slot = sl;
         float gmul = 1.f;
         int ebase = 0;
         if (a.secondary) {
           const int ps = a.row_slot[row];
-          slot = ps * k + lane;
+          slot = ps * k + sl;
           gmul = a.gate_mult[(size_t)t * a.k1 + ps];
           ebase = g * a.expert_stride;
         }
         a.out_idx[(size_t)t * a.K + slot] = ebase + idx_j;
         a.out_gate[(size_t)t * a.K + slot] = gmul * gate_j;
       }
-      if (lane == 0) {
+      if (live && sl == 0) {
 #pragma unroll
         for (int j = 0; j < KM; ++j)
-          if (S[j].i >= 0 && S[j].i < nb) kept_s[w][S[j].i >> 5] |= 1u << (S[j].i & 31);
-        thr_s[w][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
-        thr_s[w][1] = S[K1 - 2].v;
+          if (S[j].i >= 0 && S[j].i < nb)
+            kept_s[rloc * nwords + (S[j].i >> 5)] |= 1u << (S[j].i & 31);
+        thr_s[rloc][0] = S[K1 - 1].v;  // -inf if the (k+1)-th does not exist
+        thr_s[rloc][1] = S[K1 - 2].v;
         if (EX && a.kth)  // kept for the backward pass's load gradient
           a.kth[row] = make_int4(__float_as_int(S[K1 - 1].v), S[K1 - 1].i,
                                  __float_as_int(S[K1 - 2].v), S[K1 - 2].i);
-        sm_s[w][0] = M;
-        sm_s[w][1] = SE;
+        sm_s[rloc][0] = M;
+        sm_s[rloc][1] = SE;
       }
       if (stats) {
         // router statistics of the row, a second pass over its clean logits
         // (cache hits): sum c^2 and an online softmax with S = sum e^(c-m),
         // Q = sum e^(c-m) (c-m), the entropy being log S - Q/S
         float zs = 0.f, sm = -INFINITY, ss = 0.f, sq = 0.f;
-        for (int i = lane; i < nb; i += 32) {
+        for (int i = sl; i < nbe; i += LPR) {
           const float v = crow[i];
           zs = fmaf(v, v, zs);
           if (v > sm) {  // rescale to the new maximum
@@ -329,6 +347,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) {
+          if (off >= LPR) continue;
           zs += __shfl_xor_sync(0xffffffffu, zs, off);
           const float om = __shfl_xor_sync(0xffffffffu, sm, off);
           const float os = __shfl_xor_sync(0xffffffffu, ss, off);
@@ -340,7 +359,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
           ss = ss * r1 + os * r2;
           sm = m2;
         }
-        if (lane == 0) {
+        if (live && sl == 0) {
           rz += zs;
           rh += logf(ss) - sq / ss;
         }
@@ -348,8 +367,8 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
     }
     __syncthreads();
 
-    // ================= pass 2: this block's rows into the column sums
-    const int nrow_blk = min(NW, row_end - rb);
+    // ================= pass 2: this round's rows into the column sums
+    const int nrow_blk = min(NR, row_end - rb);
     if (rg < RG) {
 #pragma unroll
       for (int u = 0; u < MAXQ; ++u) {
@@ -376,7 +395,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
             }
           }
           const float thr_kept = thr_s[r][0], thr_out = thr_s[r][1];
-          const uint32_t kbits = kept_s[r][i0 >> 5] >> (i0 & 31);  // the quad's 4 bits
+          const uint32_t kbits = kept_s[r * nwords + (i0 >> 5)] >> (i0 & 31);  // the quad's 4 bits
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const bool kept = (kbits >> j) & 1u;
@@ -400,8 +419,14 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
   }
   if (bad && a.status) atomicOr(a.status, MOE_STATUS_NONFINITE);
 
-  if (stats) {  // the tile's statistics: warps added in warp order
+  if (stats) {  // the tile's statistics: a warp's rows, then warps in warp order
     __shared__ float st_s[NW][2];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {  // the row groups' leaders (other lanes hold 0)
+      if (off < LPR) continue;
+      rz += __shfl_xor_sync(0xffffffffu, rz, off);
+      rh += __shfl_xor_sync(0xffffffffu, rh, off);
+    }
     if (lane == 0) {
       st_s[w][0] = rz;
       st_s[w][1] = rh;
@@ -501,16 +526,24 @@ int launch_route(const RouteArgs &a, int tiles_upper, cudaStream_t st) {
     return launch("route_topk", kern, dim3(tiles_upper), dim3(NW * 32), 0, st, a);
   };
   const bool wide = a.nb > 4 * 4 * NW * 32;  // more than 4096 columns
+  const bool narrow = a.nb <= 128 && a.RT >= 2 * NW;
   const bool st_on = a.stats_part != nullptr || a.kth != nullptr || a.gate_raw != nullptr;
   if (a.router == MOE_ROUTER_SWITCH) {
     if (a.k != 1 || wide) return MOE_EINVAL;
-    return st_on ? go(route_kernel<2, 4, true, true>) : go(route_kernel<2, 4, true, false>);
+    if (narrow)
+      return st_on ? go(route_kernel<2, 4, true, true, true>) : go(route_kernel<2, 4, true, false, true>);
+    return st_on ? go(route_kernel<2, 4, true, true, false>) : go(route_kernel<2, 4, true, false, false>);
   }
-#define MOE_ROUTE_CASE(K1)                                                                   \
-  case K1:                                                                                   \
-    if (st_on)                                                                               \
-      return wide ? go(route_kernel<K1, 8, false, true>) : go(route_kernel<K1, 4, false, true>); \
-    return wide ? go(route_kernel<K1, 8, false, false>) : go(route_kernel<K1, 4, false, false>);
+#define MOE_ROUTE_CASE(K1)                                                               \
+  case K1:                                                                               \
+    if (narrow)                                                                          \
+      return st_on ? go(route_kernel<K1, 4, false, true, true>)                          \
+                   : go(route_kernel<K1, 4, false, false, true>);                        \
+    if (st_on)                                                                           \
+      return wide ? go(route_kernel<K1, 8, false, true, false>)                          \
+                  : go(route_kernel<K1, 4, false, true, false>);                         \
+    return wide ? go(route_kernel<K1, 8, false, false, false>)                           \
+                : go(route_kernel<K1, 4, false, false, false>);
   switch (a.k + 1) {
     MOE_ROUTE_CASE(2)
     MOE_ROUTE_CASE(3)
