@@ -30,7 +30,7 @@ oracle itself (the reference arm of this comparison).
 ``--backward``: one step is the forward pass followed by the backward pass
 (``moe_backward``: dx and every parameter's gradient for an upstream gradient
 dy plus the weighted balancing losses); the metric is then training tokens/s
-(default workload lm-flat: the backward pass covers flat layers).
+(default workload: hierarchical, as for the forward pass).
 """
 from __future__ import annotations
 
@@ -763,8 +763,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=None,
-                    help="default: hierarchical (the largest single-GPU workload); lm-flat with "
-                         "--backward (the backward pass covers flat layers)")
+                    help="default: hierarchical (the largest single-GPU workload), also with "
+                         "--backward")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--gate", default="fp32", choices=["fp32", "tf32x3"],
                     help="gate projections: fp32 multiply-adds or the 3-pass TF32 tensor-core split")
@@ -785,7 +785,7 @@ def main():
         raise SystemExit("--warmup must be at least 3")
 
     from sparsely_gated_mixture_gate_b200 import synth
-    name = args.workload or ("lm-flat" if args.backward else "hierarchical")
+    name = args.workload or "hierarchical"
     w = (synth.WORKLOADS.get(name) or synth.VARIANTS[name]).with_(
         gate_precision=1 if args.gate == "tf32x3" else 0)
     world, rank, local = dist_info()

@@ -175,14 +175,25 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
         bv[0] = load_b(B, k0 + BK, 0);
         bv[1] = load_b(B, k0 + BK, 1);
       }
+      // the fragments of step kk + 1 are read while step kk's FMAs run
+      float4 fa0[2], fa1[2], fb0[2], fb1[2];
+      fa0[0] = *reinterpret_cast<const float4 *>(&As[buf][0][ty * 4]);
+      fa1[0] = *reinterpret_cast<const float4 *>(&As[buf][0][64 + ty * 4]);
+      fb0[0] = *reinterpret_cast<const float4 *>(&Bs[buf][0][tx * 4]);
+      fb1[0] = *reinterpret_cast<const float4 *>(&Bs[buf][0][64 + tx * 4]);
 #pragma unroll
       for (int kk = 0; kk < BK; ++kk) {
-        const float4 a0 = *reinterpret_cast<const float4 *>(&As[buf][kk][ty * 4]);
-        const float4 a1 = *reinterpret_cast<const float4 *>(&As[buf][kk][64 + ty * 4]);
-        const float4 b0 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][tx * 4]);
-        const float4 b1 = *reinterpret_cast<const float4 *>(&Bs[buf][kk][64 + tx * 4]);
-        const float av8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        const float bv8[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+        const int cur = kk & 1, nxt = cur ^ 1;
+        if (kk + 1 < BK) {
+          fa0[nxt] = *reinterpret_cast<const float4 *>(&As[buf][kk + 1][ty * 4]);
+          fa1[nxt] = *reinterpret_cast<const float4 *>(&As[buf][kk + 1][64 + ty * 4]);
+          fb0[nxt] = *reinterpret_cast<const float4 *>(&Bs[buf][kk + 1][tx * 4]);
+          fb1[nxt] = *reinterpret_cast<const float4 *>(&Bs[buf][kk + 1][64 + tx * 4]);
+        }
+        const float av8[8] = {fa0[cur].x, fa0[cur].y, fa0[cur].z, fa0[cur].w,
+                              fa1[cur].x, fa1[cur].y, fa1[cur].z, fa1[cur].w};
+        const float bv8[8] = {fb0[cur].x, fb0[cur].y, fb0[cur].z, fb0[cur].w,
+                              fb1[cur].x, fb1[cur].y, fb1[cur].z, fb1[cur].w};
 #pragma unroll
         for (int i = 0; i < 8; ++i)
 #pragma unroll
