@@ -193,7 +193,7 @@ __device__ void write_plan(const int *counts, int n, const PlanOut &o) {
       ucoff[e] = (int)q;
       if (seg_mblk) seg_mblk[e] = (int)pm;
       if (seg_tiles) seg_tiles[e] = (int)pt;
-      if (tab1) {  // expert GEMM tile tables
+      if (tab1 && !(seg_mblk && mblk_rows == kExpertBM)) {  // else dispatch_tiles_kernel
         write_tiles(tab1, nblk1, e, (int)pm, (int)mb, (int)p, (int)kept);
         write_tiles(tab2, nblk2, e, (int)pm, (int)mb, (int)p, (int)kept);
         for (long long j = 0; j < mb; ++j) mdone[pm + j] = 0;
@@ -366,6 +366,21 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
   }
 }
 
+// The expert GEMM's tile tables from the offsets and M-block prefix the scan
+// wrote: one thread per expert, so the tables (six 16-byte entries an expert
+// at d = 512, f = 1024) are written by many SMs instead of the scan's last block.
+__global__ void dispatch_tiles_kernel(const int *offsets, const int *mprefix, int n, int4 *tab1,
+                                      int nblk1, int4 *tab2, int nblk2, int *mdone) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= n) return;
+  const int row = offsets[e], rows = offsets[e + 1] - row;
+  const int mb_base = mprefix[e], mb = mprefix[e + 1] - mb_base;
+  write_tiles(tab1, nblk1, e, mb_base, mb, row, rows);
+  write_tiles(tab2, nblk2, e, mb_base, mb, row, rows);
+  for (int j = 0; j < mb; ++j) mdone[mb_base + j] = 0;
+  if (e == n - 1) mdone[mb_base + mb] = 0;  // the count over all M-blocks
+}
+
 __global__ void __launch_bounds__(SCAN_NT) expert_plan_kernel(const int *offsets, int n,
                                                               int *mprefix, int4 *tab1, int nblk1,
                                                               int4 *tab2, int nblk2, int *mdone) {
@@ -427,6 +442,10 @@ int launch_dispatch(const DispatchArgs &a, cudaStream_t st) {
   o.mdone = a.mdone;
   MOE_TRY(launch("dispatch_scan", dispatch_scan_kernel, dim3((unsigned)ceil_div(a.n, 32)),
                  dim3(SCAN_NT), 0, st, (const int *)a.hist, B, a.n, a.base, a.counts, a.ticket, o));
+  if (a.tab1 && a.seg_mblk && a.mblk_rows == kExpertBM)  // the tile tables, off the scan's last block
+    MOE_TRY(launch("dispatch_tiles", dispatch_tiles_kernel, dim3((unsigned)ceil_div(a.n, 128)),
+                   dim3(128), 0, st, (const int *)a.offsets, (const int *)a.seg_mblk, a.n, a.tab1,
+                   a.nblk1, a.tab2, a.nblk2, a.mdone));
   if (B == 0) return MOE_OK;
   const dim3 grid((unsigned)ceil_div(a.T, NT / 32));
   const long long C = a.C;
