@@ -97,6 +97,9 @@ CASES = {
                                                   **LOSSES),
     "hier-f32": W["hierarchical"].with_(T=64, d=32, n=4 * 4, hier_a=4, hier_b=4, f=32,
                                         expert_bf16=0, **LOSSES),
+    # 64 experts in routing tiles of 20 rows: the routing kernel's two-rows-per-warp
+    # instance, whose thresholds and kept gates the gate's backward reads
+    "narrow-routing": W["lm-flat"].with_(T=20000, n=64, k=2, d=32, f=32, **LOSSES),
 }
 
 GRAD_KEYS = [("dx", "dx"), ("dWg", "dWg"), ("dbg", "dbg"), ("dWn", "dWn"), ("dW1", "dW1"),

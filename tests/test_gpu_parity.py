@@ -73,6 +73,14 @@ SMALL = {
     "stats-sigmoid": V["deepseek-tiny"].with_(router_stats=1),
     "stats-hier": W["hierarchical"].with_(T=200, d=64, n=8 * 16, hier_a=8, hier_b=16, f=64,
                                           router_stats=1),
+    # rows of at most 128 experts in tiles of 16+ rows: the routing kernel's
+    # several-rows-per-warp instance (4 rows a warp at 64 experts and tiles of
+    # 32+ rows, else 2), on each router
+    "narrow-noisy-64": W["lm-flat"].with_(T=40000, n=64, k=2, d=32, f=32),
+    "narrow-switch-64": W["switch-top1"].with_(T=40000, d=32, n=64, f=32),
+    "narrow-switch-128-stats": W["switch-top1"].with_(T=40000, d=32, n=128, f=32, router_stats=1),
+    "narrow-sigmoid-100": V["deepseek-tiny"].with_(T=20000, n=100, k=4, d=32, f=32),
+    "narrow-noisy-96-stats": W["lm-flat"].with_(T=20000, n=96, k=3, d=32, f=32, router_stats=1),
 }
 
 
