@@ -34,16 +34,4 @@ __device__ __forceinline__ void insert(Cand (&L)[K1], float v, int i) {
   }
 }
 
-// An unsigned key that orders non-NaN floats as their values do (-0 and +0
-// share a key, as they compare equal); 0 is below every value's key and
-// marks an empty slot.
-__device__ __forceinline__ uint32_t order_key(float v) {
-  uint32_t b = __float_as_uint(v);
-  if (b == 0x80000000u) b = 0u;  // -0 -> +0
-  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
-}
-__device__ __forceinline__ float order_key_value(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
 }  // namespace moe
