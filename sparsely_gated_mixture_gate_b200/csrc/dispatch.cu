@@ -135,13 +135,13 @@ __device__ __forceinline__ void block_exclusive_scan4(long long (&v)[4]) {
 
 constexpr int SCAN_NT = 1024, SCAN_PER = 8;  // n <= 8192
 
-// One expert's tiles of a grouped GEMM: N-block major, M-block minor; the
-// last field packs the N-block (8 bits) and the global M-block index.
+// One expert's tiles of a grouped GEMM: entry (global M-block) * nblk + N-block;
+// the last field packs the N-block (8 bits) and the global M-block index.
 __device__ __forceinline__ void write_tiles(int4 *tab, int nblk, int e, int mb_base, int mbe,
                                             int row_base, int rows) {
-  for (int nbk = 0; nbk < nblk; ++nbk)
-    for (int mb = 0; mb < mbe; ++mb)
-      tab[(size_t)(mb_base * nblk + nbk * mbe + mb)] =
+  for (int mb = 0; mb < mbe; ++mb)
+    for (int nbk = 0; nbk < nblk; ++nbk)
+      tab[(size_t)(mb_base + mb) * nblk + nbk] =
           make_int4(e, row_base + mb * kExpertBM, min(kExpertBM, rows - mb * kExpertBM),
                     nbk | ((mb_base + mb) << 8));
 }
@@ -288,11 +288,11 @@ __global__ void __launch_bounds__(NT) dispatch_place_kernel(
       shared_mprefix[1] = mbe;
     }
     for (int i = threadIdx.x; i < mbe * nblk1; i += NT) {
-      const int nbk = i / mbe, mb = i - nbk * mbe;
+      const int mb = i / nblk1, nbk = i - mb * nblk1;  // entry: M-block * nblk + N-block
       shared_tab1[i] = make_int4(0, mb * kExpertBM, min(kExpertBM, T - mb * kExpertBM), nbk | (mb << 8));
     }
     for (int i = threadIdx.x; i < mbe * nblk2; i += NT) {
-      const int nbk = i / mbe, mb = i - nbk * mbe;
+      const int mb = i / nblk2, nbk = i - mb * nblk2;
       shared_tab2[i] = make_int4(0, mb * kExpertBM, min(kExpertBM, T - mb * kExpertBM), nbk | (mb << 8));
     }
     for (int i = threadIdx.x; i <= mbe; i += NT) shared_mdone[i] = 0;

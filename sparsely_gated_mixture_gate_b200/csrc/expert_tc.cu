@@ -13,14 +13,20 @@
 // with the same tiles (N = f, then N = d); their B operands are the weights
 // as stored, i.e. MN-major (N contiguous), loaded as four 64-column boxes.
 //
-// One persistent kernel runs both, one CTA per SM, 320 threads.  Every CTA
-// takes its share of GEMM1's tiles and then of GEMM2's, so GEMM2 starts on
-// the SMs that finish GEMM1 first; a GEMM2 tile of M-block m waits (bounded)
-// until the epilogues of all GEMM1 tiles of m have published their rows of
-// hid (a counter per M-block, and one for all of GEMM1: once a CTA has seen
-// all of GEMM1 published, its later GEMM2 tiles need no check).  The launch
-// is cooperative, so every CTA is resident and no wait can depend on a CTA
-// that has not started.
+// One persistent kernel runs both, one CTA per SM, 320 threads.  The two
+// GEMMs' tiles form one list (see tile_at): M-block by M-block, the GEMM1
+// tiles of M-block s and then the GEMM2 tiles of M-block s - lag, where the
+// lag is a few waves of tiles.  So an M-block's rows of hid are read back
+// by GEMM2 a few waves after they were written, from L2, instead of after
+// the whole of GEMM1.  CTA i takes tiles i, i + grid, ...  A GEMM2 tile of
+// M-block m waits (bounded) until the epilogues of all GEMM1 tiles of m have
+// published their rows of hid (a counter per M-block, and one for all of
+// GEMM1: once a CTA has seen all of GEMM1 published, its later GEMM2 tiles
+// need no check).  Every GEMM1 tile of m comes before the GEMM2 tiles of m in
+// the list, and every CTA runs its tiles in list order, so the unfinished
+// tile earliest in the list never waits on a later one; the launch is
+// cooperative, so every CTA is resident and no wait can depend on a CTA that
+// has not started.
 //   warp 0  TMA producer: 128x64 A tile + 256x64 B tile per stage (128-byte
 //           swizzle), 4 stages, mbarrier transaction counts
 //   warp 1  MMA issuer: tcgen05.mma kind::f16 (bf16 x bf16 -> fp32), M=128,
@@ -34,9 +40,9 @@
 //           row segments, masked to the expert's valid rows; the hidden layer's
 //           stores carry an evict-last L2 policy (GEMM2 reads it back)
 // Two accumulators of 256 columns (all 512 TMEM columns) let the epilogue of
-// one tile overlap the main loop of the next.  Tiles are ordered expert by
-// expert, N-block by N-block, M-block fastest, so the M-blocks that share a
-// weight tile run at the same time and the weights stream from HBM once.
+// one tile overlap the main loop of the next.  M-blocks are numbered expert by
+// expert, so the M-blocks that share a weight tile run at about the same time
+// and the weights stream from HBM once.
 // No cluster multicast anywhere.
 //
 // Every wait is bounded (about two seconds of %globaltimer); a wait that runs
@@ -64,6 +70,7 @@ constexpr int EPI_STAGE_BYTES = 32 * 128;    // per epilogue warp: 32 rows x 64 
 constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES + NUM_EPI_WARPS * EPI_STAGE_BYTES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr unsigned long long kWaitNs = 2000000000ull;
+constexpr int kLagWaves = 3;  // see tile_at
 
 // instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
 // = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N>>3 at bits
@@ -91,7 +98,25 @@ struct FfnArgs {
   int *status;
   unsigned long long xwait_ns;  // limit of a GEMM2 tile's wait for its M-block of hid
   int withhold_mblk;     // test hook: this M-block's GEMM1 tiles never publish (-1: none)
+  int lag;               // M-blocks between a GEMM1 M-block and GEMM2's in the tile list
 };
+
+// Tile c of the list: the GEMM1 tiles of M-blocks 0 .. lag-1, then for s =
+// lag, lag+1, ... the GEMM1 tiles of M-block s followed by the GEMM2 tiles of
+// M-block s - lag, then the GEMM2 tiles of the last lag M-blocks.  The tile
+// tables are M-block major (entry M-block * nblk + N-block).  Returns the
+// GEMM (0, 1) and the entry of its table.
+__device__ __forceinline__ int2 tile_at(int c, int mtotal, int n1, int n2, int lag) {
+  const int lead = min(lag, mtotal);
+  if (c < lead * n1) return make_int2(0, c);
+  c -= lead * n1;
+  const int w = n1 + n2, both = (mtotal - lead) * w;
+  if (c < both) {
+    const int s = c / w, r = c - s * w;
+    return r < n1 ? make_int2(0, (lead + s) * n1 + r) : make_int2(1, s * n2 + (r - n1));
+  }
+  return make_int2(1, (mtotal - lead) * n2 + (c - both));
+}
 
 __device__ __forceinline__ int ld_acquire(const int *p) {
   int v;
@@ -170,11 +195,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     for (int s = 0; s < STAGES; ++s) issued[s] = -1;
     bool g1_all = false;  // all of GEMM1's hid seen published (acquire + proxy fence done)
     auto entry = [&](int t) {
-      return t < total ? __ldg(a.g[t >= T1].tiles + (t >= T1 ? t - T1 : t)) : make_int4(0, 0, 0, 0);
+      if (t >= total) return make_int4(0, 0, 0, 0);
+      const int2 w = tile_at(t, mtotal, a.g[0].nblk, a.g[1].nblk, a.lag);
+      return __ldg(a.g[w.x].tiles + w.y);
     };
     int4 ti = entry(blockIdx.x);
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      const int which = tile >= T1;
+      const int which = tile_at(tile, mtotal, a.g[0].nblk, a.g[1].nblk, a.lag).x;
       const GemmArgs &g = a.g[which];
       const int4 next = entry(tile + gridDim.x);  // fetched while this tile's loads go out
       if (which && !g1_all) {
@@ -224,7 +251,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     uint32_t phase = 0, acc_phase = 0;
     bool issued_any = false;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      const int nkb = (a.g[tile >= T1].K + BK - 1) / BK;
+      const int nkb = (a.g[tile_at(tile, mtotal, a.g[0].nblk, a.g[1].nblk, a.lag).x].K + BK - 1) / BK;
       if (!mbar_wait(tempty(acc), acc_phase ^ 1u, abort_flag, kWaitNs)) { failed = true; break; }
       tc_fence_after();
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BN);
@@ -268,9 +295,10 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     int acc = 0;
     uint32_t acc_phase = 0;
     for (int tile = blockIdx.x; tile < total && !failed; tile += gridDim.x) {
-      const int which = tile >= T1;
+      const int2 wt = tile_at(tile, mtotal, a.g[0].nblk, a.g[1].nblk, a.lag);
+      const int which = wt.x;
       const GemmArgs &g = a.g[which];
-      const int4 ti = __ldg(g.tiles + (which ? tile - T1 : tile));
+      const int4 ti = __ldg(g.tiles + wt.y);
       const int e = ti.x, nbk = ti.w & 0xFF;
       // bias of this warp's 128 columns, lane l holding columns l, l+32, ...;
       // loaded before the wait so the latency hides behind the main loop
@@ -454,6 +482,8 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   const int ctas = ffn_ctas();
   if (ctas < 1) return MOE_ECUDA;
   const int grid = (int)(upper < ctas ? upper : ctas);
+  // a GEMM2 tile follows its M-block's GEMM1 tiles by kLagWaves waves of tiles
+  f.lag = (int)ceil_div((int64_t)kLagWaves * grid, nblk1 + nblk2);
 
   // cooperative: all CTAs resident at once (a GEMM2 tile waits on other
   // CTAs' GEMM1 tiles)
