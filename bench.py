@@ -535,6 +535,8 @@ def run_ours(args, w, world, rank, local, steps=None, warmup=None, alt_gate=None
     route_ms = sum(per_kernel[k]["ms"] / t_steps for k in route_names)
     route_bytes = sum(kernel_work(w, k, S_kept)[2] for k in route_names)
 
+    routing = routing_report(w, layer)
+
     line = {
         "metric": METRIC_TRAIN if dy is not None else METRIC, "value": round(value, 1),
         "unit": "tokens/s", "n_gpus": world,
@@ -579,10 +581,31 @@ def run_ours(args, w, world, rank, local, steps=None, warmup=None, alt_gate=None
         "alt_gate_mode": alt,
         "wall_s": round(wall, 3),
         "device_status": st,
+        "routing": routing,
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
     return line
+
+
+def routing_report(w, layer):
+    """The last step's routing outcome, read back after the timed region: the
+    per-expert slot counts (the load histogram, summarised), the balancing
+    losses and the drop rate, from the layer's own outputs."""
+    counts = layer.counts.double().cpu()
+    losses = layer.losses.double().cpu().tolist()
+    mean = float(counts.mean())
+    hist = {"experts": int(counts.numel()), "min": int(counts.min()), "max": int(counts.max()),
+            "mean": round(mean, 3), "std": round(float(counts.std(unbiased=False)), 3),
+            "max_over_mean": round(float(counts.max()) / mean, 3) if mean > 0 else None,
+            "empty_experts": int((counts == 0).sum())}
+    rep = {"counts": hist, "L_importance": losses[0], "L_load": losses[1],
+           "cv2_importance": losses[5], "cv2_load": losses[6],
+           "drop_rate": losses[4], "dropped_slots": int(losses[7])}
+    if w.router == 1:  # Switch: N * sum f_i P_i and its alpha-weighted loss
+        rep["switch_aux"] = losses[2]
+        rep["L_aux"] = losses[3]
+    return rep
 
 
 def per_config_summary(line):
@@ -594,7 +617,7 @@ def per_config_summary(line):
            "expert_ffn_tflops": line["expert_ffn_tflops"],
            "expert_ffn_frac_bf16_peak": line["expert_ffn_frac_bf16_peak"],
            "routing_frac_hbm": line["routing_frac_hbm"], "clocks": line["clocks"],
-           "device_status": line["device_status"]}
+           "device_status": line["device_status"], "routing": line["routing"]}
     ks = {}
     for name in ("gate_gemm_fp32", "route_topk", "dispatch_place", "combine", "expert_ffn_tcgen05"):
         if name in line["kernels"] and "roofline" in line["kernels"][name]:
