@@ -15,10 +15,12 @@
 //
 // One persistent kernel runs both, one CTA per SM, 320 threads.  The two
 // GEMMs' tiles form one list (see tile_at): M-block by M-block, the GEMM1
-// tiles of M-block s and then the GEMM2 tiles of M-block s - lag, where the
-// lag is a few waves of tiles.  So an M-block's rows of hid are read back
-// by GEMM2 a few waves after they were written, from L2, instead of after
-// the whole of GEMM1.  CTA i takes tiles i, i + grid, ...  A GEMM2 tile of
+// tiles of M-block s and then the GEMM2 tiles of M-block s - lag.  When the
+// experts stream their weights at the HBM limit (few rows per expert) the
+// lag is a few waves of tiles, so an M-block's rows of hid are read back by
+// GEMM2 a few waves after they were written, from L2, instead of after the
+// whole of GEMM1; otherwise the lag covers every M-block and all of GEMM1
+// runs first (see kInterleaveMaxRows).  CTA i takes tiles i, i + grid, ...  A GEMM2 tile of
 // M-block m waits (bounded) until the epilogues of all GEMM1 tiles of m have
 // published their rows of hid (a counter per M-block, and one for all of
 // GEMM1: once a CTA has seen all of GEMM1 published, its later GEMM2 tiles
@@ -50,6 +52,7 @@
 // drains the copies and MMAs this CTA issued (again bounded), frees its
 // tensor memory and returns.
 #include <atomic>
+#include <climits>
 
 #include "tc_common.cuh"
 
@@ -71,6 +74,14 @@ constexpr int SMEM_BYTES = STAGES * STAGE_BYTES + 1024 + BAR_BYTES + NUM_EPI_WAR
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
 constexpr unsigned long long kWaitNs = 2000000000ull;
 constexpr int kLagWaves = 3;  // see tile_at
+// Interleave only while the experts average fewer rows than this: each byte of
+// expert weights then feeds fewer FLOPs than about 0.75 x (bf16 tensor peak /
+// HBM bandwidth), so the weights stream at the HBM limit and the hidden
+// layer's DRAM round trip competes with them.  With more rows the GEMMs sit
+// near the tensor-bound ridge, that round trip costs nothing HBM cannot
+// spare, and interleaving measured 3-8% slower (switch-top1, 256 rows per
+// expert) than running all of GEMM1 first.
+constexpr int kInterleaveMaxRows = 192;
 
 // instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9
 // = 1), B bf16 (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N>>3 at bits
@@ -482,8 +493,12 @@ int launch_expert_bf16(const ExpertArgs &a, cudaStream_t st) {
   const int ctas = ffn_ctas();
   if (ctas < 1) return MOE_ECUDA;
   const int grid = (int)(upper < ctas ? upper : ctas);
-  // a GEMM2 tile follows its M-block's GEMM1 tiles by kLagWaves waves of tiles
-  f.lag = (int)ceil_div((int64_t)kLagWaves * grid, nblk1 + nblk2);
+  // a GEMM2 tile follows its M-block's GEMM1 tiles by kLagWaves waves of tiles;
+  // a lag of every M-block runs all of GEMM1 first
+  const int64_t mblk_upper = ceil_div(a.S, BM) + a.n;
+  f.lag = (int64_t)a.S < (int64_t)kInterleaveMaxRows * a.n
+              ? (int)ceil_div((int64_t)kLagWaves * grid, nblk1 + nblk2)
+              : (int)(mblk_upper < INT_MAX ? mblk_upper : INT_MAX);
 
   // cooperative: all CTAs resident at once (a GEMM2 tile waits on other
   // CTAs' GEMM1 tiles)

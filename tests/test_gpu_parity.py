@@ -258,6 +258,10 @@ SKEWED = [
     (256, 1024, [4000, 0, 3, 0]),
     # GEMM2 with more N-blocks than GEMM1, ragged tails
     (768, 256, [1, 2000, 0, 900, 5]),
+    # fewer than 192 rows per expert on average, so GEMM2 tiles are interleaved
+    # a few waves behind GEMM1's; one expert spans 313 M-blocks, more than
+    # that lag, so its GEMM2 tiles wait on M-blocks finished moments before
+    (128, 256, [40000] + [40] * 299),
 ]
 
 
