@@ -15,8 +15,8 @@ LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["moe_api.cu", "gate_gemm.cu", "route.cu", "dispatch.cu", "expert_tc.cu",
            "expert_f32.cu", "combine.cu", "stats.cu", "dispatch_static.cu", "tc_common.cu", "gate_tc.cu",
            "backward.cu", "grad_gemm.cu", "wgrad_tc.cu", "fma_probe.cu", "ep.cu",
-           "gate_cutlass.cu", "backward_hier.cu"]
-HEADERS = ["internal.h", "philox.cuh", "tc_common.cuh", "route_common.cuh", "phi.cuh"]
+           "backward_hier.cu"]
+HEADERS = ["internal.h", "philox.cuh", "tc_common.cuh", "route_common.cuh", "phi.cuh", "fma2.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr"]
@@ -27,19 +27,6 @@ def _nvcc() -> str:
         if cand and os.path.exists(cand):
             return cand
     raise RuntimeError("nvcc not found")
-
-
-def cutlass_include() -> str:
-    """The CUTLASS header tree vendored in the image (flashinfer's copy), for
-    the SIMT GEMM templates of gate_cutlass.cu."""
-    import importlib.util
-    spec = importlib.util.find_spec("flashinfer")
-    if spec is None or not spec.submodule_search_locations:
-        raise RuntimeError("CUTLASS headers not found (flashinfer/data/cutlass/include)")
-    inc = os.path.join(list(spec.submodule_search_locations)[0], "data", "cutlass", "include")
-    if not os.path.exists(os.path.join(inc, "cutlass", "cutlass.h")):
-        raise RuntimeError(f"CUTLASS headers not found under {inc}")
-    return inc
 
 
 def _newest(paths):
@@ -60,8 +47,6 @@ def build(force: bool = False, verbose: bool = False) -> str:
         if not force and os.path.exists(o) and os.path.getmtime(o) >= max(dep_time, os.path.getmtime(s)):
             return o
         cmd = [nvcc, *ARCH, *FLAGS, "-c", s, "-o", o]
-        if src == "gate_cutlass.cu":
-            cmd[1:1] = ["-I", cutlass_include()]
         if verbose:
             print(" ".join(cmd))
         subprocess.check_call(cmd)

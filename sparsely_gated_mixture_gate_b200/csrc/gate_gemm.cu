@@ -18,7 +18,12 @@
 // reads of a warp are broadcast / conflict free.  Double-buffered shared
 // memory, global loads of the next K-slice overlap the FMAs of the current,
 // and the register fragments of the next k step are read during the FMAs of
-// this one.
+// this one.  The multiply-adds are packed (fma.rn.f32x2: two independent
+// fp32 FMAs, each rounded as fmaf would): the accumulators of columns j, j+1
+// form a pair, multiplied by the pair (a_i, a_i) and the pair (b_j, b_j+1),
+// so one instruction does two of the 64 per k step and the FMA issue slots
+// halve; every output is still one fmaf chain over k in order.
+#include "fma2.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -109,11 +114,12 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
     }
   };
 
-  float acc[8][8];
+  // accumulator pairs: acc2[i][j] holds columns 2j, 2j+1 of row i
+  unsigned long long acc2[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc2[i][j] = 0ull;
 
   const int tx = tid & 15, ty = tid >> 4;
   const int nk = (a.d + BK - 1) / BK;
@@ -147,18 +153,29 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
       }
       const float ar_[8] = {fa0[cur].x, fa0[cur].y, fa0[cur].z, fa0[cur].w,
                             fa1[cur].x, fa1[cur].y, fa1[cur].z, fa1[cur].w};
-      const float br_[8] = {fb0[cur].x, fb0[cur].y, fb0[cur].z, fb0[cur].w,
-                            fb1[cur].x, fb1[cur].y, fb1[cur].z, fb1[cur].w};
+      unsigned long long bp[4];
+      bp[0] = pack2(fb0[cur].x, fb0[cur].y);
+      bp[1] = pack2(fb0[cur].z, fb0[cur].w);
+      bp[2] = pack2(fb1[cur].x, fb1[cur].y);
+      bp[3] = pack2(fb1[cur].z, fb1[cur].w);
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
+      for (int i = 0; i < 8; ++i) {
+        const unsigned long long ap = pack2(ar_[i], ar_[i]);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(ar_[i], br_[j], acc[i][j]);
+        for (int j = 0; j < 4; ++j) fma2(acc2[i][j], ap, bp[j]);
+      }
     }
     if (kt + 1 < nk) {
       store_tiles(buf ^ 1, av, bv);
     }
     __syncthreads();
   }
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack2(acc2[i][j], acc[i][2 * j], acc[i][2 * j + 1]);
 
   // ---- epilogue: columns [0, nb) are c (+ bias), [nb, 2 nb) are s = Softplus
   const float *bias = a.bias ? a.bias + (size_t)g * nb : nullptr;
@@ -203,7 +220,6 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
 }  // namespace
 
 int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st) {
-  if (gate_gemm_cutlass_applies(a)) return launch_gate_gemm_cutlass(a, st);
   const int ncol = a.noise ? 2 * a.nb : a.nb;
   dim3 grid(mblk_upper, (ncol + BN - 1) / BN);
   return launch("gate_gemm_fp32", gate_gemm_kernel, grid, dim3(NT), 0, st, a);

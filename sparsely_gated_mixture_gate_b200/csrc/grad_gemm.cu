@@ -18,6 +18,7 @@
 // A grouped mode serves the hierarchical layer's secondary gates: one launch
 // over the groups' row segments, along K (the weight gradients, A's rows
 // gathered by token) or along M (the input gradient, one weight pair per group).
+#include "fma2.cuh"
 #include "internal.h"
 
 namespace moe {
@@ -148,11 +149,13 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
     }
   };
 
-  float acc[8][8];
+  // accumulator pairs: acc2[i][j] holds columns 2j, 2j+1 of row i (packed
+  // FMAs, see fma2.cuh)
+  unsigned long long acc2[8][4];
 #pragma unroll
   for (int i = 0; i < 8; ++i)
 #pragma unroll
-    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+    for (int j = 0; j < 4; ++j) acc2[i][j] = 0ull;
 
   // the pairs whose products are summed: pair 1 only with ksum
   const int npair = a.ksum ? 2 : 1;
@@ -192,12 +195,17 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
         }
         const float av8[8] = {fa0[cur].x, fa0[cur].y, fa0[cur].z, fa0[cur].w,
                               fa1[cur].x, fa1[cur].y, fa1[cur].z, fa1[cur].w};
-        const float bv8[8] = {fb0[cur].x, fb0[cur].y, fb0[cur].z, fb0[cur].w,
-                              fb1[cur].x, fb1[cur].y, fb1[cur].z, fb1[cur].w};
+        unsigned long long bp[4];
+        bp[0] = pack2(fb0[cur].x, fb0[cur].y);
+        bp[1] = pack2(fb0[cur].z, fb0[cur].w);
+        bp[2] = pack2(fb1[cur].x, fb1[cur].y);
+        bp[3] = pack2(fb1[cur].z, fb1[cur].w);
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
+        for (int i = 0; i < 8; ++i) {
+          const unsigned long long ap = pack2(av8[i], av8[i]);
 #pragma unroll
-          for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av8[i], bv8[j], acc[i][j]);
+          for (int j = 0; j < 4; ++j) fma2(acc2[i][j], ap, bp[j]);
+        }
       }
       if (more) {
         store(buf ^ 1, av, bv);
@@ -206,6 +214,12 @@ __global__ void __launch_bounds__(NT, 2) sgemm_kernel(SgemmArgs a) {
       }
     }
   }
+
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) unpack2(acc2[i][j], acc[i][2 * j], acc[i][2 * j + 1]);
 
   // output rows ty*4+i (i<4) and 64+ty*4+i-4, columns tx*4+j and 64+tx*4+j-4
   float *const C = (prob ? a.C[1] : a.C[0]) + offC;

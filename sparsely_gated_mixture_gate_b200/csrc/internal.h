@@ -101,11 +101,6 @@ struct GateGemmArgs {
   int *status;
 };
 int launch_gate_gemm(const GateGemmArgs &a, int mblk_upper, cudaStream_t st);
-// the flat gate with at least kGateCutlassMinCols columns per projection runs
-// on CUTLASS's SIMT GEMM (gate_cutlass.cu); same results, bit for bit
-constexpr int kGateCutlassMinCols = 2048;
-bool gate_gemm_cutlass_applies(const GateGemmArgs &a);
-int launch_gate_gemm_cutlass(const GateGemmArgs &a, cudaStream_t st);
 // the same on the tensor cores (three-pass TF32 split); xhi/xlo: [R][d],
 // whi/wlo: [G][nb*(noise?2:1)][d] scratch
 int launch_gate_tf32x3(const GateGemmArgs &a, int mblk_upper, float *xhi, float *xlo, float *whi,

@@ -144,7 +144,7 @@ GUARD_CASES = {
     "hier-T777": synth.WORKLOADS["hierarchical"].with_(T=777, d=40, f=24, n=4 * 8, hier_a=4,
                                                        hier_b=8),
     "sigmoid-shared-T33": synth.VARIANTS["deepseek-tiny"].with_(T=33, d=40, f=24),
-    # 2048 experts: the gate's projections on the CUTLASS SIMT path
+    # 2048 experts: a wide gate (16 column tiles per projection)
     "wide-gate-T33": synth.WORKLOADS["many-expert"].with_(T=33, d=40, f=24, n=2048, k=2),
 }
 

@@ -528,13 +528,13 @@ def test_shard_with_token_base_draws_the_batch_noise(name):
     assert not torch.equal(other["topk_gate"], whole["topk_gate"][h:])
 
 
-def test_wide_gate_paths_route_alike():
-    """Flat gates of 2048 or more columns take the CUTLASS SIMT mainloop,
-    narrower ones the library's own SIMT kernel; both compute each logit as
-    the same fp32 FMA chain over d in order with the same epilogue rounding.
-    Run the same 2044 experts through both: at 2048 columns the four extra
-    experts carry a bias of -1e30 (never kept, never a threshold), so the
-    routing, the gates and the smoothed Load of the 2044 must agree exactly."""
+def test_wide_gate_tiling_routes_alike():
+    """Every logit is one fp32 FMA chain over d in order, whatever column tile
+    of the gate GEMM it falls in, and the routing kernel's result does not
+    depend on how many columns share a row.  Run the same 2044 experts as a
+    gate of 2044 columns and of 2048, where the four extra experts carry a
+    bias of -1e30 (never kept, never a threshold): the routing, the gates and
+    the smoothed Load of the 2044 must agree exactly."""
     w = W["many-expert"].with_(T=1000, d=256, n=2048, k=4)
     inp = to_dev(synth.make_inputs(w, experts=False))
     inp["bg"][2044:] = -1e30
