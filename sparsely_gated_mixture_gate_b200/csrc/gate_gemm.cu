@@ -158,12 +158,13 @@ __global__ void __launch_bounds__(NT, 2) gate_gemm_kernel(GateGemmArgs a) {
       bp[1] = pack2(fb0[cur].z, fb0[cur].w);
       bp[2] = pack2(fb1[cur].x, fb1[cur].y);
       bp[3] = pack2(fb1[cur].z, fb1[cur].w);
+      unsigned long long ap[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const unsigned long long ap = pack2(ar_[i], ar_[i]);
+      for (int i = 0; i < 8; ++i) ap[i] = pack2(ar_[i], ar_[i]);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) fma2(acc2[i][j], ap, bp[j]);
-      }
+      for (int j = 0; j < 4; ++j)  // each B pair over the eight rows (measured 1% faster)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) fma2(acc2[i][j], ap[i], bp[j]);
     }
     if (kt + 1 < nk) {
       store_tiles(buf ^ 1, av, bv);
