@@ -11,9 +11,13 @@
 //
 // One persistent kernel, one CTA per SM, 320 threads, the same roles as the
 // forward's expert kernel:
-//   warp 0  TMA producer: per stage the A tile (128 M x 64 rows, two 64-column
-//           boxes) and the B tile (256 N x 64 rows, four boxes), 128-byte
-//           swizzle, 4 stages
+//   warp 0  TMA producer: per stage the A tile (128 M x 32 rows, two 64-column
+//           boxes) and the B tile (256 N x 32 rows, four boxes), 128-byte
+//           swizzle, 8 stages.  32-row K steps: the hierarchical layer's
+//           experts hold ~32 rows each, and 64-row steps loaded as many rows
+//           of the next expert as of their own (measured: 32-row steps 6% and
+//           4-9% faster than 64-row steps on the hierarchical layer and at 256
+//           experts of ~128 rows; 16-row steps 6% slower on the latter)
 //   warp 1  MMA: tcgen05.mma kind::f16 with both operands MN-major (M=128,
 //           N=256, K=16).  The last K step of an expert reads rows that
 //           belong to the next expert (or the zero fill past the end); the
@@ -35,8 +39,8 @@ namespace moe {
 namespace {
 using namespace tc;
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
-constexpr int BOX = 64 * BK * 2;  // one 64-column x 64-row box, 8 KiB
+constexpr int BM = 128, BN = 256, BK = 32, STAGES = 8;
+constexpr int BOX = 64 * BK * 2;  // one 64-column x BK-row box, 4 KiB
 constexpr int A_BYTES = BM * BK * 2;
 constexpr int B_BYTES = BN * BK * 2;
 constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
@@ -49,6 +53,8 @@ constexpr int EPI_STAGE_BYTES = 32 * 128;  // per epilogue warp: 32 rows x 32 fp
 constexpr int SMEM_BYTES =
     STAGES * STAGE_BYTES + 1024 + BAR_BYTES + NUM_EPI_WARPS * EPI_STAGE_BYTES;
 static_assert(SMEM_BYTES <= 232448, "shared memory per CTA");
+// full/empty per stage, tfull/tempty per accumulator, drain; then the TMEM slot and abort flag
+static_assert((2 * STAGES + 5) * 8 + 8 <= BAR_BYTES, "barrier area");
 constexpr unsigned long long kWaitNs = 2000000000ull;
 
 // kind::f16, D fp32, A and B bf16, both MN-major (bits 15, 16), N>>3, M>>4
@@ -306,7 +312,7 @@ int launch_wgrad_bf16(const WgradArgs &a, cudaStream_t st) {
     *out = per_sm * num_sms();
     return MOE_OK;
   }, &ctas));
-  // rows beyond S read as zero; every box is 64 columns x 64 rows
+  // rows beyond S read as zero; every box is 64 columns x BK rows
   const uint64_t S = (uint64_t)(a.S > 0 ? a.S : 1);
   CUtensorMap mA0, mB0, mA1, mB1;
   MOE_TRY(tc::make_map_2d(&mA0, a.dy_perm, 2, (uint64_t)a.d, S, BK));
