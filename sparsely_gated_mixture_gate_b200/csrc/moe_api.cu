@@ -191,7 +191,7 @@ Layout make_layout(const moe_config &c) {
   L.c2 = hier ? bp.take(4 * R2 * (size_t)c.hier_b) : 0;
   L.s2 = hier ? bp.take(4 * R2 * (size_t)c.hier_b) : 0;
   const size_t lp1 = (size_t)L.tiles1 * ng, lp2 = (size_t)L.tiles2_upper * (size_t)c.hier_b;
-  L.load_part = bp.take(4 * (lp1 > lp2 ? lp1 : lp2));
+  L.load_part = bp.take(4 * lp1);
   L.psum_part = bp.take(c.router == MOE_ROUTER_SWITCH ? 4 * (size_t)L.tiles1 * n : 0);
   L.prob_sum = bp.take(4 * n);
   L.stats_part = bp.take(c.router_stats ? 8 * (size_t)L.tiles1 : 0);
@@ -212,7 +212,8 @@ Layout make_layout(const moe_config &c) {
     L.g_row_of = bp.take(4 * T * k1);
     L.g_mblk = bp.take(4 * (a + 1));
     L.g_tiles = bp.take(4 * (a + 1));
-    L.load2_part = L.load_part;  // the primary partial sums are reduced first
+    // its own buffer: both levels' partial sums are reduced after the secondary routing
+    L.load2_part = bp.take(4 * lp2);
     L.load2 = bp.take(4 * n);
   } else {
     L.pidx = L.pgate = L.load_p = L.g_hist = L.g_base = L.g_counts = L.g_offsets = L.g_ucoff =
@@ -446,9 +447,7 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r.out_gate = pgate;
   r.K = k1;
   MOE_TRY(launch_route(r, L.tiles1, st));
-  MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, a, at<float>(ws, L.load_p), st));
-  if (r.stats_part)
-    MOE_TRY(launch_route_reduce(r.stats_part, nullptr, 1, L.tiles1, 2, at<float>(ws, L.rstats), st));
+  // (the primary gate's Load and statistics are reduced below, with the secondary Load)
 
   // ---- tokens grouped by their kept groups (stable), tile prefixes per group
   DispatchArgs da{};
@@ -516,10 +515,20 @@ int run_gate(const moe_config &c, const Layout &L, const float *x, const moe_gat
   r2.load_part = at<float>(ws, L.load2_part);
   r2.psum_part = nullptr;
   MOE_TRY(launch_route(r2, L.tiles2_upper, st));
-  MOE_TRY(launch_route_reduce(r2.load_part, da.seg_tiles, a, 0, b, at<float>(ws, L.load2), st));
+  // the Load of both levels and the statistics feed only the balancing losses:
+  // with a side stream they are reduced there, off the dispatch -> experts chain
+  cudaStream_t rs = st;
+  if (side) {
+    MOE_TRY(stream_after(side->s, st, side->fork_gate));
+    rs = side->s;
+  }
+  MOE_TRY(launch_route_reduce(r.load_part, nullptr, 1, L.tiles1, a, at<float>(ws, L.load_p), rs));
+  if (r.stats_part)
+    MOE_TRY(launch_route_reduce(r.stats_part, nullptr, 1, L.tiles1, 2, at<float>(ws, L.rstats), rs));
+  MOE_TRY(launch_route_reduce(r2.load_part, da.seg_tiles, a, 0, b, at<float>(ws, L.load2), rs));
   MOE_TRY(launch_hier_load(at<float>(ws, L.load_p), at<float>(ws, L.load2), da.counts, a, b, load,
-                           st));
-  if (prob_sum && cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, st) != cudaSuccess)
+                           rs));
+  if (prob_sum && cudaMemsetAsync(prob_sum, 0, 4 * (size_t)c.n, rs) != cudaSuccess)
     return MOE_ECUDA;
   return MOE_OK;
 }
