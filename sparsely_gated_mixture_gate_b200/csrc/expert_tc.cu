@@ -20,11 +20,11 @@
 // lag is a few waves of tiles, so an M-block's rows of hid are read back by
 // GEMM2 a few waves after they were written, from L2, instead of after the
 // whole of GEMM1; otherwise the lag covers every M-block and all of GEMM1
-// runs first (see kInterleaveMaxRows).  CTA i takes tiles i, i + grid, ...  A GEMM2 tile of
-// M-block m waits (bounded) until the epilogues of all GEMM1 tiles of m have
-// published their rows of hid (a counter per M-block, and one for all of
-// GEMM1: once a CTA has seen all of GEMM1 published, its later GEMM2 tiles
-// need no check).  Every GEMM1 tile of m comes before the GEMM2 tiles of m in
+// runs first (see kInterleaveMaxRows).  CTA i takes tiles i, i + grid, ...
+// A GEMM2 tile of M-block m waits (bounded) until the epilogues of all GEMM1
+// tiles of m have published their rows of hid (a counter per M-block, and one
+// for all of GEMM1: once a CTA has seen all of GEMM1 published, its later
+// GEMM2 tiles need no check).  Every GEMM1 tile of m comes before the GEMM2 tiles of m in
 // the list, and every CTA runs its tiles in list order, so the unfinished
 // tile earliest in the list never waits on a later one; the launch is
 // cooperative, so every CTA is resident and no wait can depend on a CTA that
