@@ -13,9 +13,9 @@
 //   Router statistics ([MoE-intro] 第三部分, optional): per row |c|^2 and the
 //   entropy of softmax(c), summed over the tile's rows in a fixed order.
 // Pass 1, one warp per row (rows of at most 128 columns: four rows per warp, 8
-// lanes each, in tiles of at least 32 rows, else two rows of 16 lanes; four
-// rows per warp halve the rounds and their barriers, 8% faster at 131072 rows
-// of 128): each lane scans column quads 4m .. 4m+3 (16-byte
+// lanes each; against two rows of 16 lanes, the rounds and their barriers
+// halve: 8-26% faster, most where the tiles are short): each lane scans
+// column quads 4m .. 4m+3 (16-byte
 // loads, one Philox call per quad) and keeps a sorted list of its k + 1 best
 // columns (ranked by H, then the lower column index); the warp merges the 32
 // lists with shuffles.  Rows of 512 columns or more rank quads instead, by
@@ -167,7 +167,7 @@ __global__ void __launch_bounds__(NW * 32, (MAXQ > 4 || SW) ? 3 : 4) route_kerne
 
   // pass 1: rows per warp and lanes per row; NR rows per round
   const bool by_quad = nb >= 512;  // rank quads: at least four quads per lane
-  const int RPW = !NARROW ? 1 : (a.RT >= 4 * NW) ? 4 : 2;
+  const int RPW = NARROW ? 4 : 1;
   const int LPR = 32 / RPW, sub = lane / LPR, sl = lane % LPR;
   const int NR = NW * RPW;
   // pass-2 thread layout: thread per column quad; with fewer quads than
